@@ -1,0 +1,161 @@
+"""Oracle for draft-token verification (speculative decoding).
+
+TEST INFRASTRUCTURE ONLY: a plain, slow, double-precision CPU statement of the
+verification step, written from the pages' prose (see ``oracle.cpp`` for the
+sources and readings). Only ``tests/``, ``__graft_entry__.smoke()`` and the
+CPU-baseline leg of ``bench.py`` may import it. It shares no code with the
+CUDA library and does not import it.
+
+Every function takes numpy arrays and returns numpy arrays. Logits are either
+float32 arrays or bfloat16 bit patterns held in uint16 arrays.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "oracle.cpp")
+_LIB = os.path.join(_HERE, "liboracle.so")
+
+FLAG_RATIO = 1
+FLAG_CDF = 2
+FLAG_TOPP = 4
+FLAG_TREE = 8
+DIAG_Q_ZERO = 16
+PARITY_FLAGS = FLAG_RATIO | FLAG_CDF | FLAG_TOPP | FLAG_TREE
+
+
+def build(force: bool = False) -> str:
+    """Compile the oracle into liboracle.so (plain g++, no GPU)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        cmd = ["g++", "-O2", "-std=c++17", "-ffp-contract=off", "-shared", "-fPIC",
+               "-pthread", _SRC, "-o", _LIB + ".tmp"]
+        subprocess.run(cmd, check=True)
+        os.replace(_LIB + ".tmp", _LIB)
+    return _LIB
+
+
+_lib = None
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        _lib = ctypes.CDLL(build())
+        P = ctypes.c_void_p
+        I = ctypes.c_int
+        D = ctypes.c_double
+        _lib.oracle_transform_rows.argtypes = [P, I, I, I, D, I, D, P, P, P, P, I]
+        _lib.oracle_verify_chain.argtypes = [P, P, I, I, I, I, P, P, D, I, D, P, P, P, I]
+        _lib.oracle_verify_chain_f64u.argtypes = [P, P, I, I, I, I, P, P, D, I, D, P, P, P, I]
+        _lib.oracle_verify_tree_typical.argtypes = [P, I, I, I, I, P, P, D, D, D, P, I, P, P, I]
+        _lib.oracle_residual_sample.argtypes = [P, P, I, I, P, P, P, I]
+        for f in (_lib.oracle_transform_rows, _lib.oracle_verify_chain,
+                  _lib.oracle_verify_chain_f64u,
+                  _lib.oracle_verify_tree_typical, _lib.oracle_residual_sample):
+            f.restype = I
+    return _lib
+
+
+def _ptr(a):
+    return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _dtype_code(logits: np.ndarray) -> int:
+    if logits.dtype == np.float32:
+        return 0
+    if logits.dtype == np.uint16:
+        return 1
+    raise TypeError("logits must be float32 or uint16 (bfloat16 bit patterns)")
+
+
+def _threads(threads):
+    return (os.cpu_count() or 1) if threads is None else int(threads)
+
+
+def transform_rows(logits, temp, top_k=0, top_p=1.0, threads=None):
+    """Rows of logits [..., V] -> (probs float64 [..., V], entropy, topp_margin, valid)."""
+    logits = np.ascontiguousarray(logits)
+    V = logits.shape[-1]
+    rows = logits.size // V
+    probs = np.zeros((rows, V), np.float64)
+    ent = np.zeros(rows, np.float64)
+    marg = np.zeros(rows, np.float64)
+    valid = np.zeros(rows, np.int32)
+    rc = _load().oracle_transform_rows(_ptr(logits), _dtype_code(logits), rows, V, float(temp),
+                                       int(top_k), float(top_p), _ptr(probs), _ptr(ent),
+                                       _ptr(marg), _ptr(valid), _threads(threads))
+    if rc != 0:
+        raise ValueError("oracle_transform_rows rejected its arguments")
+    shp = logits.shape[:-1]
+    return probs.reshape(*shp, V), ent.reshape(shp), marg.reshape(shp), valid.reshape(shp)
+
+
+def verify_chain(target, draft, draft_tokens, uniforms, temp, top_k=0, top_p=1.0, threads=None):
+    """Chain verification. target [B,K+1,V], draft [B,K,V] (unused when temp == 0),
+    draft_tokens int32 [B,K], uniforms float32 [B,K+1] (float64 uniforms select the
+    double-precision entry, used by the exact-integration tests).
+    Returns (accepted_len int32 [B], out_tokens int32 [B,K+1], flags int32 [B])."""
+    target = np.ascontiguousarray(target)
+    B, K1, V = target.shape
+    K = K1 - 1
+    if draft is not None:
+        draft = np.ascontiguousarray(draft)
+        assert draft.shape == (B, K, V) and draft.dtype == target.dtype
+    toks = np.ascontiguousarray(draft_tokens, dtype=np.int32).reshape(B, K)
+    uniforms = np.asarray(uniforms)
+    wide = uniforms.dtype == np.float64  # double uniforms: exact-integration pins only
+    u = np.ascontiguousarray(uniforms, dtype=np.float64 if wide else np.float32).reshape(B, K + 1)
+    acc = np.zeros(B, np.int32)
+    out = np.zeros((B, K + 1), np.int32)
+    flags = np.zeros(B, np.int32)
+    fn = _load().oracle_verify_chain_f64u if wide else _load().oracle_verify_chain
+    rc = fn(_ptr(target), _ptr(draft), _dtype_code(target), B, K, V,
+            _ptr(toks), _ptr(u), float(temp), int(top_k), float(top_p),
+            _ptr(acc), _ptr(out), _ptr(flags), _threads(threads))
+    if rc != 0:
+        raise ValueError("oracle_verify_chain rejected its arguments")
+    return acc, out, flags
+
+
+def verify_tree_typical(target, node_tokens, parent_idx, eps, delta, temp=1.0, path_cap=None,
+                        threads=None):
+    """Typical acceptance over a candidate tree. target [B,N,V], node_tokens int32 [B,N],
+    parent_idx int32 [N]. Returns (best_path int32 [B,path_cap], accepted_len [B], flags [B])."""
+    target = np.ascontiguousarray(target)
+    B, N, V = target.shape
+    cap = N if path_cap is None else int(path_cap)
+    toks = np.ascontiguousarray(node_tokens, dtype=np.int32).reshape(B, N)
+    par = np.ascontiguousarray(parent_idx, dtype=np.int32).reshape(N)
+    path = np.zeros((B, cap), np.int32)
+    acc = np.zeros(B, np.int32)
+    flags = np.zeros(B, np.int32)
+    rc = _load().oracle_verify_tree_typical(_ptr(target), _dtype_code(target), B, N, V,
+                                            _ptr(toks), _ptr(par), float(eps), float(delta),
+                                            float(temp), _ptr(path), cap, _ptr(acc),
+                                            _ptr(flags), _threads(threads))
+    if rc != 0:
+        raise ValueError("oracle_verify_tree_typical rejected its arguments")
+    return path, acc, flags
+
+
+def residual_sample(p, q, uniforms, threads=None):
+    """Inverse-CDF draw per row from norm(max(0, p - q)) (q None: from p).
+    p, q float32 [rows, V]; uniforms float32 [rows]. Returns (tokens int32, flags int32)."""
+    p = np.ascontiguousarray(p, dtype=np.float32)
+    rows, V = p.shape
+    if q is not None:
+        q = np.ascontiguousarray(q, dtype=np.float32)
+        assert q.shape == p.shape
+    u = np.ascontiguousarray(uniforms, dtype=np.float32).reshape(rows)
+    toks = np.zeros(rows, np.int32)
+    flags = np.zeros(rows, np.int32)
+    rc = _load().oracle_residual_sample(_ptr(p), _ptr(q), rows, V, _ptr(u), _ptr(toks),
+                                        _ptr(flags), _threads(threads))
+    if rc != 0:
+        raise ValueError("oracle_residual_sample rejected its arguments")
+    return toks, flags

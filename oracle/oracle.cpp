@@ -1,0 +1,485 @@
+// Oracle for draft-token verification in speculative decoding.
+//
+// TEST INFRASTRUCTURE ONLY. This is a plain, slow, double-precision CPU
+// statement of what the verification step computes. Only the test suite, the
+// smoke check and the benchmark's CPU-baseline leg may load it; the library
+// under test never does, and the two share no code, header or table.
+//
+// Sources (cited by page and section):
+//   [SD]  taking-lying-flat.github.io/blog/posts/spec-decoding-i/ — notes on
+//         "Fast Inference from Transformers via Speculative Decoding"
+//         (section "Speculative Decoding"), "Accelerating Large Language Model
+//         Decoding with Speculative Sampling" (section "Speculative Sampling")
+//         and MEDUSA (section "Key Components").
+//   [SV]  blog.csdn.net/yorkhunter/article/details/139214590 — survey
+//         translation, section "推测解码" (blockwise parallel decoding,
+//         MEDUSA typical acceptance).
+// The pages lost their formulas in extraction; the surviving prose fixes the
+// structure, and the formulas used here are the standard ones that prose
+// describes: accept x with probability min(1, p(x)/q(x)), resample from
+// norm(max(0, p - q)), bonus token from p after K acceptances, MEDUSA typical
+// acceptance p(x) > min(eps, delta * exp(-H(p))).
+//
+// Readings where the pages are silent (each one is listed in the design notes):
+//   * p is the target distribution, q the draft distribution.
+//   * accept iff u < min(1, r), strict; r = +inf when q(x) = 0 < p(x), r = 0
+//     when both are 0.
+//   * uniforms per batch row: u[0..K-1] for the K accept tests, u[K] for the
+//     single resample-or-bonus draw.
+//   * transforms in the order temperature -> top-k -> softmax -> top-p ->
+//     renormalise; ties broken by the lower token id; the top-p crossing token
+//     is kept.
+//   * inverse CDF in ascending token id: the smallest v with res[v] > 0 and
+//     C_v > w * S; if rounding leaves none, the largest v with res[v] > 0.
+//   * an empty residual (p == q) falls back to p.
+//   * entropy in nats; tree: node 0 is accepted unconditionally, node c is
+//     tested with p at its parent, the deepest accepted node wins with the
+//     lowest index on ties.
+//   * a row holding NaN or +inf, or whose logits are all -inf, is invalid;
+//     a batch row that needs an invalid row, or an out-of-range token, is an
+//     error row (accepted_len = -1, all outputs -1).
+
+#include <algorithm>
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <limits>
+#include <thread>
+#include <vector>
+
+namespace {
+
+const double kInf = std::numeric_limits<double>::infinity();
+
+// Flag bits: decisions that fp32 and fp64 arithmetic may take differently.
+enum : int32_t {
+  FLAG_RATIO = 1,      // |u_i - r_i| < 1e-5 at a tested position
+  FLAG_CDF = 2,        // inverse-CDF boundary within 1e-6 * S of w * S
+  FLAG_TOPP = 4,       // top-p cumulative mass boundary within 1e-6 of top_p
+  FLAG_TREE = 8,       // |p - thr| / thr < 1e-5 at a tested tree node
+  DIAG_Q_ZERO = 16,    // a tested draft token had q(x) = 0 (not a parity flag)
+};
+
+double bf16_bits_to_double(uint16_t h) {
+  uint32_t u = uint32_t(h) << 16;
+  float f;
+  std::memcpy(&f, &u, sizeof f);
+  return double(f);
+}
+
+// dtype 0 = float32, 1 = bfloat16 (raw 16-bit patterns).
+void load_row(const void* base, int dtype, size_t row, int V, std::vector<double>& l) {
+  l.resize(size_t(V));
+  if (dtype == 0) {
+    const float* p = static_cast<const float*>(base) + row * size_t(V);
+    for (int v = 0; v < V; ++v) l[v] = double(p[v]);
+  } else {
+    const uint16_t* p = static_cast<const uint16_t*>(base) + row * size_t(V);
+    for (int v = 0; v < V; ++v) l[v] = bf16_bits_to_double(p[v]);
+  }
+}
+
+bool row_valid(const std::vector<double>& l) {
+  double mx = -kInf;
+  for (double x : l) {
+    if (std::isnan(x) || x == kInf) return false;
+    if (x > mx) mx = x;
+  }
+  return mx > -kInf;
+}
+
+int argmax_lowest(const std::vector<double>& l) {
+  int best = 0;
+  for (int v = 1; v < int(l.size()); ++v)
+    if (l[v] > l[best]) best = v;
+  return best;
+}
+
+struct Dist {
+  std::vector<double> p;
+  double entropy = 0.0;
+  double topp_margin = kInf;  // min distance of the nucleus boundary sums to top_p
+};
+
+// The sampling transform of [SD] "Speculative Sampling" (last bullet): the
+// probabilities are transformed first, then the rejection scheme applies.
+// Temperature T divides the logits; top-k keeps the k highest logits (lower id
+// first on ties); softmax over the kept set; top-p keeps the shortest prefix of
+// the probability-sorted kept tokens whose mass reaches top_p, then
+// renormalises. T == 0 is the greedy limit: a one-hot at the argmax.
+Dist transform(const std::vector<double>& l, double T, int top_k, double top_p) {
+  const int V = int(l.size());
+  Dist d;
+  d.p.assign(size_t(V), 0.0);
+  if (T == 0.0) {
+    d.p[argmax_lowest(l)] = 1.0;
+    return d;
+  }
+  std::vector<char> kept(static_cast<size_t>(V), 1);
+  if (top_k >= 1 && top_k < V) {
+    std::vector<int> order(static_cast<size_t>(V));
+    for (int v = 0; v < V; ++v) order[v] = v;
+    std::partial_sort(order.begin(), order.begin() + top_k, order.end(), [&](int a, int b) {
+      if (l[a] != l[b]) return l[a] > l[b];
+      return a < b;
+    });
+    std::fill(kept.begin(), kept.end(), 0);
+    for (int j = 0; j < top_k; ++j) kept[order[j]] = 1;
+  }
+  double zmax = -kInf;
+  for (int v = 0; v < V; ++v)
+    if (kept[v] && l[v] / T > zmax) zmax = l[v] / T;
+  std::vector<double> e(static_cast<size_t>(V), 0.0);
+  double Z = 0.0;
+  for (int v = 0; v < V; ++v)
+    if (kept[v]) {
+      e[v] = std::exp(l[v] / T - zmax);
+      Z += e[v];
+    }
+  for (int v = 0; v < V; ++v) d.p[v] = e[v] / Z;
+
+  if (top_p < 1.0) {
+    std::vector<int> order;
+    for (int v = 0; v < V; ++v)
+      if (kept[v]) order.push_back(v);
+    std::sort(order.begin(), order.end(), [&](int a, int b) {
+      if (d.p[a] != d.p[b]) return d.p[a] > d.p[b];
+      return a < b;
+    });
+    double cum = 0.0, prev = 0.0;
+    size_t n_keep = order.size();
+    for (size_t j = 0; j < order.size(); ++j) {
+      prev = cum;
+      cum += d.p[order[j]];
+      if (cum >= top_p) {
+        n_keep = j + 1;
+        break;
+      }
+    }
+    if (n_keep < order.size() || cum >= top_p)
+      d.topp_margin = std::min(std::fabs(cum - top_p), std::fabs(prev - top_p));
+    else
+      d.topp_margin = std::fabs(cum - top_p);
+    std::fill(kept.begin(), kept.end(), 0);
+    for (size_t j = 0; j < n_keep; ++j) kept[order[j]] = 1;
+    double Zp = 0.0;
+    for (int v = 0; v < V; ++v)
+      if (kept[v]) Zp += e[v];
+    for (int v = 0; v < V; ++v) d.p[v] = kept[v] ? e[v] / Zp : 0.0;
+  }
+  double H = 0.0;
+  for (int v = 0; v < V; ++v)
+    if (d.p[v] > 0.0) H -= d.p[v] * std::log(d.p[v]);
+  d.entropy = H;
+  return d;
+}
+
+struct Draw {
+  int token = -1;
+  bool flag = false;
+};
+
+// Inverse-CDF draw in ascending token id: the smallest v with res[v] > 0 whose
+// cumulative sum exceeds w * S. If rounding leaves none, the largest v with
+// res[v] > 0 is taken (and the draw is flagged as sitting on an edge).
+Draw inverse_cdf(const std::vector<double>& res, double w) {
+  Draw out;
+  double S = 0.0;
+  for (double r : res) S += r;
+  const double target = w * S;
+  double C = 0.0;
+  for (int v = 0; v < int(res.size()); ++v) {
+    const double before = C;
+    C += res[v];
+    if (res[v] > 0.0 && C > target) {
+      out.token = v;
+      out.flag = std::fabs(before - target) < 1e-6 * S || std::fabs(C - target) < 1e-6 * S;
+      return out;
+    }
+  }
+  for (int v = int(res.size()) - 1; v >= 0; --v)
+    if (res[v] > 0.0) {
+      out.token = v;
+      out.flag = true;
+      return out;
+    }
+  return out;
+}
+
+// Residual distribution of [SD] "Speculative Decoding": after rejecting x at
+// position i, resample from norm(max(0, p_i - q_i)); an empty residual (only
+// possible when p_i == q_i) falls back to p_i.
+std::vector<double> residual(const std::vector<double>& p, const std::vector<double>& q) {
+  std::vector<double> r(p.size());
+  double S = 0.0;
+  for (size_t v = 0; v < p.size(); ++v) {
+    r[v] = std::max(0.0, p[v] - q[v]);
+    S += r[v];
+  }
+  if (S == 0.0) return p;
+  return r;
+}
+
+struct ChainArgs {
+  const void* target;
+  const void* draft;
+  int dtype, B, K, V;
+  const int32_t* draft_tokens;
+  const double* uniforms;
+  double T;
+  int top_k;
+  double top_p;
+  int32_t* accepted_len;
+  int32_t* out_tokens;
+  int32_t* flags;
+};
+
+void chain_error(const ChainArgs& a, int b) {
+  a.accepted_len[b] = -1;
+  for (int j = 0; j <= a.K; ++j) a.out_tokens[size_t(b) * (a.K + 1) + j] = -1;
+}
+
+// One batch row of chain verification: [SD] "Speculative Decoding" (accept
+// x_i left to right, stop at the first rejection and resample it, bonus token
+// after K acceptances) and "Speculative Sampling" (the acceptance ratio and
+// the residual). T == 0 is the greedy longest-prefix rule of blockwise
+// parallel decoding ([SV], "推测解码").
+void chain_row(const ChainArgs& a, int b) {
+  const int K = a.K, V = a.V;
+  const int32_t* x = a.draft_tokens + size_t(b) * K;
+  const double* u = a.uniforms + size_t(b) * (K + 1);
+  int32_t* out = a.out_tokens + size_t(b) * (K + 1);
+  int32_t flag = 0;
+  std::vector<double> lp, lq;
+  int acc = K;
+  int emitted = -1;
+
+  if (a.T == 0.0) {
+    for (int i = 0; i <= K; ++i) {
+      load_row(a.target, a.dtype, size_t(b) * (K + 1) + i, V, lp);
+      if (!row_valid(lp)) return chain_error(a, b);
+      const int g = argmax_lowest(lp);
+      if (i == K) {
+        emitted = g;
+        break;
+      }
+      if (x[i] < 0 || x[i] >= V) return chain_error(a, b);
+      if (x[i] != g) {
+        acc = i;
+        emitted = g;
+        break;
+      }
+    }
+  } else {
+    for (int i = 0; i <= K; ++i) {
+      load_row(a.target, a.dtype, size_t(b) * (K + 1) + i, V, lp);
+      if (!row_valid(lp)) return chain_error(a, b);
+      const Dist P = transform(lp, a.T, a.top_k, a.top_p);
+      if (P.topp_margin < 1e-6) flag |= FLAG_TOPP;
+      if (i == K) {  // every draft accepted: bonus token from p at position K+1
+        const Draw d = inverse_cdf(P.p, u[K]);
+        emitted = d.token;
+        if (d.flag) flag |= FLAG_CDF;
+        break;
+      }
+      if (x[i] < 0 || x[i] >= V) return chain_error(a, b);
+      load_row(a.draft, a.dtype, size_t(b) * K + i, V, lq);
+      if (!row_valid(lq)) return chain_error(a, b);
+      const Dist Q = transform(lq, a.T, a.top_k, a.top_p);
+      if (Q.topp_margin < 1e-6) flag |= FLAG_TOPP;
+      const double px = P.p[x[i]], qx = Q.p[x[i]];
+      double r;
+      if (qx > 0.0) {
+        r = px / qx;
+      } else {
+        r = px > 0.0 ? kInf : 0.0;
+        flag |= DIAG_Q_ZERO;
+      }
+      const double ui = u[i];
+      if (std::isfinite(r) && std::fabs(ui - r) < 1e-5) flag |= FLAG_RATIO;
+      if (ui < std::min(1.0, r)) continue;
+      acc = i;
+      const Draw d = inverse_cdf(residual(P.p, Q.p), u[K]);
+      emitted = d.token;
+      if (d.flag) flag |= FLAG_CDF;
+      break;
+    }
+  }
+  a.accepted_len[b] = acc;
+  for (int j = 0; j < acc; ++j) out[j] = x[j];
+  out[acc] = emitted;
+  for (int j = acc + 1; j <= K; ++j) out[j] = -1;
+  if (a.flags) a.flags[b] = flag;
+}
+
+template <class F>
+void parallel_rows(int n, int threads, F&& f) {
+  if (threads <= 1 || n <= 1) {
+    for (int i = 0; i < n; ++i) f(i);
+    return;
+  }
+  threads = std::min(threads, n);
+  std::vector<std::thread> pool;
+  for (int t = 0; t < threads; ++t)
+    pool.emplace_back([&, t] {
+      for (int i = t; i < n; i += threads) f(i);
+    });
+  for (auto& th : pool) th.join();
+}
+
+}  // namespace
+
+extern "C" {
+
+// Transform rows of logits into probabilities (double) and entropies (nats).
+// valid[r] = 0 marks an invalid row (its probabilities are left at 0).
+int oracle_transform_rows(const void* logits, int dtype, int rows, int V, double T, int top_k,
+                          double top_p, double* probs, double* entropy, double* topp_margin,
+                          int32_t* valid, int threads) {
+  if (!logits || rows < 0 || V <= 0 || !(T >= 0.0)) return -1;
+  parallel_rows(rows, threads, [&](int r) {
+    std::vector<double> l;
+    load_row(logits, dtype, size_t(r), V, l);
+    double* pr = probs ? probs + size_t(r) * V : nullptr;
+    if (!row_valid(l)) {
+      if (pr) std::fill(pr, pr + V, 0.0);
+      if (entropy) entropy[r] = 0.0;
+      if (topp_margin) topp_margin[r] = kInf;
+      if (valid) valid[r] = 0;
+      return;
+    }
+    const Dist d = transform(l, T, top_k, top_p);
+    if (pr) std::copy(d.p.begin(), d.p.end(), pr);
+    if (entropy) entropy[r] = d.entropy;
+    if (topp_margin) topp_margin[r] = d.topp_margin;
+    if (valid) valid[r] = 1;
+  });
+  return 0;
+}
+
+// Chain verification over B batch rows (see chain_row), with the uniforms
+// given in double precision. flags may be NULL.
+int oracle_verify_chain_f64u(const void* target, const void* draft, int dtype, int B, int K,
+                             int V, const int32_t* draft_tokens, const double* uniforms, double T,
+                             int top_k, double top_p, int32_t* accepted_len, int32_t* out_tokens,
+                             int32_t* flags, int threads) {
+  if (!target || (T != 0.0 && !draft) || B < 0 || K < 0 || V <= 0 || !draft_tokens ||
+      !uniforms || !accepted_len || !out_tokens || !(T >= 0.0))
+    return -1;
+  ChainArgs a{target, draft, dtype, B, K, V, draft_tokens, uniforms, T, top_k, top_p,
+              accepted_len, out_tokens, flags};
+  parallel_rows(B, threads, [&](int b) { chain_row(a, b); });
+  return 0;
+}
+
+// The same with float32 uniforms (the library's interface); each is widened
+// exactly to double.
+int oracle_verify_chain(const void* target, const void* draft, int dtype, int B, int K, int V,
+                        const int32_t* draft_tokens, const float* uniforms, double T, int top_k,
+                        double top_p, int32_t* accepted_len, int32_t* out_tokens, int32_t* flags,
+                        int threads) {
+  if (!uniforms || B < 0 || K < 0) return -1;
+  std::vector<double> u(size_t(B) * size_t(K + 1));
+  for (size_t j = 0; j < u.size(); ++j) u[j] = double(uniforms[j]);
+  return oracle_verify_chain_f64u(target, draft, dtype, B, K, V, draft_tokens, u.data(), T, top_k,
+                                  top_p, accepted_len, out_tokens, flags, threads);
+}
+
+// MEDUSA typical acceptance over a candidate tree ([SD] "Key Components";
+// [SV] "推测解码"). Node n's logits give the next-token distribution after n;
+// node 0 (the greedy first token) is accepted unconditionally; node c >= 1 is
+// accepted iff its parent is and p_parent(tok_c) > min(eps, delta *
+// exp(-H(p_parent))). The deepest accepted node (lowest index on ties) and its
+// root-first ancestor chain are returned. T is the softmax temperature (1 in
+// the library's interface; 0 gives the greedy limit).
+int oracle_verify_tree_typical(const void* target, int dtype, int B, int N, int V,
+                               const int32_t* node_tokens, const int32_t* parent_idx, double eps,
+                               double delta, double T, int32_t* best_path, int path_cap,
+                               int32_t* accepted_len, int32_t* flags, int threads) {
+  if (!target || B < 0 || N <= 0 || V <= 0 || !node_tokens || !parent_idx || !best_path ||
+      path_cap <= 0 || !accepted_len || !(T >= 0.0))
+    return -1;
+  bool tree_ok = parent_idx[0] == -1;
+  std::vector<int> depth(static_cast<size_t>(N), 0);
+  for (int c = 1; c < N && tree_ok; ++c) {
+    const int pa = parent_idx[c];
+    if (pa < 0 || pa >= c)
+      tree_ok = false;
+    else
+      depth[c] = depth[pa] + 1;
+  }
+  parallel_rows(B, threads, [&](int b) {
+    int32_t* path = best_path + size_t(b) * path_cap;
+    auto fail = [&]() {
+      accepted_len[b] = -1;
+      for (int j = 0; j < path_cap; ++j) path[j] = -1;
+      if (flags) flags[b] = 0;
+    };
+    if (!tree_ok) return fail();
+    int32_t flag = 0;
+    std::vector<char> acc(static_cast<size_t>(N), 0);
+    std::vector<char> have(static_cast<size_t>(N), 0);
+    std::vector<Dist> dist(static_cast<size_t>(N));
+    acc[0] = 1;
+    std::vector<double> l;
+    for (int c = 1; c < N; ++c) {
+      const int pa = parent_idx[c];
+      if (!acc[pa]) continue;
+      if (!have[pa]) {
+        load_row(target, dtype, size_t(b) * N + pa, V, l);
+        if (!row_valid(l)) return fail();
+        dist[pa] = transform(l, T, 0, 1.0);
+        have[pa] = 1;
+      }
+      const int tok = node_tokens[size_t(b) * N + c];
+      if (tok < 0 || tok >= V) return fail();
+      const double p = dist[pa].p[tok];
+      const double thr = std::min(eps, delta * std::exp(-dist[pa].entropy));
+      if (thr > 0.0 && std::fabs(p - thr) / thr < 1e-5) flag |= FLAG_TREE;
+      acc[c] = p > thr;
+    }
+    int best = 0;
+    for (int c = 1; c < N; ++c)
+      if (acc[c] && depth[c] > depth[best]) best = c;
+    const int len = depth[best] + 1;
+    if (len > path_cap) return fail();
+    for (int j = 0; j < path_cap; ++j) path[j] = -1;
+    for (int n = best, j = len - 1; j >= 0; --j, n = (n > 0 ? parent_idx[n] : -1)) path[j] = n;
+    accepted_len[b] = len;
+    if (flags) flags[b] = flag;
+  });
+  return 0;
+}
+
+// Inverse-CDF draw from norm(max(0, p - q)) (q == NULL: from p) for explicit
+// probability rows. Rows holding a negative, NaN or infinite entry, or with
+// no positive mass, give token -1.
+int oracle_residual_sample(const float* p, const float* q, int rows, int V, const float* uniforms,
+                           int32_t* tokens, int32_t* flags, int threads) {
+  if (!p || rows < 0 || V <= 0 || !uniforms || !tokens) return -1;
+  parallel_rows(rows, threads, [&](int r) {
+    std::vector<double> pr(static_cast<size_t>(V)), qr(size_t(V), 0.0);
+    bool ok = true;
+    for (int v = 0; v < V; ++v) {
+      pr[v] = double(p[size_t(r) * V + v]);
+      if (!(pr[v] >= 0.0) || pr[v] == kInf) ok = false;
+      if (q) {
+        qr[v] = double(q[size_t(r) * V + v]);
+        if (!(qr[v] >= 0.0) || qr[v] == kInf) ok = false;
+      }
+    }
+    double mass = 0.0;
+    for (double x : pr) mass += x;
+    if (!ok || !(mass > 0.0)) {
+      tokens[r] = -1;
+      if (flags) flags[r] = 0;
+      return;
+    }
+    const Draw d = inverse_cdf(q ? residual(pr, qr) : pr, double(uniforms[r]));
+    tokens[r] = d.token;
+    if (flags) flags[r] = d.flag ? FLAG_CDF : 0;
+  });
+  return 0;
+}
+
+}  // extern "C"

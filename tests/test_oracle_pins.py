@@ -1,0 +1,436 @@
+"""Pins of the oracle to what the pages and the mathematics fix (no GPU).
+
+Sources: taking-lying-flat.github.io/blog/posts/spec-decoding-i/ (sections
+"Speculative Decoding", "Speculative Sampling", "Key Components") and
+blog.csdn.net/yorkhunter/article/details/139214590 (section "推测解码").
+Each test names the property it pins; none re-types the oracle's formula.
+"""
+from __future__ import annotations
+
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+from scipy.special import softmax
+from scipy.stats import chisquare
+from scipy.stats import entropy as scipy_entropy
+
+import oracle
+import specgen
+from tests._helpers import chain_case, check_chain_invariants, draft_tokens, f32_logits, to_f64
+
+GOLD = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
+
+
+def _load(name):
+    with open(os.path.join(GOLD, name)) as f:
+        return json.load(f)
+
+
+# --------------------------------------------------------------------------- golden (hand-derived)
+
+@pytest.mark.parametrize("case", _load("chain_handworked.json")["cases"], ids=lambda c: c["name"])
+def test_golden_chain(case):
+    target = f32_logits(case["target"])[None]
+    K = target.shape[1] - 1
+    draft = None if case["draft"] is None else f32_logits(case["draft"])[None]
+    toks = np.array([case["tokens"]], np.int32)
+    u = np.array([case["u"]], np.float32)
+    acc, out, _ = oracle.verify_chain(target, draft, toks, u, case["temp"])
+    assert int(acc[0]) == case["accepted_len"]
+    assert out[0].tolist() == case["out"]
+    assert K == len(case["tokens"])
+
+
+@pytest.mark.parametrize("case", _load("transform_handworked.json")["cases"],
+                         ids=lambda c: c["name"])
+def test_golden_transform(case):
+    logits = f32_logits([case["logits"]])
+    probs, _, _, valid = oracle.transform_rows(logits, case["temp"], case["top_k"], case["top_p"])
+    expect = np.array([eval(s, {"e": math.e}) for s in case["expect"]], np.float64)
+    assert valid[0] == 1
+    np.testing.assert_allclose(probs[0], expect, rtol=0, atol=case["tol"])
+
+
+@pytest.mark.parametrize("case", _load("tree_handworked.json")["cases"], ids=lambda c: c["name"])
+def test_golden_tree(case):
+    logits = f32_logits(case["logits"])[None]
+    toks = np.array([case["tokens"]], np.int32)
+    par = np.array(case["parent"], np.int32)
+    path, acc, _ = oracle.verify_tree_typical(logits, toks, par, case["eps"], case["delta"])
+    assert int(acc[0]) == case["accepted_len"]
+    n = case["accepted_len"]
+    assert path[0, :n].tolist() == case["path"]
+    assert np.all(path[0, n:] == -1)
+
+
+# --------------------------------------------------------------------------- T1: exact enumeration
+
+def _bisect(pred, n, iters=70):
+    """Boundary t_j in [0,1] of n monotone predicates (False below t_j, True from t_j on)."""
+    lo, hi = np.zeros(n), np.ones(n)
+    at_zero = pred(np.zeros(n))
+    for _ in range(iters):
+        mid = 0.5 * (lo + hi)
+        r = pred(mid)
+        hi = np.where(r, mid, hi)
+        lo = np.where(r, lo, mid)
+    return np.where(at_zero, 0.0, hi)
+
+
+def _enumerate_chain(V, temp, top_k, top_p, seed, ties=False):
+    """Exact output law of one K=2 round, integrated over (u_0, u_1, w) by locating every
+    decision boundary of the oracle (black box) to double precision."""
+    g = np.random.default_rng(seed)
+
+    def logits(*shape):
+        x = g.normal(0.0, 1.5, size=shape)
+        if ties:
+            x = np.round(x * 2) / 2
+        return x.astype(np.float32)
+
+    t1, d1 = logits(V), logits(V)
+    t2, d2 = logits(V, V), logits(V, V)          # indexed by x1
+    t3 = logits(V, V, V)                        # indexed by (x1, x2)
+    X1, X2 = np.meshgrid(np.arange(V), np.arange(V), indexing="ij")
+    X1, X2 = X1.ravel(), X2.ravel()
+    n = V * V
+    target = np.stack([np.broadcast_to(t1, (n, V)), t2[X1], t3[X1, X2]], axis=1).copy()
+    draft = np.stack([np.broadcast_to(d1, (n, V)), d2[X1]], axis=1).copy()
+    toks = np.stack([X1, X2], axis=1).astype(np.int32)
+
+    def run(u0, u1, w):
+        u = np.stack([np.broadcast_to(u0, (n,)), np.broadcast_to(u1, (n,)),
+                      np.broadcast_to(w, (n,))], axis=1).astype(np.float64)
+        acc, out, _ = oracle.verify_chain(target, draft, toks, u, temp, top_k, top_p, threads=1)
+        return acc, out
+
+    below1 = 1.0 - 2.0 ** -53
+    tau1 = _bisect(lambda u: run(u, 0.0, 0.5)[0] < 1, n)
+    tau2 = _bisect(lambda u: run(0.0, u, 0.5)[0] < 2, n)
+
+    def law(u0, u1, slot):
+        b = np.zeros((n, V + 1))
+        b[:, V] = 1.0
+        for v in range(1, V):
+            b[:, v] = _bisect(lambda w: run(u0, u1, w)[1][:, slot] >= v, n)
+        return np.diff(b, axis=1)  # [n, V] probability of each token
+
+    R1 = law(below1, 0.0, 0)
+    R2 = law(0.0, below1, 1)
+    BON = law(0.0, 0.0, 2)
+
+    def tp(rows):
+        return oracle.transform_rows(rows, temp, top_k, top_p)[0]
+
+    P1, Q1 = tp(t1[None])[0], tp(d1[None])[0]
+    P2, Q2, P3 = tp(t2), tp(d2), tp(t3.reshape(V * V, V)).reshape(V, V, V)
+    return dict(V=V, X1=X1, X2=X2, tau1=tau1, tau2=tau2, R1=R1, R2=R2, BON=BON,
+                P1=P1, Q1=Q1, P2=P2, Q2=Q2, P3=P3, t1=t1, t2=t2, t3=t3)
+
+
+def _check_law(E, atol=1e-12):
+    V, X1, X2 = E["V"], E["X1"], E["X2"]
+    P1, Q1, P2, Q2, P3 = E["P1"], E["Q1"], E["P2"], E["Q2"], E["P3"]
+    first = np.zeros(V)
+    for x1 in range(V):
+        j = x1 * V  # any x2: position-1 decisions do not depend on x2
+        first[x1] += Q1[x1] * E["tau1"][j]
+        first += Q1[x1] * (1.0 - E["tau1"][j]) * E["R1"][j]
+    np.testing.assert_allclose(first, P1, rtol=0, atol=atol)
+    for x1 in range(V):
+        if Q1[x1] * E["tau1"][x1 * V] == 0.0:
+            continue
+        second = np.zeros(V)
+        for x2 in range(V):
+            j = x1 * V + x2
+            second[x2] += Q2[x1, x2] * E["tau2"][j]
+            second += Q2[x1, x2] * (1.0 - E["tau2"][j]) * E["R2"][j]
+        np.testing.assert_allclose(second, P2[x1], rtol=0, atol=atol)
+    for j in range(V * V):
+        if E["tau1"][j] * E["tau2"][j] > 0.0:
+            np.testing.assert_allclose(E["BON"][j], P3[X1[j], X2[j]], rtol=0, atol=atol)
+
+
+def test_T1_exact_law_equals_target_no_transform():
+    """Each emitted token follows p exactly, whatever q is (distribution preservation,
+    'Speculative Decoding' / 'Speculative Sampling'); here p and q are plain softmaxes,
+    checked against scipy's softmax."""
+    E = _enumerate_chain(V=8, temp=1.0, top_k=0, top_p=1.0, seed=11)
+    np.testing.assert_allclose(E["P1"], softmax(E["t1"].astype(np.float64)), rtol=1e-14)
+    _check_law(E)
+
+
+@pytest.mark.parametrize("temp,top_k,top_p,ties", [(0.7, 0, 1.0, False), (1.0, 3, 1.0, True),
+                                                  (1.3, 0, 0.8, False), (0.9, 5, 0.7, True)])
+def test_T1_exact_law_equals_transformed_target(temp, top_k, top_p, ties):
+    """With temperature/top-k/top-p the emitted tokens follow the transformed p
+    ('Speculative Sampling', last bullet)."""
+    E = _enumerate_chain(V=8, temp=temp, top_k=top_k, top_p=top_p, seed=23, ties=ties)
+    _check_law(E)
+
+
+# --------------------------------------------------------------------------- T2: p == q
+
+@pytest.mark.parametrize("temp,top_k,top_p", [(1.0, 0, 1.0), (0.8, 7, 1.0), (1.2, 0, 0.85)])
+def test_T2_equal_distributions_always_accept(temp, top_k, top_p):
+    """With identical target and draft distributions the ratio rule accepts with
+    probability 1 ('Key Components', contrast with independent sampling)."""
+    g = np.random.default_rng(5)
+    B, K, V = 64, 4, 40
+    target = g.normal(0, 2, size=(B, K + 1, V)).astype(np.float32)
+    draft = target[:, :K].copy()
+    toks = g.integers(0, V, size=(B, K)).astype(np.int32)
+    probs = oracle.transform_rows(draft, temp, top_k, top_p)[0]
+    for b in range(B):                       # keep draft tokens inside q's support
+        for i in range(K):
+            if probs[b, i, toks[b, i]] == 0.0:
+                toks[b, i] = int(np.argmax(probs[b, i]))
+    u = g.random((B, K + 1)).astype(np.float32)
+    u[:, :K] = np.minimum(u[:, :K], np.float32(1.0 - 2 ** -24))
+    acc, out, _ = oracle.verify_chain(target, draft, toks, u, temp, top_k, top_p)
+    assert np.all(acc == K)
+    assert np.array_equal(out[:, :K], toks)
+
+
+# --------------------------------------------------------------------------- T3: emit count
+
+@pytest.mark.parametrize("cfg", [specgen.CFG1, specgen.CFG2, specgen.CFG3, specgen.CFG5],
+                         ids=lambda c: c.name)
+def test_T3_emit_count_on_workloads(cfg):
+    """Every round emits at least 1 and at most K+1 tokens ('Speculative Sampling')."""
+    B = min(cfg.B, 3)
+    target, draft, toks, u, temp = chain_case(cfg, B)
+    acc, out, flags = oracle.verify_chain(target, draft, toks, u, temp, cfg.top_k, cfg.top_p)
+    check_chain_invariants(acc, out, toks, cfg.K, cfg.V)
+
+
+# --------------------------------------------------------------------------- T4: greedy
+
+def test_T4_greedy_is_longest_argmax_prefix():
+    """Temperature 0: keep the longest prefix equal to the target's greedy predictions
+    (blockwise parallel decoding in '推测解码'), ties to the lowest id as numpy.argmax does."""
+    g = np.random.default_rng(7)
+    B, K, V = 200, 6, 30
+    vals = np.round(g.normal(0, 1, size=(B, K + 1, V)) * 2) / 2   # many ties
+    target = specgen.f32_to_bf16_bits(vals.astype(np.float32))
+    am = np.argmax(to_f64(target), axis=2)
+    toks = np.where(g.random((B, K)) < 0.8, am[:, :K], g.integers(0, V, (B, K))).astype(np.int32)
+    u = g.random((B, K + 1)).astype(np.float32)
+    acc, out, _ = oracle.verify_chain(target, None, toks, u, 0.0)
+    for b in range(B):
+        a = 0
+        while a < K and toks[b, a] == am[b, a]:
+            a += 1
+        assert acc[b] == a
+        assert out[b, :a].tolist() == toks[b, :a].tolist()
+        assert out[b, a] == am[b, a]
+        assert np.all(out[b, a + 1:] == -1)
+
+
+# --------------------------------------------------------------------------- T5: transforms
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("temp", [0.3, 1.0, 2.5])
+def test_T5_identity_transform_is_softmax(dtype, temp):
+    g = np.random.default_rng(3)
+    x = g.normal(0, 3, size=(20, 257)).astype(np.float32)
+    logits = specgen.f32_to_bf16_bits(x) if dtype == "bf16" else x
+    for k, p in [(0, 1.0), (257, 1.0), (-1, 1.0), (0, 1.5)]:
+        probs, ent, _, valid = oracle.transform_rows(logits, temp, k, p)
+        ref = softmax(to_f64(logits) / temp, axis=1)
+        np.testing.assert_allclose(probs, ref, rtol=1e-13, atol=1e-300)
+        np.testing.assert_allclose(probs.sum(1), 1.0, rtol=0, atol=1e-14)
+        np.testing.assert_allclose(ent, scipy_entropy(ref, axis=1), rtol=1e-9, atol=1e-14)
+        assert valid.all()
+
+
+def test_T5_topk_is_renormalised_lexsort_prefix():
+    g = np.random.default_rng(4)
+    V = 64
+    x = np.round(g.normal(0, 1, size=(50, V)) * 3) / 3          # ties
+    logits = specgen.f32_to_bf16_bits(x.astype(np.float32))
+    l = to_f64(logits)
+    for k in (1, 2, 5, 17, 63):
+        probs = oracle.transform_rows(logits, 0.8, k, 1.0)[0]
+        for r in range(l.shape[0]):
+            keep = np.lexsort((np.arange(V), -l[r]))[:k]
+            ref = np.zeros(V)
+            ref[keep] = softmax(l[r, keep] / 0.8)
+            np.testing.assert_allclose(probs[r], ref, rtol=1e-13, atol=1e-300)
+
+
+def test_T5_topp_keeps_tokens_whose_preceding_mass_is_below_top_p():
+    """Nucleus = the tokens whose exclusive cumulative mass (in descending-probability,
+    ascending-id order) is below top_p: the same set as 'shortest prefix reaching top_p'."""
+    g = np.random.default_rng(9)
+    V = 48
+    x = np.round(g.normal(0, 1.2, size=(80, V)) * 4) / 4
+    logits = x.astype(np.float32)
+    l = logits.astype(np.float64)
+    for top_p in (0.05, 0.5, 0.9, 0.999):
+        probs, _, marg, _ = oracle.transform_rows(logits, 1.0, 0, top_p)
+        for r in range(l.shape[0]):
+            base = softmax(l[r])
+            order = np.lexsort((np.arange(V), -base))
+            excl = np.concatenate([[0.0], np.cumsum(base[order])[:-1]])
+            keep = order[excl < top_p]
+            ref = np.zeros(V)
+            ref[keep] = base[keep] / base[keep].sum()
+            if marg[r] > 1e-9:
+                np.testing.assert_allclose(probs[r], ref, rtol=1e-12, atol=1e-300)
+
+
+def test_T5_entropy_closed_forms():
+    V = 1000
+    uniform = np.zeros((1, V), np.float32)
+    _, ent, _, _ = oracle.transform_rows(uniform, 1.0)
+    assert abs(ent[0] - math.log(V)) < 1e-12
+    onehot = np.full((1, V), -np.inf, np.float32)
+    onehot[0, 17] = 3.0
+    probs, ent, _, valid = oracle.transform_rows(onehot, 1.0)
+    assert valid[0] == 1 and ent[0] == 0.0 and probs[0, 17] == 1.0
+    _, ent_k, _, _ = oracle.transform_rows(uniform, 1.0, top_k=10)
+    assert abs(ent_k[0] - math.log(10)) < 1e-12
+
+
+def test_T5_bf16_decoding_and_invalid_rows():
+    bits = np.array([[0x3F80, 0x0000, 0xC000, 0xFF80]], np.uint16)   # 1, 0, -2, -inf
+    probs, _, _, valid = oracle.transform_rows(bits, 1.0)
+    ref = softmax(np.array([1.0, 0.0, -2.0, -np.inf]))
+    np.testing.assert_allclose(probs[0], ref, rtol=1e-15)
+    bad = np.array([[0x7FC0, 0, 0, 0], [0x7F80, 0, 0, 0], [0xFF80] * 4, [0xFFC0, 0, 0, 0]],
+                   np.uint16)                                      # NaN, +inf, all -inf, -NaN
+    _, _, _, valid = oracle.transform_rows(bad, 1.0)
+    assert valid.tolist() == [0, 0, 0, 0]
+
+
+def test_T5_greedy_limit_is_onehot():
+    logits = np.array([[1.0, 3.0, 3.0, 2.0]], np.float32)
+    probs, ent, _, _ = oracle.transform_rows(logits, 0.0)
+    assert probs[0].tolist() == [0.0, 1.0, 0.0, 0.0] and ent[0] == 0.0
+
+
+# --------------------------------------------------------------------------- T6/T7: tree
+
+def _random_tree(g, N):
+    par = np.array([-1] + [int(g.integers(0, c)) for c in range(1, N)], np.int32)
+    return par
+
+
+def _tree_brute(l, toks, par, eps, delta, temp):
+    """Evaluate the typical criterion on every edge of every root-to-node path."""
+    N, V = l.shape
+    def dist(n):
+        if temp == 0.0:
+            p = np.zeros(V)
+            p[np.argmax(l[n])] = 1.0
+            return p, 0.0
+        p = softmax(l[n] / temp)
+        return p, scipy_entropy(p)
+    ok = np.zeros(N, bool)
+    for c in range(1, N):
+        p, H = dist(par[c])
+        ok[c] = p[toks[c]] > min(eps, delta * math.exp(-H))
+    best, best_depth = 0, 0
+    for c in range(1, N):
+        path, n = [], c
+        while n > 0:
+            path.append(n)
+            n = par[n]
+        if all(ok[m] for m in path) and len(path) > best_depth:
+            best, best_depth = c, len(path)
+    path, n = [best], best
+    while n > 0:
+        n = par[n]
+        path.append(n)
+    return path[::-1]
+
+
+@pytest.mark.parametrize("seed", range(6))
+def test_T6_tree_matches_path_enumeration(seed):
+    g = np.random.default_rng(100 + seed)
+    B, N, V = 6, 14, 16
+    par = _random_tree(g, N)
+    toks = g.integers(0, V, size=(B, N)).astype(np.int32)
+    x = g.normal(0, 1.5, size=(B, N, V))
+    for b in range(B):                    # favour children's tokens so paths get deep
+        for c in range(1, N):
+            if g.random() < 0.7:
+                x[b, par[c], toks[b, c]] += 2.5
+    logits = x.astype(np.float32)
+    eps, delta = 0.09, 0.3
+    path, acc, _ = oracle.verify_tree_typical(logits, toks, par, eps, delta)
+    for b in range(B):
+        ref = _tree_brute(logits[b].astype(np.float64), toks[b], par, eps, delta, 1.0)
+        assert acc[b] == len(ref)
+        assert path[b, :len(ref)].tolist() == ref
+
+
+@pytest.mark.parametrize("seed", range(3))
+def test_T7_tree_at_temperature_zero_is_greedy(seed):
+    """At temperature 0 typical acceptance reduces to greedy matching ('Key Components')."""
+    g = np.random.default_rng(200 + seed)
+    B, N, V = 8, 12, 10
+    par = _random_tree(g, N)
+    l = g.permuted(np.tile(np.arange(V, dtype=np.float64), (B, N, 1)), axis=2)  # distinct
+    am = np.argmax(l, axis=2)
+    toks = np.where(g.random((B, N)) < 0.6, am[np.arange(B)[:, None], par[None, :].clip(0)],
+                    g.integers(0, V, (B, N))).astype(np.int32)
+    logits = l.astype(np.float32)
+    for temp in (0.0, 1e-3):
+        path, acc, _ = oracle.verify_tree_typical(logits, toks, par, 0.09, 0.3, temp=temp)
+        for b in range(B):
+            ref = _tree_brute(l[b], toks[b], par, 0.09, 0.3, 0.0)
+            # greedy matching: accepted iff every token on the path equals its parent's argmax
+            for n in ref[1:]:
+                assert toks[b, n] == np.argmax(l[b, par[n]])
+            assert path[b, :len(ref)].tolist() == ref and acc[b] == len(ref)
+
+
+def test_tree_workload_structure_and_invalid_parent():
+    par, depth, rank = specgen.tree_structure((4, 3, 2, 2), 64)
+    assert np.bincount(depth).tolist() == [1, 4, 12, 24, 23]
+    assert par[0] == -1 and np.all(par[1:] < np.arange(1, 64)) and np.all(par[1:] >= 0)
+    logits = np.zeros((2, 3, 4), np.float32)
+    toks = np.zeros((2, 3), np.int32)
+    path, acc, _ = oracle.verify_tree_typical(logits, toks, np.array([-1, 2, 0], np.int32),
+                                              0.09, 0.3)
+    assert acc.tolist() == [-1, -1] and np.all(path == -1)
+
+
+# --------------------------------------------------------------------------- errors
+
+def test_chain_error_rows_are_procedural():
+    """An invalid row or token only matters once the scan reaches it."""
+    V, K = 6, 3
+    target = np.zeros((3, K + 1, V), np.float32)
+    draft = np.zeros((3, K, V), np.float32)
+    draft[:, :, 0] = 5.0                      # q concentrated on token 0, p uniform
+    toks = np.zeros((3, K), np.int32)         # r = (1/6)/q(0) < 1
+    u = np.full((3, K + 1), 0.999, np.float32)  # reject at position 0
+    target[1, 2, 0] = np.nan                  # after the stop: harmless
+    toks[2, 0] = V                            # at the first test: error
+    acc, out, _ = oracle.verify_chain(target, draft, toks, u, 1.0)
+    assert acc.tolist() == [0, 0, -1]
+    assert np.all(out[2] == -1)
+
+
+# --------------------------------------------------------------------------- T8: Monte Carlo
+
+def test_T8_monte_carlo_first_token_frequencies():
+    """Sanity (not a pin): emitted first tokens over many seeded rounds follow p_1."""
+    g = np.random.default_rng(12)
+    B, K, V = 20000, 3, 20
+    t = g.normal(0, 1.5, size=(K + 1, V)).astype(np.float32)
+    d = (t[:K] + g.normal(0, 1.0, size=(K, V))).astype(np.float32)
+    target = np.broadcast_to(t, (B, K + 1, V)).copy()
+    draft = np.broadcast_to(d, (B, K, V)).copy()
+    toks = draft_tokens(draft, 1.0, 0, 1.0, g.random((B, K)).astype(np.float32), 4096)
+    u = g.random((B, K + 1)).astype(np.float32)
+    acc, out, _ = oracle.verify_chain(target, draft, toks, u, 1.0)
+    counts = np.bincount(out[:, 0], minlength=V)
+    p1 = softmax(t[0].astype(np.float64))
+    assert chisquare(counts, p1 * B).pvalue > 1e-4
