@@ -1,0 +1,149 @@
+// Chain verification, after the row statistics: one thread block per batch row.
+//
+// Warp 0 evaluates every position at once — the ratio test u_i < min(1, p_i(x_i) /
+// q_i(x_i)) (or x_i == argmax p_i in the greedy form) — and a ballot finds the first
+// position that stops the scan: a rejection, the bonus position K, or a data error.
+// The whole block then draws the emitted token: from norm(max(0, p_a - q_a)) after a
+// rejection at a (p_a if that residual is empty), from p_K when all K drafts were
+// accepted. "Speculative Decoding" and "Speculative Sampling" (spec-decoding-i notes);
+// greedy longest-prefix verification from blockwise parallel decoding ("推测解码").
+#pragma once
+
+#include "draw.cuh"
+
+namespace sv {
+
+struct ChainJob {
+  const void* target;     // [B][K+1][V]
+  const void* draft;      // [B][K][V]
+  int B, K, V;
+  const int32_t* tokens;  // [B][K]
+  const float* uniforms;  // [B][K+1]
+  const RowStats* stats;  // target rows [B*(K+1)], then draft rows [B*K]
+  int greedy;
+  int32_t* accepted_len;  // [B]
+  int32_t* out_tokens;    // [B][K+1]
+};
+
+enum : int { EV_ACCEPT = 0, EV_STOP = 1, EV_ERROR = 2, EV_TIMEOUT = 3 };
+
+__device__ __forceinline__ int row_event(const RowStats& s) {
+  return s.status == ROW_OK ? EV_ACCEPT : (s.status == ROW_TIMEOUT ? EV_TIMEOUT : EV_ERROR);
+}
+
+template <typename T>
+__global__ void __launch_bounds__(kThreads) chain_finish_kernel(const ChainJob j) {
+  __shared__ DrawSmem sm;
+  __shared__ int s_a, s_ev;
+  const int b = blockIdx.x;
+  const int K = j.K, V = j.V;
+  const RowStats* ts = j.stats + size_t(b) * (K + 1);
+  const RowStats* ds = j.stats + size_t(j.B) * (K + 1) + size_t(b) * K;
+  const T* trow0 = static_cast<const T*>(j.target) + size_t(b) * (K + 1) * V;
+  const T* drow0 = j.greedy ? nullptr : static_cast<const T*>(j.draft) + size_t(b) * K * V;
+  const int32_t* x = j.tokens + size_t(b) * K;
+  const float* u = j.uniforms + size_t(b) * (K + 1);
+
+  if (threadIdx.x < 32) {
+    const int lane = threadIdx.x;
+    int a = -1, ev = EV_STOP;
+    for (int base = 0; base <= K && a < 0; base += 32) {
+      const int i = base + lane;
+      int e = EV_ACCEPT;
+      if (i <= K) {
+        const RowStats sp = ts[i];
+        e = row_event(sp);
+        if (e == EV_ACCEPT) {
+          if (i == K) {
+            e = EV_STOP;
+          } else {
+            const int xi = x[i];
+            if (xi < 0 || xi >= V) {
+              e = EV_ERROR;
+            } else if (j.greedy) {
+              e = (xi == sp.argmax) ? EV_ACCEPT : EV_STOP;
+            } else {
+              const RowStats sq = ds[i];
+              e = row_event(sq);
+              if (e == EV_ACCEPT) {
+                const float lp = Elem<T>::load(trow0, size_t(i) * V + xi);
+                const float lq = Elem<T>::load(drow0, size_t(i) * V + xi);
+                const float p = prob<T>(sp, lp, xi);
+                const float q = prob<T>(sq, lq, xi);
+                const float r = q > 0.0f ? p / q : (p > 0.0f ? INFINITY : 0.0f);
+                e = (u[i] < fminf(1.0f, r)) ? EV_ACCEPT : EV_STOP;
+              }
+            }
+          }
+        }
+      }
+      const unsigned stop = __ballot_sync(0xffffffffu, i <= K && e != EV_ACCEPT);
+      if (stop) {
+        const int L = __ffs(stop) - 1;
+        a = base + L;
+        ev = __shfl_sync(0xffffffffu, e, L);
+      }
+    }
+    if (lane == 0) {
+      s_a = a;
+      s_ev = ev;
+    }
+  }
+  __syncthreads();
+  const int a = s_a, ev = s_ev;
+  int32_t* out = j.out_tokens + size_t(b) * (K + 1);
+  if (ev != EV_STOP) {
+    if (threadIdx.x == 0) j.accepted_len[b] = ev == EV_TIMEOUT ? -2 : -1;
+    for (int k = threadIdx.x; k <= K; k += kThreads) out[k] = ev == EV_TIMEOUT ? -2 : -1;
+    return;
+  }
+  int tok;
+  if (j.greedy) {
+    tok = ts[a].argmax;
+  } else {
+    const RowStats sp = ts[a];
+    const T* prow = trow0 + size_t(a) * V;
+    const bool pal = (reinterpret_cast<uintptr_t>(prow) & 15u) == 0;
+    const float w = u[K];
+    tok = -1;
+    if (a < K) {
+      const RowStats sq = ds[a];
+      const T* qrow = drow0 + size_t(a) * V;
+      const bool qal = (reinterpret_cast<uintptr_t>(qrow) & 15u) == 0;
+      tok = inverse_cdf_draw(
+          [&](int v0, unsigned long long* r) {
+            float lp[8], lq[8];
+            load8<T>(prow, v0, V, pal, lp);
+            load8<T>(qrow, v0, V, qal, lq);
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+              const int v = v0 + k;
+              const float d = (v < V) ? prob<T>(sp, lp[k], v) - prob<T>(sq, lq[k], v) : 0.0f;
+              r[k] = to_fx(fmaxf(d, 0.0f));
+            }
+          },
+          V, w, sm);
+    }
+    if (tok < 0) {  // bonus position, or an empty residual: draw from p
+      tok = inverse_cdf_draw(
+          [&](int v0, unsigned long long* r) {
+            float lp[8];
+            load8<T>(prow, v0, V, pal, lp);
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+              const int v = v0 + k;
+              r[k] = (v < V) ? to_fx(prob<T>(sp, lp[k], v)) : 0ull;
+            }
+          },
+          V, w, sm);
+    }
+  }
+  if (threadIdx.x == 0) {
+    j.accepted_len[b] = a;
+    for (int k = 0; k < a; ++k) out[k] = x[k];
+    out[a] = tok;
+    for (int k = a + 1; k <= K; ++k) out[k] = -1;
+  }
+}
+
+}  // namespace sv

@@ -1,0 +1,247 @@
+// Shared device helpers for libspecverify (sm_100a).
+#pragma once
+
+#include <cooperative_groups.h>
+#include <cuda_bf16.h>
+#include <cstdint>
+
+namespace cg = cooperative_groups;
+
+namespace sv {
+
+constexpr int kThreads = 256;
+constexpr int kWarps = kThreads / 32;
+// Masses in [0, 1] are summed as unsigned 64-bit fixed point with 42 fraction bits:
+// integer sums are exact and independent of summation order, so every reduction is
+// deterministic; V <= 2^20 keeps any sum below 2^62.
+constexpr float kFxF = 4398046511104.0f;  // 2^42
+constexpr double kFxInv = 1.0 / 4398046511104.0;
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr unsigned long long kWaitLimitNs = 2000000000ull;  // bound on any copy wait
+
+enum : int32_t { ROW_OK = 0, ROW_INVALID = 1, ROW_TIMEOUT = 2 };
+
+// Per-logit-row statistics that define the transformed distribution:
+//   p(v) = kept(v) ? exp2((l_v - m) * c) / z : 0,
+//   kept(v) = key(l_v) > thr_key || (key(l_v) == thr_key && v <= cutoff),
+// with c = log2(e) / T. thr_key = 0 keeps every row entry.
+struct RowStats {
+  float m;           // largest logit
+  float z;           // sum over the kept set of exp2((l - m) * c)
+  float entropy;     // entropy (nats) of the transformed distribution, if computed
+  uint32_t thr_key;  // boundary key of the kept prefix in (value desc, id asc) order
+  int32_t cutoff;    // largest kept id among entries whose key equals thr_key
+  int32_t argmax;    // lowest id holding the largest logit
+  int32_t status;    // ROW_OK / ROW_INVALID / ROW_TIMEOUT
+  float c;           // log2(e) / T
+};
+static_assert(sizeof(RowStats) == 32, "RowStats is 32 bytes");
+
+// ------------------------------------------------------------------------- keys
+// Order-preserving unsigned key of a float value (larger value -> larger key);
+// -0 maps to the key of +0 so equal values have equal keys. A bfloat16 value's key
+// is the top 16 bits of its float key.
+__device__ __forceinline__ uint32_t f32_key(float x) {
+  uint32_t u = __float_as_uint(x);
+  if (u == 0x80000000u) u = 0u;
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+template <typename T>
+struct Elem;
+
+template <>
+struct Elem<float> {
+  static constexpr int kBytes = 4;
+  static constexpr int kPerVec = 4;     // elements per 16-byte vector
+  static constexpr int kKeyBits = 32;
+  __device__ static __forceinline__ void unpack(const uint4& w, float* x) {
+    x[0] = __uint_as_float(w.x);
+    x[1] = __uint_as_float(w.y);
+    x[2] = __uint_as_float(w.z);
+    x[3] = __uint_as_float(w.w);
+  }
+  __device__ static __forceinline__ float load(const void* base, size_t i) {
+    return __ldg(static_cast<const float*>(base) + i);
+  }
+  __device__ static __forceinline__ uint32_t key(float x) { return f32_key(x); }
+};
+
+template <>
+struct Elem<__nv_bfloat16> {
+  static constexpr int kBytes = 2;
+  static constexpr int kPerVec = 8;
+  static constexpr int kKeyBits = 16;
+  __device__ static __forceinline__ void unpack(const uint4& w, float* x) {
+    const uint32_t a[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      x[2 * k] = __uint_as_float(a[k] << 16);
+      x[2 * k + 1] = __uint_as_float(a[k] & 0xFFFF0000u);
+    }
+  }
+  __device__ static __forceinline__ float load(const void* base, size_t i) {
+    const unsigned short h = __ldg(static_cast<const unsigned short*>(base) + i);
+    return __uint_as_float(uint32_t(h) << 16);
+  }
+  __device__ static __forceinline__ uint32_t key(float x) { return f32_key(x) >> 16; }
+};
+
+__device__ __forceinline__ bool kept(uint32_t key, int id, uint32_t thr_key, int cutoff) {
+  return key > thr_key || (key == thr_key && id <= cutoff);
+}
+
+// 2^x with the SFU instruction (approximate, flushes denormal results to zero).
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// Unnormalised weight exp((l - m) / T) of one logit, as exp2((l - m) * c).
+__device__ __forceinline__ float weight(float l, float m, float c) { return ex2((l - m) * c); }
+
+__device__ __forceinline__ unsigned long long to_fx(float mass01) {
+  return __float2ull_rn(mass01 * kFxF);
+}
+
+// ------------------------------------------------------------------------- PTX: bulk copies
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ unsigned long long global_timer_ns() {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count)
+               : "memory");
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)),
+               "r"(bytes)
+               : "memory");
+}
+
+// 1-D bulk copy global -> this CTA's shared memory, completing on `bar`.
+// dst and src 16-byte aligned, bytes a multiple of 16. Streamed data: evict-first in L2.
+__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes,
+                                         uint64_t* bar) {
+  uint64_t policy;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(policy));
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1], %2, [%3], %4;" ::"r"(smem_u32(dst)),
+      "l"(src), "r"(bytes), "r"(smem_u32(bar)), "l"(policy)
+      : "memory");
+}
+
+// Waits for phase `parity` of `bar` to complete; gives up after kWaitLimitNs.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
+  const uint32_t addr = smem_u32(bar);
+  const unsigned long long t0 = global_timer_ns();
+  for (uint32_t it = 0;; ++it) {
+    uint32_t done;
+    asm volatile(
+        "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
+        " selp.u32 %0, 1, 0, p;\n}"
+        : "=r"(done)
+        : "r"(addr), "r"(parity)
+        : "memory");
+    if (done) return true;
+    if ((it & 255u) == 255u && global_timer_ns() - t0 > kWaitLimitNs) return false;
+  }
+}
+
+// ------------------------------------------------------------------------- reductions
+__device__ __forceinline__ unsigned long long warp_sum_u64(unsigned long long v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+__device__ __forceinline__ double warp_sum_f64(double v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+__device__ __forceinline__ uint32_t warp_sum_u32(uint32_t v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+// Block-wide sums (all threads get the result). `scratch` holds kWarps entries.
+__device__ __forceinline__ unsigned long long block_sum_u64(unsigned long long v,
+                                                            unsigned long long* scratch) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  v = warp_sum_u64(v);
+  __syncthreads();
+  if (lane == 0) scratch[warp] = v;
+  __syncthreads();
+  unsigned long long t = 0;
+#pragma unroll
+  for (int w = 0; w < kWarps; ++w) t += scratch[w];
+  return t;
+}
+__device__ __forceinline__ double block_sum_f64(double v, double* scratch) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  v = warp_sum_f64(v);
+  __syncthreads();
+  if (lane == 0) scratch[warp] = v;
+  __syncthreads();
+  double t = 0.0;
+#pragma unroll
+  for (int w = 0; w < kWarps; ++w) t += scratch[w];
+  return t;
+}
+__device__ __forceinline__ uint32_t block_sum_u32(uint32_t v, uint32_t* scratch) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  v = warp_sum_u32(v);
+  __syncthreads();
+  if (lane == 0) scratch[warp] = v;
+  __syncthreads();
+  uint32_t t = 0;
+#pragma unroll
+  for (int w = 0; w < kWarps; ++w) t += scratch[w];
+  return t;
+}
+
+// Block-wide exclusive prefix sum in thread order; returns the exclusive prefix and
+// writes the block total to *total.
+template <typename U>
+__device__ __forceinline__ U block_exclusive_scan(U v, U* scratch, U* total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  U inc = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const U n = __shfl_up_sync(0xffffffffu, inc, o);
+    if (lane >= o) inc += n;
+  }
+  __syncthreads();
+  if (lane == 31) scratch[warp] = inc;
+  __syncthreads();
+  U before = 0, all = 0;
+#pragma unroll
+  for (int w = 0; w < kWarps; ++w) {
+    if (w < warp) before += scratch[w];
+    all += scratch[w];
+  }
+  *total = all;
+  return before + inc - v;
+}
+
+// (max value, lowest index) combine; NaN never reaches it (rows with NaN are invalid).
+__device__ __forceinline__ void maxloc_combine(float& m, int& i, float m2, int i2) {
+  if (m2 > m || (m2 == m && i2 < i)) {
+    m = m2;
+    i = i2;
+  }
+}
+
+}  // namespace sv

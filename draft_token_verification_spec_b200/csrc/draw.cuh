@@ -1,0 +1,133 @@
+// Deterministic inverse-CDF draw over one vocabulary row (one thread block).
+//
+// The draw returns the smallest token id v (ascending) with res[v] > 0 whose
+// cumulative mass C_v exceeds w * S, S the total; if rounding leaves none, the largest
+// v with res[v] > 0. Masses are fixed point (42 fraction bits), so every partial sum
+// is exact and the result does not depend on how the sum is split across threads.
+// The row is read in chunks of 2048 entries (8 consecutive entries per thread); the
+// first pass records each chunk's mass, the second re-reads only the chunk that holds
+// the crossing. This is the resampling step of "Speculative Decoding" /
+// "Speculative Sampling" (spec-decoding-i notes) with the reading that the draw
+// walks token ids in ascending order.
+#pragma once
+
+#include <climits>
+
+#include "common.cuh"
+
+namespace sv {
+
+constexpr int kDrawChunk = kThreads * 8;
+constexpr int kMaxDrawChunks = (1 << 20) / kDrawChunk;  // V <= 2^20
+
+struct DrawSmem {
+  unsigned long long chunk[kMaxDrawChunks];
+  unsigned long long scr[kWarps];
+  unsigned long long total;
+  int best;
+  int sel_chunk;
+  int fallback;
+  unsigned long long sel_before;
+};
+
+// f(v0, r) fills r[0..7] with the fixed-point masses of entries v0..v0+7 (0 past V).
+// Returns -1 when the whole row has zero mass.
+template <typename F>
+__device__ int inverse_cdf_draw(F&& f, int V, float w, DrawSmem& sm) {
+  const int nch = (V + kDrawChunk - 1) / kDrawChunk;
+  for (int ch = 0; ch < nch; ++ch) {
+    unsigned long long r[8];
+    f(ch * kDrawChunk + threadIdx.x * 8, r);
+    unsigned long long t = 0;
+#pragma unroll
+    for (int k = 0; k < 8; ++k) t += r[k];
+    t = block_sum_u64(t, sm.scr);
+    if (threadIdx.x == 0) sm.chunk[ch] = t;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    unsigned long long S = 0;
+    for (int ch = 0; ch < nch; ++ch) S += sm.chunk[ch];
+    const double target = double(w) * double(S);
+    unsigned long long cum = 0;
+    int sel = -1, last_pos = -1;
+    unsigned long long last_before = 0, sel_before = 0;
+    for (int ch = 0; ch < nch; ++ch) {
+      const unsigned long long s = sm.chunk[ch];
+      if (s > 0) {
+        last_pos = ch;
+        last_before = cum;
+        if (sel < 0 && double(cum + s) > target) {
+          sel = ch;
+          sel_before = cum;
+        }
+      }
+      cum += s;
+    }
+    sm.fallback = 0;
+    if (sel < 0) {
+      sel = last_pos;
+      sel_before = last_before;
+      sm.fallback = 1;
+    }
+    sm.sel_chunk = sel;
+    sm.sel_before = sel_before;
+    sm.total = S;
+    sm.best = sm.fallback ? -1 : INT_MAX;
+  }
+  __syncthreads();
+  const int sel = sm.sel_chunk;
+  if (sel < 0) return -1;
+  const double target = double(w) * double(sm.total);
+  unsigned long long r[8];
+  const int v0 = sel * kDrawChunk + threadIdx.x * 8;
+  f(v0, r);
+  unsigned long long t = 0;
+#pragma unroll
+  for (int k = 0; k < 8; ++k) t += r[k];
+  unsigned long long total;
+  unsigned long long cum = sm.sel_before + block_exclusive_scan<unsigned long long>(t, sm.scr, &total);
+  if (sm.fallback) {
+    int last = -1;
+#pragma unroll
+    for (int k = 0; k < 8; ++k)
+      if (r[k] > 0) last = v0 + k;
+    if (last >= 0) atomicMax(&sm.best, last);
+  } else {
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      cum += r[k];
+      if (r[k] > 0 && double(cum) > target) {
+        atomicMin(&sm.best, v0 + k);
+        break;
+      }
+    }
+  }
+  __syncthreads();
+  const int tok = sm.best;
+  __syncthreads();
+  return tok;
+}
+
+// Loads entries v0..v0+7 of a logit row as floats (-inf past V): 16-byte vector loads
+// when the row is 16-byte aligned and the 8 entries are inside it.
+template <typename T>
+__device__ __forceinline__ void load8(const T* row, int v0, int V, bool aligned, float* x) {
+  if (aligned && v0 + 8 <= V) {
+    constexpr int P = Elem<T>::kPerVec;
+    const uint4* p = reinterpret_cast<const uint4*>(row + v0);
+#pragma unroll
+    for (int q = 0; q < 8 / P; ++q) Elem<T>::unpack(__ldg(p + q), x + q * P);
+  } else {
+#pragma unroll
+    for (int k = 0; k < 8; ++k) x[k] = (v0 + k < V) ? Elem<T>::load(row, size_t(v0 + k)) : -INFINITY;
+  }
+}
+
+// Probability of entry v under the transformed distribution described by s.
+template <typename T>
+__device__ __forceinline__ float prob(const RowStats& s, float l, int v) {
+  return kept(Elem<T>::key(l), v, s.thr_key, s.cutoff) ? weight(l, s.m, s.c) / s.z : 0.0f;
+}
+
+}  // namespace sv

@@ -1,0 +1,296 @@
+// libspecverify C ABI: argument checks, workspace layout and kernel launches.
+// The operations and their sources are documented in include/specverify.h.
+#include <atomic>
+#include <cmath>
+#include <cstring>
+
+#include "chain.cuh"
+#include "probs.cuh"
+#include "row_stats.cuh"
+#include "specverify.h"
+#include "tree.cuh"
+
+namespace {
+
+using sv::kThreads;
+
+// Slice of a logit row per CTA: small enough that two or three CTAs share an SM and
+// one CTA's computation overlaps another's copies.
+constexpr size_t kSliceTargetBytes = 64 * 1024;
+constexpr size_t kMaxDynSmem = 227 * 1024 - sizeof(sv::RowAux) - 1024;
+constexpr size_t kStatsOffset = 256;  // the device status word lives at offset 0
+
+std::atomic<void*> g_ev_before{nullptr};
+std::atomic<void*> g_ev_after{nullptr};
+
+struct RowPlan {
+  int C;        // CTAs per cluster (one cluster per row)
+  int slice;    // elements per CTA
+  size_t dyn;   // dynamic shared memory per CTA
+};
+
+bool plan_rows(int V, int elem_bytes, RowPlan* pl) {
+  int C = 1;
+  while (C < 16 && size_t((V + C - 1) / C) * elem_bytes > kSliceTargetBytes) C *= 2;
+  const int slice = ((V + C - 1) / C + 15) / 16 * 16;
+  const size_t dyn = (size_t(slice) * elem_bytes + 16 + 127) / 128 * 128;
+  if (dyn > kMaxDynSmem) return false;
+  *pl = RowPlan{C, slice, dyn};
+  return true;
+}
+
+template <typename T>
+cudaError_t launch_row_stats(const sv::RowJob& job, const RowPlan& pl, cudaStream_t s) {
+  auto k = sv::row_stats_kernel<T>;
+  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       int(pl.dyn));
+  if (e != cudaSuccess) return e;
+  if (pl.C > 8) {
+    e = cudaFuncSetAttribute(k, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+    if (e != cudaSuccess) return e;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(unsigned(job.rows * pl.C), 1, 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = pl.dyn;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = unsigned(pl.C);
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, k, job);
+}
+
+cudaError_t launch_row_stats_dt(spec_dtype dt, const sv::RowJob& job, const RowPlan& pl,
+                                cudaStream_t s) {
+  return dt == SPEC_BF16 ? launch_row_stats<__nv_bfloat16>(job, pl, s)
+                         : launch_row_stats<float>(job, pl, s);
+}
+
+int elem_bytes(spec_dtype dt) { return dt == SPEC_BF16 ? 2 : 4; }
+
+bool dtype_ok(int dt) { return dt == SPEC_F32 || dt == SPEC_BF16; }
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+size_t stats_bytes(long long rows) { return kStatsOffset + size_t(rows) * sizeof(sv::RowStats); }
+
+// Grid limit: rows * C must fit a 1-D grid.
+bool rows_fit(long long rows, int C) { return rows * C <= 0x7fffffffLL; }
+
+spec_status check_launch(cudaError_t e) { return e == cudaSuccess ? SPEC_OK : SPEC_ERR_CUDA; }
+
+}  // namespace
+
+extern "C" {
+
+const char* spec_status_string(int status) {
+  switch (status) {
+    case SPEC_OK: return "SPEC_OK";
+    case SPEC_ERR_INVALID_ARG: return "SPEC_ERR_INVALID_ARG";
+    case SPEC_ERR_UNSUPPORTED: return "SPEC_ERR_UNSUPPORTED";
+    case SPEC_ERR_CUDA: return "SPEC_ERR_CUDA";
+    case SPEC_ERR_WORKSPACE: return "SPEC_ERR_WORKSPACE";
+    case SPEC_ERR_DEVICE_TIMEOUT: return "SPEC_ERR_DEVICE_TIMEOUT";
+    default: return "unknown spec_status";
+  }
+}
+
+size_t spec_workspace_size(int B, int K_or_N, int V) {
+  if (B <= 0 || K_or_N <= 0 || V <= 0) return 0;
+  return stats_bytes((long long)B * (2LL * K_or_N + 1));
+}
+
+spec_status spec_verify_chain(const void* target_logits, const void* draft_logits,
+                              spec_dtype dtype, int B, int K, int V,
+                              const int32_t* draft_tokens, const float* uniforms, float temp,
+                              int top_k, float top_p, int32_t* accepted_len,
+                              int32_t* out_tokens, void* workspace, size_t workspace_bytes,
+                              void* stream) {
+  const bool greedy = temp == 0.0f;
+  if (!target_logits || (!greedy && !draft_logits) || !dtype_ok(dtype) || B <= 0 || K <= 0 ||
+      V <= 0 || !draft_tokens || !uniforms || !accepted_len || !out_tokens ||
+      !std::isfinite(temp) || temp < 0.0f || !(top_p > 0.0f))
+    return SPEC_ERR_INVALID_ARG;
+  if (V > SPEC_MAX_VOCAB) return SPEC_ERR_UNSUPPORTED;
+  const long long rows = (long long)B * (greedy ? K + 1 : 2LL * K + 1);
+  if (!workspace || !aligned16(workspace) || workspace_bytes < stats_bytes(rows))
+    return SPEC_ERR_WORKSPACE;
+  RowPlan pl;
+  if (!plan_rows(V, elem_bytes(dtype), &pl) || !rows_fit(rows, pl.C) || B > 0x7fffffff)
+    return SPEC_ERR_UNSUPPORTED;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int32_t* dev_status = static_cast<int32_t*>(workspace);
+  sv::RowStats* stats =
+      reinterpret_cast<sv::RowStats*>(static_cast<char*>(workspace) + kStatsOffset);
+  if (cudaMemsetAsync(dev_status, 0, sizeof(int32_t), s) != cudaSuccess) return SPEC_ERR_CUDA;
+
+  sv::RowJob rj = {};
+  rj.base0 = target_logits;
+  rj.base1 = draft_logits;
+  rj.rows0 = (long long)B * (K + 1);
+  rj.rows = rows;
+  rj.V = V;
+  rj.slice = pl.slice;
+  rj.c = greedy ? 0.0f : sv::kLog2e / temp;
+  rj.inv_t = greedy ? 0.0f : 1.0f / temp;
+  rj.top_k = (top_k >= 1 && top_k < V) ? top_k : 0;
+  rj.top_p = top_p < 1.0f ? top_p : 1.0f;
+  rj.flags = greedy ? sv::RS_GREEDY : 0;
+  rj.stats = stats;
+  rj.dev_status = dev_status;
+  void* evb = g_ev_before.load();
+  void* eva = g_ev_after.load();
+  if (evb) cudaEventRecord(static_cast<cudaEvent_t>(evb), s);
+  if (launch_row_stats_dt(dtype, rj, pl, s) != cudaSuccess) return SPEC_ERR_CUDA;
+  if (eva) cudaEventRecord(static_cast<cudaEvent_t>(eva), s);
+
+  sv::ChainJob cj = {};
+  cj.target = target_logits;
+  cj.draft = draft_logits;
+  cj.B = B;
+  cj.K = K;
+  cj.V = V;
+  cj.tokens = draft_tokens;
+  cj.uniforms = uniforms;
+  cj.stats = stats;
+  cj.greedy = greedy ? 1 : 0;
+  cj.accepted_len = accepted_len;
+  cj.out_tokens = out_tokens;
+  if (dtype == SPEC_BF16)
+    sv::chain_finish_kernel<__nv_bfloat16><<<B, kThreads, 0, s>>>(cj);
+  else
+    sv::chain_finish_kernel<float><<<B, kThreads, 0, s>>>(cj);
+  return check_launch(cudaGetLastError());
+}
+
+spec_status spec_verify_tree_typical(const void* target_logits, spec_dtype dtype, int B, int N,
+                                     int V, const int32_t* node_tokens,
+                                     const int32_t* parent_idx, float eps, float delta,
+                                     int32_t* best_path, int path_cap, int32_t* accepted_len,
+                                     void* workspace, size_t workspace_bytes, void* stream) {
+  if (!target_logits || !dtype_ok(dtype) || B <= 0 || N <= 0 || V <= 0 || !node_tokens ||
+      !parent_idx || !best_path || path_cap <= 0 || !accepted_len || !std::isfinite(eps) ||
+      !std::isfinite(delta))
+    return SPEC_ERR_INVALID_ARG;
+  if (V > SPEC_MAX_VOCAB || N > SPEC_MAX_TREE_NODES) return SPEC_ERR_UNSUPPORTED;
+  const long long rows = (long long)B * N;
+  if (!workspace || !aligned16(workspace) || workspace_bytes < stats_bytes(rows))
+    return SPEC_ERR_WORKSPACE;
+  RowPlan pl;
+  if (!plan_rows(V, elem_bytes(dtype), &pl) || !rows_fit(rows, pl.C)) return SPEC_ERR_UNSUPPORTED;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int32_t* dev_status = static_cast<int32_t*>(workspace);
+  sv::RowStats* stats =
+      reinterpret_cast<sv::RowStats*>(static_cast<char*>(workspace) + kStatsOffset);
+  if (cudaMemsetAsync(dev_status, 0, sizeof(int32_t), s) != cudaSuccess) return SPEC_ERR_CUDA;
+
+  sv::RowJob rj = {};
+  rj.base0 = target_logits;
+  rj.base1 = target_logits;
+  rj.rows0 = rows;
+  rj.rows = rows;
+  rj.V = V;
+  rj.slice = pl.slice;
+  rj.c = sv::kLog2e;
+  rj.inv_t = 1.0f;
+  rj.top_k = 0;
+  rj.top_p = 1.0f;
+  rj.flags = sv::RS_ENTROPY;
+  rj.stats = stats;
+  rj.dev_status = dev_status;
+  void* evb = g_ev_before.load();
+  void* eva = g_ev_after.load();
+  if (evb) cudaEventRecord(static_cast<cudaEvent_t>(evb), s);
+  if (launch_row_stats_dt(dtype, rj, pl, s) != cudaSuccess) return SPEC_ERR_CUDA;
+  if (eva) cudaEventRecord(static_cast<cudaEvent_t>(eva), s);
+
+  sv::TreeJob tj = {};
+  tj.target = target_logits;
+  tj.B = B;
+  tj.N = N;
+  tj.V = V;
+  tj.tokens = node_tokens;
+  tj.parent = parent_idx;
+  tj.eps = eps;
+  tj.delta = delta;
+  tj.stats = stats;
+  tj.best_path = best_path;
+  tj.path_cap = path_cap;
+  tj.accepted_len = accepted_len;
+  const size_t dyn = size_t(N) * (4 + 4 + 1 + 1) + 16;
+  if (dtype == SPEC_BF16)
+    sv::tree_finish_kernel<__nv_bfloat16><<<B, kThreads, dyn, s>>>(tj);
+  else
+    sv::tree_finish_kernel<float><<<B, kThreads, dyn, s>>>(tj);
+  return check_launch(cudaGetLastError());
+}
+
+spec_status spec_logits_to_probs(const void* logits, spec_dtype dtype, int rows, int V,
+                                 float temp, int top_k, float top_p, float* probs,
+                                 float* entropy, void* stream) {
+  if (!logits || !dtype_ok(dtype) || rows <= 0 || V <= 0 || !probs || !std::isfinite(temp) ||
+      temp < 0.0f || !(top_p > 0.0f))
+    return SPEC_ERR_INVALID_ARG;
+  if (V > SPEC_MAX_VOCAB) return SPEC_ERR_UNSUPPORTED;
+  RowPlan pl;
+  if (!plan_rows(V, elem_bytes(dtype), &pl) || !rows_fit(rows, pl.C)) return SPEC_ERR_UNSUPPORTED;
+  const bool greedy = temp == 0.0f;
+  sv::RowJob rj = {};
+  rj.base0 = logits;
+  rj.base1 = logits;
+  rj.rows0 = rows;
+  rj.rows = rows;
+  rj.V = V;
+  rj.slice = pl.slice;
+  rj.c = greedy ? 0.0f : sv::kLog2e / temp;
+  rj.inv_t = greedy ? 0.0f : 1.0f / temp;
+  rj.top_k = (top_k >= 1 && top_k < V) ? top_k : 0;
+  rj.top_p = top_p < 1.0f ? top_p : 1.0f;
+  rj.flags = sv::RS_WRITE_PROBS | (greedy ? sv::RS_GREEDY : 0) |
+             ((entropy && !greedy) ? sv::RS_ENTROPY : 0);
+  rj.stats = nullptr;
+  rj.probs = probs;
+  rj.entropy = entropy;
+  rj.dev_status = nullptr;
+  return check_launch(launch_row_stats_dt(dtype, rj, pl, static_cast<cudaStream_t>(stream)));
+}
+
+spec_status spec_residual_sample(const float* p, const float* q, int rows, int V,
+                                 const float* uniforms, int32_t* tokens, void* stream) {
+  if (!p || rows <= 0 || V <= 0 || !uniforms || !tokens) return SPEC_ERR_INVALID_ARG;
+  if (V > SPEC_MAX_VOCAB) return SPEC_ERR_UNSUPPORTED;
+  sv::ResidualJob j = {p, q, rows, V, uniforms, tokens};
+  sv::residual_sample_kernel<<<rows, kThreads, 0, static_cast<cudaStream_t>(stream)>>>(j);
+  return check_launch(cudaGetLastError());
+}
+
+spec_status spec_get_device_status(const void* workspace, int32_t* status_out, void* stream) {
+  if (!workspace || !status_out) return SPEC_ERR_INVALID_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int32_t h = 0;
+  if (cudaMemcpyAsync(&h, workspace, sizeof h, cudaMemcpyDeviceToHost, s) != cudaSuccess ||
+      cudaStreamSynchronize(s) != cudaSuccess)
+    return SPEC_ERR_CUDA;
+  *status_out = h ? SPEC_ERR_DEVICE_TIMEOUT : SPEC_OK;
+  return SPEC_OK;
+}
+
+void spec_set_row_kernel_events(void* before, void* after) {
+  g_ev_before.store(before);
+  g_ev_after.store(after);
+}
+
+int spec_kernels_per_call(const char* entry_point) {
+  if (!entry_point) return -1;
+  if (!std::strcmp(entry_point, "spec_verify_chain")) return 2;
+  if (!std::strcmp(entry_point, "spec_verify_tree_typical")) return 2;
+  if (!std::strcmp(entry_point, "spec_logits_to_probs")) return 1;
+  if (!std::strcmp(entry_point, "spec_residual_sample")) return 1;
+  return -1;
+}
+
+}  // extern "C"

@@ -1,0 +1,105 @@
+// MEDUSA typical acceptance over a candidate tree, after the row statistics: one
+// thread block per batch row ("Key Components", spec-decoding-i notes; "推测解码").
+//
+// Threads test every non-root node in parallel: p_parent(tok_c) > min(eps, delta *
+// exp(-H(p_parent))), p the temperature-1 softmax of the parent's logits. One thread
+// then resolves ancestry in index order (parents precede children): a node is
+// accepted iff its parent is and its own test passes; the root is accepted
+// unconditionally. The deepest accepted node (lowest index on ties) and its
+// root-first ancestor chain are written out.
+#pragma once
+
+#include "draw.cuh"
+
+namespace sv {
+
+struct TreeJob {
+  const void* target;        // [B][N][V]
+  int B, N, V;
+  const int32_t* tokens;     // [B][N]
+  const int32_t* parent;     // [N]
+  float eps, delta;
+  const RowStats* stats;     // [B*N]
+  int32_t* best_path;        // [B][path_cap]
+  int path_cap;
+  int32_t* accepted_len;     // [B]
+};
+
+enum : int8_t { ND_REJECT = 0, ND_ACCEPT = 1, ND_ERROR = 2, ND_TIMEOUT = 3 };
+
+template <typename T>
+__global__ void __launch_bounds__(kThreads) tree_finish_kernel(const TreeJob j) {
+  extern __shared__ __align__(16) unsigned char tsm[];
+  const int N = j.N, V = j.V, b = blockIdx.x;
+  int32_t* par = reinterpret_cast<int32_t*>(tsm);           // [N]
+  int32_t* depth = par + N;                                  // [N]
+  int8_t* test = reinterpret_cast<int8_t*>(depth + N);       // [N]
+  int8_t* acc = test + N;                                    // [N]
+  __shared__ int s_bad_tree;
+  if (threadIdx.x == 0) s_bad_tree = 0;
+  __syncthreads();
+  const RowStats* st = j.stats + size_t(b) * N;
+  const T* rows = static_cast<const T*>(j.target) + size_t(b) * N * V;
+  const int32_t* tok = j.tokens + size_t(b) * N;
+  for (int c = threadIdx.x; c < N; c += kThreads) {
+    const int pa = j.parent[c];
+    par[c] = pa;
+    const bool ok_edge = (c == 0) ? (pa == -1) : (pa >= 0 && pa < c);
+    if (!ok_edge) s_bad_tree = 1;
+    int8_t t = ND_ACCEPT;
+    if (c > 0 && ok_edge) {
+      const RowStats s = st[pa];
+      if (s.status != ROW_OK) {
+        t = s.status == ROW_TIMEOUT ? ND_TIMEOUT : ND_ERROR;
+      } else {
+        const int tk = tok[c];
+        if (tk < 0 || tk >= V) {
+          t = ND_ERROR;
+        } else {
+          const float l = Elem<T>::load(rows, size_t(pa) * V + tk);
+          const float p = prob<T>(s, l, tk);
+          const float thr = fminf(j.eps, j.delta * expf(-s.entropy));
+          t = p > thr ? ND_ACCEPT : ND_REJECT;
+        }
+      }
+    }
+    test[c] = t;
+  }
+  __syncthreads();
+  int32_t* path = j.best_path + size_t(b) * j.path_cap;
+  __shared__ int s_len, s_err;
+  if (threadIdx.x == 0) {
+    int err = s_bad_tree ? ND_ERROR : 0, best = 0;
+    if (!err) {
+      acc[0] = 1;
+      depth[0] = 0;
+      for (int c = 1; c < N && !err; ++c) {
+        const int pa = par[c];
+        depth[c] = depth[pa] + 1;
+        acc[c] = 0;
+        if (acc[pa]) {
+          if (test[c] >= ND_ERROR) {
+            err = test[c];
+          } else {
+            acc[c] = test[c];
+            if (acc[c] && depth[c] > depth[best]) best = c;
+          }
+        }
+      }
+    }
+    int len = err ? 0 : depth[best] + 1;
+    if (!err && len > j.path_cap) err = ND_ERROR;
+    if (!err) {
+      for (int n = best, k = len - 1; k >= 0; --k, n = (n > 0 ? par[n] : -1)) path[k] = n;
+    }
+    s_len = len;
+    s_err = err;
+    j.accepted_len[b] = err ? (err == ND_TIMEOUT ? -2 : -1) : len;
+  }
+  __syncthreads();
+  const int fill_from = s_err ? 0 : s_len;
+  const int fill = s_err == ND_TIMEOUT ? -2 : -1;
+  for (int k = fill_from + threadIdx.x; k < j.path_cap; k += kThreads) path[k] = fill;
+}
+
+}  // namespace sv

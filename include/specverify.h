@@ -1,0 +1,159 @@
+/* libspecverify — draft-token verification for speculative decoding on B200 (sm_100a).
+ *
+ * The library verifies the drafts of one speculative-decoding round on the GPU:
+ *   - chain speculative sampling (temperature / top-k / top-p, ratio test,
+ *     residual resample, bonus token) and its temperature-0 greedy form;
+ *   - MEDUSA typical acceptance over a candidate tree;
+ *   - the probability transform and the residual draw as separate calls.
+ *
+ * Sources, by page and section (the pages carry prose; their formulas were lost
+ * in extraction and are restated here in the standard form that prose describes):
+ *   [SD] taking-lying-flat.github.io/blog/posts/spec-decoding-i/ —
+ *        "Speculative Decoding" (accept, resample at the first rejection, bonus
+ *        token), "Speculative Sampling" (acceptance probability min(1, p/q), residual
+ *        norm(max(0, p - q)), transforms applied before the rejection scheme),
+ *        "Key Components" (MEDUSA tree, typical acceptance).
+ *   [SV] blog.csdn.net/yorkhunter/article/details/139214590 — "推测解码"
+ *        (blockwise parallel decoding: greedy longest-prefix verification; MEDUSA
+ *        typical acceptance, first token greedy, longest accepted prefix).
+ *
+ * Conventions for every call
+ *   - Pointers named *_logits, *_tokens, uniforms, parent_idx, workspace and all
+ *     outputs are DEVICE pointers, allocated and owned by the caller. The library
+ *     allocates nothing and keeps no pointer after a call returns.
+ *   - Work is enqueued on `stream` (a cudaStream_t passed as void*, NULL = legacy
+ *     default stream). Calls are asynchronous: they return before the GPU runs, and
+ *     no call synchronises the host (except spec_get_device_status).
+ *   - Logit tensors are row-major with the vocabulary contiguous, element type
+ *     SPEC_F32 (float) or SPEC_BF16 (bfloat16 bit patterns). 1 <= V <= SPEC_MAX_VOCAB.
+ *   - The return value reports argument and launch errors only, before or at launch;
+ *     on error nothing has been enqueued (SPEC_ERR_CUDA: a launch may have failed
+ *     part-way).
+ *   - Data errors are reported in-band per batch row: accepted_len[b] = -1 and every
+ *     other output of that row = -1. A row is in error when the verification reaches
+ *     a logit row that holds NaN or +inf or is entirely -inf, or a token outside
+ *     [0, V). Rows the rule never reaches (positions after the first rejection, tree
+ *     nodes under a rejected parent) are not inspected.
+ *   - accepted_len[b] = -2 marks a row whose device-side copy wait exceeded its time
+ *     limit (about 2 s); spec_get_device_status then returns SPEC_ERR_DEVICE_TIMEOUT.
+ *   - Results are deterministic: the same inputs give the same outputs, bit for bit.
+ *   - Temperature: temp == 0 selects the greedy limit; temp must be finite and >= 0.
+ *     top_k <= 0 or top_k >= V disables top-k; top_p >= 1 disables top-p; top_p must
+ *     be > 0. Transforms are applied in the order temperature -> top-k -> softmax ->
+ *     top-p -> renormalise, ties broken by the lower token id, the token whose mass
+ *     crosses top_p kept.
+ */
+#ifndef SPECVERIFY_H
+#define SPECVERIFY_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  SPEC_OK = 0,
+  SPEC_ERR_INVALID_ARG = -1,    /* NULL where required, bad size, bad dtype, bad knob */
+  SPEC_ERR_UNSUPPORTED = -2,    /* valid but beyond this build's limits */
+  SPEC_ERR_CUDA = -3,           /* a CUDA runtime call or launch failed */
+  SPEC_ERR_WORKSPACE = -4,      /* workspace NULL, misaligned or too small */
+  SPEC_ERR_DEVICE_TIMEOUT = -5  /* reported by spec_get_device_status only */
+} spec_status;
+
+typedef enum { SPEC_F32 = 0, SPEC_BF16 = 1 } spec_dtype;
+
+#define SPEC_MAX_VOCAB (1 << 20)
+#define SPEC_MAX_TREE_NODES 4096
+
+/* Human-readable name of a status code (static string). */
+const char* spec_status_string(int status);
+
+/* Bytes of workspace that spec_verify_chain(B, K, V) and spec_verify_tree_typical(B,
+ * N = K_or_N, V) need; either call accepts any workspace at least this large. The
+ * workspace must be 16-byte aligned. Returns 0 for invalid sizes. */
+size_t spec_workspace_size(int B, int K_or_N, int V);
+
+/* Chain verification of one round — [SD] "Speculative Decoding", "Speculative
+ * Sampling"; greedy form [SV] "推测解码".
+ *   target_logits [B][K+1][V]: target scores for draft positions 1..K and the bonus
+ *                  position K+1 (row i = distribution p_i of token i given the prefix).
+ *   draft_logits  [B][K][V]:   draft scores q_i (may be NULL iff temp == 0).
+ *   draft_tokens  [B][K] int32: the drafted tokens x_i.
+ *   uniforms      [B][K+1] float in [0,1): u[0..K-1] for the accept tests,
+ *                  u[K] for the single resample-or-bonus draw.
+ *   accepted_len  [B] int32 out: a in [0, K]; a + 1 tokens are emitted.
+ *   out_tokens    [B][K+1] int32 out: x_0..x_{a-1}, then the drawn token, then -1.
+ * With temp > 0: x_i is accepted iff u_i < min(1, p_i(x_i) / q_i(x_i)) (r = +inf when
+ * q_i(x_i) = 0 < p_i(x_i), r = 0 when both are 0), scanning i = 0.. and stopping at
+ * the first rejection, whose token is redrawn from norm(max(0, p_a - q_a)) (p_a when
+ * that is empty); if all K are accepted the bonus token is drawn from p_K. A draw
+ * returns the smallest token id v (ascending) with mass > 0 whose cumulative mass
+ * exceeds u[K] times the total. With temp == 0: a is the length of the longest
+ * prefix with x_i == argmax p_i (lowest id on ties) and the emitted token is
+ * argmax p_a. K >= 1, B >= 1. */
+spec_status spec_verify_chain(const void* target_logits, const void* draft_logits,
+                              spec_dtype dtype, int B, int K, int V,
+                              const int32_t* draft_tokens, const float* uniforms, float temp,
+                              int top_k, float top_p, int32_t* accepted_len,
+                              int32_t* out_tokens, void* workspace, size_t workspace_bytes,
+                              void* stream);
+
+/* MEDUSA typical acceptance over a candidate tree — [SD] "Key Components";
+ * [SV] "推测解码".
+ *   target_logits [B][N][V]: row n = the target's next-token scores after node n.
+ *   node_tokens   [B][N] int32: token of each node; node 0 is the root (the greedy
+ *                  first token, accepted unconditionally; its token is not read).
+ *   parent_idx    [N] int32, shared by the batch: parent_idx[0] = -1 and
+ *                  0 <= parent_idx[c] < c (parents precede children). A violation
+ *                  puts every batch row in error.
+ *   best_path     [B][path_cap] int32 out: node indices of the chosen path, root
+ *                  first, -1 padded. A path longer than path_cap is a row error.
+ *   accepted_len  [B] int32 out: nodes on the path, root included (>= 1).
+ * Node c >= 1 is accepted iff its parent is and p(tok_c) > min(eps, delta *
+ * exp(-H(p))), with p = softmax of the parent's row (temperature 1) and H its entropy
+ * in nats; the deepest accepted node wins, the lowest node index on ties.
+ * 1 <= N <= SPEC_MAX_TREE_NODES, eps and delta finite. */
+spec_status spec_verify_tree_typical(const void* target_logits, spec_dtype dtype, int B, int N,
+                                     int V, const int32_t* node_tokens,
+                                     const int32_t* parent_idx, float eps, float delta,
+                                     int32_t* best_path, int path_cap, int32_t* accepted_len,
+                                     void* workspace, size_t workspace_bytes, void* stream);
+
+/* The sampling transform alone — [SD] "Speculative Sampling" (last bullet).
+ *   logits [rows][V]; probs [rows][V] float out: the transformed distribution
+ *   (temp == 0: one-hot at the argmax); entropy [rows] float out or NULL: its
+ *   entropy in nats. Rows that hold NaN or +inf, or are entirely -inf, get NaN
+ *   probabilities and entropy. rows >= 1. */
+spec_status spec_logits_to_probs(const void* logits, spec_dtype dtype, int rows, int V,
+                                 float temp, int top_k, float top_p, float* probs,
+                                 float* entropy, void* stream);
+
+/* Residual draw alone — [SD] "Speculative Sampling".
+ *   p, q [rows][V] float probability rows (q may be NULL: draw from p);
+ *   uniforms [rows] float; tokens [rows] int32 out.
+ * Draws from norm(max(0, p - q)) (from p when that is empty) with the same
+ * inverse-CDF rule as spec_verify_chain. A row holding an entry that is NaN or
+ * outside [0, 1], or whose p has no positive entry, gets token -1. rows >= 1. */
+spec_status spec_residual_sample(const float* p, const float* q, int rows, int V,
+                                 const float* uniforms, int32_t* tokens, void* stream);
+
+/* Copies the device status word of `workspace` to the host (synchronises `stream`):
+ * SPEC_OK, or SPEC_ERR_DEVICE_TIMEOUT if a kernel of an earlier call on this
+ * workspace gave up waiting for a copy. The word is cleared by every verify call. */
+spec_status spec_get_device_status(const void* workspace, int32_t* status_out, void* stream);
+
+/* Timing hook for measurement tools: while set, every spec_verify_chain and
+ * spec_verify_tree_typical call records `before` (a cudaEvent_t) on its stream just
+ * before its row-statistics kernel and `after` just after it. NULL, NULL clears. */
+void spec_set_row_kernel_events(void* before, void* after);
+
+/* Number of kernels each call enqueues (for launch accounting). */
+int spec_kernels_per_call(const char* entry_point);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SPECVERIFY_H */

@@ -55,7 +55,8 @@ const double kInf = std::numeric_limits<double>::infinity();
 enum : int32_t {
   FLAG_RATIO = 1,      // |u_i - r_i| < 1e-5 at a tested position
   FLAG_CDF = 2,        // inverse-CDF boundary within 1e-6 * S of w * S
-  FLAG_TOPP = 4,       // top-p cumulative mass boundary within 1e-6 of top_p
+  FLAG_TOPP = 4,       // a top-p boundary within 1e-6 of top_p, whose other side
+                       // changes the row's output
   FLAG_TREE = 8,       // |p - thr| / thr < 1e-5 at a tested tree node
   DIAG_Q_ZERO = 16,    // a tested draft token had q(x) = 0 (not a parity flag)
 };
@@ -98,7 +99,12 @@ int argmax_lowest(const std::vector<double>& l) {
 struct Dist {
   std::vector<double> p;
   double entropy = 0.0;
-  double topp_margin = kInf;  // min distance of the nucleus boundary sums to top_p
+  // Distances to top_p of the cumulative mass that first reaches it (margin_reach)
+  // and of the one just before (margin_prev): how close the nucleus is to one more
+  // or one fewer token. Infinite when top-p is off.
+  double margin_reach = kInf;
+  double margin_prev = kInf;
+  double topp_margin() const { return std::min(margin_reach, margin_prev); }
 };
 
 // The sampling transform of [SD] "Speculative Sampling" (last bullet): the
@@ -107,7 +113,9 @@ struct Dist {
 // first on ties); softmax over the kept set; top-p keeps the shortest prefix of
 // the probability-sorted kept tokens whose mass reaches top_p, then
 // renormalises. T == 0 is the greedy limit: a one-hot at the argmax.
-Dist transform(const std::vector<double>& l, double T, int top_k, double top_p) {
+// alt = +1 / -1 keeps one token more / fewer than the nucleus (used only to decide
+// whether a near-tie at the top-p boundary can change a verification outcome).
+Dist transform(const std::vector<double>& l, double T, int top_k, double top_p, int alt = 0) {
   const int V = int(l.size());
   Dist d;
   d.p.assign(size_t(V), 0.0);
@@ -156,10 +164,10 @@ Dist transform(const std::vector<double>& l, double T, int top_k, double top_p) 
         break;
       }
     }
-    if (n_keep < order.size() || cum >= top_p)
-      d.topp_margin = std::min(std::fabs(cum - top_p), std::fabs(prev - top_p));
-    else
-      d.topp_margin = std::fabs(cum - top_p);
+    d.margin_reach = std::fabs(cum - top_p);
+    d.margin_prev = std::fabs(prev - top_p);
+    if (alt > 0) n_keep = std::min(n_keep + 1, order.size());
+    if (alt < 0) n_keep = std::max<size_t>(n_keep - 1, 1);
     std::fill(kept.begin(), kept.end(), 0);
     for (size_t j = 0; j < n_keep; ++j) kept[order[j]] = 1;
     double Zp = 0.0;
@@ -237,33 +245,52 @@ struct ChainArgs {
 void chain_error(const ChainArgs& a, int b) {
   a.accepted_len[b] = -1;
   for (int j = 0; j <= a.K; ++j) a.out_tokens[size_t(b) * (a.K + 1) + j] = -1;
+  if (a.flags) a.flags[b] = 0;
 }
 
-// One batch row of chain verification: [SD] "Speculative Decoding" (accept
-// x_i left to right, stop at the first rejection and resample it, bonus token
-// after K acceptances) and "Speculative Sampling" (the acceptance ratio and
-// the residual). T == 0 is the greedy longest-prefix rule of blockwise
-// parallel decoding ([SV], "推测解码").
-void chain_row(const ChainArgs& a, int b) {
+// A transformed row to evaluate with one token more (alt = +1) or fewer (alt = -1) in
+// its nucleus: kind 0 = target row, 1 = draft row, at position pos.
+struct Override {
+  int kind = -1, pos = -1, alt = 0;
+};
+
+struct Outcome {
+  bool error = false;
+  int acc = 0;
+  std::vector<int32_t> out;
+  int32_t flag = 0;
+  std::vector<Override> near_ties;  // top-p boundaries within 1e-6 on decision rows
+};
+
+// One batch row of chain verification: [SD] "Speculative Decoding" (accept x_i left to
+// right, stop at the first rejection and resample it, bonus token after K acceptances)
+// and "Speculative Sampling" (the acceptance ratio and the residual). T == 0 is the
+// greedy longest-prefix rule of blockwise parallel decoding ([SV], "推测解码").
+Outcome chain_eval(const ChainArgs& a, int b, const Override& ov) {
   const int K = a.K, V = a.V;
   const int32_t* x = a.draft_tokens + size_t(b) * K;
   const double* u = a.uniforms + size_t(b) * (K + 1);
-  int32_t* out = a.out_tokens + size_t(b) * (K + 1);
-  int32_t flag = 0;
+  Outcome o;
+  o.out.assign(size_t(K + 1), -1);
   std::vector<double> lp, lq;
   int acc = K;
   int emitted = -1;
+  auto note = [&](const Dist& d, int kind, int pos) {
+    if (d.margin_reach < 1e-6) o.near_ties.push_back({kind, pos, +1});
+    if (d.margin_prev < 1e-6) o.near_ties.push_back({kind, pos, -1});
+  };
+  auto alt_of = [&](int kind, int pos) { return (ov.kind == kind && ov.pos == pos) ? ov.alt : 0; };
 
   if (a.T == 0.0) {
     for (int i = 0; i <= K; ++i) {
       load_row(a.target, a.dtype, size_t(b) * (K + 1) + i, V, lp);
-      if (!row_valid(lp)) return chain_error(a, b);
+      if (!row_valid(lp)) return o.error = true, o;
       const int g = argmax_lowest(lp);
       if (i == K) {
         emitted = g;
         break;
       }
-      if (x[i] < 0 || x[i] >= V) return chain_error(a, b);
+      if (x[i] < 0 || x[i] >= V) return o.error = true, o;
       if (x[i] != g) {
         acc = i;
         emitted = g;
@@ -273,42 +300,56 @@ void chain_row(const ChainArgs& a, int b) {
   } else {
     for (int i = 0; i <= K; ++i) {
       load_row(a.target, a.dtype, size_t(b) * (K + 1) + i, V, lp);
-      if (!row_valid(lp)) return chain_error(a, b);
-      const Dist P = transform(lp, a.T, a.top_k, a.top_p);
-      if (P.topp_margin < 1e-6) flag |= FLAG_TOPP;
+      if (!row_valid(lp)) return o.error = true, o;
+      const Dist P = transform(lp, a.T, a.top_k, a.top_p, alt_of(0, i));
+      note(P, 0, i);
       if (i == K) {  // every draft accepted: bonus token from p at position K+1
         const Draw d = inverse_cdf(P.p, u[K]);
         emitted = d.token;
-        if (d.flag) flag |= FLAG_CDF;
+        if (d.flag) o.flag |= FLAG_CDF;
         break;
       }
-      if (x[i] < 0 || x[i] >= V) return chain_error(a, b);
+      if (x[i] < 0 || x[i] >= V) return o.error = true, o;
       load_row(a.draft, a.dtype, size_t(b) * K + i, V, lq);
-      if (!row_valid(lq)) return chain_error(a, b);
-      const Dist Q = transform(lq, a.T, a.top_k, a.top_p);
-      if (Q.topp_margin < 1e-6) flag |= FLAG_TOPP;
+      if (!row_valid(lq)) return o.error = true, o;
+      const Dist Q = transform(lq, a.T, a.top_k, a.top_p, alt_of(1, i));
+      note(Q, 1, i);
       const double px = P.p[x[i]], qx = Q.p[x[i]];
       double r;
       if (qx > 0.0) {
         r = px / qx;
       } else {
         r = px > 0.0 ? kInf : 0.0;
-        flag |= DIAG_Q_ZERO;
+        o.flag |= DIAG_Q_ZERO;
       }
       const double ui = u[i];
-      if (std::isfinite(r) && std::fabs(ui - r) < 1e-5) flag |= FLAG_RATIO;
+      if (std::isfinite(r) && std::fabs(ui - r) < 1e-5) o.flag |= FLAG_RATIO;
       if (ui < std::min(1.0, r)) continue;
       acc = i;
       const Draw d = inverse_cdf(residual(P.p, Q.p), u[K]);
       emitted = d.token;
-      if (d.flag) flag |= FLAG_CDF;
+      if (d.flag) o.flag |= FLAG_CDF;
       break;
     }
   }
-  a.accepted_len[b] = acc;
-  for (int j = 0; j < acc; ++j) out[j] = x[j];
-  out[acc] = emitted;
-  for (int j = acc + 1; j <= K; ++j) out[j] = -1;
+  o.acc = acc;
+  for (int j = 0; j < acc; ++j) o.out[j] = x[j];
+  o.out[acc] = emitted;
+  return o;
+}
+
+// Evaluates a batch row and sets its flags. A top-p near-tie flags the row only when
+// evaluating it with the other nucleus changes the row's output.
+void chain_row(const ChainArgs& a, int b) {
+  const Outcome base = chain_eval(a, b, Override{});
+  if (base.error) return chain_error(a, b);
+  int32_t flag = base.flag;
+  for (const Override& t : base.near_ties) {
+    const Outcome alt = chain_eval(a, b, t);
+    if (alt.error || alt.acc != base.acc || alt.out != base.out) flag |= FLAG_TOPP;
+  }
+  a.accepted_len[b] = base.acc;
+  std::copy(base.out.begin(), base.out.end(), a.out_tokens + size_t(b) * (a.K + 1));
   if (a.flags) a.flags[b] = flag;
 }
 
@@ -351,7 +392,7 @@ int oracle_transform_rows(const void* logits, int dtype, int rows, int V, double
     const Dist d = transform(l, T, top_k, top_p);
     if (pr) std::copy(d.p.begin(), d.p.end(), pr);
     if (entropy) entropy[r] = d.entropy;
-    if (topp_margin) topp_margin[r] = d.topp_margin;
+    if (topp_margin) topp_margin[r] = d.topp_margin();
     if (valid) valid[r] = 1;
   });
   return 0;
@@ -452,8 +493,8 @@ int oracle_verify_tree_typical(const void* target, int dtype, int B, int N, int 
 }
 
 // Inverse-CDF draw from norm(max(0, p - q)) (q == NULL: from p) for explicit
-// probability rows. Rows holding a negative, NaN or infinite entry, or with
-// no positive mass, give token -1.
+// probability rows. Entries are probabilities: a row holding an entry that is
+// NaN or outside [0, 1], or whose p has no positive entry, gives token -1.
 int oracle_residual_sample(const float* p, const float* q, int rows, int V, const float* uniforms,
                            int32_t* tokens, int32_t* flags, int threads) {
   if (!p || rows < 0 || V <= 0 || !uniforms || !tokens) return -1;
@@ -462,10 +503,10 @@ int oracle_residual_sample(const float* p, const float* q, int rows, int V, cons
     bool ok = true;
     for (int v = 0; v < V; ++v) {
       pr[v] = double(p[size_t(r) * V + v]);
-      if (!(pr[v] >= 0.0) || pr[v] == kInf) ok = false;
+      if (!(pr[v] >= 0.0 && pr[v] <= 1.0)) ok = false;
       if (q) {
         qr[v] = double(q[size_t(r) * V + v]);
-        if (!(qr[v] >= 0.0) || qr[v] == kInf) ok = false;
+        if (!(qr[v] >= 0.0 && qr[v] <= 1.0)) ok = false;
       }
     }
     double mass = 0.0;
