@@ -1,0 +1,379 @@
+"""Benchmark: chain verification of the B=512, K=8, V=151936 bfloat16 workload (top-k 50,
+temperature 0.8) on N GPUs, one process per GPU (weak scaling: every rank verifies its
+own batch; no collective on the data path).
+
+One step = one spec_verify_chain call over one batch (row statistics + accept scan +
+draw). Prints one JSON line (rank 0). `--impl reference` times the CPU oracle instead.
+"""
+from __future__ import annotations
+
+import argparse
+import dataclasses
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import specgen  # noqa: E402
+
+METRIC = "verified draft positions/sec and achieved HBM GB/s (fraction of 8 TB/s)"
+UNIT = "positions/s"
+L2_NOTE = "inputs larger than L2 (126 MB); no flush between steps"
+
+
+def log(*a):
+    print(*a, file=sys.stderr, flush=True)
+
+
+def workload(cfg: specgen.ChainConfig, greedy: bool) -> dict:
+    name = f"chain_B{cfg.B}_K{cfg.K}_V{cfg.V}_{cfg.dtype}_T{0.0 if greedy else cfg.temp:g}"
+    if not greedy:
+        name += (f"_topk{cfg.top_k}" if cfg.top_k else "") + \
+            (f"_topp{cfg.top_p:g}" if cfg.top_p < 1 else "")
+    name += f"_zipf{cfg.zipf:g}" if cfg.zipf else ""
+    return {"workload": name, "B": cfg.B, "K": cfg.K,
+            "V": cfg.V, "logits": cfg.dtype, "temperature": 0.0 if greedy else cfg.temp,
+            "top_k": 0 if greedy else cfg.top_k, "top_p": cfg.top_p, "l2": L2_NOTE}
+
+
+def algorithmic_bytes(cfg, greedy: bool) -> int:
+    """One read of every logit row the step must read: B*(2K+1) rows (B*(K+1) greedy)."""
+    rows = cfg.B * ((cfg.K + 1) if greedy else (2 * cfg.K + 1))
+    return rows * cfg.V * (2 if cfg.dtype == "bf16" else 4)
+
+
+def measured_peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return json.load(f), "measured"
+    except OSError:
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}, "fallback"
+
+
+def read_profile_traffic(name: str):
+    """Per-launch DRAM traffic of the row kernel from a committed ncu summary, if any."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            return json.load(f).get(name)
+    except (OSError, ValueError):
+        return None
+
+
+class ClockSampler:
+    """nvidia-smi SM clock / throttle-reason sampling during the timed region."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{index}.csv")
+
+    def start(self):
+        try:
+            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.index}",
+                                          f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
+                                          "-lms", "50"], stdout=self.fh,
+                                         stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"samples": 0}
+        self.proc.terminate()
+        self.proc.wait(timeout=10)
+        self.fh.close()
+        sm, mx, reasons = [], 0.0, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as f:
+            for line in f:
+                p = [x.strip() for x in line.split(",")]
+                if len(p) < 9:
+                    continue
+                try:
+                    sm.append(float(p[1]))
+                    mx = max(mx, float(p[2]))
+                except ValueError:
+                    continue
+                for n, v in zip(names, p[5:9]):
+                    if v.lower() == "active":
+                        reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx or None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def run_ours(args, cfg, greedy, rank, world):
+    import torch
+
+    import draft_token_verification_spec_b200 as sv
+
+    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", 0)))
+    torch.cuda.set_device(dev)
+    sv.lib()  # fail loudly if the CUDA library is missing
+    t0 = time.time()
+    target, draft = specgen.chain_logits(cfg)
+    u = specgen.chain_uniforms(cfg)
+    pick = specgen.drafter_uniforms(cfg)
+    log(f"[rank {rank}] generated inputs in {time.time() - t0:.1f}s")
+
+    def to_dev(a):
+        if a.dtype == np.uint16:
+            return torch.from_numpy(a.view(np.int16)).to(dev).view(torch.bfloat16)
+        return torch.from_numpy(a).to(dev)
+
+    tg, dg, ug = to_dev(target), to_dev(draft), to_dev(u)
+    # the drafter: x_i ~ transformed q_i (temperature 0: argmax), drawn on the GPU with
+    # the library's own transform and draw
+    if greedy:
+        xg = dg.float().argmax(dim=2).to(torch.int32).contiguous()
+    else:
+        probs, _ = sv.spec_logits_to_probs(dg, cfg.temp, cfg.top_k, cfg.top_p, with_entropy=False)
+        xg = sv.spec_residual_sample(probs.view(-1, cfg.V), None,
+                                     to_dev(pick).view(-1)).view(cfg.B, cfg.K)
+        del probs
+    torch.cuda.synchronize()
+    temp = 0.0 if greedy else cfg.temp
+    acc = torch.empty(cfg.B, dtype=torch.int32, device=dev)
+    out = torch.empty((cfg.B, cfg.K + 1), dtype=torch.int32, device=dev)
+    ws = torch.empty(sv.spec_workspace_size(cfg.B, cfg.K, cfg.V), dtype=torch.uint8, device=dev)
+
+    def step():
+        sv.spec_verify_chain(tg, None if greedy else dg, xg, ug, temp, cfg.top_k, cfg.top_p,
+                             accepted_len=acc, out_tokens=out, workspace=ws)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    status = sv.spec_get_device_status(ws)
+    assert status == 0, f"device status {status}"
+    accl = acc.cpu().numpy()
+    assert accl.min() >= 0, "error rows in the benchmark batch"
+
+    pairs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+             for _ in range(args.steps)]
+    for a, b in pairs:  # torch creates an event on its first record; the library re-records it
+        a.record()
+        b.record()
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(dev.index)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    time.sleep(0.2)
+    start.record()
+    for i in range(args.steps):
+        sv.spec_set_row_kernel_events(*pairs[i])
+        step()
+    end.record()
+    torch.cuda.synchronize()
+    clock_info = clocks.stop()
+    sv.spec_set_row_kernel_events(None, None)
+    if world > 1:
+        torch.distributed.barrier()
+    ms = start.elapsed_time(end)
+    row_ms = [a.elapsed_time(b) for a, b in pairs]
+    t = torch.tensor([ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    ms_max = float(t.item())
+    positions = cfg.B * cfg.K * world * args.steps
+    value = positions / (ms_max / 1e3)
+
+    # end to end through the same call: pinned host inputs in, results out, every step
+    e2e_steps = max(3, min(args.steps, 10))
+    h_t = torch.from_numpy(target.view(np.int16)).pin_memory() if target.dtype == np.uint16 \
+        else torch.from_numpy(target).pin_memory()
+    h_d = torch.from_numpy(draft.view(np.int16)).pin_memory() if draft.dtype == np.uint16 \
+        else torch.from_numpy(draft).pin_memory()
+    h_x = xg.cpu().pin_memory()
+    h_u = torch.from_numpy(u).pin_memory()
+    h_acc = torch.empty(cfg.B, dtype=torch.int32).pin_memory()
+    h_out = torch.empty((cfg.B, cfg.K + 1), dtype=torch.int32).pin_memory()
+    tg_raw = tg.view(torch.int16) if tg.dtype == torch.bfloat16 else tg
+    dg_raw = dg.view(torch.int16) if dg.dtype == torch.bfloat16 else dg
+    h2d = h_t.numel() * h_t.element_size() + (0 if greedy else h_d.numel() * h_d.element_size()) \
+        + h_x.numel() * 4 + h_u.numel() * 4
+    d2h = h_acc.numel() * 4 + h_out.numel() * 4
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    e0.record()
+    for _ in range(e2e_steps):
+        tg_raw.copy_(h_t, non_blocking=True)
+        if not greedy:
+            dg_raw.copy_(h_d, non_blocking=True)
+        xg.copy_(h_x, non_blocking=True)
+        ug.copy_(h_u, non_blocking=True)
+        step()
+        h_acc.copy_(acc, non_blocking=True)
+        h_out.copy_(out, non_blocking=True)
+    e1.record()
+    torch.cuda.synchronize()
+    e2e_ms = torch.tensor([e0.elapsed_time(e1) / e2e_steps], dtype=torch.float64, device=dev)
+    if world > 1:
+        torch.distributed.all_reduce(e2e_ms, op=torch.distributed.ReduceOp.MAX)
+    e2e_value = cfg.B * cfg.K * world / (float(e2e_ms.item()) / 1e3)
+
+    kernels_per_step = sv.spec_kernels_per_call("spec_verify_chain")
+    row_avg_ms = float(np.mean(row_ms))
+    alg = algorithmic_bytes(cfg, greedy)
+    peaks, peak_src = measured_peaks()
+    achieved = alg / (row_avg_ms / 1e3) / 1e9
+    return {
+        "value": value, "ms_per_step": ms_max / args.steps,
+        "roofline": {"bound": "hbm", "achieved": round(achieved, 1),
+                     "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                     "frac": round(achieved / peaks["hbm_gbs"], 4),
+                     "peak_source": peak_src + " (STREAM-style copy)",
+                     "frac_of_8TBs": round(achieved / 8000.0, 4),
+                     "kernel": "row_stats_kernel", "kernel_ms": round(row_avg_ms, 4),
+                     "algorithmic_bytes": alg,
+                     "traffic": read_profile_traffic(workload(cfg, greedy)["workload"])},
+        "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": int(h2d),
+                "d2h_bytes_per_step": int(d2h), "steps": e2e_steps},
+        "gpu_launches": kernels_per_step * args.steps,
+        "clocks": clock_info,
+        "acceptance": {"mean_accepted_len": float(accl.mean()),
+                       "emitted_per_round": float(accl.mean() + 1)},
+    }
+
+
+def oracle_drafts(cfg, target, draft, B, greedy):
+    import oracle
+
+    pick = specgen.drafter_uniforms(cfg, B)
+    if greedy:
+        lf = specgen.bf16_bits_to_f32(draft) if draft.dtype == np.uint16 else draft
+        return np.argmax(lf, axis=2).astype(np.int32)
+    toks = np.empty((B, cfg.K), np.int32)
+    for b in range(B):
+        probs = oracle.transform_rows(draft[b], cfg.temp, cfg.top_k, cfg.top_p)[0]
+        toks[b] = oracle.residual_sample(probs.astype(np.float32), None, pick[b])[0]
+    return toks
+
+
+def time_oracle(cfg, greedy, rows: int, threads: int):
+    """Seconds the oracle takes to verify `rows` batch rows of the workload."""
+    import oracle
+
+    target, draft = specgen.chain_logits(cfg, rows)
+    u = specgen.chain_uniforms(cfg, rows)
+    toks = oracle_drafts(cfg, target, draft, rows, greedy)
+    t0 = time.perf_counter()
+    oracle.verify_chain(target, None if greedy else draft, toks, u, 0.0 if greedy else cfg.temp,
+                        cfg.top_k, cfg.top_p, threads=threads)
+    return time.perf_counter() - t0
+
+
+def cpu_baseline(cfg, greedy, budget_s: float = 15.0) -> dict:
+    threads = os.cpu_count() or 1
+    rows = max(1, threads)
+    dt = time_oracle(cfg, greedy, rows, threads)
+    grow = int(min(cfg.B, max(rows, rows * budget_s / max(dt, 1e-3) / 2)))
+    if grow > rows:
+        rows, dt = grow, time_oracle(cfg, greedy, grow, threads)
+    return {"value": rows * cfg.K / dt, "unit": UNIT, "cores": threads, "kind": "oracle",
+            "sample": f"first {rows} of {cfg.B} batch rows ({rows * cfg.K} positions), "
+                      f"{threads} threads over batch rows, {dt:.1f}s"}
+
+
+def run_reference(args, cfg, greedy) -> dict:
+    """The oracle, as it stands, on the host cores: each step verifies a bounded sample."""
+    import oracle
+
+    threads = os.cpu_count() or 1
+    wave = time_oracle(cfg, greedy, threads, threads)  # one batch row per thread
+    waves = int(150.0 / max(1, args.steps + args.warmup) / max(wave, 1e-4))
+    per_step = min(cfg.B, threads * max(1, waves))
+    target, draft = specgen.chain_logits(cfg, per_step)
+    u = specgen.chain_uniforms(cfg, per_step)
+    toks = oracle_drafts(cfg, target, draft, per_step, greedy)
+    temp = 0.0 if greedy else cfg.temp
+
+    def step():
+        oracle.verify_chain(target, None if greedy else draft, toks, u, temp, cfg.top_k,
+                            cfg.top_p, threads=threads)
+
+    for _ in range(args.warmup):
+        step()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        step()
+    dt = time.perf_counter() - t0
+    value = per_step * cfg.K * args.steps / dt
+    sample = (f"first {per_step} of {cfg.B} batch rows per step ({per_step * cfg.K} positions), "
+              f"{threads} threads over batch rows")
+    return {"value": value, "ms_per_step": dt / args.steps * 1e3,
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--config", type=int, default=5, choices=sorted(specgen.CHAIN_CONFIGS))
+    ap.add_argument("--greedy", action="store_true", help="temperature-0 variant")
+    ap.add_argument("--batch", type=int, default=None,
+                    help="override the batch size (smaller cases for profiler captures)")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    assert args.warmup >= 3, "at least 3 warm-up steps"
+    cfg = specgen.CHAIN_CONFIGS[args.config]
+    if args.batch:
+        cfg = dataclasses.replace(cfg, B=args.batch)
+    rank = int(os.environ.get("RANK", 0))
+    world = int(os.environ.get("WORLD_SIZE", 1))
+    base = {"metric": METRIC, "unit": UNIT, "n_gpus": args.gpus, "steps": args.steps,
+            "warmup": args.warmup, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "data": "synthetic (seeded generator; no dataset)",
+            "config": workload(cfg, args.greedy)}
+
+    if args.impl == "reference":
+        if rank != 0:
+            return
+        res = run_reference(args, cfg, args.greedy)
+        print(json.dumps({**base, "impl": "reference", "dtype": "f64", **res}), flush=True)
+        return
+
+    if world > 1:
+        import datetime
+
+        import torch
+        torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", 0)))
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+    try:
+        res = run_ours(args, cfg, args.greedy, rank, world)
+        if rank == 0:
+            line = {**base, "dtype": "f32", "value": res.pop("value"),
+                    "ms_per_step": res.pop("ms_per_step"), **res}
+            if not args.no_cpu_baseline:
+                line["cpu_baseline"] = cpu_baseline(cfg, args.greedy)
+            print(json.dumps(line), flush=True)
+    finally:
+        if world > 1:
+            import torch
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -170,7 +170,7 @@ def tree_inputs(cfg: TreeConfig, B: int | None = None):
             s = cfg.heads[d - 1] if d >= 1 else 1
             order = np.lexsort((np.arange(V), -h))  # descending value, lower id first
             head_tok[b, d, :s] = order[:s]
-    tokens = head_tok[:, depth, rank].astype(np.int32)
+    tokens = np.ascontiguousarray(head_tok[:, depth, rank], dtype=np.int32)
     st = np.uint16 if cfg.dtype == "bf16" else np.float32
     logits = np.empty((B, N, V), st)
     child0 = {int(parent[c]): c for c in range(N - 1, 0, -1) if rank[c] == 0}

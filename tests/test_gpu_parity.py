@@ -31,25 +31,26 @@ def gpu_chain(target, draft, toks, u, temp, top_k=0, top_p=1.0):
     return acc.cpu().numpy(), out.cpu().numpy()
 
 
-def assert_chain_parity(acc_g, out_g, acc_r, out_r, flags, rows=None):
+def assert_chain_parity(acc_g, out_g, acc_r, out_r, flags, budget=False):
     ok = (flags & oracle.PARITY_FLAGS) == 0
     same = (acc_g == acc_r) & np.all(out_g == out_r, axis=1)
     bad = np.nonzero(~same & ok)[0]
     assert bad.size == 0, (f"{bad.size} unflagged mismatches, first rows {bad[:5].tolist()}: "
                            f"gpu {acc_g[bad[:3]]} {out_g[bad[:3]]} oracle {acc_r[bad[:3]]} "
                            f"{out_r[bad[:3]]}")
-    _STATS["rows"] += len(acc_r)
-    _STATS["flagged"] += int((~ok).sum())
+    if budget:  # workload rows only; the edge-case tests build exact ties on purpose
+        _STATS["rows"] += len(acc_r)
+        _STATS["flagged"] += int((~ok).sum())
     return int((~ok).sum())
 
 
-def run_case(target, draft, toks, u, temp, top_k=0, top_p=1.0, rows=None):
+def run_case(target, draft, toks, u, temp, top_k=0, top_p=1.0, rows=None, budget=False):
     acc_g, out_g = gpu_chain(target, draft, toks, u, temp, top_k, top_p)
     if rows is None:
         rows = np.arange(target.shape[0])
     acc_r, out_r, flags = oracle.verify_chain(target[rows], None if draft is None else draft[rows],
                                               toks[rows], u[rows], temp, top_k, top_p)
-    assert_chain_parity(acc_g[rows], out_g[rows], acc_r, out_r, flags)
+    assert_chain_parity(acc_g[rows], out_g[rows], acc_r, out_r, flags, budget)
     return acc_g, out_g
 
 
@@ -59,7 +60,7 @@ def run_case(target, draft, toks, u, temp, top_k=0, top_p=1.0, rows=None):
                                    (specgen.CFG5, 6)], ids=lambda x: getattr(x, "name", str(x)))
 def test_chain_workloads_small_batch(cfg, B):
     target, draft, toks, u, temp = chain_case(cfg, B)
-    acc, out = run_case(target, draft, toks, u, temp, cfg.top_k, cfg.top_p)
+    acc, out = run_case(target, draft, toks, u, temp, cfg.top_k, cfg.top_p, budget=True)
     check_chain_invariants(acc, out, toks, cfg.K, cfg.V)
 
 
@@ -76,9 +77,10 @@ def test_chain_cfg5_full_size_sampled_rows():
     cfg = specgen.CFG5
     target, draft, toks, u, temp = chain_case(cfg)
     rows = np.unique(np.linspace(0, cfg.B - 1, 24).astype(int))
-    acc, out = run_case(target, draft, toks, u, temp, cfg.top_k, cfg.top_p, rows=rows)
+    acc, out = run_case(target, draft, toks, u, temp, cfg.top_k, cfg.top_p, rows=rows,
+                        budget=True)
     check_chain_invariants(acc, out, toks, cfg.K, cfg.V)
-    acc_g, out_g = run_case(target, None, toks, u, 0.0)         # greedy: every row
+    acc_g, out_g = run_case(target, None, toks, u, 0.0, budget=True)  # greedy: every row
     check_chain_invariants(acc_g, out_g, toks, cfg.K, cfg.V)
 
 
@@ -86,16 +88,17 @@ def test_chain_cfg3_full_size_sampled_rows():
     cfg = specgen.CFG3
     target, draft, toks, u, temp = chain_case(cfg)
     rows = np.unique(np.linspace(0, cfg.B - 1, 16).astype(int))
-    acc, out = run_case(target, draft, toks, u, temp, cfg.top_k, cfg.top_p, rows=rows)
+    acc, out = run_case(target, draft, toks, u, temp, cfg.top_k, cfg.top_p, rows=rows,
+                        budget=True)
     check_chain_invariants(acc, out, toks, cfg.K, cfg.V)
 
 
 def test_chain_cfg2_full_size_all_rows():
     cfg = specgen.CFG2
     target, draft, toks, u, temp = chain_case(cfg)
-    run_case(target, draft, toks, u, temp)
+    run_case(target, draft, toks, u, temp, budget=True)
     target, draft, toks, u, _ = chain_case(cfg, greedy=True)
-    run_case(target, None, toks, u, 0.0)
+    run_case(target, None, toks, u, 0.0, budget=True)
 
 
 # ------------------------------------------------------------------ edge cases
@@ -140,7 +143,7 @@ def test_chain_sixteen_cta_cluster():
 def test_chain_many_positions(K):
     target, draft, toks, u = _rand_chain(K, 6, K, 300, "bf16", draft_noise=0.05)
     acc, out = run_case(target, draft, toks, u, 1.0)
-    assert acc.max() > 2
+    assert acc.max() >= min(K, 3)
 
 
 @pytest.mark.parametrize("top_k,top_p", [(1, 1.0), (2, 1.0), (9, 1.0), (299, 1.0), (0, 1e-4),
@@ -323,7 +326,8 @@ def test_residual_sample(V, with_q):
 
 
 def test_flagged_row_budget():
-    """Over every chain row checked in this module, flagged rows stay under 1e-4."""
+    """Over the workload rows checked in this module, flagged rows stay under 1e-4 (at
+    most one when fewer than 10^4 rows were checked)."""
     if _STATS["rows"] == 0:
         pytest.skip("run with the other parity tests")
     assert _STATS["flagged"] <= max(1, 1e-4 * _STATS["rows"]), _STATS
