@@ -22,11 +22,13 @@ constexpr unsigned long long kWaitLimitNs = 2000000000ull;  // bound on any copy
 enum : int32_t { ROW_OK = 0, ROW_INVALID = 1, ROW_TIMEOUT = 2 };
 
 // Per-logit-row statistics that define the transformed distribution:
-//   p(v) = kept(v) ? exp2((l_v - m) * c) / z : 0,
+//   p(v) = kept(v) ? exp2(l_v * c - mc) / z : 0,
 //   kept(v) = key(l_v) > thr_key || (key(l_v) == thr_key && v <= cutoff),
-// with c = log2(e) / T. thr_key = 0 keeps every row entry.
+// with c = log2(e) / T and mc = fl(m * c), m the largest logit. thr_key = 0 keeps every
+// row entry. The rounding of mc scales every weight of the row by the same factor, so
+// it cancels in p.
 struct RowStats {
-  float m;           // largest logit
+  float mc;          // fl(m * c), m the largest logit
   float z;           // sum over the kept set of exp2((l - m) * c)
   float entropy;     // entropy (nats) of the transformed distribution, if computed
   uint32_t thr_key;  // boundary key of the kept prefix in (value desc, id asc) order
@@ -47,6 +49,13 @@ __device__ __forceinline__ uint32_t f32_key(float x) {
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
+// max with NaN propagation (PTX max.NaN).
+__device__ __forceinline__ float fmax_nan(float a, float b) {
+  float r;
+  asm("max.NaN.f32 %0, %1, %2;" : "=f"(r) : "f"(a), "f"(b));
+  return r;
+}
+
 template <typename T>
 struct Elem;
 
@@ -65,6 +74,16 @@ struct Elem<float> {
     return __ldg(static_cast<const float*>(base) + i);
   }
   __device__ static __forceinline__ uint32_t key(float x) { return f32_key(x); }
+  // Largest value of a 16-byte vector; NaN if any entry is NaN.
+  __device__ static __forceinline__ float vmax_nan(const uint4& w) {
+    return fmax_nan(fmax_nan(__uint_as_float(w.x), __uint_as_float(w.y)),
+                    fmax_nan(__uint_as_float(w.z), __uint_as_float(w.w)));
+  }
+  // Largest value of a 16-byte vector (entries are not NaN).
+  __device__ static __forceinline__ float vmax(const uint4& w) {
+    return fmaxf(fmaxf(__uint_as_float(w.x), __uint_as_float(w.y)),
+                 fmaxf(__uint_as_float(w.z), __uint_as_float(w.w)));
+  }
 };
 
 template <>
@@ -85,6 +104,19 @@ struct Elem<__nv_bfloat16> {
     return __uint_as_float(uint32_t(h) << 16);
   }
   __device__ static __forceinline__ uint32_t key(float x) { return f32_key(x) >> 16; }
+  __device__ static __forceinline__ __nv_bfloat162 pair(uint32_t u) {
+    return *reinterpret_cast<const __nv_bfloat162*>(&u);
+  }
+  // Largest value of a 16-byte vector (packed bf16x2 max); NaN if any entry is NaN.
+  __device__ static __forceinline__ float vmax_nan(const uint4& w) {
+    const __nv_bfloat162 r = __hmax2_nan(__hmax2_nan(pair(w.x), pair(w.y)),
+                                         __hmax2_nan(pair(w.z), pair(w.w)));
+    return fmax_nan(__low2float(r), __high2float(r));
+  }
+  __device__ static __forceinline__ float vmax(const uint4& w) {
+    const __nv_bfloat162 r = __hmax2(__hmax2(pair(w.x), pair(w.y)), __hmax2(pair(w.z), pair(w.w)));
+    return fmaxf(__low2float(r), __high2float(r));
+  }
 };
 
 __device__ __forceinline__ bool kept(uint32_t key, int id, uint32_t thr_key, int cutoff) {
@@ -98,8 +130,11 @@ __device__ __forceinline__ float ex2(float x) {
   return y;
 }
 
-// Unnormalised weight exp((l - m) / T) of one logit, as exp2((l - m) * c).
-__device__ __forceinline__ float weight(float l, float m, float c) { return ex2((l - m) * c); }
+// Exponent l * c - mc = (l - m) / T in log2 units, with one rounding (FFMA).
+__device__ __forceinline__ float wexp(float l, float c, float mc) { return fmaf(l, c, -mc); }
+
+// Unnormalised weight exp((l - m) / T) of one logit.
+__device__ __forceinline__ float weight(float l, float c, float mc) { return ex2(wexp(l, c, mc)); }
 
 __device__ __forceinline__ unsigned long long to_fx(float mass01) {
   return __float2ull_rn(mass01 * kFxF);

@@ -127,7 +127,7 @@ __device__ __forceinline__ void load8(const T* row, int v0, int V, bool aligned,
 // Probability of entry v under the transformed distribution described by s.
 template <typename T>
 __device__ __forceinline__ float prob(const RowStats& s, float l, int v) {
-  return kept(Elem<T>::key(l), v, s.thr_key, s.cutoff) ? weight(l, s.m, s.c) / s.z : 0.0f;
+  return kept(Elem<T>::key(l), v, s.thr_key, s.cutoff) ? weight(l, s.c, s.mc) / s.z : 0.0f;
 }
 
 }  // namespace sv
