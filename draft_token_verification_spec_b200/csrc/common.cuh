@@ -19,7 +19,9 @@ constexpr double kFxInv = 1.0 / 4398046511104.0;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;  // bound on any copy wait
 
-enum : int32_t { ROW_OK = 0, ROW_INVALID = 1, ROW_TIMEOUT = 2 };
+// ROW_FALLBACK: the streaming kernel could not settle the row from its candidates;
+// the cluster kernel recomputes it (never seen by consumers).
+enum : int32_t { ROW_OK = 0, ROW_INVALID = 1, ROW_TIMEOUT = 2, ROW_FALLBACK = 3 };
 
 // Per-logit-row statistics that define the transformed distribution:
 //   p(v) = kept(v) ? exp2(l_v * c - mc) / z : 0,
@@ -135,6 +137,10 @@ __device__ __forceinline__ float wexp(float l, float c, float mc) { return fmaf(
 
 // Unnormalised weight exp((l - m) / T) of one logit.
 __device__ __forceinline__ float weight(float l, float c, float mc) { return ex2(wexp(l, c, mc)); }
+
+// Entropy term e * zx of one entry; an entry of weight 0 (a -inf logit) contributes 0,
+// not 0 * -inf.
+__device__ __forceinline__ float ent_term(float e, float zx) { return e > 0.0f ? e * zx : 0.0f; }
 
 __device__ __forceinline__ unsigned long long to_fx(float mass01) {
   return __float2ull_rn(mass01 * kFxF);

@@ -1,18 +1,23 @@
-// Row statistics kernel: one thread-block cluster per logit row.
+// Row statistics kernel: persistent thread-block clusters, one logit row per cluster
+// at a time.
 //
-// Each CTA of the cluster stages a contiguous slice of the row in shared memory with
-// 1-D bulk copies (cp.async.bulk, completion on an mbarrier); the cluster then combines
-// its partial results through distributed shared memory (DSMEM):
-//   - the row maximum (packed bf16x2 max with NaN propagation) and row validity;
-//   - greedy: the lowest index holding the maximum;
-//   - no truncation: the softmax normaliser (and entropy) in one exp pass;
-//   - top-k (fast path, k <= 256): t0 = the largest over the cluster's CTAs of each
-//     CTA's k-th largest per-thread maximum, so at least k entries reach t0; a filter
-//     pass keeps the few entries >= t0, every CTA gathers them and selects the top k
-//     exactly with a local radix select — no exp over the row;
-//   - otherwise (top-p, or a fast path that does not apply): exact selection by radix
+// A cluster of C CTAs walks rows cid, cid + G, cid + 2G, ... (G clusters resident). Each
+// CTA owns a contiguous slice of every row and keeps a ring of kNBuf slice buffers in
+// shared memory: while it works on one row, 1-D bulk copies (cp.async.bulk, completion
+// on an mbarrier per buffer) bring in the next rows' slices. Per row the cluster
+// combines partial results through distributed shared memory (DSMEM):
+//   - the row maximum (packed bf16x2 max with NaN propagation), validity and, in greedy
+//     mode, the lowest index holding the maximum — one exchange;
+//   - no truncation: the softmax normaliser (and entropy term) in one exp pass;
+//   - top-k (fast path, k <= 256): every warp takes the ceil(k/8)-th largest of its
+//     per-thread maxima by a ballot radix select; the smallest of a CTA's warp values
+//     is a value that k of its entries reach, and the largest over the cluster (t0)
+//     rides in the maximum exchange. A filter pass keeps the few entries >= t0, every
+//     CTA gathers them and selects the top k exactly — no exp over the row;
+//   - otherwise (top-p, or a fast path that does not fit): exact selection by radix
 //     select over order-preserving keys, 8 bits per level, with fixed-point masses.
-// It stores a RowStats record or writes the transformed probabilities.
+// It stores a RowStats record (and the kept ids of top-k rows) or writes the
+// transformed probabilities.
 //
 // This is the sampling transform of "Speculative Sampling" (spec-decoding-i notes, last
 // bullet: transform the probabilities first, then apply the rejection scheme) and the
@@ -27,9 +32,15 @@ namespace sv {
 
 enum : int { RS_GREEDY = 1, RS_ENTROPY = 2, RS_WRITE_PROBS = 4 };
 
+#ifndef SV_NBUF
+#define SV_NBUF 2
+#endif
+constexpr int kNBuf = SV_NBUF;     // slice buffers per CTA (ring)
 constexpr int kBulkChunk = 16384;
 constexpr int kCandCap = 512;      // candidates one CTA may hold in the top-k filter
 constexpr int kGatherCap = 1024;   // candidates a cluster may hold for exact selection
+constexpr int kMaxCluster = 16;
+constexpr int kKeptCap = 256;      // kept ids listed per top-k row (top_k <= 256)
 constexpr float kS1Fx = 4294967296.0f;  // 2^32: signed fixed point for entropy terms
 
 struct RowJob {
@@ -39,19 +50,24 @@ struct RowJob {
   long long rows;
   int V;
   int slice;           // elements per CTA slice (multiple of 16)
+  int slice_bytes;     // bytes reserved per slice buffer (multiple of 128)
   float c;             // log2(e) / T   (unused in greedy mode)
   float inv_t;         // 1 / T
   int top_k;           // 1 <= top_k < V, else off
   float top_p;         // < 1: on
   int flags;
   RowStats* stats;     // [rows] or NULL
+  int32_t* kept_n;     // [rows] or NULL: number of ids in kept_ids (0: no list)
+  int32_t* kept_ids;   // [rows][kKeptCap] or NULL: the kept set of top-k rows
   float* probs;        // RS_WRITE_PROBS: [rows][V]
   float* entropy;      // RS_WRITE_PROBS: [rows] or NULL
   int32_t* dev_status; // set to 1 on a copy timeout (may be NULL)
+  const int32_t* row_list;   // if set: process rows row_list[0 .. *row_count) only
+  const int32_t* row_count;
 };
 
 struct __align__(16) RowAux {
-  uint64_t bar;
+  uint64_t bar[kNBuf];
   // exchange slots, double-buffered by phase
   float xm[2];
   int xi[2];
@@ -80,49 +96,69 @@ struct __align__(16) RowAux {
   uint32_t scr_u32[kWarps];
   float scr_m[kWarps];
   int scr_i[kWarps];
+  float scr_t[kWarps];
   long long scr_s64[kWarps];
+  int cnt_off[kMaxCluster + 1];
   uint32_t lh[256];  // CTA-local histogram
   int found_bin;
   int found;
   unsigned long long found_above;
   int ccount;
-  uint32_t sel_key;
   int sel_id;
+  int broken;        // a copy wait timed out: no further copies are issued
+  int pending;       // bit b: a copy into buffer b was issued and not yet waited for
 };
 
-// Stages n elements starting at g into buf; element j lands at byte pad + j * E with
-// pad = g mod 16, so the 16-byte-aligned middle of the slice moves by bulk copy and
-// the unaligned head and tail (< 16 bytes each) by plain loads. Returns false if the
-// copy did not complete within the wait limit.
+// Where one CTA's slice of a row lives and how it is split: the 16-byte-aligned middle
+// moves by bulk copy, the unaligned head and tail (< 16 bytes each) by plain loads.
+// Element j of the slice lands at byte pad + j * E of the buffer.
+struct SliceLoc {
+  const unsigned char* g;
+  int n, pad, head, mid, tail;
+};
+
 template <typename T>
-__device__ bool stage_slice(const T* g, int n, unsigned char* buf, uint64_t* bar, int* pad_out) {
+__device__ __forceinline__ SliceLoc slice_loc(const RowJob& job, long long row, int rank) {
   constexpr int E = Elem<T>::kBytes;
-  const uintptr_t a = reinterpret_cast<uintptr_t>(g);
-  const int pad = int(a & 15u);
-  const int bytes = n * E;
-  const int head = min(bytes, (16 - pad) & 15);
-  const int mid = ((bytes - head) >> 4) << 4;
-  const int tail = bytes - head - mid;
-  *pad_out = pad;
-  if (threadIdx.x == 0) mbar_init(bar, 1);
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    mbar_arrive_expect_tx(bar, uint32_t(mid));
-    const char* gs = reinterpret_cast<const char*>(g) + head;
-    unsigned char* d = buf + pad + head;
-    for (int off = 0; off < mid; off += kBulkChunk)
-      bulk_g2s(d + off, gs + off, uint32_t(min(kBulkChunk, mid - off)), bar);
-  }
-  const int hE = head / E, tE = tail / E;
+  const int V = job.V;
+  const T* src = (row < job.rows0)
+                     ? static_cast<const T*>(job.base0) + size_t(row) * V
+                     : static_cast<const T*>(job.base1) + size_t(row - job.rows0) * V;
+  SliceLoc s;
+  const int s0 = rank * job.slice;
+  s.n = max(0, min(V - s0, job.slice));
+  s.g = reinterpret_cast<const unsigned char*>(src + s0);
+  s.pad = int(reinterpret_cast<uintptr_t>(s.g) & 15u);
+  const int bytes = s.n * E;
+  s.head = min(bytes, (16 - s.pad) & 15);
+  s.mid = ((bytes - s.head) >> 4) << 4;
+  s.tail = bytes - s.head - s.mid;
+  return s;
+}
+
+// Thread 0: starts the bulk copy of a slice into buf.
+__device__ __forceinline__ void issue_slice(const SliceLoc& s, unsigned char* buf, uint64_t* bar) {
+  mbar_arrive_expect_tx(bar, uint32_t(s.mid));
+  unsigned char* d = buf + s.pad + s.head;
+  for (int off = 0; off < s.mid; off += kBulkChunk)
+    bulk_g2s(d + off, s.g + s.head + off, uint32_t(min(kBulkChunk, s.mid - off)), bar);
+}
+
+// All threads: plain loads of the head and tail, then wait for the bulk copy. Returns
+// false if the copy did not complete within the wait limit.
+template <typename T>
+__device__ __forceinline__ bool finish_slice(const SliceLoc& s, unsigned char* buf,
+                                             uint64_t* bar, uint32_t parity) {
+  constexpr int E = Elem<T>::kBytes;
+  const int hE = s.head / E, tE = s.tail / E;
   for (int j = threadIdx.x; j < hE + tE; j += kThreads) {
-    const int e = (j < hE) ? j : (n - tE + (j - hE));
+    const int e = (j < hE) ? j : (s.n - tE + (j - hE));
     if (E == 2)
-      reinterpret_cast<uint16_t*>(buf + pad)[e] = reinterpret_cast<const uint16_t*>(g)[e];
+      reinterpret_cast<uint16_t*>(buf + s.pad)[e] = reinterpret_cast<const uint16_t*>(s.g)[e];
     else
-      reinterpret_cast<uint32_t*>(buf + pad)[e] = reinterpret_cast<const uint32_t*>(g)[e];
+      reinterpret_cast<uint32_t*>(buf + s.pad)[e] = reinterpret_cast<const uint32_t*>(s.g)[e];
   }
-  bool ok = mbar_wait(bar, 0);
-  if (!ok) mbar_wait(bar, 0);  // give an in-flight copy one more bounded chance to land
+  const bool ok = mbar_wait(bar, parity);
   __syncthreads();
   return ok;
 }
@@ -268,33 +304,15 @@ struct RowCtx {
     return aux->ccount;
   }
 
-  // k-th largest (1 <= k <= kThreads) of the keys the block's threads pass in, by an
-  // 8-bit-per-level radix select over a CTA-local histogram.
-  __device__ uint32_t block_kth_key(uint32_t key, int k) {
-    constexpr int KB = Elem<T>::kKeyBits;
-    uint32_t prefix = 0, pmask = 0, need = uint32_t(k);
-    for (int shift = KB - 8; shift >= 0; shift -= 8) {
-      aux->lh[threadIdx.x] = 0;
-      __syncthreads();
-      if ((key & pmask) == prefix) atomicAdd(&aux->lh[(key >> shift) & 255u], 1u);
-      __syncthreads();
-      find_desc_bin<uint32_t>(aux->lh, need);
-      __syncthreads();
-      need -= uint32_t(aux->found_above);
-      prefix |= uint32_t(aux->found_bin) << shift;
-      pmask |= 255u << shift;
-      __syncthreads();
-    }
-    return prefix;
-  }
-
   template <typename U>
   __device__ __forceinline__ U* remote(U* p, int r) const {
     return cl.map_shared_rank(p, r);
   }
 
-  // Cluster-wide (max, lowest index, OR of flags, max of t).
-  __device__ void xchg_maxloc(float& m, int& i, int& bad, float& t) {
+  // Row exchange: cluster-wide (max, lowest index on ties, OR of flags, max of t), where
+  // t enters per warp and is reduced by its minimum within each CTA. Lanes 0..C-1 of
+  // every warp read the C ranks' slots in parallel; no block barrier follows.
+  __device__ void xchg_row(float& m, int& i, int& bad, float& t) {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {
@@ -306,25 +324,38 @@ struct RowCtx {
     if (lane == 0) {
       aux->scr_m[warp] = m;
       aux->scr_i[warp] = i;
+      aux->scr_t[warp] = t;
     }
     __syncthreads();
     if (threadIdx.x == 0) {
-      float M = aux->scr_m[0];
+      float M = aux->scr_m[0], Tm = aux->scr_t[0];
       int I = aux->scr_i[0];
-      for (int w = 1; w < kWarps; ++w) maxloc_combine(M, I, aux->scr_m[w], aux->scr_i[w]);
+      for (int w = 1; w < kWarps; ++w) {
+        maxloc_combine(M, I, aux->scr_m[w], aux->scr_i[w]);
+        Tm = fminf(Tm, aux->scr_t[w]);
+      }
       aux->xm[ph] = M;
       aux->xi[ph] = I;
       aux->xbad[ph] = bad;
-      aux->xt[ph] = t;
+      aux->xt[ph] = Tm;
     }
     cl.sync();
     float M = -INFINITY, Tm = -INFINITY;
     int I = INT_MAX, Bd = 0;
-    for (int r = 0; r < C; ++r) {
-      const RowAux* ra = remote(aux, r);
-      maxloc_combine(M, I, ra->xm[ph], ra->xi[ph]);
-      Bd |= ra->xbad[ph];
-      Tm = fmaxf(Tm, ra->xt[ph]);
+    if (lane < C) {
+      const RowAux* ra = remote(aux, lane);
+      M = ra->xm[ph];
+      I = ra->xi[ph];
+      Bd = ra->xbad[ph];
+      Tm = ra->xt[ph];
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const float m2 = __shfl_xor_sync(0xffffffffu, M, o);
+      const int i2 = __shfl_xor_sync(0xffffffffu, I, o);
+      maxloc_combine(M, I, m2, i2);
+      Bd |= __shfl_xor_sync(0xffffffffu, Bd, o);
+      Tm = fmaxf(Tm, __shfl_xor_sync(0xffffffffu, Tm, o));
     }
     m = M;
     i = I;
@@ -333,57 +364,8 @@ struct RowCtx {
     ph ^= 1;
   }
 
-  // Cluster-wide minimum (each thread passes a value; NaN never occurs here).
-  __device__ float xchg_min(float v) {
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) v = fminf(v, __shfl_xor_sync(0xffffffffu, v, o));
-    __syncthreads();
-    if (lane == 0) aux->scr_m[warp] = v;
-    __syncthreads();
-    if (threadIdx.x == 0) {
-      float M = aux->scr_m[0];
-      for (int w = 1; w < kWarps; ++w) M = fminf(M, aux->scr_m[w]);
-      aux->xm[ph] = M;
-    }
-    cl.sync();
-    float M = INFINITY;
-    for (int r = 0; r < C; ++r) M = fminf(M, remote(aux, r)->xm[ph]);
-    ph ^= 1;
-    return M;
-  }
-
-  // Cluster-wide minimum of an int (the lowest index of something).
-  __device__ int xchg_min_int(int v) {
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) v = min(v, __shfl_xor_sync(0xffffffffu, v, o));
-    __syncthreads();
-    if (lane == 0) aux->scr_i[warp] = v;
-    __syncthreads();
-    if (threadIdx.x == 0) {
-      int M = aux->scr_i[0];
-      for (int w = 1; w < kWarps; ++w) M = min(M, aux->scr_i[w]);
-      aux->xi[ph] = M;
-    }
-    cl.sync();
-    int M = INT_MAX;
-    for (int r = 0; r < C; ++r) M = min(M, remote(aux, r)->xi[ph]);
-    ph ^= 1;
-    return M;
-  }
-
-  __device__ unsigned long long xchg_sum_u64(unsigned long long v) {
-    v = block_sum_u64(v, aux->scr_u64);
-    if (threadIdx.x == 0) aux->xu64[ph] = v;
-    cl.sync();
-    unsigned long long s = 0;
-    for (int r = 0; r < C; ++r) s += remote(aux, r)->xu64[ph];
-    ph ^= 1;
-    return s;
-  }
-
-  // Two sums in one exchange (fixed-point mass and float entropy term).
+  // Cluster sums of a fixed-point mass and a float term (parallel remote reads; the
+  // shuffle tree fixes the summation order).
   __device__ void xchg_sum_u64_f64(unsigned long long& a, double& b) {
     a = block_sum_u64(a, aux->scr_u64);
     b = block_sum_f64(b, aux->scr_f64);
@@ -392,25 +374,28 @@ struct RowCtx {
       aux->xf64[ph] = b;
     }
     cl.sync();
+    const int lane = threadIdx.x & 31;
     unsigned long long s = 0;
     double t = 0.0;
-    for (int r = 0; r < C; ++r) {
-      s += remote(aux, r)->xu64[ph];
-      t += remote(aux, r)->xf64[ph];
+    if (lane < C) {
+      s = remote(aux, lane)->xu64[ph];
+      t = remote(aux, lane)->xf64[ph];
     }
-    a = s;
-    b = t;
+    a = warp_sum_u64(s);
+    b = warp_sum_f64(t);
     ph ^= 1;
   }
 
+  __device__ unsigned long long xchg_sum_u64(unsigned long long v) {
+    double unused = 0.0;
+    xchg_sum_u64_f64(v, unused);
+    return v;
+  }
+
   __device__ double xchg_sum_f64(double v) {
-    v = block_sum_f64(v, aux->scr_f64);
-    if (threadIdx.x == 0) aux->xf64[ph] = v;
-    cl.sync();
-    double s = 0.0;
-    for (int r = 0; r < C; ++r) s += remote(aux, r)->xf64[ph];
-    ph ^= 1;
-    return s;
+    unsigned long long unused = 0;
+    xchg_sum_u64_f64(unused, v);
+    return v;
   }
 
   __device__ long long block_sum_s64(long long v) {
@@ -630,36 +615,41 @@ struct RowCtx {
   }
 
   // ---------------------------------------------------------------- top-k fast path
-  // t0 is a lower bound on the row's k-th largest value (some CTA holds k entries >= t0).
-  // Collects the entries >= t0, gathers them in every CTA, and selects the top k among
-  // them exactly. Returns false (uniformly across the cluster) when the candidates do not
-  // fit; the caller then runs radix_topk.
+  // t0 is a value that at least k entries of the row reach. Collects the entries >= t0,
+  // gathers them in every CTA, and selects the top k among them exactly. Returns false
+  // (uniformly across the cluster) when the candidates do not fit; the caller then runs
+  // radix_topk. On success rank 0 of the cluster lists the kept ids.
   __device__ bool filter_topk(int k, float t0, float c, float mc, bool want_ent, uint32_t& thr,
-                              int& cut, unsigned long long& zfx, double& S1) {
+                              int& cut, unsigned long long& zfx, double& S1, int32_t* ids_out,
+                              int32_t* n_out) {
     constexpr int KB = Elem<T>::kKeyBits;
+    const int lane = threadIdx.x & 31;
     const int mine = collect_at_least(t0);
     if (threadIdx.x == 0) aux->xcnt[ph] = uint32_t(mine);
     cl.sync();
-    int total = 0, ovf = 0;
-    for (int q = 0; q < C; ++q) {
-      const int cq = int(remote(aux, q)->xcnt[ph]);
-      ovf |= cq > kCandCap;
-      total += cq;
-    }
-    const int slot = ph;
-    ph ^= 1;
-    if (ovf || total < k || total > kGatherCap) return false;
-    // every CTA gathers the cluster's candidates
-    for (int i = threadIdx.x; i < total; i += kThreads) {
-      int q = 0, base = 0;
-      for (;; ++q) {
-        const int cq = int(remote(aux, q)->xcnt[slot]);
-        if (i < base + cq) break;
-        base += cq;
+    if (threadIdx.x < 32) {  // counts of every rank -> offsets
+      const int cq = lane < C ? int(remote(aux, lane)->xcnt[ph]) : 0;
+      int inc = cq;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int u = __shfl_up_sync(0xffffffffu, inc, o);
+        if (lane >= o) inc += u;
       }
+      const unsigned big = __ballot_sync(0xffffffffu, cq > kCandCap);
+      if (lane <= C) aux->cnt_off[lane] = inc - cq;  // lane C holds the total
+      if (lane == 0) aux->found = big ? 1 : 0;
+    }
+    ph ^= 1;
+    __syncthreads();
+    const int total = aux->cnt_off[C];
+    if (aux->found || total < k || total > kGatherCap) return false;
+    // every CTA gathers the cluster's candidates (one remote load per candidate)
+    for (int i = threadIdx.x; i < total; i += kThreads) {
+      int q = 0;
+      while (i >= aux->cnt_off[q + 1]) ++q;
       const RowAux* ra = remote(aux, q);
-      aux->u.f.gval[i] = ra->u.f.cval[i - base];
-      aux->u.f.gid[i] = ra->u.f.cid[i - base];
+      aux->u.f.gval[i] = ra->u.f.cval[i - aux->cnt_off[q]];
+      aux->u.f.gid[i] = ra->u.f.cid[i - aux->cnt_off[q]];
     }
     __syncthreads();
     // k-th largest key among the candidates (every entry >= t0 is one, so this is the
@@ -685,8 +675,6 @@ struct RowCtx {
     thr = prefix;
     cut = INT_MAX;
     if (need < cnt_eq) {  // keep the `need` lowest ids among the entries equal to the k-th
-      if (threadIdx.x == 0) aux->sel_id = INT_MAX;
-      __syncthreads();
       for (int i = threadIdx.x; i < total; i += kThreads) {
         if (Elem<T>::key(aux->u.f.gval[i]) != prefix) continue;
         const int ii = aux->u.f.gid[i];
@@ -702,45 +690,60 @@ struct RowCtx {
     // on the order the candidates arrived in
     unsigned long long z = 0;
     long long s1 = 0;
+    const bool list = ids_out != nullptr && cl.block_rank() == 0;
+    if (threadIdx.x == 0) aux->ccount = 0;
+    __syncthreads();
     for (int i = threadIdx.x; i < total; i += kThreads) {
       const float xi = aux->u.f.gval[i];
       if (!kept(Elem<T>::key(xi), aux->u.f.gid[i], thr, cut)) continue;
       const float zx = wexp(xi, c, mc);
       const float e = ex2(zx);
       z += to_fx(e);
-      if (want_ent) s1 += __float2ll_rn(e * zx * kS1Fx);
+      if (want_ent) s1 += __float2ll_rn(ent_term(e, zx) * kS1Fx);
+      if (list) ids_out[atomicAdd(&aux->ccount, 1)] = aux->u.f.gid[i];
     }
     zfx = block_sum_u64(z, aux->scr_u64);
     S1 = double(block_sum_s64(s1)) / double(kS1Fx);
+    if (list && threadIdx.x == 0) *n_out = k;
     return true;
   }
 };
 
-template <typename T>
-__global__ void __launch_bounds__(kThreads) row_stats_kernel(const RowJob job) {
-  extern __shared__ __align__(128) unsigned char slice_buf[];
-  __shared__ RowAux aux;
-  RowCtx<T> ctx{slice_buf, 0, 0, 0, 0, &aux, cg::this_cluster(), 0, 0};
-  ctx.C = int(ctx.cl.num_blocks());
-  const int rank = int(ctx.cl.block_rank());
-  const long long row = blockIdx.x / ctx.C;
-  const int V = job.V;
-  const T* src = (row < job.rows0)
-                     ? static_cast<const T*>(job.base0) + size_t(row) * V
-                     : static_cast<const T*>(job.base1) + size_t(row - job.rows0) * V;
-  ctx.s0 = rank * job.slice;
-  ctx.n = max(0, min(V - ctx.s0, job.slice));
-  bool copied = true;
-  if (ctx.n > 0) {
-    copied = stage_slice<T>(src + ctx.s0, ctx.n, slice_buf, &aux.bar, &ctx.pad);
-    ctx.nvec = (ctx.pad + ctx.n * Elem<T>::kBytes + 15) >> 4;
+// j-th largest (1 <= j <= 32) of the keys the 32 lanes pass in (ballot radix select).
+template <int KB>
+__device__ __forceinline__ uint32_t warp_kth_key(uint32_t key, int j) {
+  uint32_t prefix = 0;
+  int need = j;
+#pragma unroll
+  for (int b = KB - 1; b >= 0; --b) {
+    const uint32_t cand = prefix | (1u << b);
+    const int cnt = __popc(__ballot_sync(0xffffffffu, (key >> b) == (cand >> b)));
+    if (cnt >= need)
+      prefix = cand;
+    else
+      need -= cnt;
   }
+  return prefix;
+}
 
+template <typename T>
+__device__ __forceinline__ float key_value(uint32_t k) {
+  if (Elem<T>::kKeyBits == 16)
+    return __uint_as_float(((k & 0x8000u) ? (k & 0x7FFFu) : (~k & 0xFFFFu)) << 16);
+  return __uint_as_float((k & 0x80000000u) ? (k & 0x7FFFFFFFu) : ~k);
+}
+
+// One row: every CTA of the cluster holds its slice in ctx.buf.
+template <typename T>
+__device__ void process_row(RowCtx<T>& ctx, const RowJob& job, long long row, bool copied) {
+  const int V = job.V;
+  const int rank = int(ctx.cl.block_rank());
   const bool greedy = (job.flags & RS_GREEDY) != 0;
   const bool want_ent = (job.flags & RS_ENTROPY) != 0;
   const bool topk = !greedy && job.top_k >= 1 && job.top_k < V;
   const bool topp = !greedy && job.top_p < 1.0f;
-  const bool fast_topk = topk && !topp && job.top_k <= kThreads;
+  const int jw = (job.top_k + kWarps - 1) / kWarps;  // per-warp order statistic for t0
+  const bool fast_topk = topk && !topp && jw <= 32;
 
   // ---- maximum (with its lowest index in greedy mode) and validity
   int vbest = -1;
@@ -748,16 +751,11 @@ __global__ void __launch_bounds__(kThreads) row_stats_kernel(const RowJob job) {
   int bad = copied ? ((mt != mt || mt == INFINITY) ? 1 : 0) : 2;
   float m = (mt != mt) ? -INFINITY : mt;
   int am = greedy ? ctx.first_equal(vbest, m) : INT_MAX;
-  // top-k: this CTA's k-th largest per-thread maximum; the largest over the cluster is
-  // a value that at least k entries reach
+  // top-k: each warp's jw-th largest per-thread maximum; a CTA's smallest warp value is
+  // reached by >= 8 * jw >= k of its entries, so the cluster's largest such value is t0
   float t0 = -INFINITY;
-  if (fast_topk) {
-    const uint32_t kk = ctx.block_kth_key(Elem<T>::key(m), job.top_k);
-    t0 = (Elem<T>::kKeyBits == 16)
-             ? __uint_as_float(((kk & 0x8000u) ? (kk & 0x7FFFu) : (~kk & 0xFFFFu)) << 16)
-             : __uint_as_float((kk & 0x80000000u) ? (kk & 0x7FFFFFFFu) : ~kk);
-  }
-  ctx.xchg_maxloc(m, am, bad, t0);
+  if (fast_topk) t0 = key_value<T>(warp_kth_key<Elem<T>::kKeyBits>(Elem<T>::key(m), jw));
+  ctx.xchg_row(m, am, bad, t0);
   const int status = (bad & 2) ? ROW_TIMEOUT : ((bad & 1) || m == -INFINITY) ? ROW_INVALID : ROW_OK;
   if ((bad & 2) && job.dev_status && threadIdx.x == 0) atomicOr(job.dev_status, 1);
 
@@ -768,10 +766,9 @@ __global__ void __launch_bounds__(kThreads) row_stats_kernel(const RowJob job) {
   unsigned long long zfx = 0;
   double S1 = 0.0;  // sum over the kept set of weight * (l - m) * c  (log2 units)
   bool have_s1 = false;
+  bool listed = false;
 
-  if (status == ROW_OK && greedy) {
-    // the lowest index holding the maximum came with the exchange
-  } else if (status == ROW_OK) {
+  if (status == ROW_OK && !greedy) {
     if (!topk && !topp) {
       // ---- no truncation: one exp pass for the normaliser (and the entropy term)
       float s_a = 0.0f, s_b = 0.0f, h = 0.0f;
@@ -780,12 +777,12 @@ __global__ void __launch_bounds__(kThreads) row_stats_kernel(const RowJob job) {
           const float zx = wexp(x, c, mc);
           const float e = ex2(zx);
           s_a += e;
-          h = fmaf(e, zx, h);
+          h += ent_term(e, zx);
         });
       } else {
         constexpr int P = Elem<T>::kPerVec;
         for (int v = threadIdx.x; v < ctx.nvec; v += kThreads) {
-          const uint4 w = reinterpret_cast<const uint4*>(slice_buf)[v];
+          const uint4 w = reinterpret_cast<const uint4*>(ctx.buf)[v];
           float x[P];
           Elem<T>::unpack(w, x);
           const int j0 = ctx.first_elem(v);
@@ -812,7 +809,14 @@ __global__ void __launch_bounds__(kThreads) row_stats_kernel(const RowJob job) {
       have_s1 = true;
     } else {
       bool done = false;
-      if (fast_topk) done = ctx.filter_topk(job.top_k, t0, c, mc, want_ent, thr, cut, zfx, S1);
+      if (fast_topk) {
+        int32_t* ids = (job.kept_ids && job.top_k <= kKeptCap)
+                           ? job.kept_ids + size_t(row) * kKeptCap
+                           : nullptr;
+        done = ctx.filter_topk(job.top_k, t0, c, mc, want_ent, thr, cut, zfx, S1, ids,
+                               job.kept_n ? job.kept_n + row : nullptr);
+        listed = done && ids != nullptr;
+      }
       if (done) {
         have_s1 = true;
       } else {
@@ -826,12 +830,13 @@ __global__ void __launch_bounds__(kThreads) row_stats_kernel(const RowJob job) {
       ctx.each([&](int id, float x) {
         if (kept(Elem<T>::key(x), id, thr, cut)) {
           const float zx = wexp(x, c, mc);
-          h = fmaf(ex2(zx), zx, h);
+          h += ent_term(ex2(zx), zx);
         }
       });
       S1 = ctx.xchg_sum_f64(double(h));
     }
   }
+  if (!listed && job.kept_n && rank == 0 && threadIdx.x == 0) job.kept_n[row] = 0;
 
   const double Z = double(zfx) * kFxInv;
   const double ent = (status == ROW_OK && !greedy && want_ent)
@@ -845,7 +850,7 @@ __global__ void __launch_bounds__(kThreads) row_stats_kernel(const RowJob job) {
     st.entropy = float(ent);
     st.thr_key = thr;
     st.cutoff = cut;
-    st.argmax = am;
+    st.argmax = greedy ? am : -1;
     st.status = status;
     st.c = c;
     job.stats[row] = st;
@@ -863,6 +868,88 @@ __global__ void __launch_bounds__(kThreads) row_stats_kernel(const RowJob job) {
     }
     if (job.entropy && rank == 0 && threadIdx.x == 0)
       job.entropy[row] = status != ROW_OK ? NAN : (greedy ? 0.0f : float(ent));
+  }
+}
+
+template <typename T>
+__global__ void __launch_bounds__(kThreads) row_stats_kernel(const RowJob job) {
+  extern __shared__ __align__(128) unsigned char ring[];
+  __shared__ RowAux aux;
+  RowCtx<T> ctx{ring, 0, 0, 0, 0, &aux, cg::this_cluster(), 0, 0};
+  ctx.C = int(ctx.cl.num_blocks());
+  const int rank = int(ctx.cl.block_rank());
+  const long long cid = blockIdx.x / ctx.C;
+  const long long G = gridDim.x / ctx.C;
+  if (threadIdx.x == 0) {
+    for (int b = 0; b < kNBuf; ++b) mbar_init(&aux.bar[b], 1);
+    aux.broken = 0;
+    aux.pending = 0;
+  }
+  __syncthreads();
+  auto buffer = [&](long long it) { return ring + size_t(it % kNBuf) * job.slice_bytes; };
+  // rows: all of them, or the listed ones (rows another kernel could not settle)
+  const long long nrows = job.row_list ? (long long)*job.row_count : job.rows;
+  auto row_of = [&](long long li) { return job.row_list ? (long long)job.row_list[li] : li; };
+  // prologue: the first kNBuf - 1 rows of this cluster
+  if (threadIdx.x == 0) {
+    for (int it = 0; it < kNBuf - 1; ++it) {
+      const long long li = cid + it * G;
+      if (li >= nrows) break;
+      const SliceLoc s = slice_loc<T>(job, row_of(li), rank);
+      if (s.n > 0) {
+        issue_slice(s, buffer(it), &aux.bar[it % kNBuf]);
+        aux.pending |= 1 << (it % kNBuf);
+      }
+    }
+  }
+  for (long long it = 0;; ++it) {
+    const long long li = cid + it * G;
+    if (li >= nrows) break;
+    const long long row = row_of(li);
+    // keep kNBuf - 1 rows in flight: the buffer refilled here was last read by
+    // iteration it - 1, which every thread of this CTA has finished
+    if (threadIdx.x == 0 && !aux.broken) {
+      const long long ahead = it + kNBuf - 1;
+      const long long ali = cid + ahead * G;
+      if (ali < nrows) {
+        const SliceLoc s = slice_loc<T>(job, row_of(ali), rank);
+        if (s.n > 0) {
+          issue_slice(s, buffer(ahead), &aux.bar[ahead % kNBuf]);
+          aux.pending |= 1 << (ahead % kNBuf);
+        }
+      }
+    }
+    __syncthreads();
+    const SliceLoc s = slice_loc<T>(job, row, rank);
+    const int b = int(it % kNBuf);
+    bool copied = true;
+    if (s.n > 0) {
+      if (!aux.broken && (aux.pending & (1 << b))) {
+        copied = finish_slice<T>(s, buffer(it), &aux.bar[b], uint32_t((it / kNBuf) & 1));
+        if (threadIdx.x == 0) {
+          if (copied)
+            aux.pending &= ~(1 << b);
+          else
+            aux.broken = 1;
+        }
+      } else {
+        copied = false;  // an earlier copy timed out: this row is reported, not read
+      }
+    }
+    ctx.buf = buffer(it);
+    ctx.s0 = rank * job.slice;
+    ctx.n = s.n;
+    ctx.pad = s.pad;
+    ctx.nvec = s.n > 0 ? (s.pad + s.n * Elem<T>::kBytes + 15) >> 4 : 0;
+    process_row<T>(ctx, job, row, copied);
+    __syncthreads();
+  }
+  // a copy that timed out may still land: give each one more bounded wait
+  if (aux.broken && threadIdx.x == 0) {
+    for (int b = 0; b < kNBuf; ++b)
+      if (aux.pending & (1 << b)) {
+        if (!mbar_wait(&aux.bar[b], 0)) mbar_wait(&aux.bar[b], 1);
+      }
   }
   ctx.cl.sync();  // no CTA leaves while a peer may still read its shared memory
 }

@@ -3,20 +3,28 @@
 #include <atomic>
 #include <cmath>
 #include <cstring>
+#include <map>
+#include <mutex>
+#include <tuple>
 
 #include "chain.cuh"
 #include "probs.cuh"
 #include "row_stats.cuh"
 #include "specverify.h"
+#include "stream.cuh"
 #include "tree.cuh"
 
 namespace {
 
 using sv::kThreads;
 
-// Slice of a logit row per CTA: small enough that two or three CTAs share an SM and
-// one CTA's computation overlaps another's copies.
-constexpr size_t kSliceTargetBytes = 64 * 1024;
+// Slice of a logit row per CTA: each CTA keeps sv::kNBuf slices in flight, and two
+// CTAs share an SM, so one CTA's computation overlaps the other's copies and its own
+// next rows' copies.
+#ifndef SV_SLICE_KB
+#define SV_SLICE_KB 40
+#endif
+constexpr size_t kSliceTargetBytes = SV_SLICE_KB * 1024;
 constexpr size_t kMaxDynSmem = 227 * 1024 - sizeof(sv::RowAux) - 1024;
 constexpr size_t kStatsOffset = 256;  // the device status word lives at offset 0
 
@@ -24,33 +32,80 @@ std::atomic<void*> g_ev_before{nullptr};
 std::atomic<void*> g_ev_after{nullptr};
 
 struct RowPlan {
-  int C;        // CTAs per cluster (one cluster per row)
-  int slice;    // elements per CTA
-  size_t dyn;   // dynamic shared memory per CTA
+  int C;             // CTAs per cluster (one cluster per row at a time)
+  int slice;         // elements per CTA
+  int slice_bytes;   // bytes per slice buffer
+  size_t dyn;        // dynamic shared memory per CTA (the ring of slice buffers)
 };
 
 bool plan_rows(int V, int elem_bytes, RowPlan* pl) {
   int C = 1;
-  while (C < 16 && size_t((V + C - 1) / C) * elem_bytes > kSliceTargetBytes) C *= 2;
+  while (C < sv::kMaxCluster && size_t((V + C - 1) / C) * elem_bytes > kSliceTargetBytes) C *= 2;
   const int slice = ((V + C - 1) / C + 15) / 16 * 16;
-  const size_t dyn = (size_t(slice) * elem_bytes + 16 + 127) / 128 * 128;
+  const int slice_bytes = int((size_t(slice) * elem_bytes + 16 + 127) / 128 * 128);
+  const size_t dyn = size_t(slice_bytes) * sv::kNBuf;
   if (dyn > kMaxDynSmem) return false;
-  *pl = RowPlan{C, slice, dyn};
+  *pl = RowPlan{C, slice, slice_bytes, dyn};
   return true;
+}
+
+// Lets the row kernel take any ring size this build plans (per function and device; the
+// largest value, so a later, smaller launch can never lower it below a cached shape).
+template <typename T>
+cudaError_t allow_row_kernel_smem() {
+  auto k = sv::row_stats_kernel<T>;
+  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       int(kMaxDynSmem));
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(k, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+  return e;
+}
+
+// Clusters of the row kernel that fit on the device at once (cached per device and shape).
+template <typename T>
+int resident_clusters(const RowPlan& pl, cudaError_t* err) {
+  static std::mutex mu;
+  static std::map<std::tuple<int, int, size_t>, int> cache;
+  int dev = 0;
+  *err = cudaGetDevice(&dev);
+  if (*err != cudaSuccess) return 0;
+  const auto key = std::make_tuple(dev, pl.C, pl.dyn);
+  {
+    std::lock_guard<std::mutex> lock(mu);
+    auto it = cache.find(key);
+    if (it != cache.end()) return it->second;
+  }
+  auto k = sv::row_stats_kernel<T>;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(unsigned(pl.C), 1, 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = pl.dyn;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = unsigned(pl.C);
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int n = 0;
+  *err = cudaOccupancyMaxActiveClusters(&n, k, &cfg);
+  if (*err != cudaSuccess) return 0;
+  std::lock_guard<std::mutex> lock(mu);
+  cache[key] = n;
+  return n;
 }
 
 template <typename T>
 cudaError_t launch_row_stats(const sv::RowJob& job, const RowPlan& pl, cudaStream_t s) {
   auto k = sv::row_stats_kernel<T>;
-  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       int(pl.dyn));
+  cudaError_t e = allow_row_kernel_smem<T>();
   if (e != cudaSuccess) return e;
-  if (pl.C > 8) {
-    e = cudaFuncSetAttribute(k, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
-    if (e != cudaSuccess) return e;
-  }
+  const int clusters = resident_clusters<T>(pl, &e);
+  if (e != cudaSuccess) return e;
+  if (clusters < 1) return cudaErrorInvalidConfiguration;
+  const long long G = job.rows < clusters ? job.rows : clusters;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(unsigned(job.rows * pl.C), 1, 1);
+  cfg.gridDim = dim3(unsigned(G * pl.C), 1, 1);
   cfg.blockDim = dim3(kThreads, 1, 1);
   cfg.dynamicSmemBytes = pl.dyn;
   cfg.stream = s;
@@ -70,16 +125,99 @@ cudaError_t launch_row_stats_dt(spec_dtype dt, const sv::RowJob& job, const RowP
                          : launch_row_stats<float>(job, pl, s);
 }
 
+// ------------------------------------------------------------------ streaming kernel
+constexpr size_t kStreamBufBytes = (sv::kChunkBytes + 16 + 127) / 128 * 128;
+constexpr size_t kStreamDyn = kStreamBufBytes * sv::kSBuf;
+
+// Resident CTAs of the streaming kernel (cached per device): it is persistent.
+template <typename T>
+int stream_grid(cudaError_t* err) {
+  static std::mutex mu;
+  static std::map<int, int> cache;
+  int dev = 0;
+  *err = cudaGetDevice(&dev);
+  if (*err != cudaSuccess) return 0;
+  {
+    std::lock_guard<std::mutex> lock(mu);
+    auto it = cache.find(dev);
+    if (it != cache.end()) return it->second;
+  }
+  auto k = sv::stream_rows_kernel<T>;
+  *err = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, int(kStreamDyn));
+  if (*err != cudaSuccess) return 0;
+  int per_sm = 0, sms = 0;
+  *err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k, kThreads, kStreamDyn);
+  if (*err == cudaSuccess) *err = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (*err != cudaSuccess) return 0;
+  std::lock_guard<std::mutex> lock(mu);
+  cache[dev] = per_sm * sms;
+  return per_sm * sms;
+}
+
+template <typename T>
+cudaError_t launch_stream(const sv::StreamJob& job, cudaStream_t s) {
+  cudaError_t e = cudaSuccess;
+  const int grid = stream_grid<T>(&e);
+  if (e != cudaSuccess) return e;
+  if (grid < 1) return cudaErrorInvalidConfiguration;
+  auto k = sv::stream_rows_kernel<T>;
+  e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, int(kStreamDyn));
+  if (e != cudaSuccess) return e;
+  const long long g = job.r.rows < grid ? job.r.rows : grid;
+  k<<<unsigned(g), kThreads, kStreamDyn, s>>>(job);
+  return cudaGetLastError();
+}
+
+// Row statistics for a verify call: the streaming kernel settles the rows it can and
+// lists the rest, which the cluster kernel then finishes exactly.
+cudaError_t row_stage(spec_dtype dt, const sv::RowJob& rj, const RowPlan& pl, int32_t* fb_rows,
+                      int32_t* fb_count, cudaStream_t s) {
+  const int E = dt == SPEC_BF16 ? 2 : 4;
+  sv::StreamJob sj = {};
+  sj.r = rj;
+  sj.chunk = sv::kChunkBytes / E;
+  sj.nchunk = (rj.V + sj.chunk - 1) / sj.chunk;
+  sj.chunk_bytes = int(kStreamBufBytes);
+  const bool topk = !(rj.flags & sv::RS_GREEDY) && rj.top_k >= 1 && rj.top_k < rj.V;
+  const bool topp = !(rj.flags & sv::RS_GREEDY) && rj.top_p < 1.0f;
+  sj.topp_span = topp ? float(std::log(double(rj.V) / (1.0 - double(rj.top_p))) / rj.inv_t) : 0.0f;
+  sj.fb_rows = fb_rows;
+  sj.fb_count = fb_count;
+  cudaError_t e = dt == SPEC_BF16 ? launch_stream<__nv_bfloat16>(sj, s) : launch_stream<float>(sj, s);
+  if (e != cudaSuccess || !(topk || topp)) return e;
+  sv::RowJob fj = rj;
+  fj.row_list = fb_rows;
+  fj.row_count = fb_count;
+  return launch_row_stats_dt(dt, fj, pl, s);
+}
+
 int elem_bytes(spec_dtype dt) { return dt == SPEC_BF16 ? 2 : 4; }
 
 bool dtype_ok(int dt) { return dt == SPEC_F32 || dt == SPEC_BF16; }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-size_t stats_bytes(long long rows) { return kStatsOffset + size_t(rows) * sizeof(sv::RowStats); }
+// Workspace: [header: status word, fallback count | RowStats per row | kept-id count per
+// row | kept ids per row | fallback row list].
+struct WsLayout {
+  size_t stats, kept_n, kept_ids, fb_rows, total;
+};
 
-// Grid limit: rows * C must fit a 1-D grid.
-bool rows_fit(long long rows, int C) { return rows * C <= 0x7fffffffLL; }
+size_t up256(size_t x) { return (x + 255) / 256 * 256; }
+
+WsLayout ws_layout(long long rows) {
+  WsLayout w;
+  w.stats = kStatsOffset;
+  w.kept_n = w.stats + up256(size_t(rows) * sizeof(sv::RowStats));
+  w.kept_ids = w.kept_n + up256(size_t(rows) * sizeof(int32_t));
+  w.fb_rows = w.kept_ids + up256(size_t(rows) * sv::kKeptCap * sizeof(int32_t));
+  w.total = w.fb_rows + up256(size_t(rows) * sizeof(int32_t));
+  return w;
+}
+
+size_t stats_bytes(long long rows) { return ws_layout(rows).total; }
+
+bool rows_fit(long long rows, int) { return rows <= 0x7fffffffLL; }
 
 spec_status check_launch(cudaError_t e) { return e == cudaSuccess ? SPEC_OK : SPEC_ERR_CUDA; }
 
@@ -124,17 +262,21 @@ spec_status spec_verify_chain(const void* target_logits, const void* draft_logit
     return SPEC_ERR_UNSUPPORTED;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   int32_t* dev_status = static_cast<int32_t*>(workspace);
-  sv::RowStats* stats =
-      reinterpret_cast<sv::RowStats*>(static_cast<char*>(workspace) + kStatsOffset);
-  if (cudaMemsetAsync(dev_status, 0, sizeof(int32_t), s) != cudaSuccess) return SPEC_ERR_CUDA;
+  const WsLayout wl = ws_layout(rows);
+  char* ws = static_cast<char*>(workspace);
+  sv::RowStats* stats = reinterpret_cast<sv::RowStats*>(ws + wl.stats);
+  if (cudaMemsetAsync(dev_status, 0, 2 * sizeof(int32_t), s) != cudaSuccess) return SPEC_ERR_CUDA;
 
   sv::RowJob rj = {};
+  rj.kept_n = reinterpret_cast<int32_t*>(ws + wl.kept_n);
+  rj.kept_ids = reinterpret_cast<int32_t*>(ws + wl.kept_ids);
   rj.base0 = target_logits;
   rj.base1 = draft_logits;
   rj.rows0 = (long long)B * (K + 1);
   rj.rows = rows;
   rj.V = V;
   rj.slice = pl.slice;
+  rj.slice_bytes = pl.slice_bytes;
   rj.c = greedy ? 0.0f : sv::kLog2e / temp;
   rj.inv_t = greedy ? 0.0f : 1.0f / temp;
   rj.top_k = (top_k >= 1 && top_k < V) ? top_k : 0;
@@ -145,7 +287,9 @@ spec_status spec_verify_chain(const void* target_logits, const void* draft_logit
   void* evb = g_ev_before.load();
   void* eva = g_ev_after.load();
   if (evb) cudaEventRecord(static_cast<cudaEvent_t>(evb), s);
-  if (launch_row_stats_dt(dtype, rj, pl, s) != cudaSuccess) return SPEC_ERR_CUDA;
+  if (row_stage(dtype, rj, pl, reinterpret_cast<int32_t*>(ws + wl.fb_rows), dev_status + 1, s) !=
+      cudaSuccess)
+    return SPEC_ERR_CUDA;
   if (eva) cudaEventRecord(static_cast<cudaEvent_t>(eva), s);
 
   sv::ChainJob cj = {};
@@ -184,9 +328,10 @@ spec_status spec_verify_tree_typical(const void* target_logits, spec_dtype dtype
   if (!plan_rows(V, elem_bytes(dtype), &pl) || !rows_fit(rows, pl.C)) return SPEC_ERR_UNSUPPORTED;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   int32_t* dev_status = static_cast<int32_t*>(workspace);
-  sv::RowStats* stats =
-      reinterpret_cast<sv::RowStats*>(static_cast<char*>(workspace) + kStatsOffset);
-  if (cudaMemsetAsync(dev_status, 0, sizeof(int32_t), s) != cudaSuccess) return SPEC_ERR_CUDA;
+  const WsLayout wl = ws_layout(rows);
+  char* ws = static_cast<char*>(workspace);
+  sv::RowStats* stats = reinterpret_cast<sv::RowStats*>(ws + wl.stats);
+  if (cudaMemsetAsync(dev_status, 0, 2 * sizeof(int32_t), s) != cudaSuccess) return SPEC_ERR_CUDA;
 
   sv::RowJob rj = {};
   rj.base0 = target_logits;
@@ -195,6 +340,7 @@ spec_status spec_verify_tree_typical(const void* target_logits, spec_dtype dtype
   rj.rows = rows;
   rj.V = V;
   rj.slice = pl.slice;
+  rj.slice_bytes = pl.slice_bytes;
   rj.c = sv::kLog2e;
   rj.inv_t = 1.0f;
   rj.top_k = 0;
@@ -205,7 +351,9 @@ spec_status spec_verify_tree_typical(const void* target_logits, spec_dtype dtype
   void* evb = g_ev_before.load();
   void* eva = g_ev_after.load();
   if (evb) cudaEventRecord(static_cast<cudaEvent_t>(evb), s);
-  if (launch_row_stats_dt(dtype, rj, pl, s) != cudaSuccess) return SPEC_ERR_CUDA;
+  if (row_stage(dtype, rj, pl, reinterpret_cast<int32_t*>(ws + wl.fb_rows), dev_status + 1, s) !=
+      cudaSuccess)
+    return SPEC_ERR_CUDA;
   if (eva) cudaEventRecord(static_cast<cudaEvent_t>(eva), s);
 
   sv::TreeJob tj = {};
@@ -246,6 +394,7 @@ spec_status spec_logits_to_probs(const void* logits, spec_dtype dtype, int rows,
   rj.rows = rows;
   rj.V = V;
   rj.slice = pl.slice;
+  rj.slice_bytes = pl.slice_bytes;
   rj.c = greedy ? 0.0f : sv::kLog2e / temp;
   rj.inv_t = greedy ? 0.0f : 1.0f / temp;
   rj.top_k = (top_k >= 1 && top_k < V) ? top_k : 0;

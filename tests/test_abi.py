@@ -29,10 +29,17 @@ def test_status_strings_and_kernel_counts(lib):
     assert sv.spec_kernels_per_call("nope") == -1
 
 
+def _ws(rows):
+    up = lambda x: (x + 255) // 256 * 256
+    return 256 + up(32 * rows) + up(4 * rows) + up(rows * 256 * 4) + up(4 * rows)
+
+
 def test_workspace_size(lib):
+    """header, 32-byte row statistics, kept-id counts, up to 256 kept ids per row and the
+    list of rows the cluster kernel finishes"""
     assert sv.spec_workspace_size(0, 4, 10) == 0
-    assert sv.spec_workspace_size(512, 8, 151936) == 256 + 32 * 512 * 17
-    assert sv.spec_workspace_size(32, 64, 32000) == 256 + 32 * 32 * 129
+    assert sv.spec_workspace_size(512, 8, 151936) == _ws(512 * 17)
+    assert sv.spec_workspace_size(32, 64, 32000) == _ws(32 * 129)
 
 
 P = ctypes.c_void_p
