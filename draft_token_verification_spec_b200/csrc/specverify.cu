@@ -126,65 +126,88 @@ cudaError_t launch_row_stats_dt(spec_dtype dt, const sv::RowJob& job, const RowP
 }
 
 // ------------------------------------------------------------------ streaming kernel
-constexpr size_t kStreamBufBytes = (sv::kChunkBytes + 16 + 127) / 128 * 128;
-constexpr size_t kStreamDyn = kStreamBufBytes * sv::kSBuf;
+int stream_mode(const sv::RowJob& rj) {
+  if (rj.flags & sv::RS_GREEDY) return sv::SM_GREEDY;
+  if (rj.top_k >= 1 && rj.top_k < rj.V) return sv::SM_TOPK;
+  if (rj.top_p < 1.0f) return sv::SM_TOPP;
+  return sv::SM_SUMS;
+}
 
-// Resident CTAs of the streaming kernel (cached per device): it is persistent.
-template <typename T>
-int stream_grid(cudaError_t* err) {
-  static std::mutex mu;
-  static std::map<int, int> cache;
-  int dev = 0;
-  *err = cudaGetDevice(&dev);
-  if (*err != cudaSuccess) return 0;
-  {
+template <typename T, int M>
+struct StreamKernel {
+  // Resident CTAs (cached per device): the kernel is persistent.
+  static int grid(cudaError_t* err) {
+    static std::mutex mu;
+    static std::map<int, int> cache;
+    int dev = 0;
+    *err = cudaGetDevice(&dev);
+    if (*err != cudaSuccess) return 0;
+    {
+      std::lock_guard<std::mutex> lock(mu);
+      auto it = cache.find(dev);
+      if (it != cache.end()) return it->second;
+    }
+    auto k = sv::stream_rows_kernel<T, M>;
+    const size_t dyn = sv::stream_dyn_bytes(M);
+    *err = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, int(dyn));
+    if (*err != cudaSuccess) return 0;
+    int per_sm = 0, sms = 0;
+    *err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k, sv::kStreamThreads, dyn);
+    if (*err == cudaSuccess)
+      *err = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (*err != cudaSuccess) return 0;
     std::lock_guard<std::mutex> lock(mu);
-    auto it = cache.find(dev);
-    if (it != cache.end()) return it->second;
+    cache[dev] = per_sm * sms;
+    return per_sm * sms;
   }
-  auto k = sv::stream_rows_kernel<T>;
-  *err = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, int(kStreamDyn));
-  if (*err != cudaSuccess) return 0;
-  int per_sm = 0, sms = 0;
-  *err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k, kThreads, kStreamDyn);
-  if (*err == cudaSuccess) *err = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  if (*err != cudaSuccess) return 0;
-  std::lock_guard<std::mutex> lock(mu);
-  cache[dev] = per_sm * sms;
-  return per_sm * sms;
-}
+
+  static cudaError_t launch(const sv::StreamJob& job, cudaStream_t s) {
+    cudaError_t e = cudaSuccess;
+    const int g = grid(&e);
+    if (e != cudaSuccess) return e;
+    if (g < 1) return cudaErrorInvalidConfiguration;
+    auto k = sv::stream_rows_kernel<T, M>;
+    const size_t dyn = sv::stream_dyn_bytes(M);
+    // set on every launch: the attribute is per device, the cache is not
+    e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, int(dyn));
+    if (e != cudaSuccess) return e;
+    const long long n = job.r.rows < g ? job.r.rows : g;
+    k<<<unsigned(n), sv::kStreamThreads, dyn, s>>>(job);
+    return cudaGetLastError();
+  }
+};
 
 template <typename T>
-cudaError_t launch_stream(const sv::StreamJob& job, cudaStream_t s) {
-  cudaError_t e = cudaSuccess;
-  const int grid = stream_grid<T>(&e);
-  if (e != cudaSuccess) return e;
-  if (grid < 1) return cudaErrorInvalidConfiguration;
-  auto k = sv::stream_rows_kernel<T>;
-  e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, int(kStreamDyn));
-  if (e != cudaSuccess) return e;
-  const long long g = job.r.rows < grid ? job.r.rows : grid;
-  k<<<unsigned(g), kThreads, kStreamDyn, s>>>(job);
-  return cudaGetLastError();
+cudaError_t launch_stream(const sv::StreamJob& job, int mode, cudaStream_t s) {
+  switch (mode) {
+    case sv::SM_GREEDY: return StreamKernel<T, sv::SM_GREEDY>::launch(job, s);
+    case sv::SM_SUMS: return StreamKernel<T, sv::SM_SUMS>::launch(job, s);
+    case sv::SM_TOPK: return StreamKernel<T, sv::SM_TOPK>::launch(job, s);
+    default: return StreamKernel<T, sv::SM_TOPP>::launch(job, s);
+  }
 }
 
-// Row statistics for a verify call: the streaming kernel settles the rows it can and
-// lists the rest, which the cluster kernel then finishes exactly.
+// Row statistics for a verify call. The streaming kernel settles the rows it can; in the
+// candidate modes it lists the rest, which the cluster kernel then finishes exactly. A
+// top-k above the candidate path's limit goes to the cluster kernel for every row.
 cudaError_t row_stage(spec_dtype dt, const sv::RowJob& rj, const RowPlan& pl, int32_t* fb_rows,
                       int32_t* fb_count, cudaStream_t s) {
+  const int mode = stream_mode(rj);
+  if (mode == sv::SM_TOPK && rj.top_k > sv::kStreamMaxTopK)
+    return launch_row_stats_dt(dt, rj, pl, s);
   const int E = dt == SPEC_BF16 ? 2 : 4;
   sv::StreamJob sj = {};
   sj.r = rj;
   sj.chunk = sv::kChunkBytes / E;
   sj.nchunk = (rj.V + sj.chunk - 1) / sj.chunk;
-  sj.chunk_bytes = int(kStreamBufBytes);
-  const bool topk = !(rj.flags & sv::RS_GREEDY) && rj.top_k >= 1 && rj.top_k < rj.V;
-  const bool topp = !(rj.flags & sv::RS_GREEDY) && rj.top_p < 1.0f;
-  sj.topp_span = topp ? float(std::log(double(rj.V) / (1.0 - double(rj.top_p))) / rj.inv_t) : 0.0f;
+  sj.topp_span = rj.top_p < 1.0f
+                     ? float(std::log(double(rj.V) / (1.0 - double(rj.top_p))) / rj.inv_t)
+                     : 0.0f;
   sj.fb_rows = fb_rows;
   sj.fb_count = fb_count;
-  cudaError_t e = dt == SPEC_BF16 ? launch_stream<__nv_bfloat16>(sj, s) : launch_stream<float>(sj, s);
-  if (e != cudaSuccess || !(topk || topp)) return e;
+  cudaError_t e = dt == SPEC_BF16 ? launch_stream<__nv_bfloat16>(sj, mode, s)
+                                  : launch_stream<float>(sj, mode, s);
+  if (e != cudaSuccess || (mode != sv::SM_TOPK && mode != sv::SM_TOPP)) return e;
   sv::RowJob fj = rj;
   fj.row_list = fb_rows;
   fj.row_count = fb_count;
@@ -435,7 +458,7 @@ void spec_set_row_kernel_events(void* before, void* after) {
 
 int spec_kernels_per_call(const char* entry_point) {
   if (!entry_point) return -1;
-  if (!std::strcmp(entry_point, "spec_verify_chain")) return 2;
+  if (!std::strcmp(entry_point, "spec_verify_chain")) return 3;
   if (!std::strcmp(entry_point, "spec_verify_tree_typical")) return 2;
   if (!std::strcmp(entry_point, "spec_logits_to_probs")) return 1;
   if (!std::strcmp(entry_point, "spec_residual_sample")) return 1;

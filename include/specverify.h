@@ -149,7 +149,9 @@ spec_status spec_get_device_status(const void* workspace, int32_t* status_out, v
  * before its row-statistics kernel and `after` just after it. NULL, NULL clears. */
 void spec_set_row_kernel_events(void* before, void* after);
 
-/* Number of kernels each call enqueues (for launch accounting). */
+/* Largest number of kernels one call enqueues (for launch accounting): the row
+ * statistics kernel, the exact finisher for rows it lists (chain calls with top-k or
+ * top-p only) and the per-batch-row kernel. -1 for an unknown name. */
 int spec_kernels_per_call(const char* entry_point);
 
 #ifdef __cplusplus

@@ -25,7 +25,7 @@ def test_every_declared_function_is_exported(lib):
 def test_status_strings_and_kernel_counts(lib):
     assert sv.status_string(0) == "SPEC_OK"
     assert sv.status_string(-4) == "SPEC_ERR_WORKSPACE"
-    assert sv.spec_kernels_per_call("spec_verify_chain") == 2
+    assert sv.spec_kernels_per_call("spec_verify_chain") == 3
     assert sv.spec_kernels_per_call("nope") == -1
 
 
