@@ -5,11 +5,15 @@
 // position that stops the scan: a rejection, the bonus position K, or a data error.
 // The whole block then draws the emitted token: from norm(max(0, p_a - q_a)) after a
 // rejection at a (p_a if that residual is empty), from p_K when all K drafts were
-// accepted. "Speculative Decoding" and "Speculative Sampling" (spec-decoding-i notes);
+// accepted. When the row of p_a lists its kept ids (top-k rows), the draw runs over
+// that support only: the residual and p both vanish outside it. "Speculative Decoding" and "Speculative Sampling" (spec-decoding-i notes);
 // greedy longest-prefix verification from blockwise parallel decoding ("推测解码").
 #pragma once
 
 #include "draw.cuh"
+#include "row_stats.cuh"
+
+static_assert(sv::kSparseCap >= sv::kKeptCap, "a listed kept set fits one sparse draw");
 
 namespace sv {
 
@@ -20,6 +24,8 @@ struct ChainJob {
   const int32_t* tokens;  // [B][K]
   const float* uniforms;  // [B][K+1]
   const RowStats* stats;  // target rows [B*(K+1)], then draft rows [B*K]
+  const int32_t* kept_n;  // [rows] or NULL: ids listed per row (0: none)
+  const int32_t* kept_ids;  // [rows][kKeptCap]
   int greedy;
   int32_t* accepted_len;  // [B]
   int32_t* out_tokens;    // [B][K+1]
@@ -105,37 +111,59 @@ __global__ void __launch_bounds__(kThreads) chain_finish_kernel(const ChainJob j
     const T* prow = trow0 + size_t(a) * V;
     const bool pal = (reinterpret_cast<uintptr_t>(prow) & 15u) == 0;
     const float w = u[K];
+    const size_t prow_idx = size_t(b) * (K + 1) + a;
+    const int nk = j.kept_n ? j.kept_n[prow_idx] : 0;
     tok = -1;
-    if (a < K) {
-      const RowStats sq = ds[a];
-      const T* qrow = drow0 + size_t(a) * V;
-      const bool qal = (reinterpret_cast<uintptr_t>(qrow) & 15u) == 0;
-      tok = inverse_cdf_draw(
-          [&](int v0, unsigned long long* r) {
-            float lp[8], lq[8];
-            load8<T>(prow, v0, V, pal, lp);
-            load8<T>(qrow, v0, V, qal, lq);
+    if (nk > 0 && nk <= kSparseCap) {
+      const int32_t* ids = j.kept_ids + prow_idx * kKeptCap;
+      if (a < K) {
+        const RowStats sq = ds[a];
+        const T* qrow = drow0 + size_t(a) * V;
+        tok = sparse_draw(
+            ids, nk,
+            [&](int v) {
+              const float d = prob<T>(sp, Elem<T>::load(prow, size_t(v)), v) -
+                              prob<T>(sq, Elem<T>::load(qrow, size_t(v)), v);
+              return to_fx(fmaxf(d, 0.0f));
+            },
+            w, sm);
+      }
+      if (tok < 0)
+        tok = sparse_draw(
+            ids, nk, [&](int v) { return to_fx(prob<T>(sp, Elem<T>::load(prow, size_t(v)), v)); },
+            w, sm);
+    } else {
+      if (a < K) {
+        const RowStats sq = ds[a];
+        const T* qrow = drow0 + size_t(a) * V;
+        const bool qal = (reinterpret_cast<uintptr_t>(qrow) & 15u) == 0;
+        tok = inverse_cdf_draw(
+            [&](int v0, unsigned long long* r) {
+              float lp[8], lq[8];
+              load8<T>(prow, v0, V, pal, lp);
+              load8<T>(qrow, v0, V, qal, lq);
 #pragma unroll
-            for (int k = 0; k < 8; ++k) {
-              const int v = v0 + k;
-              const float d = (v < V) ? prob<T>(sp, lp[k], v) - prob<T>(sq, lq[k], v) : 0.0f;
-              r[k] = to_fx(fmaxf(d, 0.0f));
-            }
-          },
-          V, w, sm);
-    }
-    if (tok < 0) {  // bonus position, or an empty residual: draw from p
-      tok = inverse_cdf_draw(
-          [&](int v0, unsigned long long* r) {
-            float lp[8];
-            load8<T>(prow, v0, V, pal, lp);
+              for (int k = 0; k < 8; ++k) {
+                const int v = v0 + k;
+                const float d = (v < V) ? prob<T>(sp, lp[k], v) - prob<T>(sq, lq[k], v) : 0.0f;
+                r[k] = to_fx(fmaxf(d, 0.0f));
+              }
+            },
+            V, w, sm);
+      }
+      if (tok < 0) {  // bonus position, or an empty residual: draw from p
+        tok = inverse_cdf_draw(
+            [&](int v0, unsigned long long* r) {
+              float lp[8];
+              load8<T>(prow, v0, V, pal, lp);
 #pragma unroll
-            for (int k = 0; k < 8; ++k) {
-              const int v = v0 + k;
-              r[k] = (v < V) ? to_fx(prob<T>(sp, lp[k], v)) : 0ull;
-            }
-          },
-          V, w, sm);
+              for (int k = 0; k < 8; ++k) {
+                const int v = v0 + k;
+                r[k] = (v < V) ? to_fx(prob<T>(sp, lp[k], v)) : 0ull;
+              }
+            },
+            V, w, sm);
+      }
     }
   }
   if (threadIdx.x == 0) {

@@ -19,9 +19,11 @@ namespace sv {
 
 constexpr int kDrawChunk = kThreads * 8;
 constexpr int kMaxDrawChunks = (1 << 20) / kDrawChunk;  // V <= 2^20
+constexpr int kSparseCap = kThreads;                    // support of a sparse draw
 
 struct DrawSmem {
   unsigned long long chunk[kMaxDrawChunks];
+  int ids[kSparseCap];
   unsigned long long scr[kWarps];
   unsigned long long total;
   int best;
@@ -105,6 +107,45 @@ __device__ int inverse_cdf_draw(F&& f, int V, float w, DrawSmem& sm) {
   }
   __syncthreads();
   const int tok = sm.best;
+  __syncthreads();
+  return tok;
+}
+
+// The same draw when every entry outside ids[0..n) (distinct ids, any order, n <= kThreads)
+// has mass 0: the support is sorted by id and one block-wide prefix sum replaces the pass
+// over the row. mass(v) gives the fixed-point mass of entry v; the result is identical
+// to inverse_cdf_draw over the whole row with the same masses.
+template <typename F>
+__device__ int sparse_draw(const int32_t* ids, int n, F&& mass, float w, DrawSmem& sm) {
+  const int t = threadIdx.x;
+  const int my = t < n ? ids[t] : INT_MAX;
+  if (t < n) sm.ids[t] = my;
+  if (t == 0) sm.best = INT_MAX;
+  __syncthreads();
+  int rank = 0;
+  if (t < n)
+    for (int j = 0; j < n; ++j) rank += sm.ids[j] < my ? 1 : 0;
+  __syncthreads();
+  if (t < n) sm.ids[rank] = my;
+  __syncthreads();
+  const int v = t < n ? sm.ids[t] : -1;
+  const unsigned long long r = t < n ? mass(v) : 0ull;
+  unsigned long long S;
+  const unsigned long long ex = block_exclusive_scan<unsigned long long>(r, sm.scr, &S);
+  const double target = double(w) * double(S);
+  if (r > 0 && double(ex + r) > target) atomicMin(&sm.best, v);
+  __syncthreads();
+  int tok = sm.best;
+  if (S == 0) {
+    tok = -1;
+  } else if (tok == INT_MAX) {  // rounding left none: the largest id with mass
+    __syncthreads();
+    if (t == 0) sm.best = -1;
+    __syncthreads();
+    if (r > 0) atomicMax(&sm.best, v);
+    __syncthreads();
+    tok = sm.best;
+  }
   __syncthreads();
   return tok;
 }

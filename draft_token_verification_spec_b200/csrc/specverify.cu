@@ -324,6 +324,8 @@ spec_status spec_verify_chain(const void* target_logits, const void* draft_logit
   cj.tokens = draft_tokens;
   cj.uniforms = uniforms;
   cj.stats = stats;
+  cj.kept_n = rj.kept_n;
+  cj.kept_ids = rj.kept_ids;
   cj.greedy = greedy ? 1 : 0;
   cj.accepted_len = accepted_len;
   cj.out_tokens = out_tokens;
