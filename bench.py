@@ -68,6 +68,22 @@ def read_profile_traffic(name: str):
         return None
 
 
+def max_over_ranks(x: float, device, world: int) -> float:
+    """The largest x over all ranks (device-timed durations: the job ends with the slowest)."""
+    if world <= 1:
+        return float(x)
+    import torch
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_value(B: int, K: int, world: int, steps: int, ms_max: float) -> float:
+    """Verified draft positions per second over the whole job: every rank verifies B*K
+    positions per step, and the job takes the slowest rank's time."""
+    return B * K * world * steps / (ms_max / 1e3)
+
+
 class ClockSampler:
     """nvidia-smi SM clock / throttle-reason sampling during the timed region."""
     Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
@@ -186,12 +202,8 @@ def run_ours(args, cfg, greedy, rank, world):
         torch.distributed.barrier()
     ms = start.elapsed_time(end)
     row_ms = [a.elapsed_time(b) for a, b in pairs]
-    t = torch.tensor([ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-    ms_max = float(t.item())
-    positions = cfg.B * cfg.K * world * args.steps
-    value = positions / (ms_max / 1e3)
+    ms_max = max_over_ranks(ms, dev, world)
+    value = job_value(cfg.B, cfg.K, world, args.steps, ms_max)
 
     # end to end through the same call: pinned host inputs in, results out, every step
     e2e_steps = max(3, min(args.steps, 10))
@@ -224,10 +236,8 @@ def run_ours(args, cfg, greedy, rank, world):
         h_out.copy_(out, non_blocking=True)
     e1.record()
     torch.cuda.synchronize()
-    e2e_ms = torch.tensor([e0.elapsed_time(e1) / e2e_steps], dtype=torch.float64, device=dev)
-    if world > 1:
-        torch.distributed.all_reduce(e2e_ms, op=torch.distributed.ReduceOp.MAX)
-    e2e_value = cfg.B * cfg.K * world / (float(e2e_ms.item()) / 1e3)
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e2e_steps, dev, world)
+    e2e_value = job_value(cfg.B, cfg.K, world, 1, e2e_ms)
 
     # the row kernel, the exact finisher (candidate modes only) and the per-batch-row kernel
     candidates = not greedy and ((0 < cfg.top_k < cfg.V) or cfg.top_p < 1.0)
