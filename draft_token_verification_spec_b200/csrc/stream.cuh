@@ -21,8 +21,14 @@
 // starts from a value that k entries of the first chunk reach (per-warp order statistics of
 // per-thread maxima); top-p from (first-chunk maximum - T ln(V / (1 - top_p))), below which
 // the whole row holds less than 1 - top_p of the mass, and follows the running maximum.
-// When the list would overflow it is cut to the top k (top-k) or about kKeep (top-p)
-// entries by count.
+// Top-p also bounds the first chunk's candidates: the threshold is raised to the smallest
+// of the largest kChunk0Vecs vector maxima (so at most 8 x that many entries pass), if that
+// is higher. The consumer warps exchange their counts (and the row maximum) every
+// kXchgTopK chunks (top-k) or every chunk (top-p); when the list is about to overflow, or
+// its projected size at the row end exceeds the capacity, it is cut by count: to the top k
+// (top-k), or to the top max(kKeepFloor, kKeepTarget * seen / V) entries seen so far
+// (top-p), which for rows whose values do not drift along the vocabulary leaves about
+// kKeepTarget candidates at the row end.
 //
 // At the end of a row the CTA selects among the candidates over a histogram of log-weight
 // bins (1/32 of a log2 unit each, relative to the row maximum; bins only coarsen the
@@ -58,7 +64,10 @@ static_assert(kChunkBytes % (16 * kThreads) == 0, "chunk = whole vectors per con
 static_assert((kRing & (kRing - 1)) == 0 && kRing <= 8, "ring depth: power of two <= 8");
 constexpr int kStreamThreads = kThreads + 32;   // eight consumer warps + the producer
 constexpr int kCap = 4096;                      // candidates per row
-constexpr int kKeep = 1024;                     // top-p: candidates a cut keeps (about)
+constexpr int kKeepFloor = 512;                 // top-p: a cut keeps at least this many
+constexpr int kKeepTarget = 3 * kCap / 4;       // top-p: candidates a cut aims at by row end
+constexpr int kChunk0Vecs = 384;                // top-p: vectors of the first chunk kept
+constexpr int kXchgTopK = 4;                    // top-k: chunks between count exchanges
 constexpr int kBins = 1024;                     // log-weight bins
 constexpr float kBinScale = 32.0f;              // bins per log2 unit of weight
 constexpr int kMemberCap = 512;                 // members of the crossing bin
@@ -86,7 +95,7 @@ struct StreamJob {
 struct __align__(16) StreamAux {
   uint64_t full[kRing];    // completes when a chunk's bytes have landed
   uint64_t empty[kRing];   // completes when the eight consumer warps are done with it
-  float red_f[2][kWarps];  // per-chunk exchange, double-buffered by chunk parity
+  float red_f[2][kWarps];  // count exchange, double-buffered by exchange parity
   int red_i[2][kWarps];
   unsigned long long scr_u64[kWarps];
   long long scr_s64[kWarps];
@@ -549,6 +558,8 @@ __global__ void __launch_bounds__(kStreamThreads, (kMode <= SM_SUMS ? 3 : 2))
   int cnt = 0;            // candidates appended this row (uniform)
   bool overflow = false;  // (uniform)
   bool row_timeout = false;
+  int wacc = 0, wlen = 0, xpar = 0;  // count exchange: this warp's appends, chunks, parity
+  int single = 0;                    // entries this thread appended one by one
   long long row = blockIdx.x;
   int q = 0, b = 0;
 
@@ -591,7 +602,34 @@ __global__ void __launch_bounds__(kStreamThreads, (kMode <= SM_SUMS ? 3 : 2))
               key_value<T>(warp_kth_key<Elem<T>::kKeyBits>(Elem<T>::key(pm), jw));
           thr = creduce<float>(tw, aux.scr_f, OpMin());
         } else {
-          thr = creduce<float>(pm, aux.scr_f, OpMaxNan()) - job.topp_span;
+          const float m0 = creduce<float>(pm, aux.scr_f, OpMaxNan());
+          float t0 = m0 - job.topp_span;
+          if (m0 > -INFINITY && m0 < INFINITY) {
+            // the vectors whose maxima fall in the bins up to the one where kChunk0Vecs of
+            // them are reached; the smallest such maximum bounds what this chunk appends
+            const float mc0 = m0 * c;
+            for (int i = threadIdx.x; i < kBins; i += kThreads) cs.hcnt[i] = 0;
+            csync();
+#pragma unroll
+            for (int u = 0; u < kVecPerThread; ++u) {
+              const int v = u * kThreads + int(threadIdx.x);
+              const bool ok = v >= v_lo && v < v_hi && vm[u] > -INFINITY;
+              hist_add(cs.hcnt, ok ? bin_of(vm[u], c, mc0) : 0, ok);
+            }
+            csync();
+            cs.hist_find((unsigned long long)kChunk0Vecs, false);
+            const int bsel = aux.sel_found ? aux.sel_bin : kBins - 1;
+            float tv = INFINITY;
+#pragma unroll
+            for (int u = 0; u < kVecPerThread; ++u) {
+              const int v = u * kThreads + int(threadIdx.x);
+              if (v >= v_lo && v < v_hi && vm[u] > -INFINITY && bin_of(vm[u], c, mc0) <= bsel)
+                tv = fminf(tv, vm[u]);
+            }
+            tv = creduce<float>(tv, aux.scr_f, OpMin());
+            if (tv < INFINITY) t0 = fmaxf(t0, tv);
+          }
+          thr = t0;
         }
       }
     }
@@ -646,7 +684,6 @@ __global__ void __launch_bounds__(kStreamThreads, (kMode <= SM_SUMS ? 3 : 2))
         }
       }
     }
-    int single = 0;  // entries this thread appended one by one (edge elements)
     if (edge) {
       for (int j = e_lo; j < e_hi; ++j) {
         const float x = Elem<T>::load(s.g, j);
@@ -654,7 +691,7 @@ __global__ void __launch_bounds__(kStreamThreads, (kMode <= SM_SUMS ? 3 : 2))
         if (kCand && x >= thr) {
           const int pos = atomicAdd(&aux.ccount, 1);
           if (pos < kCap) cs.cand[pos] = make_comp(Elem<T>::key(x), base + j);
-          ++single;
+          ++single;  // entries this thread appended one by one (edge elements)
         }
       }
     }
@@ -663,33 +700,48 @@ __global__ void __launch_bounds__(kStreamThreads, (kMode <= SM_SUMS ? 3 : 2))
     if (lane == 0) mbar_arrive(&aux.empty[b]);
 
     if constexpr (kCand) {
-      // per-chunk exchange: the row maximum so far and the entries appended
-      const int par = int(g & 1);
-      float wm = st.mt;
+      wacc += wadd;
+      ++wlen;
+      constexpr int R = kMode == SM_TOPK ? kXchgTopK : 1;
+      if (wlen == R || q == nchunk - 1) {
+        // exchange: the row maximum so far and the entries appended since the last one
+        float wm = st.mt;
 #pragma unroll
-      for (int o = 16; o > 0; o >>= 1) wm = fmax_nan(wm, __shfl_xor_sync(0xffffffffu, wm, o));
-      const int wsingle = __reduce_add_sync(0xffffffffu, single);
-      if (lane == 0) {
-        aux.red_f[par][warp] = wm;
-        aux.red_i[par][warp] = wadd + wsingle;
-      }
-      csync();
-      float mrow = aux.red_f[par][0];
-      int added = aux.red_i[par][0];
+        for (int o = 16; o > 0; o >>= 1) wm = fmax_nan(wm, __shfl_xor_sync(0xffffffffu, wm, o));
+        const int wsingle = __reduce_add_sync(0xffffffffu, single);
+        if (lane == 0) {
+          aux.red_f[xpar][warp] = wm;
+          aux.red_i[xpar][warp] = wacc + wsingle;
+        }
+        csync();
+        float mrow = aux.red_f[xpar][0];
+        int added = aux.red_i[xpar][0];
 #pragma unroll
-      for (int ww = 1; ww < kWarps; ++ww) {
-        mrow = fmax_nan(mrow, aux.red_f[par][ww]);
-        added += aux.red_i[par][ww];
-      }
-      cnt += added;
-      if (kMode == SM_TOPP) thr = fmaxf(thr, mrow - job.topp_span);
-      if (cnt > kCap) {
-        overflow = true;
-      } else if (q + 1 < nchunk && cnt + added + added / 2 > kCap) {
-        // the next chunk could overflow the list: cut it by count
-        const int keep = kMode == SM_TOPK ? rj.top_k : kKeep;
-        if (keep < cnt && mrow > -INFINITY && mrow < INFINITY)
-          cnt = cs.cut(cnt, keep, c, mrow * c, &thr);
+        for (int ww = 1; ww < kWarps; ++ww) {
+          mrow = fmax_nan(mrow, aux.red_f[xpar][ww]);
+          added += aux.red_i[xpar][ww];
+        }
+        xpar ^= 1;
+        cnt += added;
+        if (kMode == SM_TOPP) thr = fmaxf(thr, mrow - job.topp_span);
+        const int rem = nchunk - 1 - q;  // chunks of this row still to come
+        if (cnt > kCap) {
+          overflow = true;
+        } else if (rem > 0 && (cnt + added + added / 2 > kCap ||
+                               (cnt >= kCap / 4 &&
+                                cnt + (long long)added * rem / wlen > kCap))) {
+          // about to overflow, or projected to: cut the list by count
+          int keep = rj.top_k;
+          if (kMode == SM_TOPP) {
+            const long long seen = min((long long)(q + 1) * job.chunk, (long long)rj.V);
+            keep = max(kKeepFloor, int((long long)kKeepTarget * seen / rj.V));
+          }
+          if (keep < cnt && mrow > -INFINITY && mrow < INFINITY)
+            cnt = cs.cut(cnt, keep, c, mrow * c, &thr);
+        }
+        wacc = 0;
+        single = 0;
+        wlen = 0;
       }
     }
 
