@@ -21,6 +21,8 @@ HEADER_PATH = os.path.join(os.path.dirname(_PKG), "include", "specverify.h")
 
 SPEC_F32, SPEC_BF16 = 0, 1
 SPEC_OK = 0
+SPEC_ERR_INVALID_ARG, SPEC_ERR_UNSUPPORTED, SPEC_ERR_CUDA, SPEC_ERR_WORKSPACE = -1, -2, -3, -4
+SPEC_ERR_DEVICE_TIMEOUT = -5
 SPEC_MAX_VOCAB = 1 << 20
 SPEC_MAX_TREE_NODES = 4096
 
@@ -41,6 +43,7 @@ def _declare(lib):
         "spec_status_string": ([I], ctypes.c_char_p),
         "spec_workspace_size": ([I, I, I], Z),
         "spec_verify_chain": ([P, P, I, I, I, I, P, P, F, I, F, P, P, P, Z, P], I),
+        "spec_verify_chain_noalloc": ([P, P, I, I, I, I, P, P, F, I, F, P, P, P], I),
         "spec_verify_tree_typical": ([P, I, I, I, I, P, P, F, F, P, I, P, P, Z, P], I),
         "spec_logits_to_probs": ([P, I, I, I, F, I, F, P, P, P], I),
         "spec_residual_sample": ([P, P, I, I, P, P, P], I),
@@ -141,6 +144,31 @@ def spec_verify_chain(target_logits, draft_logits, draft_tokens, uniforms, temp,
         _ptr(t), _ptr(d), _dtype(t), B, K, V, _ptr(x), _ptr(u), float(temp), int(top_k),
         float(top_p), _ptr(accepted_len), _ptr(out_tokens), _ptr(workspace),
         workspace.numel() * workspace.element_size(), _stream(stream, t.device)))
+    return accepted_len, out_tokens
+
+
+def spec_verify_chain_noalloc(target_logits, draft_logits, draft_tokens, uniforms, temp,
+                              top_k=0, top_p=1.0, accepted_len=None, out_tokens=None,
+                              stream=None):
+    """spec_verify_chain with the library's static scratch instead of a workspace (calls on
+    one device must not overlap). Returns (accepted_len [B], out_tokens [B,K+1])."""
+    t = _dev(target_logits, "target_logits")
+    B, K1, V = t.shape
+    K = K1 - 1
+    d = None if draft_logits is None else _dev(draft_logits, "draft_logits", t.dtype)
+    if d is not None and tuple(d.shape) != (B, K, V):
+        raise ValueError("draft_logits must be [B, K, V]")
+    x = _dev(draft_tokens, "draft_tokens", torch.int32)
+    u = _dev(uniforms, "uniforms", torch.float32)
+    if tuple(x.shape) != (B, K) or tuple(u.shape) != (B, K + 1):
+        raise ValueError("draft_tokens must be [B, K] and uniforms [B, K+1]")
+    if accepted_len is None:
+        accepted_len = torch.empty(B, dtype=torch.int32, device=t.device)
+    if out_tokens is None:
+        out_tokens = torch.empty((B, K + 1), dtype=torch.int32, device=t.device)
+    _check("spec_verify_chain_noalloc", lib().spec_verify_chain_noalloc(
+        _ptr(t), _ptr(d), _dtype(t), B, K, V, _ptr(x), _ptr(u), float(temp), int(top_k),
+        float(top_p), _ptr(accepted_len), _ptr(out_tokens), _stream(stream, t.device)))
     return accepted_len, out_tokens
 
 

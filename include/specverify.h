@@ -139,6 +139,33 @@ spec_status spec_logits_to_probs(const void* logits, spec_dtype dtype, int rows,
 spec_status spec_residual_sample(const float* p, const float* q, int rows, int V,
                                  const float* uniforms, int32_t* tokens, void* stream);
 
+/* spec_verify_chain without a caller workspace. The pages have no counterpart: they
+ * state the verification rule, not an interface; this call is the library's own.
+ *
+ * For callers that cannot allocate device memory around the call: code recording a
+ * stream capture it does not own, plain C hosts with no device allocator, decode loops
+ * whose memory pool is fixed at start-up. Arguments, semantics and outputs are those of
+ * spec_verify_chain minus workspace / workspace_bytes. The scratch is one device array of
+ * SPEC_STATIC_SCRATCH_BYTES inside the library, one per device; the call allocates
+ * nothing and looks the array's address up once per device (with that device current).
+ *   - A call whose spec_workspace_size(B, K, V) exceeds SPEC_STATIC_SCRATCH_BYTES returns
+ *     SPEC_ERR_WORKSPACE before any CUDA call (8 MiB holds about 7,800 logit rows,
+ *     B * (2K + 1)).
+ *   - Every call on a device uses the same scratch: calls that overlap in time (on
+ *     different streams, or from host threads without ordering) race on it and give
+ *     undefined results. Order them (one stream, or events).
+ *   - Make the first call on each device outside any stream capture: it resolves the
+ *     array's address, which may load the library's device code.
+ *   - spec_get_device_status cannot see this scratch: a row whose copy wait timed out
+ *     shows as accepted_len[b] = -2. */
+#define SPEC_STATIC_SCRATCH_BYTES ((size_t)8 << 20)
+spec_status spec_verify_chain_noalloc(const void* target_logits, const void* draft_logits,
+                                      spec_dtype dtype, int B, int K, int V,
+                                      const int32_t* draft_tokens, const float* uniforms,
+                                      float temp, int top_k, float top_p,
+                                      int32_t* accepted_len, int32_t* out_tokens,
+                                      void* stream);
+
 /* Copies the device status word of `workspace` to the host (synchronises `stream`):
  * SPEC_OK, or SPEC_ERR_DEVICE_TIMEOUT if a kernel of an earlier call on this
  * workspace gave up waiting for a copy. The word is cleared by every verify call. */

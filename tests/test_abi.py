@@ -97,3 +97,13 @@ def test_probs_and_residual_invalid_args(lib):
     assert lib.spec_residual_sample(None, None, 4, 10, P(16), P(16), None) == -1
     assert lib.spec_residual_sample(P(16), None, 0, 10, P(16), P(16), None) == -1
     assert lib.spec_residual_sample(P(16), None, 4, 10, P(16), None, None) == -1
+
+
+def test_noalloc_limits_on_the_host(lib):
+    """The static-scratch call rejects sizes beyond its scratch before any CUDA call."""
+    args = lambda B, K, V: (P(16), P(16), 1, B, K, V, P(16), P(16), 1.0, 0, 1.0, P(16), P(16), None)
+    assert lib.spec_verify_chain_noalloc(*args(0, 8, 151936)) == -1
+    assert lib.spec_verify_chain_noalloc(*args(4, 0, 151936)) == -1
+    big = 1024  # 1024 * 17 rows need more than the 8 MiB scratch
+    assert sv.spec_workspace_size(big, 8, 151936) > 8 << 20
+    assert lib.spec_verify_chain_noalloc(*args(big, 8, 151936)) == -4

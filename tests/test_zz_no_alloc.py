@@ -1,0 +1,67 @@
+"""spec_verify_chain_noalloc (static scratch) against spec_verify_chain (caller workspace):
+identical outputs on two no-alloc calls in a row, so nothing carries over in the scratch from
+one call into the next. The file is collected last on purpose; the test must pass both alone
+and after every other test."""
+import numpy as np
+import pytest
+import torch
+
+import draft_token_verification_spec_b200 as sv
+import specgen
+
+pytestmark = pytest.mark.gpu
+
+
+def _inputs(cfg, B, dev):
+    t, d = specgen.chain_logits(cfg, B)
+    u = specgen.chain_uniforms(cfg, B)
+
+    def to(a):
+        if a.dtype == np.uint16:
+            return torch.from_numpy(a.view(np.int16)).to(dev).view(torch.bfloat16)
+        return torch.from_numpy(a).to(dev)
+
+    tg, dg = to(t), to(d)
+    x = dg.float().argmax(-1).to(torch.int32).contiguous()  # valid draft tokens
+    return tg, dg, x, to(u)
+
+
+# (config, batch, greedy): top-k rows with kept-id lists and sparse draws, then top-p rows
+# (candidate cuts, the exact finisher list); plain sampling, then greedy
+PAIRS = [
+    ((specgen.CFG5, 8, False), (specgen.CFG3, 8, False)),
+    ((specgen.CFG2, 16, False), (specgen.CFG2, 16, True)),
+]
+
+
+@pytest.mark.parametrize("pair", PAIRS, ids=["topk_then_topp", "sampling_then_greedy"])
+def test_noalloc_matches_workspace_call_on_two_calls_in_a_row(cuda_device, pair):
+    runs = []
+    for cfg, B, greedy in pair:
+        tg, dg, x, u = _inputs(cfg, B, cuda_device)
+        temp = 0.0 if greedy else cfg.temp
+        d = None if greedy else dg
+        ref = sv.spec_verify_chain(tg, d, x, u, temp, cfg.top_k, cfg.top_p)
+        runs.append((tg, d, x, u, temp, cfg, ref))
+    torch.cuda.synchronize()
+    outs = [sv.spec_verify_chain_noalloc(tg, d, x, u, temp, cfg.top_k, cfg.top_p)
+            for tg, d, x, u, temp, cfg, _ in runs]  # back to back on one stream
+    torch.cuda.synchronize()
+    for (tg, d, x, u, temp, cfg, (acc_r, out_r)), (acc, out) in zip(runs, outs):
+        assert int(acc_r.min()) >= 0, cfg.name
+        assert torch.equal(acc, acc_r), cfg.name
+        assert torch.equal(out, out_r), cfg.name
+
+
+def test_noalloc_rejects_a_batch_beyond_its_scratch(cuda_device):
+    cfg = specgen.CFG5
+    V = cfg.V
+    assert sv.spec_workspace_size(64, cfg.K, V) <= 8 << 20
+    assert sv.spec_workspace_size(1024, cfg.K, V) > 8 << 20
+    t = torch.zeros((1024, cfg.K + 1, V), dtype=torch.bfloat16, device=cuda_device)
+    d = torch.zeros((1024, cfg.K, V), dtype=torch.bfloat16, device=cuda_device)
+    x = torch.zeros((1024, cfg.K), dtype=torch.int32, device=cuda_device)
+    u = torch.zeros((1024, cfg.K + 1), dtype=torch.float32, device=cuda_device)
+    with pytest.raises(sv.SpecError) as e:
+        sv.spec_verify_chain_noalloc(t, d, x, u, 1.0)
+    assert e.value.status == sv.SPEC_ERR_WORKSPACE
