@@ -183,20 +183,29 @@ __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t by
       : "memory");
 }
 
+// One wait on phase `parity` of `bar`: true once it has completed. While it has not, the
+// thread is suspended for up to kWaitHintNs (it wakes when the phase completes), so a
+// waiting warp takes no issue slots from the warps that share its scheduler.
+constexpr uint32_t kWaitHintNs = 20000;
+__device__ __forceinline__ bool mbar_try_wait(uint32_t addr, uint32_t parity) {
+  uint32_t done;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n"
+      " selp.u32 %0, 1, 0, p;\n}"
+      : "=r"(done)
+      : "r"(addr), "r"(parity), "r"(kWaitHintNs)
+      : "memory");
+  return done != 0;
+}
+
 // Waits for phase `parity` of `bar` to complete; gives up after kWaitLimitNs.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
   const uint32_t addr = smem_u32(bar);
+  if (mbar_try_wait(addr, parity)) return true;
   const unsigned long long t0 = global_timer_ns();
   for (uint32_t it = 0;; ++it) {
-    uint32_t done;
-    asm volatile(
-        "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
-        " selp.u32 %0, 1, 0, p;\n}"
-        : "=r"(done)
-        : "r"(addr), "r"(parity)
-        : "memory");
-    if (done) return true;
-    if ((it & 255u) == 255u && global_timer_ns() - t0 > kWaitLimitNs) return false;
+    if (mbar_try_wait(addr, parity)) return true;
+    if ((it & 15u) == 15u && global_timer_ns() - t0 > kWaitLimitNs) return false;
   }
 }
 
