@@ -198,7 +198,7 @@ cudaError_t row_stage(spec_dtype dt, const sv::RowJob& rj, const RowPlan& pl, in
   const int E = dt == SPEC_BF16 ? 2 : 4;
   sv::StreamJob sj = {};
   sj.r = rj;
-  sj.chunk = sv::kChunkBytes / E;
+  sj.chunk = sv::stream_chunk_bytes(mode) / E;
   sj.nchunk = (rj.V + sj.chunk - 1) / sj.chunk;
   sj.topp_span = rj.top_p < 1.0f
                      ? float(std::log(double(rj.V) / (1.0 - double(rj.top_p))) / rj.inv_t)

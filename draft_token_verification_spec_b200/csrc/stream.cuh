@@ -2,14 +2,15 @@
 // with a producer warp feeding eight consumer warps.
 //
 // A CTA walks rows blockIdx.x, blockIdx.x + gridDim.x, ... cut into chunks of kChunkBytes.
-// Warp 8 (the producer, one elected lane) keeps a ring of kRing chunk buffers in shared
+// Warp 8 (the producer, one elected lane) keeps a ring of chunk buffers (Ring<mode>) in shared
 // memory full with 1-D bulk copies (cp.async.bulk; a "full" mbarrier per buffer completes
 // when the bytes land) and runs ahead across row boundaries; it reuses a buffer once the
 // eight consumer warps have arrived on its "empty" mbarrier. Consumers synchronise among
 // themselves only with named barrier 1, so the producer is never held up by their row-end
 // work. Nothing is shared between CTAs.
 //
-// Per chunk each consumer thread takes four 16-byte vectors and updates, as the mode needs:
+// Per chunk each consumer thread takes eight (greedy, sums) or four (candidate modes)
+// 16-byte vectors and updates, as the mode needs:
 //   SM_GREEDY  its running maximum (packed bf16x2 max, NaN propagating) and the lowest index
 //              holding it;
 //   SM_SUMS    an online softmax sum (and entropy term), rescaled when its maximum grows;
@@ -23,12 +24,13 @@
 // the whole row holds less than 1 - top_p of the mass, and follows the running maximum.
 // Top-p also bounds the first chunk's candidates: the threshold is raised to the smallest
 // of the largest kChunk0Vecs vector maxima (so at most 8 x that many entries pass), if that
-// is higher. The consumer warps exchange their counts (and the row maximum) every
-// kXchgTopK chunks (top-k) or every chunk (top-p); when the list is about to overflow, or
-// its projected size at the row end exceeds the capacity, it is cut by count: to the top k
-// (top-k), or to the top max(kKeepFloor, kKeepTarget * seen / V) entries seen so far
-// (top-p), which for rows whose values do not drift along the vocabulary leaves about
-// kKeepTarget candidates at the row end.
+// is higher. The consumer warps exchange their counts (and the row maximum) after the first
+// chunk, then every kXchgTopK chunks (top-k) or every chunk (top-p). The list is cut by
+// count when it is about to overflow, when its projected size at the row end exceeds the
+// capacity, or (top-k) when it holds more than 2k entries: to the top k of the entries
+// seen so far (top-k), or to the top max(kKeepFloor, kKeepTarget * seen / V) (top-p), which
+// for rows whose values do not drift along the vocabulary leaves about kKeepTarget
+// candidates at the row end. Appends are warp-aggregated (one shared atomic per warp).
 //
 // At the end of a row the CTA selects among the candidates over a histogram of log-weight
 // bins (1/32 of a log2 unit each, relative to the row maximum; bins only coarsen the
@@ -50,18 +52,39 @@
 
 namespace sv {
 
-#ifndef SV_RING_NBUF
-#define SV_RING_NBUF 4
+// Ring of chunk buffers per CTA. Greedy and plain sums (three CTAs per SM) stream two
+// 32 KB chunks; the candidate modes (two CTAs per SM, with an exchange every few chunks)
+// four 16 KB chunks, so more copies are in flight while the consumers synchronise.
+#ifndef SV_RING_NBUF_PLAIN
+#define SV_RING_NBUF_PLAIN 2
 #endif
-#ifndef SV_RING_KB
-#define SV_RING_KB 16
+#ifndef SV_RING_KB_PLAIN
+#define SV_RING_KB_PLAIN 32
 #endif
-constexpr int kRing = SV_RING_NBUF;             // chunk buffers per CTA
-constexpr int kChunkBytes = SV_RING_KB * 1024;  // bytes of logits per chunk
-constexpr int kRingBufBytes = kChunkBytes + 128;  // a chunk starts up to 15 bytes in
-constexpr int kVecPerThread = kChunkBytes / (16 * kThreads);
-static_assert(kChunkBytes % (16 * kThreads) == 0, "chunk = whole vectors per consumer");
-static_assert((kRing & (kRing - 1)) == 0 && kRing <= 8, "ring depth: power of two <= 8");
+#ifndef SV_RING_NBUF_CAND
+#define SV_RING_NBUF_CAND 4
+#endif
+#ifndef SV_RING_KB_CAND
+#define SV_RING_KB_CAND 16
+#endif
+constexpr int kMaxRing = 4;
+
+enum : int { SM_GREEDY = 0, SM_SUMS = 1, SM_TOPK = 2, SM_TOPP = 3 };
+
+template <int kMode>
+struct Ring {
+  static constexpr int kBuf = kMode <= SM_SUMS ? SV_RING_NBUF_PLAIN : SV_RING_NBUF_CAND;
+  static constexpr int kBytes = (kMode <= SM_SUMS ? SV_RING_KB_PLAIN : SV_RING_KB_CAND) * 1024;
+  static constexpr int kBufBytes = kBytes + 128;  // a chunk starts up to 15 bytes in
+  static constexpr int kVec = kBytes / (16 * kThreads);  // vectors per consumer thread
+  static_assert(kBytes % (16 * kThreads) == 0, "chunk = whole vectors per consumer");
+  static_assert((kBuf & (kBuf - 1)) == 0 && kBuf <= kMaxRing, "ring depth: power of two");
+};
+
+__host__ __device__ constexpr int stream_chunk_bytes(int mode) {
+  return (mode <= SM_SUMS ? SV_RING_KB_PLAIN : SV_RING_KB_CAND) * 1024;
+}
+
 constexpr int kStreamThreads = kThreads + 32;   // eight consumer warps + the producer
 constexpr int kCap = 4096;                      // candidates per row
 constexpr int kKeepFloor = 512;                 // top-p: a cut keeps at least this many
@@ -73,12 +96,11 @@ constexpr float kBinScale = 32.0f;              // bins per log2 unit of weight
 constexpr int kMemberCap = 512;                 // members of the crossing bin
 constexpr int kStreamMaxTopK = kKeptCap;        // top-k the candidate path takes
 
-enum : int { SM_GREEDY = 0, SM_SUMS = 1, SM_TOPK = 2, SM_TOPP = 3 };
-
 // Dynamic shared memory of one CTA: the ring, then (candidate modes) the candidate list,
 // the bin counts and the bin masses (whose space the crossing bin's members reuse).
 __host__ __device__ constexpr size_t stream_dyn_bytes(int mode) {
-  return size_t(kRing) * kRingBufBytes +
+  return (mode <= SM_SUMS ? size_t(Ring<SM_SUMS>::kBuf) * Ring<SM_SUMS>::kBufBytes
+                          : size_t(Ring<SM_TOPK>::kBuf) * Ring<SM_TOPK>::kBufBytes) +
          (mode >= SM_TOPK ? size_t(kCap) * 8 + size_t(kBins) * 4 + size_t(kBins) * 8 : 0);
 }
 static_assert(2 * kMemberCap * 8 <= kBins * 8, "members and their weights fit the masses");
@@ -93,8 +115,8 @@ struct StreamJob {
 };
 
 struct __align__(16) StreamAux {
-  uint64_t full[kRing];    // completes when a chunk's bytes have landed
-  uint64_t empty[kRing];   // completes when the eight consumer warps are done with it
+  uint64_t full[kMaxRing];   // completes when a chunk's bytes have landed
+  uint64_t empty[kMaxRing];  // completes when the eight consumer warps are done with it
   float red_f[2][kWarps];  // count exchange, double-buffered by exchange parity
   int red_i[2][kWarps];
   unsigned long long scr_u64[kWarps];
@@ -490,6 +512,8 @@ __global__ void __launch_bounds__(kStreamThreads, (kMode <= SM_SUMS ? 3 : 2))
     stream_rows_kernel(const StreamJob job) {
   constexpr bool kCand = kMode == SM_TOPK || kMode == SM_TOPP;
   constexpr int E = Elem<T>::kBytes, P = Elem<T>::kPerVec;
+  using RG = Ring<kMode>;
+  constexpr int kRing = RG::kBuf, kRingBufBytes = RG::kBufBytes, kVecPerThread = RG::kVec;
   extern __shared__ __align__(128) unsigned char smem[];
   __shared__ StreamAux aux;
   unsigned char* ring = smem;
@@ -636,19 +660,27 @@ __global__ void __launch_bounds__(kStreamThreads, (kMode <= SM_SUMS ? 3 : 2))
 
     // ---- the chunk pass
     uint32_t cm[kVecPerThread];
+    float vmax4 = -INFINITY;
 #pragma unroll
     for (int u = 0; u < kVecPerThread; ++u) {
       const int v = u * kThreads + int(threadIdx.x);
       const int j0 = base + (16 * v - s.pad) / E;
       st.vec(w[u], vm[u], j0, c, want_ent);
       cm[u] = 0;
-      if constexpr (kCand) {
-        if (v >= v_lo && v < v_hi && vm[u] >= thr) {
-          float x[P];
-          Elem<T>::unpack(w[u], x);
+      vmax4 = fmaxf(vmax4, vm[u]);  // pad vectors hold -inf; NaN never passes a filter
+    }
+    if constexpr (kCand) {
+      if (vmax4 >= thr) {
 #pragma unroll
-          for (int k = 0; k < P; ++k)
-            if (x[k] >= thr) cm[u] |= 1u << k;
+        for (int u = 0; u < kVecPerThread; ++u) {
+          const int v = u * kThreads + int(threadIdx.x);
+          if (v >= v_lo && v < v_hi && vm[u] >= thr) {
+            float x[P];
+            Elem<T>::unpack(w[u], x);
+#pragma unroll
+            for (int k = 0; k < P; ++k)
+              if (x[k] >= thr) cm[u] |= 1u << k;
+          }
         }
       }
     }
@@ -657,7 +689,7 @@ __global__ void __launch_bounds__(kStreamThreads, (kMode <= SM_SUMS ? 3 : 2))
       int my = 0;
 #pragma unroll
       for (int u = 0; u < kVecPerThread; ++u) my += __popc(cm[u]);
-      if (__any_sync(0xffffffffu, my != 0)) {
+      if (__any_sync(0xffffffffu, my != 0)) {  // one shared atomic for the warp
         int inc = my;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
@@ -703,7 +735,7 @@ __global__ void __launch_bounds__(kStreamThreads, (kMode <= SM_SUMS ? 3 : 2))
       wacc += wadd;
       ++wlen;
       constexpr int R = kMode == SM_TOPK ? kXchgTopK : 1;
-      if (wlen == R || q == nchunk - 1) {
+      if (wlen == R || q == nchunk - 1 || q == 0) {
         // exchange: the row maximum so far and the entries appended since the last one
         float wm = st.mt;
 #pragma unroll
@@ -727,10 +759,12 @@ __global__ void __launch_bounds__(kStreamThreads, (kMode <= SM_SUMS ? 3 : 2))
         const int rem = nchunk - 1 - q;  // chunks of this row still to come
         if (cnt > kCap) {
           overflow = true;
-        } else if (rem > 0 && (cnt + added + added / 2 > kCap ||
+        } else if (rem > 0 && ((kMode == SM_TOPK && cnt > 2 * rj.top_k) ||
+                               cnt + added + added / 2 > kCap ||
                                (cnt >= kCap / 4 &&
                                 cnt + (long long)added * rem / wlen > kCap))) {
-          // about to overflow, or projected to: cut the list by count
+          // top-k: more than 2k candidates; or about to overflow, or projected to: cut
+          // the list by count (top-k: to the exact k-th of the entries seen so far)
           int keep = rj.top_k;
           if (kMode == SM_TOPP) {
             const long long seen = min((long long)(q + 1) * job.chunk, (long long)rj.V);
