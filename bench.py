@@ -59,13 +59,21 @@ def measured_peaks():
 
 
 def read_profile_traffic(name: str):
-    """Per-launch DRAM traffic of the row kernel from a committed ncu summary, if any."""
-    path = os.path.join(ROOT, "profiles", "traffic.json")
+    """Per-launch DRAM traffic (read + write bytes) of the row-statistics kernel for this
+    workload, from the committed ncu summary; None if there is none or the kernel source
+    has changed since the counters were taken."""
+    import hashlib
     try:
-        with open(path) as f:
-            return json.load(f).get(name)
+        with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
+            rec = json.load(f)
+        with open(os.path.join(ROOT, "draft_token_verification_spec_b200", "csrc",
+                               "stream.cuh"), "rb") as f:
+            sha = hashlib.sha256(f.read()).hexdigest()[:16]
     except (OSError, ValueError):
         return None
+    if rec.get("stream_cuh_sha256_16") != sha:
+        return None
+    return rec.get("traffic", {}).get(name)
 
 
 def max_over_ranks(x: float, device, world: int) -> float:
