@@ -24,8 +24,8 @@
 // the whole row holds less than 1 - top_p of the mass, and follows the running maximum.
 // Top-p also bounds the first chunk's candidates: the threshold is raised to the smallest
 // of the largest kChunk0Vecs vector maxima (so at most 8 x that many entries pass), if that
-// is higher. The consumer warps exchange their counts (and the row maximum) after every
-// chunk (top-p), or after the first chunk and at the row end (top-k: the cut after the first
+// is higher. The consumer warps exchange their counts (and the row maximum) after the first
+// chunk, at the row end and (top-p) every kXchgTopP chunks (top-k: the cut after the first
 // chunk leaves a threshold that later chunks of usual rows rarely reach; a list that still
 // overflows sends the row to the exact finisher). The list is cut by
 // count when it is about to overflow, when its projected size at the row end exceeds the
@@ -90,7 +90,8 @@ __host__ __device__ constexpr int stream_chunk_bytes(int mode) {
 constexpr int kStreamThreads = kThreads + 32;   // eight consumer warps + the producer
 constexpr int kCap = 4096;                      // candidates per row
 constexpr int kKeepFloor = 512;                 // top-p: a cut keeps at least this many
-constexpr int kKeepTarget = 3 * kCap / 4;       // top-p: candidates a cut aims at by row end
+constexpr int kKeepTarget = 3 * kCap / 8;       // top-p: candidates a cut aims at by row end
+constexpr int kXchgTopP = 4;                    // top-p: chunks between count exchanges
 constexpr int kChunk0Vecs = 384;                // top-p: vectors of the first chunk kept
 constexpr int kBins = 1024;                     // log-weight bins
 constexpr float kBinScale = 32.0f;              // bins per log2 unit of weight
@@ -735,7 +736,7 @@ __global__ void __launch_bounds__(kStreamThreads, (kMode <= SM_SUMS ? 3 : 2))
     if constexpr (kCand) {
       wacc += wadd;
       ++wlen;
-      if (kMode == SM_TOPP || q == 0 || q == nchunk - 1) {
+      if ((kMode == SM_TOPP && wlen == kXchgTopP) || q == 0 || q == nchunk - 1) {
         // exchange: the row maximum so far and the entries appended since the last one
         float wm = st.mt;
 #pragma unroll
