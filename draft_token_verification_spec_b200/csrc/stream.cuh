@@ -34,10 +34,14 @@
 // for rows whose values do not drift along the vocabulary leaves about kKeepTarget
 // candidates at the row end. Appends are warp-aggregated (one shared atomic per warp).
 //
-// At the end of a row the CTA selects among the candidates over a histogram of log-weight
-// bins (1/32 of a log2 unit each, relative to the row maximum; bins only coarsen the
-// order, they never reorder it): the bin where the count (top-k) or mass (top-p) crosses
-// the target, then the exact crossing candidate among that bin's members. It writes the
+// At the end of a row the CTA selects among the candidates. Top-k lists of at most
+// kRankMax entries are ranked directly (each candidate counts the larger composites; the
+// top-p crossing within the top k accumulates their weights the same way). Longer lists go
+// over a histogram of log-weight bins (1/32 of a log2 unit each, relative to the row
+// maximum; bins only coarsen the order, they never reorder it): the bin where the count
+// (top-k) or mass (top-p) crosses the target, then the exact crossing candidate among that
+// bin's members. The cut after a top-k row's first chunk ranks the same way when the list
+// is short, and keeps the list as it is. It writes the
 // RowStats record (and the kept ids of top-k rows). Rows the candidates cannot settle
 // (list overflow, too many members in the crossing bin, or candidates holding less than
 // top_p of the mass) are marked ROW_FALLBACK and listed; the cluster kernel
@@ -96,6 +100,7 @@ constexpr int kChunk0Vecs = 384;                // top-p: vectors of the first c
 constexpr int kBins = 1024;                     // log-weight bins
 constexpr float kBinScale = 32.0f;              // bins per log2 unit of weight
 constexpr int kMemberCap = 512;                 // members of the crossing bin
+constexpr int kRankMax = 1024;                  // lists this short are ranked directly
 constexpr int kStreamMaxTopK = kKeptCap;        // top-k the candidate path takes
 
 // Dynamic shared memory of one CTA: the ring, then (candidate modes) the candidate list,
@@ -409,6 +414,50 @@ struct CandSet {
     csync();
     *thr = fmaxf(*thr, key_value<T>(kmin_all));
     return int(total);
+  }
+
+  // Short lists (n <= kRankMax, flat): the k-th largest composite among cand[0..n) that are
+  // >= lim, by counting for each the larger ones (composites are distinct) ->
+  // aux->sel_comp. The caller has synchronised the list. False if there is none.
+  __device__ bool rank_select(int n, uint64_t lim, int k) {
+    if (threadIdx.x == 0) aux->sel_comp = 0;
+    csync();
+    for (int i = threadIdx.x; i < n; i += kThreads) {
+      const uint64_t e = cand[i];
+      if (e < lim) continue;
+      int above = 0;
+      for (int j = 0; j < n; ++j) above += cand[j] > e ? 1 : 0;
+      if (above == k - 1) aux->sel_comp = e;
+    }
+    csync();
+    return aux->sel_comp != 0;
+  }
+
+  // Short lists: among the candidates >= lim, in composite order, the one where the mass
+  // accumulated from the top first reaches top_p of their total -> aux->sel_comp.
+  __device__ bool rank_mass(int n, uint64_t lim, float top_p, float c, float mc) {
+    unsigned long long* mw = hmass;  // one weight per list slot (0 below lim)
+    unsigned long long z = 0;
+    for (int i = threadIdx.x; i < n; i += kThreads) {
+      const uint64_t e = cand[i];
+      const unsigned long long w = e >= lim ? to_fx(weight(key_value<T>(comp_key(e)), c, mc)) : 0ull;
+      mw[i] = w;
+      z += w;
+    }
+    z = creduce<unsigned long long>(z, aux->scr_u64, OpSum());  // also orders mw
+    unsigned long long target = (unsigned long long)ceil(double(top_p) * double(z));
+    if (target < 1) target = 1;
+    if (threadIdx.x == 0) aux->sel_comp = 0;
+    csync();
+    for (int i = threadIdx.x; i < n; i += kThreads) {
+      const uint64_t e = cand[i];
+      if (e < lim) continue;
+      unsigned long long above = 0;
+      for (int j = 0; j < n; ++j) above += cand[j] > e ? mw[j] : 0ull;
+      if (above < target && target <= above + mw[i]) aux->sel_comp = e;
+    }
+    csync();
+    return aux->sel_comp != 0;
   }
 
   // Fixed-point sum of the weights of the candidates with composite >= lim.
@@ -736,7 +785,7 @@ __global__ void __launch_bounds__(kStreamThreads, (kMode <= SM_SUMS ? 3 : 2))
     if constexpr (kCand) {
       wacc += wadd;
       ++wlen;
-      if ((kMode == SM_TOPP && wlen == kXchgTopP) || q == 0 || q == nchunk - 1) {
+      if ((kMode == SM_TOPP && wlen == kXchgTopP && q != nchunk - 1) || q == 0) {
         // exchange: the row maximum so far and the entries appended since the last one
         float wm = st.mt;
 #pragma unroll
@@ -771,8 +820,13 @@ __global__ void __launch_bounds__(kStreamThreads, (kMode <= SM_SUMS ? 3 : 2))
             const long long seen = min((long long)(q + 1) * job.chunk, (long long)rj.V);
             keep = max(kKeepFloor, int((long long)kKeepTarget * seen / rj.V));
           }
-          if (keep < cnt && mrow > -INFINITY && mrow < INFINITY)
+          if (kMode == SM_TOPK && cnt <= kRankMax) {
+            // the exact k-th of the entries seen so far becomes the threshold; the entries
+            // below it stay in the list (the row-end selection ranks past them)
+            if (cs.rank_select(cnt, 0, keep)) thr = fmaxf(thr, key_value<T>(comp_key(aux.sel_comp)));
+          } else if (keep < cnt && mrow > -INFINITY && mrow < INFINITY) {
             cnt = cs.cut(cnt, keep, c, mrow * c, &thr);
+          }
         }
         wacc = 0;
         single = 0;
@@ -783,6 +837,7 @@ __global__ void __launch_bounds__(kStreamThreads, (kMode <= SM_SUMS ? 3 : 2))
     if (q == nchunk - 1) {
       // ---------------------------------------------------------------- row end
       const bool tmo = csync_or(row_timeout);
+      const int nall = aux.ccount;  // every append of the row is done (candidate modes)
       const float m = creduce<float>(st.mt, aux.scr_f, OpMaxNan());
       int status = tmo ? ROW_TIMEOUT
                        : ((m != m || m == INFINITY || m == -INFINITY) ? ROW_INVALID : ROW_OK);
@@ -810,28 +865,35 @@ __global__ void __launch_bounds__(kStreamThreads, (kMode <= SM_SUMS ? 3 : 2))
         }
       } else {
         if (status == ROW_OK) {
-          const int n = min(cnt, kCap);
-          bool ok = !overflow;
+          const int n = min(nall, kCap);
+          bool ok = !overflow && nall <= kCap;
           uint64_t cstar = 0;
           if constexpr (kMode == SM_TOPK) {
             ok = ok && n >= rj.top_k;
-            if (ok) {  // the k-th candidate by count
+            if (ok && n <= kRankMax) {  // short list: rank directly
+              ok = cs.rank_select(n, 0, rj.top_k);
+              cstar = aux.sel_comp;
+              if (ok && rj.top_p < 1.0f) {
+                ok = cs.rank_mass(n, cstar, rj.top_p, c, mc);
+                cstar = aux.sel_comp;
+              }
+            } else if (ok) {  // the k-th candidate by count, over log-weight bins
               cs.hist_build(n, 0, c, mc, false);
               cs.hist_find((unsigned long long)rj.top_k, false);
               ok = aux.sel_found &&
                    cs.resolve(n, 0, c, mc, false, (unsigned long long)rj.top_k - aux.sel_before);
               cstar = aux.sel_comp;
-            }
-            if (ok && rj.top_p < 1.0f) {  // then the top-p crossing within the top k
-              const unsigned long long zk = cs.mass_from(n, cstar, c, mc);
-              unsigned long long target =
-                  (unsigned long long)ceil(double(rj.top_p) * double(zk));
-              if (target < 1) target = 1;
-              cs.hist_build(n, cstar, c, mc, true);
-              cs.hist_find(target, true);
-              ok = aux.sel_found &&
-                   cs.resolve(n, cstar, c, mc, true, target - aux.sel_before);
-              cstar = aux.sel_comp;
+              if (ok && rj.top_p < 1.0f) {  // then the top-p crossing within the top k
+                const unsigned long long zk = cs.mass_from(n, cstar, c, mc);
+                unsigned long long target =
+                    (unsigned long long)ceil(double(rj.top_p) * double(zk));
+                if (target < 1) target = 1;
+                cs.hist_build(n, cstar, c, mc, true);
+                cs.hist_find(target, true);
+                ok = aux.sel_found &&
+                     cs.resolve(n, cstar, c, mc, true, target - aux.sel_before);
+                cstar = aux.sel_comp;
+              }
             }
           } else {  // top-p over the whole row: the mass target from the online sums
             float sc = 0.0f;
@@ -900,6 +962,9 @@ __global__ void __launch_bounds__(kStreamThreads, (kMode <= SM_SUMS ? 3 : 2))
       st.reset();
       thr = -INFINITY;
       cnt = 0;
+      wacc = 0;  // appends since the last exchange belong to this row
+      single = 0;
+      wlen = 0;
       overflow = false;
       row_timeout = false;
       if constexpr (kCand) {
