@@ -54,8 +54,9 @@ def _load():
         _lib.oracle_verify_chain_f64u.argtypes = [P, P, I, I, I, I, P, P, D, I, D, P, P, P, I]
         _lib.oracle_verify_tree_typical.argtypes = [P, I, I, I, I, P, P, D, D, D, P, I, P, P, I]
         _lib.oracle_residual_sample.argtypes = [P, P, I, I, P, P, P, I]
+        _lib.oracle_verify_tree_greedy.argtypes = [P, I, I, I, I, P, P, P, I, P, P, I]
         for f in (_lib.oracle_transform_rows, _lib.oracle_verify_chain,
-                  _lib.oracle_verify_chain_f64u,
+                  _lib.oracle_verify_chain_f64u, _lib.oracle_verify_tree_greedy,
                   _lib.oracle_verify_tree_typical, _lib.oracle_residual_sample):
             f.restype = I
     return _lib
@@ -141,6 +142,26 @@ def verify_tree_typical(target, node_tokens, parent_idx, eps, delta, temp=1.0, p
     if rc != 0:
         raise ValueError("oracle_verify_tree_typical rejected its arguments")
     return path, acc, flags
+
+
+def verify_tree_greedy(target, node_tokens, parent_idx, path_cap=None, threads=None):
+    """Greedy verification over a candidate tree. target [B,N,V], node_tokens int32 [B,N],
+    parent_idx int32 [N]. Returns (best_path int32 [B,path_cap], accepted_len [B],
+    next_token [B])."""
+    target = np.ascontiguousarray(target)
+    B, N, V = target.shape
+    cap = N if path_cap is None else int(path_cap)
+    toks = np.ascontiguousarray(node_tokens, dtype=np.int32).reshape(B, N)
+    par = np.ascontiguousarray(parent_idx, dtype=np.int32).reshape(N)
+    path = np.zeros((B, cap), np.int32)
+    acc = np.zeros(B, np.int32)
+    nxt = np.zeros(B, np.int32)
+    rc = _load().oracle_verify_tree_greedy(_ptr(target), _dtype_code(target), B, N, V,
+                                           _ptr(toks), _ptr(par), _ptr(path), cap, _ptr(acc),
+                                           _ptr(nxt), _threads(threads))
+    if rc != 0:
+        raise ValueError("oracle_verify_tree_greedy rejected its arguments")
+    return path, acc, nxt
 
 
 def residual_sample(p, q, uniforms, threads=None):

@@ -492,6 +492,74 @@ int oracle_verify_tree_typical(const void* target, int dtype, int B, int N, int 
   return 0;
 }
 
+// Greedy verification over a candidate tree: several draft continuations checked against
+// the target at once, the longest correct one kept ([SV] "推测解码": blockwise parallel
+// decoding accepts a draft token while it equals the target's argmax; Lookahead decoding
+// verifies candidate branches in parallel and keeps the longest correct one). Node n's
+// logits give the next-token distribution after n; node 0 is accepted; node c >= 1 is
+// accepted iff its parent is and node_tokens[c] is the argmax of the parent's logits
+// (lowest id on ties). The deepest accepted node (lowest index on ties) and its root-first
+// ancestor chain are returned, and next_token = the argmax of that node's logits (the
+// token the round emits after the path). Rows the rule reads must be valid.
+int oracle_verify_tree_greedy(const void* target, int dtype, int B, int N, int V,
+                              const int32_t* node_tokens, const int32_t* parent_idx,
+                              int32_t* best_path, int path_cap, int32_t* accepted_len,
+                              int32_t* next_token, int threads) {
+  if (!target || B < 0 || N <= 0 || V <= 0 || !node_tokens || !parent_idx || !best_path ||
+      path_cap <= 0 || !accepted_len)
+    return -1;
+  bool tree_ok = parent_idx[0] == -1;
+  std::vector<int> depth(static_cast<size_t>(N), 0);
+  for (int c = 1; c < N && tree_ok; ++c) {
+    const int pa = parent_idx[c];
+    if (pa < 0 || pa >= c)
+      tree_ok = false;
+    else
+      depth[c] = depth[pa] + 1;
+  }
+  parallel_rows(B, threads, [&](int b) {
+    int32_t* path = best_path + size_t(b) * path_cap;
+    auto fail = [&]() {
+      accepted_len[b] = -1;
+      for (int j = 0; j < path_cap; ++j) path[j] = -1;
+      if (next_token) next_token[b] = -1;
+    };
+    if (!tree_ok) return fail();
+    std::vector<int> arg(static_cast<size_t>(N), -1);  // argmax of node n's row, once read
+    std::vector<double> l;
+    auto argmax_of = [&](int n) {
+      if (arg[n] < 0) {
+        load_row(target, dtype, size_t(b) * N + n, V, l);
+        if (!row_valid(l)) return -1;
+        arg[n] = argmax_lowest(l);
+      }
+      return arg[n];
+    };
+    std::vector<char> acc(static_cast<size_t>(N), 0);
+    acc[0] = 1;
+    for (int c = 1; c < N; ++c) {
+      const int pa = parent_idx[c];
+      if (!acc[pa]) continue;
+      const int g = argmax_of(pa);
+      if (g < 0) return fail();
+      const int tok = node_tokens[size_t(b) * N + c];
+      if (tok < 0 || tok >= V) return fail();
+      acc[c] = tok == g;
+    }
+    int best = 0;
+    for (int c = 1; c < N; ++c)
+      if (acc[c] && depth[c] > depth[best]) best = c;
+    const int len = depth[best] + 1;
+    const int g = argmax_of(best);
+    if (len > path_cap || g < 0) return fail();
+    for (int j = 0; j < path_cap; ++j) path[j] = -1;
+    for (int n = best, j = len - 1; j >= 0; --j, n = (n > 0 ? parent_idx[n] : -1)) path[j] = n;
+    accepted_len[b] = len;
+    if (next_token) next_token[b] = g;
+  });
+  return 0;
+}
+
 // Inverse-CDF draw from norm(max(0, p - q)) (q == NULL: from p) for explicit
 // probability rows. Entries are probabilities: a row holding an entry that is
 // NaN or outside [0, 1], or whose p has no positive entry, gives token -1.

@@ -390,6 +390,95 @@ def test_T7_tree_at_temperature_zero_is_greedy(seed):
             assert path[b, :len(ref)].tolist() == ref and acc[b] == len(ref)
 
 
+def _greedy_tree_brute(l, toks, par):
+    """Every root-to-node path checked edge by edge against numpy's argmax (first index on
+    ties); the deepest fully matching node, lowest index first; its row's argmax."""
+    N = l.shape[0]
+    best, best_depth = 0, 0
+    for c in range(1, N):
+        path, n = [], c
+        while n > 0:
+            path.append(n)
+            n = par[n]
+        if all(toks[m] == np.argmax(l[par[m]]) for m in path) and len(path) > best_depth:
+            best, best_depth = c, len(path)
+    path, n = [best], best
+    while n > 0:
+        n = par[n]
+        path.append(n)
+    return path[::-1], int(np.argmax(l[best]))
+
+
+@pytest.mark.parametrize("seed", range(6))
+def test_tree_greedy_matches_path_enumeration(seed):
+    g = np.random.default_rng(300 + seed)
+    B, N, V = 8, 14, 12
+    par = _random_tree(g, N)
+    l = np.round(g.normal(0, 1.0, size=(B, N, V)), 1)     # coarse values: ties occur
+    am = np.argmax(l, axis=2)
+    toks = np.where(g.random((B, N)) < 0.7, am[np.arange(B)[:, None], par[None, :].clip(0)],
+                    g.integers(0, V, (B, N))).astype(np.int32)
+    logits = l.astype(np.float32)
+    assert np.array_equal(logits.astype(np.float64), l.astype(np.float32).astype(np.float64))
+    path, acc, nxt = oracle.verify_tree_greedy(logits, toks, par)
+    deep = 0
+    for b in range(B):
+        ref, ref_next = _greedy_tree_brute(logits[b].astype(np.float64), toks[b], par)
+        assert acc[b] == len(ref) and path[b, :len(ref)].tolist() == ref
+        assert np.all(path[b, len(ref):] == -1) and nxt[b] == ref_next
+        deep = max(deep, len(ref))
+    assert deep >= 3
+
+
+def test_tree_greedy_is_typical_acceptance_at_temperature_zero():
+    """Greedy tree verification is the T -> 0 limit of MEDUSA typical acceptance: the
+    typical test against a one-hot distribution passes exactly for the argmax token."""
+    g = np.random.default_rng(400)
+    B, N, V = 10, 16, 9
+    par = _random_tree(g, N)
+    l = g.permuted(np.tile(np.arange(V, dtype=np.float64), (B, N, 1)), axis=2)
+    am = np.argmax(l, axis=2)
+    toks = np.where(g.random((B, N)) < 0.65, am[np.arange(B)[:, None], par[None, :].clip(0)],
+                    g.integers(0, V, (B, N))).astype(np.int32)
+    logits = l.astype(np.float32)
+    p_g, a_g, _ = oracle.verify_tree_greedy(logits, toks, par)
+    p_t, a_t, _ = oracle.verify_tree_typical(logits, toks, par, 0.5, 0.5, temp=0.0)
+    assert np.array_equal(a_g, a_t) and np.array_equal(p_g, p_t)
+
+
+def test_tree_greedy_on_a_path_is_chain_greedy():
+    """A tree that is one path (parent = previous node) verifies like the greedy chain:
+    node c's token is draft x_(c-1) against target row c-1; the emitted token after the
+    accepted prefix is the chain's correction or bonus token."""
+    g = np.random.default_rng(500)
+    B, K, V = 12, 6, 20
+    l = g.normal(0, 2.0, size=(B, K + 1, V)).astype(np.float32)
+    am = np.argmax(l, axis=2)
+    x = np.where(g.random((B, K)) < 0.75, am[:, :K], g.integers(0, V, (B, K))).astype(np.int32)
+    acc_c, out_c, _ = oracle.verify_chain(l, None, x, np.zeros((B, K + 1), np.float32), 0.0)
+    par = np.arange(-1, K, dtype=np.int32)
+    toks = np.concatenate([np.zeros((B, 1), np.int32), x], axis=1)
+    path, acc_t, nxt = oracle.verify_tree_greedy(l, toks, par)
+    assert np.array_equal(acc_t, acc_c + 1)
+    for b in range(B):
+        assert path[b, :acc_t[b]].tolist() == list(range(acc_t[b]))
+        assert nxt[b] == out_c[b, acc_c[b]]
+
+
+def test_tree_greedy_errors_only_where_the_rule_reads():
+    V = 6
+    par = np.array([-1, 0, 0, 1], np.int32)
+    l = np.zeros((2, 4, V), np.float32)
+    l[:, 0, 2] = 1.0                 # root row argmax 2
+    l[:, 1, 4] = 1.0                 # node 1 row argmax 4
+    l[:, 2, :] = np.nan              # node 2's row: never read (no child of node 2)
+    l[1, 1, 3] = np.inf              # batch row 1: node 1's row invalid, and it is read
+    toks = np.array([[0, 2, 5, 4], [0, 2, 5, 4]], np.int32)
+    path, acc, nxt = oracle.verify_tree_greedy(l, toks, par)
+    assert acc.tolist() == [3, -1] and path[0, :3].tolist() == [0, 1, 3]
+    assert nxt[0] == int(np.argmax(l[0, 3])) and nxt[1] == -1 and np.all(path[1] == -1)
+
+
 def test_tree_workload_structure_and_invalid_parent():
     par, depth, rank = specgen.tree_structure((4, 3, 2, 2), 64)
     assert np.bincount(depth).tolist() == [1, 4, 12, 24, 23]
