@@ -244,6 +244,75 @@ bool rows_fit(long long rows, int) { return rows <= 0x7fffffffLL; }
 
 spec_status check_launch(cudaError_t e) { return e == cudaSuccess ? SPEC_OK : SPEC_ERR_CUDA; }
 
+// Tree verification, typical or greedy acceptance (the two public calls below).
+spec_status verify_tree(const void* target_logits, spec_dtype dtype, int B, int N, int V,
+                        const int32_t* node_tokens, const int32_t* parent_idx, float eps,
+                        float delta, bool greedy, int32_t* best_path, int path_cap,
+                        int32_t* accepted_len, int32_t* next_token, void* workspace,
+                        size_t workspace_bytes, void* stream) {
+  if (!target_logits || !dtype_ok(dtype) || B <= 0 || N <= 0 || V <= 0 || !node_tokens ||
+      !parent_idx || !best_path || path_cap <= 0 || !accepted_len ||
+      (!greedy && (!std::isfinite(eps) || !std::isfinite(delta))))
+    return SPEC_ERR_INVALID_ARG;
+  if (V > SPEC_MAX_VOCAB || N > SPEC_MAX_TREE_NODES) return SPEC_ERR_UNSUPPORTED;
+  const long long rows = (long long)B * N;
+  if (!workspace || !aligned16(workspace) || workspace_bytes < stats_bytes(rows))
+    return SPEC_ERR_WORKSPACE;
+  RowPlan pl;
+  if (!plan_rows(V, elem_bytes(dtype), &pl) || !rows_fit(rows, pl.C)) return SPEC_ERR_UNSUPPORTED;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int32_t* dev_status = static_cast<int32_t*>(workspace);
+  const WsLayout wl = ws_layout(rows);
+  char* ws = static_cast<char*>(workspace);
+  sv::RowStats* stats = reinterpret_cast<sv::RowStats*>(ws + wl.stats);
+  if (cudaMemsetAsync(dev_status, 0, 2 * sizeof(int32_t), s) != cudaSuccess) return SPEC_ERR_CUDA;
+
+  sv::RowJob rj = {};
+  rj.base0 = target_logits;
+  rj.base1 = target_logits;
+  rj.rows0 = rows;
+  rj.rows = rows;
+  rj.V = V;
+  rj.slice = pl.slice;
+  rj.slice_bytes = pl.slice_bytes;
+  rj.c = greedy ? 0.0f : sv::kLog2e;
+  rj.inv_t = greedy ? 0.0f : 1.0f;
+  rj.top_k = 0;
+  rj.top_p = 1.0f;
+  rj.flags = greedy ? sv::RS_GREEDY : sv::RS_ENTROPY;
+  rj.stats = stats;
+  rj.dev_status = dev_status;
+  void* evb = g_ev_before.load();
+  void* eva = g_ev_after.load();
+  if (evb) cudaEventRecord(static_cast<cudaEvent_t>(evb), s);
+  if (row_stage(dtype, rj, pl, reinterpret_cast<int32_t*>(ws + wl.fb_rows), dev_status + 1, s) !=
+      cudaSuccess)
+    return SPEC_ERR_CUDA;
+  if (eva) cudaEventRecord(static_cast<cudaEvent_t>(eva), s);
+
+  sv::TreeJob tj = {};
+  tj.target = target_logits;
+  tj.B = B;
+  tj.N = N;
+  tj.V = V;
+  tj.tokens = node_tokens;
+  tj.parent = parent_idx;
+  tj.eps = eps;
+  tj.delta = delta;
+  tj.stats = stats;
+  tj.best_path = best_path;
+  tj.path_cap = path_cap;
+  tj.accepted_len = accepted_len;
+  tj.greedy = greedy ? 1 : 0;
+  tj.next_token = next_token;
+  const size_t dyn = size_t(N) * (4 + 4 + 1 + 1) + 16;
+  if (dtype == SPEC_BF16)
+    sv::tree_finish_kernel<__nv_bfloat16><<<B, kThreads, dyn, s>>>(tj);
+  else
+    sv::tree_finish_kernel<float><<<B, kThreads, dyn, s>>>(tj);
+  return check_launch(cudaGetLastError());
+}
+
 }  // namespace
 
 extern "C" {
@@ -341,65 +410,19 @@ spec_status spec_verify_tree_typical(const void* target_logits, spec_dtype dtype
                                      const int32_t* parent_idx, float eps, float delta,
                                      int32_t* best_path, int path_cap, int32_t* accepted_len,
                                      void* workspace, size_t workspace_bytes, void* stream) {
-  if (!target_logits || !dtype_ok(dtype) || B <= 0 || N <= 0 || V <= 0 || !node_tokens ||
-      !parent_idx || !best_path || path_cap <= 0 || !accepted_len || !std::isfinite(eps) ||
-      !std::isfinite(delta))
-    return SPEC_ERR_INVALID_ARG;
-  if (V > SPEC_MAX_VOCAB || N > SPEC_MAX_TREE_NODES) return SPEC_ERR_UNSUPPORTED;
-  const long long rows = (long long)B * N;
-  if (!workspace || !aligned16(workspace) || workspace_bytes < stats_bytes(rows))
-    return SPEC_ERR_WORKSPACE;
-  RowPlan pl;
-  if (!plan_rows(V, elem_bytes(dtype), &pl) || !rows_fit(rows, pl.C)) return SPEC_ERR_UNSUPPORTED;
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
-  int32_t* dev_status = static_cast<int32_t*>(workspace);
-  const WsLayout wl = ws_layout(rows);
-  char* ws = static_cast<char*>(workspace);
-  sv::RowStats* stats = reinterpret_cast<sv::RowStats*>(ws + wl.stats);
-  if (cudaMemsetAsync(dev_status, 0, 2 * sizeof(int32_t), s) != cudaSuccess) return SPEC_ERR_CUDA;
+  return verify_tree(target_logits, dtype, B, N, V, node_tokens, parent_idx, eps, delta, false,
+                     best_path, path_cap, accepted_len, nullptr, workspace, workspace_bytes,
+                     stream);
+}
 
-  sv::RowJob rj = {};
-  rj.base0 = target_logits;
-  rj.base1 = target_logits;
-  rj.rows0 = rows;
-  rj.rows = rows;
-  rj.V = V;
-  rj.slice = pl.slice;
-  rj.slice_bytes = pl.slice_bytes;
-  rj.c = sv::kLog2e;
-  rj.inv_t = 1.0f;
-  rj.top_k = 0;
-  rj.top_p = 1.0f;
-  rj.flags = sv::RS_ENTROPY;
-  rj.stats = stats;
-  rj.dev_status = dev_status;
-  void* evb = g_ev_before.load();
-  void* eva = g_ev_after.load();
-  if (evb) cudaEventRecord(static_cast<cudaEvent_t>(evb), s);
-  if (row_stage(dtype, rj, pl, reinterpret_cast<int32_t*>(ws + wl.fb_rows), dev_status + 1, s) !=
-      cudaSuccess)
-    return SPEC_ERR_CUDA;
-  if (eva) cudaEventRecord(static_cast<cudaEvent_t>(eva), s);
-
-  sv::TreeJob tj = {};
-  tj.target = target_logits;
-  tj.B = B;
-  tj.N = N;
-  tj.V = V;
-  tj.tokens = node_tokens;
-  tj.parent = parent_idx;
-  tj.eps = eps;
-  tj.delta = delta;
-  tj.stats = stats;
-  tj.best_path = best_path;
-  tj.path_cap = path_cap;
-  tj.accepted_len = accepted_len;
-  const size_t dyn = size_t(N) * (4 + 4 + 1 + 1) + 16;
-  if (dtype == SPEC_BF16)
-    sv::tree_finish_kernel<__nv_bfloat16><<<B, kThreads, dyn, s>>>(tj);
-  else
-    sv::tree_finish_kernel<float><<<B, kThreads, dyn, s>>>(tj);
-  return check_launch(cudaGetLastError());
+spec_status spec_verify_tree_greedy(const void* target_logits, spec_dtype dtype, int B, int N,
+                                    int V, const int32_t* node_tokens, const int32_t* parent_idx,
+                                    int32_t* best_path, int path_cap, int32_t* accepted_len,
+                                    int32_t* next_token, void* workspace, size_t workspace_bytes,
+                                    void* stream) {
+  return verify_tree(target_logits, dtype, B, N, V, node_tokens, parent_idx, 0.0f, 0.0f, true,
+                     best_path, path_cap, accepted_len, next_token, workspace, workspace_bytes,
+                     stream);
 }
 
 spec_status spec_logits_to_probs(const void* logits, spec_dtype dtype, int rows, int V,
@@ -462,6 +485,7 @@ int spec_kernels_per_call(const char* entry_point) {
   if (!entry_point) return -1;
   if (!std::strcmp(entry_point, "spec_verify_chain")) return 3;
   if (!std::strcmp(entry_point, "spec_verify_tree_typical")) return 2;
+  if (!std::strcmp(entry_point, "spec_verify_tree_greedy")) return 2;
   if (!std::strcmp(entry_point, "spec_logits_to_probs")) return 1;
   if (!std::strcmp(entry_point, "spec_residual_sample")) return 1;
   return -1;

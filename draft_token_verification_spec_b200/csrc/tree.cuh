@@ -1,12 +1,16 @@
-// MEDUSA typical acceptance over a candidate tree, after the row statistics: one
-// thread block per batch row ("Key Components", spec-decoding-i notes; "推测解码").
+// Verification over a candidate tree, after the row statistics: one thread block per batch
+// row. Typical acceptance (MEDUSA, "Key Components", spec-decoding-i notes; "推测解码"), or
+// greedy acceptance (blockwise parallel decoding / Lookahead, "推测解码": several candidate
+// branches checked against the target's argmax at once, the longest correct one kept).
 //
-// Threads test every non-root node in parallel: p_parent(tok_c) > min(eps, delta *
-// exp(-H(p_parent))), p the temperature-1 softmax of the parent's logits. One thread
+// Threads test every non-root node in parallel: typical, p_parent(tok_c) > min(eps,
+// delta * exp(-H(p_parent))), p the temperature-1 softmax of the parent's logits; greedy,
+// tok_c == the argmax of the parent's logits (lowest id on ties). One thread
 // then resolves ancestry in index order (parents precede children): a node is
 // accepted iff its parent is and its own test passes; the root is accepted
 // unconditionally. The deepest accepted node (lowest index on ties) and its
-// root-first ancestor chain are written out.
+// root-first ancestor chain are written out; in greedy mode also the argmax of the deepest
+// node's row, the token the round emits after the path.
 #pragma once
 
 #include "draw.cuh"
@@ -23,6 +27,8 @@ struct TreeJob {
   int32_t* best_path;        // [B][path_cap]
   int path_cap;
   int32_t* accepted_len;     // [B]
+  int greedy;                // greedy acceptance (stats hold each row's argmax)
+  int32_t* next_token;       // [B] or NULL (greedy mode)
 };
 
 enum : int8_t { ND_REJECT = 0, ND_ACCEPT = 1, ND_ERROR = 2, ND_TIMEOUT = 3 };
@@ -55,6 +61,8 @@ __global__ void __launch_bounds__(kThreads) tree_finish_kernel(const TreeJob j) 
         const int tk = tok[c];
         if (tk < 0 || tk >= V) {
           t = ND_ERROR;
+        } else if (j.greedy) {
+          t = tk == s.argmax ? ND_ACCEPT : ND_REJECT;
         } else {
           const float l = Elem<T>::load(rows, size_t(pa) * V + tk);
           const float p = prob<T>(s, l, tk);
@@ -89,6 +97,15 @@ __global__ void __launch_bounds__(kThreads) tree_finish_kernel(const TreeJob j) 
     }
     int len = err ? 0 : depth[best] + 1;
     if (!err && len > j.path_cap) err = ND_ERROR;
+    int next = -1;
+    if (!err && j.greedy) {  // the deepest node's own row is read for the next token
+      const RowStats sb = st[best];
+      if (sb.status != ROW_OK)
+        err = sb.status == ROW_TIMEOUT ? ND_TIMEOUT : ND_ERROR;
+      else
+        next = sb.argmax;
+    }
+    if (j.next_token) j.next_token[b] = err ? (err == ND_TIMEOUT ? -2 : -1) : next;
     if (!err) {
       for (int n = best, k = len - 1; k >= 0; --k, n = (n > 0 ? par[n] : -1)) path[k] = n;
     }

@@ -70,8 +70,9 @@ typedef enum { SPEC_F32 = 0, SPEC_BF16 = 1 } spec_dtype;
 /* Human-readable name of a status code (static string). */
 const char* spec_status_string(int status);
 
-/* Bytes of workspace that spec_verify_chain(B, K, V) and spec_verify_tree_typical(B,
- * N = K_or_N, V) need; either call accepts any workspace at least this large. The
+/* Bytes of workspace that spec_verify_chain(B, K, V), spec_verify_tree_typical(B,
+ * N = K_or_N, V) and spec_verify_tree_greedy(B, N, V) need; each call accepts any
+ * workspace at least this large. The
  * workspace must be 16-byte aligned. Returns 0 for invalid sizes. */
 size_t spec_workspace_size(int B, int K_or_N, int V);
 
@@ -120,6 +121,25 @@ spec_status spec_verify_tree_typical(const void* target_logits, spec_dtype dtype
                                      const int32_t* parent_idx, float eps, float delta,
                                      int32_t* best_path, int path_cap, int32_t* accepted_len,
                                      void* workspace, size_t workspace_bytes, void* stream);
+
+/* Greedy verification over a candidate tree: several candidate continuations checked
+ * against the target at once, the longest correct one kept — [SV] "推测解码" (blockwise
+ * parallel decoding accepts a draft token while it equals the target's argmax; Lookahead
+ * decoding verifies candidate branches in parallel and keeps the longest correct prefix).
+ * Branches that share a prefix share their nodes; independent branches all hang off node
+ * 0. Layout, conventions and outputs as spec_verify_tree_typical, plus
+ *   next_token    [B] int32 out or NULL: the argmax of the deepest accepted node's row,
+ *                  the token the round emits after the path (-1 on an error row).
+ * Node c >= 1 is accepted iff its parent is and node_tokens[b][c] is the argmax of the
+ * parent's row (lowest id on ties); the deepest accepted node wins, the lowest node
+ * index on ties. Only argmaxes are computed: the row stage reads each row once and does
+ * no exp. The deepest accepted node's own row must be valid (it gives next_token).
+ * 1 <= N <= SPEC_MAX_TREE_NODES. */
+spec_status spec_verify_tree_greedy(const void* target_logits, spec_dtype dtype, int B, int N,
+                                    int V, const int32_t* node_tokens, const int32_t* parent_idx,
+                                    int32_t* best_path, int path_cap, int32_t* accepted_len,
+                                    int32_t* next_token, void* workspace, size_t workspace_bytes,
+                                    void* stream);
 
 /* The sampling transform alone — [SD] "Speculative Sampling" (last bullet).
  *   logits [rows][V]; probs [rows][V] float out: the transformed distribution

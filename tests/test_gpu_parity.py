@@ -262,6 +262,67 @@ def test_tree_invalid_inputs():
     assert np.all(one[1] == 1) and np.all(one[0][:, 0] == 0)
 
 
+# ------------------------------------------------------------------ greedy tree (multi-branch)
+
+def assert_tree_greedy_parity(logits, toks, par, path_cap=None):
+    path_g, len_g, nxt_g = sv.spec_verify_tree_greedy(dev(logits), dev(toks), dev(par),
+                                                      path_cap=path_cap)
+    torch.cuda.synchronize()
+    path_r, len_r, nxt_r = oracle.verify_tree_greedy(logits, toks, par, path_cap=path_cap)
+    # argmax decisions on exact logits: bit-exact, no flags
+    assert np.array_equal(len_g.cpu().numpy(), len_r)
+    assert np.array_equal(path_g.cpu().numpy(), path_r)
+    assert np.array_equal(nxt_g.cpu().numpy(), nxt_r)
+    return len_r
+
+
+def _greedy_tree_tokens(g, logits_f32, par, p_match):
+    """Node tokens that follow the parent's argmax with probability p_match (deep paths)."""
+    am = np.argmax(logits_f32, axis=2)
+    B, N = am.shape
+    return np.where(g.random((B, N)) < p_match, am[np.arange(B)[:, None], par[None, :].clip(0)],
+                    g.integers(0, logits_f32.shape[2], (B, N))).astype(np.int32)
+
+
+def test_tree_greedy_workload_full_size():
+    """The 32 x 64-node tree workload, tokens following the parent's argmax often."""
+    cfg = specgen.CFG4
+    logits, _, par = specgen.tree_inputs(cfg)
+    g = np.random.default_rng(7)
+    toks = _greedy_tree_tokens(g, specgen.bf16_bits_to_f32(logits), par, 0.8)
+    lens = assert_tree_greedy_parity(logits, toks, par)
+    assert lens.max() >= 4
+
+
+@pytest.mark.parametrize("dtype,V", [("bf16", 32000), ("f32", 1000), ("bf16", 151936),
+                                     ("bf16", 17), ("f32", 4099)])
+def test_tree_greedy_random(dtype, V):
+    g = np.random.default_rng(V)
+    B, N = 6, 30
+    par = np.array([-1] + [int(g.integers(max(0, c - 5), c)) for c in range(1, N)], np.int32)
+    x = np.round(g.normal(0, 2.0, (B, N, V)), 1).astype(np.float32)  # ties at the maximum
+    logits = x if dtype == "f32" else specgen.f32_to_bf16_bits(x)
+    lf = x if dtype == "f32" else specgen.bf16_bits_to_f32(logits)
+    toks = _greedy_tree_tokens(g, lf, par, 0.85)
+    assert_tree_greedy_parity(logits, toks, par)
+    assert_tree_greedy_parity(logits, toks, par, path_cap=3)   # too-long paths: error rows
+
+
+def test_tree_greedy_invalid_inputs():
+    B, N, V = 3, 5, 20
+    logits = np.zeros((B, N, V), np.float32)
+    logits[:, :, 7] = 1.0
+    toks = np.full((B, N), 7, np.int32)
+    par = np.array([-1, 0, 0, 1, 3], np.int32)
+    logits[1, 1, 4] = np.nan      # read: node 1 is accepted and has a child
+    toks[2, 3] = 99               # out of range on an accepted path
+    lens = assert_tree_greedy_parity(logits, toks, par)
+    assert lens.tolist() == [4, -1, -1]
+    bad_par = np.array([-1, 0, 3, 1, 1], np.int32)
+    path, plen, nxt = sv.spec_verify_tree_greedy(dev(logits), dev(toks), dev(bad_par))
+    assert np.all(plen.cpu().numpy() == -1) and np.all(nxt.cpu().numpy() == -1)
+
+
 # ------------------------------------------------------------------ transform and residual draw
 
 @pytest.mark.parametrize("dtype,V", [("bf16", 32000), ("f32", 1000), ("bf16", 128256), ("f32", 40000),
