@@ -4,11 +4,13 @@
 // cumulative mass C_v exceeds w * S, S the total; if rounding leaves none, the largest
 // v with res[v] > 0. Masses are fixed point (42 fraction bits), so every partial sum
 // is exact and the result does not depend on how the sum is split across threads.
-// The row is read in chunks of 2048 entries (8 consecutive entries per thread); the
-// first pass records each chunk's mass, the second re-reads only the chunk that holds
-// the crossing. This is the resampling step of "Speculative Decoding" /
-// "Speculative Sampling" (spec-decoding-i notes) with the reading that the draw
-// walks token ids in ascending order.
+// The row is read in chunks of kThreads * m groups of 8 entries (m groups per thread,
+// m = 1 unless the row has more than kMaxDrawChunks such chunks). The first pass records
+// each warp's share of each chunk's mass with no block barrier; one barrier later the
+// chunk totals locate the chunk that holds the crossing, and only that chunk is read
+// again. This is the resampling step of "Speculative Decoding" / "Speculative Sampling"
+// (spec-decoding-i notes) with the reading that the draw walks token ids in ascending
+// order.
 #pragma once
 
 #include <climits>
@@ -17,60 +19,68 @@
 
 namespace sv {
 
-constexpr int kDrawChunk = kThreads * 8;
-constexpr int kMaxDrawChunks = (1 << 20) / kDrawChunk;  // V <= 2^20
+constexpr int kMaxDrawChunks = 128;
 constexpr int kSparseCap = kThreads;                    // support of a sparse draw
 
 struct DrawSmem {
-  unsigned long long chunk[kMaxDrawChunks];
+  unsigned long long wchunk[kMaxDrawChunks][kWarps];   // per-warp mass of each chunk
   int ids[kSparseCap];
   unsigned long long scr[kWarps];
   unsigned long long total;
-  int best;
+  unsigned long long sel_before;
   int sel_chunk;
   int fallback;
-  unsigned long long sel_before;
+  int best;
 };
 
 // f(v0, r) fills r[0..7] with the fixed-point masses of entries v0..v0+7 (0 past V).
 // Returns -1 when the whole row has zero mass.
 template <typename F>
 __device__ int inverse_cdf_draw(F&& f, int V, float w, DrawSmem& sm) {
-  const int nch = (V + kDrawChunk - 1) / kDrawChunk;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int G = (V + 7) / 8;
+  const int m = max(1, (G + kThreads * kMaxDrawChunks - 1) / (kThreads * kMaxDrawChunks));
+  const int CG = kThreads * m;  // groups per chunk
+  const int nch = (G + CG - 1) / CG;
   for (int ch = 0; ch < nch; ++ch) {
-    unsigned long long r[8];
-    f(ch * kDrawChunk + threadIdx.x * 8, r);
     unsigned long long t = 0;
+    for (int i = 0; i < m; ++i) {
+      const int g = ch * CG + i * kThreads + int(threadIdx.x);  // coalesced within a warp
+      if (g < G) {
+        unsigned long long r[8];
+        f(g * 8, r);
 #pragma unroll
-    for (int k = 0; k < 8; ++k) t += r[k];
-    t = block_sum_u64(t, sm.scr);
-    if (threadIdx.x == 0) sm.chunk[ch] = t;
+        for (int k = 0; k < 8; ++k) t += r[k];
+      }
+    }
+    t = warp_sum_u64(t);
+    if (lane == 0) sm.wchunk[ch][warp] = t;
   }
   __syncthreads();
   if (threadIdx.x == 0) {
     unsigned long long S = 0;
-    for (int ch = 0; ch < nch; ++ch) S += sm.chunk[ch];
+    for (int ch = 0; ch < nch; ++ch)
+      for (int ww = 0; ww < kWarps; ++ww) S += sm.wchunk[ch][ww];
     const double target = double(w) * double(S);
-    unsigned long long cum = 0;
-    int sel = -1, last_pos = -1;
-    unsigned long long last_before = 0, sel_before = 0;
+    unsigned long long cum = 0, sel_before = 0, last_before = 0;
+    int sel = -1, last = -1;
     for (int ch = 0; ch < nch; ++ch) {
-      const unsigned long long s = sm.chunk[ch];
-      if (s > 0) {
-        last_pos = ch;
+      unsigned long long c = 0;
+      for (int ww = 0; ww < kWarps; ++ww) c += sm.wchunk[ch][ww];
+      if (c > 0) {
+        last = ch;
         last_before = cum;
-        if (sel < 0 && double(cum + s) > target) {
+        if (sel < 0 && double(cum + c) > target) {
           sel = ch;
           sel_before = cum;
         }
       }
-      cum += s;
+      cum += c;
     }
-    sm.fallback = 0;
+    sm.fallback = sel < 0;
     if (sel < 0) {
-      sel = last_pos;
+      sel = last;
       sel_before = last_before;
-      sm.fallback = 1;
     }
     sm.sel_chunk = sel;
     sm.sel_before = sel_before;
@@ -79,31 +89,47 @@ __device__ int inverse_cdf_draw(F&& f, int V, float w, DrawSmem& sm) {
   }
   __syncthreads();
   const int sel = sm.sel_chunk;
-  if (sel < 0) return -1;
+  if (sel < 0) {
+    __syncthreads();
+    return -1;
+  }
   const double target = double(w) * double(sm.total);
-  unsigned long long r[8];
-  const int v0 = sel * kDrawChunk + threadIdx.x * 8;
-  f(v0, r);
-  unsigned long long t = 0;
+  // the chunk again, in token order: thread t takes groups t, t + kThreads, ... of it;
+  // group j of the chunk is entry range [8 (sel * CG + j), +8)
+  unsigned long long rr[8];
+  unsigned long long own = 0;  // this thread's mass, in the order that scans below expect
+  // order within the chunk: i-major (i * kThreads + t), so a scan per i keeps token order
+  unsigned long long before = sm.sel_before;
+  for (int i = 0; i < m; ++i) {
+    const int g = sel * CG + i * kThreads + int(threadIdx.x);
+    if (g < G) {
+      f(g * 8, rr);
+    } else {
 #pragma unroll
-  for (int k = 0; k < 8; ++k) t += r[k];
-  unsigned long long total;
-  unsigned long long cum = sm.sel_before + block_exclusive_scan<unsigned long long>(t, sm.scr, &total);
-  if (sm.fallback) {
-    int last = -1;
+      for (int k = 0; k < 8; ++k) rr[k] = 0ull;
+    }
+    own = 0;
 #pragma unroll
-    for (int k = 0; k < 8; ++k)
-      if (r[k] > 0) last = v0 + k;
-    if (last >= 0) atomicMax(&sm.best, last);
-  } else {
+    for (int k = 0; k < 8; ++k) own += rr[k];
+    unsigned long long total;
+    unsigned long long cum = before + block_exclusive_scan<unsigned long long>(own, sm.scr, &total);
+    if (sm.fallback) {
+      int lst = -1;
 #pragma unroll
-    for (int k = 0; k < 8; ++k) {
-      cum += r[k];
-      if (r[k] > 0 && double(cum) > target) {
-        atomicMin(&sm.best, v0 + k);
-        break;
+      for (int k = 0; k < 8; ++k)
+        if (rr[k] > 0) lst = g * 8 + k;
+      if (lst >= 0) atomicMax(&sm.best, lst);
+    } else {
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        cum += rr[k];
+        if (rr[k] > 0 && double(cum) > target) {
+          atomicMin(&sm.best, g * 8 + k);
+          break;
+        }
       }
     }
+    before += total;
   }
   __syncthreads();
   const int tok = sm.best;
