@@ -1,5 +1,6 @@
 // Row statistics kernel: persistent thread-block clusters, one logit row per cluster
-// at a time.
+// at a time. It computes spec_logits_to_probs, finishes the rows the streaming kernel
+// (stream.cuh) lists as unsettled, and takes top-k above the streaming kernel's limit.
 //
 // A cluster of C CTAs walks rows cid, cid + G, cid + 2G, ... (G clusters resident). Each
 // CTA owns a contiguous slice of every row and keeps a ring of kNBuf slice buffers in

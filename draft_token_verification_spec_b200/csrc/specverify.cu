@@ -18,9 +18,10 @@ namespace {
 
 using sv::kThreads;
 
-// Slice of a logit row per CTA: each CTA keeps sv::kNBuf slices in flight, and two
-// CTAs share an SM, so one CTA's computation overlaps the other's copies and its own
-// next rows' copies.
+// Cluster kernel (spec_logits_to_probs, the exact finisher of listed rows, top-k above
+// the streaming limit): a slice of a logit row per CTA; each CTA keeps sv::kNBuf slices in
+// flight, and two CTAs share an SM, so one CTA's computation overlaps the other's copies
+// and its own next rows' copies.
 #ifndef SV_SLICE_KB
 #define SV_SLICE_KB 40
 #endif

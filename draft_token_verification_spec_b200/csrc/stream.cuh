@@ -1,11 +1,11 @@
 // Streaming row statistics kernel: one CTA per logit row at a time, persistent over rows,
 // with a producer warp feeding eight consumer warps.
 //
-// A CTA walks rows blockIdx.x, blockIdx.x + gridDim.x, ... cut into chunks of kChunkBytes.
-// Warp 8 (the producer, one elected lane) keeps a ring of chunk buffers (Ring<mode>) in shared
-// memory full with 1-D bulk copies (cp.async.bulk; a "full" mbarrier per buffer completes
-// when the bytes land) and runs ahead across row boundaries; it reuses a buffer once the
-// eight consumer warps have arrived on its "empty" mbarrier. Consumers synchronise among
+// A CTA walks rows blockIdx.x, blockIdx.x + gridDim.x, ... cut into chunks (Ring<mode>).
+// Warp 8 (the producer, one elected lane) keeps a ring of chunk buffers in shared memory
+// full with 1-D bulk copies (cp.async.bulk; a "full" mbarrier per buffer completes when
+// the bytes land) and runs ahead across row boundaries; it reuses a buffer once the eight
+// consumer warps have arrived on its "empty" mbarrier. Consumers synchronise among
 // themselves only with named barrier 1, so the producer is never held up by their row-end
 // work. Nothing is shared between CTAs.
 //
@@ -15,41 +15,43 @@
 //              holding it;
 //   SM_SUMS    an online softmax sum (and entropy term), rescaled when its maximum grows;
 //   SM_TOPK    the running maximum, and appends the entries >= a threshold to the CTA's
-//              candidate list;
+//              candidate list (warp-aggregated: one shared atomic per warp);
 //   SM_TOPP    the online sum and the candidate list.
 // Candidates are 64-bit composites (key << 32 | ~id): the order of composites is the order
-// (value desc, id asc) that top-k and top-p use, so the k-th candidate is unique. Top-k
-// starts from a value that k entries of the first chunk reach (per-warp order statistics of
-// per-thread maxima); top-p from (first-chunk maximum - T ln(V / (1 - top_p))), below which
-// the whole row holds less than 1 - top_p of the mass, and follows the running maximum.
-// Top-p also bounds the first chunk's candidates: the threshold is raised to the smallest
-// of the largest kChunk0Vecs vector maxima (so at most 8 x that many entries pass), if that
-// is higher. The consumer warps exchange their counts (and the row maximum) after the first
-// chunk, at the row end and (top-p) every kXchgTopP chunks (top-k: the cut after the first
-// chunk leaves a threshold that later chunks of usual rows rarely reach; a list that still
-// overflows sends the row to the exact finisher). The list is cut by
-// count when it is about to overflow, when its projected size at the row end exceeds the
-// capacity, or (top-k) when it holds more than 2k entries: to the top k of the entries
-// seen so far (top-k), or to the top max(kKeepFloor, kKeepTarget * seen / V) (top-p), which
-// for rows whose values do not drift along the vocabulary leaves about kKeepTarget
-// candidates at the row end. Appends are warp-aggregated (one shared atomic per warp).
+// (value desc, id asc) that top-k and top-p use, so the k-th candidate is unique.
+//
+// Top-k: the first threshold is a value that k entries of the first chunk reach (per-warp
+// order statistics of per-thread maxima). After the first chunk the consumer warps exchange
+// their counts once, and a list of more than 2k entries sets the threshold to the exact
+// k-th of the chunk (ranked directly, the list kept as it is; longer lists are cut over
+// log-weight bins). Later chunks of usual rows rarely reach it; no further exchange runs,
+// and a list that still overflows sends the row to the exact finisher.
+//
+// Top-p: the threshold starts at (first-chunk maximum - T ln(V / (1 - top_p))), below
+// which the whole row holds less than 1 - top_p of the mass, raised to the smallest of
+// the largest kChunk0Vecs vector maxima of the first chunk (so at most 8 x that many
+// entries pass) if that is higher. The warps exchange counts and the row maximum after the
+// first chunk and then every kXchgTopP chunks: the threshold follows the maximum, and the
+// list is cut by count when it is about to overflow or its projected size at the row end
+// exceeds the capacity, to the top max(kKeepFloor, kKeepTarget * seen / V) entries seen so
+// far (about kKeepTarget candidates at the row end for rows whose values do not drift
+// along the vocabulary).
 //
 // At the end of a row the CTA selects among the candidates. Top-k lists of at most
 // kRankMax entries are ranked directly (each candidate counts the larger composites; the
-// top-p crossing within the top k accumulates their weights the same way). Longer lists go
+// top-p crossing within the top k accumulates their weights the same way). Other lists go
 // over a histogram of log-weight bins (1/32 of a log2 unit each, relative to the row
 // maximum; bins only coarsen the order, they never reorder it): the bin where the count
 // (top-k) or mass (top-p) crosses the target, then the exact crossing candidate among that
-// bin's members. The cut after a top-k row's first chunk ranks the same way when the list
-// is short, and keeps the list as it is. It writes the
-// RowStats record (and the kept ids of top-k rows). Rows the candidates cannot settle
-// (list overflow, too many members in the crossing bin, or candidates holding less than
-// top_p of the mass) are marked ROW_FALLBACK and listed; the cluster kernel
-// (row_stats.cuh) then finishes them exactly.
+// bin's members. It writes the RowStats record (and the kept ids of top-k rows). Rows the
+// candidates cannot settle (list overflow, too many members in the crossing bin, or
+// candidates holding less than top_p of the mass) are marked ROW_FALLBACK and listed; the
+// cluster kernel (row_stats.cuh) then finishes them exactly.
 //
 // This is the sampling transform of "Speculative Sampling" (spec-decoding-i notes, last
-// bullet: transform the probabilities first, then apply the rejection scheme) and the
-// entropy used by MEDUSA typical acceptance ("Key Components").
+// bullet: transform the probabilities first, then apply the rejection scheme), the argmax
+// of the greedy forms and the entropy used by MEDUSA typical acceptance ("Key
+// Components").
 #pragma once
 
 #include <climits>
