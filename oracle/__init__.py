@@ -55,6 +55,12 @@ def _load():
         _lib.oracle_verify_tree_typical.argtypes = [P, I, I, I, I, P, P, D, D, D, P, I, P, P, I]
         _lib.oracle_residual_sample.argtypes = [P, P, I, I, P, P, P, I]
         _lib.oracle_verify_tree_greedy.argtypes = [P, I, I, I, I, P, P, P, I, P, P, I]
+        _lib.oracle_verify_tree_sampling.argtypes = [P, P, I, I, I, I, P, P, P, D, I, D, P, I, P,
+                                                     P, P, I]
+        _lib.oracle_verify_tree_sampling_f64u.argtypes = \
+            _lib.oracle_verify_tree_sampling.argtypes
+        _lib.oracle_verify_tree_sampling.restype = I
+        _lib.oracle_verify_tree_sampling_f64u.restype = I
         for f in (_lib.oracle_transform_rows, _lib.oracle_verify_chain,
                   _lib.oracle_verify_chain_f64u, _lib.oracle_verify_tree_greedy,
                   _lib.oracle_verify_tree_typical, _lib.oracle_residual_sample):
@@ -162,6 +168,36 @@ def verify_tree_greedy(target, node_tokens, parent_idx, path_cap=None, threads=N
     if rc != 0:
         raise ValueError("oracle_verify_tree_greedy rejected its arguments")
     return path, acc, nxt
+
+
+def verify_tree_sampling(target, draft, node_tokens, parent_idx, uniforms, temp, top_k=0,
+                         top_p=1.0, path_cap=None, threads=None):
+    """Rejection sampling over a candidate tree. target and draft [B,N,V] (draft unused
+    when temp == 0), node_tokens int32 [B,N], parent_idx int32 [N], uniforms [B,N+1]
+    (float64 uniforms select the double-precision entry). Returns (best_path [B,path_cap],
+    accepted_len [B], next_token [B], flags [B])."""
+    target = np.ascontiguousarray(target)
+    B, N, V = target.shape
+    if draft is not None:
+        draft = np.ascontiguousarray(draft)
+        assert draft.shape == target.shape and draft.dtype == target.dtype
+    cap = N if path_cap is None else int(path_cap)
+    toks = np.ascontiguousarray(node_tokens, dtype=np.int32).reshape(B, N)
+    par = np.ascontiguousarray(parent_idx, dtype=np.int32).reshape(N)
+    uniforms = np.asarray(uniforms)
+    wide = uniforms.dtype == np.float64
+    u = np.ascontiguousarray(uniforms, dtype=np.float64 if wide else np.float32).reshape(B, N + 1)
+    path = np.zeros((B, cap), np.int32)
+    acc = np.zeros(B, np.int32)
+    nxt = np.zeros(B, np.int32)
+    flags = np.zeros(B, np.int32)
+    fn = _load().oracle_verify_tree_sampling_f64u if wide else _load().oracle_verify_tree_sampling
+    rc = fn(_ptr(target), _ptr(draft), _dtype_code(target), B, N, V, _ptr(toks), _ptr(par),
+            _ptr(u), float(temp), int(top_k), float(top_p), _ptr(path), cap, _ptr(acc),
+            _ptr(nxt), _ptr(flags), _threads(threads))
+    if rc != 0:
+        raise ValueError("oracle_verify_tree_sampling rejected its arguments")
+    return path, acc, nxt, flags
 
 
 def residual_sample(p, q, uniforms, threads=None):

@@ -560,6 +560,128 @@ int oracle_verify_tree_greedy(const void* target, int dtype, int B, int N, int V
   return 0;
 }
 
+// Rejection sampling over a candidate tree ([SD] "Key Components": MEDUSA's step (3) may
+// reuse the rejection rule of speculative sampling so that the output keeps the target
+// distribution). Node n's target row gives p_n, its draft row q_n, the distribution its
+// children's tokens were drawn from (independently). From the root: at the current node,
+// the children are tried in index order; child c is accepted iff u[c] < min(1, p'(x_c) /
+// q(x_c)), p' the current residual (p_n at first); a rejection replaces p' by
+// norm(max(0, p' - q_n)) (unchanged if that is empty). An accepted child becomes the current
+// node. When no child is accepted (or there is none) the emitted token is drawn from p' by
+// the inverse CDF with u[N]. The accepted path (root first) and that token are returned.
+// T == 0 is the greedy limit: the first child whose token is the argmax of p_n is accepted,
+// and the emitted token is that argmax. uniforms [B][N + 1] (u[0] unused).
+int oracle_verify_tree_sampling_f64u(const void* target, const void* draft, int dtype, int B,
+                                     int N, int V, const int32_t* node_tokens,
+                                     const int32_t* parent_idx, const double* uniforms, double T,
+                                     int top_k, double top_p, int32_t* best_path, int path_cap,
+                                     int32_t* accepted_len, int32_t* next_token, int32_t* flags,
+                                     int threads) {
+  if (!target || (T != 0.0 && !draft) || B < 0 || N <= 0 || V <= 0 || !node_tokens ||
+      !parent_idx || !uniforms || !best_path || path_cap <= 0 || !accepted_len || !(T >= 0.0))
+    return -1;
+  bool tree_ok = parent_idx[0] == -1;
+  std::vector<std::vector<int>> kids(static_cast<size_t>(N));
+  for (int c = 1; c < N && tree_ok; ++c) {
+    const int pa = parent_idx[c];
+    if (pa < 0 || pa >= c)
+      tree_ok = false;
+    else
+      kids[pa].push_back(c);  // index order
+  }
+  parallel_rows(B, threads, [&](int b) {
+    int32_t* path = best_path + size_t(b) * path_cap;
+    auto fail = [&]() {
+      accepted_len[b] = -1;
+      for (int j = 0; j < path_cap; ++j) path[j] = -1;
+      if (next_token) next_token[b] = -1;
+      if (flags) flags[b] = 0;
+    };
+    if (!tree_ok) return fail();
+    const int32_t* tok = node_tokens + size_t(b) * N;
+    const double* u = uniforms + size_t(b) * (N + 1);
+    int32_t flag = 0;
+    std::vector<int> nodes{0};
+    std::vector<double> lp, lq;
+    int cur = 0, emitted = -1;
+    for (;;) {
+      load_row(target, dtype, size_t(b) * N + cur, V, lp);
+      if (!row_valid(lp)) return fail();
+      const Dist pd = transform(lp, T, top_k, top_p);
+      if (pd.topp_margin() < 1e-6) flag |= FLAG_TOPP;
+      int next = -1;
+      if (T == 0.0) {
+        const int g = argmax_lowest(lp);
+        for (int c : kids[cur]) {
+          if (tok[c] < 0 || tok[c] >= V) return fail();
+          if (tok[c] == g) {
+            next = c;
+            break;
+          }
+        }
+        if (next < 0) emitted = g;
+      } else {
+        std::vector<double> r = pd.p;  // the current residual, normalised
+        if (!kids[cur].empty()) {
+          load_row(draft, dtype, size_t(b) * N + cur, V, lq);
+          if (!row_valid(lq)) return fail();
+          const Dist qd = transform(lq, T, top_k, top_p);
+          if (qd.topp_margin() < 1e-6) flag |= FLAG_TOPP;
+          for (int c : kids[cur]) {
+            const int x = tok[c];
+            if (x < 0 || x >= V) return fail();
+            const double px = r[x], qx = qd.p[x];
+            const double ratio = qx > 0.0 ? px / qx : (px > 0.0 ? kInf : 0.0);
+            if (std::fabs(u[c] - ratio) < 1e-5) flag |= FLAG_RATIO;
+            if (u[c] < std::min(1.0, ratio)) {
+              next = c;
+              break;
+            }
+            std::vector<double> rn(static_cast<size_t>(V));
+            double S = 0.0;
+            for (int v = 0; v < V; ++v) {
+              rn[v] = std::max(0.0, r[v] - qd.p[v]);
+              S += rn[v];
+            }
+            if (S > 0.0) {
+              for (int v = 0; v < V; ++v) r[v] = rn[v] / S;
+            }
+          }
+        }
+        if (next < 0) {
+          const Draw d = inverse_cdf(r, u[N]);
+          if (d.flag) flag |= FLAG_CDF;
+          emitted = d.token;
+        }
+      }
+      if (next < 0) break;
+      nodes.push_back(next);
+      cur = next;
+    }
+    const int len = int(nodes.size());
+    if (len > path_cap || emitted < 0) return fail();
+    for (int j = 0; j < path_cap; ++j) path[j] = j < len ? nodes[j] : -1;
+    accepted_len[b] = len;
+    if (next_token) next_token[b] = emitted;
+    if (flags) flags[b] = flag;
+  });
+  return 0;
+}
+
+// The same with float32 uniforms (the library's interface), each widened exactly.
+int oracle_verify_tree_sampling(const void* target, const void* draft, int dtype, int B, int N,
+                                int V, const int32_t* node_tokens, const int32_t* parent_idx,
+                                const float* uniforms, double T, int top_k, double top_p,
+                                int32_t* best_path, int path_cap, int32_t* accepted_len,
+                                int32_t* next_token, int32_t* flags, int threads) {
+  if (!uniforms || B < 0 || N <= 0) return -1;
+  std::vector<double> u(size_t(B) * size_t(N + 1));
+  for (size_t j = 0; j < u.size(); ++j) u[j] = double(uniforms[j]);
+  return oracle_verify_tree_sampling_f64u(target, draft, dtype, B, N, V, node_tokens, parent_idx,
+                                          u.data(), T, top_k, top_p, best_path, path_cap,
+                                          accepted_len, next_token, flags, threads);
+}
+
 // Inverse-CDF draw from norm(max(0, p - q)) (q == NULL: from p) for explicit
 // probability rows. Entries are probabilities: a row holding an entry that is
 // NaN or outside [0, 1], or whose p has no positive entry, gives token -1.

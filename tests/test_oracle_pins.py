@@ -479,6 +479,162 @@ def test_tree_greedy_errors_only_where_the_rule_reads():
     assert nxt[0] == int(np.argmax(l[0, 3])) and nxt[1] == -1 and np.all(path[1] == -1)
 
 
+# --------------------------------------------------------------------------- tree sampling
+
+def _tree_sampling_first_token_law(V, m, temp, top_k, top_p, seed):
+    """Exact law of the first token after the root of one round, the root holding m leaf
+    children whose tokens are drawn independently from q_root: every tuple of child tokens
+    is enumerated, and each acceptance threshold and the final draw's CDF are located by
+    bisection on the oracle's decisions (black box)."""
+    g = np.random.default_rng(seed)
+    t_root = g.normal(0, 1.5, V).astype(np.float32)
+    d_root = g.normal(0, 1.5, V).astype(np.float32)
+    grids = np.meshgrid(*[np.arange(V)] * m, indexing="ij")
+    X = np.stack([x.ravel() for x in grids], axis=1)           # [n, m] child tokens
+    n, N = X.shape[0], m + 1
+    target = np.zeros((n, N, V), np.float32)
+    target[:, 0] = t_root
+    target[:, 1:] = g.normal(0, 1.0, (n, m, V)).astype(np.float32)  # leaf rows (bonus only)
+    draft = np.zeros((n, N, V), np.float32)
+    draft[:, 0] = d_root
+    draft[:, 1:] = 1.0
+    toks = np.concatenate([np.zeros((n, 1), np.int32), X.astype(np.int32)], axis=1)
+    par = np.array([-1] + [0] * m, np.int32)
+    below1 = 1.0 - 2.0 ** -53
+
+    def run(us, w):
+        u = np.zeros((n, N + 1))
+        for j, uj in enumerate(us):
+            u[:, j + 1] = uj
+        u[:, N] = w
+        path, acc, nxt, _ = oracle.verify_tree_sampling(target, draft, toks, par, u, temp,
+                                                        top_k, top_p, threads=1)
+        return path, acc, nxt
+
+    a = np.zeros((n, m))
+    for j in range(m):
+        def not_accepted_at_j(uj, j=j):
+            us = [below1] * j + [uj] + [0.0] * (m - j - 1)
+            path, acc, _ = run(us, 0.5)
+            return ~((acc >= 2) & (path[:, 1] == j + 1))
+        a[:, j] = _bisect(not_accepted_at_j, n)
+    b = np.zeros((n, V + 1))
+    b[:, V] = 1.0
+    for v in range(1, V):
+        b[:, v] = _bisect(lambda w: run([below1] * m, w)[2] >= v, n)
+    draw = np.diff(b, axis=1)
+    q = oracle.transform_rows(d_root[None], temp, top_k, top_p)[0][0]
+    p = oracle.transform_rows(t_root[None], temp, top_k, top_p)[0][0]
+    law = np.zeros(V)
+    for t in range(n):
+        w_t = np.prod(q[X[t]])
+        if w_t == 0.0:
+            continue
+        reach = 1.0
+        for j in range(m):
+            law[X[t, j]] += w_t * reach * a[t, j]
+            reach *= 1.0 - a[t, j]
+        law += w_t * reach * draw[t]
+    return law, p
+
+
+@pytest.mark.parametrize("m,temp,top_k,top_p,seed", [
+    (1, 1.0, 0, 1.0, 0), (2, 1.0, 0, 1.0, 1), (3, 1.0, 0, 1.0, 2), (2, 0.7, 3, 1.0, 3),
+    (2, 1.3, 0, 0.8, 4), (3, 0.9, 3, 0.9, 5)])
+def test_tree_sampling_keeps_the_target_distribution(m, temp, top_k, top_p, seed):
+    """The first emitted token is distributed exactly as the transformed p_root, whatever
+    the number of candidate children drawn from q_root ("Key Components": the rejection
+    rule keeps the original model's output distribution)."""
+    law, p = _tree_sampling_first_token_law(4, m, temp, top_k, top_p, seed)
+    np.testing.assert_allclose(law, p, rtol=0, atol=1e-12)
+
+
+def test_tree_sampling_with_p_equal_q_follows_first_children():
+    g = np.random.default_rng(600)
+    B, N, V = 6, 12, 9
+    par = _random_tree(g, N)
+    t = g.normal(0, 1.5, (B, N, V)).astype(np.float32)
+    toks = g.integers(0, V, (B, N)).astype(np.int32)
+    u = g.random((B, N + 1)).astype(np.float32) * np.float32(0.999)
+    path, acc, nxt, _ = oracle.verify_tree_sampling(t, t, toks, par, u, 1.0)
+    for b in range(B):
+        ref, n_ = [0], 0
+        while True:
+            kids = [c for c in range(1, N) if par[c] == n_]
+            if not kids:
+                break
+            n_ = kids[0]
+            ref.append(n_)
+        assert path[b, :acc[b]].tolist() == ref
+        assert 0 <= nxt[b] < V
+
+
+def test_tree_sampling_at_temperature_zero_is_greedy_tree():
+    """With distinct sibling tokens, only one child can match the argmax: the T = 0 limit
+    walks the same path as greedy tree verification and emits the same next token."""
+    g = np.random.default_rng(700)
+    B, N, V = 10, 16, 40
+    par = _random_tree(g, N)
+    l = g.normal(0, 2.0, (B, N, V)).astype(np.float32)
+    am = np.argmax(l, axis=2)
+    toks = np.zeros((B, N), np.int32)
+    for b in range(B):
+        for pa in range(N):
+            kids = [c for c in range(1, N) if par[c] == pa]
+            vals = g.permutation(V)[:len(kids)]
+            if kids and g.random() < 0.8:
+                vals[g.integers(0, len(kids))] = am[b, pa] if am[b, pa] not in vals else vals[0]
+            for c, v in zip(kids, vals):
+                toks[b, c] = v
+    u = g.random((B, N + 1)).astype(np.float32)
+    path_s, acc_s, nxt_s, _ = oracle.verify_tree_sampling(l, None, toks, par, u, 0.0)
+    path_g, acc_g, nxt_g = oracle.verify_tree_greedy(l, toks, par)
+    assert np.array_equal(acc_s, acc_g) and np.array_equal(path_s, path_g)
+    assert np.array_equal(nxt_s, nxt_g)
+    assert acc_g.max() >= 3
+
+
+@pytest.mark.parametrize("temp,top_k,top_p", [(1.0, 0, 1.0), (0.8, 5, 1.0), (1.2, 0, 0.85)])
+def test_tree_sampling_on_a_path_is_chain_sampling(temp, top_k, top_p):
+    """A tree that is one path verifies like the chain: node c is draft x_(c-1) tested with
+    uniform u[c] against target row c-1 and draft row c-1; the final draw uses u[N] like
+    the chain's u[K]."""
+    g = np.random.default_rng(800)
+    B, K, V = 16, 5, 24
+    target = g.normal(0, 2.0, (B, K + 1, V)).astype(np.float32)
+    dk = (target[:, :K] + g.normal(0, 0.7, (B, K, V))).astype(np.float32)
+    x = draft_tokens(dk, temp, top_k, top_p, g.random((B, K)).astype(np.float32))
+    uc = g.random((B, K + 1)).astype(np.float32)
+    acc_c, out_c, fl_c = oracle.verify_chain(target, dk, x, uc, temp, top_k, top_p)
+    par = np.arange(-1, K, dtype=np.int32)
+    draft = np.concatenate([dk, np.zeros((B, 1, V), np.float32)], axis=1)
+    toks = np.concatenate([np.zeros((B, 1), np.int32), x], axis=1)
+    ut = np.concatenate([np.zeros((B, 1), np.float32), uc], axis=1)   # u[c] = chain u[c-1]
+    path, acc_t, nxt, fl_t = oracle.verify_tree_sampling(target, draft, toks, par, ut, temp,
+                                                         top_k, top_p)
+    assert np.array_equal(acc_t, acc_c + 1)
+    for b in range(B):
+        assert path[b, :acc_t[b]].tolist() == list(range(acc_t[b]))
+        assert nxt[b] == out_c[b, acc_c[b]]
+    assert acc_c.min() == 0 and acc_c.max() >= 2
+
+
+def test_tree_sampling_errors_only_where_the_rule_reads():
+    V = 6
+    par = np.array([-1, 0, 0, 1], np.int32)
+    t = np.zeros((2, 4, V), np.float32)
+    d = np.zeros((2, 4, V), np.float32)
+    t[:, 2, :] = np.nan              # node 2's target row: never read (node 2 has no child,
+    d[:, 2, :] = np.nan              # and is not on an accepted path here)
+    d[:, 3, :] = np.nan              # node 3 is a leaf: its draft row is never read
+    toks = np.array([[0, 1, 2, 3], [0, 1, 2, 3]], np.int32)
+    u = np.zeros((2, 5), np.float32)           # u = 0: every tested child is accepted
+    d[1, 1, 0] = np.inf              # batch row 1: node 1's draft row is read (node 3 is its child)
+    path, acc, nxt, _ = oracle.verify_tree_sampling(t, d, toks, par, u, 1.0)
+    assert acc.tolist() == [3, -1] and path[0, :3].tolist() == [0, 1, 3]
+    assert nxt[1] == -1 and np.all(path[1] == -1)
+
+
 def test_tree_workload_structure_and_invalid_parent():
     par, depth, rank = specgen.tree_structure((4, 3, 2, 2), 64)
     assert np.bincount(depth).tolist() == [1, 4, 12, 24, 23]
