@@ -46,6 +46,8 @@ def _declare(lib):
         "spec_verify_chain_noalloc": ([P, P, I, I, I, I, P, P, F, I, F, P, P, P], I),
         "spec_verify_tree_typical": ([P, I, I, I, I, P, P, F, F, P, I, P, P, Z, P], I),
         "spec_verify_tree_greedy": ([P, I, I, I, I, P, P, P, I, P, P, P, Z, P], I),
+        "spec_verify_tree_sampling": ([P, P, I, I, I, I, P, P, P, F, I, F, P, I, P, P, P, Z, P],
+                                      I),
         "spec_logits_to_probs": ([P, I, I, I, F, I, F, P, P, P], I),
         "spec_residual_sample": ([P, P, I, I, P, P, P], I),
         "spec_get_device_status": ([P, P, P], I),
@@ -223,6 +225,39 @@ def spec_verify_tree_greedy(target_logits, node_tokens, parent_idx, path_cap=Non
         _ptr(t), _dtype(t), B, N, V, _ptr(nt), _ptr(par), _ptr(best_path), cap,
         _ptr(accepted_len), _ptr(next_token), _ptr(workspace),
         workspace.numel() * workspace.element_size(), _stream(stream, t.device)))
+    return best_path, accepted_len, next_token
+
+
+def spec_verify_tree_sampling(target_logits, draft_logits, node_tokens, parent_idx, uniforms,
+                              temp, top_k=0, top_p=1.0, path_cap=None, best_path=None,
+                              accepted_len=None, next_token=None, workspace=None, stream=None):
+    """Rejection sampling over a candidate tree. target and draft [B,N,V] (draft None when
+    temp == 0), node_tokens int32 [B,N], parent_idx int32 [N], uniforms float32 [B,N+1].
+    Returns (best_path [B,path_cap], accepted_len [B], next_token [B])."""
+    t = _dev(target_logits, "target_logits")
+    B, N, V = t.shape
+    d = None if draft_logits is None else _dev(draft_logits, "draft_logits", t.dtype)
+    if d is not None and tuple(d.shape) != (B, N, V):
+        raise ValueError("draft_logits must be [B, N, V]")
+    nt = _dev(node_tokens, "node_tokens", torch.int32)
+    par = _dev(parent_idx, "parent_idx", torch.int32)
+    u = _dev(uniforms, "uniforms", torch.float32)
+    if tuple(nt.shape) != (B, N) or tuple(par.shape) != (N,) or tuple(u.shape) != (B, N + 1):
+        raise ValueError("node_tokens must be [B, N], parent_idx [N] and uniforms [B, N+1]")
+    cap = N if path_cap is None else int(path_cap)
+    if best_path is None:
+        best_path = torch.empty((B, cap), dtype=torch.int32, device=t.device)
+    if accepted_len is None:
+        accepted_len = torch.empty(B, dtype=torch.int32, device=t.device)
+    if next_token is None:
+        next_token = torch.empty(B, dtype=torch.int32, device=t.device)
+    if workspace is None:
+        workspace = torch.empty(spec_workspace_size(B, N, V), dtype=torch.uint8, device=t.device)
+    _check("spec_verify_tree_sampling", lib().spec_verify_tree_sampling(
+        _ptr(t), _ptr(d), _dtype(t), B, N, V, _ptr(nt), _ptr(par), _ptr(u), float(temp),
+        int(top_k), float(top_p), _ptr(best_path), cap, _ptr(accepted_len), _ptr(next_token),
+        _ptr(workspace), workspace.numel() * workspace.element_size(),
+        _stream(stream, t.device)))
     return best_path, accepted_len, next_token
 
 

@@ -13,6 +13,7 @@
 #include "specverify.h"
 #include "stream.cuh"
 #include "tree.cuh"
+#include "tree_sample.cuh"
 
 namespace {
 
@@ -426,6 +427,89 @@ spec_status spec_verify_tree_greedy(const void* target_logits, spec_dtype dtype,
                      stream);
 }
 
+spec_status spec_verify_tree_sampling(const void* target_logits, const void* draft_logits,
+                                      spec_dtype dtype, int B, int N, int V,
+                                      const int32_t* node_tokens, const int32_t* parent_idx,
+                                      const float* uniforms, float temp, int top_k, float top_p,
+                                      int32_t* best_path, int path_cap, int32_t* accepted_len,
+                                      int32_t* next_token, void* workspace,
+                                      size_t workspace_bytes, void* stream) {
+  const bool greedy = temp == 0.0f;
+  if (!target_logits || (!greedy && !draft_logits) || !dtype_ok(dtype) || B <= 0 || N <= 0 ||
+      V <= 0 || !node_tokens || !parent_idx || !uniforms || !best_path || path_cap <= 0 ||
+      !accepted_len || !std::isfinite(temp) || temp < 0.0f || !(top_p > 0.0f))
+    return SPEC_ERR_INVALID_ARG;
+  if (V > SPEC_MAX_VOCAB || N > SPEC_MAX_TREE_NODES) return SPEC_ERR_UNSUPPORTED;
+  const long long rows = (long long)B * N * (greedy ? 1 : 2);
+  if (!workspace || !aligned16(workspace) || workspace_bytes < stats_bytes(rows))
+    return SPEC_ERR_WORKSPACE;
+  RowPlan pl;
+  if (!plan_rows(V, elem_bytes(dtype), &pl) || !rows_fit(rows, pl.C) || B > 0x7fffffff)
+    return SPEC_ERR_UNSUPPORTED;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int32_t* dev_status = static_cast<int32_t*>(workspace);
+  const WsLayout wl = ws_layout(rows);
+  char* ws = static_cast<char*>(workspace);
+  sv::RowStats* stats = reinterpret_cast<sv::RowStats*>(ws + wl.stats);
+  if (cudaMemsetAsync(dev_status, 0, 2 * sizeof(int32_t), s) != cudaSuccess) return SPEC_ERR_CUDA;
+
+  sv::RowJob rj = {};
+  rj.kept_n = reinterpret_cast<int32_t*>(ws + wl.kept_n);
+  rj.kept_ids = reinterpret_cast<int32_t*>(ws + wl.kept_ids);
+  rj.base0 = target_logits;
+  rj.base1 = draft_logits;
+  rj.rows0 = (long long)B * N;
+  rj.rows = rows;
+  rj.V = V;
+  rj.slice = pl.slice;
+  rj.slice_bytes = pl.slice_bytes;
+  rj.c = greedy ? 0.0f : sv::kLog2e / temp;
+  rj.inv_t = greedy ? 0.0f : 1.0f / temp;
+  rj.top_k = (top_k >= 1 && top_k < V) ? top_k : 0;
+  rj.top_p = top_p < 1.0f ? top_p : 1.0f;
+  rj.flags = greedy ? sv::RS_GREEDY : 0;
+  rj.stats = stats;
+  rj.dev_status = dev_status;
+  void* evb = g_ev_before.load();
+  void* eva = g_ev_after.load();
+  if (evb) cudaEventRecord(static_cast<cudaEvent_t>(evb), s);
+  if (row_stage(dtype, rj, pl, reinterpret_cast<int32_t*>(ws + wl.fb_rows), dev_status + 1, s) !=
+      cudaSuccess)
+    return SPEC_ERR_CUDA;
+  if (eva) cudaEventRecord(static_cast<cudaEvent_t>(eva), s);
+
+  sv::TreeSampleJob tj = {};
+  tj.target = target_logits;
+  tj.draft = draft_logits;
+  tj.B = B;
+  tj.N = N;
+  tj.V = V;
+  tj.tokens = node_tokens;
+  tj.parent = parent_idx;
+  tj.uniforms = uniforms;
+  tj.stats = stats;
+  tj.kept_n = rj.kept_n;
+  tj.kept_ids = rj.kept_ids;
+  tj.greedy = greedy ? 1 : 0;
+  tj.best_path = best_path;
+  tj.path_cap = path_cap;
+  tj.accepted_len = accepted_len;
+  tj.next_token = next_token;
+  const size_t dyn = size_t(N) * 16 + 16;  // child lists, path, normalisers
+  cudaError_t e;
+  if (dtype == SPEC_BF16) {
+    e = cudaFuncSetAttribute(sv::tree_sample_kernel<__nv_bfloat16>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, int(dyn));
+    if (e == cudaSuccess) sv::tree_sample_kernel<__nv_bfloat16><<<B, kThreads, dyn, s>>>(tj);
+  } else {
+    e = cudaFuncSetAttribute(sv::tree_sample_kernel<float>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, int(dyn));
+    if (e == cudaSuccess) sv::tree_sample_kernel<float><<<B, kThreads, dyn, s>>>(tj);
+  }
+  if (e != cudaSuccess) return SPEC_ERR_CUDA;
+  return check_launch(cudaGetLastError());
+}
+
 spec_status spec_logits_to_probs(const void* logits, spec_dtype dtype, int rows, int V,
                                  float temp, int top_k, float top_p, float* probs,
                                  float* entropy, void* stream) {
@@ -487,6 +571,7 @@ int spec_kernels_per_call(const char* entry_point) {
   if (!std::strcmp(entry_point, "spec_verify_chain")) return 3;
   if (!std::strcmp(entry_point, "spec_verify_tree_typical")) return 2;
   if (!std::strcmp(entry_point, "spec_verify_tree_greedy")) return 2;
+  if (!std::strcmp(entry_point, "spec_verify_tree_sampling")) return 3;
   if (!std::strcmp(entry_point, "spec_logits_to_probs")) return 1;
   if (!std::strcmp(entry_point, "spec_residual_sample")) return 1;
   return -1;

@@ -71,8 +71,8 @@ typedef enum { SPEC_F32 = 0, SPEC_BF16 = 1 } spec_dtype;
 const char* spec_status_string(int status);
 
 /* Bytes of workspace that spec_verify_chain(B, K, V), spec_verify_tree_typical(B,
- * N = K_or_N, V) and spec_verify_tree_greedy(B, N, V) need; each call accepts any
- * workspace at least this large. The
+ * N = K_or_N, V), spec_verify_tree_greedy(B, N, V) and spec_verify_tree_sampling(B, N, V)
+ * need; each call accepts any workspace at least this large. The
  * workspace must be 16-byte aligned. Returns 0 for invalid sizes. */
 size_t spec_workspace_size(int B, int K_or_N, int V);
 
@@ -140,6 +140,34 @@ spec_status spec_verify_tree_greedy(const void* target_logits, spec_dtype dtype,
                                     int32_t* best_path, int path_cap, int32_t* accepted_len,
                                     int32_t* next_token, void* workspace, size_t workspace_bytes,
                                     void* stream);
+
+/* Rejection sampling over a candidate tree — [SD] "Key Components" (MEDUSA's step (3)
+ * may reuse the rejection rule of speculative sampling, which keeps the target's output
+ * distribution), with the rule of "Speculative Decoding" / "Speculative Sampling".
+ *   target_logits [B][N][V]: row n = the target's scores after node n (p_n).
+ *   draft_logits  [B][N][V]: row n = the drafter's scores after node n (q_n); the
+ *                  children of n carry tokens drawn independently from q_n. NULL allowed
+ *                  iff temp == 0.
+ *   node_tokens, parent_idx, best_path, path_cap, accepted_len: as
+ *                  spec_verify_tree_typical; next_token [B] out or NULL: the token emitted
+ *                  after the path.
+ *   uniforms      [B][N+1] float in [0,1): u[c] tests child c (u[0] unused), u[N] is the
+ *                  final draw.
+ * From the root, at the current node n the children are tried in index order: child c
+ * is accepted iff u[c] < min(1, r(x_c)/q_n(x_c)), r the current residual (p_n at first);
+ * a rejection replaces r by norm(max(0, r - q_n)) (unchanged if that is empty). An
+ * accepted child becomes the current node; when none is accepted the emitted token is
+ * drawn from r with u[N] (the inverse CDF of spec_verify_chain). temp, top_k, top_p
+ * transform p and q as in spec_verify_chain; temp == 0 accepts the first child whose
+ * token is the argmax of p_n and emits that argmax. The draws and tests read only the
+ * rows on the walked path. 1 <= N <= SPEC_MAX_TREE_NODES. */
+spec_status spec_verify_tree_sampling(const void* target_logits, const void* draft_logits,
+                                      spec_dtype dtype, int B, int N, int V,
+                                      const int32_t* node_tokens, const int32_t* parent_idx,
+                                      const float* uniforms, float temp, int top_k, float top_p,
+                                      int32_t* best_path, int path_cap, int32_t* accepted_len,
+                                      int32_t* next_token, void* workspace,
+                                      size_t workspace_bytes, void* stream);
 
 /* The sampling transform alone — [SD] "Speculative Sampling" (last bullet).
  *   logits [rows][V]; probs [rows][V] float out: the transformed distribution

@@ -323,6 +323,98 @@ def test_tree_greedy_invalid_inputs():
     assert np.all(plen.cpu().numpy() == -1) and np.all(nxt.cpu().numpy() == -1)
 
 
+# ------------------------------------------------------------------ tree rejection sampling
+
+def _tree_children_from_q(g, draft, par, temp, top_k, top_p):
+    """Node tokens: each child drawn from the transformed draft distribution of its parent
+    (independently), the way a drafter proposes them."""
+    B, N, V = draft.shape
+    q = oracle.transform_rows(draft, temp, top_k, top_p)[0].reshape(B, N, V)
+    toks = np.zeros((B, N), np.int32)
+    for b in range(B):
+        for c in range(1, N):
+            pr = q[b, par[c]]
+            toks[b, c] = g.choice(V, p=pr / pr.sum())
+    return toks
+
+
+def assert_tree_sampling_parity(target, draft, toks, par, u, temp, top_k=0, top_p=1.0,
+                                path_cap=None, flag_budget=20):
+    path_g, len_g, nxt_g = sv.spec_verify_tree_sampling(
+        dev(target), None if draft is None else dev(draft), dev(toks), dev(par), dev(u), temp,
+        top_k, top_p, path_cap=path_cap)
+    torch.cuda.synchronize()
+    path_r, len_r, nxt_r, flags = oracle.verify_tree_sampling(target, draft, toks, par, u, temp,
+                                                              top_k, top_p, path_cap=path_cap)
+    len_g, path_g, nxt_g = len_g.cpu().numpy(), path_g.cpu().numpy(), nxt_g.cpu().numpy()
+    ok = (flags & oracle.PARITY_FLAGS) == 0
+    same = (len_g == len_r) & np.all(path_g == path_r, axis=1) & (nxt_g == nxt_r)
+    bad = np.nonzero(~same & ok)[0]
+    assert bad.size == 0, (bad[:5], len_g[bad[:5]], len_r[bad[:5]], nxt_g[bad[:5]], nxt_r[bad[:5]])
+    # a flag marks a decision inside the fp32/fp64 window (a draw on a token holding under
+    # 1e-6 of the mass, a ratio within 1e-5 of its uniform)
+    assert (~ok).sum() <= max(1, len(ok) // flag_budget), (~ok).sum()
+    return len_r
+
+
+@pytest.mark.parametrize("dtype,V,temp,top_k,top_p", [
+    ("bf16", 32000, 1.0, 0, 1.0), ("f32", 1000, 0.8, 20, 1.0), ("bf16", 151936, 0.8, 50, 1.0),
+    ("bf16", 4099, 1.2, 0, 0.9), ("f32", 17, 1.0, 0, 1.0), ("bf16", 32000, 0.0, 0, 1.0),
+    ("bf16", 32000, 0.9, 40, 0.8)])
+def test_tree_sampling_random(dtype, V, temp, top_k, top_p):
+    g = np.random.default_rng(V + int(temp * 10) + top_k)
+    B, N = 8, 24
+    par = np.array([-1] + [int(g.integers(max(0, c - 4), c)) for c in range(1, N)], np.int32)
+    t = g.normal(0, 2.0, (B, N, V)).astype(np.float32)
+    d = (t + g.normal(0, 0.8, (B, N, V))).astype(np.float32)
+    to = (lambda a: a) if dtype == "f32" else specgen.f32_to_bf16_bits
+    target, draft = to(t), to(d)
+    if temp > 0:
+        toks = _tree_children_from_q(g, draft, par, temp, top_k, top_p)
+    else:  # greedy limit: children mostly on the parent's argmax
+        lf = t if dtype == "f32" else specgen.bf16_bits_to_f32(target)
+        toks = _greedy_tree_tokens(g, lf, par, 0.7)
+    u = (g.integers(0, 1 << 24, (B, N + 1)) / float(1 << 24)).astype(np.float32)
+    lens = assert_tree_sampling_parity(target, None if temp == 0 else draft, toks, par, u, temp,
+                                       top_k, top_p)
+    assert lens.max() >= 2
+    assert_tree_sampling_parity(target, None if temp == 0 else draft, toks, par, u, temp,
+                                top_k, top_p, path_cap=2)
+
+
+def test_tree_sampling_workload_shape():
+    """The 32 x 64-node tree shape at V=32000 (bfloat16), children drawn from the drafter."""
+    cfg = specgen.CFG4
+    par, _, _ = specgen.tree_structure(cfg.heads, cfg.N)
+    g = np.random.default_rng(11)
+    B, N, V = cfg.B, cfg.N, cfg.V
+    prior = -1.1 * np.log1p(np.arange(V))          # the Zipf log-prior of the chain workloads
+    t = (g.normal(0, 3.0, (B, N, V)) + prior).astype(np.float32)
+    d = (t + g.normal(0, 1.0, (B, N, V))).astype(np.float32)
+    target, draft = specgen.f32_to_bf16_bits(t), specgen.f32_to_bf16_bits(d)
+    toks = _tree_children_from_q(g, draft, par, 1.0, 0, 1.0)
+    u = (g.integers(0, 1 << 24, (B, N + 1)) / float(1 << 24)).astype(np.float32)
+    lens = assert_tree_sampling_parity(target, draft, toks, par, u, 1.0, flag_budget=8)
+    assert lens.max() >= 3
+
+
+def test_tree_sampling_invalid_inputs():
+    B, N, V = 3, 5, 20
+    t = np.zeros((B, N, V), np.float32)
+    d = np.zeros((B, N, V), np.float32)
+    toks = np.zeros((B, N), np.int32)
+    par = np.array([-1, 0, 0, 1, 3], np.int32)
+    u = np.zeros((B, N + 1), np.float32)   # every tested child accepted
+    d[1, 1, 3] = np.nan                    # read: node 1 is accepted and has a child
+    toks[2, 1] = 99                        # out of range, tested first at the root
+    lens = assert_tree_sampling_parity(t, d, toks, par, u, 1.0)
+    assert lens.tolist() == [4, -1, -1]
+    bad_par = np.array([-1, 0, 3, 1, 1], np.int32)
+    path, plen, nxt = sv.spec_verify_tree_sampling(dev(t), dev(d), dev(toks), dev(bad_par),
+                                                   dev(u), 1.0)
+    assert np.all(plen.cpu().numpy() == -1) and np.all(nxt.cpu().numpy() == -1)
+
+
 # ------------------------------------------------------------------ transform and residual draw
 
 @pytest.mark.parametrize("dtype,V", [("bf16", 32000), ("f32", 1000), ("bf16", 128256), ("f32", 40000),
