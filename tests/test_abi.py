@@ -90,6 +90,45 @@ def test_tree_invalid_args(lib):
     assert f(*args) == -4
 
 
+def test_tree_greedy_invalid_args(lib):
+    f = lib.spec_verify_tree_greedy
+    ok = [P(16), 1, 2, 8, 100, P(16), P(16), P(16), 8, P(16), P(16), P(256), 1 << 20, None]
+    for i, v in [(0, None), (1, 7), (2, 0), (3, 0), (4, 0), (5, None), (6, None), (7, None),
+                 (8, 0), (9, None)]:
+        args = list(ok)
+        args[i] = v
+        assert f(*args) == -1, i
+    args = list(ok)
+    args[3] = 5000
+    assert f(*args) == -2
+    args = list(ok)
+    args[12] = 10
+    assert f(*args) == -4
+
+
+def test_tree_sampling_invalid_args(lib):
+    f = lib.spec_verify_tree_sampling
+    ok = [P(16), P(16), 1, 2, 8, 100, P(16), P(16), P(16), 1.0, 0, 1.0, P(16), 8, P(16), P(16),
+          P(256), 1 << 20, None]
+    for i, v in [(0, None), (1, None), (2, 7), (3, 0), (4, 0), (5, 0), (6, None), (7, None),
+                 (8, None), (9, -1.0), (9, float("nan")), (11, 0.0), (12, None), (13, 0),
+                 (14, None)]:
+        args = list(ok)
+        args[i] = v
+        assert f(*args) == -1, i
+    args = list(ok)
+    args[1] = None
+    args[9] = 0.0          # the greedy limit needs no draft logits: passes the host checks
+    args[16] = None        # (and then stops at the missing workspace)
+    assert f(*args) == -4
+    args = list(ok)
+    args[4] = 5000
+    assert f(*args) == -2
+    args = list(ok)
+    args[17] = 10
+    assert f(*args) == -4
+
+
 def test_probs_and_residual_invalid_args(lib):
     assert lib.spec_logits_to_probs(None, 1, 4, 10, 1.0, 0, 1.0, P(16), None, None) == -1
     assert lib.spec_logits_to_probs(P(16), 1, 4, 10, 1.0, 0, 0.0, P(16), None, None) == -1
