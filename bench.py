@@ -253,6 +253,7 @@ def run_ours(args, cfg, greedy, rank, world):
     row_avg_ms = float(np.mean(row_ms))
     alg = algorithmic_bytes(cfg, greedy)
     peaks, peak_src = measured_peaks()
+    traffic = read_profile_traffic(workload(cfg, greedy)["workload"])
     achieved = alg / (row_avg_ms / 1e3) / 1e9
     return {
         "value": value, "ms_per_step": ms_max / args.steps,
@@ -263,13 +264,19 @@ def run_ours(args, cfg, greedy, rank, world):
                      "frac_of_8TBs": round(achieved / 8000.0, 4),
                      "kernel": "stream_rows_kernel", "kernel_ms": round(row_avg_ms, 4),
                      "algorithmic_bytes": alg,
-                     "traffic": read_profile_traffic(workload(cfg, greedy)["workload"])},
+                     "traffic": traffic},
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": int(h2d),
                 "d2h_bytes_per_step": int(d2h), "steps": e2e_steps},
         "gpu_launches": kernels_per_step * args.steps,
         "clocks": clock_info,
         "acceptance": {"mean_accepted_len": float(accl.mean()),
-                       "emitted_per_round": float(accl.mean() + 1)},
+                       "emitted_per_round": float(accl.mean() + 1),
+                       "histogram": np.bincount(accl, minlength=cfg.K + 1).tolist()},
+        # one read of every logit row, per verified draft position (the minimum the step
+        # must move), and what the row kernel's counted DRAM traffic gives per position
+        "bytes_per_position": {"algorithmic": alg / (cfg.B * cfg.K),
+                               "counted": (None if traffic is None
+                                           else traffic / (cfg.B * cfg.K))},
     }
 
 
