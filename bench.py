@@ -58,17 +58,23 @@ def measured_peaks():
         return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}, "fallback"
 
 
+def kernel_code(src: str) -> str:
+    """The source without its // comments and blank lines: what the counters depend on."""
+    lines = (ln.split("//", 1)[0].rstrip() for ln in src.splitlines())
+    return "\n".join(ln for ln in lines if ln.strip())
+
+
 def read_profile_traffic(name: str):
     """Per-launch DRAM traffic (read + write bytes) of the row-statistics kernel for this
-    workload, from the committed ncu summary; None if there is none or the kernel source
-    has changed since the counters were taken."""
+    workload, from the committed ncu summary; None if there is none or the kernel code
+    (comments aside) has changed since the counters were taken."""
     import hashlib
     try:
         with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
             rec = json.load(f)
         with open(os.path.join(ROOT, "draft_token_verification_spec_b200", "csrc",
-                               "stream.cuh"), "rb") as f:
-            sha = hashlib.sha256(f.read()).hexdigest()[:16]
+                               "stream.cuh")) as f:
+            sha = hashlib.sha256(kernel_code(f.read()).encode()).hexdigest()[:16]
     except (OSError, ValueError):
         return None
     if rec.get("stream_cuh_sha256_16") != sha:
