@@ -76,6 +76,11 @@ struct Elem<float> {
     return __ldg(static_cast<const float*>(base) + i);
   }
   __device__ static __forceinline__ uint32_t key(float x) { return f32_key(x); }
+  // Key of entry k of a 16-byte vector, from its bits.
+  __device__ static __forceinline__ uint32_t key_at(const uint4& w, int k) {
+    const uint32_t b = k < 2 ? (k == 0 ? w.x : w.y) : (k == 2 ? w.z : w.w);
+    return f32_key(__uint_as_float(b));
+  }
   // Largest value of a 16-byte vector; NaN if any entry is NaN.
   __device__ static __forceinline__ float vmax_nan(const uint4& w) {
     return fmax_nan(fmax_nan(__uint_as_float(w.x), __uint_as_float(w.y)),
@@ -106,6 +111,14 @@ struct Elem<__nv_bfloat16> {
     return __uint_as_float(uint32_t(h) << 16);
   }
   __device__ static __forceinline__ uint32_t key(float x) { return f32_key(x) >> 16; }
+  // Key of entry k of a 16-byte vector, from its 16 bits (-0 maps to the key of +0).
+  __device__ static __forceinline__ uint32_t key_at(const uint4& w, int k) {
+    const int q = k >> 1;
+    const uint32_t b = q < 2 ? (q == 0 ? w.x : w.y) : (q == 2 ? w.z : w.w);
+    uint32_t h = (k & 1) ? (b >> 16) : (b & 0xFFFFu);
+    if (h == 0x8000u) h = 0u;
+    return (h & 0x8000u) ? (~h & 0xFFFFu) : (h | 0x8000u);
+  }
   __device__ static __forceinline__ __nv_bfloat162 pair(uint32_t u) {
     return *reinterpret_cast<const __nv_bfloat162*>(&u);
   }

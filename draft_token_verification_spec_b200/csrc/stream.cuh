@@ -9,8 +9,8 @@
 // themselves only with named barrier 1, so the producer is never held up by their row-end
 // work. Nothing is shared between CTAs.
 //
-// Per chunk each consumer thread takes eight (greedy, sums) or four (candidate modes)
-// 16-byte vectors and updates, as the mode needs:
+// Per chunk each consumer thread takes eight 16-byte vectors and updates, as the mode
+// needs:
 //   SM_GREEDY  its running maximum (packed bf16x2 max, NaN propagating) and the lowest index
 //              holding it;
 //   SM_SUMS    an online softmax sum (and entropy term), rescaled when its maximum grows;
@@ -60,9 +60,9 @@
 
 namespace sv {
 
-// Ring of chunk buffers per CTA. Greedy and plain sums (three CTAs per SM) stream two
-// 32 KB chunks; the candidate modes (two CTAs per SM, with an exchange every few chunks)
-// four 16 KB chunks, so more copies are in flight while the consumers synchronise.
+// Ring of chunk buffers per CTA: two 32 KB chunks, in every mode (three CTAs per SM for
+// greedy and plain sums; two for the candidate modes, whose list and histogram take the
+// rest of the shared memory). The depth and chunk size of each kind are build-time knobs.
 #ifndef SV_RING_NBUF_PLAIN
 #define SV_RING_NBUF_PLAIN 2
 #endif
@@ -70,10 +70,10 @@ namespace sv {
 #define SV_RING_KB_PLAIN 32
 #endif
 #ifndef SV_RING_NBUF_CAND
-#define SV_RING_NBUF_CAND 4
+#define SV_RING_NBUF_CAND 2
 #endif
 #ifndef SV_RING_KB_CAND
-#define SV_RING_KB_CAND 16
+#define SV_RING_KB_CAND 32
 #endif
 constexpr int kMaxRing = 4;
 
@@ -755,16 +755,11 @@ __global__ void __launch_bounds__(kStreamThreads, (kMode <= SM_SUMS ? 3 : 2))
         int pos = __shfl_sync(0xffffffffu, wbase, 31) + inc - my;
 #pragma unroll
         for (int u = 0; u < kVecPerThread; ++u) {
-          if (!cm[u]) continue;
-          float x[P];
-          Elem<T>::unpack(w[u], x);
           const int j0 = base + (16 * (u * kThreads + int(threadIdx.x)) - s.pad) / E;
-#pragma unroll
-          for (int k = 0; k < P; ++k) {
-            if (cm[u] & (1u << k)) {
-              if (pos < kCap) cs.cand[pos] = make_comp(Elem<T>::key(x[k]), j0 + k);
-              ++pos;
-            }
+          for (uint32_t m = cm[u]; m != 0; m &= m - 1) {  // the set bits only
+            const int k = __ffs(m) - 1;
+            if (pos < kCap) cs.cand[pos] = make_comp(Elem<T>::key_at(w[u], k), j0 + k);
+            ++pos;
           }
         }
       }
