@@ -510,12 +510,16 @@ struct RowAcc {
   }
 
   // One 16-byte vector whose first element has row index j0 (entries outside the chunk
-  // hold -inf). vm = its largest value.
-  __device__ __forceinline__ void vec(const uint4& w, float vm, int j0, float c, bool want_ent) {
+  // hold -inf). vm = its largest value. Top-p: returns the mask of its entries >= t, from
+  // the values the sums unpacked (0 in the other modes).
+  __device__ __forceinline__ uint32_t vec(const uint4& w, float vm, int j0, float c,
+                                          bool want_ent, float t) {
     constexpr int P = Elem<T>::kPerVec;
+    uint32_t cm = 0;
     if (!(vm > -INFINITY)) {  // all -inf (weight 0), or a NaN
       mt = fmax_nan(mt, vm);
-      return;
+      if (kMode == SM_TOPP && vm >= t) cm = (1u << P) - 1u;  // all -inf, and t = -inf
+      return cm;
     }
     if constexpr (kMode == SM_GREEDY) {
       if (vm > mt) {  // later vectors hold higher indices: strict > keeps the lowest
@@ -541,8 +545,14 @@ struct RowAcc {
         }
         s += s2;
       }
+      if (kMode == SM_TOPP && vm >= t) {
+#pragma unroll
+        for (int k = 0; k < P; ++k)
+          if (x[k] >= t) cm |= 1u << k;
+      }
     }
     mt = fmax_nan(mt, vm);
+    return cm;
   }
 
   // One element outside the vector path (chunk head or tail), row index j.
@@ -718,11 +728,10 @@ __global__ void __launch_bounds__(kStreamThreads, (kMode <= SM_SUMS ? 3 : 2))
     for (int u = 0; u < kVecPerThread; ++u) {
       const int v = u * kThreads + int(threadIdx.x);
       const int j0 = base + (16 * v - s.pad) / E;
-      st.vec(w[u], vm[u], j0, c, want_ent);
-      cm[u] = 0;
+      cm[u] = st.vec(w[u], vm[u], j0, c, want_ent, (v >= v_lo && v < v_hi) ? thr : INFINITY);
       vmax4 = fmaxf(vmax4, vm[u]);  // pad vectors hold -inf; NaN never passes a filter
     }
-    if constexpr (kCand) {
+    if constexpr (kMode == SM_TOPK) {
       if (vmax4 >= thr) {
 #pragma unroll
         for (int u = 0; u < kVecPerThread; ++u) {
