@@ -9,13 +9,14 @@
 // themselves only with named barrier 1, so the producer is never held up by their row-end
 // work. Nothing is shared between CTAs.
 //
-// Per chunk each consumer thread takes eight 16-byte vectors and updates, as the mode
-// needs:
+// Per chunk each consumer thread takes eight (top-k: seven) 16-byte vectors and updates,
+// as the mode needs:
 //   SM_GREEDY  its running maximum (packed bf16x2 max, NaN propagating) and the lowest index
 //              holding it;
 //   SM_SUMS    an online softmax sum (and entropy term), rescaled when its maximum grows;
 //   SM_TOPK    the running maximum, and appends the entries >= a threshold to the CTA's
-//              candidate list (warp-aggregated: one shared atomic per warp);
+//              candidate list (warp-aggregated: one shared atomic per warp, then each lane
+//              writes only the set bits of its vectors' masks);
 //   SM_TOPP    the online sum and the candidate list.
 // Candidates are 64-bit composites (key << 32 | ~id): the order of composites is the order
 // (value desc, id asc) that top-k and top-p use, so the k-th candidate is unique.
@@ -23,9 +24,9 @@
 // Top-k: the first threshold is a value that k entries of the first chunk reach (per-warp
 // order statistics of per-thread maxima). After the first chunk the consumer warps exchange
 // their counts once, and a list of more than 2k entries sets the threshold to the exact
-// k-th of the chunk (ranked directly, the list kept as it is; longer lists are cut over
-// log-weight bins). Later chunks of usual rows rarely reach it; no further exchange runs,
-// and a list that still overflows sends the row to the exact finisher.
+// k-th of the chunk (ranked directly, the list kept as it is). Later chunks of usual rows
+// rarely reach it; no further exchange runs, and a list that outgrows kCapTopK sends the row
+// to the exact finisher. The short list keeps a top-k CTA small enough for three per SM.
 //
 // Top-p: the threshold starts at (first-chunk maximum - T ln(V / (1 - top_p))), below
 // which the whole row holds less than 1 - top_p of the mass, raised to the smallest of
@@ -37,16 +38,16 @@
 // far (about kKeepTarget candidates at the row end for rows whose values do not drift
 // along the vocabulary).
 //
-// At the end of a row the CTA selects among the candidates. Top-k lists of at most
-// kRankMax entries are ranked directly (each candidate counts the larger composites; the
-// top-p crossing within the top k accumulates their weights the same way). Other lists go
-// over a histogram of log-weight bins (1/32 of a log2 unit each, relative to the row
-// maximum; bins only coarsen the order, they never reorder it): the bin where the count
-// (top-k) or mass (top-p) crosses the target, then the exact crossing candidate among that
-// bin's members. It writes the RowStats record (and the kept ids of top-k rows). Rows the
-// candidates cannot settle (list overflow, too many members in the crossing bin, or
-// candidates holding less than top_p of the mass) are marked ROW_FALLBACK and listed; the
-// cluster kernel (row_stats.cuh) then finishes them exactly.
+// At the end of a row the CTA selects among the candidates. Top-k lists are ranked directly
+// (each candidate counts the larger composites); with top-p as well, the top k go to their
+// rank slots and a block scan of their weights finds the crossing. Top-p lists go over a
+// histogram of log-weight bins (1/32 of a log2 unit each, relative to the row maximum; bins
+// only coarsen the order, they never reorder it): the bin where the mass crosses the
+// target, then the exact crossing candidate among that bin's members. It writes the
+// RowStats record (and the kept ids of top-k rows). Rows the candidates cannot settle (list
+// overflow, too many members in the crossing bin, or candidates holding less than top_p of
+// the mass) are marked ROW_FALLBACK and listed; the cluster kernel (row_stats.cuh) then
+// finishes them exactly.
 //
 // This is the sampling transform of "Speculative Sampling" (spec-decoding-i notes, last
 // bullet: transform the probabilities first, then apply the rejection scheme), the argmax
@@ -60,9 +61,11 @@
 
 namespace sv {
 
-// Ring of chunk buffers per CTA: two 32 KB chunks, in every mode (three CTAs per SM for
-// greedy and plain sums; two for the candidate modes, whose list and histogram take the
-// rest of the shared memory). The depth and chunk size of each kind are build-time knobs.
+// Ring of chunk buffers per CTA: two chunks in every mode. Greedy and plain sums stream
+// 32 KB chunks at three CTAs per SM; top-k 28 KB chunks at three CTAs per SM (its list of
+// kCapTopK candidates and the top k in rank order fill the rest); top-p 32 KB chunks at two
+// CTAs per SM (its larger list and the log-weight histogram take the rest). The depth and
+// chunk size of each kind are build-time knobs.
 #ifndef SV_RING_NBUF_PLAIN
 #define SV_RING_NBUF_PLAIN 2
 #endif
@@ -75,6 +78,9 @@ namespace sv {
 #ifndef SV_RING_KB_CAND
 #define SV_RING_KB_CAND 32
 #endif
+#ifndef SV_RING_KB_TOPK
+#define SV_RING_KB_TOPK 28
+#endif
 constexpr int kMaxRing = 4;
 
 enum : int { SM_GREEDY = 0, SM_SUMS = 1, SM_TOPK = 2, SM_TOPP = 3 };
@@ -82,7 +88,9 @@ enum : int { SM_GREEDY = 0, SM_SUMS = 1, SM_TOPK = 2, SM_TOPP = 3 };
 template <int kMode>
 struct Ring {
   static constexpr int kBuf = kMode <= SM_SUMS ? SV_RING_NBUF_PLAIN : SV_RING_NBUF_CAND;
-  static constexpr int kBytes = (kMode <= SM_SUMS ? SV_RING_KB_PLAIN : SV_RING_KB_CAND) * 1024;
+  static constexpr int kBytes =
+      (kMode <= SM_SUMS ? SV_RING_KB_PLAIN : (kMode == SM_TOPK ? SV_RING_KB_TOPK : SV_RING_KB_CAND)) *
+      1024;
   static constexpr int kBufBytes = kBytes + 128;  // a chunk starts up to 15 bytes in
   static constexpr int kVec = kBytes / (16 * kThreads);  // vectors per consumer thread
   static_assert(kBytes % (16 * kThreads) == 0, "chunk = whole vectors per consumer");
@@ -90,11 +98,13 @@ struct Ring {
 };
 
 __host__ __device__ constexpr int stream_chunk_bytes(int mode) {
-  return (mode <= SM_SUMS ? SV_RING_KB_PLAIN : SV_RING_KB_CAND) * 1024;
+  return mode <= SM_SUMS ? Ring<SM_SUMS>::kBytes
+                         : (mode == SM_TOPK ? Ring<SM_TOPK>::kBytes : Ring<SM_TOPP>::kBytes);
 }
 
 constexpr int kStreamThreads = kThreads + 32;   // eight consumer warps + the producer
-constexpr int kCap = 4096;                      // candidates per row
+constexpr int kCap = 4096;                      // top-p: candidates per row
+constexpr int kCapTopK = 1024;                  // top-k: candidates per row
 constexpr int kKeepFloor = 512;                 // top-p: a cut keeps at least this many
 constexpr int kKeepTarget = 3 * kCap / 8;       // top-p: candidates a cut aims at by row end
 constexpr int kXchgTopP = 4;                    // top-p: chunks between count exchanges
@@ -105,14 +115,20 @@ constexpr int kMemberCap = 512;                 // members of the crossing bin
 constexpr int kRankMax = 1024;                  // lists this short are ranked directly
 constexpr int kStreamMaxTopK = kKeptCap;        // top-k the candidate path takes
 
-// Dynamic shared memory of one CTA: the ring, then (candidate modes) the candidate list,
-// the bin counts and the bin masses (whose space the crossing bin's members reuse).
+// Dynamic shared memory of one CTA: the ring, then top-k: the candidate list and the top k
+// in rank order; top-p: the candidate list, the bin counts and the bin masses (whose space
+// the crossing bin's members reuse).
 __host__ __device__ constexpr size_t stream_dyn_bytes(int mode) {
-  return (mode <= SM_SUMS ? size_t(Ring<SM_SUMS>::kBuf) * Ring<SM_SUMS>::kBufBytes
-                          : size_t(Ring<SM_TOPK>::kBuf) * Ring<SM_TOPK>::kBufBytes) +
-         (mode >= SM_TOPK ? size_t(kCap) * 8 + size_t(kBins) * 4 + size_t(kBins) * 8 : 0);
+  return mode <= SM_SUMS ? size_t(Ring<SM_SUMS>::kBuf) * Ring<SM_SUMS>::kBufBytes
+         : mode == SM_TOPK
+             ? size_t(Ring<SM_TOPK>::kBuf) * Ring<SM_TOPK>::kBufBytes + size_t(kCapTopK) * 8 +
+                   size_t(kKeptCap) * 8
+             : size_t(Ring<SM_TOPP>::kBuf) * Ring<SM_TOPP>::kBufBytes + size_t(kCap) * 8 +
+                   size_t(kBins) * 4 + size_t(kBins) * 8;
 }
 static_assert(2 * kMemberCap * 8 <= kBins * 8, "members and their weights fit the masses");
+static_assert(kCapTopK <= kRankMax, "every top-k list is ranked directly");
+static_assert(kStreamMaxTopK <= kThreads, "the top k in rank order: one per thread");
 
 struct StreamJob {
   RowJob r;             // rows, element type, transform, outputs
@@ -274,9 +290,10 @@ __device__ __forceinline__ int bin_of(float x, float c, float mc) {
 
 template <typename T>
 struct CandSet {
-  uint64_t* cand;              // [kCap]
-  uint32_t* hcnt;              // [kBins]
-  unsigned long long* hmass;   // [kBins]; members and their weights reuse it
+  uint64_t* cand;              // [kCap] (top-k: [kCapTopK])
+  uint32_t* hcnt;              // [kBins] (top-p only)
+  unsigned long long* hmass;   // [kBins]; members and their weights reuse it (top-p only)
+  uint64_t* ranked;            // [kKeptCap]: the top k in rank order (top-k only)
   StreamAux* aux;
 
   // Histogram of the candidates i < n with composite >= lim: counts, and (mass) the sum of
@@ -435,41 +452,29 @@ struct CandSet {
     return aux->sel_comp != 0;
   }
 
-  // Short lists: among the candidates >= lim, in composite order, the one where the mass
-  // accumulated from the top first reaches top_p of their total -> aux->sel_comp.
-  __device__ bool rank_mass(int n, uint64_t lim, float top_p, float c, float mc) {
-    unsigned long long* mw = hmass;  // one weight per list slot (0 below lim)
-    unsigned long long z = 0;
+  // Top-k lists (n <= kRankMax): the top k of cand[0..n) (k <= kThreads) in rank order, then
+  // the one where the mass accumulated from the top first reaches top_p of their total ->
+  // aux->sel_comp. The caller has synchronised the list, and read aux->sel_comp if it needs
+  // it, before the call.
+  __device__ bool rank_topp(int n, int k, float top_p, float c, float mc) {
     for (int i = threadIdx.x; i < n; i += kThreads) {
       const uint64_t e = cand[i];
-      const unsigned long long w = e >= lim ? to_fx(weight(key_value<T>(comp_key(e)), c, mc)) : 0ull;
-      mw[i] = w;
-      z += w;
+      int above = 0;
+      for (int j = 0; j < n; ++j) above += cand[j] > e ? 1 : 0;
+      if (above < k) ranked[above] = e;
     }
-    z = creduce<unsigned long long>(z, aux->scr_u64, OpSum());  // also orders mw
-    unsigned long long target = (unsigned long long)ceil(double(top_p) * double(z));
-    if (target < 1) target = 1;
     if (threadIdx.x == 0) aux->sel_comp = 0;
     csync();
-    for (int i = threadIdx.x; i < n; i += kThreads) {
-      const uint64_t e = cand[i];
-      if (e < lim) continue;
-      unsigned long long above = 0;
-      for (int j = 0; j < n; ++j) above += cand[j] > e ? mw[j] : 0ull;
-      if (above < target && target <= above + mw[i]) aux->sel_comp = e;
-    }
+    const bool mine = int(threadIdx.x) < k;
+    const uint64_t e = mine ? ranked[threadIdx.x] : 0ull;
+    const unsigned long long w = mine ? to_fx(weight(key_value<T>(comp_key(e)), c, mc)) : 0ull;
+    unsigned long long z;
+    const unsigned long long ex = cscan<unsigned long long>(w, aux->scr_u64, &z);
+    unsigned long long target = (unsigned long long)ceil(double(top_p) * double(z));
+    if (target < 1) target = 1;
+    if (mine && ex < target && target <= ex + w) aux->sel_comp = e;
     csync();
     return aux->sel_comp != 0;
-  }
-
-  // Fixed-point sum of the weights of the candidates with composite >= lim.
-  __device__ unsigned long long mass_from(int n, uint64_t lim, float c, float mc) {
-    unsigned long long z = 0;
-    for (int i = threadIdx.x; i < n; i += kThreads) {
-      const uint64_t e = cand[i];
-      if (e >= lim) z += to_fx(weight(key_value<T>(comp_key(e)), c, mc));
-    }
-    return creduce<unsigned long long>(z, aux->scr_u64, OpSum());
   }
 };
 
@@ -571,9 +576,10 @@ struct RowAcc {
 // ------------------------------------------------------------------ kernel
 // Greedy and plain-sum CTAs need no candidate list and fit three to an SM.
 template <typename T, int kMode>
-__global__ void __launch_bounds__(kStreamThreads, (kMode <= SM_SUMS ? 3 : 2))
+__global__ void __launch_bounds__(kStreamThreads, (kMode == SM_TOPP ? 2 : 3))
     stream_rows_kernel(const StreamJob job) {
   constexpr bool kCand = kMode == SM_TOPK || kMode == SM_TOPP;
+  constexpr int kCapM = kMode == SM_TOPK ? kCapTopK : kCap;  // candidates per row
   constexpr int E = Elem<T>::kBytes, P = Elem<T>::kPerVec;
   using RG = Ring<kMode>;
   constexpr int kRing = RG::kBuf, kRingBufBytes = RG::kBufBytes, kVecPerThread = RG::kVec;
@@ -636,8 +642,15 @@ __global__ void __launch_bounds__(kStreamThreads, (kMode <= SM_SUMS ? 3 : 2))
   const float c = rj.c;
   CandSet<T> cs;
   cs.cand = reinterpret_cast<uint64_t*>(smem + size_t(kRing) * kRingBufBytes);
-  cs.hcnt = reinterpret_cast<uint32_t*>(cs.cand + kCap);
-  cs.hmass = reinterpret_cast<unsigned long long*>(cs.hcnt + kBins);
+  if (kMode == SM_TOPK) {
+    cs.ranked = cs.cand + kCapTopK;
+    cs.hcnt = nullptr;
+    cs.hmass = nullptr;
+  } else {
+    cs.ranked = nullptr;
+    cs.hcnt = reinterpret_cast<uint32_t*>(cs.cand + kCap);
+    cs.hmass = reinterpret_cast<unsigned long long*>(cs.hcnt + kBins);
+  }
   cs.aux = &aux;
   RowAcc<T, kMode> st;
   st.reset();
@@ -767,7 +780,7 @@ __global__ void __launch_bounds__(kStreamThreads, (kMode <= SM_SUMS ? 3 : 2))
           const int j0 = base + (16 * (u * kThreads + int(threadIdx.x)) - s.pad) / E;
           for (uint32_t m = cm[u]; m != 0; m &= m - 1) {  // the set bits only
             const int k = __ffs(m) - 1;
-            if (pos < kCap) cs.cand[pos] = make_comp(Elem<T>::key_at(w[u], k), j0 + k);
+            if (pos < kCapM) cs.cand[pos] = make_comp(Elem<T>::key_at(w[u], k), j0 + k);
             ++pos;
           }
         }
@@ -779,7 +792,7 @@ __global__ void __launch_bounds__(kStreamThreads, (kMode <= SM_SUMS ? 3 : 2))
         st.scalar(x, base + j, c, want_ent);
         if (kCand && x >= thr) {
           const int pos = atomicAdd(&aux.ccount, 1);
-          if (pos < kCap) cs.cand[pos] = make_comp(Elem<T>::key(x), base + j);
+          if (pos < kCapM) cs.cand[pos] = make_comp(Elem<T>::key(x), base + j);
           ++single;  // entries this thread appended one by one (edge elements)
         }
       }
@@ -813,12 +826,12 @@ __global__ void __launch_bounds__(kStreamThreads, (kMode <= SM_SUMS ? 3 : 2))
         cnt += added;
         if (kMode == SM_TOPP) thr = fmaxf(thr, mrow - job.topp_span);
         const int rem = nchunk - 1 - q;  // chunks of this row still to come
-        if (cnt > kCap) {
+        if (cnt > kCapM) {
           overflow = true;
         } else if (rem > 0 && ((kMode == SM_TOPK && cnt > 2 * rj.top_k) ||
-                               cnt + added + added / 2 > kCap ||
-                               (cnt >= kCap / 4 &&
-                                cnt + (long long)added * rem / wlen > kCap))) {
+                               cnt + added + added / 2 > kCapM ||
+                               (cnt >= kCapM / 4 &&
+                                cnt + (long long)added * rem / wlen > kCapM))) {
           // top-k: more than 2k candidates; or about to overflow, or projected to: cut
           // the list by count (top-k: to the exact k-th of the entries seen so far)
           int keep = rj.top_k;
@@ -826,10 +839,11 @@ __global__ void __launch_bounds__(kStreamThreads, (kMode <= SM_SUMS ? 3 : 2))
             const long long seen = min((long long)(q + 1) * job.chunk, (long long)rj.V);
             keep = max(kKeepFloor, int((long long)kKeepTarget * seen / rj.V));
           }
-          if (kMode == SM_TOPK && cnt <= kRankMax) {
+          if constexpr (kMode == SM_TOPK) {
             // the exact k-th of the entries seen so far becomes the threshold; the entries
             // below it stay in the list (the row-end selection ranks past them)
-            if (cs.rank_select(cnt, 0, keep)) thr = fmaxf(thr, key_value<T>(comp_key(aux.sel_comp)));
+            if (cnt >= keep && cs.rank_select(cnt, 0, keep))
+              thr = fmaxf(thr, key_value<T>(comp_key(aux.sel_comp)));
           } else if (keep < cnt && mrow > -INFINITY && mrow < INFINITY) {
             cnt = cs.cut(cnt, keep, c, mrow * c, &thr);
           }
@@ -871,35 +885,18 @@ __global__ void __launch_bounds__(kStreamThreads, (kMode <= SM_SUMS ? 3 : 2))
         }
       } else {
         if (status == ROW_OK) {
-          const int n = min(nall, kCap);
-          bool ok = !overflow && nall <= kCap;
+          const int n = min(nall, kCapM);
+          bool ok = !overflow && nall <= kCapM;
           uint64_t cstar = 0;
           if constexpr (kMode == SM_TOPK) {
             ok = ok && n >= rj.top_k;
-            if (ok && n <= kRankMax) {  // short list: rank directly
-              ok = cs.rank_select(n, 0, rj.top_k);
-              cstar = aux.sel_comp;
-              if (ok && rj.top_p < 1.0f) {
-                ok = cs.rank_mass(n, cstar, rj.top_p, c, mc);
-                cstar = aux.sel_comp;
+            if (ok) {  // every list is short (kCapTopK <= kRankMax): rank directly
+              if (rj.top_p < 1.0f) {  // the top-p crossing within the top k
+                ok = cs.rank_topp(n, rj.top_k, rj.top_p, c, mc);
+              } else {
+                ok = cs.rank_select(n, 0, rj.top_k);
               }
-            } else if (ok) {  // the k-th candidate by count, over log-weight bins
-              cs.hist_build(n, 0, c, mc, false);
-              cs.hist_find((unsigned long long)rj.top_k, false);
-              ok = aux.sel_found &&
-                   cs.resolve(n, 0, c, mc, false, (unsigned long long)rj.top_k - aux.sel_before);
               cstar = aux.sel_comp;
-              if (ok && rj.top_p < 1.0f) {  // then the top-p crossing within the top k
-                const unsigned long long zk = cs.mass_from(n, cstar, c, mc);
-                unsigned long long target =
-                    (unsigned long long)ceil(double(rj.top_p) * double(zk));
-                if (target < 1) target = 1;
-                cs.hist_build(n, cstar, c, mc, true);
-                cs.hist_find(target, true);
-                ok = aux.sel_found &&
-                     cs.resolve(n, cstar, c, mc, true, target - aux.sel_before);
-                cstar = aux.sel_comp;
-              }
             }
           } else {  // top-p over the whole row: the mass target from the online sums
             float sc = 0.0f;

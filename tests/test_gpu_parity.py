@@ -132,6 +132,27 @@ def test_chain_ragged_vocab(dtype, V):
         run_case(target, draft, toks, u, 1.1, top_p=0.8)
 
 
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+@pytest.mark.parametrize("trend", [-1.0, 0.0, 1.0])
+@pytest.mark.parametrize("top_k,top_p", [(50, 1.0), (50, 0.9), (256, 0.95), (3, 0.5)])
+def test_chain_topk_multichunk_trends(dtype, trend, top_k, top_p):
+    """Top-k, alone and with top-p, over rows of several streamed chunks whose values fall
+    along the vocabulary (the first chunk holds the top), stay level, or rise (later chunks
+    keep adding candidates, up to the list's capacity and past it, so rows go to the exact
+    finisher)."""
+    B, K, V = 6, 3, 60000
+    g = np.random.default_rng(7000 + int(10 * trend) + top_k)
+    ramp = trend * 1.2 * np.log1p(np.arange(V))
+    t = g.normal(0, 3.0, size=(B, K + 1, V)) + ramp
+    d = t[:, :K] + g.normal(0, 1.0, size=(B, K, V))
+    conv = (lambda a: specgen.f32_to_bf16_bits(a.astype(np.float32))) if dtype == "bf16" \
+        else (lambda a: a.astype(np.float32))
+    target, draft = conv(t), conv(d)
+    toks = draft_tokens(draft, 0.8, top_k, top_p, g.random((B, K)).astype(np.float32))
+    u = g.random((B, K + 1)).astype(np.float32)
+    run_case(target, draft, toks, u, 0.8, top_k, top_p)
+
+
 def test_chain_sixteen_cta_cluster():
     """V = 300000 bfloat16 (600 KB rows) spreads each row over a 16-CTA cluster."""
     target, draft, toks, u = _rand_chain(3, 3, 2, 300000, "bf16", sigma=3.0)
