@@ -9,8 +9,8 @@
 // themselves only with named barrier 1, so the producer is never held up by their row-end
 // work. Nothing is shared between CTAs.
 //
-// Per chunk each consumer thread takes eight (top-k: seven) 16-byte vectors and updates,
-// as the mode needs:
+// Per chunk each consumer thread takes eight 16-byte vectors and updates, as the mode
+// needs:
 //   SM_GREEDY  its running maximum (packed bf16x2 max, NaN propagating) and the lowest index
 //              holding it;
 //   SM_SUMS    an online softmax sum (and entropy term), rescaled when its maximum grows;
@@ -61,11 +61,10 @@
 
 namespace sv {
 
-// Ring of chunk buffers per CTA: two chunks in every mode. Greedy and plain sums stream
-// 32 KB chunks at three CTAs per SM; top-k 28 KB chunks at three CTAs per SM (its list of
-// kCapTopK candidates and the top k in rank order fill the rest); top-p 32 KB chunks at two
-// CTAs per SM (its larger list and the log-weight histogram take the rest). The depth and
-// chunk size of each kind are build-time knobs.
+// Ring of chunk buffers per CTA: two 32 KB chunks in every mode. Greedy, plain sums and
+// top-k run three CTAs per SM (top-k adds its list of kCapTopK candidates and the top k in
+// rank order, which just fits); top-p two (its larger list and the log-weight histogram
+// take the rest). The depth and chunk size of each kind are build-time knobs.
 #ifndef SV_RING_NBUF_PLAIN
 #define SV_RING_NBUF_PLAIN 2
 #endif
@@ -79,7 +78,7 @@ namespace sv {
 #define SV_RING_KB_CAND 32
 #endif
 #ifndef SV_RING_KB_TOPK
-#define SV_RING_KB_TOPK 28
+#define SV_RING_KB_TOPK 32
 #endif
 constexpr int kMaxRing = 4;
 
@@ -159,6 +158,11 @@ struct __align__(16) StreamAux {
   int mcount;
   int broken;   // a copy or buffer wait timed out: the CTA stops reading rows
 };
+
+// Three top-k CTAs per SM: ring, list, ranked top k, this record and the 1 KB the hardware
+// reserves per CTA, within the SM's 228 KB.
+static_assert(3 * (stream_dyn_bytes(SM_TOPK) + sizeof(StreamAux) + 1024) <= 228 * 1024,
+              "three top-k CTAs per SM");
 
 // ------------------------------------------------------------------ consumer barriers
 // Named barrier 1 over the 256 consumer threads (the producer warp never joins it).
