@@ -159,6 +159,22 @@ __device__ __forceinline__ unsigned long long to_fx(float mass01) {
   return __float2ull_rn(mass01 * kFxF);
 }
 
+// Fixed-point masses (< 2^45) summed in shared memory as three 15-bit limbs with 32-bit
+// atomics: a 64-bit shared atomic add is many times slower, most of all when lanes collide
+// on one address. A histogram of n bins keeps limb i of bin b at l[i * n + b]; up to 2^16
+// adds per bin cannot overflow a limb, and the sum is exact.
+__device__ __forceinline__ void limb_add(uint32_t* l, int n, int b, unsigned long long w) {
+  const uint32_t w0 = uint32_t(w & 0x7FFFu), w1 = uint32_t((w >> 15) & 0x7FFFu),
+                 w2 = uint32_t(w >> 30);
+  if (w0) atomicAdd(&l[b], w0);
+  if (w1) atomicAdd(&l[n + b], w1);
+  if (w2) atomicAdd(&l[2 * n + b], w2);
+}
+__device__ __forceinline__ unsigned long long limb_get(const uint32_t* l, int n, int b) {
+  return (unsigned long long)l[b] + ((unsigned long long)l[n + b] << 15) +
+         ((unsigned long long)l[2 * n + b] << 30);
+}
+
 // ------------------------------------------------------------------------- PTX: bulk copies
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));

@@ -81,7 +81,7 @@ struct __align__(16) RowAux {
   union {
     struct {  // radix select
       uint32_t hcnt[2][256];
-      unsigned long long hmass[2][256];
+      uint32_t hlimb[2][3 * 256];  // masses as 15-bit limbs (limb_add)
       uint32_t tot_cnt[256];
       unsigned long long tot_mass[256];
     } g;
@@ -164,38 +164,6 @@ __device__ __forceinline__ bool finish_slice(const SliceLoc& s, unsigned char* b
   return ok;
 }
 
-// Adds one count and the fixed-point mass w (<= 2^43) to bin `bin` of hc and hm for every
-// lane with `in`. Where the warp's lanes fall in few distinct bins (the usual case for the
-// high bits of float keys, whose exponents cluster), lanes sharing a bin are combined first:
-// one pair of atomics per distinct bin instead of many 64-bit atomics on one address. Every
-// lane of the warp calls it. The sums are exact, so the result does not depend on the path.
-// (A count alone is cheaper with plain 32-bit atomics.)
-__device__ __forceinline__ void hist_add_mass(uint32_t* hc, unsigned long long* hm, uint32_t bin,
-                                              unsigned long long w, bool in) {
-  const int lane = threadIdx.x & 31;
-  const unsigned peers = __match_any_sync(0xffffffffu, in ? bin : 0xFFFFFFFFu);
-  const unsigned lead = __ballot_sync(0xffffffffu, in && lane == __ffs(peers) - 1);
-  if (__popc(lead) > 8) {  // many distinct bins: each lane adds its own
-    if (in) {
-      atomicAdd(&hc[bin], 1u);
-      atomicAdd(&hm[bin], w);
-    }
-    return;
-  }
-  for (unsigned L = lead; L != 0; L &= L - 1) {
-    const int src = __ffs(L) - 1;
-    const uint32_t b = __shfl_sync(0xffffffffu, bin, src);
-    const bool mine = in && bin == b;
-    // w in two 21-bit halves: a sum of 32 of either cannot overflow 32 bits
-    const uint32_t hi = __reduce_add_sync(0xffffffffu, mine ? uint32_t(w >> 21) : 0u);
-    const uint32_t lo = __reduce_add_sync(0xffffffffu, mine ? uint32_t(w & 0x1FFFFFu) : 0u);
-    if (lane == src) {
-      atomicAdd(&hc[b], uint32_t(__popc(peers)));
-      atomicAdd(&hm[b], ((unsigned long long)hi << 21) + lo);
-    }
-  }
-}
-
 template <typename T>
 struct RowCtx {
   const unsigned char* buf;
@@ -231,27 +199,6 @@ struct RowCtx {
           const int j = j0 + k;
           if (j >= 0 && j < n) f(s0 + j, x[k]);
         }
-      }
-    }
-  }
-
-  // Like each(), but every lane of a warp calls f(global id, value, ok) the same number of
-  // times (ok false for places past the slice), so f may use warp-wide intrinsics.
-  template <typename F>
-  __device__ __forceinline__ void each_warp(F&& f) const {
-    constexpr int P = Elem<T>::kPerVec;
-    const int vend = (nvec + kThreads - 1) / kThreads * kThreads;
-    for (int v = threadIdx.x; v < vend; v += kThreads) {
-      const bool vin = v < nvec;
-      uint4 w = make_uint4(0u, 0u, 0u, 0u);
-      if (vin) w = reinterpret_cast<const uint4*>(buf)[v];
-      float x[P];
-      Elem<T>::unpack(w, x);
-      const int j0 = first_elem(v);
-#pragma unroll
-      for (int k = 0; k < P; ++k) {
-        const int j = j0 + k;
-        f(s0 + j, x[k], vin && j >= 0 && j < n);
       }
     }
   }
@@ -621,16 +568,17 @@ struct RowCtx {
     unsigned long long before = 0, mass_eq = 0;
     for (int shift = KB - 8; shift >= 0; shift -= 8) {
       uint32_t* hc = aux->u.g.hcnt[ph];
-      unsigned long long* hm = aux->u.g.hmass[ph];
-      for (int i = threadIdx.x; i < 256; i += kThreads) {
-        hc[i] = 0;
-        hm[i] = 0;
-      }
+      uint32_t* hl = aux->u.g.hlimb[ph];
+      for (int i = threadIdx.x; i < 256; i += kThreads) hc[i] = 0;
+      for (int i = threadIdx.x; i < 3 * 256; i += kThreads) hl[i] = 0;
       __syncthreads();
-      each_warp([&](int id, float x, bool ok) {
+      each([&](int id, float x) {
         const uint32_t key = Elem<T>::key(x);
-        const bool in = ok && (key & pmask) == prefix && kept(key, id, thr_k, cut_k);
-        hist_add_mass(hc, hm, (key >> shift) & 255u, in ? to_fx(weight(x, c, mc)) : 0ull, in);
+        if ((key & pmask) == prefix && kept(key, id, thr_k, cut_k)) {
+          const uint32_t bin = (key >> shift) & 255u;
+          atomicAdd(&hc[bin], 1u);
+          limb_add(hl, 256, int(bin), to_fx(weight(x, c, mc)));
+        }
       });
       __syncthreads();
       cl.sync();
@@ -639,7 +587,7 @@ struct RowCtx {
         unsigned long long sm = 0;
         for (int r = 0; r < C; ++r) {
           sc += remote(aux->u.g.hcnt[ph], r)[threadIdx.x];
-          sm += remote(aux->u.g.hmass[ph], r)[threadIdx.x];
+          sm += limb_get(remote(aux->u.g.hlimb[ph], r), 256, int(threadIdx.x));
         }
         aux->u.g.tot_cnt[threadIdx.x] = sc;
         aux->u.g.tot_mass[threadIdx.x] = sm;

@@ -115,17 +115,17 @@ constexpr int kRankMax = 1024;                  // lists this short are ranked d
 constexpr int kStreamMaxTopK = kKeptCap;        // top-k the candidate path takes
 
 // Dynamic shared memory of one CTA: the ring, then top-k: the candidate list and the top k
-// in rank order; top-p: the candidate list, the bin counts and the bin masses (whose space
-// the crossing bin's members reuse).
+// in rank order; top-p: the candidate list, the bin counts and the bin masses as 15-bit
+// limbs (whose space the crossing bin's members reuse).
 __host__ __device__ constexpr size_t stream_dyn_bytes(int mode) {
   return mode <= SM_SUMS ? size_t(Ring<SM_SUMS>::kBuf) * Ring<SM_SUMS>::kBufBytes
          : mode == SM_TOPK
              ? size_t(Ring<SM_TOPK>::kBuf) * Ring<SM_TOPK>::kBufBytes + size_t(kCapTopK) * 8 +
                    size_t(kKeptCap) * 8
              : size_t(Ring<SM_TOPP>::kBuf) * Ring<SM_TOPP>::kBufBytes + size_t(kCap) * 8 +
-                   size_t(kBins) * 4 + size_t(kBins) * 8;
+                   size_t(kBins) * 4 + size_t(kBins) * 12;
 }
-static_assert(2 * kMemberCap * 8 <= kBins * 8, "members and their weights fit the masses");
+static_assert(2 * kMemberCap * 8 <= 3 * kBins * 4, "members and their weights fit the masses");
 static_assert(kCapTopK <= kRankMax, "every top-k list is ranked directly");
 static_assert(kStreamMaxTopK <= kThreads, "the top k in rank order: one per thread");
 
@@ -163,6 +163,8 @@ struct __align__(16) StreamAux {
 // reserves per CTA, within the SM's 228 KB.
 static_assert(3 * (stream_dyn_bytes(SM_TOPK) + sizeof(StreamAux) + 1024) <= 228 * 1024,
               "three top-k CTAs per SM");
+static_assert(2 * (stream_dyn_bytes(SM_TOPP) + sizeof(StreamAux) + 1024) <= 228 * 1024,
+              "two top-p CTAs per SM");
 
 // ------------------------------------------------------------------ consumer barriers
 // Named barrier 1 over the 256 consumer threads (the producer warp never joins it).
@@ -296,17 +298,17 @@ template <typename T>
 struct CandSet {
   uint64_t* cand;              // [kCap] (top-k: [kCapTopK])
   uint32_t* hcnt;              // [kBins] (top-p only)
-  unsigned long long* hmass;   // [kBins]; members and their weights reuse it (top-p only)
+  uint32_t* hlimb;             // [3][kBins]: bin masses as limbs; members and their weights
+                               // reuse it (top-p only)
   uint64_t* ranked;            // [kKeptCap]: the top k in rank order (top-k only)
   StreamAux* aux;
 
   // Histogram of the candidates i < n with composite >= lim: counts, and (mass) the sum of
   // their fixed-point weights.
   __device__ void hist_build(int n, uint64_t lim, float c, float mc, bool mass) {
-    for (int i = threadIdx.x; i < kBins; i += kThreads) {
-      hcnt[i] = 0;
-      if (mass) hmass[i] = 0;
-    }
+    for (int i = threadIdx.x; i < kBins; i += kThreads) hcnt[i] = 0;
+    if (mass)
+      for (int i = threadIdx.x; i < 3 * kBins; i += kThreads) hlimb[i] = 0;
     csync();
     for (int i0 = 0; i0 < n; i0 += kThreads) {
       const int i = i0 + threadIdx.x;
@@ -324,7 +326,7 @@ struct CandSet {
       hist_add(hcnt, b, ok);
       if (mass && ok) {
         const unsigned long long w = to_fx(weight(x, c, mc));
-        if (w) atomicAdd(&hmass[b], w);
+        limb_add(hlimb, kBins, b, w);
       }
     }
     csync();
@@ -340,7 +342,7 @@ struct CandSet {
 #pragma unroll
     for (int q = 0; q < kPer; ++q) {
       const int b = threadIdx.x * kPer + q;
-      part[q] = mass ? hmass[b] : (unsigned long long)hcnt[b];
+      part[q] = mass ? limb_get(hlimb, kBins, b) : (unsigned long long)hcnt[b];
       tsum += part[q];
     }
     unsigned long long total;
@@ -372,8 +374,8 @@ struct CandSet {
                           unsigned long long need) {
     if (aux->sel_cnt > uint32_t(kMemberCap)) return false;  // uniform
     const int bsel = aux->sel_bin;
-    uint64_t* mem = reinterpret_cast<uint64_t*>(hmass);
-    unsigned long long* mw = hmass + kMemberCap;
+    uint64_t* mem = reinterpret_cast<uint64_t*>(hlimb);
+    unsigned long long* mw = reinterpret_cast<unsigned long long*>(hlimb) + kMemberCap;
     if (threadIdx.x == 0) {
       aux->mcount = 0;
       aux->sel_comp = 0;
@@ -649,11 +651,11 @@ __global__ void __launch_bounds__(kStreamThreads, (kMode == SM_TOPP ? 2 : 3))
   if (kMode == SM_TOPK) {
     cs.ranked = cs.cand + kCapTopK;
     cs.hcnt = nullptr;
-    cs.hmass = nullptr;
+    cs.hlimb = nullptr;
   } else {
     cs.ranked = nullptr;
     cs.hcnt = reinterpret_cast<uint32_t*>(cs.cand + kCap);
-    cs.hmass = reinterpret_cast<unsigned long long*>(cs.hcnt + kBins);
+    cs.hlimb = cs.hcnt + kBins;
   }
   cs.aux = &aux;
   RowAcc<T, kMode> st;
