@@ -441,6 +441,29 @@ struct CandSet {
     return int(total);
   }
 
+  // Top-k lists: keeps the candidates of cand[0..n) (n <= kCapTopK) whose composite is
+  // >= lim, in place; returns their count (also the list's new fill count).
+  __device__ int compact_ge(int n, uint64_t lim) {
+    constexpr int kPer = kCapTopK / kThreads;
+    uint64_t v[kPer];
+    uint32_t keepm = 0;
+    const int lo = threadIdx.x * kPer;
+#pragma unroll
+    for (int q = 0; q < kPer; ++q) {
+      const int i = lo + q;
+      v[q] = i < n ? cand[i] : 0ull;
+      if (i < n && v[q] >= lim) keepm |= 1u << q;
+    }
+    uint32_t total;
+    uint32_t pos = cscan<uint32_t>(uint32_t(__popc(keepm)), aux->scr_u32, &total);
+#pragma unroll
+    for (int q = 0; q < kPer; ++q)
+      if (keepm & (1u << q)) cand[pos++] = v[q];
+    if (threadIdx.x == 0) aux->ccount = int(total);
+    csync();
+    return int(total);
+  }
+
   // Short lists (n <= kRankMax, flat): the k-th largest composite among cand[0..n) that are
   // >= lim, by counting for each the larger ones (composites are distinct) ->
   // aux->sel_comp. The caller has synchronised the list. False if there is none.
@@ -594,6 +617,9 @@ __global__ void __launch_bounds__(kStreamThreads, (kMode == SM_TOPP ? 2 : 3))
   unsigned char* ring = smem;
   const RowJob& rj = job.r;
   const int nchunk = job.nchunk;
+  // top-k: chunks between count exchanges, so that about kCapTopK / 2 entries can arrive
+  // between two even when every chunk brings k new ones
+  const int xchg_k = kMode == SM_TOPK ? max(1, (kCapTopK / 2) / max(1, rj.top_k)) : 0;
   const long long nrows_mine =
       rj.rows > blockIdx.x ? (rj.rows - 1 - blockIdx.x) / gridDim.x + 1 : 0;
   const long long items = nrows_mine * nchunk;
@@ -810,7 +836,8 @@ __global__ void __launch_bounds__(kStreamThreads, (kMode == SM_TOPP ? 2 : 3))
     if constexpr (kCand) {
       wacc += wadd;
       ++wlen;
-      if ((kMode == SM_TOPP && wlen == kXchgTopP && q != nchunk - 1) || q == 0) {
+      if ((kMode == SM_TOPP && wlen == kXchgTopP && q != nchunk - 1) ||
+          (kMode == SM_TOPK && wlen == xchg_k && q != nchunk - 1) || q == 0) {
         // exchange: the row maximum so far and the entries appended since the last one
         float wm = st.mt;
 #pragma unroll
@@ -834,7 +861,7 @@ __global__ void __launch_bounds__(kStreamThreads, (kMode == SM_TOPP ? 2 : 3))
         const int rem = nchunk - 1 - q;  // chunks of this row still to come
         if (cnt > kCapM) {
           overflow = true;
-        } else if (rem > 0 && ((kMode == SM_TOPK && cnt > 2 * rj.top_k) ||
+        } else if (rem > 0 && ((kMode == SM_TOPK && cnt > rj.top_k) ||
                                cnt + added + added / 2 > kCapM ||
                                (cnt >= kCapM / 4 &&
                                 cnt + (long long)added * rem / wlen > kCapM))) {
@@ -846,10 +873,14 @@ __global__ void __launch_bounds__(kStreamThreads, (kMode == SM_TOPP ? 2 : 3))
             keep = max(kKeepFloor, int((long long)kKeepTarget * seen / rj.V));
           }
           if constexpr (kMode == SM_TOPK) {
-            // the exact k-th of the entries seen so far becomes the threshold; the entries
-            // below it stay in the list (the row-end selection ranks past them)
-            if (cnt >= keep && cs.rank_select(cnt, 0, keep))
-              thr = fmaxf(thr, key_value<T>(comp_key(aux.sel_comp)));
+            // the exact k-th of the entries seen so far becomes the threshold; a short list
+            // keeps the entries below it (the row-end selection ranks past them), one past
+            // half the capacity drops them
+            if (cnt >= keep && cs.rank_select(cnt, 0, keep)) {
+              const uint64_t kth = aux.sel_comp;
+              thr = fmaxf(thr, key_value<T>(comp_key(kth)));
+              if (cnt > kCapTopK / 2) cnt = cs.compact_ge(cnt, kth);
+            }
           } else if (keep < cnt && mrow > -INFINITY && mrow < INFINITY) {
             cnt = cs.cut(cnt, keep, c, mrow * c, &thr);
           }
