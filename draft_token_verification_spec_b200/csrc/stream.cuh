@@ -245,6 +245,27 @@ __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
 
+// The j-th largest (1 <= j <= 32 N) of the warp's 32 N keys (N per lane), by a radix walk
+// from the top bit with warp-wide counts; every lane calls it.
+template <int KB, int N>
+__device__ __forceinline__ uint32_t warp_kth_key_n(const uint32_t (&key)[N], int j) {
+  uint32_t prefix = 0;
+  int need = j;
+#pragma unroll 1
+  for (int b = KB - 1; b >= 0; --b) {
+    const uint32_t cand = prefix | (1u << b);
+    uint32_t c = 0;
+#pragma unroll
+    for (int i = 0; i < N; ++i) c += (key[i] >> b) == (cand >> b) ? 1u : 0u;
+    const int cnt = int(__reduce_add_sync(0xffffffffu, c));
+    if (cnt >= need)
+      prefix = cand;
+    else
+      need -= cnt;
+  }
+  return prefix;
+}
+
 // ------------------------------------------------------------------ chunks
 // Chunk q of a row: element j lands at byte pad + j * E of its buffer (pad = the source
 // address mod 16); the 16-byte-aligned middle [pad + head, pad + head + mid) moves by
@@ -730,9 +751,19 @@ __global__ void __launch_bounds__(kStreamThreads, (kMode == SM_TOPP ? 2 : 3))
           for (int j = e_lo; j < e_hi; ++j) pm = fmax_nan(pm, Elem<T>::load(s.g, j));
         if constexpr (kMode == SM_TOPK) {
           const int jw = (rj.top_k + kWarps - 1) / kWarps;  // <= 32: top_k <= 256
-          const float tw =
-              key_value<T>(warp_kth_key<Elem<T>::kKeyBits>(Elem<T>::key(pm), jw));
-          thr = creduce<float>(tw, aux.scr_f, OpMin());
+          uint32_t kw;
+          if (jw <= 16) {  // a value that jw of the warp's per-thread maxima reach
+            kw = warp_kth_key<Elem<T>::kKeyBits>(Elem<T>::key(pm), jw);
+          } else {
+            // large k: a per-thread maximum stands for eight vectors, too coarse a step;
+            // a value that jw of the warp's vector maxima reach (vectors outside the
+            // chunk hold -inf)
+            uint32_t kv[kVecPerThread];
+#pragma unroll
+            for (int u = 0; u < kVecPerThread; ++u) kv[u] = Elem<T>::key(vm[u]);
+            kw = warp_kth_key_n<Elem<T>::kKeyBits, kVecPerThread>(kv, jw);
+          }
+          thr = creduce<float>(key_value<T>(kw), aux.scr_f, OpMin());
         } else {
           const float m0 = creduce<float>(pm, aux.scr_f, OpMaxNan());
           float t0 = m0 - job.topp_span;
