@@ -22,11 +22,14 @@
 // (value desc, id asc) that top-k and top-p use, so the k-th candidate is unique.
 //
 // Top-k: the first threshold is a value that k entries of the first chunk reach (per-warp
-// order statistics of per-thread maxima). After the first chunk the consumer warps exchange
-// their counts once, and a list of more than 2k entries sets the threshold to the exact
-// k-th of the chunk (ranked directly, the list kept as it is). Later chunks of usual rows
-// rarely reach it; no further exchange runs, and a list that outgrows kCapTopK sends the row
-// to the exact finisher. The short list keeps a top-k CTA small enough for three per SM.
+// order statistics of per-thread maxima; of vector maxima for k > 128). After the first
+// chunk the consumer warps exchange their counts, and a list of more than k entries sets the
+// threshold to the exact k-th seen so far (ranked directly, the list kept as it is). Further
+// exchanges run every (kCapTopK / 2) / k chunks, so about half the list can fill between
+// two even if every chunk brings k new entries; one past half the capacity is cut to its top
+// k. Rows whose values do not grow along the vocabulary rarely reach the threshold again, and
+// a list that still outgrows kCapTopK sends the row to the exact finisher. The short list
+// keeps a top-k CTA small enough for three per SM.
 //
 // Top-p: the threshold starts at (first-chunk maximum - T ln(V / (1 - top_p))), below
 // which the whole row holds less than 1 - top_p of the mass, raised to the smallest of
