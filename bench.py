@@ -107,12 +107,13 @@ class ClockSampler:
     def __init__(self, index: int):
         self.index = index
         self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{index}.csv")
+        self.path = None
 
     def start(self):
         try:
-            os.makedirs(os.path.dirname(self.path), exist_ok=True)
-            self.fh = open(self.path, "w")
+            import tempfile
+            fd, self.path = tempfile.mkstemp(prefix=f"clocks_gpu{self.index}_", suffix=".csv")
+            self.fh = os.fdopen(fd, "w")
             self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.index}",
                                           f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
                                           "-lms", "50"], stdout=self.fh,
@@ -126,6 +127,9 @@ class ClockSampler:
         self.proc.terminate()
         self.proc.wait(timeout=10)
         self.fh.close()
+        if os.environ.get("SPEC_CLOCKS_CSV"):  # keep the raw samples where the caller asks
+            import shutil
+            shutil.copyfile(self.path, os.environ["SPEC_CLOCKS_CSV"])
         sm, mx, reasons = [], 0.0, set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         with open(self.path) as f:
@@ -141,6 +145,7 @@ class ClockSampler:
                 for n, v in zip(names, p[5:9]):
                     if v.lower() == "active":
                         reasons.add(n)
+        os.unlink(self.path)
         return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx or None,
                 "reasons": sorted(reasons), "samples": len(sm)}
 

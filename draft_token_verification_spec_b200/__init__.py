@@ -143,10 +143,11 @@ def spec_verify_chain(target_logits, draft_logits, draft_tokens, uniforms, temp,
         out_tokens = torch.empty((B, K + 1), dtype=torch.int32, device=t.device)
     if workspace is None:
         workspace = torch.empty(spec_workspace_size(B, K, V), dtype=torch.uint8, device=t.device)
-    _check("spec_verify_chain", lib().spec_verify_chain(
-        _ptr(t), _ptr(d), _dtype(t), B, K, V, _ptr(x), _ptr(u), float(temp), int(top_k),
-        float(top_p), _ptr(accepted_len), _ptr(out_tokens), _ptr(workspace),
-        workspace.numel() * workspace.element_size(), _stream(stream, t.device)))
+    with torch.cuda.device(t.device):  # launches go to the tensors' device
+        _check("spec_verify_chain", lib().spec_verify_chain(
+            _ptr(t), _ptr(d), _dtype(t), B, K, V, _ptr(x), _ptr(u), float(temp), int(top_k),
+            float(top_p), _ptr(accepted_len), _ptr(out_tokens), _ptr(workspace),
+            workspace.numel() * workspace.element_size(), _stream(stream, t.device)))
     return accepted_len, out_tokens
 
 
@@ -169,9 +170,10 @@ def spec_verify_chain_noalloc(target_logits, draft_logits, draft_tokens, uniform
         accepted_len = torch.empty(B, dtype=torch.int32, device=t.device)
     if out_tokens is None:
         out_tokens = torch.empty((B, K + 1), dtype=torch.int32, device=t.device)
-    _check("spec_verify_chain_noalloc", lib().spec_verify_chain_noalloc(
-        _ptr(t), _ptr(d), _dtype(t), B, K, V, _ptr(x), _ptr(u), float(temp), int(top_k),
-        float(top_p), _ptr(accepted_len), _ptr(out_tokens), _stream(stream, t.device)))
+    with torch.cuda.device(t.device):  # launches go to the tensors' device
+        _check("spec_verify_chain_noalloc", lib().spec_verify_chain_noalloc(
+            _ptr(t), _ptr(d), _dtype(t), B, K, V, _ptr(x), _ptr(u), float(temp), int(top_k),
+            float(top_p), _ptr(accepted_len), _ptr(out_tokens), _stream(stream, t.device)))
     return accepted_len, out_tokens
 
 
@@ -193,10 +195,11 @@ def spec_verify_tree_typical(target_logits, node_tokens, parent_idx, eps, delta,
         accepted_len = torch.empty(B, dtype=torch.int32, device=t.device)
     if workspace is None:
         workspace = torch.empty(spec_workspace_size(B, N, V), dtype=torch.uint8, device=t.device)
-    _check("spec_verify_tree_typical", lib().spec_verify_tree_typical(
-        _ptr(t), _dtype(t), B, N, V, _ptr(nt), _ptr(par), float(eps), float(delta),
-        _ptr(best_path), cap, _ptr(accepted_len), _ptr(workspace),
-        workspace.numel() * workspace.element_size(), _stream(stream, t.device)))
+    with torch.cuda.device(t.device):  # launches go to the tensors' device
+        _check("spec_verify_tree_typical", lib().spec_verify_tree_typical(
+            _ptr(t), _dtype(t), B, N, V, _ptr(nt), _ptr(par), float(eps), float(delta),
+            _ptr(best_path), cap, _ptr(accepted_len), _ptr(workspace),
+            workspace.numel() * workspace.element_size(), _stream(stream, t.device)))
     return best_path, accepted_len
 
 
@@ -221,10 +224,11 @@ def spec_verify_tree_greedy(target_logits, node_tokens, parent_idx, path_cap=Non
         next_token = torch.empty(B, dtype=torch.int32, device=t.device)
     if workspace is None:
         workspace = torch.empty(spec_workspace_size(B, N, V), dtype=torch.uint8, device=t.device)
-    _check("spec_verify_tree_greedy", lib().spec_verify_tree_greedy(
-        _ptr(t), _dtype(t), B, N, V, _ptr(nt), _ptr(par), _ptr(best_path), cap,
-        _ptr(accepted_len), _ptr(next_token), _ptr(workspace),
-        workspace.numel() * workspace.element_size(), _stream(stream, t.device)))
+    with torch.cuda.device(t.device):  # launches go to the tensors' device
+        _check("spec_verify_tree_greedy", lib().spec_verify_tree_greedy(
+            _ptr(t), _dtype(t), B, N, V, _ptr(nt), _ptr(par), _ptr(best_path), cap,
+            _ptr(accepted_len), _ptr(next_token), _ptr(workspace),
+            workspace.numel() * workspace.element_size(), _stream(stream, t.device)))
     return best_path, accepted_len, next_token
 
 
@@ -253,11 +257,12 @@ def spec_verify_tree_sampling(target_logits, draft_logits, node_tokens, parent_i
         next_token = torch.empty(B, dtype=torch.int32, device=t.device)
     if workspace is None:
         workspace = torch.empty(spec_workspace_size(B, N, V), dtype=torch.uint8, device=t.device)
-    _check("spec_verify_tree_sampling", lib().spec_verify_tree_sampling(
-        _ptr(t), _ptr(d), _dtype(t), B, N, V, _ptr(nt), _ptr(par), _ptr(u), float(temp),
-        int(top_k), float(top_p), _ptr(best_path), cap, _ptr(accepted_len), _ptr(next_token),
-        _ptr(workspace), workspace.numel() * workspace.element_size(),
-        _stream(stream, t.device)))
+    with torch.cuda.device(t.device):  # launches go to the tensors' device
+        _check("spec_verify_tree_sampling", lib().spec_verify_tree_sampling(
+            _ptr(t), _ptr(d), _dtype(t), B, N, V, _ptr(nt), _ptr(par), _ptr(u), float(temp),
+            int(top_k), float(top_p), _ptr(best_path), cap, _ptr(accepted_len), _ptr(next_token),
+            _ptr(workspace), workspace.numel() * workspace.element_size(),
+            _stream(stream, t.device)))
     return best_path, accepted_len, next_token
 
 
@@ -272,9 +277,10 @@ def spec_logits_to_probs(logits, temp, top_k=0, top_p=1.0, with_entropy=True, pr
         probs = torch.empty(lg.shape, dtype=torch.float32, device=lg.device)
     if with_entropy and entropy is None:
         entropy = torch.empty(lg.shape[:-1], dtype=torch.float32, device=lg.device)
-    _check("spec_logits_to_probs", lib().spec_logits_to_probs(
-        _ptr(lg), _dtype(lg), rows, V, float(temp), int(top_k), float(top_p), _ptr(probs),
-        _ptr(entropy), _stream(stream, lg.device)))
+    with torch.cuda.device(lg.device):  # launches go to the tensors' device
+        _check("spec_logits_to_probs", lib().spec_logits_to_probs(
+            _ptr(lg), _dtype(lg), rows, V, float(temp), int(top_k), float(top_p), _ptr(probs),
+            _ptr(entropy), _stream(stream, lg.device)))
     return probs, entropy
 
 
@@ -289,15 +295,17 @@ def spec_residual_sample(p, q, uniforms, tokens=None, stream=None):
     u = _dev(uniforms, "uniforms", torch.float32)
     if tokens is None:
         tokens = torch.empty(rows, dtype=torch.int32, device=pp.device)
-    _check("spec_residual_sample", lib().spec_residual_sample(
-        _ptr(pp), _ptr(qq), rows, V, _ptr(u), _ptr(tokens), _stream(stream, pp.device)))
+    with torch.cuda.device(pp.device):  # launches go to the tensors' device
+        _check("spec_residual_sample", lib().spec_residual_sample(
+            _ptr(pp), _ptr(qq), rows, V, _ptr(u), _ptr(tokens), _stream(stream, pp.device)))
     return tokens
 
 
 def spec_get_device_status(workspace, stream=None) -> int:
     out = ctypes.c_int32(0)
-    _check("spec_get_device_status", lib().spec_get_device_status(
-        _ptr(workspace), ctypes.byref(out), _stream(stream, workspace.device)))
+    with torch.cuda.device(workspace.device):  # launches go to the tensors' device
+        _check("spec_get_device_status", lib().spec_get_device_status(
+            _ptr(workspace), ctypes.byref(out), _stream(stream, workspace.device)))
     return int(out.value)
 
 

@@ -10,7 +10,8 @@
 // one statically sized __device__ array (one instance per device the module is loaded on).
 // It allocates nothing: no cudaMalloc/cudaFree, no allocating library routine. The array's
 // address is looked up once per device with cudaGetSymbolAddress, with that device
-// current, and cached. What must start at zero (the status word and the fallback count)
+// current, and cached; the logits must be device memory of the current device (checked
+// before any launch). What must start at zero (the status word and the fallback count)
 // spec_verify_chain clears on every call; everything else it writes before reading.
 #include <cuda_runtime.h>
 
@@ -39,16 +40,31 @@ void* device_scratch() {
   return g_scratch_addr[dev];
 }
 
+// True when p is device (or managed) memory of the current device. The scratch is chosen
+// by the current device, so logits on another device would have this call's kernels write
+// the wrong device's array.
+bool on_current_device(const void* p) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) return false;
+  cudaPointerAttributes at = {};
+  if (cudaPointerGetAttributes(&at, p) != cudaSuccess) {
+    cudaGetLastError();  // a failed query leaves a (non-sticky) error behind: clear it
+    return false;
+  }
+  return (at.type == cudaMemoryTypeDevice || at.type == cudaMemoryTypeManaged) && at.device == dev;
+}
+
 }  // namespace
 
 extern "C" spec_status spec_verify_chain_noalloc(
     const void* target_logits, const void* draft_logits, spec_dtype dtype, int B, int K, int V,
     const int32_t* draft_tokens, const float* uniforms, float temp, int top_k, float top_p,
     int32_t* accepted_len, int32_t* out_tokens, void* stream) {
-  if (B <= 0 || K <= 0 || V <= 0) return SPEC_ERR_INVALID_ARG;
+  if (B <= 0 || K <= 0 || V <= 0 || !target_logits) return SPEC_ERR_INVALID_ARG;
   const size_t need = spec_workspace_size(B, K, V);
   if (need == 0) return SPEC_ERR_INVALID_ARG;
   if (need > SPEC_STATIC_SCRATCH_BYTES) return SPEC_ERR_WORKSPACE;  // before any CUDA call
+  if (!on_current_device(target_logits)) return SPEC_ERR_INVALID_ARG;
   void* scratch = device_scratch();
   if (!scratch) return SPEC_ERR_CUDA;
   return spec_verify_chain(target_logits, draft_logits, dtype, B, K, V, draft_tokens, uniforms,

@@ -204,6 +204,9 @@ spec_status spec_residual_sample(const float* p, const float* q, int rows, int V
  *     undefined results. Order them (one stream, or events).
  *   - Make the first call on each device outside any stream capture: it resolves the
  *     array's address, which may load the library's device code.
+ *   - The scratch is the current device's: make the device that holds the tensors current
+ *     before the call. target_logits that is not device (or managed) memory of the current
+ *     device gets SPEC_ERR_INVALID_ARG before any launch.
  *   - spec_get_device_status cannot see this scratch: a row whose copy wait timed out
  *     shows as accepted_len[b] = -2. */
 #define SPEC_STATIC_SCRATCH_BYTES ((size_t)8 << 20)

@@ -121,8 +121,8 @@ def _rand_chain(seed, B, K, V, dtype, sigma=2.0, quant=None, temp=1.0, top_k=0, 
 @pytest.mark.parametrize("dtype", ["bf16", "f32"])
 @pytest.mark.parametrize("V", [1, 2, 17, 1001, 4099, 40000])
 def test_chain_ragged_vocab(dtype, V):
-    """Odd V makes rows start off 16-byte boundaries (plain-load head/tail); large V
-    splits a row over a cluster of CTAs."""
+    """Odd V makes rows start off 16-byte boundaries (plain-load chunk head and tail); large
+    V streams a row as several chunks."""
     B, K = 12, 3
     target, draft, toks, u = _rand_chain(V + (dtype == "f32"), B, K, V, dtype)
     run_case(target, draft, toks, u, 1.0)
@@ -154,7 +154,8 @@ def test_chain_topk_multichunk_trends(dtype, trend, top_k, top_p):
 
 
 def test_chain_sixteen_cta_cluster():
-    """V = 300000 bfloat16 (600 KB rows) spreads each row over a 16-CTA cluster."""
+    """V = 300000 bfloat16 (600 KB rows): ten streamed chunks per row, and the exact finisher
+    (one row per thread-block cluster) for rows the candidates cannot settle."""
     target, draft, toks, u = _rand_chain(3, 3, 2, 300000, "bf16", sigma=3.0)
     run_case(target, draft, toks, u, 1.0, top_k=40)
     run_case(target, draft, toks, u, 1.0, top_p=0.7)

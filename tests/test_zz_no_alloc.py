@@ -65,3 +65,24 @@ def test_noalloc_rejects_a_batch_beyond_its_scratch(cuda_device):
     with pytest.raises(sv.SpecError) as e:
         sv.spec_verify_chain_noalloc(t, d, x, u, 1.0)
     assert e.value.status == sv.SPEC_ERR_WORKSPACE
+
+
+def test_noalloc_rejects_logits_off_the_current_device(cuda_device):
+    """The scratch is the current device's, so logits that are not that device's memory
+    (here: plain host memory) are refused before any launch."""
+    import ctypes
+
+    B, K, V = 2, 2, 64
+    host = np.zeros((B, K + 1, V), np.float32)
+    d = torch.zeros((B, K, V), dtype=torch.float32, device=cuda_device)
+    x = torch.zeros((B, K), dtype=torch.int32, device=cuda_device)
+    u = torch.zeros((B, K + 1), dtype=torch.float32, device=cuda_device)
+    acc = torch.empty(B, dtype=torch.int32, device=cuda_device)
+    out = torch.empty((B, K + 1), dtype=torch.int32, device=cuda_device)
+    torch.cuda.synchronize()
+    rc = sv.lib().spec_verify_chain_noalloc(
+        host.ctypes.data_as(ctypes.c_void_p), ctypes.c_void_p(d.data_ptr()), sv.SPEC_F32, B, K,
+        V, ctypes.c_void_p(x.data_ptr()), ctypes.c_void_p(u.data_ptr()), 1.0, 0, 1.0,
+        ctypes.c_void_p(acc.data_ptr()), ctypes.c_void_p(out.data_ptr()), None)
+    assert rc == sv.SPEC_ERR_INVALID_ARG
+    torch.cuda.synchronize()  # nothing was launched, and the context is healthy
