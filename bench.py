@@ -150,6 +150,155 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples": len(sm)}
 
 
+def _events(n):
+    import torch
+    pairs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+             for _ in range(n)]
+    for a, b in pairs:  # torch creates an event on its first record; the library re-records it
+        a.record()
+        b.record()
+    return pairs
+
+
+def time_calls(step, steps: int, warmup: int):
+    """Device time of `steps` calls of step() after `warmup` untimed ones: (total ms, the
+    row-statistics stage of each call in ms, from the library's timing hook)."""
+    import torch
+
+    import draft_token_verification_spec_b200 as sv
+
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+    pairs = _events(steps)
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    start.record()
+    for i in range(steps):
+        sv.spec_set_row_kernel_events(*pairs[i])
+        step()
+    end.record()
+    torch.cuda.synchronize()
+    sv.spec_set_row_kernel_events(None, None)
+    return start.elapsed_time(end), [a.elapsed_time(b) for a, b in pairs]
+
+
+def roofline_entry(alg: int, row_ms: float, kernel: str = "stream_rows_kernel") -> dict:
+    peaks, peak_src = measured_peaks()
+    achieved = alg / (row_ms / 1e3) / 1e9
+    return {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"],
+            "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4),
+            "peak_source": peak_src + " (STREAM-style copy)",
+            "frac_of_8TBs": round(achieved / 8000.0, 4), "kernel": kernel,
+            "kernel_ms": round(row_ms, 4), "algorithmic_bytes": alg}
+
+
+def chain_device_inputs(cfg, greedy, dev):
+    """Generator logits and uniforms on the device, and drafter tokens x_i ~ transformed q_i
+    (temperature 0: the draft argmax) drawn with the library's own transform and draw."""
+    import torch
+
+    import draft_token_verification_spec_b200 as sv
+
+    target, draft = specgen.chain_logits(cfg)
+    u = specgen.chain_uniforms(cfg)
+    pick = specgen.drafter_uniforms(cfg)
+
+    def to_dev(a):
+        if a.dtype == np.uint16:
+            return torch.from_numpy(a.view(np.int16)).to(dev).view(torch.bfloat16)
+        return torch.from_numpy(a).to(dev)
+
+    tg, dg, ug = to_dev(target), to_dev(draft), to_dev(u)
+    if greedy:
+        xg = dg.float().argmax(dim=2).to(torch.int32).contiguous()
+    else:
+        probs, _ = sv.spec_logits_to_probs(dg, cfg.temp, cfg.top_k, cfg.top_p, with_entropy=False)
+        xg = sv.spec_residual_sample(probs.view(-1, cfg.V), None,
+                                     to_dev(pick).view(-1)).view(cfg.B, cfg.K)
+        del probs
+    torch.cuda.synchronize()
+    return target, draft, u, tg, dg, ug, xg
+
+
+def per_config_chain(cfg, greedy, args, dev) -> dict:
+    """One workload timed like the headline (same steps and warm-up), device-resident
+    inputs, plus the oracle on the host cores over a bounded sample."""
+    import torch
+
+    import draft_token_verification_spec_b200 as sv
+
+    _, _, _, tg, dg, ug, xg = chain_device_inputs(cfg, greedy, dev)
+    temp = 0.0 if greedy else cfg.temp
+    acc = torch.empty(cfg.B, dtype=torch.int32, device=dev)
+    out = torch.empty((cfg.B, cfg.K + 1), dtype=torch.int32, device=dev)
+    ws = torch.empty(sv.spec_workspace_size(cfg.B, cfg.K, cfg.V), dtype=torch.uint8, device=dev)
+
+    def step():
+        sv.spec_verify_chain(tg, None if greedy else dg, xg, ug, temp, cfg.top_k, cfg.top_p,
+                             accepted_len=acc, out_tokens=out, workspace=ws)
+
+    ms, row_ms = time_calls(step, args.steps, args.warmup)
+    accl = acc.cpu().numpy()
+    assert accl.min() >= 0 and sv.spec_get_device_status(ws) == 0, cfg.name
+    row = float(np.mean(row_ms))
+    res = {"workload": workload(cfg, greedy)["workload"], "metric_unit": UNIT,
+           "value": cfg.B * cfg.K * args.steps / (ms / 1e3), "ms_per_step": ms / args.steps,
+           "row_stage_ms": round(row, 4),
+           "roofline": roofline_entry(algorithmic_bytes(cfg, greedy), row),
+           "mean_accepted_len": float(accl.mean())}
+    del tg, dg, ug, xg, ws
+    torch.cuda.empty_cache()
+    if not args.no_cpu_baseline:
+        res["cpu_baseline"] = cpu_baseline(cfg, greedy, budget_s=4.0)
+    return res
+
+
+def tree_streamed_rows(parent) -> int:
+    """Logit rows of one batch row that typical acceptance reads: the rows of nodes with a
+    child (a node's row is read only to test its children)."""
+    par = np.asarray(parent)
+    return int(np.unique(par[1:][(par[1:] >= 0)]).size)
+
+
+def per_config_tree(cfg, args, dev) -> dict:
+    """The MEDUSA-tree workload under typical acceptance: verified positions = B * (N - 1)
+    candidate nodes per call."""
+    import torch
+
+    import draft_token_verification_spec_b200 as sv
+
+    logits, toks, par = specgen.tree_inputs(cfg)
+    lg = torch.from_numpy(logits.view(np.int16)).to(dev).view(torch.bfloat16)
+    tk, pa = torch.from_numpy(toks).to(dev), torch.from_numpy(par).to(dev)
+    path = torch.empty((cfg.B, cfg.N), dtype=torch.int32, device=dev)
+    plen = torch.empty(cfg.B, dtype=torch.int32, device=dev)
+    ws = torch.empty(sv.spec_workspace_size(cfg.B, cfg.N, cfg.V), dtype=torch.uint8, device=dev)
+
+    def step():
+        sv.spec_verify_tree_typical(lg, tk, pa, cfg.eps, cfg.delta, best_path=path,
+                                    accepted_len=plen, workspace=ws)
+
+    ms, row_ms = time_calls(step, args.steps, args.warmup)
+    lens = plen.cpu().numpy()
+    assert lens.min() >= 1 and sv.spec_get_device_status(ws) == 0
+    row = float(np.mean(row_ms))
+    alg = cfg.B * tree_streamed_rows(par) * cfg.V * 2
+    res = {"workload": cfg.name, "metric_unit": UNIT,
+           "value": cfg.B * (cfg.N - 1) * args.steps / (ms / 1e3), "ms_per_step": ms / args.steps,
+           "row_stage_ms": round(row, 4), "roofline": roofline_entry(alg, row),
+           "mean_accepted_len": float(lens.mean())}
+    if not args.no_cpu_baseline:
+        import oracle
+        threads = os.cpu_count() or 1
+        t0 = time.perf_counter()
+        oracle.verify_tree_typical(logits, toks, par, cfg.eps, cfg.delta, threads=threads)
+        dt = time.perf_counter() - t0
+        res["cpu_baseline"] = {"value": cfg.B * (cfg.N - 1) / dt, "unit": UNIT, "cores": threads,
+                               "kind": "oracle",
+                               "sample": f"all {cfg.B} batch rows, {threads} threads, {dt:.2f}s"}
+    return res
+
+
 def run_ours(args, cfg, greedy, rank, world):
     import torch
 
@@ -159,27 +308,8 @@ def run_ours(args, cfg, greedy, rank, world):
     torch.cuda.set_device(dev)
     sv.lib()  # fail loudly if the CUDA library is missing
     t0 = time.time()
-    target, draft = specgen.chain_logits(cfg)
-    u = specgen.chain_uniforms(cfg)
-    pick = specgen.drafter_uniforms(cfg)
+    target, draft, u, tg, dg, ug, xg = chain_device_inputs(cfg, greedy, dev)
     log(f"[rank {rank}] generated inputs in {time.time() - t0:.1f}s")
-
-    def to_dev(a):
-        if a.dtype == np.uint16:
-            return torch.from_numpy(a.view(np.int16)).to(dev).view(torch.bfloat16)
-        return torch.from_numpy(a).to(dev)
-
-    tg, dg, ug = to_dev(target), to_dev(draft), to_dev(u)
-    # the drafter: x_i ~ transformed q_i (temperature 0: argmax), drawn on the GPU with
-    # the library's own transform and draw
-    if greedy:
-        xg = dg.float().argmax(dim=2).to(torch.int32).contiguous()
-    else:
-        probs, _ = sv.spec_logits_to_probs(dg, cfg.temp, cfg.top_k, cfg.top_p, with_entropy=False)
-        xg = sv.spec_residual_sample(probs.view(-1, cfg.V), None,
-                                     to_dev(pick).view(-1)).view(cfg.B, cfg.K)
-        del probs
-    torch.cuda.synchronize()
     temp = 0.0 if greedy else cfg.temp
     acc = torch.empty(cfg.B, dtype=torch.int32, device=dev)
     out = torch.empty((cfg.B, cfg.K + 1), dtype=torch.int32, device=dev)
@@ -197,11 +327,7 @@ def run_ours(args, cfg, greedy, rank, world):
     accl = acc.cpu().numpy()
     assert accl.min() >= 0, "error rows in the benchmark batch"
 
-    pairs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-             for _ in range(args.steps)]
-    for a, b in pairs:  # torch creates an event on its first record; the library re-records it
-        a.record()
-        b.record()
+    pairs = _events(args.steps)
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     clocks = ClockSampler(dev.index)
     if world > 1:
@@ -263,19 +389,11 @@ def run_ours(args, cfg, greedy, rank, world):
     kernels_per_step = 3 if candidates else 2
     row_avg_ms = float(np.mean(row_ms))
     alg = algorithmic_bytes(cfg, greedy)
-    peaks, peak_src = measured_peaks()
     traffic = read_profile_traffic(workload(cfg, greedy)["workload"])
-    achieved = alg / (row_avg_ms / 1e3) / 1e9
+    del h_t, h_d
     return {
         "value": value, "ms_per_step": ms_max / args.steps,
-        "roofline": {"bound": "hbm", "achieved": round(achieved, 1),
-                     "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                     "frac": round(achieved / peaks["hbm_gbs"], 4),
-                     "peak_source": peak_src + " (STREAM-style copy)",
-                     "frac_of_8TBs": round(achieved / 8000.0, 4),
-                     "kernel": "stream_rows_kernel", "kernel_ms": round(row_avg_ms, 4),
-                     "algorithmic_bytes": alg,
-                     "traffic": traffic},
+        "roofline": {**roofline_entry(alg, row_avg_ms), "traffic": traffic},
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": int(h2d),
                 "d2h_bytes_per_step": int(d2h), "steps": e2e_steps},
         "gpu_launches": kernels_per_step * args.steps,
@@ -330,6 +448,21 @@ def cpu_baseline(cfg, greedy, budget_s: float = 15.0) -> dict:
                       f"{threads} threads over batch rows, {dt:.1f}s"}
 
 
+def per_config_all(args) -> list:
+    """Every other workload, one entry each (1 GPU): the three other chain workloads, the
+    temperature-0 variants of the two that have one, and the MEDUSA tree."""
+    import torch
+
+    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", 0)))
+    out = []
+    for cfg, greedy in [(specgen.CFG1, False), (specgen.CFG2, False), (specgen.CFG2, True),
+                        (specgen.CFG3, False), (specgen.CFG5, True)]:
+        out.append(per_config_chain(cfg, greedy, args, dev))
+        log(f"per-config {out[-1]['workload']}: {out[-1]['ms_per_step']:.4f} ms")
+    out.append(per_config_tree(specgen.CFG4, args, dev))
+    return out
+
+
 def run_reference(args, cfg, greedy) -> dict:
     """The oracle, as it stands, on the host cores: each step verifies a bounded sample."""
     import oracle
@@ -374,6 +507,8 @@ def main():
     ap.add_argument("--batch", type=int, default=None,
                     help="override the batch size (smaller cases for profiler captures)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-per-config", action="store_true",
+                    help="time only the headline workload")
     args = ap.parse_args()
     assert args.warmup >= 3, "at least 3 warm-up steps"
     cfg = specgen.CHAIN_CONFIGS[args.config]
@@ -406,6 +541,9 @@ def main():
                     "ms_per_step": res.pop("ms_per_step"), **res}
             if not args.no_cpu_baseline:
                 line["cpu_baseline"] = cpu_baseline(cfg, args.greedy)
+            if world == 1 and not args.no_per_config and args.config == 5 and not args.greedy \
+                    and not args.batch:
+                line["per_config"] = per_config_all(args)
             print(json.dumps(line), flush=True)
     finally:
         if world > 1:

@@ -264,7 +264,7 @@ spec_status verify_tree(const void* target_logits, spec_dtype dtype, int B, int 
   if (!plan_rows(V, elem_bytes(dtype), &pl) || !rows_fit(rows, pl.C)) return SPEC_ERR_UNSUPPORTED;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   int32_t* dev_status = static_cast<int32_t*>(workspace);
-  const WsLayout wl = ws_layout(rows);
+  const WsLayout wl = ws_layout(rows);  // the kept-id area (unused by trees) holds the row map
   char* ws = static_cast<char*>(workspace);
   sv::RowStats* stats = reinterpret_cast<sv::RowStats*>(ws + wl.stats);
   if (cudaMemsetAsync(dev_status, 0, 2 * sizeof(int32_t), s) != cudaSuccess) return SPEC_ERR_CUDA;
@@ -284,6 +284,16 @@ spec_status verify_tree(const void* target_logits, spec_dtype dtype, int B, int 
   rj.flags = greedy ? sv::RS_GREEDY : sv::RS_ENTROPY;
   rj.stats = stats;
   rj.dev_status = dev_status;
+  if (!greedy) {
+    // typical acceptance reads only the rows of nodes with a child (greedy also reads the
+    // deepest accepted node's own row, which may be a leaf): list them on the device
+    int32_t* map = reinterpret_cast<int32_t*>(ws + wl.kept_ids);
+    int32_t* count = dev_status + 2;
+    sv::tree_parent_rows_kernel<<<1, kThreads, 0, s>>>(parent_idx, N, B, map, count);
+    if (cudaGetLastError() != cudaSuccess) return SPEC_ERR_CUDA;
+    rj.row_list = map;
+    rj.row_count = count;
+  }
   void* evb = g_ev_before.load();
   void* eva = g_ev_after.load();
   if (evb) cudaEventRecord(static_cast<cudaEvent_t>(evb), s);
@@ -569,7 +579,7 @@ void spec_set_row_kernel_events(void* before, void* after) {
 int spec_kernels_per_call(const char* entry_point) {
   if (!entry_point) return -1;
   if (!std::strcmp(entry_point, "spec_verify_chain")) return 3;
-  if (!std::strcmp(entry_point, "spec_verify_tree_typical")) return 2;
+  if (!std::strcmp(entry_point, "spec_verify_tree_typical")) return 3;
   if (!std::strcmp(entry_point, "spec_verify_tree_greedy")) return 2;
   if (!std::strcmp(entry_point, "spec_verify_tree_sampling")) return 3;
   if (!std::strcmp(entry_point, "spec_logits_to_probs")) return 1;

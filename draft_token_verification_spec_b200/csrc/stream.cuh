@@ -644,8 +644,12 @@ __global__ void __launch_bounds__(kStreamThreads, (kMode == SM_TOPP ? 2 : 3))
   // top-k: chunks between count exchanges, so that about kCapTopK / 2 entries can arrive
   // between two even when every chunk brings k new ones
   const int xchg_k = kMode == SM_TOPK ? max(1, (kCapTopK / 2) / max(1, rj.top_k)) : 0;
+  // rows [0, rows), or the rows row_list[0 .. *row_count) when a list is given (logical index
+  // lr -> row row_of(lr); statistics and outputs are indexed by the row itself)
+  const long long nrows = rj.row_list ? (long long)*rj.row_count : rj.rows;
+  auto row_of = [&](long long lr) { return rj.row_list ? (long long)rj.row_list[lr] : lr; };
   const long long nrows_mine =
-      rj.rows > blockIdx.x ? (rj.rows - 1 - blockIdx.x) / gridDim.x + 1 : 0;
+      nrows > blockIdx.x ? (nrows - 1 - blockIdx.x) / gridDim.x + 1 : 0;
   const long long items = nrows_mine * nchunk;
 
   if (threadIdx.x == 0) {
@@ -662,7 +666,7 @@ __global__ void __launch_bounds__(kStreamThreads, (kMode == SM_TOPP ? 2 : 3))
   if (threadIdx.x >= kThreads) {
     if (threadIdx.x == kThreads) {
       uint32_t issued = 0, lastpar = 0;
-      long long row = blockIdx.x;
+      long long lr = blockIdx.x, row = nrows_mine > 0 ? row_of(lr) : 0;
       int q = 0, b = 0;
       for (long long g = 0; g < items; ++g) {
         // buffer b last held item g - kRing: wait until every consumer warp is done with it
@@ -681,7 +685,8 @@ __global__ void __launch_bounds__(kStreamThreads, (kMode == SM_TOPP ? 2 : 3))
         lastpar = (lastpar & ~(1u << b)) | (uint32_t((g / kRing) & 1) << b);
         if (++q == nchunk) {
           q = 0;
-          row += gridDim.x;
+          lr += gridDim.x;
+          if (g + 1 < items) row = row_of(lr);
         }
         if (++b == kRing) b = 0;
       }
@@ -716,7 +721,7 @@ __global__ void __launch_bounds__(kStreamThreads, (kMode == SM_TOPP ? 2 : 3))
   bool row_timeout = false;
   int wacc = 0, wlen = 0, xpar = 0;  // count exchange: this warp's appends, chunks, parity
   int single = 0;                    // entries this thread appended one by one
-  long long row = blockIdx.x;
+  long long lr = blockIdx.x, row = nrows_mine > 0 ? row_of(lr) : 0;
   int q = 0, b = 0;
 
   for (long long g = 0; g < items; ++g) {
@@ -1049,7 +1054,8 @@ __global__ void __launch_bounds__(kStreamThreads, (kMode == SM_TOPP ? 2 : 3))
     if (++b == kRing) b = 0;
     if (++q == nchunk) {
       q = 0;
-      row += gridDim.x;
+      lr += gridDim.x;
+      if (g + 1 < items) row = row_of(lr);
     }
   }
 }

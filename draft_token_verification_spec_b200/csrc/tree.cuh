@@ -33,6 +33,40 @@ struct TreeJob {
 
 enum : int8_t { ND_REJECT = 0, ND_ACCEPT = 1, ND_ERROR = 2, ND_TIMEOUT = 3 };
 
+constexpr int kTreeMaxNodes = 4096;  // SPEC_MAX_TREE_NODES
+
+// Typical acceptance reads a node's row only to test the node's children, so only rows of
+// nodes with a child are streamed. One block lists them for every batch row, parents in
+// index order: map[b * P + j] = b * N + (j-th node with a child), *count = B * P. Malformed
+// parent entries are skipped here (the finisher rejects the tree).
+__global__ void __launch_bounds__(kThreads)
+    tree_parent_rows_kernel(const int32_t* parent, int N, int B, int32_t* map, int32_t* count) {
+  __shared__ uint8_t has_child[kTreeMaxNodes];
+  __shared__ int32_t plist[kTreeMaxNodes];
+  __shared__ uint32_t scr[kWarps];
+  for (int c = threadIdx.x; c < N; c += kThreads) has_child[c] = 0;
+  __syncthreads();
+  for (int c = 1 + threadIdx.x; c < N; c += kThreads) {
+    const int pa = parent[c];
+    if (pa >= 0 && pa < c) has_child[pa] = 1;
+  }
+  __syncthreads();
+  int P = 0;
+  for (int base = 0; base < N; base += kThreads) {
+    const int c = base + int(threadIdx.x);
+    const uint32_t f = (c < N && has_child[c]) ? 1u : 0u;
+    uint32_t total;
+    const uint32_t pos = block_exclusive_scan<uint32_t>(f, scr, &total);
+    if (f) plist[P + int(pos)] = c;
+    P += int(total);
+  }
+  __syncthreads();
+  const long long n = (long long)B * P;
+  for (long long i = threadIdx.x; i < n; i += kThreads)
+    map[i] = int32_t((i / P) * N + plist[i % P]);
+  if (threadIdx.x == 0) *count = int32_t(n);
+}
+
 template <typename T>
 __global__ void __launch_bounds__(kThreads) tree_finish_kernel(const TreeJob j) {
   extern __shared__ __align__(16) unsigned char tsm[];

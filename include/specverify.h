@@ -114,7 +114,8 @@ spec_status spec_verify_chain(const void* target_logits, const void* draft_logit
  *   accepted_len  [B] int32 out: nodes on the path, root included (>= 1).
  * Node c >= 1 is accepted iff its parent is and p(tok_c) > min(eps, delta *
  * exp(-H(p))), with p = softmax of the parent's row (temperature 1) and H its entropy
- * in nats; the deepest accepted node wins, the lowest node index on ties.
+ * in nats; the deepest accepted node wins, the lowest node index on ties. Only the rows
+ * of nodes that have a child are read (a leaf's row is never inspected).
  * 1 <= N <= SPEC_MAX_TREE_NODES, eps and delta finite. */
 spec_status spec_verify_tree_typical(const void* target_logits, spec_dtype dtype, int B, int N,
                                      int V, const int32_t* node_tokens,
@@ -229,7 +230,8 @@ void spec_set_row_kernel_events(void* before, void* after);
 
 /* Largest number of kernels one call enqueues (for launch accounting): the row
  * statistics kernel, the exact finisher for rows it lists (chain calls with top-k or
- * top-p only) and the per-batch-row kernel. -1 for an unknown name. */
+ * top-p only), the per-batch-row kernel, and for typical acceptance the kernel that lists
+ * the rows of nodes with a child. -1 for an unknown name. */
 int spec_kernels_per_call(const char* entry_point);
 
 #ifdef __cplusplus

@@ -284,6 +284,22 @@ def test_tree_invalid_inputs():
     assert np.all(one[1] == 1) and np.all(one[0][:, 0] == 0)
 
 
+def test_tree_leaf_rows_are_never_read():
+    """Typical acceptance streams only the rows of nodes with a child: NaN or +inf in every
+    leaf's row leaves the result unchanged (the rule never reads a leaf's row)."""
+    cfg = specgen.CFG4
+    logits, toks, par = specgen.tree_inputs(
+        specgen.TreeConfig(**{**cfg.__dict__, "coverage_boost": 6.0}), 6)
+    leaves = np.setdiff1d(np.arange(cfg.N), par[1:])
+    bad = logits.copy()
+    bad[:, leaves, 5] = 0x7FC0     # NaN
+    bad[:, leaves, 9] = 0x7F80     # +inf
+    path_g, len_g = gpu_tree(bad, toks, par, cfg.eps, cfg.delta)
+    path_r, len_r, _ = oracle.verify_tree_typical(logits, toks, par, cfg.eps, cfg.delta)
+    assert np.array_equal(len_g, len_r) and np.array_equal(path_g, path_r)
+    assert len_g.min() >= 1
+
+
 # ------------------------------------------------------------------ greedy tree (multi-branch)
 
 def assert_tree_greedy_parity(logits, toks, par, path_cap=None):

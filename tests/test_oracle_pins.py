@@ -679,3 +679,87 @@ def test_T8_monte_carlo_first_token_frequencies():
     counts = np.bincount(out[:, 0], minlength=V)
     p1 = softmax(t[0].astype(np.float64))
     assert chisquare(counts, p1 * B).pvalue > 1e-4
+
+
+# --------------------------------------------------------------------------- explicit-row draw
+
+def _ln(x):
+    return math.log(x) if x > 0 else None
+
+
+def test_residual_sample_validity_rule():
+    """The explicit-probability draw ("Speculative Sampling": resample from norm(max(0, p - q)))
+    takes probabilities: an entry outside [0, 1] or NaN, in p or in q, or a p with no positive
+    mass, gives token -1; every other row gives a token (hand-derived cases)."""
+    V = 4
+    good = [0.5, 0.25, 0.25, 0.0]
+    rows_p = [good, [1.5, 0.0, 0.0, 0.0], [0.5, -0.25, 0.5, 0.25], [0.5, math.nan, 0.25, 0.25],
+              [0.0, 0.0, 0.0, 0.0], good, good]
+    rows_q = [good, good, good, good, good, [0.25, 1.25, 0.0, 0.0], [0.25, math.nan, 0.0, 0.0]]
+    p = np.array(rows_p, np.float32)
+    q = np.array(rows_q, np.float32)
+    u = np.full(len(rows_p), 0.25, np.float32)
+    tok, _ = oracle.residual_sample(p, q, u)
+    # row 0: p == q, empty residual, falls back to p: w*S = 0.25 < C_0 = 0.5 -> token 0
+    assert tok.tolist() == [0, -1, -1, -1, -1, -1, -1]
+    tok_p, _ = oracle.residual_sample(p, None, u)          # q absent: only p is checked
+    assert tok_p.tolist() == [0, -1, -1, -1, -1, 0, 0]
+
+
+@pytest.mark.parametrize("w,expect", [(0.4, 0), (0.5, 2), (0.6, 2), (0.0, 0), (0.999, 2)])
+def test_residual_sample_dyadic_golden(w, expect):
+    """p = (1/2, 1/4, 1/4, 0), q = (1/4, 1/4, 0, 1/2): max(0, p - q) = (1/4, 0, 1/4, 0),
+    S = 1/2. The smallest id whose cumulative mass exceeds w*S: C_0 = 1/4, C_2 = 1/2, so
+    w*S < 1/4 (w < 1/2) gives token 0 and w >= 1/2 gives token 2 (strict '>' at the edge)."""
+    p = np.array([[0.5, 0.25, 0.25, 0.0]], np.float32)
+    q = np.array([[0.25, 0.25, 0.0, 0.5]], np.float32)
+    tok, _ = oracle.residual_sample(p, q, np.array([w], np.float32))
+    assert int(tok[0]) == expect
+
+
+# --------------------------------------------------------------------------- top-p near ties
+
+def _near_tie_case(x0, draft0):
+    """K = 1, V = 4, top_p = 0.75. Target row 0 is p = (4, 2, 1, 1)/8: the two largest
+    tokens hold exactly 0.75, so the nucleus {0, 1} sits on the top-p boundary (one more
+    token, 2, on the other side). Target row 1 (the bonus) is (1, 2, 3, 10)/16, whose
+    nucleus {3, 2} is far from the boundary (0.8125 and 0.625). u = (0, 0.3)."""
+    target = f32_logits([[_ln(4), _ln(2), 0.0, 0.0], [0.0, _ln(2), _ln(3), _ln(10)]])[None]
+    draft = f32_logits([draft0])[None]
+    toks = np.array([[x0]], np.int32)
+    u = np.array([[0.0, 0.3]], np.float32)
+    return oracle.verify_chain(target, draft, toks, u, 1.0, 0, 0.75)
+
+
+def test_topp_near_tie_flags_only_when_the_other_nucleus_changes_the_output():
+    """A top-p boundary within the precision window flags a row only if evaluating the row
+    with the other nucleus (one token more or fewer) changes its output ("Speculative
+    Sampling": the transform decides p and q before the ratio test)."""
+    # x = 2 lies outside {0, 1} but inside {0, 1, 2}; q = (1, 1, 14)/16 keeps {2}, q(2) = 1.
+    # Nucleus {0, 1}: p(2) = 0, r = 0, u = 0 is not < 0 -> reject, redraw from p.
+    # Nucleus {0, 1, 2}: p(2) = 1/7 > 0 -> accept, bonus token. Different outputs: flagged.
+    acc, out, flags = _near_tie_case(2, [0.0, 0.0, _ln(14), None])
+    assert int(flags[0]) & oracle.FLAG_TOPP
+    assert int(acc[0]) == 0 and int(out[0, 0]) in (0, 1)
+    # x = 0 lies inside both nuclei; q = (14, 1, 1)/16 keeps {0}, q(0) = 1, r = 2/3 or 4/7,
+    # u = 0 accepts either way; the bonus draw from (3, 10)/13 at w = 0.3 gives token 3
+    # (C_2 = 3/13 < 0.3). Same output: not flagged.
+    acc, out, flags = _near_tie_case(0, [_ln(14), 0.0, 0.0, None])
+    assert int(flags[0]) & oracle.PARITY_FLAGS == 0
+    assert int(acc[0]) == 1 and out[0].tolist() == [0, 3]
+
+
+def test_topp_near_tie_below_the_boundary_tries_one_token_fewer():
+    """Cumulative mass just below top_p before the crossing token (p = (4, 2, 1, 1)/8,
+    top_p = 0.75 + 5e-7: {0, 1} holds 0.75, so the nucleus is {0, 1, 2} with the boundary
+    5e-7 away). The alternative nucleus {0, 1} drops token 2: a draft x = 2 accepted with
+    {0, 1, 2} is rejected with {0, 1}, so the row is flagged; x = 0 is not."""
+    target = f32_logits([[_ln(4), _ln(2), 0.0, 0.0], [0.0, _ln(2), _ln(3), _ln(10)]])[None]
+    u = np.array([[0.0, 0.3]], np.float32)
+    top_p = 0.75 + 5e-7
+    d2 = f32_logits([[0.0, 0.0, _ln(14), None]])[None]
+    acc, out, flags = oracle.verify_chain(target, d2, np.array([[2]], np.int32), u, 1.0, 0, top_p)
+    assert int(acc[0]) == 1 and int(flags[0]) & oracle.FLAG_TOPP
+    d0 = f32_logits([[_ln(14), 0.0, 0.0, None]])[None]
+    acc, out, flags = oracle.verify_chain(target, d0, np.array([[0]], np.int32), u, 1.0, 0, top_p)
+    assert int(acc[0]) == 1 and int(flags[0]) & oracle.PARITY_FLAGS == 0
