@@ -6,8 +6,15 @@
 // The whole block then draws the emitted token: from norm(max(0, p_a - q_a)) after a
 // rejection at a (p_a if that residual is empty), from p_K when all K drafts were
 // accepted. When the row of p_a lists its kept ids (top-k rows), the draw runs over
-// that support only: the residual and p both vanish outside it. "Speculative Decoding" and "Speculative Sampling" (spec-decoding-i notes);
-// greedy longest-prefix verification from blockwise parallel decoding ("推测解码").
+// that support only: the residual and p both vanish outside it. "Speculative Decoding"
+// and "Speculative Sampling" (spec-decoding-i notes); greedy longest-prefix verification
+// from blockwise parallel decoding ("推测解码").
+//
+// The ratio tests and the draw are taken in double precision: p(v) = exp((l_v - m) / T) / zd
+// over the kept set, zd the double normaliser of the row statistics. A row whose statistics
+// carry no zd (untruncated rows, rows the exact finisher settled) has it summed here, by the
+// whole block, the first time the scan reaches it. The draw's masses are doubles summed as
+// exact 128-bit fixed point.
 #pragma once
 
 #include "draw.cuh"
@@ -27,11 +34,13 @@ struct ChainJob {
   const int32_t* kept_n;  // [rows] or NULL: ids listed per row (0: none)
   const int32_t* kept_ids;  // [rows][kKeptCap]
   int greedy;
+  float temp;             // the temperature as given (sampling)
   int32_t* accepted_len;  // [B]
   int32_t* out_tokens;    // [B][K+1]
 };
 
-enum : int { EV_ACCEPT = 0, EV_STOP = 1, EV_ERROR = 2, EV_TIMEOUT = 3 };
+// EV_NEEDZ: the test at this position needs a normaliser that the block must sum first.
+enum : int { EV_ACCEPT = 0, EV_STOP = 1, EV_ERROR = 2, EV_TIMEOUT = 3, EV_NEEDZ = 4 };
 
 __device__ __forceinline__ int row_event(const RowStats& s) {
   return s.status == ROW_OK ? EV_ACCEPT : (s.status == ROW_TIMEOUT ? EV_TIMEOUT : EV_ERROR);
@@ -40,7 +49,8 @@ __device__ __forceinline__ int row_event(const RowStats& s) {
 template <typename T>
 __global__ void __launch_bounds__(kThreads) chain_finish_kernel(const ChainJob j) {
   __shared__ DrawSmem sm;
-  __shared__ int s_a, s_ev;
+  __shared__ int s_a, s_ev, s_zpos;
+  __shared__ double s_z[2];  // zd of p and q at position s_zpos, summed by the block
   const int b = blockIdx.x;
   const int K = j.K, V = j.V;
   const RowStats* ts = j.stats + size_t(b) * (K + 1);
@@ -49,53 +59,78 @@ __global__ void __launch_bounds__(kThreads) chain_finish_kernel(const ChainJob j
   const T* drow0 = j.greedy ? nullptr : static_cast<const T*>(j.draft) + size_t(b) * K * V;
   const int32_t* x = j.tokens + size_t(b) * K;
   const float* u = j.uniforms + size_t(b) * (K + 1);
+  const double Tt = double(j.temp);
+  if (threadIdx.x == 0) s_zpos = -1;
+  __syncthreads();
 
-  if (threadIdx.x < 32) {
-    const int lane = threadIdx.x;
-    int a = -1, ev = EV_STOP;
-    for (int base = 0; base <= K && a < 0; base += 32) {
-      const int i = base + lane;
-      int e = EV_ACCEPT;
-      if (i <= K) {
-        const RowStats sp = ts[i];
-        e = row_event(sp);
-        if (e == EV_ACCEPT) {
-          if (i == K) {
-            e = EV_STOP;
-          } else {
-            const int xi = x[i];
-            if (xi < 0 || xi >= V) {
-              e = EV_ERROR;
-            } else if (j.greedy) {
-              e = (xi == sp.argmax) ? EV_ACCEPT : EV_STOP;
+  for (int start = 0;;) {
+    if (threadIdx.x < 32) {
+      const int lane = threadIdx.x;
+      const int zpos = s_zpos;
+      int a = -1, ev = EV_STOP;
+      for (int base = start; base <= K && a < 0; base += 32) {
+        const int i = base + lane;
+        int e = EV_ACCEPT;
+        if (i <= K) {
+          const RowStats sp = ts[i];
+          e = row_event(sp);
+          if (e == EV_ACCEPT) {
+            if (i == K) {
+              e = EV_STOP;
             } else {
-              const RowStats sq = ds[i];
-              e = row_event(sq);
-              if (e == EV_ACCEPT) {
-                const float lp = Elem<T>::load(trow0, size_t(i) * V + xi);
-                const float lq = Elem<T>::load(drow0, size_t(i) * V + xi);
-                const float p = prob<T>(sp, lp, xi);
-                const float q = prob<T>(sq, lq, xi);
-                const float r = q > 0.0f ? p / q : (p > 0.0f ? INFINITY : 0.0f);
-                e = (u[i] < fminf(1.0f, r)) ? EV_ACCEPT : EV_STOP;
+              const int xi = x[i];
+              if (xi < 0 || xi >= V) {
+                e = EV_ERROR;
+              } else if (j.greedy) {
+                e = (xi == sp.argmax) ? EV_ACCEPT : EV_STOP;
+              } else {
+                const RowStats sq = ds[i];
+                e = row_event(sq);
+                if (e == EV_ACCEPT) {
+                  const double zp = i == zpos ? s_z[0] : sp.zd;
+                  const double zq = i == zpos ? s_z[1] : sq.zd;
+                  if (zp < 0.0 || zq < 0.0) {
+                    e = EV_NEEDZ;
+                  } else {
+                    const float lp = Elem<T>::load(trow0, size_t(i) * V + xi);
+                    const float lq = Elem<T>::load(drow0, size_t(i) * V + xi);
+                    const double p = prob_d<T>(sp, zp, Tt, lp, xi);
+                    const double q = prob_d<T>(sq, zq, Tt, lq, xi);
+                    const double r = q > 0.0 ? p / q : (p > 0.0 ? double(INFINITY) : 0.0);
+                    e = (double(u[i]) < fmin(1.0, r)) ? EV_ACCEPT : EV_STOP;
+                  }
+                }
               }
             }
           }
         }
+        const unsigned stop = __ballot_sync(0xffffffffu, i <= K && e != EV_ACCEPT);
+        if (stop) {
+          const int L = __ffs(stop) - 1;
+          a = base + L;
+          ev = __shfl_sync(0xffffffffu, e, L);
+        }
       }
-      const unsigned stop = __ballot_sync(0xffffffffu, i <= K && e != EV_ACCEPT);
-      if (stop) {
-        const int L = __ffs(stop) - 1;
-        a = base + L;
-        ev = __shfl_sync(0xffffffffu, e, L);
+      if (lane == 0) {
+        s_a = a;
+        s_ev = ev;
       }
     }
-    if (lane == 0) {
-      s_a = a;
-      s_ev = ev;
+    __syncthreads();
+    if (s_ev != EV_NEEDZ) break;
+    // the first position still to test lacks a normaliser: the block sums it, then the
+    // scan resumes there (the positions before it are accepted)
+    const int i = s_a;
+    const double zp = row_zd<T>(ts[i], trow0 + size_t(i) * V, V, Tt, sm.scr);
+    const double zq = row_zd<T>(ds[i], drow0 + size_t(i) * V, V, Tt, sm.scr);
+    if (threadIdx.x == 0) {
+      s_z[0] = zp;
+      s_z[1] = zq;
+      s_zpos = i;
     }
+    start = i;
+    __syncthreads();
   }
-  __syncthreads();
   const int a = s_a, ev = s_ev;
   int32_t* out = j.out_tokens + size_t(b) * (K + 1);
   if (ev != EV_STOP) {
@@ -113,53 +148,62 @@ __global__ void __launch_bounds__(kThreads) chain_finish_kernel(const ChainJob j
     const float w = u[K];
     const size_t prow_idx = size_t(b) * (K + 1) + a;
     const int nk = j.kept_n ? j.kept_n[prow_idx] : 0;
+    // the normalisers the test at a used (the bonus draw needs none: it scales by its total)
+    const double zp = a < K ? (a == s_zpos ? s_z[0] : sp.zd) : 1.0;
     tok = -1;
     if (nk > 0 && nk <= kSparseCap) {
       const int32_t* ids = j.kept_ids + prow_idx * kKeptCap;
       if (a < K) {
         const RowStats sq = ds[a];
+        const double zq = a == s_zpos ? s_z[1] : sq.zd;
         const T* qrow = drow0 + size_t(a) * V;
         tok = sparse_draw(
             ids, nk,
             [&](int v) {
-              const float d = prob<T>(sp, Elem<T>::load(prow, size_t(v)), v) -
-                              prob<T>(sq, Elem<T>::load(qrow, size_t(v)), v);
-              return to_fx(fmaxf(d, 0.0f));
+              const double d = prob_d<T>(sp, zp, Tt, Elem<T>::load(prow, size_t(v)), v) -
+                               prob_d<T>(sq, zq, Tt, Elem<T>::load(qrow, size_t(v)), v);
+              return fx_from(fmax(d, 0.0));
             },
             w, sm);
       }
       if (tok < 0)
         tok = sparse_draw(
-            ids, nk, [&](int v) { return to_fx(prob<T>(sp, Elem<T>::load(prow, size_t(v)), v)); },
+            ids, nk,
+            [&](int v) {
+              return fx_from(kept_weight_d<T>(sp, Tt, Elem<T>::load(prow, size_t(v)), v));
+            },
             w, sm);
     } else {
       if (a < K) {
         const RowStats sq = ds[a];
+        const double zq = a == s_zpos ? s_z[1] : sq.zd;
         const T* qrow = drow0 + size_t(a) * V;
         const bool qal = (reinterpret_cast<uintptr_t>(qrow) & 15u) == 0;
         tok = inverse_cdf_draw(
-            [&](int v0, unsigned long long* r) {
+            [&](int v0, Fx128* r) {
               float lp[8], lq[8];
               load8<T>(prow, v0, V, pal, lp);
               load8<T>(qrow, v0, V, qal, lq);
 #pragma unroll
               for (int k = 0; k < 8; ++k) {
                 const int v = v0 + k;
-                const float d = (v < V) ? prob<T>(sp, lp[k], v) - prob<T>(sq, lq[k], v) : 0.0f;
-                r[k] = to_fx(fmaxf(d, 0.0f));
+                const double d = (v < V) ? prob_d<T>(sp, zp, Tt, lp[k], v) -
+                                               prob_d<T>(sq, zq, Tt, lq[k], v)
+                                         : 0.0;
+                r[k] = fx_from(fmax(d, 0.0));
               }
             },
             V, w, sm);
       }
       if (tok < 0) {  // bonus position, or an empty residual: draw from p
         tok = inverse_cdf_draw(
-            [&](int v0, unsigned long long* r) {
+            [&](int v0, Fx128* r) {
               float lp[8];
               load8<T>(prow, v0, V, pal, lp);
 #pragma unroll
               for (int k = 0; k < 8; ++k) {
                 const int v = v0 + k;
-                r[k] = (v < V) ? to_fx(prob<T>(sp, lp[k], v)) : 0ull;
+                r[k] = (v < V) ? fx_from(kept_weight_d<T>(sp, Tt, lp[k], v)) : fx_zero();
               }
             },
             V, w, sm);

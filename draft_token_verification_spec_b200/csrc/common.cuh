@@ -29,6 +29,10 @@ enum : int32_t { ROW_OK = 0, ROW_INVALID = 1, ROW_TIMEOUT = 2, ROW_FALLBACK = 3 
 // with c = log2(e) / T and mc = fl(m * c), m the largest logit. thr_key = 0 keeps every
 // row entry. The rounding of mc scales every weight of the row by the same factor, so
 // it cancels in p.
+//
+// The decisions of the sampling rule (the ratio test, the residual and bonus draws) use the
+// double-precision view of the same distribution: p(v) = kept(v) ? exp((l_v - m) / T) / zd : 0,
+// with zd the double sum over the kept set (zd < 0: not computed here; the consumer sums it).
 struct RowStats {
   float mc;          // fl(m * c), m the largest logit
   float z;           // sum over the kept set of exp2((l - m) * c)
@@ -38,8 +42,11 @@ struct RowStats {
   int32_t argmax;    // lowest id holding the largest logit
   int32_t status;    // ROW_OK / ROW_INVALID / ROW_TIMEOUT
   float c;           // log2(e) / T
+  float m;           // the largest logit (exact)
+  int32_t pad;
+  double zd;         // sum over the kept set of exp((l - m) / T) in double, or -1
 };
-static_assert(sizeof(RowStats) == 32, "RowStats is 32 bytes");
+static_assert(sizeof(RowStats) == 48, "RowStats is 48 bytes");
 
 // ------------------------------------------------------------------------- keys
 // Order-preserving unsigned key of a float value (larger value -> larger key);
@@ -173,6 +180,59 @@ __device__ __forceinline__ void limb_add(uint32_t* l, int n, int b, unsigned lon
 __device__ __forceinline__ unsigned long long limb_get(const uint32_t* l, int n, int b) {
   return (unsigned long long)l[b] + ((unsigned long long)l[n + b] << 15) +
          ((unsigned long long)l[2 * n + b] << 30);
+}
+
+// ------------------------------------------------------------------------- exact wide sums
+// Nonnegative doubles below 2^27 as unsigned 128-bit fixed point with 100 fraction bits.
+// Conversion drops only what lies below 2^-100; sums of converted values are exact, so they
+// do not depend on the order of the terms (deterministic reductions over lists that arrive
+// in any order), and 2^20 terms below 1 each stay far below the range.
+struct Fx128 {
+  unsigned long long lo, hi;
+};
+__device__ __forceinline__ Fx128 fx_zero() { return Fx128{0ull, 0ull}; }
+__device__ __forceinline__ Fx128 fx_add(Fx128 a, Fx128 b) {
+  Fx128 r;
+  r.lo = a.lo + b.lo;
+  r.hi = a.hi + b.hi + (r.lo < a.lo ? 1ull : 0ull);
+  return r;
+}
+__device__ __forceinline__ bool fx_is_zero(Fx128 a) { return (a.lo | a.hi) == 0ull; }
+// x in [0, 2^27): x * 2^100 truncated to an integer.
+__device__ __forceinline__ Fx128 fx_from(double x) {
+  const unsigned long long bits = static_cast<unsigned long long>(__double_as_longlong(x));
+  const int E = int((bits >> 52) & 0x7FFu);
+  if (E == 0 || (bits >> 63)) return fx_zero();  // zero, subnormal (< 2^-1022) or negative
+  const unsigned long long m = (bits & ((1ull << 52) - 1ull)) | (1ull << 52);
+  const int sh = E - 975;  // x * 2^100 = m * 2^(E - 1075 + 100)
+  Fx128 r;
+  if (sh >= 64) {
+    r.hi = m << (sh - 64);
+    r.lo = 0ull;
+  } else if (sh > 0) {
+    r.hi = m >> (64 - sh);
+    r.lo = m << sh;
+  } else if (sh > -64) {
+    r.hi = 0ull;
+    r.lo = m >> (-sh);
+  } else {
+    r = fx_zero();
+  }
+  return r;
+}
+__device__ __forceinline__ double fx_to_double(Fx128 a) {
+  return ldexp(double(a.hi), -36) + ldexp(double(a.lo), -100);
+}
+__device__ __forceinline__ Fx128 fx_shfl_xor(Fx128 a, int o) {
+  return Fx128{__shfl_xor_sync(0xffffffffu, a.lo, o), __shfl_xor_sync(0xffffffffu, a.hi, o)};
+}
+__device__ __forceinline__ Fx128 fx_shfl_up(Fx128 a, int o) {
+  return Fx128{__shfl_up_sync(0xffffffffu, a.lo, o), __shfl_up_sync(0xffffffffu, a.hi, o)};
+}
+__device__ __forceinline__ Fx128 warp_sum_fx(Fx128 v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fx_add(v, fx_shfl_xor(v, o));
+  return v;
 }
 
 // ------------------------------------------------------------------------- PTX: bulk copies
@@ -313,6 +373,45 @@ __device__ __forceinline__ U block_exclusive_scan(U v, U* scratch, U* total) {
   }
   *total = all;
   return before + inc - v;
+}
+
+// Block-wide sum of Fx128 (all threads get it); scratch holds kWarps entries.
+__device__ __forceinline__ Fx128 block_sum_fx(Fx128 v, Fx128* scratch) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  v = warp_sum_fx(v);
+  __syncthreads();
+  if (lane == 0) scratch[warp] = v;
+  __syncthreads();
+  Fx128 t = fx_zero();
+#pragma unroll
+  for (int w = 0; w < kWarps; ++w) t = fx_add(t, scratch[w]);
+  return t;
+}
+
+// Block-wide exclusive prefix sum of Fx128 in thread order; *total = the sum.
+__device__ __forceinline__ Fx128 block_exclusive_scan_fx(Fx128 v, Fx128* scratch, Fx128* total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  Fx128 inc = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const Fx128 n = fx_shfl_up(inc, o);
+    if (lane >= o) inc = fx_add(inc, n);
+  }
+  __syncthreads();
+  if (lane == 31) scratch[warp] = inc;
+  __syncthreads();
+  Fx128 before = fx_zero(), all = fx_zero();
+#pragma unroll
+  for (int w = 0; w < kWarps; ++w) {
+    if (w < warp) before = fx_add(before, scratch[w]);
+    all = fx_add(all, scratch[w]);
+  }
+  *total = all;
+  // inclusive - v, computed as before + (inc - v) without a subtraction: scan of the
+  // exclusive within-warp prefix
+  Fx128 ex = fx_shfl_up(inc, 1);
+  if (lane == 0) ex = fx_zero();
+  return fx_add(before, ex);
 }
 
 // (max value, lowest index) combine; NaN never reaches it (rows with NaN are invalid).

@@ -1,6 +1,7 @@
 // Inverse-CDF draw from explicit probability rows: norm(max(0, p - q)), or p when q
 // is absent or the residual is empty ("Speculative Sampling", spec-decoding-i notes).
-// One thread block per row; the same deterministic draw as chain verification.
+// One thread block per row; the same deterministic draw as chain verification, on the
+// exact double differences of the float inputs.
 #pragma once
 
 #include "draw.cuh"
@@ -40,22 +41,22 @@ __global__ void __launch_bounds__(kThreads) residual_sample_kernel(const Residua
   int tok = -1;
   if (qr) {
     tok = inverse_cdf_draw(
-        [&](int v0, unsigned long long* r) {
+        [&](int v0, Fx128* r) {
 #pragma unroll
           for (int k = 0; k < 8; ++k) {
             const int v = v0 + k;
-            r[k] = (v < V) ? to_fx(fmaxf(pr[v] - qr[v], 0.0f)) : 0ull;
+            r[k] = (v < V) ? fx_from(fmax(double(pr[v]) - double(qr[v]), 0.0)) : fx_zero();
           }
         },
         V, w, sm);
   }
   if (tok < 0) {
     tok = inverse_cdf_draw(
-        [&](int v0, unsigned long long* r) {
+        [&](int v0, Fx128* r) {
 #pragma unroll
           for (int k = 0; k < 8; ++k) {
             const int v = v0 + k;
-            r[k] = (v < V) ? to_fx(pr[v]) : 0ull;
+            r[k] = (v < V) ? fx_from(double(pr[v])) : fx_zero();
           }
         },
         V, w, sm);

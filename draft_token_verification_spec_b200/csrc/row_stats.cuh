@@ -54,6 +54,7 @@ struct RowJob {
   int slice_bytes;     // bytes reserved per slice buffer (multiple of 128)
   float c;             // log2(e) / T   (unused in greedy mode)
   float inv_t;         // 1 / T
+  float temp;          // T as given (the double-precision view uses it)
   int top_k;           // 1 <= top_k < V, else off
   float top_p;         // < 1: on
   int flags;
@@ -65,6 +66,8 @@ struct RowJob {
   int32_t* dev_status; // set to 1 on a copy timeout (may be NULL)
   const int32_t* row_list;   // if set: process rows row_list[0 .. *row_count) only
   const int32_t* row_count;
+  int32_t* refine_rows;      // if set: top-p rows whose boundary is re-decided in double
+  int32_t* refine_count;
 };
 
 struct __align__(16) RowAux {
@@ -836,6 +839,9 @@ __device__ void process_row(RowCtx<T>& ctx, const RowJob& job, long long row, bo
     }
   }
   if (!listed && job.kept_n && rank == 0 && threadIdx.x == 0) job.kept_n[row] = 0;
+  // a top-p boundary this kernel placed with fp32 masses: re-decided in double afterwards
+  if (status == ROW_OK && topp && !topk && job.refine_rows && rank == 0 && threadIdx.x == 0)
+    job.refine_rows[atomicAdd(job.refine_count, 1)] = int32_t(row);
 
   const double Z = double(zfx) * kFxInv;
   const double ent = (status == ROW_OK && !greedy && want_ent)
@@ -852,6 +858,9 @@ __device__ void process_row(RowCtx<T>& ctx, const RowJob& job, long long row, bo
     st.argmax = greedy ? am : -1;
     st.status = status;
     st.c = c;
+    st.m = m;
+    st.pad = 0;
+    st.zd = -1.0;  // the consumer sums the double normaliser when it needs it
     job.stats[row] = st;
   }
   if (job.flags & RS_WRITE_PROBS) {

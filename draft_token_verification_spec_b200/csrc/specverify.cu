@@ -9,6 +9,7 @@
 
 #include "chain.cuh"
 #include "probs.cuh"
+#include "refine.cuh"
 #include "row_stats.cuh"
 #include "specverify.h"
 #include "stream.cuh"
@@ -189,11 +190,48 @@ cudaError_t launch_stream(const sv::StreamJob& job, int mode, cudaStream_t s) {
   }
 }
 
+// Blocks of the top-p refinement: one per SM (each walks the listed rows).
+template <typename T>
+cudaError_t launch_refine(const sv::RefineJob& j, cudaStream_t s) {
+  static std::mutex mu;
+  static std::map<int, int> sms_of;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  int sms = 0;
+  {
+    std::lock_guard<std::mutex> lock(mu);
+    auto it = sms_of.find(dev);
+    if (it != sms_of.end()) sms = it->second;
+  }
+  if (sms == 0) {
+    e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return e;
+    std::lock_guard<std::mutex> lock(mu);
+    sms_of[dev] = sms;
+  }
+  const size_t dyn = size_t(sv::kRefineCap) * sizeof(uint64_t);
+  e = cudaFuncSetAttribute(sv::topp_refine_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           int(dyn));
+  if (e != cudaSuccess) return e;
+  const long long g = j.r.rows < sms ? j.r.rows : sms;
+  sv::topp_refine_kernel<T><<<unsigned(g), kThreads, dyn, s>>>(j);
+  return cudaGetLastError();
+}
+
 // Row statistics for a verify call. The streaming kernel settles the rows it can; in the
 // candidate modes it lists the rest, which the cluster kernel then finishes exactly. A
-// top-k above the candidate path's limit goes to the cluster kernel for every row.
-cudaError_t row_stage(spec_dtype dt, const sv::RowJob& rj, const RowPlan& pl, int32_t* fb_rows,
-                      int32_t* fb_count, cudaStream_t s) {
+// top-k above the candidate path's limit goes to the cluster kernel for every row. Pure
+// top-p rows whose boundary was placed with fp32 masses too close to call (and every top-p
+// row the cluster kernel settled) then get it placed again in double precision
+// (refine_rows, when given).
+cudaError_t row_stage(spec_dtype dt, sv::RowJob rj, const RowPlan& pl, int32_t* fb_rows,
+                      int32_t* fb_count, int32_t* refine_rows, int32_t* refine_count,
+                      int32_t* unresolved, cudaStream_t s) {
+  const bool refine = refine_rows && rj.top_p < 1.0f && rj.top_k == 0 &&
+                      !(rj.flags & sv::RS_GREEDY);
+  rj.refine_rows = refine ? refine_rows : nullptr;
+  rj.refine_count = refine ? refine_count : nullptr;
   const int mode = stream_mode(rj);
   if (mode == sv::SM_TOPK && rj.top_k > sv::kStreamMaxTopK)
     return launch_row_stats_dt(dt, rj, pl, s);
@@ -213,7 +251,14 @@ cudaError_t row_stage(spec_dtype dt, const sv::RowJob& rj, const RowPlan& pl, in
   sv::RowJob fj = rj;
   fj.row_list = fb_rows;
   fj.row_count = fb_count;
-  return launch_row_stats_dt(dt, fj, pl, s);
+  e = launch_row_stats_dt(dt, fj, pl, s);
+  if (e != cudaSuccess || !refine) return e;
+  sv::RefineJob rf = {};
+  rf.r = rj;
+  rf.rows = refine_rows;
+  rf.count = refine_count;
+  rf.unresolved = unresolved;
+  return dt == SPEC_BF16 ? launch_refine<__nv_bfloat16>(rf, s) : launch_refine<float>(rf, s);
 }
 
 int elem_bytes(spec_dtype dt) { return dt == SPEC_BF16 ? 2 : 4; }
@@ -222,11 +267,14 @@ bool dtype_ok(int dt) { return dt == SPEC_F32 || dt == SPEC_BF16; }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-// Workspace: [header: status word, fallback count | RowStats per row | kept-id count per
-// row | kept ids per row | fallback row list].
+// Workspace: [header | RowStats per row | kept-id count per row | kept ids per row |
+// fallback row list | refinement row list]. Header words (int32): 0 the device status,
+// 1 the fallback count, 2 the tree row-list count, 3 the refinement count, 4 rows left
+// unrefined; the rest of the 256 bytes is unused.
 struct WsLayout {
-  size_t stats, kept_n, kept_ids, fb_rows, total;
+  size_t stats, kept_n, kept_ids, fb_rows, refine_rows, total;
 };
+constexpr int kHeaderWords = 5;
 
 size_t up256(size_t x) { return (x + 255) / 256 * 256; }
 
@@ -236,7 +284,8 @@ WsLayout ws_layout(long long rows) {
   w.kept_n = w.stats + up256(size_t(rows) * sizeof(sv::RowStats));
   w.kept_ids = w.kept_n + up256(size_t(rows) * sizeof(int32_t));
   w.fb_rows = w.kept_ids + up256(size_t(rows) * sv::kKeptCap * sizeof(int32_t));
-  w.total = w.fb_rows + up256(size_t(rows) * sizeof(int32_t));
+  w.refine_rows = w.fb_rows + up256(size_t(rows) * sizeof(int32_t));
+  w.total = w.refine_rows + up256(size_t(rows) * sizeof(int32_t));
   return w;
 }
 
@@ -267,7 +316,8 @@ spec_status verify_tree(const void* target_logits, spec_dtype dtype, int B, int 
   const WsLayout wl = ws_layout(rows);  // the kept-id area (unused by trees) holds the row map
   char* ws = static_cast<char*>(workspace);
   sv::RowStats* stats = reinterpret_cast<sv::RowStats*>(ws + wl.stats);
-  if (cudaMemsetAsync(dev_status, 0, 2 * sizeof(int32_t), s) != cudaSuccess) return SPEC_ERR_CUDA;
+  if (cudaMemsetAsync(dev_status, 0, kHeaderWords * sizeof(int32_t), s) != cudaSuccess)
+    return SPEC_ERR_CUDA;
 
   sv::RowJob rj = {};
   rj.base0 = target_logits;
@@ -279,6 +329,7 @@ spec_status verify_tree(const void* target_logits, spec_dtype dtype, int B, int 
   rj.slice_bytes = pl.slice_bytes;
   rj.c = greedy ? 0.0f : sv::kLog2e;
   rj.inv_t = greedy ? 0.0f : 1.0f;
+  rj.temp = 1.0f;
   rj.top_k = 0;
   rj.top_p = 1.0f;
   rj.flags = greedy ? sv::RS_GREEDY : sv::RS_ENTROPY;
@@ -297,8 +348,8 @@ spec_status verify_tree(const void* target_logits, spec_dtype dtype, int B, int 
   void* evb = g_ev_before.load();
   void* eva = g_ev_after.load();
   if (evb) cudaEventRecord(static_cast<cudaEvent_t>(evb), s);
-  if (row_stage(dtype, rj, pl, reinterpret_cast<int32_t*>(ws + wl.fb_rows), dev_status + 1, s) !=
-      cudaSuccess)
+  if (row_stage(dtype, rj, pl, reinterpret_cast<int32_t*>(ws + wl.fb_rows), dev_status + 1,
+                nullptr, nullptr, nullptr, s) != cudaSuccess)
     return SPEC_ERR_CUDA;
   if (eva) cudaEventRecord(static_cast<cudaEvent_t>(eva), s);
 
@@ -369,7 +420,8 @@ spec_status spec_verify_chain(const void* target_logits, const void* draft_logit
   const WsLayout wl = ws_layout(rows);
   char* ws = static_cast<char*>(workspace);
   sv::RowStats* stats = reinterpret_cast<sv::RowStats*>(ws + wl.stats);
-  if (cudaMemsetAsync(dev_status, 0, 2 * sizeof(int32_t), s) != cudaSuccess) return SPEC_ERR_CUDA;
+  if (cudaMemsetAsync(dev_status, 0, kHeaderWords * sizeof(int32_t), s) != cudaSuccess)
+    return SPEC_ERR_CUDA;
 
   sv::RowJob rj = {};
   rj.kept_n = reinterpret_cast<int32_t*>(ws + wl.kept_n);
@@ -383,6 +435,7 @@ spec_status spec_verify_chain(const void* target_logits, const void* draft_logit
   rj.slice_bytes = pl.slice_bytes;
   rj.c = greedy ? 0.0f : sv::kLog2e / temp;
   rj.inv_t = greedy ? 0.0f : 1.0f / temp;
+  rj.temp = temp;
   rj.top_k = (top_k >= 1 && top_k < V) ? top_k : 0;
   rj.top_p = top_p < 1.0f ? top_p : 1.0f;
   rj.flags = greedy ? sv::RS_GREEDY : 0;
@@ -391,8 +444,9 @@ spec_status spec_verify_chain(const void* target_logits, const void* draft_logit
   void* evb = g_ev_before.load();
   void* eva = g_ev_after.load();
   if (evb) cudaEventRecord(static_cast<cudaEvent_t>(evb), s);
-  if (row_stage(dtype, rj, pl, reinterpret_cast<int32_t*>(ws + wl.fb_rows), dev_status + 1, s) !=
-      cudaSuccess)
+  if (row_stage(dtype, rj, pl, reinterpret_cast<int32_t*>(ws + wl.fb_rows), dev_status + 1,
+                reinterpret_cast<int32_t*>(ws + wl.refine_rows), dev_status + 3, dev_status + 4,
+                s) != cudaSuccess)
     return SPEC_ERR_CUDA;
   if (eva) cudaEventRecord(static_cast<cudaEvent_t>(eva), s);
 
@@ -408,6 +462,7 @@ spec_status spec_verify_chain(const void* target_logits, const void* draft_logit
   cj.kept_n = rj.kept_n;
   cj.kept_ids = rj.kept_ids;
   cj.greedy = greedy ? 1 : 0;
+  cj.temp = temp;
   cj.accepted_len = accepted_len;
   cj.out_tokens = out_tokens;
   if (dtype == SPEC_BF16)
@@ -461,7 +516,8 @@ spec_status spec_verify_tree_sampling(const void* target_logits, const void* dra
   const WsLayout wl = ws_layout(rows);
   char* ws = static_cast<char*>(workspace);
   sv::RowStats* stats = reinterpret_cast<sv::RowStats*>(ws + wl.stats);
-  if (cudaMemsetAsync(dev_status, 0, 2 * sizeof(int32_t), s) != cudaSuccess) return SPEC_ERR_CUDA;
+  if (cudaMemsetAsync(dev_status, 0, kHeaderWords * sizeof(int32_t), s) != cudaSuccess)
+    return SPEC_ERR_CUDA;
 
   sv::RowJob rj = {};
   rj.kept_n = reinterpret_cast<int32_t*>(ws + wl.kept_n);
@@ -475,6 +531,7 @@ spec_status spec_verify_tree_sampling(const void* target_logits, const void* dra
   rj.slice_bytes = pl.slice_bytes;
   rj.c = greedy ? 0.0f : sv::kLog2e / temp;
   rj.inv_t = greedy ? 0.0f : 1.0f / temp;
+  rj.temp = temp;
   rj.top_k = (top_k >= 1 && top_k < V) ? top_k : 0;
   rj.top_p = top_p < 1.0f ? top_p : 1.0f;
   rj.flags = greedy ? sv::RS_GREEDY : 0;
@@ -483,8 +540,9 @@ spec_status spec_verify_tree_sampling(const void* target_logits, const void* dra
   void* evb = g_ev_before.load();
   void* eva = g_ev_after.load();
   if (evb) cudaEventRecord(static_cast<cudaEvent_t>(evb), s);
-  if (row_stage(dtype, rj, pl, reinterpret_cast<int32_t*>(ws + wl.fb_rows), dev_status + 1, s) !=
-      cudaSuccess)
+  if (row_stage(dtype, rj, pl, reinterpret_cast<int32_t*>(ws + wl.fb_rows), dev_status + 1,
+                reinterpret_cast<int32_t*>(ws + wl.refine_rows), dev_status + 3, dev_status + 4,
+                s) != cudaSuccess)
     return SPEC_ERR_CUDA;
   if (eva) cudaEventRecord(static_cast<cudaEvent_t>(eva), s);
 
@@ -501,11 +559,12 @@ spec_status spec_verify_tree_sampling(const void* target_logits, const void* dra
   tj.kept_n = rj.kept_n;
   tj.kept_ids = rj.kept_ids;
   tj.greedy = greedy ? 1 : 0;
+  tj.temp = temp;
   tj.best_path = best_path;
   tj.path_cap = path_cap;
   tj.accepted_len = accepted_len;
   tj.next_token = next_token;
-  const size_t dyn = size_t(N) * 16 + 16;  // child lists, path, normalisers
+  const size_t dyn = size_t(N) * 20 + 16;  // normalisers (double), child lists, path
   cudaError_t e;
   if (dtype == SPEC_BF16) {
     e = cudaFuncSetAttribute(sv::tree_sample_kernel<__nv_bfloat16>,
@@ -540,6 +599,7 @@ spec_status spec_logits_to_probs(const void* logits, spec_dtype dtype, int rows,
   rj.slice_bytes = pl.slice_bytes;
   rj.c = greedy ? 0.0f : sv::kLog2e / temp;
   rj.inv_t = greedy ? 0.0f : 1.0f / temp;
+  rj.temp = temp;
   rj.top_k = (top_k >= 1 && top_k < V) ? top_k : 0;
   rj.top_p = top_p < 1.0f ? top_p : 1.0f;
   rj.flags = sv::RS_WRITE_PROBS | (greedy ? sv::RS_GREEDY : 0) |
@@ -578,10 +638,10 @@ void spec_set_row_kernel_events(void* before, void* after) {
 
 int spec_kernels_per_call(const char* entry_point) {
   if (!entry_point) return -1;
-  if (!std::strcmp(entry_point, "spec_verify_chain")) return 3;
+  if (!std::strcmp(entry_point, "spec_verify_chain")) return 4;
   if (!std::strcmp(entry_point, "spec_verify_tree_typical")) return 3;
   if (!std::strcmp(entry_point, "spec_verify_tree_greedy")) return 2;
-  if (!std::strcmp(entry_point, "spec_verify_tree_sampling")) return 3;
+  if (!std::strcmp(entry_point, "spec_verify_tree_sampling")) return 4;
   if (!std::strcmp(entry_point, "spec_logits_to_probs")) return 1;
   if (!std::strcmp(entry_point, "spec_residual_sample")) return 1;
   return -1;

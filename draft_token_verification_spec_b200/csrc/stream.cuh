@@ -59,7 +59,9 @@
 #pragma once
 
 #include <climits>
+#include <cstddef>
 
+#include "draw.cuh"
 #include "row_stats.cuh"
 
 namespace sv {
@@ -116,6 +118,11 @@ constexpr float kBinScale = 32.0f;              // bins per log2 unit of weight
 constexpr int kMemberCap = 512;                 // members of the crossing bin
 constexpr int kRankMax = 1024;                  // lists this short are ranked directly
 constexpr int kStreamMaxTopK = kKeptCap;        // top-k the candidate path takes
+// Top-p: a bound on the error, relative to the row's total mass, of the fp32 masses that
+// place the nucleus boundary (each weight: the exponent's rounding and the rounding of
+// log2(e)/T, ex2.approx, the per-vector fp32 sum; the tail below 2^-24 of the maximum holds
+// at most V * 2^-24 of it). A boundary within it is re-decided in double precision.
+constexpr float kToppGuard = 6e-6f;
 
 // Dynamic shared memory of one CTA: the ring, then top-k: the candidate list and the top k
 // in rank order; top-p: the candidate list, the bin counts and the bin masses as 15-bit
@@ -146,7 +153,7 @@ struct __align__(16) StreamAux {
   uint64_t empty[kMaxRing];  // completes when the eight consumer warps are done with it
   float red_f[2][kWarps];  // count exchange, double-buffered by exchange parity
   int red_i[2][kWarps];
-  unsigned long long scr_u64[kWarps];
+  unsigned long long scr_u64[kWarps];  // scr_u64 and scr_s64 together also hold kWarps Fx128
   long long scr_s64[kWarps];
   double scr_f64[kWarps];
   float scr_f[kWarps];
@@ -154,6 +161,8 @@ struct __align__(16) StreamAux {
   uint32_t scr_u32[kWarps];
   unsigned long long sel_before;
   unsigned long long sel_comp;
+  unsigned long long sel_mabove;  // resolve: mass of the crossing bin's members above it
+  unsigned long long sel_mw;      // resolve: the crossing member's own mass
   uint32_t sel_cnt;
   int sel_bin;
   int sel_found;
@@ -161,6 +170,10 @@ struct __align__(16) StreamAux {
   int mcount;
   int broken;   // a copy or buffer wait timed out: the CTA stops reading rows
 };
+
+__device__ __forceinline__ Fx128* scr_fx(StreamAux& a) { return reinterpret_cast<Fx128*>(a.scr_u64); }
+static_assert(offsetof(StreamAux, scr_s64) == offsetof(StreamAux, scr_u64) + 8 * kWarps,
+              "scr_u64 and scr_s64 are adjacent");
 
 // Three top-k CTAs per SM: ring, list, ranked top k, this record and the 1 KB the hardware
 // reserves per CTA, within the SM's 228 KB.
@@ -233,6 +246,43 @@ __device__ __forceinline__ U cscan(U v, U* scr, U* total) {
   }
   *total = all;
   return before + inc - v;
+}
+
+// Fx128 sum over the consumer threads (all of them get it).
+__device__ __forceinline__ Fx128 creduce_fx(Fx128 v, Fx128* scr) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  v = warp_sum_fx(v);
+  csync();
+  if (lane == 0) scr[warp] = v;
+  csync();
+  Fx128 t = scr[0];
+#pragma unroll
+  for (int w = 1; w < kWarps; ++w) t = fx_add(t, scr[w]);
+  return t;
+}
+
+// Exclusive Fx128 prefix sum over the consumer threads in thread order; *total = the sum.
+__device__ __forceinline__ Fx128 cscan_fx(Fx128 v, Fx128* scr, Fx128* total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  Fx128 inc = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const Fx128 n = fx_shfl_up(inc, o);
+    if (lane >= o) inc = fx_add(inc, n);
+  }
+  csync();
+  if (lane == 31) scr[warp] = inc;
+  csync();
+  Fx128 before = fx_zero(), all = fx_zero();
+#pragma unroll
+  for (int w = 0; w < kWarps; ++w) {
+    if (w < warp) before = fx_add(before, scr[w]);
+    all = fx_add(all, scr[w]);
+  }
+  *total = all;
+  Fx128 ex = fx_shfl_up(inc, 1);
+  if (lane == 0) ex = fx_zero();
+  return fx_add(before, ex);
 }
 
 // Counts into hist[bin] with one shared atomic per distinct bin per warp; every lane of
@@ -423,7 +473,11 @@ struct CandSet {
       unsigned long long above = 0;
       for (int j = 0; j < m; ++j)
         if (mem[j] > ei) above += mw[j];
-      if (above < need && need <= above + mw[i]) aux->sel_comp = ei;
+      if (above < need && need <= above + mw[i]) {
+        aux->sel_comp = ei;
+        aux->sel_mabove = above;
+        aux->sel_mw = mw[i];
+      }
     }
     csync();
     return aux->sel_comp != 0;
@@ -507,9 +561,9 @@ struct CandSet {
 
   // Top-k lists (n <= kRankMax): the top k of cand[0..n) (k <= kThreads) in rank order, then
   // the one where the mass accumulated from the top first reaches top_p of their total ->
-  // aux->sel_comp. The caller has synchronised the list, and read aux->sel_comp if it needs
-  // it, before the call.
-  __device__ bool rank_topp(int n, int k, float top_p, float c, float mc) {
+  // aux->sel_comp, with the weights exp((l - m) / T) in double summed exactly. The caller has
+  // synchronised the list, and read aux->sel_comp if it needs it, before the call.
+  __device__ bool rank_topp(int n, int k, float top_p, float m, double Tt) {
     for (int i = threadIdx.x; i < n; i += kThreads) {
       const uint64_t e = cand[i];
       int above = 0;
@@ -520,12 +574,12 @@ struct CandSet {
     csync();
     const bool mine = int(threadIdx.x) < k;
     const uint64_t e = mine ? ranked[threadIdx.x] : 0ull;
-    const unsigned long long w = mine ? to_fx(weight(key_value<T>(comp_key(e)), c, mc)) : 0ull;
-    unsigned long long z;
-    const unsigned long long ex = cscan<unsigned long long>(w, aux->scr_u64, &z);
-    unsigned long long target = (unsigned long long)ceil(double(top_p) * double(z));
-    if (target < 1) target = 1;
-    if (mine && ex < target && target <= ex + w) aux->sel_comp = e;
+    const Fx128 w = mine ? fx_from(weight_d(key_value<T>(comp_key(e)), m, Tt)) : fx_zero();
+    Fx128 z;
+    const Fx128 ex = cscan_fx(w, scr_fx(*aux), &z);
+    const double target = double(top_p) * fx_to_double(z);
+    if (mine && fx_to_double(ex) < target && target <= fx_to_double(fx_add(ex, w)))
+      aux->sel_comp = e;
     csync();
     return aux->sel_comp != 0;
   }
@@ -539,6 +593,11 @@ struct RowAcc {
   int am;     // greedy: lowest index holding mt
   float mct;  // fl(mt * c): the online sums are relative to it
   float s, h; // online weight sum and entropy term (log2 units)
+  // top-p: the online weight sum as 42-bit fixed point. Each vector's eight weights are
+  // summed in fp32 and added exactly, and a new maximum rescales the sum in double by the
+  // exact power of two between the two references, so the sum's error stays within a few
+  // fp32 roundings per weight (the bound the top-p decision's guard relies on).
+  unsigned long long sfx;
 
   __device__ void reset() {
     mt = -INFINITY;
@@ -546,12 +605,15 @@ struct RowAcc {
     mct = 0.0f;
     s = 0.0f;
     h = 0.0f;
+    sfx = 0ull;
   }
 
   // Raises the running maximum to vm (> mt), rescaling the online sums.
   __device__ __forceinline__ void raise_max(float vm, float c) {
     const float nm = vm * c;
-    if (s != 0.0f || h != 0.0f) {
+    if constexpr (kMode == SM_TOPP) {
+      if (sfx) sfx = __double2ull_rn(double(sfx) * exp2(double(mct) - double(nm)));
+    } else if (s != 0.0f || h != 0.0f) {
       const float d = nm - mct;  // > 0
       const float scale = ex2(-d);
       h = scale * (h - d * s);
@@ -563,8 +625,12 @@ struct RowAcc {
   __device__ __forceinline__ void add(float x, float c, bool want_ent) {
     const float zx = wexp(x, c, mct);
     const float e = ex2(zx);
-    s += e;
-    if (want_ent) h += ent_term(e, zx);
+    if constexpr (kMode == SM_TOPP) {
+      sfx += to_fx(e);
+    } else {
+      s += e;
+      if (want_ent) h += ent_term(e, zx);
+    }
   }
 
   // One 16-byte vector whose first element has row index j0 (entries outside the chunk
@@ -591,7 +657,15 @@ struct RowAcc {
       if (vm > mt) raise_max(vm, c);
       float x[P];
       Elem<T>::unpack(w, x);
-      if (want_ent) {
+      if (kMode == SM_TOPP) {
+        float s1 = 0.0f, s2 = 0.0f;
+#pragma unroll
+        for (int k = 0; k < P; k += 2) {
+          s1 += ex2(wexp(x[k], c, mct));
+          s2 += ex2(wexp(x[k + 1], c, mct));
+        }
+        sfx += to_fx(s1 + s2);
+      } else if (want_ent) {
 #pragma unroll
         for (int k = 0; k < P; ++k) add(x[k], c, true);
       } else {
@@ -701,6 +775,7 @@ __global__ void __launch_bounds__(kStreamThreads, (kMode == SM_TOPP ? 2 : 3))
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const bool want_ent = (rj.flags & RS_ENTROPY) != 0;
   const float c = rj.c;
+  const double Tt = double(rj.temp);
   CandSet<T> cs;
   cs.cand = reinterpret_cast<uint64_t*>(smem + size_t(kRing) * kRingBufBytes);
   if (kMode == SM_TOPK) {
@@ -943,6 +1018,7 @@ __global__ void __launch_bounds__(kStreamThreads, (kMode == SM_TOPP ? 2 : 3))
       int cutoff = INT_MAX, am = -1;
       unsigned long long zfx = 0;
       double S1 = 0.0;
+      double zd = -1.0;  // the double normaliser, where the kept set is in the list
       bool listed = false;
       if constexpr (kMode == SM_GREEDY) {
         if (status == ROW_OK)
@@ -968,17 +1044,17 @@ __global__ void __launch_bounds__(kStreamThreads, (kMode == SM_TOPP ? 2 : 3))
             ok = ok && n >= rj.top_k;
             if (ok) {  // every list is short (kCapTopK <= kRankMax): rank directly
               if (rj.top_p < 1.0f) {  // the top-p crossing within the top k
-                ok = cs.rank_topp(n, rj.top_k, rj.top_p, c, mc);
+                ok = cs.rank_topp(n, rj.top_k, rj.top_p, m, Tt);
               } else {
                 ok = cs.rank_select(n, 0, rj.top_k);
               }
               cstar = aux.sel_comp;
             }
           } else {  // top-p over the whole row: the mass target from the online sums
-            float sc = 0.0f;
-            if (st.s != 0.0f) sc = ex2(-(mc - st.mct)) * st.s;
-            const unsigned long long zall =
-                creduce<unsigned long long>(to_fx(sc), aux.scr_u64, OpSum());
+            const unsigned long long zt =
+                st.sfx ? __double2ull_rn(double(st.sfx) * exp2(double(st.mct) - double(mc)))
+                       : 0ull;
+            const unsigned long long zall = creduce<unsigned long long>(zt, aux.scr_u64, OpSum());
             unsigned long long target =
                 (unsigned long long)ceil(double(rj.top_p) * double(zall));
             if (target < 1) target = 1;
@@ -987,6 +1063,16 @@ __global__ void __launch_bounds__(kStreamThreads, (kMode == SM_TOPP ? 2 : 3))
               cs.hist_find(target, true);  // not found: the candidates hold too little mass
               ok = aux.sel_found && cs.resolve(n, 0, c, mc, true, target - aux.sel_before);
               cstar = aux.sel_comp;
+              if (ok && rj.refine_rows) {
+                // the fp32 masses before and through the crossing; within the guard of the
+                // target the decision goes to the double-precision refinement
+                const unsigned long long before = aux.sel_before + aux.sel_mabove;
+                const unsigned long long through = before + aux.sel_mw;
+                const unsigned long long g =
+                    (unsigned long long)ceil(double(kToppGuard) * double(zall)) + 1ull;
+                if ((target - before <= g || through - target <= g) && threadIdx.x == 0)
+                  rj.refine_rows[atomicAdd(rj.refine_count, 1)] = int32_t(row);
+              }
             }
           }
           if (!ok) {
@@ -998,18 +1084,22 @@ __global__ void __launch_bounds__(kStreamThreads, (kMode == SM_TOPP ? 2 : 3))
             csync();
             unsigned long long z = 0;
             long long s1 = 0;
+            Fx128 zdx = fx_zero();
             for (int i = threadIdx.x; i < n; i += kThreads) {
               const uint64_t e = cs.cand[i];
               if (e < cstar) continue;
-              const float zx = wexp(key_value<T>(comp_key(e)), c, mc);
+              const float xv = key_value<T>(comp_key(e));
+              const float zx = wexp(xv, c, mc);
               const float ex = ex2(zx);
               z += to_fx(ex);
+              zdx = fx_add(zdx, fx_from(weight_d(xv, m, Tt)));
               if (want_ent) s1 += __float2ll_rn(ent_term(ex, zx) * kS1Fx);
               if (list) {
                 const int slot = atomicAdd(&aux.mcount, 1);
                 if (slot < kKeptCap) rj.kept_ids[size_t(row) * kKeptCap + slot] = comp_id(e);
               }
             }
+            zd = fx_to_double(creduce_fx(zdx, scr_fx(aux)));
             zfx = creduce<unsigned long long>(z, aux.scr_u64, OpSum());
             S1 = double(creduce<long long>(s1, aux.scr_s64, OpSum())) / double(kS1Fx);
             thr_key = comp_key(cstar);
@@ -1035,6 +1125,9 @@ __global__ void __launch_bounds__(kStreamThreads, (kMode == SM_TOPP ? 2 : 3))
         rs.argmax = am;
         rs.status = status;
         rs.c = c;
+        rs.m = m;
+        rs.pad = 0;
+        rs.zd = status == ROW_OK ? zd : -1.0;
         rj.stats[row] = rs;
       }
       // the next row starts clean

@@ -11,6 +11,11 @@
 // unconditionally. The deepest accepted node (lowest index on ties) and its
 // root-first ancestor chain are written out; in greedy mode also the argmax of the deepest
 // node's row, the token the round emits after the path.
+//
+// The typical test is taken with the fp32 row statistics. A test whose p lies within
+// kTreeGuard (relative) of its threshold, a margin well above the fp32 statistics' error,
+// is taken again in double precision: the block sums exp(l - m) and exp(l - m) * (m - l)
+// over the parent's row exactly (Fx128), giving p and the entropy in double.
 #pragma once
 
 #include "draw.cuh"
@@ -31,7 +36,13 @@ struct TreeJob {
   int32_t* next_token;       // [B] or NULL (greedy mode)
 };
 
-enum : int8_t { ND_REJECT = 0, ND_ACCEPT = 1, ND_ERROR = 2, ND_TIMEOUT = 3 };
+enum : int8_t { ND_REJECT = 0, ND_ACCEPT = 1, ND_ERROR = 2, ND_TIMEOUT = 3, ND_NEAR = 4 };
+
+// Relative distance of p from the typical threshold below which the test is re-taken in
+// double precision. The fp32 statistics err by far less: per-thread fp32 sums of at most
+// V / 256 + 16 terms (2^-24 each), ex2.approx and exponent roundings; they move p by under
+// 3e-4 relative and the entropy by under 3e-3 for V <= 2^20.
+constexpr float kTreeGuard = 3e-2f;
 
 constexpr int kTreeMaxNodes = 4096;  // SPEC_MAX_TREE_NODES
 
@@ -101,13 +112,45 @@ __global__ void __launch_bounds__(kThreads) tree_finish_kernel(const TreeJob j) 
           const float l = Elem<T>::load(rows, size_t(pa) * V + tk);
           const float p = prob<T>(s, l, tk);
           const float thr = fminf(j.eps, j.delta * expf(-s.entropy));
-          t = p > thr ? ND_ACCEPT : ND_REJECT;
+          t = fabsf(p - thr) <= kTreeGuard * thr ? ND_NEAR : (p > thr ? ND_ACCEPT : ND_REJECT);
         }
       }
     }
     test[c] = t;
   }
   __syncthreads();
+  if (!j.greedy) {  // tests too close to call in fp32: again in double, one at a time
+    __shared__ Fx128 zscr[kWarps];
+    for (int c = 1; c < N; ++c) {
+      if (test[c] != ND_NEAR) continue;  // uniform: test[] is in shared memory
+      const int pa = par[c];
+      const RowStats s = st[pa];
+      const T* prow = rows + size_t(pa) * V;
+      const bool al = (reinterpret_cast<uintptr_t>(prow) & 15u) == 0;
+      Fx128 z = fx_zero(), h = fx_zero();
+      for (int v0 = int(threadIdx.x) * 8; v0 < V; v0 += kThreads * 8) {
+        float x[8];
+        load8<T>(prow, v0, V, al, x);
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          if (v0 + k >= V || !(x[k] > -INFINITY)) continue;
+          const double d = double(s.m) - double(x[k]);  // >= 0, exact
+          const double e = exp(-d);
+          z = fx_add(z, fx_from(e));
+          h = fx_add(h, fx_from(e * d));
+        }
+      }
+      const double zd = fx_to_double(block_sum_fx(z, zscr));
+      const double hd = fx_to_double(block_sum_fx(h, zscr));
+      if (threadIdx.x == 0) {
+        const double H = log(zd) + hd / zd;  // -sum p ln p
+        const double p = exp(double(Elem<T>::load(prow, size_t(tok[c]))) - double(s.m)) / zd;
+        const double thr = fmin(double(j.eps), double(j.delta) * exp(-H));
+        test[c] = p > thr ? ND_ACCEPT : ND_REJECT;
+      }
+      __syncthreads();
+    }
+  }
   int32_t* path = j.best_path + size_t(b) * j.path_cap;
   __shared__ int s_len, s_err;
   if (threadIdx.x == 0) {

@@ -10,7 +10,9 @@
 // recursion r_j(v) = max(0, r_(j-1)(v) - q_n(v)) / z_j. An accepted child becomes the current
 // node; when none is accepted the emitted token is drawn from r by the inverse CDF with
 // u[N]. In the greedy limit the first child whose token is the argmax of p_n is accepted and
-// the emitted token is that argmax.
+// the emitted token is that argmax. The tests, the residual chain and the draw are taken in
+// double precision (p(v) = exp((l_v - m) / T) / zd over the kept set, masses summed as exact
+// 128-bit fixed point).
 #pragma once
 
 #include "chain.cuh"
@@ -28,6 +30,7 @@ struct TreeSampleJob {
   const int32_t* kept_n;    // [2*B*N] or NULL: ids listed per row (0: none)
   const int32_t* kept_ids;  // [rows][kKeptCap]
   int greedy;
+  float temp;               // the temperature as given (sampling)
   int32_t* best_path;       // [B][path_cap]
   int path_cap;
   int32_t* accepted_len;    // [B]
@@ -38,10 +41,11 @@ template <typename T>
 __global__ void __launch_bounds__(kThreads) tree_sample_kernel(const TreeSampleJob j) {
   extern __shared__ __align__(16) unsigned char tsm[];
   const int N = j.N, V = j.V, b = blockIdx.x;
-  int32_t* kstart = reinterpret_cast<int32_t*>(tsm);  // [N+1] children of n: kids[kstart[n]..)
+  double* zs = reinterpret_cast<double*>(tsm);        // [N] normalisers of the residual chain
+  int32_t* kstart = reinterpret_cast<int32_t*>(zs + N);  // [N+1] children of n: kids[kstart[n]..)
   int32_t* kids = kstart + N + 1;                      // [N]
   int32_t* path = kids + N;                            // [N] nodes on the accepted path
-  float* zs = reinterpret_cast<float*>(path + N);      // [N] normalisers of the residual chain
+  const double Tt = double(j.temp);
   __shared__ DrawSmem sm;
   __shared__ int s_bad;
   const int32_t* par = j.parent;
@@ -101,12 +105,15 @@ __global__ void __launch_bounds__(kThreads) tree_sample_kernel(const TreeSampleJ
           break;
         }
       }
+      // the double normalisers of p_n and (with children) q_n; every thread gets them
+      const double zp = row_zd<T>(sp, prow, V, Tt, sm.scr);
+      const double zq = k1 > k0 ? row_zd<T>(sq, qrow, V, Tt, sm.scr) : 1.0;
       int nrej = 0;
       // the current residual at v: the recursion over the rejections so far
-      auto resid = [&](int v, float pv, float qv) {
-        float r = pv;
+      auto resid = [&](double pv, double qv) {
+        double r = pv;
         for (int i = 0; i < nrej; ++i)
-          if (zs[i] > 0.0f) r = fmaxf(r - qv, 0.0f) / zs[i];
+          if (zs[i] > 0.0) r = fmax(r - qv, 0.0) / zs[i];
         return r;
       };
       for (int i = k0; i < k1 && next < 0; ++i) {
@@ -116,32 +123,32 @@ __global__ void __launch_bounds__(kThreads) tree_sample_kernel(const TreeSampleJ
           err = EV_ERROR;
           break;
         }
-        const float px = prob<T>(sp, Elem<T>::load(prow, size_t(x)), x);
-        const float qx = prob<T>(sq, Elem<T>::load(qrow, size_t(x)), x);
-        const float rx = resid(x, px, qx);
-        const float ratio = qx > 0.0f ? rx / qx : (rx > 0.0f ? INFINITY : 0.0f);
-        if (u[c] < fminf(1.0f, ratio)) {
+        const double px = prob_d<T>(sp, zp, Tt, Elem<T>::load(prow, size_t(x)), x);
+        const double qx = prob_d<T>(sq, zq, Tt, Elem<T>::load(qrow, size_t(x)), x);
+        const double rx = resid(px, qx);
+        const double ratio = qx > 0.0 ? rx / qx : (rx > 0.0 ? double(INFINITY) : 0.0);
+        if (double(u[c]) < fmin(1.0, ratio)) {
           next = c;
           break;
         }
         // rejected: the normaliser of max(0, r - q) over the row
-        unsigned long long zsum = 0;
+        Fx128 zsum = fx_zero();
         if (sparse) {
           for (int t = threadIdx.x; t < nk; t += kThreads) {
             const int v = ids[t];
-            const float pv = prob<T>(sp, Elem<T>::load(prow, size_t(v)), v);
-            const float qv = prob<T>(sq, Elem<T>::load(qrow, size_t(v)), v);
-            zsum += to_fx(fmaxf(resid(v, pv, qv) - qv, 0.0f));
+            const double pv = prob_d<T>(sp, zp, Tt, Elem<T>::load(prow, size_t(v)), v);
+            const double qv = prob_d<T>(sq, zq, Tt, Elem<T>::load(qrow, size_t(v)), v);
+            zsum = fx_add(zsum, fx_from(fmax(resid(pv, qv) - qv, 0.0)));
           }
         } else {
           for (int v = threadIdx.x; v < V; v += kThreads) {
-            const float pv = prob<T>(sp, Elem<T>::load(prow, size_t(v)), v);
-            const float qv = prob<T>(sq, Elem<T>::load(qrow, size_t(v)), v);
-            zsum += to_fx(fmaxf(resid(v, pv, qv) - qv, 0.0f));
+            const double pv = prob_d<T>(sp, zp, Tt, Elem<T>::load(prow, size_t(v)), v);
+            const double qv = prob_d<T>(sq, zq, Tt, Elem<T>::load(qrow, size_t(v)), v);
+            zsum = fx_add(zsum, fx_from(fmax(resid(pv, qv) - qv, 0.0)));
           }
         }
-        zsum = block_sum_u64(zsum, sm.scr);
-        if (threadIdx.x == 0) zs[nrej] = float(double(zsum) * kFxInv);
+        zsum = block_sum_fx(zsum, sm.scr);
+        if (threadIdx.x == 0) zs[nrej] = fx_to_double(zsum);
         __syncthreads();
         ++nrej;
       }
@@ -151,29 +158,30 @@ __global__ void __launch_bounds__(kThreads) tree_sample_kernel(const TreeSampleJ
           emitted = sparse_draw(
               ids, nk,
               [&](int v) {
-                const float pv = prob<T>(sp, Elem<T>::load(prow, size_t(v)), v);
-                const float qv = k1 > k0 ? prob<T>(sq, Elem<T>::load(qrow, size_t(v)), v) : 0.0f;
-                return to_fx(resid(v, pv, qv));
+                const double pv = prob_d<T>(sp, zp, Tt, Elem<T>::load(prow, size_t(v)), v);
+                const double qv =
+                    k1 > k0 ? prob_d<T>(sq, zq, Tt, Elem<T>::load(qrow, size_t(v)), v) : 0.0;
+                return fx_from(resid(pv, qv));
               },
               w, sm);
         } else {
           const bool pal = (reinterpret_cast<uintptr_t>(prow) & 15u) == 0;
           const bool qal = (reinterpret_cast<uintptr_t>(qrow) & 15u) == 0;
           emitted = inverse_cdf_draw(
-              [&](int v0, unsigned long long* r) {
+              [&](int v0, Fx128* r) {
                 float lp[8], lq[8];
                 load8<T>(prow, v0, V, pal, lp);
                 if (k1 > k0) load8<T>(qrow, v0, V, qal, lq);
 #pragma unroll
                 for (int k = 0; k < 8; ++k) {
                   const int v = v0 + k;
-                  float m = 0.0f;
+                  double mv = 0.0;
                   if (v < V) {
-                    const float pv = prob<T>(sp, lp[k], v);
-                    const float qv = k1 > k0 ? prob<T>(sq, lq[k], v) : 0.0f;
-                    m = resid(v, pv, qv);
+                    const double pv = prob_d<T>(sp, zp, Tt, lp[k], v);
+                    const double qv = k1 > k0 ? prob_d<T>(sq, zq, Tt, lq[k], v) : 0.0;
+                    mv = resid(pv, qv);
                   }
-                  r[k] = to_fx(m);
+                  r[k] = fx_from(mv);
                 }
               },
               V, w, sm);

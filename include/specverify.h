@@ -198,7 +198,7 @@ spec_status spec_residual_sample(const float* p, const float* q, int rows, int V
  * SPEC_STATIC_SCRATCH_BYTES inside the library, one per device; the call allocates
  * nothing and looks the array's address up once per device (with that device current).
  *   - A call whose spec_workspace_size(B, K, V) exceeds SPEC_STATIC_SCRATCH_BYTES returns
- *     SPEC_ERR_WORKSPACE before any CUDA call (8 MiB holds about 7,800 logit rows,
+ *     SPEC_ERR_WORKSPACE before any CUDA call (8 MiB holds about 7,700 logit rows,
  *     B * (2K + 1)).
  *   - Every call on a device uses the same scratch: calls that overlap in time (on
  *     different streams, or from host threads without ordering) race on it and give
@@ -230,8 +230,9 @@ void spec_set_row_kernel_events(void* before, void* after);
 
 /* Largest number of kernels one call enqueues (for launch accounting): the row
  * statistics kernel, the exact finisher for rows it lists (chain calls with top-k or
- * top-p only), the per-batch-row kernel, and for typical acceptance the kernel that lists
- * the rows of nodes with a child. -1 for an unknown name. */
+ * top-p only), the double-precision placement of top-p boundaries (top-p without top-k),
+ * the per-batch-row kernel, and for typical acceptance the kernel that lists the rows of
+ * nodes with a child. -1 for an unknown name. */
 int spec_kernels_per_call(const char* entry_point);
 
 #ifdef __cplusplus

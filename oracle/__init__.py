@@ -28,6 +28,17 @@ FLAG_TREE = 8
 DIAG_Q_ZERO = 16
 PARITY_FLAGS = FLAG_RATIO | FLAG_CDF | FLAG_TOPP | FLAG_TREE
 
+# Widths of the precision windows behind the flags (ratio, cdf_rel, cdf_abs, topp, tree):
+# a flag marks a decision that arithmetic of lower precision than the oracle's may take
+# the other way. They change only the flags, never a result.
+#   CRITERION: the widest the acceptance criterion allows: |u - r| < 1e-5, a CDF edge
+#              within 1e-6 * S of w * S (and 1e-6 on a top-p boundary, relative 1e-5 on a
+#              tree threshold, this build's extensions of the same idea).
+#   FP64:      for a verifier that takes these decisions in double precision: double
+#              rounding over up to 2^20 terms moves a sum by at most ~1.2e-10 of it.
+CRITERION = (1e-5, 1e-6, 0.0, 1e-6, 1e-5)
+FP64 = (1e-9, 1e-9, 1e-10, 1e-10, 1e-9)
+
 
 def build(force: bool = False) -> str:
     """Compile the oracle into liboracle.so (plain g++, no GPU)."""
@@ -50,13 +61,14 @@ def _load():
         I = ctypes.c_int
         D = ctypes.c_double
         _lib.oracle_transform_rows.argtypes = [P, I, I, I, D, I, D, P, P, P, P, I]
-        _lib.oracle_verify_chain.argtypes = [P, P, I, I, I, I, P, P, D, I, D, P, P, P, I]
-        _lib.oracle_verify_chain_f64u.argtypes = [P, P, I, I, I, I, P, P, D, I, D, P, P, P, I]
-        _lib.oracle_verify_tree_typical.argtypes = [P, I, I, I, I, P, P, D, D, D, P, I, P, P, I]
-        _lib.oracle_residual_sample.argtypes = [P, P, I, I, P, P, P, I]
+        _lib.oracle_verify_chain.argtypes = [P, P, I, I, I, I, P, P, D, I, D, P, P, P, I, P]
+        _lib.oracle_verify_chain_f64u.argtypes = [P, P, I, I, I, I, P, P, D, I, D, P, P, P, I, P]
+        _lib.oracle_verify_tree_typical.argtypes = [P, I, I, I, I, P, P, D, D, D, P, I, P, P, I,
+                                                    P]
+        _lib.oracle_residual_sample.argtypes = [P, P, I, I, P, P, P, I, P]
         _lib.oracle_verify_tree_greedy.argtypes = [P, I, I, I, I, P, P, P, I, P, P, I]
         _lib.oracle_verify_tree_sampling.argtypes = [P, P, I, I, I, I, P, P, P, D, I, D, P, I, P,
-                                                     P, P, I]
+                                                     P, P, I, P]
         _lib.oracle_verify_tree_sampling_f64u.argtypes = \
             _lib.oracle_verify_tree_sampling.argtypes
         _lib.oracle_verify_tree_sampling.restype = I
@@ -84,6 +96,12 @@ def _threads(threads):
     return (os.cpu_count() or 1) if threads is None else int(threads)
 
 
+def _win(windows):
+    w = np.ascontiguousarray(CRITERION if windows is None else windows, dtype=np.float64)
+    assert w.shape == (5,)
+    return w
+
+
 def transform_rows(logits, temp, top_k=0, top_p=1.0, threads=None):
     """Rows of logits [..., V] -> (probs float64 [..., V], entropy, topp_margin, valid)."""
     logits = np.ascontiguousarray(logits)
@@ -102,10 +120,12 @@ def transform_rows(logits, temp, top_k=0, top_p=1.0, threads=None):
     return probs.reshape(*shp, V), ent.reshape(shp), marg.reshape(shp), valid.reshape(shp)
 
 
-def verify_chain(target, draft, draft_tokens, uniforms, temp, top_k=0, top_p=1.0, threads=None):
+def verify_chain(target, draft, draft_tokens, uniforms, temp, top_k=0, top_p=1.0, threads=None,
+                 windows=None):
     """Chain verification. target [B,K+1,V], draft [B,K,V] (unused when temp == 0),
     draft_tokens int32 [B,K], uniforms float32 [B,K+1] (float64 uniforms select the
     double-precision entry, used by the exact-integration tests).
+    windows: the flag windows (CRITERION by default, see above).
     Returns (accepted_len int32 [B], out_tokens int32 [B,K+1], flags int32 [B])."""
     target = np.ascontiguousarray(target)
     B, K1, V = target.shape
@@ -120,17 +140,18 @@ def verify_chain(target, draft, draft_tokens, uniforms, temp, top_k=0, top_p=1.0
     acc = np.zeros(B, np.int32)
     out = np.zeros((B, K + 1), np.int32)
     flags = np.zeros(B, np.int32)
+    w = _win(windows)
     fn = _load().oracle_verify_chain_f64u if wide else _load().oracle_verify_chain
     rc = fn(_ptr(target), _ptr(draft), _dtype_code(target), B, K, V,
             _ptr(toks), _ptr(u), float(temp), int(top_k), float(top_p),
-            _ptr(acc), _ptr(out), _ptr(flags), _threads(threads))
+            _ptr(acc), _ptr(out), _ptr(flags), _threads(threads), _ptr(w))
     if rc != 0:
         raise ValueError("oracle_verify_chain rejected its arguments")
     return acc, out, flags
 
 
 def verify_tree_typical(target, node_tokens, parent_idx, eps, delta, temp=1.0, path_cap=None,
-                        threads=None):
+                        threads=None, windows=None):
     """Typical acceptance over a candidate tree. target [B,N,V], node_tokens int32 [B,N],
     parent_idx int32 [N]. Returns (best_path int32 [B,path_cap], accepted_len [B], flags [B])."""
     target = np.ascontiguousarray(target)
@@ -144,7 +165,7 @@ def verify_tree_typical(target, node_tokens, parent_idx, eps, delta, temp=1.0, p
     rc = _load().oracle_verify_tree_typical(_ptr(target), _dtype_code(target), B, N, V,
                                             _ptr(toks), _ptr(par), float(eps), float(delta),
                                             float(temp), _ptr(path), cap, _ptr(acc),
-                                            _ptr(flags), _threads(threads))
+                                            _ptr(flags), _threads(threads), _ptr(_win(windows)))
     if rc != 0:
         raise ValueError("oracle_verify_tree_typical rejected its arguments")
     return path, acc, flags
@@ -171,7 +192,7 @@ def verify_tree_greedy(target, node_tokens, parent_idx, path_cap=None, threads=N
 
 
 def verify_tree_sampling(target, draft, node_tokens, parent_idx, uniforms, temp, top_k=0,
-                         top_p=1.0, path_cap=None, threads=None):
+                         top_p=1.0, path_cap=None, threads=None, windows=None):
     """Rejection sampling over a candidate tree. target and draft [B,N,V] (draft unused
     when temp == 0), node_tokens int32 [B,N], parent_idx int32 [N], uniforms [B,N+1]
     (float64 uniforms select the double-precision entry). Returns (best_path [B,path_cap],
@@ -194,13 +215,13 @@ def verify_tree_sampling(target, draft, node_tokens, parent_idx, uniforms, temp,
     fn = _load().oracle_verify_tree_sampling_f64u if wide else _load().oracle_verify_tree_sampling
     rc = fn(_ptr(target), _ptr(draft), _dtype_code(target), B, N, V, _ptr(toks), _ptr(par),
             _ptr(u), float(temp), int(top_k), float(top_p), _ptr(path), cap, _ptr(acc),
-            _ptr(nxt), _ptr(flags), _threads(threads))
+            _ptr(nxt), _ptr(flags), _threads(threads), _ptr(_win(windows)))
     if rc != 0:
         raise ValueError("oracle_verify_tree_sampling rejected its arguments")
     return path, acc, nxt, flags
 
 
-def residual_sample(p, q, uniforms, threads=None):
+def residual_sample(p, q, uniforms, threads=None, windows=None):
     """Inverse-CDF draw per row from norm(max(0, p - q)) (q None: from p).
     p, q float32 [rows, V]; uniforms float32 [rows]. Returns (tokens int32, flags int32)."""
     p = np.ascontiguousarray(p, dtype=np.float32)
@@ -212,7 +233,7 @@ def residual_sample(p, q, uniforms, threads=None):
     toks = np.zeros(rows, np.int32)
     flags = np.zeros(rows, np.int32)
     rc = _load().oracle_residual_sample(_ptr(p), _ptr(q), rows, V, _ptr(u), _ptr(toks),
-                                        _ptr(flags), _threads(threads))
+                                        _ptr(flags), _threads(threads), _ptr(_win(windows)))
     if rc != 0:
         raise ValueError("oracle_residual_sample rejected its arguments")
     return toks, flags

@@ -53,13 +53,40 @@ const double kInf = std::numeric_limits<double>::infinity();
 
 // Flag bits: decisions that fp32 and fp64 arithmetic may take differently.
 enum : int32_t {
-  FLAG_RATIO = 1,      // |u_i - r_i| < 1e-5 at a tested position
-  FLAG_CDF = 2,        // inverse-CDF boundary within 1e-6 * S of w * S
-  FLAG_TOPP = 4,       // a top-p boundary within 1e-6 of top_p, whose other side
-                       // changes the row's output
-  FLAG_TREE = 8,       // |p - thr| / thr < 1e-5 at a tested tree node
+  FLAG_RATIO = 1,      // |u_i - r_i| < ratio window at a tested position
+  FLAG_CDF = 2,        // inverse-CDF boundary within cdf_rel * S + cdf_abs of w * S
+  FLAG_TOPP = 4,       // a top-p boundary within the top-p window of top_p, whose other
+                       // side changes the row's output
+  FLAG_TREE = 8,       // |p - thr| / thr < tree window at a tested tree node
   DIAG_Q_ZERO = 16,    // a tested draft token had q(x) = 0 (not a parity flag)
 };
+
+// Widths of the precision windows behind the flags. A flag marks a decision that another
+// implementation, computing in lower precision, may take the other way; the defaults are
+// the widest the acceptance criterion allows (1e-5 on the ratio, 1e-6 of S on the CDF; the
+// same 1e-6 on a top-p boundary and a relative 1e-5 on a tree threshold). A caller whose
+// arithmetic is more precise passes narrower windows. The windows change only the flags,
+// never a result.
+struct Windows {
+  double ratio = 1e-5;
+  double cdf_rel = 1e-6;
+  double cdf_abs = 0.0;
+  double topp = 1e-6;
+  double tree = 1e-5;
+};
+
+// w = {ratio, cdf_rel, cdf_abs, topp, tree}, or NULL for the defaults.
+Windows windows_from(const double* w) {
+  Windows x;
+  if (w) {
+    x.ratio = w[0];
+    x.cdf_rel = w[1];
+    x.cdf_abs = w[2];
+    x.topp = w[3];
+    x.tree = w[4];
+  }
+  return x;
+}
 
 double bf16_bits_to_double(uint16_t h) {
   uint32_t u = uint32_t(h) << 16;
@@ -190,7 +217,7 @@ struct Draw {
 // Inverse-CDF draw in ascending token id: the smallest v with res[v] > 0 whose
 // cumulative sum exceeds w * S. If rounding leaves none, the largest v with
 // res[v] > 0 is taken (and the draw is flagged as sitting on an edge).
-Draw inverse_cdf(const std::vector<double>& res, double w) {
+Draw inverse_cdf(const std::vector<double>& res, double w, const Windows& win) {
   Draw out;
   double S = 0.0;
   for (double r : res) S += r;
@@ -201,7 +228,8 @@ Draw inverse_cdf(const std::vector<double>& res, double w) {
     C += res[v];
     if (res[v] > 0.0 && C > target) {
       out.token = v;
-      out.flag = std::fabs(before - target) < 1e-6 * S || std::fabs(C - target) < 1e-6 * S;
+      const double band = win.cdf_rel * S + win.cdf_abs;
+      out.flag = std::fabs(before - target) < band || std::fabs(C - target) < band;
       return out;
     }
   }
@@ -240,6 +268,7 @@ struct ChainArgs {
   int32_t* accepted_len;
   int32_t* out_tokens;
   int32_t* flags;
+  Windows win;
 };
 
 void chain_error(const ChainArgs& a, int b) {
@@ -259,7 +288,7 @@ struct Outcome {
   int acc = 0;
   std::vector<int32_t> out;
   int32_t flag = 0;
-  std::vector<Override> near_ties;  // top-p boundaries within 1e-6 on decision rows
+  std::vector<Override> near_ties;  // top-p boundaries within the window on decision rows
 };
 
 // One batch row of chain verification: [SD] "Speculative Decoding" (accept x_i left to
@@ -276,8 +305,8 @@ Outcome chain_eval(const ChainArgs& a, int b, const Override& ov) {
   int acc = K;
   int emitted = -1;
   auto note = [&](const Dist& d, int kind, int pos) {
-    if (d.margin_reach < 1e-6) o.near_ties.push_back({kind, pos, +1});
-    if (d.margin_prev < 1e-6) o.near_ties.push_back({kind, pos, -1});
+    if (d.margin_reach < a.win.topp) o.near_ties.push_back({kind, pos, +1});
+    if (d.margin_prev < a.win.topp) o.near_ties.push_back({kind, pos, -1});
   };
   auto alt_of = [&](int kind, int pos) { return (ov.kind == kind && ov.pos == pos) ? ov.alt : 0; };
 
@@ -304,7 +333,7 @@ Outcome chain_eval(const ChainArgs& a, int b, const Override& ov) {
       const Dist P = transform(lp, a.T, a.top_k, a.top_p, alt_of(0, i));
       note(P, 0, i);
       if (i == K) {  // every draft accepted: bonus token from p at position K+1
-        const Draw d = inverse_cdf(P.p, u[K]);
+        const Draw d = inverse_cdf(P.p, u[K], a.win);
         emitted = d.token;
         if (d.flag) o.flag |= FLAG_CDF;
         break;
@@ -323,10 +352,10 @@ Outcome chain_eval(const ChainArgs& a, int b, const Override& ov) {
         o.flag |= DIAG_Q_ZERO;
       }
       const double ui = u[i];
-      if (std::isfinite(r) && std::fabs(ui - r) < 1e-5) o.flag |= FLAG_RATIO;
+      if (std::isfinite(r) && std::fabs(ui - r) < a.win.ratio) o.flag |= FLAG_RATIO;
       if (ui < std::min(1.0, r)) continue;
       acc = i;
-      const Draw d = inverse_cdf(residual(P.p, Q.p), u[K]);
+      const Draw d = inverse_cdf(residual(P.p, Q.p), u[K], a.win);
       emitted = d.token;
       if (d.flag) o.flag |= FLAG_CDF;
       break;
@@ -403,12 +432,12 @@ int oracle_transform_rows(const void* logits, int dtype, int rows, int V, double
 int oracle_verify_chain_f64u(const void* target, const void* draft, int dtype, int B, int K,
                              int V, const int32_t* draft_tokens, const double* uniforms, double T,
                              int top_k, double top_p, int32_t* accepted_len, int32_t* out_tokens,
-                             int32_t* flags, int threads) {
+                             int32_t* flags, int threads, const double* windows) {
   if (!target || (T != 0.0 && !draft) || B < 0 || K < 0 || V <= 0 || !draft_tokens ||
       !uniforms || !accepted_len || !out_tokens || !(T >= 0.0))
     return -1;
   ChainArgs a{target, draft, dtype, B, K, V, draft_tokens, uniforms, T, top_k, top_p,
-              accepted_len, out_tokens, flags};
+              accepted_len, out_tokens, flags, windows_from(windows)};
   parallel_rows(B, threads, [&](int b) { chain_row(a, b); });
   return 0;
 }
@@ -418,12 +447,12 @@ int oracle_verify_chain_f64u(const void* target, const void* draft, int dtype, i
 int oracle_verify_chain(const void* target, const void* draft, int dtype, int B, int K, int V,
                         const int32_t* draft_tokens, const float* uniforms, double T, int top_k,
                         double top_p, int32_t* accepted_len, int32_t* out_tokens, int32_t* flags,
-                        int threads) {
+                        int threads, const double* windows) {
   if (!uniforms || B < 0 || K < 0) return -1;
   std::vector<double> u(size_t(B) * size_t(K + 1));
   for (size_t j = 0; j < u.size(); ++j) u[j] = double(uniforms[j]);
   return oracle_verify_chain_f64u(target, draft, dtype, B, K, V, draft_tokens, u.data(), T, top_k,
-                                  top_p, accepted_len, out_tokens, flags, threads);
+                                  top_p, accepted_len, out_tokens, flags, threads, windows);
 }
 
 // MEDUSA typical acceptance over a candidate tree ([SD] "Key Components";
@@ -436,7 +465,9 @@ int oracle_verify_chain(const void* target, const void* draft, int dtype, int B,
 int oracle_verify_tree_typical(const void* target, int dtype, int B, int N, int V,
                                const int32_t* node_tokens, const int32_t* parent_idx, double eps,
                                double delta, double T, int32_t* best_path, int path_cap,
-                               int32_t* accepted_len, int32_t* flags, int threads) {
+                               int32_t* accepted_len, int32_t* flags, int threads,
+                               const double* windows) {
+  const Windows win = windows_from(windows);
   if (!target || B < 0 || N <= 0 || V <= 0 || !node_tokens || !parent_idx || !best_path ||
       path_cap <= 0 || !accepted_len || !(T >= 0.0))
     return -1;
@@ -476,7 +507,7 @@ int oracle_verify_tree_typical(const void* target, int dtype, int B, int N, int 
       if (tok < 0 || tok >= V) return fail();
       const double p = dist[pa].p[tok];
       const double thr = std::min(eps, delta * std::exp(-dist[pa].entropy));
-      if (thr > 0.0 && std::fabs(p - thr) / thr < 1e-5) flag |= FLAG_TREE;
+      if (thr > 0.0 && std::fabs(p - thr) / thr < win.tree) flag |= FLAG_TREE;
       acc[c] = p > thr;
     }
     int best = 0;
@@ -576,7 +607,8 @@ int oracle_verify_tree_sampling_f64u(const void* target, const void* draft, int 
                                      const int32_t* parent_idx, const double* uniforms, double T,
                                      int top_k, double top_p, int32_t* best_path, int path_cap,
                                      int32_t* accepted_len, int32_t* next_token, int32_t* flags,
-                                     int threads) {
+                                     int threads, const double* windows) {
+  const Windows win = windows_from(windows);
   if (!target || (T != 0.0 && !draft) || B < 0 || N <= 0 || V <= 0 || !node_tokens ||
       !parent_idx || !uniforms || !best_path || path_cap <= 0 || !accepted_len || !(T >= 0.0))
     return -1;
@@ -608,7 +640,7 @@ int oracle_verify_tree_sampling_f64u(const void* target, const void* draft, int 
       load_row(target, dtype, size_t(b) * N + cur, V, lp);
       if (!row_valid(lp)) return fail();
       const Dist pd = transform(lp, T, top_k, top_p);
-      if (pd.topp_margin() < 1e-6) flag |= FLAG_TOPP;
+      if (pd.topp_margin() < win.topp) flag |= FLAG_TOPP;
       int next = -1;
       if (T == 0.0) {
         const int g = argmax_lowest(lp);
@@ -626,13 +658,13 @@ int oracle_verify_tree_sampling_f64u(const void* target, const void* draft, int 
           load_row(draft, dtype, size_t(b) * N + cur, V, lq);
           if (!row_valid(lq)) return fail();
           const Dist qd = transform(lq, T, top_k, top_p);
-          if (qd.topp_margin() < 1e-6) flag |= FLAG_TOPP;
+          if (qd.topp_margin() < win.topp) flag |= FLAG_TOPP;
           for (int c : kids[cur]) {
             const int x = tok[c];
             if (x < 0 || x >= V) return fail();
             const double px = r[x], qx = qd.p[x];
             const double ratio = qx > 0.0 ? px / qx : (px > 0.0 ? kInf : 0.0);
-            if (std::fabs(u[c] - ratio) < 1e-5) flag |= FLAG_RATIO;
+            if (std::fabs(u[c] - ratio) < win.ratio) flag |= FLAG_RATIO;
             if (u[c] < std::min(1.0, ratio)) {
               next = c;
               break;
@@ -649,7 +681,7 @@ int oracle_verify_tree_sampling_f64u(const void* target, const void* draft, int 
           }
         }
         if (next < 0) {
-          const Draw d = inverse_cdf(r, u[N]);
+          const Draw d = inverse_cdf(r, u[N], win);
           if (d.flag) flag |= FLAG_CDF;
           emitted = d.token;
         }
@@ -673,20 +705,22 @@ int oracle_verify_tree_sampling(const void* target, const void* draft, int dtype
                                 int V, const int32_t* node_tokens, const int32_t* parent_idx,
                                 const float* uniforms, double T, int top_k, double top_p,
                                 int32_t* best_path, int path_cap, int32_t* accepted_len,
-                                int32_t* next_token, int32_t* flags, int threads) {
+                                int32_t* next_token, int32_t* flags, int threads,
+                                const double* windows) {
   if (!uniforms || B < 0 || N <= 0) return -1;
   std::vector<double> u(size_t(B) * size_t(N + 1));
   for (size_t j = 0; j < u.size(); ++j) u[j] = double(uniforms[j]);
   return oracle_verify_tree_sampling_f64u(target, draft, dtype, B, N, V, node_tokens, parent_idx,
                                           u.data(), T, top_k, top_p, best_path, path_cap,
-                                          accepted_len, next_token, flags, threads);
+                                          accepted_len, next_token, flags, threads, windows);
 }
 
 // Inverse-CDF draw from norm(max(0, p - q)) (q == NULL: from p) for explicit
 // probability rows. Entries are probabilities: a row holding an entry that is
 // NaN or outside [0, 1], or whose p has no positive entry, gives token -1.
 int oracle_residual_sample(const float* p, const float* q, int rows, int V, const float* uniforms,
-                           int32_t* tokens, int32_t* flags, int threads) {
+                           int32_t* tokens, int32_t* flags, int threads, const double* windows) {
+  const Windows win = windows_from(windows);
   if (!p || rows < 0 || V <= 0 || !uniforms || !tokens) return -1;
   parallel_rows(rows, threads, [&](int r) {
     std::vector<double> pr(static_cast<size_t>(V)), qr(size_t(V), 0.0);
@@ -706,7 +740,7 @@ int oracle_residual_sample(const float* p, const float* q, int rows, int V, cons
       if (flags) flags[r] = 0;
       return;
     }
-    const Draw d = inverse_cdf(q ? residual(pr, qr) : pr, double(uniforms[r]));
+    const Draw d = inverse_cdf(q ? residual(pr, qr) : pr, double(uniforms[r]), win);
     tokens[r] = d.token;
     if (flags) flags[r] = d.flag ? FLAG_CDF : 0;
   });

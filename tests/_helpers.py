@@ -38,7 +38,7 @@ def draft_tokens(draft: np.ndarray, temp: float, top_k: int, top_p: float,
     """x[b, i] ~ transformed q_i (temp 0: argmax of the draft logits)."""
     B, K, V = draft.shape
     flat = draft.reshape(B * K, V)
-    u = np.asarray(pick_uniforms, np.float32).reshape(B * K)
+    u = None if temp == 0.0 else np.asarray(pick_uniforms, np.float32).reshape(B * K)
     out = np.empty(B * K, np.int32)
     for s in range(0, B * K, chunk_rows):
         rows = flat[s:s + chunk_rows]

@@ -25,13 +25,14 @@ def test_every_declared_function_is_exported(lib):
 def test_status_strings_and_kernel_counts(lib):
     assert sv.status_string(0) == "SPEC_OK"
     assert sv.status_string(-4) == "SPEC_ERR_WORKSPACE"
-    assert sv.spec_kernels_per_call("spec_verify_chain") == 3
+    assert sv.spec_kernels_per_call("spec_verify_chain") == 4
+    assert sv.spec_kernels_per_call("spec_verify_tree_typical") == 3
     assert sv.spec_kernels_per_call("nope") == -1
 
 
 def _ws(rows):
     up = lambda x: (x + 255) // 256 * 256
-    return 256 + up(32 * rows) + up(4 * rows) + up(rows * 256 * 4) + up(4 * rows)
+    return 256 + up(48 * rows) + up(4 * rows) + up(rows * 256 * 4) + up(4 * rows) + up(4 * rows)
 
 
 def test_workspace_size(lib):

@@ -1,8 +1,19 @@
 """GPU parity: the CUDA library (through the C ABI) against the oracle, on the same
-seeded inputs. Tokens and accepted lengths must be identical except on rows the
-oracle flags (a decision within the fp32/fp64 precision window whose other side
-changes the output); flagged rows must stay under 1e-4 of all rows checked."""
+seeded inputs. Tokens, paths and accepted lengths must be identical except on rows the
+oracle flags.
+
+The library takes every sampling decision in double precision (the ratio tests, the
+residual and bonus draws, the top-p boundary when fp32 cannot settle it, the typical test
+when fp32 cannot settle it), so the oracle's flags use the FP64 windows: a row is excluded
+only when a decision lies within ~1e-9 of its boundary, where double rounding over a whole
+row could tip it. The oracle is evaluated with the knob values the library receives
+(temperature, top_p, eps and delta rounded to float32). The budget tests at the end check
+that excluded rows stay under 1e-4 of at least 10^4 rows for chain and tree verification."""
 from __future__ import annotations
+
+import dataclasses
+import os
+from concurrent.futures import ThreadPoolExecutor
 
 import numpy as np
 import pytest
@@ -15,7 +26,12 @@ from tests._helpers import chain_case, check_chain_invariants, draft_tokens
 
 pytestmark = pytest.mark.gpu
 
-_STATS = {"rows": 0, "flagged": 0}
+W = oracle.FP64
+
+
+def f32(x: float) -> float:
+    """The float32 value the C ABI receives for a knob."""
+    return float(np.float32(x))
 
 
 def dev(a: np.ndarray) -> torch.Tensor:
@@ -31,27 +47,27 @@ def gpu_chain(target, draft, toks, u, temp, top_k=0, top_p=1.0):
     return acc.cpu().numpy(), out.cpu().numpy()
 
 
-def assert_chain_parity(acc_g, out_g, acc_r, out_r, flags, budget=False):
+def assert_chain_parity(acc_g, out_g, acc_r, out_r, flags):
+    """No mismatch outside the flagged rows; returns the number of flagged rows."""
     ok = (flags & oracle.PARITY_FLAGS) == 0
     same = (acc_g == acc_r) & np.all(out_g == out_r, axis=1)
     bad = np.nonzero(~same & ok)[0]
     assert bad.size == 0, (f"{bad.size} unflagged mismatches, first rows {bad[:5].tolist()}: "
                            f"gpu {acc_g[bad[:3]]} {out_g[bad[:3]]} oracle {acc_r[bad[:3]]} "
-                           f"{out_r[bad[:3]]}")
-    if budget:  # workload rows only; the edge-case tests build exact ties on purpose
-        _STATS["rows"] += len(acc_r)
-        _STATS["flagged"] += int((~ok).sum())
+                           f"{out_r[bad[:3]]} flags {flags[bad[:3]]}")
     return int((~ok).sum())
 
 
-def run_case(target, draft, toks, u, temp, top_k=0, top_p=1.0, rows=None, budget=False):
+def oracle_chain(target, draft, toks, u, temp, top_k=0, top_p=1.0):
+    return oracle.verify_chain(target, draft, toks, u, f32(temp), top_k, f32(top_p), windows=W)
+
+
+def run_case(target, draft, toks, u, temp, top_k=0, top_p=1.0):
+    """GPU and oracle on every batch row; returns the GPU outputs and the flagged count."""
     acc_g, out_g = gpu_chain(target, draft, toks, u, temp, top_k, top_p)
-    if rows is None:
-        rows = np.arange(target.shape[0])
-    acc_r, out_r, flags = oracle.verify_chain(target[rows], None if draft is None else draft[rows],
-                                              toks[rows], u[rows], temp, top_k, top_p)
-    assert_chain_parity(acc_g[rows], out_g[rows], acc_r, out_r, flags, budget)
-    return acc_g, out_g
+    acc_r, out_r, flags = oracle_chain(target, draft, toks, u, temp, top_k, top_p)
+    nflag = assert_chain_parity(acc_g, out_g, acc_r, out_r, flags)
+    return acc_g, out_g, nflag
 
 
 # ------------------------------------------------------------------ the workloads, small batch
@@ -60,7 +76,7 @@ def run_case(target, draft, toks, u, temp, top_k=0, top_p=1.0, rows=None, budget
                                    (specgen.CFG5, 6)], ids=lambda x: getattr(x, "name", str(x)))
 def test_chain_workloads_small_batch(cfg, B):
     target, draft, toks, u, temp = chain_case(cfg, B)
-    acc, out = run_case(target, draft, toks, u, temp, cfg.top_k, cfg.top_p, budget=True)
+    acc, out, _ = run_case(target, draft, toks, u, temp, cfg.top_k, cfg.top_p)
     check_chain_invariants(acc, out, toks, cfg.K, cfg.V)
 
 
@@ -73,32 +89,33 @@ def test_chain_greedy_small_batch(cfg, B):
 
 # ------------------------------------------------------------------ full sizes (bench launch shape)
 
-def test_chain_cfg5_full_size_sampled_rows():
+def test_chain_cfg5_full_size_all_rows():
+    """The 512 x 8 x 151936 top-k 50 workload, every batch row, sampling and greedy."""
     cfg = specgen.CFG5
     target, draft, toks, u, temp = chain_case(cfg)
-    rows = np.unique(np.linspace(0, cfg.B - 1, 24).astype(int))
-    acc, out = run_case(target, draft, toks, u, temp, cfg.top_k, cfg.top_p, rows=rows,
-                        budget=True)
+    acc, out, _ = run_case(target, draft, toks, u, temp, cfg.top_k, cfg.top_p)
     check_chain_invariants(acc, out, toks, cfg.K, cfg.V)
-    acc_g, out_g = run_case(target, None, toks, u, 0.0, budget=True)  # greedy: every row
-    check_chain_invariants(acc_g, out_g, toks, cfg.K, cfg.V)
+    greedy_toks = draft_tokens(draft, 0.0, 0, 1.0, None)  # the draft argmax
+    acc_g, out_g, nflag = run_case(target, None, greedy_toks, u, 0.0)
+    assert nflag == 0
+    check_chain_invariants(acc_g, out_g, greedy_toks, cfg.K, cfg.V)
 
 
-def test_chain_cfg3_full_size_sampled_rows():
+def test_chain_cfg3_full_size_all_rows():
+    """The 256 x 7 x 128256 top-p 0.9 workload, every batch row."""
     cfg = specgen.CFG3
     target, draft, toks, u, temp = chain_case(cfg)
-    rows = np.unique(np.linspace(0, cfg.B - 1, 16).astype(int))
-    acc, out = run_case(target, draft, toks, u, temp, cfg.top_k, cfg.top_p, rows=rows,
-                        budget=True)
+    acc, out, _ = run_case(target, draft, toks, u, temp, cfg.top_k, cfg.top_p)
     check_chain_invariants(acc, out, toks, cfg.K, cfg.V)
 
 
 def test_chain_cfg2_full_size_all_rows():
     cfg = specgen.CFG2
     target, draft, toks, u, temp = chain_case(cfg)
-    run_case(target, draft, toks, u, temp, budget=True)
+    run_case(target, draft, toks, u, temp)
     target, draft, toks, u, _ = chain_case(cfg, greedy=True)
-    run_case(target, None, toks, u, 0.0, budget=True)
+    _, _, nflag = run_case(target, None, toks, u, 0.0)
+    assert nflag == 0
 
 
 # ------------------------------------------------------------------ edge cases
@@ -164,7 +181,7 @@ def test_chain_sixteen_cta_cluster():
 @pytest.mark.parametrize("K", [1, 31, 32, 40])
 def test_chain_many_positions(K):
     target, draft, toks, u = _rand_chain(K, 6, K, 300, "bf16", draft_noise=0.05)
-    acc, out = run_case(target, draft, toks, u, 1.0)
+    acc, out, _ = run_case(target, draft, toks, u, 1.0)
     assert acc.max() >= min(K, 3)
 
 
@@ -200,7 +217,7 @@ def test_chain_error_rows():
     draft[2, 0, :] = 0xFF80               # all -inf draft row at position 0: error
     toks[3, 0] = V                        # token out of range: error
     toks[4, 2] = -5                       # out of range after a likely stop
-    acc_g, out_g = run_case(target, draft, toks, u, 1.0)
+    acc_g, out_g, _ = run_case(target, draft, toks, u, 1.0)
     assert acc_g[0] == -1 and acc_g[2] == -1 and acc_g[3] == -1
     assert np.all(out_g[[0, 2, 3]] == -1)
     run_case(target, None, toks, u, 0.0)
@@ -209,7 +226,7 @@ def test_chain_error_rows():
 def test_chain_unaligned_base_pointer_and_determinism():
     B, K, V = 6, 4, 1000
     target, draft, toks, u = _rand_chain(11, B, K, V, "bf16")
-    acc_ref, out_ref, _ = oracle.verify_chain(target, draft, toks, u, 1.0, 20)
+    acc_ref, out_ref, _ = oracle_chain(target, draft, toks, u, 1.0, 20)
     # shift the tensors by one element inside a larger allocation
     tb = torch.empty(target.size + 1, dtype=torch.bfloat16, device="cuda")
     db = torch.empty(draft.size + 1, dtype=torch.bfloat16, device="cuda")
@@ -233,13 +250,19 @@ def gpu_tree(logits, toks, par, eps, delta, path_cap=None):
     return path.cpu().numpy(), plen.cpu().numpy()
 
 
-def assert_tree_parity(logits, toks, par, eps, delta, path_cap=None):
+def assert_tree_parity(logits, toks, par, eps, delta, path_cap=None, stats=None):
+    """Typical acceptance: no mismatch outside the flagged rows (a threshold within 1e-9
+    relative); `stats` accumulates rows and flagged rows."""
     path_g, len_g = gpu_tree(logits, toks, par, eps, delta, path_cap)
-    path_r, len_r, flags = oracle.verify_tree_typical(logits, toks, par, eps, delta,
-                                                      path_cap=path_cap)
+    path_r, len_r, flags = oracle.verify_tree_typical(logits, toks, par, f32(eps), f32(delta),
+                                                      path_cap=path_cap, windows=W)
     ok = (flags & oracle.PARITY_FLAGS) == 0
     same = (len_g == len_r) & np.all(path_g == path_r, axis=1)
-    assert np.all(same | ~ok), np.nonzero(~same & ok)[0]
+    bad = np.nonzero(~same & ok)[0]
+    assert bad.size == 0, (bad[:5], len_g[bad[:5]], len_r[bad[:5]])
+    if stats is not None:
+        stats["rows"] += len(ok)
+        stats["flagged"] += int((~ok).sum())
     return len_g
 
 
@@ -295,7 +318,8 @@ def test_tree_leaf_rows_are_never_read():
     bad[:, leaves, 5] = 0x7FC0     # NaN
     bad[:, leaves, 9] = 0x7F80     # +inf
     path_g, len_g = gpu_tree(bad, toks, par, cfg.eps, cfg.delta)
-    path_r, len_r, _ = oracle.verify_tree_typical(logits, toks, par, cfg.eps, cfg.delta)
+    path_r, len_r, _ = oracle.verify_tree_typical(logits, toks, par, f32(cfg.eps),
+                                                  f32(cfg.delta), windows=W)
     assert np.array_equal(len_g, len_r) and np.array_equal(path_g, path_r)
     assert len_g.min() >= 1
 
@@ -377,21 +401,24 @@ def _tree_children_from_q(g, draft, par, temp, top_k, top_p):
 
 
 def assert_tree_sampling_parity(target, draft, toks, par, u, temp, top_k=0, top_p=1.0,
-                                path_cap=None, flag_budget=20):
+                                path_cap=None, stats=None):
+    """Tree rejection sampling: no mismatch outside the flagged rows (a ratio within 1e-9 of
+    its uniform, a draw within 1e-9 of a CDF edge, a top-p boundary within 1e-10); `stats`
+    accumulates rows and flagged rows."""
     path_g, len_g, nxt_g = sv.spec_verify_tree_sampling(
         dev(target), None if draft is None else dev(draft), dev(toks), dev(par), dev(u), temp,
         top_k, top_p, path_cap=path_cap)
     torch.cuda.synchronize()
-    path_r, len_r, nxt_r, flags = oracle.verify_tree_sampling(target, draft, toks, par, u, temp,
-                                                              top_k, top_p, path_cap=path_cap)
+    path_r, len_r, nxt_r, flags = oracle.verify_tree_sampling(
+        target, draft, toks, par, u, f32(temp), top_k, f32(top_p), path_cap=path_cap, windows=W)
     len_g, path_g, nxt_g = len_g.cpu().numpy(), path_g.cpu().numpy(), nxt_g.cpu().numpy()
     ok = (flags & oracle.PARITY_FLAGS) == 0
     same = (len_g == len_r) & np.all(path_g == path_r, axis=1) & (nxt_g == nxt_r)
     bad = np.nonzero(~same & ok)[0]
     assert bad.size == 0, (bad[:5], len_g[bad[:5]], len_r[bad[:5]], nxt_g[bad[:5]], nxt_r[bad[:5]])
-    # a flag marks a decision inside the fp32/fp64 window (a draw on a token holding under
-    # 1e-6 of the mass, a ratio within 1e-5 of its uniform)
-    assert (~ok).sum() <= max(1, len(ok) // flag_budget), (~ok).sum()
+    if stats is not None:
+        stats["rows"] += len(ok)
+        stats["flagged"] += int((~ok).sum())
     return len_r
 
 
@@ -432,7 +459,7 @@ def test_tree_sampling_workload_shape():
     target, draft = specgen.f32_to_bf16_bits(t), specgen.f32_to_bf16_bits(d)
     toks = _tree_children_from_q(g, draft, par, 1.0, 0, 1.0)
     u = (g.integers(0, 1 << 24, (B, N + 1)) / float(1 << 24)).astype(np.float32)
-    lens = assert_tree_sampling_parity(target, draft, toks, par, u, 1.0, flag_budget=8)
+    lens = assert_tree_sampling_parity(target, draft, toks, par, u, 1.0)
     assert lens.max() >= 3
 
 
@@ -505,7 +532,7 @@ def test_residual_sample(V, with_q):
     u[2] = np.float32(1 - 2 ** -24)
     tok_g = sv.spec_residual_sample(dev(p), None if q is None else dev(q), dev(u))
     tok_g = tok_g.cpu().numpy()
-    tok_r, flags = oracle.residual_sample(p, q, u)
+    tok_r, flags = oracle.residual_sample(p, q, u, windows=W)
     ok = flags == 0
     assert np.all((tok_g == tok_r) | ~ok), np.nonzero((tok_g != tok_r) & ok)
     bad = p.copy()
@@ -516,9 +543,97 @@ def test_residual_sample(V, with_q):
     assert tb[:3].tolist() == [-1, -1, -1]
 
 
-def test_flagged_row_budget():
-    """Over the workload rows checked in this module, flagged rows stay under 1e-4 (at
-    most one when fewer than 10^4 rows were checked)."""
-    if _STATS["rows"] == 0:
-        pytest.skip("run with the other parity tests")
-    assert _STATS["flagged"] <= max(1, 1e-4 * _STATS["rows"]), _STATS
+
+
+# ------------------------------------------------------------------ the flagged-row budget
+# Acceptance: tokens and lengths bit-exact except flagged rows, which must stay under 1e-4 of
+# all rows. Each test below checks at least 10^4 batch rows of seeded inputs shaped like the
+# workloads (seeds beyond the workloads' own), every row against the oracle, and asserts the
+# flagged share with no floor. Inputs are generated on host threads (one generator per
+# instance; the seeded streams do not depend on the thread).
+
+def _pool_map(fn, items):
+    """fn over items on host threads, results in order as they complete."""
+    with ThreadPoolExecutor(max_workers=min(len(items), 8, os.cpu_count() or 1)) as ex:
+        yield from ex.map(fn, items)
+
+
+def _budget_report(name, stats):
+    print(f"\n{name}: {stats}", flush=True)
+    assert stats["rows"] >= 10_000, stats
+    assert stats["flagged"] < 1e-4 * stats["rows"], stats
+
+
+def test_chain_flagged_rows_under_1e4_of_10k_rows():
+    """Chain sampling on 10,240 rows of the 32,000-vocabulary Zipf workload's distribution
+    (temperature 0.7, untruncated: dense draws), 512 rows of the 128,256-vocabulary top-p 0.9
+    workload's and 512 rows of the 151,936-vocabulary top-k 50 workload's, all with seeds
+    beyond the workloads' own."""
+    cases = [(dataclasses.replace(specgen.CFG2, seed=100 + i), 512) for i in range(20)]
+    cases += [(dataclasses.replace(specgen.CFG3, seed=200 + i), 256) for i in range(2)]
+    stats = {"rows": 0, "flagged": 0}
+
+    def check(cfg, B, inputs):
+        target, draft, toks, u, temp = inputs
+        acc, out, nflag = run_case(target, draft, toks, u, temp, cfg.top_k, cfg.top_p)
+        check_chain_invariants(acc, out, toks, cfg.K, cfg.V)
+        stats["rows"] += B
+        stats["flagged"] += nflag
+
+    for (cfg, B), inputs in zip(cases, _pool_map(lambda c: chain_case(*c), cases)):
+        check(cfg, B, inputs)
+    cfg5 = dataclasses.replace(specgen.CFG5, seed=400)  # 2.6 GB: alone
+    check(cfg5, 512, chain_case(cfg5, 512))
+    _budget_report("chain", stats)
+
+
+def test_tree_typical_flagged_rows_under_1e4_of_10k_rows():
+    """Typical acceptance on 10,240 trees of the MEDUSA workload's shape (4 heads, top-(4,3,2,2)
+    truncated to 64 nodes, node logits N(0, 3^2)) over a 2,048-entry vocabulary, half of them
+    with the coverage boost that accepts deep paths."""
+    def make(i):
+        cfg = specgen.TreeConfig(**{**specgen.CFG4.__dict__, "V": 2048, "seed": 30 + i,
+                                    "coverage_boost": 6.0 if i % 2 else 0.0})
+        return cfg, specgen.tree_inputs(cfg, 512)
+    stats = {"rows": 0, "flagged": 0}
+    for cfg, (logits, toks, par) in _pool_map(make, list(range(20))):
+        assert_tree_parity(logits, toks, par, cfg.eps, cfg.delta, stats=stats)
+    _budget_report("tree typical", stats)
+
+
+def _children_from_q_fast(g, draft, par, temp, top_k, top_p):
+    """As _tree_children_from_q, vectorised over batch rows (inverse CDF per child)."""
+    B, N, V = draft.shape
+    q = oracle.transform_rows(draft, temp, top_k, top_p)[0].reshape(B, N, V)
+    cdf = np.cumsum(q, axis=2)
+    toks = np.zeros((B, N), np.int32)
+    u = g.random((B, N))
+    for c in range(1, N):
+        cc = cdf[:, par[c], :]
+        t = (cc < (u[:, c] * cc[:, -1])[:, None]).sum(axis=1)
+        toks[:, c] = np.minimum(t, V - 1)
+    return toks
+
+
+def test_tree_sampling_flagged_rows_under_1e4_of_10k_rows():
+    """Tree rejection sampling on 10,240 random trees (20 x 512) of 24 nodes over a 1,024-entry
+    vocabulary (target N(0, 2^2) plus the Zipf prior, draft = target + N(0, 0.8^2)),
+    children drawn from the drafter, at temperature 1 untruncated, 0.8 with top-k 40, and 1
+    with top-p 0.9."""
+    N, V, B = 24, 1024, 512
+    knobs = [(1.0, 0, 1.0), (0.8, 40, 1.0), (1.0, 0, 0.9)]
+
+    def make(i):
+        g = np.random.default_rng(9000 + i)
+        par = np.array([-1] + [int(g.integers(max(0, c - 4), c)) for c in range(1, N)], np.int32)
+        t = (g.normal(0, 2.0, (B, N, V)) - 1.1 * np.log1p(np.arange(V))).astype(np.float32)
+        d = (t + g.normal(0, 0.8, (B, N, V))).astype(np.float32)
+        temp, top_k, top_p = knobs[i % len(knobs)]
+        target, draft = specgen.f32_to_bf16_bits(t), specgen.f32_to_bf16_bits(d)
+        toks = _children_from_q_fast(g, draft, par, temp, top_k, top_p)
+        u = (g.integers(0, 1 << 24, (B, N + 1)) / float(1 << 24)).astype(np.float32)
+        return target, draft, toks, par, u, temp, top_k, top_p
+    stats = {"rows": 0, "flagged": 0}
+    for target, draft, toks, par, u, temp, top_k, top_p in _pool_map(make, list(range(20))):
+        assert_tree_sampling_parity(target, draft, toks, par, u, temp, top_k, top_p, stats=stats)
+    _budget_report("tree sampling", stats)
