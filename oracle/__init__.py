@@ -73,6 +73,8 @@ def _load():
             _lib.oracle_verify_tree_sampling.argtypes
         _lib.oracle_verify_tree_sampling.restype = I
         _lib.oracle_verify_tree_sampling_f64u.restype = I
+        _lib.oracle_linear_state_replay.argtypes = [P, I, I, I, I, I, P, P, P, P, P, P, I]
+        _lib.oracle_linear_state_replay.restype = I
         for f in (_lib.oracle_transform_rows, _lib.oracle_verify_chain,
                   _lib.oracle_verify_chain_f64u, _lib.oracle_verify_tree_greedy,
                   _lib.oracle_verify_tree_typical, _lib.oracle_residual_sample):
@@ -237,3 +239,27 @@ def residual_sample(p, q, uniforms, threads=None, windows=None):
     if rc != 0:
         raise ValueError("oracle_residual_sample rejected its arguments")
     return toks, flags
+
+
+def linear_state_replay(state0, alpha, beta, keys, values, steps, threads=None):
+    """Linear-attention state after each sequence's accepted prefix, replayed step by step
+    (gated delta rule S_t = alpha_t (I - beta_t k_t k_t^T) S_{t-1} + beta_t k_t v_t^T).
+    state0 float32 [B,H,dk,dv]; alpha, beta [B,H,K]; keys [B,H,K,dk]; values [B,H,K,dv];
+    steps int32 [B] (outside [0, K]: unchanged). Returns float64 [B,H,dk,dv]."""
+    state0 = np.ascontiguousarray(state0, np.float32)
+    B, H, dk, dv = state0.shape
+    alpha = np.ascontiguousarray(alpha, np.float32)
+    K = alpha.shape[2]
+    beta = np.ascontiguousarray(beta, np.float32)
+    keys = np.ascontiguousarray(keys, np.float32)
+    values = np.ascontiguousarray(values, np.float32)
+    steps = np.ascontiguousarray(steps, np.int32)
+    assert alpha.shape == beta.shape == (B, H, K)
+    assert keys.shape == (B, H, K, dk) and values.shape == (B, H, K, dv) and steps.shape == (B,)
+    out = np.zeros((B, H, dk, dv), np.float64)
+    rc = _load().oracle_linear_state_replay(_ptr(state0), B, H, dk, dv, K, _ptr(alpha),
+                                            _ptr(beta), _ptr(keys), _ptr(values), _ptr(steps),
+                                            _ptr(out), _threads(threads))
+    if rc != 0:
+        raise ValueError("oracle_linear_state_replay rejected its arguments")
+    return out

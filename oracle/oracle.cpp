@@ -747,4 +747,50 @@ int oracle_residual_sample(const float* p, const float* q, int rows, int V, cons
   return 0;
 }
 
+// State commit after verification for a linear-attention target ([SpecLA] summary: the
+// state is a dense summary updated with every token, and after the verdict it is brought to
+// the accepted prefix; the summary names the gated-delta-rule model GDN). The recurrence,
+// per sequence b and head h, with the state S in R^{dk x dv}:
+//   S_t = alpha_t (I - beta_t k_t k_t^T) S_{t-1} + beta_t k_t v_t^T,   t = 1 .. steps[b],
+// replayed here one step at a time in double (the plain definition; no compact factors).
+// state0 [B][H][dk][dv] float, alpha, beta [B][H][K], keys [B][H][K][dk], values
+// [B][H][K][dv] float; out [B][H][dk][dv] double. steps[b] outside [0, K] leaves the state
+// unchanged (an error row of the verification).
+int oracle_linear_state_replay(const float* state0, int B, int H, int dk, int dv, int K,
+                               const float* alpha, const float* beta, const float* keys,
+                               const float* values, const int32_t* steps, double* out,
+                               int threads) {
+  if (!state0 || B < 0 || H <= 0 || dk <= 0 || dv <= 0 || K < 0 || !alpha || !beta || !keys ||
+      !values || !steps || !out)
+    return -1;
+  parallel_rows(B * H, threads, [&](int bh) {
+    const int b = bh / H;
+    const size_t n = size_t(dk) * dv;
+    double* S = out + size_t(bh) * n;
+    for (size_t i = 0; i < n; ++i) S[i] = double(state0[size_t(bh) * n + i]);
+    const int a = steps[b];
+    if (a < 0 || a > K) return;
+    std::vector<double> kS(static_cast<size_t>(dv));
+    for (int t = 0; t < a; ++t) {
+      const size_t st = size_t(bh) * K + t;
+      const double al = alpha[st], be = beta[st];
+      const float* k = keys + st * dk;
+      const float* v = values + st * dv;
+      // kS = k^T S_{t-1}
+      for (int j = 0; j < dv; ++j) {
+        double acc = 0.0;
+        for (int i = 0; i < dk; ++i) acc += double(k[i]) * S[size_t(i) * dv + j];
+        kS[j] = acc;
+      }
+      // S_t = alpha (S - beta k kS^T) + beta k v^T
+      for (int i = 0; i < dk; ++i)
+        for (int j = 0; j < dv; ++j) {
+          double& x = S[size_t(i) * dv + j];
+          x = al * (x - be * double(k[i]) * kS[j]) + be * double(k[i]) * double(v[j]);
+        }
+    }
+  });
+  return 0;
+}
+
 }  // extern "C"

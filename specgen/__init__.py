@@ -1,8 +1,9 @@
 """Seeded synthetic inputs for draft-token verification.
 
 This module only draws numbers: logits with the shapes, value distributions
-and structure of the five verification workloads, uniforms, and MEDUSA-style
-candidate trees. It holds none of the verification arithmetic (no softmax,
+and structure of the five verification workloads, uniforms, MEDUSA-style
+candidate trees, and the recurrent state and per-step data of a linear-attention
+target. It holds none of the verification arithmetic (no softmax,
 no transform, no acceptance rule), and both the CUDA library's tests/bench and
 the oracle's tests consume the same bytes from it.
 
@@ -20,6 +21,7 @@ import numpy as np
 
 # Independent streams (see module docstring).
 S_TARGET, S_DRAFT, S_BOOST, S_UNIFORM, S_DRAFTPICK, S_HEADS, S_TREE = range(7)
+S_STATE, S_KEYS, S_VALUES, S_GATES, S_ACCEPT = range(7, 12)
 
 
 def rng(seed: int, stream: int) -> np.random.Generator:
@@ -181,3 +183,49 @@ def tree_inputs(cfg: TreeConfig, B: int | None = None):
                 x[n, tokens[b, c]] += np.float32(cfg.coverage_boost)
         logits[b] = _emit(x, cfg.dtype)
     return logits, tokens, parent
+
+
+@dataclass(frozen=True)
+class LinearStateConfig:
+    """A linear-attention target's recurrent state, per sequence and head, and the per-step
+    data of one verified round: the previous round's emitted token (its update was deferred)
+    plus K drafts, so K + 1 steps. A sequence whose first a drafts were accepted commits
+    a + 1 steps."""
+    name: str
+    B: int
+    H: int
+    dk: int
+    dv: int
+    K: int                 # drafts; the round holds K + 1 steps
+    accept: float          # per-draft acceptance probability (leading run of successes)
+    alpha_lo: float = 0.9  # gates alpha ~ U(alpha_lo, 1)
+    seed: int = 5
+
+
+# Gated-delta-rule state of a 1.3B-parameter class model: 16 heads, 128-wide keys, 256-wide
+# values, fp32 state (128 KiB per head); 512 sequences with 8 drafts each, acceptance 0.75.
+LSTATE = LinearStateConfig("lstate_B512_H16_dk128_dv256_K8_f32", 512, 16, 128, 256, 8, 0.75)
+
+
+def linear_state_inputs(cfg: LinearStateConfig, B: int | None = None):
+    """state0 [B,H,dk,dv] float32 ~ N(0, 1); keys [B,H,K+1,dk] unit vectors (normalised
+    N(0, I)); values [B,H,K+1,dv] ~ N(0, 1); alpha ~ U(alpha_lo, 1) and beta ~ U(0, 1)
+    [B,H,K+1]; steps [B] int32 = 1 + the number of leading accepted drafts (each accepted
+    with probability cfg.accept)."""
+    B = cfg.B if B is None else int(B)
+    H, dk, dv, S = cfg.H, cfg.dk, cfg.dv, cfg.K + 1
+    gs, gk, gv, gg, ga = (rng(cfg.seed, x) for x in (S_STATE, S_KEYS, S_VALUES, S_GATES, S_ACCEPT))
+    state = np.empty((B, H, dk, dv), np.float32)
+    keys = np.empty((B, H, S, dk), np.float32)
+    values = np.empty((B, H, S, dv), np.float32)
+    for b in range(B):
+        state[b] = gs.standard_normal((H, dk, dv), dtype=np.float32)
+        k = gk.standard_normal((H, S, dk), dtype=np.float32)
+        keys[b] = k / np.linalg.norm(k, axis=2, keepdims=True)
+        values[b] = gv.standard_normal((H, S, dv), dtype=np.float32)
+    alpha = gg.uniform(cfg.alpha_lo, 1.0, (B, H, S)).astype(np.float32)
+    beta = gg.uniform(0.0, 1.0, (B, H, S)).astype(np.float32)
+    ok = ga.random((B, cfg.K)) < cfg.accept
+    lead = np.where(ok.all(axis=1), cfg.K, np.argmin(ok, axis=1))
+    steps = (1 + lead).astype(np.int32)
+    return state, alpha, beta, keys, values, steps

@@ -763,3 +763,84 @@ def test_topp_near_tie_below_the_boundary_tries_one_token_fewer():
     d0 = f32_logits([[_ln(14), 0.0, 0.0, None]])[None]
     acc, out, flags = oracle.verify_chain(target, d0, np.array([[0]], np.int32), u, 1.0, 0, top_p)
     assert int(acc[0]) == 1 and int(flags[0]) & oracle.PARITY_FLAGS == 0
+
+
+# --------------------------------------------------------------------------- linear-state commit
+# The recurrence S_t = alpha_t (I - beta_t k_t k_t^T) S_{t-1} + beta_t k_t v_t^T (the gated
+# delta rule of the linear-attention model the SpecLA summary names); pins from its
+# properties, none re-typing the update.
+
+def _lstate(B=2, H=3, dk=8, dv=5, K=4, seed=0):
+    g = np.random.default_rng(seed)
+    S0 = g.normal(size=(B, H, dk, dv)).astype(np.float32)
+    k = g.normal(size=(B, H, K, dk))
+    k = (k / np.linalg.norm(k, axis=3, keepdims=True)).astype(np.float32)
+    v = g.normal(size=(B, H, K, dv)).astype(np.float32)
+    al = g.uniform(0.5, 1.0, (B, H, K)).astype(np.float32)
+    be = g.uniform(0.0, 1.0, (B, H, K)).astype(np.float32)
+    return S0, al, be, k, v
+
+
+def test_linear_state_without_writes_only_decays():
+    """beta = 0: no write; the state decays by the product of the gates."""
+    S0, al, be, k, v = _lstate()
+    steps = np.array([3, 4], np.int32)
+    out = oracle.linear_state_replay(S0, al, np.zeros_like(be), k, v, steps)
+    for b in range(2):
+        g = np.prod(al[b, :, :steps[b]].astype(np.float64), axis=1)
+        np.testing.assert_allclose(out[b], g[:, None, None] * S0[b], rtol=1e-12)
+
+
+def test_linear_state_full_write_stores_the_value_at_its_key():
+    """alpha = beta = 1 and a unit key: reading the state at k gives v (the delta rule
+    replaces what k retrieved), and directions orthogonal to k are untouched."""
+    S0, al, be, k, v = _lstate(B=1, H=1, dk=6, dv=4, K=1, seed=3)
+    out = oracle.linear_state_replay(S0, np.ones_like(al), np.ones_like(be), k, v,
+                                     np.array([1], np.int32))[0, 0]
+    kk = k[0, 0, 0].astype(np.float64)
+    n2 = kk @ kk                                   # 1 up to the key's float32 rounding
+    np.testing.assert_allclose(kk @ out, (1 - n2) * (kk @ S0[0, 0]) + n2 * v[0, 0, 0],
+                               rtol=1e-12, atol=1e-12)
+    assert abs(n2 - 1) < 1e-6
+    x = np.linalg.svd(kk[None])[2][1:]            # an orthonormal basis of k's complement
+    np.testing.assert_allclose(x @ out, x @ S0[0, 0].astype(np.float64), atol=1e-12)
+
+
+def test_linear_state_orthonormal_keys_keep_every_write():
+    """Orthonormal keys, alpha = beta = 1: after a steps every k_t reads back its v_t."""
+    dk, dv, K = 8, 3, 5
+    g = np.random.default_rng(4)
+    q, _ = np.linalg.qr(g.normal(size=(dk, dk)))
+    keys = q[:, :K].T.astype(np.float32)[None, None]          # [1, 1, K, dk]
+    S0 = g.normal(size=(1, 1, dk, dv)).astype(np.float32)
+    v = g.normal(size=(1, 1, K, dv)).astype(np.float32)
+    ones = np.ones((1, 1, K), np.float32)
+    out = oracle.linear_state_replay(S0, ones, ones, keys, v, np.array([K], np.int32))[0, 0]
+    np.testing.assert_allclose(keys[0, 0].astype(np.float64) @ out, v[0, 0], atol=1e-6)
+
+
+def test_linear_state_partial_write_mixes_old_and_new():
+    """A unit key with write strength beta and gate alpha: k^T S_1 = alpha (1 - beta) k^T S_0
+    + beta v (the old content is reduced by beta before the decay, the new one is not
+    decayed); with |k|^2 = n2 from the key's rounding, beta becomes beta * n2."""
+    S0, al, be, k, v = _lstate(B=1, H=1, dk=7, dv=3, K=1, seed=5)
+    out = oracle.linear_state_replay(S0, al, be, k, v, np.array([1], np.int32))[0, 0]
+    kk = k[0, 0, 0].astype(np.float64)
+    n2 = kk @ kk                                   # 1 up to the key's float32 rounding
+    a, b = float(al[0, 0, 0]), float(be[0, 0, 0])
+    np.testing.assert_allclose(kk @ out, a * (1 - b * n2) * (kk @ S0[0, 0]) + b * n2 * v[0, 0, 0],
+                               rtol=1e-10, atol=1e-12)
+
+
+def test_linear_state_prefixes_compose_and_bad_lengths_leave_the_state():
+    """Committing a steps equals committing a - 1 and then one more step from that state;
+    a length of 0 or outside [0, K] leaves the state as it was."""
+    S0, al, be, k, v = _lstate(B=1, H=2, K=4, seed=6)
+    full = oracle.linear_state_replay(S0, al, be, k, v, np.array([3], np.int32))
+    part = oracle.linear_state_replay(S0, al, be, k, v, np.array([2], np.int32))
+    step = oracle.linear_state_replay(part.astype(np.float32), al[:, :, 2:], be[:, :, 2:],
+                                      k[:, :, 2:], v[:, :, 2:], np.array([1], np.int32))
+    np.testing.assert_allclose(step, full, rtol=1e-6, atol=1e-6)   # part rounded to float32
+    for a in (0, -1, 5):
+        same = oracle.linear_state_replay(S0, al, be, k, v, np.array([a], np.int32))
+        np.testing.assert_array_equal(same, S0.astype(np.float64))
