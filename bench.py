@@ -448,9 +448,63 @@ def cpu_baseline(cfg, greedy, budget_s: float = 15.0) -> dict:
                       f"{threads} threads over batch rows, {dt:.1f}s"}
 
 
+def per_config_lstate(cfg, args, dev) -> dict:
+    """Linear-attention state commit after verification: the factors of the round's steps,
+    then the commit of each sequence's accepted prefix to its state, in place. Timed with
+    CUDA events around each commit (the factor kernel is reported beside it)."""
+    import torch
+
+    import draft_token_verification_spec_b200 as sv
+
+    state, alpha, beta, keys, values, steps = specgen.linear_state_inputs(cfg)
+    d = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(dev)
+    st, al, be, k, v, n = d(state), d(alpha), d(beta), d(keys), d(values), d(steps)
+    w, u, g = sv.spec_linear_state_factors(al, be, k, v)
+    torch.cuda.synchronize()
+    ev = _events(args.steps)
+    fev = _events(args.steps)
+    for _ in range(args.warmup):
+        sv.spec_commit_linear_state(st, k, w, u, g, n)
+    torch.cuda.synchronize()
+    for i in range(args.steps):
+        fev[i][0].record()
+        sv.spec_linear_state_factors(al, be, k, v, w, u, g)
+        fev[i][1].record()
+        ev[i][0].record()
+        sv.spec_commit_linear_state(st, k, w, u, g, n)
+        ev[i][1].record()
+    torch.cuda.synchronize()
+    ms = float(np.mean([a.elapsed_time(b) for a, b in ev]))
+    fms = float(np.mean([a.elapsed_time(b) for a, b in fev]))
+    committed = int((steps > 0).sum())
+    S = cfg.K + 1
+    alg = committed * cfg.H * cfg.dk * cfg.dv * 4 * 2 + \
+        int(steps.sum()) * cfg.H * (2 * cfg.dk + cfg.dv) * 4
+    res = {"workload": cfg.name, "metric_unit": "committed steps/s",
+           "value": float(steps.sum()) / (ms / 1e3), "ms_per_step": ms,
+           "factors_ms": round(fms, 4), "mean_steps": float(steps.mean()), "steps_per_round": S,
+           "roofline": roofline_entry(alg, ms, kernel="lstate_commit_kernel")}
+    del st, al, be, k, v, n, w, u, g
+    torch.cuda.empty_cache()
+    if not args.no_cpu_baseline:
+        import oracle
+        threads = os.cpu_count() or 1
+        rows = min(cfg.B, 4 * threads)
+        t0 = time.perf_counter()
+        oracle.linear_state_replay(state[:rows], alpha[:rows], beta[:rows], keys[:rows],
+                                   values[:rows], steps[:rows], threads=threads)
+        dt = time.perf_counter() - t0
+        res["cpu_baseline"] = {"value": float(steps[:rows].sum()) / dt,
+                               "unit": "committed steps/s", "cores": threads, "kind": "oracle",
+                               "sample": f"first {rows} of {cfg.B} sequences (step-by-step "
+                                         f"replay), {threads} threads, {dt:.2f}s"}
+    return res
+
+
 def per_config_all(args) -> list:
     """Every other workload, one entry each (1 GPU): the three other chain workloads, the
-    temperature-0 variants of the two that have one, and the MEDUSA tree."""
+    temperature-0 variants of the two that have one, the MEDUSA tree, and the
+    linear-attention state commit."""
     import torch
 
     dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", 0)))
@@ -460,6 +514,7 @@ def per_config_all(args) -> list:
         out.append(per_config_chain(cfg, greedy, args, dev))
         log(f"per-config {out[-1]['workload']}: {out[-1]['ms_per_step']:.4f} ms")
     out.append(per_config_tree(specgen.CFG4, args, dev))
+    out.append(per_config_lstate(specgen.LSTATE, args, dev))
     return out
 
 

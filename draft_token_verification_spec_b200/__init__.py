@@ -51,6 +51,8 @@ def _declare(lib):
         "spec_logits_to_probs": ([P, I, I, I, F, I, F, P, P, P], I),
         "spec_residual_sample": ([P, P, I, I, P, P, P], I),
         "spec_get_device_status": ([P, P, P], I),
+        "spec_linear_state_factors": ([P, P, P, P, I, I, I, I, I, P, P, P, P], I),
+        "spec_commit_linear_state": ([P, I, I, I, I, I, P, P, P, P, P, P], I),
         "spec_set_row_kernel_events": ([P, P], None),
         "spec_kernels_per_call": ([ctypes.c_char_p], I),
     }
@@ -299,6 +301,55 @@ def spec_residual_sample(p, q, uniforms, tokens=None, stream=None):
         _check("spec_residual_sample", lib().spec_residual_sample(
             _ptr(pp), _ptr(qq), rows, V, _ptr(u), _ptr(tokens), _stream(stream, pp.device)))
     return tokens
+
+
+def spec_linear_state_factors(alpha, beta, keys, values, w=None, u=None, gamma=None,
+                              stream=None):
+    """Compact factors of every prefix of a round's S steps (gated delta rule). alpha, beta
+    float32 [B,H,S]; keys [B,H,S,dk]; values [B,H,S,dv]. Returns (w [B,H,S,dk], u [B,H,S,dv],
+    gamma [B,H,S])."""
+    al = _dev(alpha, "alpha", torch.float32)
+    be = _dev(beta, "beta", torch.float32)
+    k = _dev(keys, "keys", torch.float32)
+    v = _dev(values, "values", torch.float32)
+    B, H, S = al.shape
+    dk, dv = k.shape[3], v.shape[3]
+    if tuple(be.shape) != (B, H, S) or tuple(k.shape[:3]) != (B, H, S) or \
+            tuple(v.shape[:3]) != (B, H, S):
+        raise ValueError("alpha, beta [B,H,S], keys [B,H,S,dk], values [B,H,S,dv]")
+    if w is None:
+        w = torch.empty((B, H, S, dk), dtype=torch.float32, device=k.device)
+    if u is None:
+        u = torch.empty((B, H, S, dv), dtype=torch.float32, device=k.device)
+    if gamma is None:
+        gamma = torch.empty((B, H, S), dtype=torch.float32, device=k.device)
+    with torch.cuda.device(k.device):  # launches go to the tensors' device
+        _check("spec_linear_state_factors", lib().spec_linear_state_factors(
+            _ptr(al), _ptr(be), _ptr(k), _ptr(v), B, H, S, dk, dv, _ptr(w), _ptr(u),
+            _ptr(gamma), _stream(stream, k.device)))
+    return w, u, gamma
+
+
+def spec_commit_linear_state(state, keys, w, u, gamma, steps, stream=None):
+    """In place: state float32 [B,H,dk,dv] becomes the state after steps[b] steps of its
+    round (keys, w [B,H,S,dk]; u [B,H,S,dv]; gamma [B,H,S]; steps int32 [B])."""
+    st = _dev(state, "state", torch.float32)
+    B, H, dk, dv = st.shape
+    k = _dev(keys, "keys", torch.float32)
+    S = k.shape[2]
+    ww = _dev(w, "w", torch.float32)
+    uu = _dev(u, "u", torch.float32)
+    g = _dev(gamma, "gamma", torch.float32)
+    n = _dev(steps, "steps", torch.int32)
+    if tuple(k.shape) != (B, H, S, dk) or tuple(ww.shape) != (B, H, S, dk) or \
+            tuple(uu.shape) != (B, H, S, dv) or tuple(g.shape) != (B, H, S) or \
+            tuple(n.shape) != (B,):
+        raise ValueError("keys, w [B,H,S,dk]; u [B,H,S,dv]; gamma [B,H,S]; steps [B]")
+    with torch.cuda.device(st.device):  # launches go to the tensors' device
+        _check("spec_commit_linear_state", lib().spec_commit_linear_state(
+            _ptr(st), B, H, dk, dv, S, _ptr(k), _ptr(ww), _ptr(uu), _ptr(g), _ptr(n),
+            _stream(stream, st.device)))
+    return st
 
 
 def spec_get_device_status(workspace, stream=None) -> int:

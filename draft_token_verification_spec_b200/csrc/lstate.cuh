@@ -1,0 +1,195 @@
+// Linear-attention state commit after verification (the SpecLA summary, gist.science: a
+// linear-attention model keeps one dense state per head that every token updates; after the
+// verdict the state is brought to the accepted prefix from small per-step "factors" saved
+// during verification, instead of replaying the accepted tokens).
+//
+// The state of one sequence and head, S in R^{dk x dv}, follows the gated delta rule
+//   S_t = alpha_t (I - beta_t k_t k_t^T) S_{t-1} + beta_t k_t v_t^T.
+// With G_t = alpha_1 ... alpha_t and the WY vectors
+//   w_t = beta_t (k_t - sum_{s<t} (k_t . k_s) w_s)                 (length dk)
+//   u_t = beta_t (v_t / G_t - sum_{s<t} (k_t . k_s) u_s)           (length dv)
+// every prefix of a steps has the closed form
+//   S_a = G_a (S_0 + sum_{t<=a} k_t (u_t - S_0^T w_t)^T),
+// because prod_{t=a..1} (I - beta_t k_t k_t^T) = I - sum_{t<=a} k_t w_t^T and the rescaled
+// state S_t / G_t follows the same rule with values v_t / G_t. The vectors of step t depend
+// only on steps <= t, so one set of factors serves every acceptance length.
+//
+//   lstate_factors_kernel: one block per (sequence, head); the Gram products k_t . k_s, the
+//     gates G_t, then w_t and u_t in step order (each step parallel over dk or dv).
+//   lstate_commit_kernel: one block per (sequence, head, 64-column tile of S); the tile stays
+//     in registers: M = U_a - W_a S_0 (a x 64; each warp owns 8 columns and reduces its
+//     16 row lanes by shuffles), then S_a = G_a (S_0 + K_a^T M), written back in place. A
+//     sequence committing 0 steps (or an invalid length) is not touched. Bandwidth-bound:
+//     one read and one write of the state per committed sequence.
+#pragma once
+
+#include "common.cuh"
+
+namespace sv {
+
+constexpr int kLsMaxSteps = 32;   // steps per round (drafts + the deferred token)
+constexpr int kLsMaxDk = 256;
+constexpr int kLsCols = 64;       // columns of S per commit block
+
+struct LsFactorJob {
+  const float* alpha;   // [B][H][S]
+  const float* beta;    // [B][H][S]
+  const float* keys;    // [B][H][S][dk]
+  const float* values;  // [B][H][S][dv]
+  int B, H, S, dk, dv;
+  float* w;             // [B][H][S][dk]
+  float* u;             // [B][H][S][dv]
+  float* gamma;         // [B][H][S]: G_t for t = 1..S
+};
+
+__global__ void __launch_bounds__(kThreads) lstate_factors_kernel(const LsFactorJob j) {
+  __shared__ float kk[kLsMaxSteps * kLsMaxDk];
+  __shared__ float gram[kLsMaxSteps][kLsMaxSteps];
+  __shared__ float g[kLsMaxSteps];
+  const int bh = blockIdx.x, S = j.S, dk = j.dk, dv = j.dv;
+  const float* kin = j.keys + size_t(bh) * S * dk;
+  for (int i = threadIdx.x; i < S * dk; i += kThreads) kk[i] = kin[i];
+  if (threadIdx.x == 0) {
+    float acc = 1.0f;
+    for (int t = 0; t < S; ++t) {
+      acc *= j.alpha[size_t(bh) * S + t];
+      g[t] = acc;
+      j.gamma[size_t(bh) * S + t] = acc;
+    }
+  }
+  __syncthreads();
+  // Gram products k_t . k_s (s < t), one warp per pair
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  for (int p = warp; p < S * S; p += kWarps) {
+    const int t = p / S, s = p % S;
+    if (s >= t) continue;
+    float acc = 0.0f;
+    for (int i = lane; i < dk; i += 32) acc += kk[t * dk + i] * kk[s * dk + i];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+    if (lane == 0) gram[t][s] = acc;
+  }
+  __syncthreads();
+  const float* bet = j.beta + size_t(bh) * S;
+  float* wout = j.w + size_t(bh) * S * dk;
+  float* uout = j.u + size_t(bh) * S * dv;
+  const float* vin = j.values + size_t(bh) * S * dv;
+  // w_t and u_t in step order; a thread owns fixed entries, so it reads back only its own
+  // earlier writes
+  for (int t = 0; t < S; ++t) {
+    const float bt = bet[t];
+    for (int i = threadIdx.x; i < dk; i += kThreads) {
+      float x = kk[t * dk + i];
+      for (int s = 0; s < t; ++s) x -= gram[t][s] * wout[s * dk + i];
+      wout[t * dk + i] = bt * x;
+    }
+    const float inv_g = 1.0f / g[t];
+    for (int i = threadIdx.x; i < dv; i += kThreads) {
+      float x = vin[t * dv + i] * inv_g;
+      for (int s = 0; s < t; ++s) x -= gram[t][s] * uout[s * dv + i];
+      uout[t * dv + i] = bt * x;
+    }
+  }
+}
+
+struct LsCommitJob {
+  float* state;         // [B][H][dk][dv], updated in place
+  int B, H, S, dk, dv;
+  const float* keys;    // [B][H][S][dk]
+  const float* w;       // [B][H][S][dk]
+  const float* u;       // [B][H][S][dv]
+  const float* gamma;   // [B][H][S]
+  const int32_t* steps; // [B]: steps to commit (0..S; anything else leaves the state)
+  int tiles;            // column tiles per head: ceil(dv / kLsCols)
+};
+
+// R rows of S per lane: dk = 16 R (16 row lanes per warp).
+// Dynamic shared memory: keys and w of S steps (S x dk each), then M (S x kLsCols).
+__host__ __device__ constexpr size_t lstate_commit_smem(int S, int dk) {
+  return size_t(S) * dk * 8 + size_t(S) * kLsCols * 4;
+}
+
+template <int R>
+__global__ void __launch_bounds__(kThreads) lstate_commit_kernel(const LsCommitJob j) {
+  extern __shared__ __align__(16) float lsm[];
+  constexpr int dk = 16 * R;
+  float* ks = lsm;                                            // [S][dk]
+  float* ws = ks + size_t(j.S) * dk;                          // [S][dk]
+  float (*mt)[kLsCols] = reinterpret_cast<float (*)[kLsCols]>(ws + size_t(j.S) * dk);
+  const long long blk = blockIdx.x;
+  const int tile = int(blk % j.tiles);
+  const long long bh = blk / j.tiles;
+  const int b = int(bh / j.H);
+  const int a = j.steps[b];
+  if (a <= 0 || a > j.S) return;  // nothing to commit (uniform)
+  const int S = j.S, dv = j.dv;
+  for (int i = threadIdx.x; i < a * dk; i += kThreads) {
+    ks[i] = j.keys[size_t(bh) * S * dk + i];
+    ws[i] = j.w[size_t(bh) * S * dk + i];
+  }
+  const float* urow = j.u + size_t(bh) * S * dv;
+  const int c0 = tile * kLsCols;
+  for (int i = threadIdx.x; i < a * kLsCols; i += kThreads) {
+    const int t = i / kLsCols, c = c0 + i % kLsCols;
+    mt[t][i % kLsCols] = c < dv ? urow[size_t(t) * dv + c] : 0.0f;
+  }
+  const float ga = j.gamma[size_t(bh) * S + a - 1];
+  __syncthreads();
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int rl = lane & 15;                          // row lane: rows rl, rl + 16, ...
+  const int cl = warp * 8 + (lane >> 4) * 4;         // first of this lane's 4 columns (in tile)
+  const int col = c0 + cl;
+  const bool live = col < dv;                        // dv % 4 == 0: a quad is all in or out
+  float* base = j.state + size_t(bh) * dk * dv;
+  float4 x[R];
+#pragma unroll
+  for (int r = 0; r < R; ++r)
+    x[r] = live ? *reinterpret_cast<const float4*>(base + size_t(rl + 16 * r) * dv + col)
+                : make_float4(0.f, 0.f, 0.f, 0.f);
+  // M[t][c] = U[t][c] - sum_i W[t][i] S[i][c]: partial sums over this lane's rows, then the
+  // 16 row lanes of the warp (xor shuffles keep them within the half-warp)
+  for (int t = 0; t < a; ++t) {
+    float4 p = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+      const float wv = ws[t * dk + rl + 16 * r];
+      p.x = fmaf(wv, x[r].x, p.x);
+      p.y = fmaf(wv, x[r].y, p.y);
+      p.z = fmaf(wv, x[r].z, p.z);
+      p.w = fmaf(wv, x[r].w, p.w);
+    }
+#pragma unroll
+    for (int o = 1; o < 16; o <<= 1) {
+      p.x += __shfl_xor_sync(0xffffffffu, p.x, o);
+      p.y += __shfl_xor_sync(0xffffffffu, p.y, o);
+      p.z += __shfl_xor_sync(0xffffffffu, p.z, o);
+      p.w += __shfl_xor_sync(0xffffffffu, p.w, o);
+    }
+    if (rl == 0) {
+      mt[t][cl + 0] -= p.x;
+      mt[t][cl + 1] -= p.y;
+      mt[t][cl + 2] -= p.z;
+      mt[t][cl + 3] -= p.w;
+    }
+  }
+  __syncwarp();  // each warp reads back only its own columns of mt
+  // S_a = G_a (S_0 + K^T M)
+#pragma unroll
+  for (int r = 0; r < R; ++r) {
+    float4 y = x[r];
+    for (int t = 0; t < a; ++t) {
+      const float kv = ks[t * dk + rl + 16 * r];
+      y.x = fmaf(kv, mt[t][cl + 0], y.x);
+      y.y = fmaf(kv, mt[t][cl + 1], y.y);
+      y.z = fmaf(kv, mt[t][cl + 2], y.z);
+      y.w = fmaf(kv, mt[t][cl + 3], y.w);
+    }
+    y.x *= ga;
+    y.y *= ga;
+    y.z *= ga;
+    y.w *= ga;
+    if (live) *reinterpret_cast<float4*>(base + size_t(rl + 16 * r) * dv + col) = y;
+  }
+}
+
+}  // namespace sv

@@ -8,6 +8,7 @@
 #include <tuple>
 
 #include "chain.cuh"
+#include "lstate.cuh"
 #include "probs.cuh"
 #include "refine.cuh"
 #include "row_stats.cuh"
@@ -376,6 +377,16 @@ spec_status verify_tree(const void* target_logits, spec_dtype dtype, int B, int 
   return check_launch(cudaGetLastError());
 }
 
+template <int R>
+cudaError_t launch_commit(const sv::LsCommitJob& j, cudaStream_t s) {
+  const size_t dyn = sv::lstate_commit_smem(j.S, 16 * R);
+  cudaError_t e = cudaFuncSetAttribute(sv::lstate_commit_kernel<R>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, int(dyn));
+  if (e != cudaSuccess) return e;
+  const long long blocks = (long long)j.B * j.H * j.tiles;
+  sv::lstate_commit_kernel<R><<<unsigned(blocks), kThreads, dyn, s>>>(j);
+  return cudaGetLastError();
+}
 }  // namespace
 
 extern "C" {
@@ -620,6 +631,44 @@ spec_status spec_residual_sample(const float* p, const float* q, int rows, int V
   return check_launch(cudaGetLastError());
 }
 
+spec_status spec_linear_state_factors(const float* alpha, const float* beta, const float* keys,
+                                      const float* values, int B, int H, int S, int dk, int dv,
+                                      float* w, float* u, float* gamma, void* stream) {
+  if (!alpha || !beta || !keys || !values || !w || !u || !gamma || B <= 0 || H <= 0 || S <= 0 ||
+      dk <= 0 || dv <= 0)
+    return SPEC_ERR_INVALID_ARG;
+  if (S > sv::kLsMaxSteps || dk > sv::kLsMaxDk || (long long)B * H > 0x7fffffffLL)
+    return SPEC_ERR_UNSUPPORTED;
+  sv::LsFactorJob j = {alpha, beta, keys, values, B, H, S, dk, dv, w, u, gamma};
+  sv::lstate_factors_kernel<<<unsigned(B * H), kThreads, 0, static_cast<cudaStream_t>(stream)>>>(
+      j);
+  return check_launch(cudaGetLastError());
+}
+
+spec_status spec_commit_linear_state(float* state, int B, int H, int dk, int dv, int S,
+                                     const float* keys, const float* w, const float* u,
+                                     const float* gamma, const int32_t* steps, void* stream) {
+  if (!state || !keys || !w || !u || !gamma || !steps || B <= 0 || H <= 0 || S <= 0 || dk <= 0 ||
+      dv <= 0)
+    return SPEC_ERR_INVALID_ARG;
+  if (S > sv::kLsMaxSteps || dv % 4 != 0 || !aligned16(state) ||
+      (dk != 32 && dk != 64 && dk != 128 && dk != 256))
+    return SPEC_ERR_UNSUPPORTED;
+  const long long blocks = (long long)B * H * ((dv + sv::kLsCols - 1) / sv::kLsCols);
+  if (blocks > 0x7fffffffLL) return SPEC_ERR_UNSUPPORTED;
+  sv::LsCommitJob j = {state, B, H, S, dk, dv, keys, w, u, gamma, steps,
+                       (dv + sv::kLsCols - 1) / sv::kLsCols};
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e;
+  switch (dk) {
+    case 32: e = launch_commit<2>(j, s); break;
+    case 64: e = launch_commit<4>(j, s); break;
+    case 128: e = launch_commit<8>(j, s); break;
+    default: e = launch_commit<16>(j, s); break;
+  }
+  return check_launch(e);
+}
+
 spec_status spec_get_device_status(const void* workspace, int32_t* status_out, void* stream) {
   if (!workspace || !status_out) return SPEC_ERR_INVALID_ARG;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
@@ -644,6 +693,8 @@ int spec_kernels_per_call(const char* entry_point) {
   if (!std::strcmp(entry_point, "spec_verify_tree_sampling")) return 4;
   if (!std::strcmp(entry_point, "spec_logits_to_probs")) return 1;
   if (!std::strcmp(entry_point, "spec_residual_sample")) return 1;
+  if (!std::strcmp(entry_point, "spec_linear_state_factors")) return 1;
+  if (!std::strcmp(entry_point, "spec_commit_linear_state")) return 1;
   return -1;
 }
 

@@ -188,6 +188,34 @@ spec_status spec_logits_to_probs(const void* logits, spec_dtype dtype, int rows,
 spec_status spec_residual_sample(const float* p, const float* q, int rows, int V,
                                  const float* uniforms, int32_t* tokens, void* stream);
 
+/* Linear-attention state commit after verification — [SpecLA] gist.science summary of
+ * "SpecLA: Efficient Speculative Decoding for Linear-Attention Models" (a linear-attention
+ * target keeps one dense state per head; after the verdict the state is brought to the
+ * accepted prefix from compact per-step factors saved during verification, with no replay).
+ * The state of sequence b, head h is S in R^{dk x dv} (row-major, float32) and follows the
+ * gated delta rule S_t = alpha_t (I - beta_t k_t k_t^T) S_{t-1} + beta_t k_t v_t^T over the
+ * S steps of one round (e.g. the previous round's emitted token, whose update was
+ * deferred, then the K drafts).
+ *
+ * spec_linear_state_factors: the factors of every prefix, from the round's per-step data.
+ *   alpha, beta [B][H][S], keys [B][H][S][dk], values [B][H][S][dv] (float32, device);
+ *   w [B][H][S][dk], u [B][H][S][dv], gamma [B][H][S] out (device, caller-allocated):
+ *   gamma_t = alpha_1 .. alpha_t, w_t = beta_t (k_t - sum_{s<t} (k_t . k_s) w_s),
+ *   u_t = beta_t (v_t / gamma_t - sum_{s<t} (k_t . k_s) u_s). 1 <= S <= 32, dk <= 256. The
+ *   values are divided by the cumulative gate, so gates far below 1 over many steps lose
+ *   float32 precision.
+ * spec_commit_linear_state: state [B][H][dk][dv] (device, 16-byte aligned) is replaced, in
+ *   place, by the state after steps[b] steps (int32 [B], device):
+ *   S_a = gamma_a (S_0 + sum_{t<=a} k_t (u_t - S_0^T w_t)^T). A sequence with steps[b] = 0,
+ *   or outside [0, S], is left untouched (not read or written). dk in {32, 64, 128, 256},
+ *   dv a multiple of 4, S <= 32. One read and one write of each committed state. */
+spec_status spec_linear_state_factors(const float* alpha, const float* beta, const float* keys,
+                                      const float* values, int B, int H, int S, int dk, int dv,
+                                      float* w, float* u, float* gamma, void* stream);
+spec_status spec_commit_linear_state(float* state, int B, int H, int dk, int dv, int S,
+                                     const float* keys, const float* w, const float* u,
+                                     const float* gamma, const int32_t* steps, void* stream);
+
 /* spec_verify_chain without a caller workspace. The pages have no counterpart: they
  * state the verification rule, not an interface; this call is the library's own.
  *
