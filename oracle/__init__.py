@@ -74,6 +74,8 @@ def _load():
         _lib.oracle_verify_tree_sampling.restype = I
         _lib.oracle_verify_tree_sampling_f64u.restype = I
         _lib.oracle_linear_state_replay.argtypes = [P, I, I, I, I, I, P, P, P, P, P, P, I]
+        _lib.oracle_lmhead_logits.argtypes = [P, P, I, I, I, P, I]
+        _lib.oracle_lmhead_logits.restype = I
         _lib.oracle_linear_state_replay.restype = I
         for f in (_lib.oracle_transform_rows, _lib.oracle_verify_chain,
                   _lib.oracle_verify_chain_f64u, _lib.oracle_verify_tree_greedy,
@@ -262,4 +264,20 @@ def linear_state_replay(state0, alpha, beta, keys, values, steps, threads=None):
                                             _ptr(out), _threads(threads))
     if rc != 0:
         raise ValueError("oracle_linear_state_replay rejected its arguments")
+    return out
+
+
+def lmhead_logits(hidden, weight, threads=None):
+    """logits [rows, V] float64 = hidden [rows, d] @ weight[V, d]^T, both bfloat16 bit
+    patterns (uint16), summed in double."""
+    hidden = np.ascontiguousarray(hidden, np.uint16)
+    weight = np.ascontiguousarray(weight, np.uint16)
+    rows, d = hidden.shape
+    V = weight.shape[0]
+    assert weight.shape == (V, d)
+    out = np.zeros((rows, V), np.float64)
+    rc = _load().oracle_lmhead_logits(_ptr(hidden), _ptr(weight), rows, V, d, _ptr(out),
+                                      _threads(threads))
+    if rc != 0:
+        raise ValueError("oracle_lmhead_logits rejected its arguments")
     return out

@@ -747,6 +747,28 @@ int oracle_residual_sample(const float* p, const float* q, int rows, int V, cons
   return 0;
 }
 
+// Logits of the scoring forward's last layer: logits[r][v] = sum_j hidden[r][j] * weight[v][j]
+// (the LM head, weight row v = token v's output embedding), in double from bfloat16 inputs.
+// The pages put the bandwidth and compute of a round in the target's forward ([SD]
+// "Speculative Sampling": scoring K drafts costs about one forward because the linear layers
+// are memory-bound at small batch); this is its final matrix product, written as plain loops.
+// hidden [rows][d], weight [V][d] bfloat16 bit patterns; out [rows][V] double.
+int oracle_lmhead_logits(const uint16_t* hidden, const uint16_t* weight, int rows, int V, int d,
+                         double* out, int threads) {
+  if (!hidden || !weight || !out || rows < 0 || V <= 0 || d <= 0) return -1;
+  parallel_rows(rows, threads, [&](int r) {
+    std::vector<double> h(static_cast<size_t>(d));
+    for (int j = 0; j < d; ++j) h[j] = bf16_bits_to_double(hidden[size_t(r) * d + j]);
+    for (int v = 0; v < V; ++v) {
+      const uint16_t* w = weight + size_t(v) * d;
+      double acc = 0.0;
+      for (int j = 0; j < d; ++j) acc += h[j] * bf16_bits_to_double(w[j]);
+      out[size_t(r) * V + v] = acc;
+    }
+  });
+  return 0;
+}
+
 // State commit after verification for a linear-attention target ([SpecLA] summary: the
 // state is a dense summary updated with every token, and after the verdict it is brought to
 // the accepted prefix; the summary names the gated-delta-rule model GDN). The recurrence,

@@ -844,3 +844,31 @@ def test_linear_state_prefixes_compose_and_bad_lengths_leave_the_state():
     for a in (0, -1, 5):
         same = oracle.linear_state_replay(S0, al, be, k, v, np.array([a], np.int32))
         np.testing.assert_array_equal(same, S0.astype(np.float64))
+
+
+# --------------------------------------------------------------------------- LM-head logits
+
+def test_lmhead_logits_exact_on_small_integers():
+    """Small integers are exact in bfloat16 and their products and sums are exact in double:
+    the logits equal the integer matrix product exactly."""
+    g = np.random.default_rng(21)
+    h = g.integers(-8, 9, (5, 33)).astype(np.float32)
+    w = g.integers(-8, 9, (70, 33)).astype(np.float32)
+    got = oracle.lmhead_logits(specgen.f32_to_bf16_bits(h), specgen.f32_to_bf16_bits(w))
+    exact = h.astype(np.int64) @ w.astype(np.int64).T
+    np.testing.assert_array_equal(got, exact.astype(np.float64))
+
+
+def test_lmhead_logits_match_numpy_matmul():
+    """Random bfloat16 inputs: the loops agree with numpy's float64 matmul (a different
+    summation order) to double rounding."""
+    g = np.random.default_rng(22)
+    hb = specgen.f32_to_bf16_bits(g.normal(size=(7, 256)).astype(np.float32))
+    wb = specgen.f32_to_bf16_bits((g.normal(size=(300, 256)) / 16).astype(np.float32))
+    got = oracle.lmhead_logits(hb, wb)
+    ref = specgen.bf16_bits_to_f32(hb).astype(np.float64) @ \
+        specgen.bf16_bits_to_f32(wb).astype(np.float64).T
+    np.testing.assert_allclose(got, ref, rtol=1e-12, atol=1e-12)
+    # a transposed operand or a dropped row would not match
+    assert not np.allclose(got[:, :7], (specgen.bf16_bits_to_f32(hb).astype(np.float64) @
+                                        specgen.bf16_bits_to_f32(hb).astype(np.float64).T)[:, :7])
