@@ -109,6 +109,15 @@ def _dev(t: torch.Tensor, name: str, dtype=None) -> torch.Tensor:
     return t
 
 
+def _on(device):
+    """Makes `device` current for the call when it is not already (launches go to the
+    tensors' device); a no-op context otherwise, so the common case costs nothing."""
+    import contextlib
+    if device.index is None or device.index == torch.cuda.current_device():
+        return contextlib.nullcontext()
+    return torch.cuda.device(device)
+
+
 def _ptr(t):
     return None if t is None else ctypes.c_void_p(t.data_ptr())
 
@@ -145,7 +154,7 @@ def spec_verify_chain(target_logits, draft_logits, draft_tokens, uniforms, temp,
         out_tokens = torch.empty((B, K + 1), dtype=torch.int32, device=t.device)
     if workspace is None:
         workspace = torch.empty(spec_workspace_size(B, K, V), dtype=torch.uint8, device=t.device)
-    with torch.cuda.device(t.device):  # launches go to the tensors' device
+    with _on(t.device):
         _check("spec_verify_chain", lib().spec_verify_chain(
             _ptr(t), _ptr(d), _dtype(t), B, K, V, _ptr(x), _ptr(u), float(temp), int(top_k),
             float(top_p), _ptr(accepted_len), _ptr(out_tokens), _ptr(workspace),
@@ -172,7 +181,7 @@ def spec_verify_chain_noalloc(target_logits, draft_logits, draft_tokens, uniform
         accepted_len = torch.empty(B, dtype=torch.int32, device=t.device)
     if out_tokens is None:
         out_tokens = torch.empty((B, K + 1), dtype=torch.int32, device=t.device)
-    with torch.cuda.device(t.device):  # launches go to the tensors' device
+    with _on(t.device):
         _check("spec_verify_chain_noalloc", lib().spec_verify_chain_noalloc(
             _ptr(t), _ptr(d), _dtype(t), B, K, V, _ptr(x), _ptr(u), float(temp), int(top_k),
             float(top_p), _ptr(accepted_len), _ptr(out_tokens), _stream(stream, t.device)))
@@ -197,7 +206,7 @@ def spec_verify_tree_typical(target_logits, node_tokens, parent_idx, eps, delta,
         accepted_len = torch.empty(B, dtype=torch.int32, device=t.device)
     if workspace is None:
         workspace = torch.empty(spec_workspace_size(B, N, V), dtype=torch.uint8, device=t.device)
-    with torch.cuda.device(t.device):  # launches go to the tensors' device
+    with _on(t.device):
         _check("spec_verify_tree_typical", lib().spec_verify_tree_typical(
             _ptr(t), _dtype(t), B, N, V, _ptr(nt), _ptr(par), float(eps), float(delta),
             _ptr(best_path), cap, _ptr(accepted_len), _ptr(workspace),
@@ -226,7 +235,7 @@ def spec_verify_tree_greedy(target_logits, node_tokens, parent_idx, path_cap=Non
         next_token = torch.empty(B, dtype=torch.int32, device=t.device)
     if workspace is None:
         workspace = torch.empty(spec_workspace_size(B, N, V), dtype=torch.uint8, device=t.device)
-    with torch.cuda.device(t.device):  # launches go to the tensors' device
+    with _on(t.device):
         _check("spec_verify_tree_greedy", lib().spec_verify_tree_greedy(
             _ptr(t), _dtype(t), B, N, V, _ptr(nt), _ptr(par), _ptr(best_path), cap,
             _ptr(accepted_len), _ptr(next_token), _ptr(workspace),
@@ -259,7 +268,7 @@ def spec_verify_tree_sampling(target_logits, draft_logits, node_tokens, parent_i
         next_token = torch.empty(B, dtype=torch.int32, device=t.device)
     if workspace is None:
         workspace = torch.empty(spec_workspace_size(B, N, V), dtype=torch.uint8, device=t.device)
-    with torch.cuda.device(t.device):  # launches go to the tensors' device
+    with _on(t.device):
         _check("spec_verify_tree_sampling", lib().spec_verify_tree_sampling(
             _ptr(t), _ptr(d), _dtype(t), B, N, V, _ptr(nt), _ptr(par), _ptr(u), float(temp),
             int(top_k), float(top_p), _ptr(best_path), cap, _ptr(accepted_len), _ptr(next_token),
@@ -279,7 +288,7 @@ def spec_logits_to_probs(logits, temp, top_k=0, top_p=1.0, with_entropy=True, pr
         probs = torch.empty(lg.shape, dtype=torch.float32, device=lg.device)
     if with_entropy and entropy is None:
         entropy = torch.empty(lg.shape[:-1], dtype=torch.float32, device=lg.device)
-    with torch.cuda.device(lg.device):  # launches go to the tensors' device
+    with _on(lg.device):
         _check("spec_logits_to_probs", lib().spec_logits_to_probs(
             _ptr(lg), _dtype(lg), rows, V, float(temp), int(top_k), float(top_p), _ptr(probs),
             _ptr(entropy), _stream(stream, lg.device)))
@@ -297,7 +306,7 @@ def spec_residual_sample(p, q, uniforms, tokens=None, stream=None):
     u = _dev(uniforms, "uniforms", torch.float32)
     if tokens is None:
         tokens = torch.empty(rows, dtype=torch.int32, device=pp.device)
-    with torch.cuda.device(pp.device):  # launches go to the tensors' device
+    with _on(pp.device):
         _check("spec_residual_sample", lib().spec_residual_sample(
             _ptr(pp), _ptr(qq), rows, V, _ptr(u), _ptr(tokens), _stream(stream, pp.device)))
     return tokens
@@ -323,7 +332,7 @@ def spec_linear_state_factors(alpha, beta, keys, values, w=None, u=None, gamma=N
         u = torch.empty((B, H, S, dv), dtype=torch.float32, device=k.device)
     if gamma is None:
         gamma = torch.empty((B, H, S), dtype=torch.float32, device=k.device)
-    with torch.cuda.device(k.device):  # launches go to the tensors' device
+    with _on(k.device):
         _check("spec_linear_state_factors", lib().spec_linear_state_factors(
             _ptr(al), _ptr(be), _ptr(k), _ptr(v), B, H, S, dk, dv, _ptr(w), _ptr(u),
             _ptr(gamma), _stream(stream, k.device)))
@@ -345,7 +354,7 @@ def spec_commit_linear_state(state, keys, w, u, gamma, steps, stream=None):
             tuple(uu.shape) != (B, H, S, dv) or tuple(g.shape) != (B, H, S) or \
             tuple(n.shape) != (B,):
         raise ValueError("keys, w [B,H,S,dk]; u [B,H,S,dv]; gamma [B,H,S]; steps [B]")
-    with torch.cuda.device(st.device):  # launches go to the tensors' device
+    with _on(st.device):
         _check("spec_commit_linear_state", lib().spec_commit_linear_state(
             _ptr(st), B, H, dk, dv, S, _ptr(k), _ptr(ww), _ptr(uu), _ptr(g), _ptr(n),
             _stream(stream, st.device)))
@@ -354,7 +363,7 @@ def spec_commit_linear_state(state, keys, w, u, gamma, steps, stream=None):
 
 def spec_get_device_status(workspace, stream=None) -> int:
     out = ctypes.c_int32(0)
-    with torch.cuda.device(workspace.device):  # launches go to the tensors' device
+    with _on(workspace.device):
         _check("spec_get_device_status", lib().spec_get_device_status(
             _ptr(workspace), ctypes.byref(out), _stream(stream, workspace.device)))
     return int(out.value)

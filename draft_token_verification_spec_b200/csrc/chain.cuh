@@ -46,11 +46,14 @@ __device__ __forceinline__ int row_event(const RowStats& s) {
   return s.status == ROW_OK ? EV_ACCEPT : (s.status == ROW_TIMEOUT ? EV_TIMEOUT : EV_ERROR);
 }
 
+constexpr int kZPos = 32;  // positions whose listed rows get their normalisers up front
+
 template <typename T>
 __global__ void __launch_bounds__(kThreads) chain_finish_kernel(const ChainJob j) {
   __shared__ DrawSmem sm;
   __shared__ int s_a, s_ev, s_zpos;
   __shared__ double s_z[2];  // zd of p and q at position s_zpos, summed by the block
+  __shared__ double s_zl[2][kZPos];  // zd of p and q at positions < kZPos (< 0: unknown)
   const int b = blockIdx.x;
   const int K = j.K, V = j.V;
   const RowStats* ts = j.stats + size_t(b) * (K + 1);
@@ -59,8 +62,35 @@ __global__ void __launch_bounds__(kThreads) chain_finish_kernel(const ChainJob j
   const T* drow0 = j.greedy ? nullptr : static_cast<const T*>(j.draft) + size_t(b) * K * V;
   const int32_t* x = j.tokens + size_t(b) * K;
   const float* u = j.uniforms + size_t(b) * (K + 1);
-  const double Tt = double(j.temp);
+  const double iT = 1.0 / double(j.temp);  // greedy rows never use it
   if (threadIdx.x == 0) s_zpos = -1;
+  const int npos = min(K + 1, kZPos);
+  if (!j.greedy) {
+    // rows that list their kept ids: the double normaliser over the list, one warp per row
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    for (int r = warp; r < 2 * npos; r += kWarps) {
+      const bool tgt = r < npos;
+      const int i = tgt ? r : r - npos;
+      double z = -1.0;
+      if (tgt || i < K) {
+        const RowStats st = tgt ? ts[i] : ds[i];
+        const size_t gr = tgt ? size_t(b) * (K + 1) + i : size_t(j.B) * (K + 1) + size_t(b) * K + i;
+        const int nk = j.kept_n ? j.kept_n[gr] : 0;
+        z = st.zd;
+        if (z < 0.0 && st.status == ROW_OK && nk > 0) {
+          const T* row = tgt ? trow0 + size_t(i) * V : drow0 + size_t(i) * V;
+          const int32_t* ids = j.kept_ids + gr * kKeptCap;
+          Fx128 acc = fx_zero();
+          for (int q = lane; q < nk; q += 32) {
+            const int v = ids[q];
+            acc = fx_add(acc, fx_from(kept_weight_d<T>(st, iT, Elem<T>::load(row, size_t(v)), v)));
+          }
+          z = fx_to_double(warp_sum_fx(acc));
+        }
+      }
+      if (lane == 0) s_zl[tgt ? 0 : 1][i] = z;
+    }
+  }
   __syncthreads();
 
   for (int start = 0;;) {
@@ -87,15 +117,15 @@ __global__ void __launch_bounds__(kThreads) chain_finish_kernel(const ChainJob j
                 const RowStats sq = ds[i];
                 e = row_event(sq);
                 if (e == EV_ACCEPT) {
-                  const double zp = i == zpos ? s_z[0] : sp.zd;
-                  const double zq = i == zpos ? s_z[1] : sq.zd;
+                  const double zp = i == zpos ? s_z[0] : (i < npos ? s_zl[0][i] : sp.zd);
+                  const double zq = i == zpos ? s_z[1] : (i < npos ? s_zl[1][i] : sq.zd);
                   if (zp < 0.0 || zq < 0.0) {
                     e = EV_NEEDZ;
                   } else {
                     const float lp = Elem<T>::load(trow0, size_t(i) * V + xi);
                     const float lq = Elem<T>::load(drow0, size_t(i) * V + xi);
-                    const double p = prob_d<T>(sp, zp, Tt, lp, xi);
-                    const double q = prob_d<T>(sq, zq, Tt, lq, xi);
+                    const double p = kept_weight_d<T>(sp, iT, lp, xi) / zp;
+                    const double q = kept_weight_d<T>(sq, iT, lq, xi) / zq;
                     const double r = q > 0.0 ? p / q : (p > 0.0 ? double(INFINITY) : 0.0);
                     e = (double(u[i]) < fmin(1.0, r)) ? EV_ACCEPT : EV_STOP;
                   }
@@ -121,8 +151,12 @@ __global__ void __launch_bounds__(kThreads) chain_finish_kernel(const ChainJob j
     // the first position still to test lacks a normaliser: the block sums it, then the
     // scan resumes there (the positions before it are accepted)
     const int i = s_a;
-    const double zp = row_zd<T>(ts[i], trow0 + size_t(i) * V, V, Tt, sm.scr);
-    const double zq = row_zd<T>(ds[i], drow0 + size_t(i) * V, V, Tt, sm.scr);
+    const size_t tr = size_t(b) * (K + 1) + i, dr = size_t(j.B) * (K + 1) + size_t(b) * K + i;
+    const int ntk = j.kept_n ? j.kept_n[tr] : 0, ndk = j.kept_n ? j.kept_n[dr] : 0;
+    const double zp = row_zd<T>(ts[i], trow0 + size_t(i) * V, V, iT, sm.scr,
+                                j.kept_ids + tr * kKeptCap, ntk);
+    const double zq = row_zd<T>(ds[i], drow0 + size_t(i) * V, V, iT, sm.scr,
+                                j.kept_ids + dr * kKeptCap, ndk);
     if (threadIdx.x == 0) {
       s_z[0] = zp;
       s_z[1] = zq;
@@ -149,19 +183,20 @@ __global__ void __launch_bounds__(kThreads) chain_finish_kernel(const ChainJob j
     const size_t prow_idx = size_t(b) * (K + 1) + a;
     const int nk = j.kept_n ? j.kept_n[prow_idx] : 0;
     // the normalisers the test at a used (the bonus draw needs none: it scales by its total)
-    const double zp = a < K ? (a == s_zpos ? s_z[0] : sp.zd) : 1.0;
+    const double izp =
+        a < K ? 1.0 / (a == s_zpos ? s_z[0] : (a < npos ? s_zl[0][a] : sp.zd)) : 1.0;
     tok = -1;
     if (nk > 0 && nk <= kSparseCap) {
       const int32_t* ids = j.kept_ids + prow_idx * kKeptCap;
       if (a < K) {
         const RowStats sq = ds[a];
-        const double zq = a == s_zpos ? s_z[1] : sq.zd;
+        const double izq = 1.0 / (a == s_zpos ? s_z[1] : (a < npos ? s_zl[1][a] : sq.zd));
         const T* qrow = drow0 + size_t(a) * V;
         tok = sparse_draw(
             ids, nk,
             [&](int v) {
-              const double d = prob_d<T>(sp, zp, Tt, Elem<T>::load(prow, size_t(v)), v) -
-                               prob_d<T>(sq, zq, Tt, Elem<T>::load(qrow, size_t(v)), v);
+              const double d = prob_d<T>(sp, izp, iT, Elem<T>::load(prow, size_t(v)), v) -
+                               prob_d<T>(sq, izq, iT, Elem<T>::load(qrow, size_t(v)), v);
               return fx_from(fmax(d, 0.0));
             },
             w, sm);
@@ -170,13 +205,13 @@ __global__ void __launch_bounds__(kThreads) chain_finish_kernel(const ChainJob j
         tok = sparse_draw(
             ids, nk,
             [&](int v) {
-              return fx_from(kept_weight_d<T>(sp, Tt, Elem<T>::load(prow, size_t(v)), v));
+              return fx_from(kept_weight_d<T>(sp, iT, Elem<T>::load(prow, size_t(v)), v));
             },
             w, sm);
     } else {
       if (a < K) {
         const RowStats sq = ds[a];
-        const double zq = a == s_zpos ? s_z[1] : sq.zd;
+        const double izq = 1.0 / (a == s_zpos ? s_z[1] : (a < npos ? s_zl[1][a] : sq.zd));
         const T* qrow = drow0 + size_t(a) * V;
         const bool qal = (reinterpret_cast<uintptr_t>(qrow) & 15u) == 0;
         tok = inverse_cdf_draw(
@@ -187,8 +222,8 @@ __global__ void __launch_bounds__(kThreads) chain_finish_kernel(const ChainJob j
 #pragma unroll
               for (int k = 0; k < 8; ++k) {
                 const int v = v0 + k;
-                const double d = (v < V) ? prob_d<T>(sp, zp, Tt, lp[k], v) -
-                                               prob_d<T>(sq, zq, Tt, lq[k], v)
+                const double d = (v < V) ? prob_d<T>(sp, izp, iT, lp[k], v) -
+                                               prob_d<T>(sq, izq, iT, lq[k], v)
                                          : 0.0;
                 r[k] = fx_from(fmax(d, 0.0));
               }
@@ -203,7 +238,7 @@ __global__ void __launch_bounds__(kThreads) chain_finish_kernel(const ChainJob j
 #pragma unroll
               for (int k = 0; k < 8; ++k) {
                 const int v = v0 + k;
-                r[k] = (v < V) ? fx_from(kept_weight_d<T>(sp, Tt, lp[k], v)) : fx_zero();
+                r[k] = (v < V) ? fx_from(kept_weight_d<T>(sp, iT, lp[k], v)) : fx_zero();
               }
             },
             V, w, sm);

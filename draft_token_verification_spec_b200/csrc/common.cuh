@@ -259,6 +259,10 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t by
                : "memory");
 }
 
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
 // 1-D bulk copy global -> this CTA's shared memory, completing on `bar`.
 // dst and src 16-byte aligned, bytes a multiple of 16. Streamed data: evict-first in L2.
 __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes,

@@ -198,37 +198,95 @@ __device__ __forceinline__ float prob(const RowStats& s, float l, int v) {
 }
 
 // ------------------------------------------------------------------ double-precision view
-// Unnormalised weight exp((l - m) / T) of a kept entry, in double (l - m is exact).
-__device__ __forceinline__ double weight_d(float l, float m, double T) {
-  return exp((double(l) - double(m)) / T);
+// 2^(j/64), j = 0..63, each the double nearest the exact value (computed to 60 digits).
+static __device__ const double kExp2J[64] = {
+    0x1.0000000000000p+0, 0x1.02c9a3e778061p+0, 0x1.059b0d3158574p+0, 0x1.0874518759bc8p+0,
+    0x1.0b5586cf9890fp+0, 0x1.0e3ec32d3d1a2p+0, 0x1.11301d0125b51p+0, 0x1.1429aaea92de0p+0,
+    0x1.172b83c7d517bp+0, 0x1.1a35beb6fcb75p+0, 0x1.1d4873168b9aap+0, 0x1.2063b88628cd6p+0,
+    0x1.2387a6e756238p+0, 0x1.26b4565e27cddp+0, 0x1.29e9df51fdee1p+0, 0x1.2d285a6e4030bp+0,
+    0x1.306fe0a31b715p+0, 0x1.33c08b26416ffp+0, 0x1.371a7373aa9cbp+0, 0x1.3a7db34e59ff7p+0,
+    0x1.3dea64c123422p+0, 0x1.4160a21f72e2ap+0, 0x1.44e086061892dp+0, 0x1.486a2b5c13cd0p+0,
+    0x1.4bfdad5362a27p+0, 0x1.4f9b2769d2ca7p+0, 0x1.5342b569d4f82p+0, 0x1.56f4736b527dap+0,
+    0x1.5ab07dd485429p+0, 0x1.5e76f15ad2148p+0, 0x1.6247eb03a5585p+0, 0x1.6623882552225p+0,
+    0x1.6a09e667f3bcdp+0, 0x1.6dfb23c651a2fp+0, 0x1.71f75e8ec5f74p+0, 0x1.75feb564267c9p+0,
+    0x1.7a11473eb0187p+0, 0x1.7e2f336cf4e62p+0, 0x1.82589994cce13p+0, 0x1.868d99b4492edp+0,
+    0x1.8ace5422aa0dbp+0, 0x1.8f1ae99157736p+0, 0x1.93737b0cdc5e5p+0, 0x1.97d829fde4e50p+0,
+    0x1.9c49182a3f090p+0, 0x1.a0c667b5de565p+0, 0x1.a5503b23e255dp+0, 0x1.a9e6b5579fdbfp+0,
+    0x1.ae89f995ad3adp+0, 0x1.b33a2b84f15fbp+0, 0x1.b7f76f2fb5e47p+0, 0x1.bcc1e904bc1d2p+0,
+    0x1.c199bdd85529cp+0, 0x1.c67f12e57d14bp+0, 0x1.cb720dcef9069p+0, 0x1.d072d4a07897cp+0,
+    0x1.d5818dcfba487p+0, 0x1.da9e603db3285p+0, 0x1.dfc97337b9b5fp+0, 0x1.e502ee78b3ff6p+0,
+    0x1.ea4afa2a490dap+0, 0x1.efa1bee615a27p+0, 0x1.f50765b6e4540p+0, 0x1.fa7c1819e90d8p+0,
+};
+
+// e^x for x <= 0 in double, by Tang's table-driven method (P. T. P. Tang, "Table-driven
+// implementation of the exponential function in IEEE floating-point arithmetic", ACM TOMS
+// 15(2), 1989): x = (64 k + j) ln2 / 64 + r with |r| <= ln2 / 128 (ln2 / 64 split into a
+// 32-bit head and a tail, so n * head is exact), e^x = 2^k 2^(j/64) e^r, and e^r by its
+// Taylor series to r^5 (the remainder is below 4e-17 of it). Relative error within a few
+// units in the last place; x below -745 (and -inf) gives 0.
+__device__ __forceinline__ double exp_neg(double x) {
+  if (!(x > -745.0)) return 0.0;
+  const double n = rint(x * 92.33248261689366);  // 64 / ln2
+  double r = fma(-n, 0x1.62e42fee00000p-7, x);
+  r = fma(-n, 0x1.a39ef35793c76p-39, r);
+  const int ni = int(n);
+  double p = fma(r, 1.0 / 120.0, 1.0 / 24.0);
+  p = fma(p, r, 1.0 / 6.0);
+  p = fma(p, r, 0.5);
+  p = fma(p, r, 1.0);
+  p = fma(p, r, 1.0);
+  const double t = __ldg(&kExp2J[ni & 63]) * p;
+  const int k = ni >> 6;  // floor(n / 64)
+  if (k >= -1022) return t * __longlong_as_double((long long)(k + 1023) << 52);
+  return ldexp(t, k);
+}
+
+// Unnormalised weight exp((l - m) / T) of a kept entry, in double (l - m is exact); iT = 1 / T.
+__device__ __forceinline__ double weight_d(float l, float m, double iT) {
+  return exp_neg((double(l) - double(m)) * iT);
 }
 
 // Weight of entry v of the row described by s (0 outside the kept set).
 template <typename T>
-__device__ __forceinline__ double kept_weight_d(const RowStats& s, double Tt, float l, int v) {
-  return kept(Elem<T>::key(l), v, s.thr_key, s.cutoff) ? weight_d(l, s.m, Tt) : 0.0;
+__device__ __forceinline__ double kept_weight_d(const RowStats& s, double iT, float l, int v) {
+  return kept(Elem<T>::key(l), v, s.thr_key, s.cutoff) ? weight_d(l, s.m, iT) : 0.0;
 }
 
-// Probability of entry v in double: kept weight / zd.
+// Probability of entry v in double: kept weight times izd = 1 / zd.
 template <typename T>
-__device__ __forceinline__ double prob_d(const RowStats& s, double zd, double Tt, float l, int v) {
-  return kept_weight_d<T>(s, Tt, l, v) / zd;
+__device__ __forceinline__ double prob_d(const RowStats& s, double izd, double iT, float l, int v) {
+  return kept_weight_d<T>(s, iT, l, v) * izd;
 }
 
 // The double normaliser of one row (every thread of the block calls it, gets the sum):
-// s.zd when the row statistics hold it, else the sum over the kept set, by a pass over the
-// row with exact Fx128 accumulation.
+// s.zd when the row statistics hold it; else the sum over the kept set with exact Fx128
+// accumulation, over the row's listed kept ids (nk > 0 of them at ids) or by a pass over the
+// row.
 template <typename T>
-__device__ double row_zd(const RowStats& s, const T* row, int V, double Tt, Fx128* scr) {
+__device__ double row_zd(const RowStats& s, const T* row, int V, double iT, Fx128* scr,
+                         const int32_t* ids = nullptr, int nk = 0) {
   if (s.zd >= 0.0) return s.zd;
+  if (ids && nk > 0) {
+    Fx128 acc = fx_zero();
+    for (int i = threadIdx.x; i < nk; i += kThreads) {
+      const int v = ids[i];
+      acc = fx_add(acc, fx_from(kept_weight_d<T>(s, iT, Elem<T>::load(row, size_t(v)), v)));
+    }
+    return fx_to_double(block_sum_fx(acc, scr));
+  }
   const bool al = (reinterpret_cast<uintptr_t>(row) & 15u) == 0;
   Fx128 acc = fx_zero();
-  for (int v0 = int(threadIdx.x) * 8; v0 < V; v0 += kThreads * 8) {
-    float x[8];
+  // two groups of 8 per iteration, both loaded before either is used
+  for (int v0 = int(threadIdx.x) * 8; v0 < V; v0 += 2 * kThreads * 8) {
+    float x[8], y[8];
+    const int v1 = v0 + kThreads * 8;
     load8<T>(row, v0, V, al, x);
+    load8<T>(row, v1, V, al, y);
 #pragma unroll
-    for (int k = 0; k < 8; ++k)
-      if (v0 + k < V) acc = fx_add(acc, fx_from(kept_weight_d<T>(s, Tt, x[k], v0 + k)));
+    for (int k = 0; k < 8; ++k) {
+      if (v0 + k < V) acc = fx_add(acc, fx_from(kept_weight_d<T>(s, iT, x[k], v0 + k)));
+      if (v1 + k < V) acc = fx_add(acc, fx_from(kept_weight_d<T>(s, iT, y[k], v1 + k)));
+    }
   }
   return fx_to_double(block_sum_fx(acc, scr));
 }

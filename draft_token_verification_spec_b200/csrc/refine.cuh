@@ -63,7 +63,7 @@ __global__ void __launch_bounds__(kThreads) topp_refine_kernel(const RefineJob j
   const RowJob& rj = j.r;
   const int V = rj.V;
   const long long nlist = *j.count;
-  const double Tt = double(rj.temp);
+  const double iT = 1.0 / double(rj.temp);
   for (long long li = blockIdx.x; li < nlist; li += gridDim.x) {
     const long long row = j.rows[li];
     const RowStats rs = rj.stats[row];
@@ -89,7 +89,7 @@ __global__ void __launch_bounds__(kThreads) topp_refine_kernel(const RefineJob j
       for (int k = 0; k < 8; ++k) {
         const int v = v0 + k;
         if (v >= V || !(x[k] > -INFINITY)) continue;  // past the row, or weight 0
-        const Fx128 fe = fx_from(weight_d(x[k], m, Tt));
+        const Fx128 fe = fx_from(weight_d(x[k], m, iT));
         zall = fx_add(zall, fe);
         const int b = bin_of(x[k], c, mc);
         const unsigned long long e = make_comp(Elem<T>::key(x[k]), v);
@@ -124,13 +124,13 @@ __global__ void __launch_bounds__(kThreads) topp_refine_kernel(const RefineJob j
     const int lo = int(threadIdx.x) * per;
     Fx128 own = fx_zero();
     for (int i = lo; i < lo + per && i < n; ++i)
-      own = fx_add(own, fx_from(weight_d(key_value<T>(comp_key(win[i])), m, Tt)));
+      own = fx_add(own, fx_from(weight_d(key_value<T>(comp_key(win[i])), m, iT)));
     Fx128 wtot;
     const Fx128 ex = block_exclusive_scan_fx(own, scr, &wtot);
     const double target = double(rj.top_p) * fx_to_double(zall);
     Fx128 cum = fx_add(above, ex);
     for (int i = lo; i < lo + per && i < n; ++i) {
-      cum = fx_add(cum, fx_from(weight_d(key_value<T>(comp_key(win[i])), m, Tt)));
+      cum = fx_add(cum, fx_from(weight_d(key_value<T>(comp_key(win[i])), m, iT)));
       if (fx_to_double(cum) >= target) {
         atomicMin(&s_best, i);
         break;
@@ -147,7 +147,7 @@ __global__ void __launch_bounds__(kThreads) topp_refine_kernel(const RefineJob j
       if (a >= target) {
         // the crossing lies above the window: the lightest entry above it, if that alone
         // holds the excess
-        const double wl = weight_d(key_value<T>(comp_key(s_lo_above)), m, Tt);
+        const double wl = weight_d(key_value<T>(comp_key(s_lo_above)), m, iT);
         if (s_lo_above != ~0ull && a - wl < target) {
           e = s_lo_above;
           zkept = a;
@@ -158,7 +158,7 @@ __global__ void __launch_bounds__(kThreads) topp_refine_kernel(const RefineJob j
       } else if (s_hi_below != 0ull) {
         // below the window: the heaviest entry after it, if it reaches the target
         const double through = fx_to_double(fx_add(above, wtot));
-        const double wh = weight_d(key_value<T>(comp_key(s_hi_below)), m, Tt);
+        const double wh = weight_d(key_value<T>(comp_key(s_hi_below)), m, iT);
         if (through + wh >= target) {
           e = s_hi_below;
           zkept = through + wh;

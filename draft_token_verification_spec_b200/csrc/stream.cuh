@@ -285,6 +285,24 @@ __device__ __forceinline__ Fx128 cscan_fx(Fx128 v, Fx128* scr, Fx128* total) {
   return fx_add(before, ex);
 }
 
+// The double-precision work at a row's end, kept out of line so that its registers do not
+// weigh on the streaming loop (the call is taken once per row): one entry's weight
+// exp((x - m) / T) as Fx128, and a thread's share of the kept candidates' weights.
+template <typename T>
+__device__ __noinline__ Fx128 weight_fx(uint32_t key, float m, double iT) {
+  return fx_from(weight_d(key_value<T>(key), m, iT));
+}
+template <typename T>
+__device__ __noinline__ Fx128 kept_weights_fx(const uint64_t* cand, int n, uint64_t cstar, float m,
+                                              double iT) {
+  Fx128 acc = fx_zero();
+  for (int i = threadIdx.x; i < n; i += kThreads) {
+    const uint64_t e = cand[i];
+    if (e >= cstar) acc = fx_add(acc, fx_from(weight_d(key_value<T>(uint32_t(e >> 32)), m, iT)));
+  }
+  return acc;
+}
+
 // Counts into hist[bin] with one shared atomic per distinct bin per warp; every lane of
 // the warp calls it.
 __device__ __forceinline__ void hist_add(uint32_t* hist, int bin, bool valid) {
@@ -294,9 +312,6 @@ __device__ __forceinline__ void hist_add(uint32_t* hist, int bin, bool valid) {
   if ((threadIdx.x & 31) == __ffs(peers) - 1) atomicAdd(&hist[bin], uint32_t(__popc(peers)));
 }
 
-__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
-  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
-}
 
 // The j-th largest (1 <= j <= 32 N) of the warp's 32 N keys (N per lane), by a radix walk
 // from the top bit with warp-wide counts; every lane calls it.
@@ -563,7 +578,7 @@ struct CandSet {
   // the one where the mass accumulated from the top first reaches top_p of their total ->
   // aux->sel_comp, with the weights exp((l - m) / T) in double summed exactly. The caller has
   // synchronised the list, and read aux->sel_comp if it needs it, before the call.
-  __device__ bool rank_topp(int n, int k, float top_p, float m, double Tt) {
+  __device__ bool rank_topp(int n, int k, float top_p, float m, double iT) {
     for (int i = threadIdx.x; i < n; i += kThreads) {
       const uint64_t e = cand[i];
       int above = 0;
@@ -574,7 +589,7 @@ struct CandSet {
     csync();
     const bool mine = int(threadIdx.x) < k;
     const uint64_t e = mine ? ranked[threadIdx.x] : 0ull;
-    const Fx128 w = mine ? fx_from(weight_d(key_value<T>(comp_key(e)), m, Tt)) : fx_zero();
+    const Fx128 w = mine ? weight_fx<T>(comp_key(e), m, iT) : fx_zero();
     Fx128 z;
     const Fx128 ex = cscan_fx(w, scr_fx(*aux), &z);
     const double target = double(top_p) * fx_to_double(z);
@@ -775,7 +790,7 @@ __global__ void __launch_bounds__(kStreamThreads, (kMode == SM_TOPP ? 2 : 3))
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const bool want_ent = (rj.flags & RS_ENTROPY) != 0;
   const float c = rj.c;
-  const double Tt = double(rj.temp);
+  const double iT = rj.temp > 0.0f ? 1.0 / double(rj.temp) : 0.0;
   CandSet<T> cs;
   cs.cand = reinterpret_cast<uint64_t*>(smem + size_t(kRing) * kRingBufBytes);
   if (kMode == SM_TOPK) {
@@ -1044,7 +1059,7 @@ __global__ void __launch_bounds__(kStreamThreads, (kMode == SM_TOPP ? 2 : 3))
             ok = ok && n >= rj.top_k;
             if (ok) {  // every list is short (kCapTopK <= kRankMax): rank directly
               if (rj.top_p < 1.0f) {  // the top-p crossing within the top k
-                ok = cs.rank_topp(n, rj.top_k, rj.top_p, m, Tt);
+                ok = cs.rank_topp(n, rj.top_k, rj.top_p, m, iT);
               } else {
                 ok = cs.rank_select(n, 0, rj.top_k);
               }
@@ -1078,13 +1093,16 @@ __global__ void __launch_bounds__(kStreamThreads, (kMode == SM_TOPP ? 2 : 3))
           if (!ok) {
             status = ROW_FALLBACK;
           } else {
-            // normaliser, entropy term and kept-id list over the kept candidates
-            const bool list = kMode == SM_TOPK && rj.top_p >= 1.0f && rj.kept_ids != nullptr;
+            // normaliser, entropy term and kept-id list over the kept candidates. Top-k rows
+            // list their kept ids (with top-p too: the nucleus within the top k), and the
+            // consumer sums the double normaliser over the list if it needs it; top-p rows
+            // are not listed and get it here.
+            const bool list = kMode == SM_TOPK && rj.kept_ids != nullptr;
             if (threadIdx.x == 0) aux.mcount = 0;
             csync();
             unsigned long long z = 0;
             long long s1 = 0;
-            Fx128 zdx = fx_zero();
+            const Fx128 zdx = list ? fx_zero() : kept_weights_fx<T>(cs.cand, n, cstar, m, iT);
             for (int i = threadIdx.x; i < n; i += kThreads) {
               const uint64_t e = cs.cand[i];
               if (e < cstar) continue;
@@ -1092,14 +1110,13 @@ __global__ void __launch_bounds__(kStreamThreads, (kMode == SM_TOPP ? 2 : 3))
               const float zx = wexp(xv, c, mc);
               const float ex = ex2(zx);
               z += to_fx(ex);
-              zdx = fx_add(zdx, fx_from(weight_d(xv, m, Tt)));
               if (want_ent) s1 += __float2ll_rn(ent_term(ex, zx) * kS1Fx);
               if (list) {
                 const int slot = atomicAdd(&aux.mcount, 1);
                 if (slot < kKeptCap) rj.kept_ids[size_t(row) * kKeptCap + slot] = comp_id(e);
               }
             }
-            zd = fx_to_double(creduce_fx(zdx, scr_fx(aux)));
+            if (!list) zd = fx_to_double(creduce_fx(zdx, scr_fx(aux)));
             zfx = creduce<unsigned long long>(z, aux.scr_u64, OpSum());
             S1 = double(creduce<long long>(s1, aux.scr_s64, OpSum())) / double(kS1Fx);
             thr_key = comp_key(cstar);
@@ -1110,7 +1127,7 @@ __global__ void __launch_bounds__(kStreamThreads, (kMode == SM_TOPP ? 2 : 3))
       }
       if (status == ROW_FALLBACK && threadIdx.x == 0)
         job.fb_rows[atomicAdd(job.fb_count, 1)] = int32_t(row);
-      if (rj.kept_n && threadIdx.x == 0) rj.kept_n[row] = listed ? rj.top_k : 0;
+      if (rj.kept_n && threadIdx.x == 0) rj.kept_n[row] = listed ? min(aux.mcount, kKeptCap) : 0;
       const double Z = double(zfx) * kFxInv;
       const double ent = (status == ROW_OK && kMode != SM_GREEDY && want_ent)
                              ? log(Z) - 0.6931471805599453 * S1 / Z

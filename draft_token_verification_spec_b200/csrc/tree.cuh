@@ -135,7 +135,7 @@ __global__ void __launch_bounds__(kThreads) tree_finish_kernel(const TreeJob j) 
         for (int k = 0; k < 8; ++k) {
           if (v0 + k >= V || !(x[k] > -INFINITY)) continue;
           const double d = double(s.m) - double(x[k]);  // >= 0, exact
-          const double e = exp(-d);
+          const double e = exp_neg(-d);
           z = fx_add(z, fx_from(e));
           h = fx_add(h, fx_from(e * d));
         }

@@ -45,7 +45,7 @@ __global__ void __launch_bounds__(kThreads) tree_sample_kernel(const TreeSampleJ
   int32_t* kstart = reinterpret_cast<int32_t*>(zs + N);  // [N+1] children of n: kids[kstart[n]..)
   int32_t* kids = kstart + N + 1;                      // [N]
   int32_t* path = kids + N;                            // [N] nodes on the accepted path
-  const double Tt = double(j.temp);
+  const double iT = j.temp > 0.0f ? 1.0 / double(j.temp) : 0.0;
   __shared__ DrawSmem sm;
   __shared__ int s_bad;
   const int32_t* par = j.parent;
@@ -106,8 +106,12 @@ __global__ void __launch_bounds__(kThreads) tree_sample_kernel(const TreeSampleJ
         }
       }
       // the double normalisers of p_n and (with children) q_n; every thread gets them
-      const double zp = row_zd<T>(sp, prow, V, Tt, sm.scr);
-      const double zq = k1 > k0 ? row_zd<T>(sq, qrow, V, Tt, sm.scr) : 1.0;
+      const size_t qrow_idx = size_t(j.B) * N + size_t(b) * N + cur;
+      const int nqk = (j.kept_n && k1 > k0) ? j.kept_n[qrow_idx] : 0;
+      const double izp = 1.0 / row_zd<T>(sp, prow, V, iT, sm.scr, ids, sparse ? nk : 0);
+      const double izq = k1 > k0 ? 1.0 / row_zd<T>(sq, qrow, V, iT, sm.scr,
+                                                    j.kept_ids + qrow_idx * kKeptCap, nqk)
+                                 : 1.0;
       int nrej = 0;
       // the current residual at v: the recursion over the rejections so far
       auto resid = [&](double pv, double qv) {
@@ -123,8 +127,8 @@ __global__ void __launch_bounds__(kThreads) tree_sample_kernel(const TreeSampleJ
           err = EV_ERROR;
           break;
         }
-        const double px = prob_d<T>(sp, zp, Tt, Elem<T>::load(prow, size_t(x)), x);
-        const double qx = prob_d<T>(sq, zq, Tt, Elem<T>::load(qrow, size_t(x)), x);
+        const double px = prob_d<T>(sp, izp, iT, Elem<T>::load(prow, size_t(x)), x);
+        const double qx = prob_d<T>(sq, izq, iT, Elem<T>::load(qrow, size_t(x)), x);
         const double rx = resid(px, qx);
         const double ratio = qx > 0.0 ? rx / qx : (rx > 0.0 ? double(INFINITY) : 0.0);
         if (double(u[c]) < fmin(1.0, ratio)) {
@@ -136,14 +140,14 @@ __global__ void __launch_bounds__(kThreads) tree_sample_kernel(const TreeSampleJ
         if (sparse) {
           for (int t = threadIdx.x; t < nk; t += kThreads) {
             const int v = ids[t];
-            const double pv = prob_d<T>(sp, zp, Tt, Elem<T>::load(prow, size_t(v)), v);
-            const double qv = prob_d<T>(sq, zq, Tt, Elem<T>::load(qrow, size_t(v)), v);
+            const double pv = prob_d<T>(sp, izp, iT, Elem<T>::load(prow, size_t(v)), v);
+            const double qv = prob_d<T>(sq, izq, iT, Elem<T>::load(qrow, size_t(v)), v);
             zsum = fx_add(zsum, fx_from(fmax(resid(pv, qv) - qv, 0.0)));
           }
         } else {
           for (int v = threadIdx.x; v < V; v += kThreads) {
-            const double pv = prob_d<T>(sp, zp, Tt, Elem<T>::load(prow, size_t(v)), v);
-            const double qv = prob_d<T>(sq, zq, Tt, Elem<T>::load(qrow, size_t(v)), v);
+            const double pv = prob_d<T>(sp, izp, iT, Elem<T>::load(prow, size_t(v)), v);
+            const double qv = prob_d<T>(sq, izq, iT, Elem<T>::load(qrow, size_t(v)), v);
             zsum = fx_add(zsum, fx_from(fmax(resid(pv, qv) - qv, 0.0)));
           }
         }
@@ -158,9 +162,9 @@ __global__ void __launch_bounds__(kThreads) tree_sample_kernel(const TreeSampleJ
           emitted = sparse_draw(
               ids, nk,
               [&](int v) {
-                const double pv = prob_d<T>(sp, zp, Tt, Elem<T>::load(prow, size_t(v)), v);
+                const double pv = prob_d<T>(sp, izp, iT, Elem<T>::load(prow, size_t(v)), v);
                 const double qv =
-                    k1 > k0 ? prob_d<T>(sq, zq, Tt, Elem<T>::load(qrow, size_t(v)), v) : 0.0;
+                    k1 > k0 ? prob_d<T>(sq, izq, iT, Elem<T>::load(qrow, size_t(v)), v) : 0.0;
                 return fx_from(resid(pv, qv));
               },
               w, sm);
@@ -177,8 +181,8 @@ __global__ void __launch_bounds__(kThreads) tree_sample_kernel(const TreeSampleJ
                   const int v = v0 + k;
                   double mv = 0.0;
                   if (v < V) {
-                    const double pv = prob_d<T>(sp, zp, Tt, lp[k], v);
-                    const double qv = k1 > k0 ? prob_d<T>(sq, zq, Tt, lq[k], v) : 0.0;
+                    const double pv = prob_d<T>(sp, izp, iT, lp[k], v);
+                    const double qv = k1 > k0 ? prob_d<T>(sq, izq, iT, lq[k], v) : 0.0;
                     mv = resid(pv, qv);
                   }
                   r[k] = fx_from(mv);
