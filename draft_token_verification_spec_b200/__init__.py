@@ -52,6 +52,8 @@ def _declare(lib):
         "spec_residual_sample": ([P, P, I, I, P, P, P], I),
         "spec_get_device_status": ([P, P, P], I),
         "spec_linear_state_factors": ([P, P, P, P, I, I, I, I, I, P, P, P, P], I),
+        "spec_lmhead_workspace_size": ([I, I, I, I, I], Z),
+        "spec_verify_chain_lmhead": ([P, P, P, P, I, I, I, I, P, P, F, I, P, P, P, P, Z, P], I),
         "spec_commit_linear_state": ([P, I, I, I, I, I, P, P, P, P, P, P], I),
         "spec_set_row_kernel_events": ([P, P], None),
         "spec_kernels_per_call": ([ctypes.c_char_p], I),
@@ -310,6 +312,49 @@ def spec_residual_sample(p, q, uniforms, tokens=None, stream=None):
         _check("spec_residual_sample", lib().spec_residual_sample(
             _ptr(pp), _ptr(qq), rows, V, _ptr(u), _ptr(tokens), _stream(stream, pp.device)))
     return tokens
+
+
+def spec_lmhead_workspace_size(B: int, K: int, V: int, d: int, top_k: int) -> int:
+    return int(lib().spec_lmhead_workspace_size(int(B), int(K), int(V), int(d), int(top_k)))
+
+
+def spec_verify_chain_lmhead(target_hidden, draft_hidden, target_weight, draft_weight,
+                             draft_tokens, uniforms, temp, top_k=0, logits_out=None,
+                             accepted_len=None, out_tokens=None, workspace=None, stream=None):
+    """Chain verification from hidden states: target_hidden bf16 [B,K+1,d], draft_hidden
+    [B,K,d] (None when temp == 0), target_weight and draft_weight bf16 [V,d] (the LM heads).
+    temp == 0 (greedy) or 1 <= top_k <= 64. logits_out: None, or float32 [B*(2K+1), V] to
+    receive the logits as well (target rows, then draft rows). Returns (accepted_len [B],
+    out_tokens [B,K+1])."""
+    ht = _dev(target_hidden, "target_hidden", torch.bfloat16)
+    B, K1, d = ht.shape
+    K = K1 - 1
+    wt = _dev(target_weight, "target_weight", torch.bfloat16)
+    V = wt.shape[0]
+    greedy = float(temp) == 0.0
+    hd = None if draft_hidden is None else _dev(draft_hidden, "draft_hidden", torch.bfloat16)
+    wd = None if draft_weight is None else _dev(draft_weight, "draft_weight", torch.bfloat16)
+    if tuple(wt.shape) != (V, d) or (hd is not None and tuple(hd.shape) != (B, K, d)) or \
+            (wd is not None and tuple(wd.shape) != (V, d)):
+        raise ValueError("hidden [B,K+1,d] / [B,K,d], weights [V,d]")
+    x = _dev(draft_tokens, "draft_tokens", torch.int32)
+    u = _dev(uniforms, "uniforms", torch.float32)
+    if accepted_len is None:
+        accepted_len = torch.empty(B, dtype=torch.int32, device=ht.device)
+    if out_tokens is None:
+        out_tokens = torch.empty((B, K + 1), dtype=torch.int32, device=ht.device)
+    if logits_out is not None:
+        _dev(logits_out, "logits_out", torch.float32)
+    if workspace is None:
+        workspace = torch.empty(spec_lmhead_workspace_size(B, K, V, d, 0 if greedy else top_k),
+                                dtype=torch.uint8, device=ht.device)
+    with _on(ht.device):
+        _check("spec_verify_chain_lmhead", lib().spec_verify_chain_lmhead(
+            _ptr(ht), _ptr(hd), _ptr(wt), _ptr(wd), B, K, V, d, _ptr(x), _ptr(u), float(temp),
+            int(top_k), _ptr(accepted_len), _ptr(out_tokens), _ptr(logits_out),
+            _ptr(workspace), workspace.numel() * workspace.element_size(),
+            _stream(stream, ht.device)))
+    return accepted_len, out_tokens
 
 
 def spec_linear_state_factors(alpha, beta, keys, values, w=None, u=None, gamma=None,

@@ -188,6 +188,32 @@ spec_status spec_logits_to_probs(const void* logits, spec_dtype dtype, int rows,
 spec_status spec_residual_sample(const float* p, const float* q, int rows, int V,
                                  const float* uniforms, int32_t* tokens, void* stream);
 
+/* Chain verification straight from the scoring forward's hidden states — [SD]
+ * "Speculative Sampling" (the K drafts are scored in one forward whose cost lies in its
+ * linear layers) and the chain rule of spec_verify_chain. The LM-head product
+ * logits = hidden . weight^T runs on the tensor cores (bf16 x bf16, fp32 accumulation) and
+ * its epilogue keeps only what the rule needs of each logit row, the top-k entries (the
+ * argmax at temperature 0), so no logit row is written to memory.
+ *   target_hidden [B][K+1][d], draft_hidden [B][K][d] (NULL iff temp == 0): bf16, row-major.
+ *   target_weight, draft_weight [V][d] bf16 (row v = token v's output embedding; the draft
+ *                  weight may be NULL iff temp == 0).
+ *   draft_tokens, uniforms, accepted_len, out_tokens: as spec_verify_chain.
+ *   temp == 0: greedy (draft rows unused); temp > 0 needs 1 <= top_k <= 64, top_k < V
+ *   (top-k sampling; other transforms return SPEC_ERR_UNSUPPORTED). The decisions are those of
+ *   spec_verify_chain applied to the fp32 logits this product computes.
+ *   logits_out: NULL, or float [B*(K+1) + B*K][V] (target rows, then draft rows) that also
+ *   receives those logits, for checking.
+ *   d a multiple of 64; hidden, weight and workspace 16-byte aligned; workspace at least
+ *   spec_lmhead_workspace_size(B, K, V, d, top_k) bytes (top_k = 0 for greedy). */
+size_t spec_lmhead_workspace_size(int B, int K, int V, int d, int top_k);
+spec_status spec_verify_chain_lmhead(const void* target_hidden, const void* draft_hidden,
+                                     const void* target_weight, const void* draft_weight, int B,
+                                     int K, int V, int d, const int32_t* draft_tokens,
+                                     const float* uniforms, float temp, int top_k,
+                                     int32_t* accepted_len, int32_t* out_tokens,
+                                     float* logits_out, void* workspace, size_t workspace_bytes,
+                                     void* stream);
+
 /* Linear-attention state commit after verification — [SpecLA] gist.science summary of
  * "SpecLA: Efficient Speculative Decoding for Linear-Attention Models" (a linear-attention
  * target keeps one dense state per head; after the verdict the state is brought to the

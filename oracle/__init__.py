@@ -26,9 +26,10 @@ FLAG_CDF = 2
 FLAG_TOPP = 4
 FLAG_TREE = 8
 DIAG_Q_ZERO = 16
-PARITY_FLAGS = FLAG_RATIO | FLAG_CDF | FLAG_TOPP | FLAG_TREE
+FLAG_GAP = 32
+PARITY_FLAGS = FLAG_RATIO | FLAG_CDF | FLAG_TOPP | FLAG_TREE | FLAG_GAP
 
-# Widths of the precision windows behind the flags (ratio, cdf_rel, cdf_abs, topp, tree):
+# Widths of the precision windows behind the flags (ratio, cdf_rel, cdf_abs, topp, tree, gap):
 # a flag marks a decision that arithmetic of lower precision than the oracle's may take
 # the other way. They change only the flags, never a result.
 #   CRITERION: the widest the acceptance criterion allows: |u - r| < 1e-5, a CDF edge
@@ -36,8 +37,12 @@ PARITY_FLAGS = FLAG_RATIO | FLAG_CDF | FLAG_TOPP | FLAG_TREE
 #              tree threshold, this build's extensions of the same idea).
 #   FP64:      for a verifier that takes these decisions in double precision: double
 #              rounding over up to 2^20 terms moves a sum by at most ~1.2e-10 of it.
-CRITERION = (1e-5, 1e-6, 0.0, 1e-6, 1e-5)
-FP64 = (1e-9, 1e-9, 1e-10, 1e-10, 1e-9)
+#   FP32_LOGITS: for a verifier that computes the logits itself with fp32 accumulation
+#              (the LM-head product): a logit gap under 1e-3 behind an argmax or top-k
+#              decision, and ratios and CDF edges within 1e-4 (relative), are flagged.
+CRITERION = (1e-5, 1e-6, 0.0, 1e-6, 1e-5, 0.0)
+FP64 = (1e-9, 1e-9, 1e-10, 1e-10, 1e-9, 0.0)
+FP32_LOGITS = (1e-4, 1e-4, 0.0, 1e-4, 1e-5, 1e-3)
 
 
 def build(force: bool = False) -> str:
@@ -93,7 +98,9 @@ def _dtype_code(logits: np.ndarray) -> int:
         return 0
     if logits.dtype == np.uint16:
         return 1
-    raise TypeError("logits must be float32 or uint16 (bfloat16 bit patterns)")
+    if logits.dtype == np.float64:
+        return 2
+    raise TypeError("logits must be float32, float64 or uint16 (bfloat16 bit patterns)")
 
 
 def _threads(threads):
@@ -102,7 +109,7 @@ def _threads(threads):
 
 def _win(windows):
     w = np.ascontiguousarray(CRITERION if windows is None else windows, dtype=np.float64)
-    assert w.shape == (5,)
+    assert w.shape == (6,)
     return w
 
 

@@ -59,6 +59,8 @@ enum : int32_t {
                        // side changes the row's output
   FLAG_TREE = 8,       // |p - thr| / thr < tree window at a tested tree node
   DIAG_Q_ZERO = 16,    // a tested draft token had q(x) = 0 (not a parity flag)
+  FLAG_GAP = 32,       // a logit gap behind a decision (argmax, top-k boundary) within the
+                       // gap window: for logits that the verifier computes itself
 };
 
 // Widths of the precision windows behind the flags. A flag marks a decision that another
@@ -73,9 +75,10 @@ struct Windows {
   double cdf_abs = 0.0;
   double topp = 1e-6;
   double tree = 1e-5;
+  double gap = 0.0;  // logit-gap window (0: off; the logits are inputs, not computed)
 };
 
-// w = {ratio, cdf_rel, cdf_abs, topp, tree}, or NULL for the defaults.
+// w = {ratio, cdf_rel, cdf_abs, topp, tree, gap}, or NULL for the defaults.
 Windows windows_from(const double* w) {
   Windows x;
   if (w) {
@@ -84,6 +87,7 @@ Windows windows_from(const double* w) {
     x.cdf_abs = w[2];
     x.topp = w[3];
     x.tree = w[4];
+    x.gap = w[5];
   }
   return x;
 }
@@ -95,10 +99,13 @@ double bf16_bits_to_double(uint16_t h) {
   return double(f);
 }
 
-// dtype 0 = float32, 1 = bfloat16 (raw 16-bit patterns).
+// dtype 0 = float32, 1 = bfloat16 (raw 16-bit patterns), 2 = float64.
 void load_row(const void* base, int dtype, size_t row, int V, std::vector<double>& l) {
   l.resize(size_t(V));
-  if (dtype == 0) {
+  if (dtype == 2) {
+    const double* p = static_cast<const double*>(base) + row * size_t(V);
+    for (int v = 0; v < V; ++v) l[v] = p[v];
+  } else if (dtype == 0) {
     const float* p = static_cast<const float*>(base) + row * size_t(V);
     for (int v = 0; v < V; ++v) l[v] = double(p[v]);
   } else {
@@ -132,6 +139,10 @@ struct Dist {
   double margin_reach = kInf;
   double margin_prev = kInf;
   double topp_margin() const { return std::min(margin_reach, margin_prev); }
+  // Logit gap at the decision the transform takes on logit order: between the k-th and the
+  // (k+1)-th largest logits under top-k, between the largest and the next at T == 0.
+  // Infinite when neither applies.
+  double logit_gap = kInf;
 };
 
 // The sampling transform of [SD] "Speculative Sampling" (last bullet): the
@@ -147,7 +158,12 @@ Dist transform(const std::vector<double>& l, double T, int top_k, double top_p, 
   Dist d;
   d.p.assign(size_t(V), 0.0);
   if (T == 0.0) {
-    d.p[argmax_lowest(l)] = 1.0;
+    const int g = argmax_lowest(l);
+    d.p[g] = 1.0;
+    double second = -kInf;
+    for (int v = 0; v < V; ++v)
+      if (v != g && l[v] > second) second = l[v];
+    d.logit_gap = l[g] - second;
     return d;
   }
   std::vector<char> kept(static_cast<size_t>(V), 1);
@@ -160,6 +176,10 @@ Dist transform(const std::vector<double>& l, double T, int top_k, double top_p, 
     });
     std::fill(kept.begin(), kept.end(), 0);
     for (int j = 0; j < top_k; ++j) kept[order[j]] = 1;
+    double next = -kInf;  // the largest logit left out
+    for (int v = 0; v < V; ++v)
+      if (!kept[v] && l[v] > next) next = l[v];
+    d.logit_gap = l[order[top_k - 1]] - next;
   }
   double zmax = -kInf;
   for (int v = 0; v < V; ++v)
@@ -315,6 +335,7 @@ Outcome chain_eval(const ChainArgs& a, int b, const Override& ov) {
       load_row(a.target, a.dtype, size_t(b) * (K + 1) + i, V, lp);
       if (!row_valid(lp)) return o.error = true, o;
       const int g = argmax_lowest(lp);
+      if (a.win.gap > 0.0 && transform(lp, 0.0, 0, 1.0).logit_gap < a.win.gap) o.flag |= FLAG_GAP;
       if (i == K) {
         emitted = g;
         break;
@@ -332,6 +353,7 @@ Outcome chain_eval(const ChainArgs& a, int b, const Override& ov) {
       if (!row_valid(lp)) return o.error = true, o;
       const Dist P = transform(lp, a.T, a.top_k, a.top_p, alt_of(0, i));
       note(P, 0, i);
+      if (P.logit_gap < a.win.gap) o.flag |= FLAG_GAP;
       if (i == K) {  // every draft accepted: bonus token from p at position K+1
         const Draw d = inverse_cdf(P.p, u[K], a.win);
         emitted = d.token;
@@ -343,6 +365,7 @@ Outcome chain_eval(const ChainArgs& a, int b, const Override& ov) {
       if (!row_valid(lq)) return o.error = true, o;
       const Dist Q = transform(lq, a.T, a.top_k, a.top_p, alt_of(1, i));
       note(Q, 1, i);
+      if (Q.logit_gap < a.win.gap) o.flag |= FLAG_GAP;
       const double px = P.p[x[i]], qx = Q.p[x[i]];
       double r;
       if (qx > 0.0) {

@@ -229,3 +229,53 @@ def linear_state_inputs(cfg: LinearStateConfig, B: int | None = None):
     lead = np.where(ok.all(axis=1), cfg.K, np.argmin(ok, axis=1))
     steps = (1 + lead).astype(np.int32)
     return state, alpha, beta, keys, values, steps
+
+
+@dataclass(frozen=True)
+class LmHeadConfig:
+    """Hidden states and output embeddings of a target and a draft model: the inputs of the
+    scoring forward's last matrix product. Hidden states ~ N(0, 1); target embeddings
+    ~ N(0, (sigma / sqrt(d))^2), so target logits are ~ N(0, sigma^2); the draft model's
+    hidden states and embeddings are the target's plus independent noise (scale h_noise,
+    w_noise relative to each), so its logits follow the target's."""
+    name: str
+    B: int
+    K: int
+    V: int
+    d: int
+    sigma: float
+    h_noise: float
+    w_noise: float
+    temp: float
+    top_k: int
+    seed: int = 6
+
+
+LMHEAD = LmHeadConfig("lmhead_B512_K8_V151936_d4096_bf16_T0.8_topk50", 512, 8, 151936, 4096,
+                      4.0, 0.5, 0.5, 0.8, 50)
+
+
+def lmhead_inputs(cfg: LmHeadConfig, B: int | None = None, V: int | None = None):
+    """(target_hidden [B, K+1, d], draft_hidden [B, K, d], target_weight [V, d],
+    draft_weight [V, d]) as bfloat16 bit patterns."""
+    B = cfg.B if B is None else int(B)
+    V = cfg.V if V is None else int(V)
+    K, d = cfg.K, cfg.d
+    gh, gw, gn = rng(cfg.seed, S_STATE), rng(cfg.seed, S_KEYS), rng(cfg.seed, S_VALUES)
+    ws = np.float32(cfg.sigma / np.sqrt(d))
+    wt = np.empty((V, d), np.uint16)
+    wd = np.empty((V, d), np.uint16)
+    for v0 in range(0, V, 4096):
+        n = min(4096, V - v0)
+        w = gw.standard_normal((n, d), dtype=np.float32) * ws
+        wt[v0:v0 + n] = f32_to_bf16_bits(w)
+        wd[v0:v0 + n] = f32_to_bf16_bits(
+            w + gn.standard_normal((n, d), dtype=np.float32) * (ws * np.float32(cfg.w_noise)))
+    ht = np.empty((B, K + 1, d), np.uint16)
+    hd = np.empty((B, K, d), np.uint16)
+    for b in range(B):
+        h = gh.standard_normal((K + 1, d), dtype=np.float32)
+        ht[b] = f32_to_bf16_bits(h)
+        hd[b] = f32_to_bf16_bits(
+            h[:K] + gh.standard_normal((K, d), dtype=np.float32) * np.float32(cfg.h_noise))
+    return ht, hd, wt, wd

@@ -872,3 +872,30 @@ def test_lmhead_logits_match_numpy_matmul():
     # a transposed operand or a dropped row would not match
     assert not np.allclose(got[:, :7], (specgen.bf16_bits_to_f32(hb).astype(np.float64) @
                                         specgen.bf16_bits_to_f32(hb).astype(np.float64).T)[:, :7])
+
+
+def test_double_logits_and_the_logit_gap_flag():
+    """Logit rows given in double give what the same values in float32 give; the gap flag
+    marks exactly the rows whose argmax or top-k boundary sits within the gap window."""
+    g = np.random.default_rng(23)
+    B, K, V = 6, 2, 40
+    t32 = g.normal(0, 2, (B, K + 1, V)).astype(np.float32)
+    d32 = (t32[:, :K] + g.normal(0, 1, (B, K, V))).astype(np.float32)
+    toks = draft_tokens(d32, 1.0, 5, 1.0, g.random((B, K)).astype(np.float32))
+    u = g.random((B, K + 1)).astype(np.float32)
+    a32 = oracle.verify_chain(t32, d32, toks, u, 1.0, 5)
+    a64 = oracle.verify_chain(t32.astype(np.float64), d32.astype(np.float64), toks, u, 1.0, 5)
+    for x, y in zip(a32, a64):
+        np.testing.assert_array_equal(x, y)
+    # greedy: row 0's argmax leads the runner-up by 5e-4, row 1's by 0.5
+    tg = np.zeros((2, 2, 8), np.float64)
+    tg[:, :, 3] = 1.0
+    tg[0, :, 5] = 1.0 - 5e-4
+    tg[1, :, 5] = 0.5
+    x = np.full((2, 1), 3, np.int32)
+    _, _, fl = oracle.verify_chain(tg, None, x, np.zeros((2, 2), np.float32), 0.0,
+                                   windows=oracle.FP32_LOGITS)
+    assert fl[0] & oracle.FLAG_GAP and not fl[1] & oracle.FLAG_GAP
+    _, _, fl = oracle.verify_chain(tg, None, x, np.zeros((2, 2), np.float32), 0.0,
+                                   windows=oracle.FP64)
+    assert not fl.any()
