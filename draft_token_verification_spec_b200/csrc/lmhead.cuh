@@ -398,11 +398,11 @@ __global__ void __launch_bounds__(kThreads) lmhead_merge_kernel(const LmMergeJob
     o.argmax = j.kept_id[size_t(row) * k];
     o.n = min(k, n);
     o.status = (s_bad || n < k || !(m > -INFINITY)) ? ROW_INVALID : ROW_OK;
-    double z = 0.0;
+    Fx128 z = fx_zero();  // exact, so it equals the same sum taken in any order
     if (j.temp > 0.0f)
       for (int i = 0; i < o.n; ++i)
-        z += weight_d(j.kept_val[size_t(row) * k + i], m, 1.0 / double(j.temp));
-    o.zd = z;
+        z = fx_add(z, fx_from(weight_d(j.kept_val[size_t(row) * k + i], m, 1.0 / double(j.temp))));
+    o.zd = fx_to_double(z);
     j.out[row] = o;
   }
 }
@@ -508,12 +508,13 @@ __global__ void __launch_bounds__(kThreads) lmhead_chain_kernel(const LmChainJob
       const LmRow sq = j.rows[drow0 + a];
       const float* qv = j.kept_val + (drow0 + a) * k;
       const int32_t* qid = j.kept_id + (drow0 + a) * k;
+      const double izp = 1.0 / sp.zd, izq = 1.0 / sq.zd;
       tok = sparse_draw(
           pid, k,
           [&](int v) {
             const float lp = lm_lookup(pv, pid, k, v), lq = lm_lookup(qv, qid, k, v);
-            const double p = weight_d(lp, sp.m, iT) / sp.zd;
-            const double q = lq > -INFINITY ? weight_d(lq, sq.m, iT) / sq.zd : 0.0;
+            const double p = weight_d(lp, sp.m, iT) * izp;
+            const double q = lq > -INFINITY ? weight_d(lq, sq.m, iT) * izq : 0.0;
             return fx_from(fmax(p - q, 0.0));
           },
           u[K], sm);

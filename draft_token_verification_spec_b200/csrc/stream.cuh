@@ -85,20 +85,24 @@ namespace sv {
 #ifndef SV_RING_KB_TOPK
 #define SV_RING_KB_TOPK 32
 #endif
+#ifndef SV_RING_NBUF_TOPK
+#define SV_RING_NBUF_TOPK 2
+#endif
 constexpr int kMaxRing = 4;
 
 enum : int { SM_GREEDY = 0, SM_SUMS = 1, SM_TOPK = 2, SM_TOPP = 3 };
 
 template <int kMode>
 struct Ring {
-  static constexpr int kBuf = kMode <= SM_SUMS ? SV_RING_NBUF_PLAIN : SV_RING_NBUF_CAND;
+  static constexpr int kBuf = kMode <= SM_SUMS ? SV_RING_NBUF_PLAIN
+                              : (kMode == SM_TOPK ? SV_RING_NBUF_TOPK : SV_RING_NBUF_CAND);
   static constexpr int kBytes =
       (kMode <= SM_SUMS ? SV_RING_KB_PLAIN : (kMode == SM_TOPK ? SV_RING_KB_TOPK : SV_RING_KB_CAND)) *
       1024;
   static constexpr int kBufBytes = kBytes + 128;  // a chunk starts up to 15 bytes in
   static constexpr int kVec = kBytes / (16 * kThreads);  // vectors per consumer thread
   static_assert(kBytes % (16 * kThreads) == 0, "chunk = whole vectors per consumer");
-  static_assert((kBuf & (kBuf - 1)) == 0 && kBuf <= kMaxRing, "ring depth: power of two");
+  static_assert(kBuf >= 2 && kBuf <= kMaxRing, "ring depth");
 };
 
 __host__ __device__ constexpr int stream_chunk_bytes(int mode) {
