@@ -13,8 +13,11 @@
 // The ratio tests and the draw are taken in double precision: p(v) = exp((l_v - m) / T) / zd
 // over the kept set, zd the double normaliser of the row statistics. A row whose statistics
 // carry no zd (untruncated rows, rows the exact finisher settled) has it summed here, by the
-// whole block, the first time the scan reaches it. The draw's masses are doubles summed as
-// exact 128-bit fixed point.
+// whole block, the first time the scan reaches a test that needs it. For untruncated rows the
+// test first uses the streaming kernel's fp32 normaliser with a bound on its error: only a
+// ratio within that bound of u needs the double one (the decision is the same either way, as
+// the true ratio lies inside the bound). The draw's masses are doubles summed as exact 128-bit
+// fixed point, with double normalisers (summed here when the scan did not need them).
 #pragma once
 
 #include "draw.cuh"
@@ -35,6 +38,10 @@ struct ChainJob {
   const int32_t* kept_ids;  // [rows][kKeptCap]
   int greedy;
   float temp;             // the temperature as given (sampling)
+  // > 0: rows without a double normaliser carry an fp32 one (RowStats::z) whose relative
+  // error is at most zguard + 2^-23 |m| log2(e) / T (untruncated rows of the streaming
+  // kernel); a ratio test that clears that margin is decided with it. 0: never.
+  float zguard;
   int32_t* accepted_len;  // [B]
   int32_t* out_tokens;    // [B][K+1]
 };
@@ -47,6 +54,43 @@ __device__ __forceinline__ int row_event(const RowStats& s) {
 }
 
 constexpr int kZPos = 32;  // positions whose listed rows get their normalisers up front
+
+// The ratio test at position i when a double normaliser is missing: each missing one is
+// replaced by the row's fp32 normaliser z, whose relative error is at most
+// e = zguard + 2^-23 |m| c (the summation and ex2 roundings of the streaming kernel, and the
+// rounding of m c and c that shifts every exponent of the row). The true ratio then lies in
+// [r (1 - g), r (1 + g)] with g twice the sum of the missing rows' e (a margin over the
+// first-order bound); a u outside that interval is decided, one inside returns EV_NEEDZ. The
+// token's own weights are doubles, and a zero weight decides exactly as the double test does.
+template <typename T>
+__device__ __forceinline__ int guarded_test(const ChainJob& j, const RowStats& sp,
+                                            const RowStats& sq, double zp, double zq,
+                                            const T* trow0, const T* drow0, int i, int xi,
+                                            int V, double iT, float ui) {
+  const float lp = Elem<T>::load(trow0, size_t(i) * V + xi);
+  const float lq = Elem<T>::load(drow0, size_t(i) * V + xi);
+  const double wp = kept_weight_d<T>(sp, iT, lp, xi);
+  const double wq = kept_weight_d<T>(sq, iT, lq, xi);
+  if (wq == 0.0) return wp > 0.0 ? EV_ACCEPT : EV_STOP;  // r = inf (u < 1) or r = 0
+  if (wp == 0.0) return EV_STOP;
+  double g = 0.0;
+  if (zp < 0.0) {
+    if (!(sp.z > 0.0f && sp.z < INFINITY)) return EV_NEEDZ;
+    zp = double(sp.z);
+    g += double(j.zguard) + 0x1p-23 * fabs(double(sp.m) * double(sp.c));
+  }
+  if (zq < 0.0) {
+    if (!(sq.z > 0.0f && sq.z < INFINITY)) return EV_NEEDZ;
+    zq = double(sq.z);
+    g += double(j.zguard) + 0x1p-23 * fabs(double(sq.m) * double(sq.c));
+  }
+  g *= 2.0;
+  const double r = (wp / zp) / (wq / zq);
+  const double uu = double(ui);
+  if (uu < fmin(1.0, r * (1.0 - g))) return EV_ACCEPT;
+  if (uu >= r * (1.0 + g)) return EV_STOP;
+  return EV_NEEDZ;
+}
 
 template <typename T>
 __global__ void __launch_bounds__(kThreads) chain_finish_kernel(const ChainJob j) {
@@ -121,6 +165,7 @@ __global__ void __launch_bounds__(kThreads) chain_finish_kernel(const ChainJob j
                   const double zq = i == zpos ? s_z[1] : (i < npos ? s_zl[1][i] : sq.zd);
                   if (zp < 0.0 || zq < 0.0) {
                     e = EV_NEEDZ;
+                    if (j.zguard > 0.0f) e = guarded_test<T>(j, sp, sq, zp, zq, trow0, drow0, i, xi, V, iT, u[i]);
                   } else {
                     const float lp = Elem<T>::load(trow0, size_t(i) * V + xi);
                     const float lq = Elem<T>::load(drow0, size_t(i) * V + xi);
@@ -182,15 +227,32 @@ __global__ void __launch_bounds__(kThreads) chain_finish_kernel(const ChainJob j
     const float w = u[K];
     const size_t prow_idx = size_t(b) * (K + 1) + a;
     const int nk = j.kept_n ? j.kept_n[prow_idx] : 0;
-    // the normalisers the test at a used (the bonus draw needs none: it scales by its total)
-    const double izp =
-        a < K ? 1.0 / (a == s_zpos ? s_z[0] : (a < npos ? s_zl[0][a] : sp.zd)) : 1.0;
+    // the double normalisers at a (the bonus draw needs none: it scales by its total); a
+    // test the fp32 normalisers decided leaves them to be summed now
+    if (a < K) {
+      const size_t dr = size_t(j.B) * (K + 1) + size_t(b) * K + a;
+      double zp = a == s_zpos ? s_z[0] : (a < npos ? s_zl[0][a] : sp.zd);
+      double zq = a == s_zpos ? s_z[1] : (a < npos ? s_zl[1][a] : ds[a].zd);
+      if (zp < 0.0)
+        zp = row_zd<T>(sp, prow, V, iT, sm.scr, j.kept_ids + prow_idx * kKeptCap, nk);
+      if (zq < 0.0)
+        zq = row_zd<T>(ds[a], drow0 + size_t(a) * V, V, iT, sm.scr, j.kept_ids + dr * kKeptCap,
+                       j.kept_n ? j.kept_n[dr] : 0);
+      __syncthreads();
+      if (threadIdx.x == 0) {
+        s_z[0] = zp;
+        s_z[1] = zq;
+        s_zpos = a;
+      }
+      __syncthreads();
+    }
+    const double izp = a < K ? 1.0 / s_z[0] : 1.0;
     tok = -1;
     if (nk > 0 && nk <= kSparseCap) {
       const int32_t* ids = j.kept_ids + prow_idx * kKeptCap;
       if (a < K) {
         const RowStats sq = ds[a];
-        const double izq = 1.0 / (a == s_zpos ? s_z[1] : (a < npos ? s_zl[1][a] : sq.zd));
+        const double izq = 1.0 / s_z[1];
         const T* qrow = drow0 + size_t(a) * V;
         tok = sparse_draw(
             ids, nk,
@@ -211,7 +273,7 @@ __global__ void __launch_bounds__(kThreads) chain_finish_kernel(const ChainJob j
     } else {
       if (a < K) {
         const RowStats sq = ds[a];
-        const double izq = 1.0 / (a == s_zpos ? s_z[1] : (a < npos ? s_zl[1][a] : sq.zd));
+        const double izq = 1.0 / s_z[1];
         const T* qrow = drow0 + size_t(a) * V;
         const bool qal = (reinterpret_cast<uintptr_t>(qrow) & 15u) == 0;
         tok = inverse_cdf_draw(

@@ -16,7 +16,8 @@
 //            K = 16, four per 64-wide stage, accumulating a 128 x 256 tile in one of two
 //            tensor-memory buffers (512 columns), tcgen05.commit releasing stages and tiles;
 //   warps 2-5 epilogue: one logit row per thread (its tensor-memory lane), 32 columns per
-//            tcgen05.ld; the row's running top-k lives in shared memory (value desc, id asc).
+//            tcgen05.ld; the row's running top-k lives in shared memory as an unsorted list
+//            of (value, id) composites whose weakest entry is the next to be replaced.
 // A work item is one 128-row tile and a chunk of consecutive 256-column tiles; at its end the
 // epilogue writes each row's top-k of that chunk, and lmhead_merge_kernel takes the exact
 // top-k of a row from its chunks. Every wait is bounded (kWaitLimitNs); a wait that runs out
@@ -137,6 +138,26 @@ struct __align__(8) LmBars {
   int broken;
 };
 
+// Work item `it`: row tile it % m_tiles of vocabulary chunk it / m_tiles. CTAs running at the
+// same time take neighbouring items, so they share a chunk of the output embeddings, which is
+// then read from HBM about once and from L2 by the other row tiles.
+struct LmItem {
+  int m0, chunk, t0, t1;
+};
+__device__ __forceinline__ LmItem lm_item(const LmJob& j, int it) {
+  LmItem w;
+  w.m0 = (it % j.m_tiles) * kLmBM;
+  w.chunk = it / j.m_tiles;
+  w.t0 = w.chunk * j.tiles_per_chunk;
+  w.t1 = min(j.n_tiles, w.t0 + j.tiles_per_chunk);
+  return w;
+}
+
+// The float whose f32_key is `key` (-0 comes back as +0).
+__device__ __forceinline__ float lm_key_value(uint32_t key) {
+  return __uint_as_float((key & 0x80000000u) ? (key & 0x7FFFFFFFu) : ~key);
+}
+
 __device__ __forceinline__ bool lm_wait(uint64_t* bar, uint32_t parity, LmBars& s,
                                         int32_t* dev_status) {
   if (*reinterpret_cast<volatile int*>(&s.broken)) return false;
@@ -154,8 +175,7 @@ __global__ void __launch_bounds__(kLmThreads, 1)
   // the ring must start on a 1024-byte boundary (swizzle atoms)
   unsigned char* ring = reinterpret_cast<unsigned char*>(
       (reinterpret_cast<uintptr_t>(lm_raw) + 1023) & ~uintptr_t(1023));
-  float* lv = reinterpret_cast<float*>(ring + size_t(kLmStages) * kLmStageBytes);  // [k][128]
-  int32_t* li = reinterpret_cast<int32_t*>(lv + kLmKMax * kLmBM);                  // [k][128]
+  uint64_t* lc = reinterpret_cast<uint64_t*>(ring + size_t(kLmStages) * kLmStageBytes);  // [k][128]
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int items = j.m_tiles * j.nchunk;
   const int kblocks = j.d / kLmBK;
@@ -190,16 +210,14 @@ __global__ void __launch_bounds__(kLmThreads, 1)
       uint32_t phase = 0;
       long long issued = 0;
       for (int it = blockIdx.x; it < items && !s.broken; it += gridDim.x) {
-        const int m0 = (it / j.nchunk) * kLmBM, chunk = it % j.nchunk;
-        const int t0 = chunk * j.tiles_per_chunk;
-        const int t1 = min(j.n_tiles, t0 + j.tiles_per_chunk);
-        for (int t = t0; t < t1; ++t) {
+        const LmItem w = lm_item(j, it);
+        for (int t = w.t0; t < w.t1; ++t) {
           for (int kb = 0; kb < kblocks; ++kb) {
             if (issued >= kLmStages && !lm_wait(&s.empty[stage], phase ^ 1u, s, j.dev_status))
               break;
             unsigned char* a = ring + size_t(stage) * kLmStageBytes;
             mbar_arrive_expect_tx(&s.full[stage], uint32_t(kLmStageBytes));
-            tma_load_2d(a, &map_h, kb * kLmBK, m0, &s.full[stage]);
+            tma_load_2d(a, &map_h, kb * kLmBK, w.m0, &s.full[stage]);
             tma_load_2d(a + kLmStageA, &map_w, kb * kLmBK, t * kLmBN, &s.full[stage]);
             ++issued;
             if (++stage == kLmStages) {
@@ -226,10 +244,8 @@ __global__ void __launch_bounds__(kLmThreads, 1)
       long long tiles = 0;
       bool any = false;
       for (int it = blockIdx.x; it < items && !s.broken; it += gridDim.x) {
-        const int chunk = it % j.nchunk;
-        const int t0 = chunk * j.tiles_per_chunk;
-        const int t1 = min(j.n_tiles, t0 + j.tiles_per_chunk);
-        for (int t = t0; t < t1 && !s.broken; ++t) {
+        const LmItem w = lm_item(j, it);
+        for (int t = w.t0; t < w.t1 && !s.broken; ++t) {
           if (tiles >= 2 && !lm_wait(&s.acc_empty[acc], acc_phase ^ 1u, s, j.dev_status)) break;
           tc_fence_after();
           const uint32_t d_tmem = tmem + uint32_t(acc * kLmBN);
@@ -270,14 +286,21 @@ __global__ void __launch_bounds__(kLmThreads, 1)
     uint32_t acc_phase = 0;
     const int k = j.k;
     for (int it = blockIdx.x; it < items && !s.broken; it += gridDim.x) {
-      const int m0 = (it / j.nchunk) * kLmBM, chunk = it % j.nchunk;
-      const int t0 = chunk * j.tiles_per_chunk;
-      const int t1 = min(j.n_tiles, t0 + j.tiles_per_chunk);
-      const int row = m0 + r;
-      int n = 0;                  // entries in this row's list
-      float thr = -INFINITY;      // the list's k-th value once it is full
-      for (int t = t0; t < t1; ++t) {
-        if (!lm_wait(&s.acc_full[acc], acc_phase, s, j.dev_status)) break;
+      const LmItem w = lm_item(j, it);
+      const int row = w.m0 + r;
+      // The row's list holds the chunk's best k entries so far as composites
+      // (key << 32 | ~id: larger is better, value desc then id asc), unsorted; once it is
+      // full, `weak` is its smallest composite and `wslot` where that sits. A new entry
+      // replaces the weakest, and one scan of the list (independent loads) finds the next.
+      int n = 0;
+      uint64_t weak = 0;
+      int wslot = 0;
+      float thr = -INFINITY;      // the weakest entry's value (a quick first test)
+      bool bad = false;           // a NaN or +inf logit in this chunk of the row
+      for (int t = w.t0; t < w.t1; ++t) {
+        // warp-uniform, as the tensor-memory loads below are .sync.aligned
+        if (!__all_sync(0xffffffffu, lm_wait(&s.acc_full[acc], acc_phase, s, j.dev_status)))
+          break;
         tc_fence_after();
         for (int cc = 0; cc < kLmBN / 32; ++cc) {
           uint32_t v[32];
@@ -287,23 +310,41 @@ __global__ void __launch_bounds__(kLmThreads, 1)
             for (int e = 0; e < 32; ++e)
               if (c0 + e < j.V) j.logits_out[size_t(row) * j.V + c0 + e] = __uint_as_float(v[e]);
           }
-#pragma unroll 4
+          // which of the 32 may enter (against the list as it stands: a superset), then
+          // those in column order; fully unrolled so v stays in registers
+          uint32_t want = 0;
+#pragma unroll
           for (int e = 0; e < 32; ++e) {
             const float x = __uint_as_float(v[e]);
-            const int id = c0 + e;
-            if (id >= j.V || !(n < k || x > thr)) continue;
-            // insert (value desc, id asc): ids arrive in ascending order, so an entry goes
-            // after every entry >= it
-            int pos = n < k ? n : k - 1;
-            while (pos > 0 && lv[(pos - 1) * kLmBM + r] < x) {
-              lv[pos * kLmBM + r] = lv[(pos - 1) * kLmBM + r];
-              li[pos * kLmBM + r] = li[(pos - 1) * kLmBM + r];
-              --pos;
+            const bool in = c0 + e < j.V;
+            bad |= in && !(x < INFINITY);
+            if (in && !(n == k && x < thr)) want |= 1u << e;
+          }
+          if (want) {
+#pragma unroll
+            for (int e = 0; e < 32; ++e) {
+              if (!((want >> e) & 1u)) continue;
+              const float x = __uint_as_float(v[e]);
+              if (n == k && x < thr) continue;
+              const uint64_t c = (uint64_t(f32_key(x)) << 32) | uint64_t(~uint32_t(c0 + e));
+              if (n < k) {
+                lc[n * kLmBM + r] = c;
+                if (++n < k) continue;
+              } else if (c > weak) {
+                lc[wslot * kLmBM + r] = c;
+              } else {
+                continue;
+              }
+              weak = ~0ull;
+              for (int i = 0; i < k; ++i) {
+                const uint64_t q = lc[i * kLmBM + r];
+                if (q < weak) {
+                  weak = q;
+                  wslot = i;
+                }
+              }
+              thr = lm_key_value(uint32_t(weak >> 32));
             }
-            lv[pos * kLmBM + r] = x;
-            li[pos * kLmBM + r] = id;
-            if (n < k) ++n;
-            if (n == k) thr = lv[(k - 1) * kLmBM + r];
           }
         }
         tc_fence_before();
@@ -314,10 +355,16 @@ __global__ void __launch_bounds__(kLmThreads, 1)
         }
       }
       if (row < j.M) {
-        const size_t o = (size_t(row) * j.nchunk + chunk) * k;
+        // the weakest entry goes to the last slot (the merge reads a chunk's k-th value
+        // there); a NaN first entry tells the merge that the row holds a NaN or +inf logit
+        const size_t o = (size_t(row) * j.nchunk + w.chunk) * k;
         for (int i = 0; i < k; ++i) {
-          j.part_val[o + i] = i < n ? lv[i * kLmBM + r] : -INFINITY;
-          j.part_id[o + i] = i < n ? li[i * kLmBM + r] : INT_MAX;
+          const int src = n < k ? i : (i == k - 1 ? wslot : (i == wslot ? k - 1 : i));
+          const uint64_t c = lc[src * kLmBM + r];
+          j.part_val[o + i] = (i == 0 && bad) ? __int_as_float(0x7fc00000)
+                              : i < n      ? lm_key_value(uint32_t(c >> 32))
+                                           : -INFINITY;
+          j.part_id[o + i] = i < n ? int32_t(~uint32_t(c)) : INT_MAX;
         }
       }
     }
@@ -384,9 +431,7 @@ __global__ void __launch_bounds__(kThreads) lmhead_merge_kernel(const LmMergeJob
     int above = 0;
     for (int q = 0; q < n; ++q) above += cand[q] > e ? 1 : 0;
     if (above < k) {
-      const uint32_t key = uint32_t(e >> 32);
-      const uint32_t u = (key & 0x80000000u) ? (key & 0x7FFFFFFFu) : ~key;
-      j.kept_val[size_t(row) * k + above] = __uint_as_float(u);
+      j.kept_val[size_t(row) * k + above] = lm_key_value(uint32_t(e >> 32));
       j.kept_id[size_t(row) * k + above] = int32_t(~uint32_t(e));
     }
   }

@@ -474,6 +474,17 @@ spec_status spec_verify_chain(const void* target_logits, const void* draft_logit
   cj.kept_ids = rj.kept_ids;
   cj.greedy = greedy ? 1 : 0;
   cj.temp = temp;
+  if (!greedy && rj.top_k == 0 && rj.top_p >= 1.0f) {
+    // untruncated rows: the streaming kernel's fp32 normaliser sums, per consumer thread,
+    // n = ceil(V / kThreads) weights in order (at most n roundings of 2^-24), each from ex2
+    // (relative error < 2^-22.7) of an exponent whose roundings shift it by at most
+    // 2^-24 (|l| + |m|) c (the |m| part is added per row by the finisher; the mean of
+    // |l - m| c under the row's own distribution is at most log2 V), and rescales the sum
+    // by ex2 at most once per 16-byte vector, n / 4 times (2^-22 each)
+    const double n = double((V + kThreads - 1) / kThreads);
+    cj.zguard = float(std::ldexp(n + std::log2(double(V)) + 16.0, -24) +
+                      std::ldexp(n / 4.0 + 8.0, -22));
+  }
   cj.accepted_len = accepted_len;
   cj.out_tokens = out_tokens;
   if (dtype == SPEC_BF16)

@@ -829,14 +829,24 @@ __global__ void __launch_bounds__(kStreamThreads, (kMode == SM_TOPP ? 2 : 3))
     const uint4* vb = reinterpret_cast<const uint4*>(ring + size_t(b) * kRingBufBytes);
     const int base = q * job.chunk;
     const int v_lo = (s.pad + s.head) >> 4, v_hi = (s.pad + s.head + s.mid) >> 4;
-    uint4 w[kVecPerThread];
+    // the chunk's vectors of this thread; top-k keeps only their maxima in registers and
+    // reads a vector again from the ring in the rare case that it holds a candidate (the
+    // buffer is released after the appends)
+    auto load_vec = [&](int v) {
+      return (copied && v >= v_lo && v < v_hi) ? vb[v] : neg_inf_vec<T>();
+    };
+    uint4 w[kMode == SM_TOPK ? 1 : kVecPerThread];
     float vm[kVecPerThread];
 #pragma unroll
     for (int u = 0; u < kVecPerThread; ++u) {
-      const int v = u * kThreads + int(threadIdx.x);
-      w[u] = (copied && v >= v_lo && v < v_hi) ? vb[v] : neg_inf_vec<T>();
-      vm[u] = Elem<T>::vmax_nan(w[u]);
+      const uint4 wu = load_vec(u * kThreads + int(threadIdx.x));
+      vm[u] = Elem<T>::vmax_nan(wu);
+      if constexpr (kMode != SM_TOPK) w[u] = wu;
     }
+    auto vec_at = [&](int u) -> uint4 {
+      if constexpr (kMode == SM_TOPK) return load_vec(u * kThreads + int(threadIdx.x));
+      else return w[u];
+    };
     // elements outside the bulk-copied middle (< 16 bytes at each end): thread 0 takes the
     // head, thread 32 the tail, from global memory
     const int head_e = s.head / E, tail_e0 = (s.head + s.mid) / E;
@@ -906,7 +916,8 @@ __global__ void __launch_bounds__(kStreamThreads, (kMode == SM_TOPP ? 2 : 3))
     for (int u = 0; u < kVecPerThread; ++u) {
       const int v = u * kThreads + int(threadIdx.x);
       const int j0 = base + (16 * v - s.pad) / E;
-      cm[u] = st.vec(w[u], vm[u], j0, c, want_ent, (v >= v_lo && v < v_hi) ? thr : INFINITY);
+      cm[u] = st.vec(kMode == SM_TOPK ? uint4{} : vec_at(u), vm[u], j0, c, want_ent,
+                     (v >= v_lo && v < v_hi) ? thr : INFINITY);
       vmax4 = fmaxf(vmax4, vm[u]);  // pad vectors hold -inf; NaN never passes a filter
     }
     if constexpr (kMode == SM_TOPK) {
@@ -916,7 +927,7 @@ __global__ void __launch_bounds__(kStreamThreads, (kMode == SM_TOPP ? 2 : 3))
           const int v = u * kThreads + int(threadIdx.x);
           if (v >= v_lo && v < v_hi && vm[u] >= thr) {
             float x[P];
-            Elem<T>::unpack(w[u], x);
+            Elem<T>::unpack(vec_at(u), x);
 #pragma unroll
             for (int k = 0; k < P; ++k)
               if (x[k] >= thr) cm[u] |= 1u << k;
@@ -943,9 +954,11 @@ __global__ void __launch_bounds__(kStreamThreads, (kMode == SM_TOPP ? 2 : 3))
 #pragma unroll
         for (int u = 0; u < kVecPerThread; ++u) {
           const int j0 = base + (16 * (u * kThreads + int(threadIdx.x)) - s.pad) / E;
+          if (cm[u] == 0) continue;
+          const uint4 wu = vec_at(u);
           for (uint32_t m = cm[u]; m != 0; m &= m - 1) {  // the set bits only
             const int k = __ffs(m) - 1;
-            if (pos < kCapM) cs.cand[pos] = make_comp(Elem<T>::key_at(w[u], k), j0 + k);
+            if (pos < kCapM) cs.cand[pos] = make_comp(Elem<T>::key_at(wu, k), j0 + k);
             ++pos;
           }
         }
@@ -1106,7 +1119,8 @@ __global__ void __launch_bounds__(kStreamThreads, (kMode == SM_TOPP ? 2 : 3))
             csync();
             unsigned long long z = 0;
             long long s1 = 0;
-            const Fx128 zdx = list ? fx_zero() : kept_weights_fx<T>(cs.cand, n, cstar, m, iT);
+            Fx128 zdx = fx_zero();
+            if constexpr (kMode == SM_TOPP) zdx = kept_weights_fx<T>(cs.cand, n, cstar, m, iT);
             for (int i = threadIdx.x; i < n; i += kThreads) {
               const uint64_t e = cs.cand[i];
               if (e < cstar) continue;
@@ -1120,7 +1134,7 @@ __global__ void __launch_bounds__(kStreamThreads, (kMode == SM_TOPP ? 2 : 3))
                 if (slot < kKeptCap) rj.kept_ids[size_t(row) * kKeptCap + slot] = comp_id(e);
               }
             }
-            if (!list) zd = fx_to_double(creduce_fx(zdx, scr_fx(aux)));
+            if constexpr (kMode == SM_TOPP) zd = fx_to_double(creduce_fx(zdx, scr_fx(aux)));
             zfx = creduce<unsigned long long>(z, aux.scr_u64, OpSum());
             S1 = double(creduce<long long>(s1, aux.scr_s64, OpSum())) / double(kS1Fx);
             thr_key = comp_key(cstar);

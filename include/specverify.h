@@ -274,7 +274,10 @@ spec_status spec_verify_chain_noalloc(const void* target_logits, const void* dra
 
 /* Copies the device status word of `workspace` to the host (synchronises `stream`):
  * SPEC_OK, or SPEC_ERR_DEVICE_TIMEOUT if a kernel of an earlier call on this
- * workspace gave up waiting for a copy. The word is cleared by every verify call. */
+ * workspace gave up waiting for a copy (or, for spec_verify_chain_lmhead, for a tensor-core
+ * stage). The word is cleared by every verify call. It works on the workspaces of
+ * spec_verify_chain, spec_verify_tree_typical, spec_verify_tree_sampling and
+ * spec_verify_chain_lmhead alike (the word is the first 4 bytes of each). */
 spec_status spec_get_device_status(const void* workspace, int32_t* status_out, void* stream);
 
 /* Timing hook for measurement tools: while set, every spec_verify_chain and

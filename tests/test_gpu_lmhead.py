@@ -61,10 +61,14 @@ def _fused(ht, hd, wt, wd, x, u, temp, top_k, want_logits=True):
     rows = B * K1 + (0 if temp == 0.0 else B * (K1 - 1))
     lo = torch.full((rows, V), float("nan"), dtype=torch.float32, device="cuda") if want_logits \
         else None
+    ws = torch.empty(sv.spec_lmhead_workspace_size(B, K, V, d, 0 if temp == 0.0 else top_k),
+                     dtype=torch.uint8, device="cuda")
     acc, out = sv.spec_verify_chain_lmhead(
         _bf(ht), None if temp == 0.0 else _bf(hd), _bf(wt), None if temp == 0.0 else _bf(wd),
-        torch.from_numpy(x).cuda(), torch.from_numpy(u).cuda(), temp, top_k, logits_out=lo)
+        torch.from_numpy(x).cuda(), torch.from_numpy(u).cuda(), temp, top_k, logits_out=lo,
+        workspace=ws)
     torch.cuda.synchronize()
+    assert sv.spec_get_device_status(ws) == sv.SPEC_OK  # no wait of the kernel ran out
     return acc.cpu().numpy(), out.cpu().numpy(), lo
 
 
@@ -99,6 +103,25 @@ def test_lmhead_fusion_equals_unfused_verification_of_its_logits(temp, top_k):
     u = np.random.default_rng(4).random((8, 6)).astype(np.float32)
     acc, out, lo = _fused(ht, hd, wt, wd, x, u, temp, top_k)
     acc_u, out_u = _unfused_on(lo, 8, 5, cfg.V, x, u, temp, top_k)
+    assert np.array_equal(acc, acc_u) and np.array_equal(out, out_u)
+    assert acc.min() >= 0
+
+
+@pytest.mark.parametrize("temp,top_k", [(0.0, 0), (0.8, 50)])
+def test_lmhead_persistent_ctas_over_many_tiles(temp, top_k):
+    """More work items than SMs (5 row tiles x up to 118 vocabulary tiles): every CTA runs
+    several items through the same stage ring and tensor-memory buffers. Logits against the
+    oracle's double product on every row, decisions against the unfused verification."""
+    cfg, ht, hd, wt, wd = _case(64, 30000, 256, K=8, seed=9, temp=temp, top_k=top_k)
+    lt, ld = _oracle_logits(ht, hd, wt, wd)
+    x = _drafts(ld, temp, top_k, 8)
+    u = np.random.default_rng(10).random((64, 9)).astype(np.float32)
+    acc, out, lo = _fused(ht, hd, wt, wd, x, u, temp, top_k)
+    got = lo.cpu().numpy().astype(np.float64)
+    ref = lt.reshape(-1, cfg.V) if temp == 0.0 else np.concatenate(
+        [lt.reshape(-1, cfg.V), ld.reshape(-1, cfg.V)])
+    assert (np.abs(got - ref) <= 1e-3 + 1e-4 * np.abs(ref)).all()
+    acc_u, out_u = _unfused_on(lo, 64, 8, cfg.V, x, u, temp, top_k)
     assert np.array_equal(acc, acc_u) and np.array_equal(out, out_u)
     assert acc.min() >= 0
 
