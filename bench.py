@@ -501,10 +501,97 @@ def per_config_lstate(cfg, args, dev) -> dict:
     return res
 
 
+def per_config_lmhead(cfg, args, dev) -> list:
+    """Chain verification from hidden states: the LM-head products of the target and draft
+    models on the tensor cores with the top-k statistics in their epilogue, then the
+    verification from those lists (spec_verify_chain_lmhead), at the configuration's top-k
+    and at temperature 0. Timed with CUDA events around each call; the roofline counts the
+    two products' FLOPs against the whole call."""
+    import torch
+
+    import draft_token_verification_spec_b200 as sv
+
+    ht, hd, wt, wd = specgen.lmhead_inputs(cfg)
+    bf = lambda a: torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).to(dev).view(
+        torch.bfloat16)
+    Ht, Hd, Wt, Wd = bf(ht), bf(hd), bf(wt), bf(wd)
+    B, K, V, d = cfg.B, cfg.K, cfg.V, cfg.d
+    # the drafter's tokens: x_i ~ its top-k distribution at temperature T (or its argmax),
+    # from a plain bf16 product and torch sampling (input preparation, not timed)
+    g = torch.Generator(device=dev)
+    g.manual_seed(cfg.seed)
+    ld = (Hd.reshape(-1, d) @ Wd.T).float()
+    vals, idx = torch.topk(ld, cfg.top_k, dim=1)
+    pick = torch.multinomial(torch.softmax(vals / cfg.temp, dim=1), 1, generator=g)
+    x_s = idx.gather(1, pick).view(B, K).to(torch.int32)
+    x_g = ld.argmax(dim=1).view(B, K).to(torch.int32)
+    del ld, vals, idx
+    u = torch.from_numpy(specgen.dyadic_uniforms(specgen.rng(cfg.seed, specgen.S_ACCEPT),
+                                                 (B, K + 1))).to(dev)
+    peaks, peak_src = measured_peaks()
+    steps = max(3, min(args.steps, 20))
+    out = []
+    for temp, top_k, x in ((cfg.temp, cfg.top_k, x_s), (0.0, 0, x_g)):
+        ws = torch.empty(sv.spec_lmhead_workspace_size(B, K, V, d, top_k), dtype=torch.uint8,
+                         device=dev)
+        acc = torch.empty(B, dtype=torch.int32, device=dev)
+        toks = torch.empty((B, K + 1), dtype=torch.int32, device=dev)
+
+        def call():
+            sv.spec_verify_chain_lmhead(Ht, None if temp == 0 else Hd, Wt,
+                                        None if temp == 0 else Wd, x, u, temp, top_k,
+                                        accepted_len=acc, out_tokens=toks, workspace=ws)
+
+        for _ in range(max(3, args.warmup)):
+            call()
+        torch.cuda.synchronize()
+        ev = _events(steps)
+        for i in range(steps):
+            ev[i][0].record()
+            call()
+            ev[i][1].record()
+        torch.cuda.synchronize()
+        ms = float(np.mean([a.elapsed_time(b) for a, b in ev]))
+        rows = B * (K + 1) + (0 if temp == 0 else B * K)
+        flops = 2.0 * rows * V * d
+        tf = flops / (ms / 1e3) / 1e12
+        name = cfg.name if temp > 0 else cfg.name.replace(f"_T{cfg.temp:g}_topk{cfg.top_k}", "_T0")
+        res = {"workload": name, "metric_unit": "positions/s",
+               "value": B * K / (ms / 1e3), "ms_per_step": ms,
+               "mean_accepted_len": float(acc.float().mean()),
+               "roofline": {"bound": "tensor", "achieved": round(tf, 1),
+                            "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                            "frac": round(tf / peaks["bf16_tflops"], 4),
+                            "peak_source": peak_src + " (cuBLAS bf16 GEMM, burst)",
+                            "kernel": "lmhead_topk_kernel (whole call timed)",
+                            "kernel_ms": round(ms, 4), "algorithmic_flops": flops}}
+        if not args.no_cpu_baseline and temp > 0:
+            import oracle
+            threads = os.cpu_count() or 1
+            t0 = time.perf_counter()
+            lt = oracle.lmhead_logits(ht[:1].reshape(-1, d), wt, threads=threads)
+            lq = oracle.lmhead_logits(hd[:1].reshape(-1, d), wd, threads=threads)
+            oracle.verify_chain(lt.reshape(1, K + 1, V), lq.reshape(1, K, V),
+                                x[:1].cpu().numpy(), u[:1].cpu().numpy(),
+                                float(np.float32(temp)), top_k)
+            dt = time.perf_counter() - t0
+            res["cpu_baseline"] = {"value": K / dt, "unit": "positions/s", "cores": threads,
+                                   "kind": "oracle",
+                                   "sample": f"1 of {B} sequences (double LM-head products "
+                                             f"and verification), {threads} threads, "
+                                             f"{dt:.1f}s"}
+        out.append(res)
+        del ws
+    del Ht, Hd, Wt, Wd
+    torch.cuda.empty_cache()
+    return out
+
+
 def per_config_all(args) -> list:
     """Every other workload, one entry each (1 GPU): the three other chain workloads, the
-    temperature-0 variants of the two that have one, the MEDUSA tree, and the
-    linear-attention state commit."""
+    temperature-0 variants of the two that have one, the MEDUSA tree, the linear-attention
+    state commit, and verification from hidden states (LM head fused; sampling and
+    temperature 0)."""
     import torch
 
     dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", 0)))
@@ -515,6 +602,7 @@ def per_config_all(args) -> list:
         log(f"per-config {out[-1]['workload']}: {out[-1]['ms_per_step']:.4f} ms")
     out.append(per_config_tree(specgen.CFG4, args, dev))
     out.append(per_config_lstate(specgen.LSTATE, args, dev))
+    out.extend(per_config_lmhead(specgen.LMHEAD, args, dev))
     return out
 
 

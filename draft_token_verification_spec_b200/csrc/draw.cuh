@@ -21,7 +21,8 @@
 namespace sv {
 
 constexpr int kMaxDrawChunks = 128;
-constexpr int kSparseCap = kThreads;                    // support of a sparse draw
+constexpr int kSparsePer = 4;                           // support entries per thread
+constexpr int kSparseCap = kSparsePer * kThreads;       // support of a sparse draw
 
 struct DrawSmem {
   Fx128 wchunk[kMaxDrawChunks][kWarps];   // per-warp mass of each chunk
@@ -137,29 +138,54 @@ __device__ int inverse_cdf_draw(F&& f, int V, float w, DrawSmem& sm) {
   return tok;
 }
 
-// The same draw when every entry outside ids[0..n) (distinct ids, any order, n <= kThreads)
-// has mass 0: the support is sorted by id and one block-wide prefix sum replaces the pass
-// over the row. mass(v) gives the Fx128 mass of entry v; the result is identical to
-// inverse_cdf_draw over the whole row with the same masses.
+// The same draw when every entry outside ids[0..n) (distinct ids, any order,
+// n <= kSparseCap) has mass 0: the support is sorted by id (each id counts the smaller ones)
+// and one block-wide prefix sum replaces the pass over the row, thread t holding sorted
+// positions [kSparsePer t, kSparsePer (t + 1)). mass(v) gives the Fx128 mass of entry v; the
+// result is identical to inverse_cdf_draw over the whole row with the same masses.
 template <typename F>
 __device__ int sparse_draw(const int32_t* ids, int n, F&& mass, float w, DrawSmem& sm) {
   const int t = threadIdx.x;
-  const int my = t < n ? ids[t] : INT_MAX;
-  if (t < n) sm.ids[t] = my;
+  int my[kSparsePer];
+#pragma unroll
+  for (int q = 0; q < kSparsePer; ++q) {
+    const int i = q * kThreads + t;
+    my[q] = i < n ? ids[i] : INT_MAX;
+    if (i < n) sm.ids[i] = my[q];
+  }
   if (t == 0) sm.best = INT_MAX;
   __syncthreads();
-  int rank = 0;
-  if (t < n)
-    for (int j = 0; j < n; ++j) rank += sm.ids[j] < my ? 1 : 0;
+  int rank[kSparsePer];
+#pragma unroll
+  for (int q = 0; q < kSparsePer; ++q) {
+    rank[q] = 0;
+    if (q * kThreads + t < n)
+      for (int j = 0; j < n; ++j) rank[q] += sm.ids[j] < my[q] ? 1 : 0;
+  }
   __syncthreads();
-  if (t < n) sm.ids[rank] = my;
+#pragma unroll
+  for (int q = 0; q < kSparsePer; ++q)
+    if (q * kThreads + t < n) sm.ids[rank[q]] = my[q];
   __syncthreads();
-  const int v = t < n ? sm.ids[t] : -1;
-  const Fx128 r = t < n ? mass(v) : fx_zero();
+  Fx128 r[kSparsePer];
+  Fx128 own = fx_zero();
+#pragma unroll
+  for (int q = 0; q < kSparsePer; ++q) {
+    const int p = kSparsePer * t + q;
+    r[q] = p < n ? mass(sm.ids[p]) : fx_zero();
+    own = fx_add(own, r[q]);
+  }
   Fx128 S;
-  const Fx128 ex = block_exclusive_scan_fx(r, sm.scr, &S);
+  Fx128 cum = block_exclusive_scan_fx(own, sm.scr, &S);
   const double target = double(w) * fx_to_double(S);
-  if (!fx_is_zero(r) && fx_to_double(fx_add(ex, r)) > target) atomicMin(&sm.best, v);
+#pragma unroll
+  for (int q = 0; q < kSparsePer; ++q) {
+    cum = fx_add(cum, r[q]);
+    if (!fx_is_zero(r[q]) && fx_to_double(cum) > target) {
+      atomicMin(&sm.best, sm.ids[kSparsePer * t + q]);
+      break;
+    }
+  }
   __syncthreads();
   int tok = sm.best;
   if (fx_is_zero(S)) {
@@ -168,7 +194,9 @@ __device__ int sparse_draw(const int32_t* ids, int n, F&& mass, float w, DrawSme
     __syncthreads();
     if (t == 0) sm.best = -1;
     __syncthreads();
-    if (!fx_is_zero(r)) atomicMax(&sm.best, v);
+#pragma unroll
+    for (int q = 0; q < kSparsePer; ++q)
+      if (!fx_is_zero(r[q])) atomicMax(&sm.best, sm.ids[kSparsePer * t + q]);
     __syncthreads();
     tok = sm.best;
   }

@@ -44,7 +44,11 @@ constexpr int kLmStageBytes = kLmStageA + kLmStageB;
 constexpr int kLmThreads = 192;
 constexpr int kLmMergeCap = 4096;                  // chunks x k a row's merge may hold
 // dynamic shared memory: the ring (1024-byte aligned atoms), then the top-k lists
-constexpr size_t kLmSmem = size_t(kLmStages) * kLmStageBytes + size_t(kLmKMax) * kLmBM * 8 + 1024;
+constexpr int kLmStageStride = 33;                 // floats per row of the epilogue's staging
+// dynamic shared memory: the ring, the top-k lists, the staging of 32 logits per row
+constexpr size_t kLmSmem = size_t(kLmStages) * kLmStageBytes + size_t(kLmKMax) * kLmBM * 8 +
+                           size_t(kLmBM) * kLmStageStride * 4 + 1024;
+static_assert(kLmSmem + 1024 <= 227 * 1024, "LM-head shared memory (dynamic and static)");
 
 // ------------------------------------------------------------------ PTX wrappers
 __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int x, int y,
@@ -176,6 +180,7 @@ __global__ void __launch_bounds__(kLmThreads, 1)
   unsigned char* ring = reinterpret_cast<unsigned char*>(
       (reinterpret_cast<uintptr_t>(lm_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* lc = reinterpret_cast<uint64_t*>(ring + size_t(kLmStages) * kLmStageBytes);  // [k][128]
+  float* stg = reinterpret_cast<float*>(lc + kLmKMax * kLmBM);  // [128][kLmStageStride]
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int items = j.m_tiles * j.nchunk;
   const int kblocks = j.d / kLmBK;
@@ -242,7 +247,6 @@ __global__ void __launch_bounds__(kLmThreads, 1)
       int acc = 0;
       uint32_t acc_phase = 0;
       long long tiles = 0;
-      bool any = false;
       for (int it = blockIdx.x; it < items && !s.broken; it += gridDim.x) {
         const LmItem w = lm_item(j, it);
         for (int t = w.t0; t < w.t1 && !s.broken; ++t) {
@@ -258,7 +262,6 @@ __global__ void __launch_bounds__(kLmThreads, 1)
             for (int k = 0; k < kLmBK / 16; ++k)  // +32 bytes per K = 16 step (>> 4: +2)
               tc_mma(d_tmem, ad + uint64_t(2 * k), bd + uint64_t(2 * k), kLmIdesc, kb > 0 || k > 0);
             tc_commit(&s.empty[stage]);  // the stage is free once these MMAs have read it
-            any = true;
             if (++stage == kLmStages) {
               stage = 0;
               phase ^= 1u;
@@ -273,7 +276,6 @@ __global__ void __launch_bounds__(kLmThreads, 1)
         }
       }
       // every MMA issued has completed before the tensor memory is freed
-      (void)any;
       tc_commit(&s.done);
       mbar_wait(&s.done, 0);
     }
@@ -310,8 +312,9 @@ __global__ void __launch_bounds__(kLmThreads, 1)
             for (int e = 0; e < 32; ++e)
               if (c0 + e < j.V) j.logits_out[size_t(row) * j.V + c0 + e] = __uint_as_float(v[e]);
           }
-          // which of the 32 may enter (against the list as it stands: a superset), then
-          // those in column order; fully unrolled so v stays in registers
+          // which of the 32 may enter (against the list as it stands: a superset); those few
+          // go through this row's staging slot in shared memory, so the list code below
+          // exists once (a small epilogue keeps the MMA warp's instructions cached)
           uint32_t want = 0;
 #pragma unroll
           for (int e = 0; e < 32; ++e) {
@@ -321,10 +324,13 @@ __global__ void __launch_bounds__(kLmThreads, 1)
             if (in && !(n == k && x < thr)) want |= 1u << e;
           }
           if (want) {
+            float* sr = stg + r * kLmStageStride;
 #pragma unroll
-            for (int e = 0; e < 32; ++e) {
-              if (!((want >> e) & 1u)) continue;
-              const float x = __uint_as_float(v[e]);
+            for (int e = 0; e < 32; ++e) sr[e] = __uint_as_float(v[e]);
+            while (want) {
+              const int e = __ffs(int(want)) - 1;
+              want &= want - 1u;
+              const float x = sr[e];
               if (n == k && x < thr) continue;
               const uint64_t c = (uint64_t(f32_key(x)) << 32) | uint64_t(~uint32_t(c0 + e));
               if (n < k) {

@@ -109,6 +109,12 @@ __host__ __device__ constexpr size_t lstate_commit_smem(int S, int dk) {
   return size_t(S) * dk * 8 + size_t(S) * kLsCols * 4;
 }
 
+// 16-byte global -> shared copy that bypasses the registers (and L1).
+__device__ __forceinline__ void ls_copy16(void* dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src)
+               : "memory");
+}
+
 template <int R>
 __global__ void __launch_bounds__(kThreads) lstate_commit_kernel(const LsCommitJob j) {
   extern __shared__ __align__(16) float lsm[];
@@ -123,18 +129,28 @@ __global__ void __launch_bounds__(kThreads) lstate_commit_kernel(const LsCommitJ
   const int a = j.steps[b];
   if (a <= 0 || a > j.S) return;  // nothing to commit (uniform)
   const int S = j.S, dv = j.dv;
-  for (int i = threadIdx.x; i < a * dk; i += kThreads) {
-    ks[i] = j.keys[size_t(bh) * S * dk + i];
-    ws[i] = j.w[size_t(bh) * S * dk + i];
-  }
-  const float* urow = j.u + size_t(bh) * S * dv;
   const int c0 = tile * kLsCols;
-  for (int i = threadIdx.x; i < a * kLsCols; i += kThreads) {
-    const int t = i / kLsCols, c = c0 + i % kLsCols;
-    mt[t][i % kLsCols] = c < dv ? urow[size_t(t) * dv + c] : 0.0f;
+  // every load is issued before any is waited for: the factors go to shared memory by
+  // asynchronous copies (keys and w of the first a steps, and this tile's columns of u; a
+  // tile past dv reads zeros), and the state tile goes to registers meanwhile
+  {
+    const float4* kin = reinterpret_cast<const float4*>(j.keys + size_t(bh) * S * dk);
+    const float4* win = reinterpret_cast<const float4*>(j.w + size_t(bh) * S * dk);
+    for (int i = threadIdx.x; i < a * dk / 4; i += kThreads) {
+      ls_copy16(ks + 4 * i, kin + i);
+      ls_copy16(ws + 4 * i, win + i);
+    }
+    const float* urow = j.u + size_t(bh) * S * dv;
+    for (int i = threadIdx.x; i < a * (kLsCols / 4); i += kThreads) {
+      const int t = i / (kLsCols / 4), c = 4 * (i % (kLsCols / 4));
+      if (c0 + c < dv)
+        ls_copy16(&mt[t][c], urow + size_t(t) * dv + c0 + c);
+      else
+        *reinterpret_cast<float4*>(&mt[t][c]) = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+    asm volatile("cp.async.commit_group;" ::: "memory");
   }
   const float ga = j.gamma[size_t(bh) * S + a - 1];
-  __syncthreads();
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int rl = lane & 15;                          // row lane: rows rl, rl + 16, ...
   const int cl = warp * 8 + (lane >> 4) * 4;         // first of this lane's 4 columns (in tile)
@@ -146,6 +162,8 @@ __global__ void __launch_bounds__(kThreads) lstate_commit_kernel(const LsCommitJ
   for (int r = 0; r < R; ++r)
     x[r] = live ? *reinterpret_cast<const float4*>(base + size_t(rl + 16 * r) * dv + col)
                 : make_float4(0.f, 0.f, 0.f, 0.f);
+  asm volatile("cp.async.wait_all;" ::: "memory");
+  __syncthreads();
   // M[t][c] = U[t][c] - sum_i W[t][i] S[i][c]: partial sums over this lane's rows, then the
   // 16 row lanes of the warp (xor shuffles keep them within the half-warp)
   for (int t = 0; t < a; ++t) {

@@ -211,7 +211,7 @@ cudaError_t launch_refine(const sv::RefineJob& j, cudaStream_t s) {
     std::lock_guard<std::mutex> lock(mu);
     sms_of[dev] = sms;
   }
-  const size_t dyn = size_t(sv::kRefineCap) * sizeof(uint64_t);
+  const size_t dyn = sv::refine_smem<T>();
   e = cudaFuncSetAttribute(sv::topp_refine_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            int(dyn));
   if (e != cudaSuccess) return e;
@@ -662,7 +662,8 @@ spec_status spec_commit_linear_state(float* state, int B, int H, int dk, int dv,
   if (!state || !keys || !w || !u || !gamma || !steps || B <= 0 || H <= 0 || S <= 0 || dk <= 0 ||
       dv <= 0)
     return SPEC_ERR_INVALID_ARG;
-  if (S > sv::kLsMaxSteps || dv % 4 != 0 || !aligned16(state) ||
+  if (S > sv::kLsMaxSteps || dv % 4 != 0 || !aligned16(state) || !aligned16(keys) ||
+      !aligned16(w) || !aligned16(u) ||
       (dk != 32 && dk != 64 && dk != 128 && dk != 256))
     return SPEC_ERR_UNSUPPORTED;
   const long long blocks = (long long)B * H * ((dv + sv::kLsCols - 1) / sv::kLsCols);

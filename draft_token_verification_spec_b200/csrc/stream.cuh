@@ -85,6 +85,9 @@ namespace sv {
 #ifndef SV_RING_KB_TOPK
 #define SV_RING_KB_TOPK 32
 #endif
+#ifndef SV_TOPK_CTAS
+#define SV_TOPK_CTAS 3        // top-k CTAs resident per SM (2 or 3)
+#endif
 #ifndef SV_RING_NBUF_TOPK
 #define SV_RING_NBUF_TOPK 2
 #endif
@@ -121,7 +124,7 @@ constexpr int kBins = 1024;                     // log-weight bins
 constexpr float kBinScale = 32.0f;              // bins per log2 unit of weight
 constexpr int kMemberCap = 512;                 // members of the crossing bin
 constexpr int kRankMax = 1024;                  // lists this short are ranked directly
-constexpr int kStreamMaxTopK = kKeptCap;        // top-k the candidate path takes
+constexpr int kStreamMaxTopK = 256;             // top-k the candidate path takes
 // Top-p: a bound on the error, relative to the row's total mass, of the fp32 masses that
 // place the nucleus boundary (each weight: the exponent's rounding and the rounding of
 // log2(e)/T, ex2.approx, the per-vector fp32 sum; the tail below 2^-24 of the maximum holds
@@ -135,7 +138,7 @@ __host__ __device__ constexpr size_t stream_dyn_bytes(int mode) {
   return mode <= SM_SUMS ? size_t(Ring<SM_SUMS>::kBuf) * Ring<SM_SUMS>::kBufBytes
          : mode == SM_TOPK
              ? size_t(Ring<SM_TOPK>::kBuf) * Ring<SM_TOPK>::kBufBytes + size_t(kCapTopK) * 8 +
-                   size_t(kKeptCap) * 8
+                   size_t(kStreamMaxTopK) * 8
              : size_t(Ring<SM_TOPP>::kBuf) * Ring<SM_TOPP>::kBufBytes + size_t(kCap) * 8 +
                    size_t(kBins) * 4 + size_t(kBins) * 12;
 }
@@ -179,10 +182,11 @@ __device__ __forceinline__ Fx128* scr_fx(StreamAux& a) { return reinterpret_cast
 static_assert(offsetof(StreamAux, scr_s64) == offsetof(StreamAux, scr_u64) + 8 * kWarps,
               "scr_u64 and scr_s64 are adjacent");
 
-// Three top-k CTAs per SM: ring, list, ranked top k, this record and the 1 KB the hardware
-// reserves per CTA, within the SM's 228 KB.
-static_assert(3 * (stream_dyn_bytes(SM_TOPK) + sizeof(StreamAux) + 1024) <= 228 * 1024,
-              "three top-k CTAs per SM");
+// SV_TOPK_CTAS top-k CTAs per SM: ring, list, ranked top k, this record and the 1 KB the
+// hardware reserves per CTA, within the SM's 228 KB.
+static_assert(SV_TOPK_CTAS >= 2 && SV_TOPK_CTAS <= 3, "top-k CTAs per SM");
+static_assert(SV_TOPK_CTAS * (stream_dyn_bytes(SM_TOPK) + sizeof(StreamAux) + 1024) <= 228 * 1024,
+              "the top-k CTAs of an SM fit its shared memory");
 static_assert(2 * (stream_dyn_bytes(SM_TOPP) + sizeof(StreamAux) + 1024) <= 228 * 1024,
               "two top-p CTAs per SM");
 
@@ -393,7 +397,7 @@ struct CandSet {
   uint32_t* hcnt;              // [kBins] (top-p only)
   uint32_t* hlimb;             // [3][kBins]: bin masses as limbs; members and their weights
                                // reuse it (top-p only)
-  uint64_t* ranked;            // [kKeptCap]: the top k in rank order (top-k only)
+  uint64_t* ranked;            // [kStreamMaxTopK]: the top k in rank order (top-k only)
   StreamAux* aux;
 
   // Histogram of the candidates i < n with composite >= lim: counts, and (mass) the sum of
@@ -722,7 +726,8 @@ struct RowAcc {
 // ------------------------------------------------------------------ kernel
 // Greedy and plain-sum CTAs need no candidate list and fit three to an SM.
 template <typename T, int kMode>
-__global__ void __launch_bounds__(kStreamThreads, (kMode == SM_TOPP ? 2 : 3))
+__global__ void __launch_bounds__(kStreamThreads,
+                                  (kMode == SM_TOPP ? 2 : (kMode == SM_TOPK ? SV_TOPK_CTAS : 3)))
     stream_rows_kernel(const StreamJob job) {
   constexpr bool kCand = kMode == SM_TOPK || kMode == SM_TOPP;
   constexpr int kCapM = kMode == SM_TOPK ? kCapTopK : kCap;  // candidates per row
@@ -1110,11 +1115,11 @@ __global__ void __launch_bounds__(kStreamThreads, (kMode == SM_TOPP ? 2 : 3))
           if (!ok) {
             status = ROW_FALLBACK;
           } else {
-            // normaliser, entropy term and kept-id list over the kept candidates. Top-k rows
-            // list their kept ids (with top-p too: the nucleus within the top k), and the
-            // consumer sums the double normaliser over the list if it needs it; top-p rows
-            // are not listed and get it here.
-            const bool list = kMode == SM_TOPK && rj.kept_ids != nullptr;
+            // normaliser, entropy term and kept-id list over the kept candidates. Rows list
+            // their kept ids (a nucleus of more than kKeptCap entries is not listed); top-k
+            // rows leave the double normaliser to the consumer, which sums it over the list
+            // if it needs it, and top-p rows get it here.
+            const bool list = rj.kept_ids != nullptr;
             if (threadIdx.x == 0) aux.mcount = 0;
             csync();
             unsigned long long z = 0;
@@ -1145,7 +1150,8 @@ __global__ void __launch_bounds__(kStreamThreads, (kMode == SM_TOPP ? 2 : 3))
       }
       if (status == ROW_FALLBACK && threadIdx.x == 0)
         job.fb_rows[atomicAdd(job.fb_count, 1)] = int32_t(row);
-      if (rj.kept_n && threadIdx.x == 0) rj.kept_n[row] = listed ? min(aux.mcount, kKeptCap) : 0;
+      if (rj.kept_n && threadIdx.x == 0)
+        rj.kept_n[row] = (listed && aux.mcount <= kKeptCap) ? aux.mcount : 0;
       const double Z = double(zfx) * kFxInv;
       const double ent = (status == ROW_OK && kMode != SM_GREEDY && want_ent)
                              ? log(Z) - 0.6931471805599453 * S1 / Z

@@ -230,7 +230,8 @@ spec_status spec_verify_chain_lmhead(const void* target_hidden, const void* draf
  *   u_t = beta_t (v_t / gamma_t - sum_{s<t} (k_t . k_s) u_s). 1 <= S <= 32, dk <= 256. The
  *   values are divided by the cumulative gate, so gates far below 1 over many steps lose
  *   float32 precision.
- * spec_commit_linear_state: state [B][H][dk][dv] (device, 16-byte aligned) is replaced, in
+ * spec_commit_linear_state: state [B][H][dk][dv] (device; it, keys, w and u 16-byte aligned,
+ *   else SPEC_ERR_UNSUPPORTED) is replaced, in
  *   place, by the state after steps[b] steps (int32 [B], device):
  *   S_a = gamma_a (S_0 + sum_{t<=a} k_t (u_t - S_0^T w_t)^T). A sequence with steps[b] = 0,
  *   or outside [0, S], is left untouched (not read or written). dk in {32, 64, 128, 256},
@@ -252,7 +253,7 @@ spec_status spec_commit_linear_state(float* state, int B, int H, int dk, int dv,
  * SPEC_STATIC_SCRATCH_BYTES inside the library, one per device; the call allocates
  * nothing and looks the array's address up once per device (with that device current).
  *   - A call whose spec_workspace_size(B, K, V) exceeds SPEC_STATIC_SCRATCH_BYTES returns
- *     SPEC_ERR_WORKSPACE before any CUDA call (8 MiB holds about 7,700 logit rows,
+ *     SPEC_ERR_WORKSPACE before any CUDA call (32 MiB holds about 8,000 logit rows,
  *     B * (2K + 1)).
  *   - Every call on a device uses the same scratch: calls that overlap in time (on
  *     different streams, or from host threads without ordering) race on it and give
@@ -264,7 +265,7 @@ spec_status spec_commit_linear_state(float* state, int B, int H, int dk, int dv,
  *     device gets SPEC_ERR_INVALID_ARG before any launch.
  *   - spec_get_device_status cannot see this scratch: a row whose copy wait timed out
  *     shows as accepted_len[b] = -2. */
-#define SPEC_STATIC_SCRATCH_BYTES ((size_t)8 << 20)
+#define SPEC_STATIC_SCRATCH_BYTES ((size_t)32 << 20)
 spec_status spec_verify_chain_noalloc(const void* target_logits, const void* draft_logits,
                                       spec_dtype dtype, int B, int K, int V,
                                       const int32_t* draft_tokens, const float* uniforms,

@@ -32,11 +32,11 @@ def test_status_strings_and_kernel_counts(lib):
 
 def _ws(rows):
     up = lambda x: (x + 255) // 256 * 256
-    return 256 + up(48 * rows) + up(4 * rows) + up(rows * 256 * 4) + up(4 * rows) + up(4 * rows)
+    return 256 + up(48 * rows) + up(4 * rows) + up(rows * 1024 * 4) + up(4 * rows) + up(4 * rows)
 
 
 def test_workspace_size(lib):
-    """header, 32-byte row statistics, kept-id counts, up to 256 kept ids per row and the
+    """header, 32-byte row statistics, kept-id counts, up to 1024 kept ids per row and the
     list of rows the cluster kernel finishes"""
     assert sv.spec_workspace_size(0, 4, 10) == 0
     assert sv.spec_workspace_size(512, 8, 151936) == _ws(512 * 17)
@@ -144,6 +144,6 @@ def test_noalloc_limits_on_the_host(lib):
     args = lambda B, K, V: (P(16), P(16), 1, B, K, V, P(16), P(16), 1.0, 0, 1.0, P(16), P(16), None)
     assert lib.spec_verify_chain_noalloc(*args(0, 8, 151936)) == -1
     assert lib.spec_verify_chain_noalloc(*args(4, 0, 151936)) == -1
-    big = 1024  # 1024 * 17 rows need more than the 8 MiB scratch
-    assert sv.spec_workspace_size(big, 8, 151936) > 8 << 20
+    big = 1024  # 1024 * 17 rows need more than the 32 MiB scratch
+    assert sv.spec_workspace_size(big, 8, 151936) > 32 << 20
     assert lib.spec_verify_chain_noalloc(*args(big, 8, 151936)) == -4
