@@ -400,9 +400,9 @@ struct CandSet {
   uint64_t* ranked;            // [kStreamMaxTopK]: the top k in rank order (top-k only)
   StreamAux* aux;
 
-  // Histogram of the candidates i < n with composite >= lim: counts, and (mass) the sum of
-  // their fixed-point weights.
-  __device__ void hist_build(int n, uint64_t lim, float c, float mc, bool mass) {
+  // Histogram of the candidates i < n with composite >= lim over log-weight bins relative to
+  // mc: counts, and (mass) the sum of their fixed-point weights 2^(x c - wref).
+  __device__ void hist_build(int n, uint64_t lim, float c, float mc, bool mass, float wref) {
     for (int i = threadIdx.x; i < kBins; i += kThreads) hcnt[i] = 0;
     if (mass)
       for (int i = threadIdx.x; i < 3 * kBins; i += kThreads) hlimb[i] = 0;
@@ -422,7 +422,7 @@ struct CandSet {
       }
       hist_add(hcnt, b, ok);
       if (mass && ok) {
-        const unsigned long long w = to_fx(weight(x, c, mc));
+        const unsigned long long w = to_fx(weight(x, c, wref));
         limb_add(hlimb, kBins, b, w);
       }
     }
@@ -468,7 +468,7 @@ struct CandSet {
   // where the count (or mass) accumulated within the bin reaches need -> aux->sel_comp.
   // Returns false if the bin has more than kMemberCap members.
   __device__ bool resolve(int n, uint64_t lim, float c, float mc, bool mass,
-                          unsigned long long need) {
+                          unsigned long long need, float wref) {
     if (aux->sel_cnt > uint32_t(kMemberCap)) return false;  // uniform
     const int bsel = aux->sel_bin;
     uint64_t* mem = reinterpret_cast<uint64_t*>(hlimb);
@@ -486,7 +486,7 @@ struct CandSet {
       const int slot = atomicAdd(&aux->mcount, 1);
       if (slot < kMemberCap) {
         mem[slot] = e;
-        mw[slot] = mass ? to_fx(weight(x, c, mc)) : 1ull;
+        mw[slot] = mass ? to_fx(weight(x, c, wref)) : 1ull;
       }
     }
     csync();
@@ -510,7 +510,7 @@ struct CandSet {
   // where the count reaches keep; returns the new count and sets *thr to the smallest kept
   // value, so the list stays "every entry seen so far that is >= thr".
   __device__ int cut(int n, int keep, float c, float mc, float* thr) {
-    hist_build(n, 0, c, mc, false);
+    hist_build(n, 0, c, mc, false, mc);
     hist_find((unsigned long long)keep, false);
     const int bsel = aux->sel_found ? aux->sel_bin : kBins - 1;
     constexpr int kPer = kCap / kThreads;
@@ -614,12 +614,13 @@ struct RowAcc {
   static constexpr bool kSums = kMode == SM_SUMS || kMode == SM_TOPP;
   float mt;   // running maximum (NaN once a NaN was seen)
   int am;     // greedy: lowest index holding mt
-  float mct;  // fl(mt * c): the online sums are relative to it
+  float mct;  // the online sums are relative to it: fl(mt * c); top-p: ceil(fl(mt * c))
   float s, h; // online weight sum and entropy term (log2 units)
-  // top-p: the online weight sum as 42-bit fixed point. Each vector's eight weights are
-  // summed in fp32 and added exactly, and a new maximum rescales the sum in double by the
-  // exact power of two between the two references, so the sum's error stays within a few
-  // fp32 roundings per weight (the bound the top-p decision's guard relies on).
+  // top-p: the online weight sum as 42-bit fixed point, relative to the integer reference
+  // mct. Each vector's eight weights are summed in fp32 and added exactly; a reference that
+  // rises by d shifts the sum right by d bits (the exact power of two, truncated below
+  // 2^-42), so the sum's error stays within a few fp32 roundings per weight (the bound the
+  // top-p decision's guard relies on) with no floating-point rescale in the loop.
   unsigned long long sfx;
 
   __device__ void reset() {
@@ -635,7 +636,15 @@ struct RowAcc {
   __device__ __forceinline__ void raise_max(float vm, float c) {
     const float nm = vm * c;
     if constexpr (kMode == SM_TOPP) {
-      if (sfx) sfx = __double2ull_rn(double(sfx) * exp2(double(mct) - double(nm)));
+      const float nr = ceilf(nm);
+      if (sfx == 0ull) {
+        mct = nr;
+      } else if (nr > mct) {
+        const float d = nr - mct;
+        sfx = d < 64.0f ? sfx >> int(d) : 0ull;
+        mct = nr;
+      }
+      return;
     } else if (s != 0.0f || h != 0.0f) {
       const float d = nm - mct;  // > 0
       const float scale = ex2(-d);
@@ -1087,18 +1096,19 @@ __global__ void __launch_bounds__(kStreamThreads,
               }
               cstar = aux.sel_comp;
             }
-          } else {  // top-p over the whole row: the mass target from the online sums
-            const unsigned long long zt =
-                st.sfx ? __double2ull_rn(double(st.sfx) * exp2(double(st.mct) - double(mc)))
-                       : 0ull;
+          } else {  // top-p over the whole row: the mass target from the online sums,
+                    // relative to the row's integer reference rref = ceil(mc)
+            const float rref = ceilf(mc);
+            const float dsh = rref - st.mct;  // >= 0 for every thread with a sum
+            const unsigned long long zt = (st.sfx && dsh < 64.0f) ? st.sfx >> int(dsh) : 0ull;
             const unsigned long long zall = creduce<unsigned long long>(zt, aux.scr_u64, OpSum());
             unsigned long long target =
                 (unsigned long long)ceil(double(rj.top_p) * double(zall));
             if (target < 1) target = 1;
             if (ok) {
-              cs.hist_build(n, 0, c, mc, true);
+              cs.hist_build(n, 0, c, mc, true, rref);
               cs.hist_find(target, true);  // not found: the candidates hold too little mass
-              ok = aux.sel_found && cs.resolve(n, 0, c, mc, true, target - aux.sel_before);
+              ok = aux.sel_found && cs.resolve(n, 0, c, mc, true, target - aux.sel_before, rref);
               cstar = aux.sel_comp;
               if (ok && rj.refine_rows) {
                 // the fp32 masses before and through the crossing; within the guard of the
