@@ -197,6 +197,13 @@ __device__ __forceinline__ Fx128 fx_add(Fx128 a, Fx128 b) {
   r.hi = a.hi + b.hi + (r.lo < a.lo ? 1ull : 0ull);
   return r;
 }
+// a * n exactly (a < 2^28 * 2^100 / n, true of any row sum here).
+__device__ __forceinline__ Fx128 fx_mul_u32(Fx128 a, uint32_t n) {
+  Fx128 r;
+  r.lo = a.lo * n;
+  r.hi = a.hi * n + __umul64hi(a.lo, uint64_t(n));
+  return r;
+}
 __device__ __forceinline__ bool fx_is_zero(Fx128 a) { return (a.lo | a.hi) == 0ull; }
 // x in [0, 2^27): x * 2^100 truncated to an integer.
 __device__ __forceinline__ Fx128 fx_from(double x) {
@@ -221,7 +228,8 @@ __device__ __forceinline__ Fx128 fx_from(double x) {
   return r;
 }
 __device__ __forceinline__ double fx_to_double(Fx128 a) {
-  return ldexp(double(a.hi), -36) + ldexp(double(a.lo), -100);
+  // exact scalings by powers of two (both products are normal doubles)
+  return double(a.hi) * 0x1.0p-36 + double(a.lo) * 0x1.0p-100;
 }
 __device__ __forceinline__ Fx128 fx_shfl_xor(Fx128 a, int o) {
   return Fx128{__shfl_xor_sync(0xffffffffu, a.lo, o), __shfl_xor_sync(0xffffffffu, a.hi, o)};

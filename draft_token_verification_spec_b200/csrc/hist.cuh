@@ -20,14 +20,6 @@ constexpr int kHistCodes = 65536;                       // every bfloat16 code
 constexpr int kHistWords = kHistCodes / 2;              // two 16-bit counters per word
 constexpr size_t kHistBytes = size_t(kHistWords) * 4;   // 128 KB of shared memory
 
-// a * n exactly (a < 2^28 * 2^100 / n, true of any row sum here).
-__device__ __forceinline__ Fx128 fx_mul_u32(Fx128 a, uint32_t n) {
-  Fx128 r;
-  r.lo = a.lo * n;
-  r.hi = a.hi * n + __umul64hi(a.lo, uint64_t(n));
-  return r;
-}
-
 __device__ __forceinline__ void hist_clear(uint32_t* hist) {
   uint4* h4 = reinterpret_cast<uint4*>(hist);
   for (int i = threadIdx.x; i < kHistWords / 4; i += kThreads) h4[i] = make_uint4(0, 0, 0, 0);

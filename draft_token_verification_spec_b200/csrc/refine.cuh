@@ -3,24 +3,32 @@
 // rejection scheme; the nucleus is the shortest prefix in (probability desc, id asc) order
 // whose mass reaches top_p, the crossing token kept).
 //
-// The streaming kernel places the boundary with fp32 masses. Rows where that placement lies
-// within its error guard of the target, and rows the exact finisher settled, are listed;
-// here one thread block per listed row places the boundary again with double weights
-// exp((l - m) / T) summed exactly (Fx128):
+// Rows whose boundary was placed within the error bound of an fp32 sum (the streaming
+// kernel's sum of the entries below its threshold), and top-p rows the exact finisher
+// settled with fp32 masses, are listed; here the boundary is placed again exactly.
+//
+// bfloat16 rows, two kernels:
+//   - topp_zexact_kernel: the row's normaliser Z = sum of exp((l - m) / T) in double, summed
+//     exactly (Fx128) by kZSlices blocks per listed row, each over a slice, into the row's
+//     accumulator (128-bit atomic adds with carry, so the total does not depend on order);
+//   - topp_finalize_kernel: one block per listed row collects every entry within two log2
+//     units of weight of the listed boundary or above it (a histogram of their codes and
+//     their 32-bit composites, as the streaming kernel keeps them) and runs the same
+//     selection with the exact Z: the code where the mass from the top reaches top_p * Z,
+//     how many of its entries (in id order) are kept, their ids.
+// float32 rows, topp_refine_kernel, one block per listed row:
 //   - one pass over the row collects, as (key << 32 | ~id) composites, the entries of a
 //     window of three log-weight bins around the listed boundary's bin (the same fp32 bin
-//     function the streaming kernel used, so the classification is identical), notes the
-//     lightest entry above the window and the heaviest below it, and lists the ids above
-//     the window. It also gathers the total mass Z and the mass above the window: for
-//     bfloat16 rows through a histogram of the row's codes (each distinct code weighed once,
-//     hist.cuh), for float32 rows entry by entry;
+//     function the streaming kernel used), notes the lightest entry above the window and
+//     the heaviest below it, and lists the ids above the window. It also sums the total
+//     mass Z and the mass above the window entry by entry;
 //   - the window is sorted (bitonic, descending composite = descending probability, then
 //     ascending id) and scanned: the first entry whose cumulative mass reaches top_p * Z is
 //     the boundary. A crossing just outside the window is taken from the noted neighbours.
 // The row statistics get the new boundary and the double normaliser of the kept set, and
 // the row's kept-id list is rewritten for the new boundary (emptied when it does not fit).
-// A row whose window overflows, or whose crossing lies further out, keeps its fp32 boundary
-// and is counted in *unresolved.
+// A row whose crossing lies outside what was collected keeps its fp32 boundary and is
+// counted in *unresolved.
 #pragma once
 
 #include "draw.cuh"
@@ -38,11 +46,165 @@ struct RefineJob {
   int32_t* unresolved;      // rows left at their fp32 boundary (may be NULL)
 };
 
-// Dynamic shared memory: the window, then (bfloat16 rows) the code histogram: one block per
-// SM.
+// Dynamic shared memory of topp_refine_kernel: the window.
 template <typename T>
 __host__ __device__ constexpr size_t refine_smem() {
   return size_t(kRefineCap) * 8 + (sizeof(T) == 2 ? kHistBytes : 0);
+}
+
+constexpr int kZSlices = 16;  // blocks per listed row summing its exact normaliser
+
+// 128-bit atomic add with carry: concurrent adds of exact terms give the exact total.
+__device__ __forceinline__ void fx_atomic_add(unsigned long long* p, Fx128 a) {
+  const unsigned long long old = atomicAdd(p, a.lo);
+  const unsigned long long carry = (old + a.lo < old) ? 1ull : 0ull;
+  if (a.hi + carry) atomicAdd(p + 1, a.hi + carry);
+}
+
+template <typename T>
+__device__ __forceinline__ const T* refine_row_ptr(const RowJob& rj, long long row) {
+  return (row < rj.rows0) ? static_cast<const T*>(rj.base0) + size_t(row) * rj.V
+                          : static_cast<const T*>(rj.base1) + size_t(row - rj.rows0) * rj.V;
+}
+
+// Exact normalisers of the listed rows: work item (li, s) adds the Fx128 sum of exp((l - m)
+// / T) over slice s of listed row li to rj.refine_z[li] (zeroed when the row was listed).
+template <typename T>
+__global__ void __launch_bounds__(kThreads) topp_zexact_kernel(const RefineJob j) {
+  __shared__ Fx128 scr[kWarps];
+  const RowJob& rj = j.r;
+  const int V = rj.V;
+  const long long items = (long long)*j.count * kZSlices;
+  const int slice = ((V + kZSlices - 1) / kZSlices + 7) / 8 * 8;
+  const double iT = 1.0 / double(rj.temp);
+  for (long long it = blockIdx.x; it < items; it += gridDim.x) {
+    const long long li = it / kZSlices;
+    const int sl = int(it % kZSlices);
+    const long long row = j.rows[li];
+    const RowStats rs = rj.stats[row];
+    if (rs.status != ROW_OK) continue;  // uniform
+    const T* src = refine_row_ptr<T>(rj, row);
+    const bool al = (reinterpret_cast<uintptr_t>(src) & 15u) == 0;
+    const int v1 = min(V, (sl + 1) * slice);
+    Fx128 acc = fx_zero();
+    // four groups of 8 per thread in flight
+    for (int v00 = sl * slice + int(threadIdx.x) * 8; v00 < v1; v00 += 8 * kThreads * 4) {
+      float x[4][8];
+#pragma unroll
+      for (int g = 0; g < 4; ++g) load8<T>(src, v00 + g * kThreads * 8, v1, al, x[g]);
+#pragma unroll
+      for (int g = 0; g < 4; ++g)
+#pragma unroll
+        for (int k = 0; k < 8; ++k)
+          if (x[g][k] > -INFINITY) acc = fx_add(acc, fx_from(weight_d(x[g][k], rs.m, iT)));
+    }
+    acc = block_sum_fx(acc, scr);
+    if (threadIdx.x == 0) fx_atomic_add(rj.refine_z + 2 * li, acc);
+  }
+}
+
+// One block per listed bfloat16 row: the boundary again, from the exact normaliser.
+template <typename T>
+__global__ void __launch_bounds__(kThreads) topp_finalize_kernel(const RefineJob j) {
+  static_assert(sizeof(T) == 2, "bfloat16 rows");
+  __shared__ StreamAux aux;
+  __shared__ uint32_t plist[kCapP];
+  __shared__ uint32_t hcnt[kPBins];
+  __shared__ uint32_t pmem[kPMem];
+  CandSet<T> cs;
+  cs.cand = nullptr;
+  cs.ranked = nullptr;
+  cs.plist = plist;
+  cs.hcnt = hcnt;
+  cs.pmem = pmem;
+  cs.aux = &aux;
+  const RowJob& rj = j.r;
+  const int V = rj.V;
+  const long long nlist = *j.count;
+  const double iT = 1.0 / double(rj.temp);
+  for (long long li = blockIdx.x; li < nlist; li += gridDim.x) {
+    const long long row = j.rows[li];
+    const RowStats rs = rj.stats[row];
+    if (rs.status != ROW_OK) continue;  // uniform
+    const T* src = refine_row_ptr<T>(rj, row);
+    const bool al = (reinterpret_cast<uintptr_t>(src) & 15u) == 0;
+    const double zt = fx_to_double(Fx128{rj.refine_z[2 * li], rj.refine_z[2 * li + 1]});
+    // collect the codes from two log2 units of weight below the listed boundary up, in a
+    // window of kPBins codes that reaches the row maximum
+    const float xlo = key_value<T>(rs.thr_key) - 1.3862944f * rj.temp;
+    uint32_t base = Elem<T>::key(xlo);
+    const uint32_t kmax = Elem<T>::key(rs.m);
+    if (kmax > base + uint32_t(kPBins - 1)) base = kmax - uint32_t(kPBins - 1);
+    const float t = key_value<T>(base);
+    for (int i = threadIdx.x; i < kPBins; i += kThreads) hcnt[i] = 0u;
+    if (threadIdx.x == 0) aux.ccount = 0;
+    __syncthreads();
+    // eight groups of 8 per thread in flight
+    for (int v00 = int(threadIdx.x) * 8; v00 < V; v00 += 8 * kThreads * 8) {
+      float x[8][8];
+#pragma unroll
+      for (int g = 0; g < 8; ++g) load8<T>(src, v00 + g * kThreads * 8, V, al, x[g]);
+#pragma unroll
+      for (int g = 0; g < 8; ++g) {
+        const int v0 = v00 + g * kThreads * 8;
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          if (x[g][k] >= t && v0 + k < V) {
+            const uint32_t rel = Elem<T>::key(x[g][k]) - base;  // < kPBins: x <= the maximum
+            const int pos = atomicAdd(&aux.ccount, 1);
+            if (pos < kCapP) plist[pos] = pcomp(rel, v0 + k);
+            atomicAdd(&hcnt[rel], 1u);
+          }
+        }
+      }
+    }
+    __syncthreads();
+    const int nall = aux.ccount;
+    if (threadIdx.x < 32) {
+      uint32_t cst = 0u;
+      double zk = -1.0;
+      int stable = 0;
+      const bool found = nall <= kCapP && cs.p_select_warp(nall, base, 0, rs.m, iT, rj.top_p, 0.0,
+                                                           zt, 0.0, &cst, &zk, &stable);
+      if (threadIdx.x == 0) {
+        aux.sel_found = found ? 1 : 0;
+        aux.sel_c32 = cst;
+        aux.sel_above = zk;
+      }
+    }
+    __syncthreads();
+    const bool ok = aux.sel_found != 0;
+    const double zkept = aux.sel_above;
+    int32_t* kids = rj.kept_ids ? rj.kept_ids + size_t(row) * kKeptCap : nullptr;
+    if (!ok) {
+      // unresolved: the listed boundary stands, with its kept list
+      if (threadIdx.x == 0 && j.unresolved) atomicAdd(j.unresolved, 1);
+      __syncthreads();
+      continue;
+    }
+    const uint32_t cstar = aux.sel_c32;
+    if (threadIdx.x == 0) aux.mcount = 0;
+    __syncthreads();
+    unsigned long long z = 0;
+    for (int i = threadIdx.x; i < nall; i += kThreads) {
+      const uint32_t e = plist[i];
+      if (e < cstar) continue;
+      z += to_fx(weight(key_value<T>(base + pcomp_rel(e)), rs.c, rs.mc));
+      const int slot = atomicAdd(&aux.mcount, 1);
+      if (kids && slot < kKeptCap) kids[slot] = pcomp_id(e);
+    }
+    const unsigned long long zf = creduce<unsigned long long>(z, aux.scr_u64, OpSum());
+    if (threadIdx.x == 0) {
+      RowStats out = rs;
+      out.thr_key = base + pcomp_rel(cstar);
+      out.cutoff = pcomp_id(cstar);
+      out.zd = zkept;
+      out.z = float(double(zf) * kFxInv);
+      rj.stats[row] = out;
+      if (rj.kept_n) rj.kept_n[row] = (kids && aux.mcount <= kKeptCap) ? aux.mcount : 0;
+    }
+    __syncthreads();
+  }
 }
 
 __device__ __forceinline__ void bitonic_sort_desc(uint64_t* a, int n2) {

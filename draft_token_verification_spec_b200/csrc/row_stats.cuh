@@ -68,6 +68,7 @@ struct RowJob {
   const int32_t* row_count;
   int32_t* refine_rows;      // if set: top-p rows whose boundary is re-decided in double
   int32_t* refine_count;
+  unsigned long long* refine_z;  // [rows][2]: their exact normalisers (Fx128), zeroed on listing
 };
 
 struct __align__(16) RowAux {
@@ -840,8 +841,12 @@ __device__ void process_row(RowCtx<T>& ctx, const RowJob& job, long long row, bo
   }
   if (!listed && job.kept_n && rank == 0 && threadIdx.x == 0) job.kept_n[row] = 0;
   // a top-p boundary this kernel placed with fp32 masses: re-decided in double afterwards
-  if (status == ROW_OK && topp && !topk && job.refine_rows && rank == 0 && threadIdx.x == 0)
-    job.refine_rows[atomicAdd(job.refine_count, 1)] = int32_t(row);
+  if (status == ROW_OK && topp && !topk && job.refine_rows && rank == 0 && threadIdx.x == 0) {
+    const int li = atomicAdd(job.refine_count, 1);
+    job.refine_rows[li] = int32_t(row);
+    job.refine_z[2 * li] = 0ull;
+    job.refine_z[2 * li + 1] = 0ull;
+  }
 
   const double Z = double(zfx) * kFxInv;
   const double ent = (status == ROW_OK && !greedy && want_ent)

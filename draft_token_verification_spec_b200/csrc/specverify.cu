@@ -191,7 +191,9 @@ cudaError_t launch_stream(const sv::StreamJob& job, int mode, cudaStream_t s) {
   }
 }
 
-// Blocks of the top-p refinement: one per SM (each walks the listed rows).
+// The top-p refinement. bfloat16 rows: the exact normalisers (four blocks per SM over the
+// (row, slice) items), then one block per listed row (one per SM, each walking the list).
+// float32 rows: one block per SM, each walking the listed rows.
 template <typename T>
 cudaError_t launch_refine(const sv::RefineJob& j, cudaStream_t s) {
   static std::mutex mu;
@@ -211,13 +213,23 @@ cudaError_t launch_refine(const sv::RefineJob& j, cudaStream_t s) {
     std::lock_guard<std::mutex> lock(mu);
     sms_of[dev] = sms;
   }
-  const size_t dyn = sv::refine_smem<T>();
-  e = cudaFuncSetAttribute(sv::topp_refine_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           int(dyn));
-  if (e != cudaSuccess) return e;
   const long long g = j.r.rows < sms ? j.r.rows : sms;
-  sv::topp_refine_kernel<T><<<unsigned(g), kThreads, dyn, s>>>(j);
-  return cudaGetLastError();
+  if constexpr (sizeof(T) == 2) {
+    const long long items = j.r.rows * sv::kZSlices;
+    const long long gz = items < 4LL * sms ? items : 4LL * sms;
+    sv::topp_zexact_kernel<T><<<unsigned(gz), kThreads, 0, s>>>(j);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    sv::topp_finalize_kernel<T><<<unsigned(g), kThreads, 0, s>>>(j);
+    return cudaGetLastError();
+  } else {
+    const size_t dyn = sv::refine_smem<T>();
+    e = cudaFuncSetAttribute(sv::topp_refine_kernel<T>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, int(dyn));
+    if (e != cudaSuccess) return e;
+    sv::topp_refine_kernel<T><<<unsigned(g), kThreads, dyn, s>>>(j);
+    return cudaGetLastError();
+  }
 }
 
 // Row statistics for a verify call. The streaming kernel settles the rows it can; in the
@@ -228,14 +240,26 @@ cudaError_t launch_refine(const sv::RefineJob& j, cudaStream_t s) {
 // (refine_rows, when given).
 cudaError_t row_stage(spec_dtype dt, sv::RowJob rj, const RowPlan& pl, int32_t* fb_rows,
                       int32_t* fb_count, int32_t* refine_rows, int32_t* refine_count,
-                      int32_t* unresolved, cudaStream_t s) {
+                      unsigned long long* refine_z, int32_t* unresolved, cudaStream_t s) {
   const bool refine = refine_rows && rj.top_p < 1.0f && rj.top_k == 0 &&
                       !(rj.flags & sv::RS_GREEDY);
   rj.refine_rows = refine ? refine_rows : nullptr;
   rj.refine_count = refine ? refine_count : nullptr;
+  rj.refine_z = refine ? refine_z : nullptr;
   const int mode = stream_mode(rj);
-  if (mode == sv::SM_TOPK && rj.top_k > sv::kStreamMaxTopK)
-    return launch_row_stats_dt(dt, rj, pl, s);
+  sv::RefineJob rf = {};
+  rf.r = rj;
+  rf.rows = refine_rows;
+  rf.count = refine_count;
+  rf.unresolved = unresolved;
+  // top-k above the candidate path's limit, and float32 top-p rows: the cluster kernel
+  // settles every row (then the refinement, for top-p)
+  if ((mode == sv::SM_TOPK && rj.top_k > sv::kStreamMaxTopK) ||
+      (mode == sv::SM_TOPP && dt != SPEC_BF16)) {
+    cudaError_t e = launch_row_stats_dt(dt, rj, pl, s);
+    if (e != cudaSuccess || !refine) return e;
+    return dt == SPEC_BF16 ? launch_refine<__nv_bfloat16>(rf, s) : launch_refine<float>(rf, s);
+  }
   const int E = dt == SPEC_BF16 ? 2 : 4;
   sv::StreamJob sj = {};
   sj.r = rj;
@@ -254,11 +278,6 @@ cudaError_t row_stage(spec_dtype dt, sv::RowJob rj, const RowPlan& pl, int32_t* 
   fj.row_count = fb_count;
   e = launch_row_stats_dt(dt, fj, pl, s);
   if (e != cudaSuccess || !refine) return e;
-  sv::RefineJob rf = {};
-  rf.r = rj;
-  rf.rows = refine_rows;
-  rf.count = refine_count;
-  rf.unresolved = unresolved;
   return dt == SPEC_BF16 ? launch_refine<__nv_bfloat16>(rf, s) : launch_refine<float>(rf, s);
 }
 
@@ -269,11 +288,12 @@ bool dtype_ok(int dt) { return dt == SPEC_F32 || dt == SPEC_BF16; }
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 // Workspace: [header | RowStats per row | kept-id count per row | kept ids per row |
-// fallback row list | refinement row list]. Header words (int32): 0 the device status,
+// fallback row list | refinement row list | exact normalisers of refined rows (Fx128)].
+// Header words (int32): 0 the device status,
 // 1 the fallback count, 2 the tree row-list count, 3 the refinement count, 4 rows left
 // unrefined; the rest of the 256 bytes is unused.
 struct WsLayout {
-  size_t stats, kept_n, kept_ids, fb_rows, refine_rows, total;
+  size_t stats, kept_n, kept_ids, fb_rows, refine_rows, refine_z, total;
 };
 constexpr int kHeaderWords = 5;
 
@@ -286,7 +306,8 @@ WsLayout ws_layout(long long rows) {
   w.kept_ids = w.kept_n + up256(size_t(rows) * sizeof(int32_t));
   w.fb_rows = w.kept_ids + up256(size_t(rows) * sv::kKeptCap * sizeof(int32_t));
   w.refine_rows = w.fb_rows + up256(size_t(rows) * sizeof(int32_t));
-  w.total = w.refine_rows + up256(size_t(rows) * sizeof(int32_t));
+  w.refine_z = w.refine_rows + up256(size_t(rows) * sizeof(int32_t));
+  w.total = w.refine_z + up256(size_t(rows) * 2 * sizeof(unsigned long long));
   return w;
 }
 
@@ -350,7 +371,7 @@ spec_status verify_tree(const void* target_logits, spec_dtype dtype, int B, int 
   void* eva = g_ev_after.load();
   if (evb) cudaEventRecord(static_cast<cudaEvent_t>(evb), s);
   if (row_stage(dtype, rj, pl, reinterpret_cast<int32_t*>(ws + wl.fb_rows), dev_status + 1,
-                nullptr, nullptr, nullptr, s) != cudaSuccess)
+                nullptr, nullptr, nullptr, nullptr, s) != cudaSuccess)
     return SPEC_ERR_CUDA;
   if (eva) cudaEventRecord(static_cast<cudaEvent_t>(eva), s);
 
@@ -456,7 +477,8 @@ spec_status spec_verify_chain(const void* target_logits, const void* draft_logit
   void* eva = g_ev_after.load();
   if (evb) cudaEventRecord(static_cast<cudaEvent_t>(evb), s);
   if (row_stage(dtype, rj, pl, reinterpret_cast<int32_t*>(ws + wl.fb_rows), dev_status + 1,
-                reinterpret_cast<int32_t*>(ws + wl.refine_rows), dev_status + 3, dev_status + 4,
+                reinterpret_cast<int32_t*>(ws + wl.refine_rows), dev_status + 3,
+                reinterpret_cast<unsigned long long*>(ws + wl.refine_z), dev_status + 4,
                 s) != cudaSuccess)
     return SPEC_ERR_CUDA;
   if (eva) cudaEventRecord(static_cast<cudaEvent_t>(eva), s);
@@ -563,7 +585,8 @@ spec_status spec_verify_tree_sampling(const void* target_logits, const void* dra
   void* eva = g_ev_after.load();
   if (evb) cudaEventRecord(static_cast<cudaEvent_t>(evb), s);
   if (row_stage(dtype, rj, pl, reinterpret_cast<int32_t*>(ws + wl.fb_rows), dev_status + 1,
-                reinterpret_cast<int32_t*>(ws + wl.refine_rows), dev_status + 3, dev_status + 4,
+                reinterpret_cast<int32_t*>(ws + wl.refine_rows), dev_status + 3,
+                reinterpret_cast<unsigned long long*>(ws + wl.refine_z), dev_status + 4,
                 s) != cudaSuccess)
     return SPEC_ERR_CUDA;
   if (eva) cudaEventRecord(static_cast<cudaEvent_t>(eva), s);

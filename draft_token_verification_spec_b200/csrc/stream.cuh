@@ -17,9 +17,9 @@
 //   SM_TOPK    the running maximum, and appends the entries >= a threshold to the CTA's
 //              candidate list (warp-aggregated: one shared atomic per warp, then each lane
 //              writes only the set bits of its vectors' masks);
-//   SM_TOPP    the online sum and the candidate list.
-// Candidates are 64-bit composites (key << 32 | ~id): the order of composites is the order
-// (value desc, id asc) that top-k and top-p use, so the k-th candidate is unique.
+//   SM_TOPP    the online sum of the entries below the threshold and the candidate list.
+// Top-k candidates are 64-bit composites (key << 32 | ~id): the order of composites is the
+// order (value desc, id asc) that top-k and top-p use, so the k-th candidate is unique.
 //
 // Top-k: the first threshold is a value that k entries of the first chunk reach (per-warp
 // order statistics of per-thread maxima; of vector maxima for k > 128). After the first
@@ -31,26 +31,30 @@
 // a list that still outgrows kCapTopK sends the row to the exact finisher. The short list
 // keeps a top-k CTA small enough for three per SM.
 //
-// Top-p: the threshold starts at (first-chunk maximum - T ln(V / (1 - top_p))), below
-// which the whole row holds less than 1 - top_p of the mass, raised to the smallest of
-// the largest kChunk0Vecs vector maxima of the first chunk (so at most 8 x that many
-// entries pass) if that is higher. The warps exchange counts and the row maximum after the
-// first chunk and then every kXchgTopP chunks: the threshold follows the maximum, and the
-// list is cut by count when it is about to overflow or its projected size at the row end
-// exceeds the capacity, to the top max(kKeepFloor, kKeepTarget * seen / V) entries seen so
-// far (about kKeepTarget candidates at the row end for rows whose values do not drift
-// along the vocabulary).
+// Top-p (bfloat16 rows): the threshold starts at (first-chunk maximum - T ln(V / (1 -
+// top_p))), below which the whole row holds less than 1 - top_p of the mass, raised to the
+// smallest of the largest kChunk0Vecs vector maxima of the first chunk if that is higher,
+// and is always an exact bfloat16 value. A candidate is a 32-bit composite of its code
+// (relative to the row's base code, the code of the first threshold) and its id, and is
+// also counted in a histogram of codes. Candidates are left out of the online fp32 sums
+// (their weight is replaced by 0 before the exponentials), so the sums hold only the
+// entries below the threshold. The warps exchange counts and the row maximum after the
+// first chunk and then every kXchgTopP chunks: the threshold follows the maximum, and a list
+// about to overflow is cut to the codes holding its top max(kKeepFloor, kKeepTarget * seen /
+// V) entries (the histogram keeps the counts of the entries cut).
 //
 // At the end of a row the CTA selects among the candidates. Top-k lists are ranked directly
 // (each candidate counts the larger composites); with top-p as well, the top k go to their
-// rank slots and a block scan of their weights finds the crossing. Top-p lists go over a
-// histogram of log-weight bins (1/32 of a log2 unit each, relative to the row maximum; bins
-// only coarsen the order, they never reorder it): the bin where the mass crosses the
-// target, then the exact crossing candidate among that bin's members. It writes the
-// RowStats record (and the kept ids of top-k rows). Rows the candidates cannot settle (list
-// overflow, too many members in the crossing bin, or candidates holding less than top_p of
-// the mass) are marked ROW_FALLBACK and listed; the cluster kernel (row_stats.cuh) then
-// finishes them exactly.
+// rank slots and a block scan of their weights finds the crossing. Top-p rows weigh the
+// histogram's codes once each in double (exp((l - m) / T)); the total plus the fp32 sum of
+// the entries below the threshold gives the mass target, a suffix scan over the codes finds
+// the code where the mass crosses it and how many of its entries (in id order) are kept,
+// and the list gives their ids. Only the sum below the threshold carries fp32 error: a
+// crossing within its error bound of the target is listed for the exact placement
+// (refine.cuh). The CTA writes the RowStats record and the kept ids. Rows the candidates
+// cannot settle (list overflow, a code outside the histogram's window, a crossing among
+// entries cut from the list or below the threshold) are marked ROW_FALLBACK and listed; the
+// cluster kernel (row_stats.cuh) then finishes them.
 //
 // This is the sampling transform of "Speculative Sampling" (spec-decoding-i notes, last
 // bullet: transform the probabilities first, then apply the rejection scheme), the argmax
@@ -66,10 +70,10 @@
 
 namespace sv {
 
-// Ring of chunk buffers per CTA: two 32 KB chunks in every mode. Greedy, plain sums and
-// top-k run three CTAs per SM (top-k adds its list of kCapTopK candidates and the top k in
-// rank order, which just fits); top-p two (its larger list and the log-weight histogram
-// take the rest). The depth and chunk size of each kind are build-time knobs.
+// Ring of chunk buffers per CTA: two 32 KB chunks (24 KB for top-p). Every mode runs three
+// CTAs per SM: top-k adds its list of kCapTopK candidates and the top k in rank order,
+// top-p its list of 32-bit candidates, the code histogram and the crossing code's members.
+// The depth and chunk size of each kind are build-time knobs.
 #ifndef SV_RING_NBUF_PLAIN
 #define SV_RING_NBUF_PLAIN 2
 #endif
@@ -80,7 +84,7 @@ namespace sv {
 #define SV_RING_NBUF_CAND 2
 #endif
 #ifndef SV_RING_KB_CAND
-#define SV_RING_KB_CAND 32
+#define SV_RING_KB_CAND 24
 #endif
 #ifndef SV_RING_KB_TOPK
 #define SV_RING_KB_TOPK 32
@@ -114,35 +118,43 @@ __host__ __device__ constexpr int stream_chunk_bytes(int mode) {
 }
 
 constexpr int kStreamThreads = kThreads + 32;   // eight consumer warps + the producer
-constexpr int kCap = 4096;                      // top-p: candidates per row
 constexpr int kCapTopK = 1024;                  // top-k: candidates per row
+constexpr int kCapP = 4096;                     // top-p: candidates per row (32-bit)
+constexpr int kPBins = 1024;                    // top-p: codes of the histogram's window
+constexpr int kPMem = 256;                      // top-p: entries of the crossing code
 constexpr int kKeepFloor = 512;                 // top-p: a cut keeps at least this many
-constexpr int kKeepTarget = 3 * kCap / 8;       // top-p: candidates a cut aims at by row end
-constexpr int kXchgTopP = 4;                    // top-p: chunks between count exchanges
-constexpr int kChunk0Vecs = 384;                // top-p: vectors of the first chunk kept
+constexpr int kKeepTarget = 3 * kCapP / 8;      // top-p: candidates a cut aims at by row end
+constexpr int kXchgTopP = 5;                    // top-p: chunks between count exchanges
 constexpr int kBins = 1024;                     // log-weight bins
 constexpr float kBinScale = 32.0f;              // bins per log2 unit of weight
-constexpr int kMemberCap = 512;                 // members of the crossing bin
 constexpr int kRankMax = 1024;                  // lists this short are ranked directly
 constexpr int kStreamMaxTopK = 256;             // top-k the candidate path takes
-// Top-p: a bound on the error, relative to the row's total mass, of the fp32 masses that
-// place the nucleus boundary (each weight: the exponent's rounding and the rounding of
-// log2(e)/T, ex2.approx, the per-vector fp32 sum; the tail below 2^-24 of the maximum holds
-// at most V * 2^-24 of it). A boundary within it is re-decided in double precision.
-constexpr float kToppGuard = 6e-6f;
+// Top-p: a bound on the error of the fp32 sum of the entries below the threshold, relative
+// to that sum, in weights exp((l - m) / T) (max 1). Per entry of depth d = (m - l) log2(e) /
+// T log2 units: c = fl(log2(e) / T) is off by 3 * 2^-24 at most (d * 3 * 2^-24 in the
+// exponent), the exponent fl(l c - r) by 2^-24 of (d + 1), ex2.approx by 2^-22 relative,
+// and the per-vector fp32 sum by 4 * 2^-24; entries with d <= 32 are thus within
+// ln2 * 2^-24 * (4 * 32 + 1) + 2^-22 + 4 * 2^-24 = 5.9e-6 of their weight, and the rest (each
+// below 2^-32, at most 2^20 of them) are off by under 1.5e-9 in all. The fixed-point sums
+// add at most 2^-42 per vector and per reference shift (kPGuardFxUnit).
+constexpr double kPGuardRel = 6.0e-6;
+constexpr double kPGuardAbs = 2.0e-9;
+constexpr double kPGuardFxUnit = 2.2737367544323206e-13;  // 2^-42
 
 // Dynamic shared memory of one CTA: the ring, then top-k: the candidate list and the top k
-// in rank order; top-p: the candidate list, the bin counts and the bin masses as 15-bit
-// limbs (whose space the crossing bin's members reuse).
+// in rank order; top-p: the candidate list, the code histogram and the crossing code's
+// members.
 __host__ __device__ constexpr size_t stream_dyn_bytes(int mode) {
   return mode <= SM_SUMS ? size_t(Ring<SM_SUMS>::kBuf) * Ring<SM_SUMS>::kBufBytes
          : mode == SM_TOPK
              ? size_t(Ring<SM_TOPK>::kBuf) * Ring<SM_TOPK>::kBufBytes + size_t(kCapTopK) * 8 +
                    size_t(kStreamMaxTopK) * 8
-             : size_t(Ring<SM_TOPP>::kBuf) * Ring<SM_TOPP>::kBufBytes + size_t(kCap) * 8 +
-                   size_t(kBins) * 4 + size_t(kBins) * 12;
+             : size_t(Ring<SM_TOPP>::kBuf) * Ring<SM_TOPP>::kBufBytes + size_t(kCapP) * 4 +
+                   size_t(kPBins) * 4 + size_t(kPMem) * 4;
 }
-static_assert(2 * kMemberCap * 8 <= 3 * kBins * 4, "members and their weights fit the masses");
+// top-p: per warp, the vectors of the first chunk whose maxima set its threshold (1 in 16)
+constexpr int kChunk0WarpVecs = Ring<SM_TOPP>::kVec * 32 / 16;
+static_assert(kPBins % kThreads == 0, "whole histogram bins per consumer thread");
 static_assert(kCapTopK <= kRankMax, "every top-k list is ranked directly");
 static_assert(kStreamMaxTopK <= kThreads, "the top k in rank order: one per thread");
 
@@ -168,8 +180,12 @@ struct __align__(16) StreamAux {
   uint32_t scr_u32[kWarps];
   unsigned long long sel_before;
   unsigned long long sel_comp;
-  unsigned long long sel_mabove;  // resolve: mass of the crossing bin's members above it
-  unsigned long long sel_mw;      // resolve: the crossing member's own mass
+  double sel_above;  // top-p: mass of the codes above the crossing code
+  double sel_w;      // top-p: weight of the crossing code
+  int sel_j;         // top-p: entries of the crossing code kept
+  int sel_stable;    // top-p: the crossing lies outside the guard
+  uint32_t sel_c32;  // top-p: the crossing composite
+  int pover;         // top-p: a candidate's code fell outside the histogram's window
   uint32_t sel_cnt;
   int sel_bin;
   int sel_found;
@@ -183,12 +199,12 @@ static_assert(offsetof(StreamAux, scr_s64) == offsetof(StreamAux, scr_u64) + 8 *
               "scr_u64 and scr_s64 are adjacent");
 
 // SV_TOPK_CTAS top-k CTAs per SM: ring, list, ranked top k, this record and the 1 KB the
-// hardware reserves per CTA, within the SM's 228 KB.
+// hardware reserves per CTA, within the SM's 228 KB; likewise three top-p CTAs.
 static_assert(SV_TOPK_CTAS >= 2 && SV_TOPK_CTAS <= 3, "top-k CTAs per SM");
 static_assert(SV_TOPK_CTAS * (stream_dyn_bytes(SM_TOPK) + sizeof(StreamAux) + 1024) <= 228 * 1024,
               "the top-k CTAs of an SM fit its shared memory");
-static_assert(2 * (stream_dyn_bytes(SM_TOPP) + sizeof(StreamAux) + 1024) <= 228 * 1024,
-              "two top-p CTAs per SM");
+static_assert(3 * (stream_dyn_bytes(SM_TOPP) + sizeof(StreamAux) + 1024) <= 228 * 1024,
+              "three top-p CTAs per SM");
 
 // ------------------------------------------------------------------ consumer barriers
 // Named barrier 1 over the 256 consumer threads (the producer warp never joins it).
@@ -295,22 +311,11 @@ __device__ __forceinline__ Fx128 cscan_fx(Fx128 v, Fx128* scr, Fx128* total) {
 
 // The double-precision work at a row's end, kept out of line so that its registers do not
 // weigh on the streaming loop (the call is taken once per row): one entry's weight
-// exp((x - m) / T) as Fx128, and a thread's share of the kept candidates' weights.
+// exp((x - m) / T) as Fx128.
 template <typename T>
 __device__ __noinline__ Fx128 weight_fx(uint32_t key, float m, double iT) {
   return fx_from(weight_d(key_value<T>(key), m, iT));
 }
-template <typename T>
-__device__ __noinline__ Fx128 kept_weights_fx(const uint64_t* cand, int n, uint64_t cstar, float m,
-                                              double iT) {
-  Fx128 acc = fx_zero();
-  for (int i = threadIdx.x; i < n; i += kThreads) {
-    const uint64_t e = cand[i];
-    if (e >= cstar) acc = fx_add(acc, fx_from(weight_d(key_value<T>(uint32_t(e >> 32)), m, iT)));
-  }
-  return acc;
-}
-
 // Counts into hist[bin] with one shared atomic per distinct bin per warp; every lane of
 // the warp calls it.
 __device__ __forceinline__ void hist_add(uint32_t* hist, int bin, bool valid) {
@@ -391,55 +396,35 @@ __device__ __forceinline__ int bin_of(float x, float c, float mc) {
   return d < float(kBins - 1) ? max(0, int(d)) : kBins - 1;
 }
 
+// Top-p candidates: 32-bit composites (rel << 20) | (2^20 - 1 - id), rel = the entry's code
+// key minus the row's base key (rel < kPBins, id < 2^20): larger composite = larger value,
+// then lower id.
+__device__ __forceinline__ uint32_t pcomp(uint32_t rel, int id) {
+  return (rel << 20) | (0xFFFFFu - uint32_t(id));
+}
+__device__ __forceinline__ uint32_t pcomp_rel(uint32_t e) { return e >> 20; }
+__device__ __forceinline__ int pcomp_id(uint32_t e) { return int(0xFFFFFu - (e & 0xFFFFFu)); }
+
 template <typename T>
 struct CandSet {
-  uint64_t* cand;              // [kCap] (top-k: [kCapTopK])
-  uint32_t* hcnt;              // [kBins] (top-p only)
-  uint32_t* hlimb;             // [3][kBins]: bin masses as limbs; members and their weights
-                               // reuse it (top-p only)
-  uint64_t* ranked;            // [kStreamMaxTopK]: the top k in rank order (top-k only)
+  uint64_t* cand;              // top-k: [kCapTopK]
+  uint64_t* ranked;            // top-k: [kStreamMaxTopK], the top k in rank order
+  uint32_t* plist;             // top-p: [kCapP] candidates
+  uint32_t* hcnt;              // top-p: [kPBins] code histogram (first chunk: vector-maxima bins)
+  uint32_t* pmem;              // top-p: [kPMem] entries of the crossing code
   StreamAux* aux;
 
-  // Histogram of the candidates i < n with composite >= lim over log-weight bins relative to
-  // mc: counts, and (mass) the sum of their fixed-point weights 2^(x c - wref).
-  __device__ void hist_build(int n, uint64_t lim, float c, float mc, bool mass, float wref) {
-    for (int i = threadIdx.x; i < kBins; i += kThreads) hcnt[i] = 0;
-    if (mass)
-      for (int i = threadIdx.x; i < 3 * kBins; i += kThreads) hlimb[i] = 0;
-    csync();
-    for (int i0 = 0; i0 < n; i0 += kThreads) {
-      const int i = i0 + threadIdx.x;
-      bool ok = false;
-      int b = 0;
-      float x = 0.0f;
-      if (i < n) {
-        const uint64_t e = cand[i];
-        ok = e >= lim;
-        if (ok) {
-          x = key_value<T>(comp_key(e));
-          b = bin_of(x, c, mc);
-        }
-      }
-      hist_add(hcnt, b, ok);
-      if (mass && ok) {
-        const unsigned long long w = to_fx(weight(x, c, wref));
-        limb_add(hlimb, kBins, b, w);
-      }
-    }
-    csync();
-  }
-
-  // The bin where the count (or mass) accumulated from bin 0 first reaches need:
-  // aux->sel_found, sel_bin, sel_before (the count or mass of the bins before it) and
-  // sel_cnt (its count).
-  __device__ void hist_find(unsigned long long need, bool mass) {
+  // The bin of hcnt[0 .. kBins) where the count accumulated from bin 0 first reaches need:
+  // aux->sel_found, sel_bin, sel_before (the count of the bins before it) and sel_cnt (its
+  // count).
+  __device__ void hist_find(unsigned long long need) {
     constexpr int kPer = kBins / kThreads;
     unsigned long long part[kPer];
     unsigned long long tsum = 0;
 #pragma unroll
     for (int q = 0; q < kPer; ++q) {
       const int b = threadIdx.x * kPer + q;
-      part[q] = mass ? limb_get(hlimb, kBins, b) : (unsigned long long)hcnt[b];
+      part[q] = (unsigned long long)hcnt[b];
       tsum += part[q];
     }
     unsigned long long total;
@@ -464,82 +449,235 @@ struct CandSet {
     csync();
   }
 
-  // Among the members of bin aux->sel_bin (composite >= lim), in composite order, the one
-  // where the count (or mass) accumulated within the bin reaches need -> aux->sel_comp.
-  // Returns false if the bin has more than kMemberCap members.
-  __device__ bool resolve(int n, uint64_t lim, float c, float mc, bool mass,
-                          unsigned long long need, float wref) {
-    if (aux->sel_cnt > uint32_t(kMemberCap)) return false;  // uniform
-    const int bsel = aux->sel_bin;
-    uint64_t* mem = reinterpret_cast<uint64_t*>(hlimb);
-    unsigned long long* mw = reinterpret_cast<unsigned long long*>(hlimb) + kMemberCap;
-    if (threadIdx.x == 0) {
-      aux->mcount = 0;
-      aux->sel_comp = 0;
-    }
-    csync();
-    for (int i = threadIdx.x; i < n; i += kThreads) {
-      const uint64_t e = cand[i];
-      if (e < lim) continue;
-      const float x = key_value<T>(comp_key(e));
-      if (bin_of(x, c, mc) != bsel) continue;
-      const int slot = atomicAdd(&aux->mcount, 1);
-      if (slot < kMemberCap) {
-        mem[slot] = e;
-        mw[slot] = mass ? to_fx(weight(x, c, wref)) : 1ull;
-      }
-    }
-    csync();
-    const int m = min(aux->mcount, kMemberCap);
-    for (int i = threadIdx.x; i < m; i += kThreads) {
-      const uint64_t ei = mem[i];
-      unsigned long long above = 0;
-      for (int j = 0; j < m; ++j)
-        if (mem[j] > ei) above += mw[j];
-      if (above < need && need <= above + mw[i]) {
-        aux->sel_comp = ei;
-        aux->sel_mabove = above;
-        aux->sel_mw = mw[i];
-      }
-    }
-    csync();
-    return aux->sel_comp != 0;
-  }
-
-  // Cuts the list cand[0..n) to the candidates in the bins (relative to mc) up to the one
-  // where the count reaches keep; returns the new count and sets *thr to the smallest kept
-  // value, so the list stays "every entry seen so far that is >= thr".
-  __device__ int cut(int n, int keep, float c, float mc, float* thr) {
-    hist_build(n, 0, c, mc, false, mc);
-    hist_find((unsigned long long)keep, false);
-    const int bsel = aux->sel_found ? aux->sel_bin : kBins - 1;
-    constexpr int kPer = kCap / kThreads;
-    uint64_t v[kPer];
-    uint32_t keepm = 0;
-    uint32_t kmin = 0xFFFFFFFFu;
-    const int lo = threadIdx.x * kPer;
+  // Top-p cut: the highest code c >= *lfloor whose entries and those above number at least
+  // keep becomes the list's floor; the list plist[0..n) keeps the candidates of codes >= c
+  // (all of them: every entry of a code at or above the floor is listed), *thr becomes
+  // that code's value. The histogram keeps every count. Returns the new count. Thread t
+  // holds the codes kPBins - 1 - kPer t down to kPBins - kPer (t + 1).
+  __device__ int p_cut(int n, int keep, uint32_t base, int* lfloor, float* thr) {
+    constexpr int kPer = kPBins / kThreads;
+    const int top = kPBins - 1 - kPer * int(threadIdx.x);
+    uint32_t part[kPer];
+    uint32_t tsum = 0;
 #pragma unroll
     for (int q = 0; q < kPer; ++q) {
-      const int i = lo + q;
-      v[q] = i < n ? cand[i] : 0ull;
-      if (i < n) {
-        const uint32_t key = comp_key(v[q]);
-        if (bin_of(key_value<T>(key), c, mc) <= bsel) {
-          keepm |= 1u << q;
-          kmin = min(kmin, key);
+      const int bb = top - q;
+      part[q] = bb >= *lfloor ? hcnt[bb] : 0u;
+      tsum += part[q];
+    }
+    uint32_t total;
+    const uint32_t ex = cscan<uint32_t>(tsum, aux->scr_u32, &total);
+    if (threadIdx.x == 0) aux->sel_found = 0;
+    csync();
+    if (ex < uint32_t(keep) && uint32_t(keep) <= ex + tsum) {
+      uint32_t acc = ex;
+#pragma unroll
+      for (int q = 0; q < kPer; ++q) {
+        acc += part[q];
+        if (acc >= uint32_t(keep)) {
+          aux->sel_bin = top - q;
+          aux->sel_found = 1;
+          break;
         }
       }
     }
-    uint32_t total;
-    uint32_t pos = cscan<uint32_t>(uint32_t(__popc(keepm)), aux->scr_u32, &total);
-#pragma unroll
-    for (int q = 0; q < kPer; ++q)
-      if (keepm & (1u << q)) cand[pos++] = v[q];
-    const uint32_t kmin_all = creduce<uint32_t>(kmin, aux->scr_u32, OpMin());
-    if (threadIdx.x == 0) aux->ccount = int(total);
     csync();
-    *thr = fmaxf(*thr, key_value<T>(kmin_all));
-    return int(total);
+    if (!aux->sel_found) return n;  // uniform: the list holds fewer than keep
+    const int cf = aux->sel_bin;
+    constexpr int kPerL = kCapP / kThreads;
+    uint32_t v[kPerL];
+    uint32_t keepm = 0;
+    const int lo = threadIdx.x * kPerL;
+#pragma unroll
+    for (int q = 0; q < kPerL; ++q) {
+      const int i = lo + q;
+      v[q] = i < n ? plist[i] : 0u;
+      if (i < n && int(pcomp_rel(v[q])) >= cf) keepm |= 1u << q;
+    }
+    uint32_t kept;
+    uint32_t pos = cscan<uint32_t>(uint32_t(__popc(keepm)), aux->scr_u32, &kept);
+#pragma unroll
+    for (int q = 0; q < kPerL; ++q)
+      if (keepm & (1u << q)) plist[pos++] = v[q];
+    if (threadIdx.x == 0) aux->ccount = int(kept);
+    csync();
+    *lfloor = cf;
+    *thr = fmaxf(*thr, key_value<T>(base + uint32_t(cf)));
+    return int(kept);
+  }
+
+  // Top-p crossing over the code histogram's occupied bins 0..btop (relative to base), by
+  // one warp (all 32 lanes call it; no block barrier): the codes are weighed once each in
+  // double, exp((l - m) / T); Z is ztot if that is >= 0, else their total plus zrest. Lane L
+  // holds per = ceil((btop + 1) / 32) codes from btop - per L down. Returns the code where
+  // the mass accumulated from the top reaches top_p * Z (-1: none), with how many of its
+  // entries are kept (*j, in id order), the mass above it (*above), its weight (*w) and
+  // whether the crossing stays put when the target moves by guard either way (*stable).
+  __device__ int p_cross_warp(int btop, uint32_t base, float m, double iT, float top_p,
+                              double zrest, double ztot, double guard, int* j, double* above,
+                              double* w, int* stable) const {
+    const int lane = threadIdx.x & 31;
+    const int per = (btop + 32) / 32;
+    const int top = btop - per * lane;
+    Fx128 tsum = fx_zero();
+#pragma unroll 4
+    for (int q = 0; q < per; ++q) {
+      const int bb = top - q;
+      const uint32_t cnt = bb >= 0 ? hcnt[bb] : 0u;
+      if (cnt)
+        tsum = fx_add(tsum, fx_mul_u32(fx_from(weight_d(key_value<T>(base + uint32_t(bb)), m, iT)),
+                                       cnt));
+    }
+    Fx128 incl = tsum;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const Fx128 nb = fx_shfl_up(incl, o);
+      if (lane >= o) incl = fx_add(incl, nb);
+    }
+    const Fx128 zh{__shfl_sync(0xffffffffu, incl.lo, 31), __shfl_sync(0xffffffffu, incl.hi, 31)};
+    Fx128 ex = fx_shfl_up(incl, 1);
+    if (lane == 0) ex = fx_zero();
+    const double target = double(top_p) * (ztot >= 0.0 ? ztot : fx_to_double(zh) + zrest);
+    const unsigned hit = __ballot_sync(
+        0xffffffffu, fx_to_double(ex) < target && target <= fx_to_double(incl));
+    if (!hit) return -1;  // the histogram holds less than the target
+    const int cl = __ffs(hit) - 1;
+    int bsel = -1, jj = 0, stb = 0;
+    double ab = 0.0, wc = 0.0;
+    if (lane == cl) {
+      Fx128 acc = ex;
+      for (int q = 0; q < per; ++q) {
+        const int bb = top - q;
+        const uint32_t cnt = bb >= 0 ? hcnt[bb] : 0u;
+        if (!cnt) continue;
+        const double wq = weight_d(key_value<T>(base + uint32_t(bb)), m, iT);
+        const Fx128 nacc = fx_add(acc, fx_mul_u32(fx_from(wq), cnt));
+        const double a = fx_to_double(acc), t = fx_to_double(nacc);
+        if (a < target && target <= t) {
+          // the fewest entries of the code that reach the target
+          int k = int(ceil((target - a) / wq));
+          k = max(1, min(int(cnt), k));
+          while (k > 1 && a + double(k - 1) * wq >= target) --k;
+          while (k < int(cnt) && a + double(k) * wq < target) ++k;
+          bsel = bb;
+          jj = k;
+          ab = a;
+          wc = wq;
+          stb = (a + double(k - 1) * wq < target - guard && a + double(k) * wq >= target + guard)
+                    ? 1 : 0;
+          break;
+        }
+        acc = nacc;
+      }
+    }
+    *j = __shfl_sync(0xffffffffu, jj, cl);
+    *stable = __shfl_sync(0xffffffffu, stb, cl);
+    *above = __shfl_sync(0xffffffffu, ab, cl);
+    *w = __shfl_sync(0xffffffffu, wc, cl);
+    return __shfl_sync(0xffffffffu, bsel, cl);
+  }
+
+  // Top-p selection over the code histogram (bins >= 0 relative to base) and the list
+  // plist[0..n) (every entry of a code >= lfloor), by one warp (all 32 lanes call it; no
+  // block barrier). The codes are weighed once each in double, exp((l - m) / T); Z is ztot
+  // if that is >= 0, else their total plus zrest (the mass of the entries outside the
+  // histogram). Finds the code where the mass accumulated from the top reaches top_p * Z,
+  // how many of its entries it keeps (j, in id order), and the crossing composite among
+  // them (*cstar), with the kept mass (*zd) and whether the crossing stays put when the
+  // target moves by guard either way (*stable). False if it cannot be settled here (no
+  // crossing within the histogram, a crossing below lfloor, or more than kPMem entries of
+  // the crossing code). Lane L holds the codes kPBins - 1 - 32 L down to kPBins - 32 (L + 1).
+  __device__ bool p_select_warp(int n, uint32_t base, int lfloor, float m, double iT,
+                                float top_p, double zrest, double ztot, double guard,
+                                uint32_t* cstar, double* zd, int* stable) const {
+    constexpr int kPerL = kPBins / 32;
+    const int lane = threadIdx.x & 31;
+    const int top = kPBins - 1 - kPerL * lane;
+    Fx128 tsum = fx_zero();
+    for (int q = 0; q < kPerL; ++q) {
+      const uint32_t cnt = hcnt[top - q];
+      if (cnt)
+        tsum = fx_add(tsum, fx_mul_u32(fx_from(weight_d(key_value<T>(base + uint32_t(top - q)),
+                                                        m, iT)),
+                                       cnt));
+    }
+    Fx128 incl = tsum;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const Fx128 nb = fx_shfl_up(incl, o);
+      if (lane >= o) incl = fx_add(incl, nb);
+    }
+    const Fx128 zh{__shfl_sync(0xffffffffu, incl.lo, 31), __shfl_sync(0xffffffffu, incl.hi, 31)};
+    Fx128 ex = fx_shfl_up(incl, 1);
+    if (lane == 0) ex = fx_zero();
+    const double target = double(top_p) * (ztot >= 0.0 ? ztot : fx_to_double(zh) + zrest);
+    const unsigned hit = __ballot_sync(
+        0xffffffffu, fx_to_double(ex) < target && target <= fx_to_double(incl));
+    if (!hit) return false;  // the histogram holds less than the target
+    const int cl = __ffs(hit) - 1;
+    int bsel = -1, j = 0, stb = 0;
+    double above = 0.0, w = 0.0;
+    if (lane == cl) {
+      Fx128 acc = ex;
+      for (int q = 0; q < kPerL; ++q) {
+        const uint32_t cnt = hcnt[top - q];
+        if (!cnt) continue;
+        const double wq = weight_d(key_value<T>(base + uint32_t(top - q)), m, iT);
+        const Fx128 nacc = fx_add(acc, fx_mul_u32(fx_from(wq), cnt));
+        const double a = fx_to_double(acc), t = fx_to_double(nacc);
+        if (a < target && target <= t) {
+          // the fewest entries of the code that reach the target
+          int jj = int(ceil((target - a) / wq));
+          jj = max(1, min(int(cnt), jj));
+          while (jj > 1 && a + double(jj - 1) * wq >= target) --jj;
+          while (jj < int(cnt) && a + double(jj) * wq < target) ++jj;
+          bsel = top - q;
+          j = jj;
+          above = a;
+          w = wq;
+          stb = (a + double(jj - 1) * wq < target - guard && a + double(jj) * wq >= target + guard)
+                    ? 1 : 0;
+          break;
+        }
+        acc = nacc;
+      }
+    }
+    bsel = __shfl_sync(0xffffffffu, bsel, cl);
+    j = __shfl_sync(0xffffffffu, j, cl);
+    stb = __shfl_sync(0xffffffffu, stb, cl);
+    above = __shfl_sync(0xffffffffu, above, cl);
+    w = __shfl_sync(0xffffffffu, w, cl);
+    if (bsel < lfloor || hcnt[bsel] > uint32_t(kPMem)) return false;  // (bsel < 0 included)
+    // the entries of the crossing code, then the j-th largest of them (the j-th lowest id)
+    int nm = 0;
+    for (int i0 = 0; i0 < n; i0 += 32) {
+      const int i = i0 + lane;
+      const uint32_t e = i < n ? plist[i] : 0u;
+      const bool is = i < n && int(pcomp_rel(e)) == bsel;
+      const unsigned bal = __ballot_sync(0xffffffffu, is);
+      const int slot = nm + __popc(bal & ((1u << lane) - 1u));
+      if (is && slot < kPMem) pmem[slot] = e;
+      nm += __popc(bal);
+    }
+    nm = min(nm, kPMem);
+    __syncwarp();
+    uint32_t cst = 0u;
+    bool got = false;
+    for (int i = lane; i < nm; i += 32) {
+      const uint32_t e = pmem[i];
+      int ab = 0;
+      for (int q = 0; q < nm; ++q) ab += pmem[q] > e ? 1 : 0;
+      if (ab == j - 1) {
+        cst = e;
+        got = true;
+      }
+    }
+    const unsigned g = __ballot_sync(0xffffffffu, got);
+    if (!g) return false;
+    *cstar = __shfl_sync(0xffffffffu, cst, __ffs(g) - 1);
+    *zd = above + double(j) * w;
+    *stable = stb;
+    return true;
   }
 
   // Top-k lists: keeps the candidates of cand[0..n) (n <= kCapTopK) whose composite is
@@ -616,11 +754,12 @@ struct RowAcc {
   int am;     // greedy: lowest index holding mt
   float mct;  // the online sums are relative to it: fl(mt * c); top-p: ceil(fl(mt * c))
   float s, h; // online weight sum and entropy term (log2 units)
-  // top-p: the online weight sum as 42-bit fixed point, relative to the integer reference
-  // mct. Each vector's eight weights are summed in fp32 and added exactly; a reference that
-  // rises by d shifts the sum right by d bits (the exact power of two, truncated below
-  // 2^-42), so the sum's error stays within a few fp32 roundings per weight (the bound the
-  // top-p decision's guard relies on) with no floating-point rescale in the loop.
+  // top-p: the online weight sum of the entries below the candidate threshold as 42-bit
+  // fixed point, relative to the integer reference mct. Each vector's weights are summed in
+  // fp32 and added exactly; a reference that rises by d shifts the sum right by d bits (the
+  // exact power of two, truncated below 2^-42), so the sum's error stays within a few fp32
+  // roundings per weight (the bound kPGuardRel states) with no floating-point rescale in the
+  // loop.
   unsigned long long sfx;
 
   __device__ void reset() {
@@ -666,16 +805,15 @@ struct RowAcc {
   }
 
   // One 16-byte vector whose first element has row index j0 (entries outside the chunk
-  // hold -inf). vm = its largest value. Top-p: returns the mask of its entries >= t, from
-  // the values the sums unpacked (0 in the other modes).
+  // hold -inf). vm = its largest value. Top-p: returns the mask of its entries >= t (the
+  // candidates, bit k for entry k), which the sums leave out; 0 in the other modes.
   __device__ __forceinline__ uint32_t vec(const uint4& w, float vm, int j0, float c,
                                           bool want_ent, float t) {
     constexpr int P = Elem<T>::kPerVec;
-    uint32_t cm = 0;
+    uint32_t cm = 0u;
     if (!(vm > -INFINITY)) {  // all -inf (weight 0), or a NaN
       mt = fmax_nan(mt, vm);
-      if (kMode == SM_TOPP && vm >= t) cm = (1u << P) - 1u;  // all -inf, and t = -inf
-      return cm;
+      return (kMode == SM_TOPP && vm >= t) ? (1u << P) - 1u : 0u;  // all -inf, t = -inf
     }
     if constexpr (kMode == SM_GREEDY) {
       if (vm > mt) {  // later vectors hold higher indices: strict > keeps the lowest
@@ -688,8 +826,32 @@ struct RowAcc {
     } else if constexpr (kSums) {
       if (vm > mt) raise_max(vm, c);
       float x[P];
-      Elem<T>::unpack(w, x);
-      if (kMode == SM_TOPP) {
+      if constexpr (kMode == SM_TOPP) {
+        // candidates become -inf (weight 0) in the copy the sums read
+        uint4 ws = w;
+        if (vm >= t) {
+          if constexpr (sizeof(T) == 2) {
+            const __nv_bfloat162 tt = __float2bfloat162_rn(t);  // t is a bfloat16 value
+            uint32_t a[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              const uint32_t mk = __hge2_mask(Elem<T>::pair(a[i]), tt);
+              a[i] = (a[i] & ~mk) | (mk & 0xFF80FF80u);
+              cm |= ((mk & 1u) | ((mk >> 15) & 2u)) << (2 * i);  // entries 2i, 2i + 1
+            }
+            ws = make_uint4(a[0], a[1], a[2], a[3]);
+          } else {
+            uint32_t a[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+              if (__uint_as_float(a[i]) >= t) {
+                a[i] = 0xFF800000u;
+                cm |= 1u << i;
+              }
+            ws = make_uint4(a[0], a[1], a[2], a[3]);
+          }
+        }
+        Elem<T>::unpack(ws, x);
         float s1 = 0.0f, s2 = 0.0f;
 #pragma unroll
         for (int k = 0; k < P; k += 2) {
@@ -698,9 +860,11 @@ struct RowAcc {
         }
         sfx += to_fx(s1 + s2);
       } else if (want_ent) {
+        Elem<T>::unpack(w, x);
 #pragma unroll
         for (int k = 0; k < P; ++k) add(x[k], c, true);
       } else {
+        Elem<T>::unpack(w, x);
         float s2 = 0.0f;
 #pragma unroll
         for (int k = 0; k < P; k += 2) {
@@ -709,23 +873,19 @@ struct RowAcc {
         }
         s += s2;
       }
-      if (kMode == SM_TOPP && vm >= t) {
-#pragma unroll
-        for (int k = 0; k < P; ++k)
-          if (x[k] >= t) cm |= 1u << k;
-      }
     }
     mt = fmax_nan(mt, vm);
     return cm;
   }
 
-  // One element outside the vector path (chunk head or tail), row index j.
-  __device__ __forceinline__ void scalar(float x, int j, float c, bool want_ent) {
+  // One element outside the vector path (chunk head or tail), row index j; top-p sums
+  // only the entries that are not candidates (sum).
+  __device__ __forceinline__ void scalar(float x, int j, float c, bool want_ent, bool sum) {
     if constexpr (kMode == SM_GREEDY) {
       if (x > mt || (x == mt && j < am)) am = j;
     } else if constexpr (kSums) {
       if (x > mt) raise_max(x, c);
-      add(x, c, want_ent);
+      if (sum) add(x, c, want_ent);
     }
     mt = fmax_nan(mt, x);
   }
@@ -735,11 +895,10 @@ struct RowAcc {
 // ------------------------------------------------------------------ kernel
 // Greedy and plain-sum CTAs need no candidate list and fit three to an SM.
 template <typename T, int kMode>
-__global__ void __launch_bounds__(kStreamThreads,
-                                  (kMode == SM_TOPP ? 2 : (kMode == SM_TOPK ? SV_TOPK_CTAS : 3)))
+__global__ void __launch_bounds__(kStreamThreads, (kMode == SM_TOPK ? SV_TOPK_CTAS : 3))
     stream_rows_kernel(const StreamJob job) {
   constexpr bool kCand = kMode == SM_TOPK || kMode == SM_TOPP;
-  constexpr int kCapM = kMode == SM_TOPK ? kCapTopK : kCap;  // candidates per row
+  constexpr int kCapM = kMode == SM_TOPK ? kCapTopK : kCapP;  // candidates per row
   constexpr int E = Elem<T>::kBytes, P = Elem<T>::kPerVec;
   using RG = Ring<kMode>;
   constexpr int kRing = RG::kBuf, kRingBufBytes = RG::kBufBytes, kVecPerThread = RG::kVec;
@@ -766,6 +925,7 @@ __global__ void __launch_bounds__(kStreamThreads,
     }
     aux.broken = 0;
     aux.ccount = 0;
+    aux.pover = 0;
   }
   __syncthreads();
 
@@ -810,20 +970,26 @@ __global__ void __launch_bounds__(kStreamThreads,
   const float c = rj.c;
   const double iT = rj.temp > 0.0f ? 1.0 / double(rj.temp) : 0.0;
   CandSet<T> cs;
-  cs.cand = reinterpret_cast<uint64_t*>(smem + size_t(kRing) * kRingBufBytes);
+  unsigned char* const cand_area = smem + size_t(kRing) * kRingBufBytes;
   if (kMode == SM_TOPK) {
+    cs.cand = reinterpret_cast<uint64_t*>(cand_area);
     cs.ranked = cs.cand + kCapTopK;
+    cs.plist = nullptr;
     cs.hcnt = nullptr;
-    cs.hlimb = nullptr;
+    cs.pmem = nullptr;
   } else {
+    cs.cand = nullptr;
     cs.ranked = nullptr;
-    cs.hcnt = reinterpret_cast<uint32_t*>(cs.cand + kCap);
-    cs.hlimb = cs.hcnt + kBins;
+    cs.plist = reinterpret_cast<uint32_t*>(cand_area);
+    cs.hcnt = cs.plist + kCapP;
+    cs.pmem = cs.hcnt + kPBins;
   }
   cs.aux = &aux;
   RowAcc<T, kMode> st;
   st.reset();
   float thr = -INFINITY;  // candidates: every entry seen this row that is >= thr (uniform)
+  uint32_t pbase = 0;     // top-p: the key of the row's histogram bin 0 (uniform)
+  int lfloor = 0;         // top-p: every entry of a code >= pbase + lfloor is listed (uniform)
   int cnt = 0;            // candidates appended this row (uniform)
   bool overflow = false;  // (uniform)
   bool row_timeout = false;
@@ -843,22 +1009,24 @@ __global__ void __launch_bounds__(kStreamThreads,
     const uint4* vb = reinterpret_cast<const uint4*>(ring + size_t(b) * kRingBufBytes);
     const int base = q * job.chunk;
     const int v_lo = (s.pad + s.head) >> 4, v_hi = (s.pad + s.head + s.mid) >> 4;
-    // the chunk's vectors of this thread; top-k keeps only their maxima in registers and
-    // reads a vector again from the ring in the rare case that it holds a candidate (the
-    // buffer is released after the appends)
+    // the chunk's vectors of this thread; the candidate modes keep only their maxima in
+    // registers and read a vector again from the ring when they need it (top-k: in the rare
+    // case that it holds a candidate; top-p: for the sums; the buffer is released after the
+    // appends)
+    constexpr bool kReload = kMode == SM_TOPK || kMode == SM_TOPP;
     auto load_vec = [&](int v) {
       return (copied && v >= v_lo && v < v_hi) ? vb[v] : neg_inf_vec<T>();
     };
-    uint4 w[kMode == SM_TOPK ? 1 : kVecPerThread];
+    uint4 w[kReload ? 1 : kVecPerThread];
     float vm[kVecPerThread];
 #pragma unroll
     for (int u = 0; u < kVecPerThread; ++u) {
       const uint4 wu = load_vec(u * kThreads + int(threadIdx.x));
       vm[u] = Elem<T>::vmax_nan(wu);
-      if constexpr (kMode != SM_TOPK) w[u] = wu;
+      if constexpr (!kReload) w[u] = wu;
     }
     auto vec_at = [&](int u) -> uint4 {
-      if constexpr (kMode == SM_TOPK) return load_vec(u * kThreads + int(threadIdx.x));
+      if constexpr (kReload) return load_vec(u * kThreads + int(threadIdx.x));
       else return w[u];
     };
     // elements outside the bulk-copied middle (< 16 bytes at each end): thread 0 takes the
@@ -891,33 +1059,51 @@ __global__ void __launch_bounds__(kStreamThreads,
           }
           thr = creduce<float>(key_value<T>(kw), aux.scr_f, OpMin());
         } else {
-          const float m0 = creduce<float>(pm, aux.scr_f, OpMaxNan());
+          // top-p: each warp takes the maximum of its share of the chunk and a value that
+          // kChunk0WarpVecs of its vector maxima reach; one exchange combines them (the
+          // smallest such value: every warp has that many vectors at or above it)
+          float wm0 = pm;
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1) wm0 = fmax_nan(wm0, __shfl_xor_sync(0xffffffffu, wm0, o));
+          uint32_t kv[kVecPerThread];
+#pragma unroll
+          for (int u = 0; u < kVecPerThread; ++u) {
+            const int v = u * kThreads + int(threadIdx.x);
+            kv[u] = (v >= v_lo && v < v_hi && vm[u] == vm[u]) ? Elem<T>::key(vm[u]) : 0u;
+          }
+          const uint32_t kw =
+              warp_kth_key_n<Elem<T>::kKeyBits, kVecPerThread>(kv, kChunk0WarpVecs);
+          for (int i = threadIdx.x; i < kPBins; i += kThreads) cs.hcnt[i] = 0;  // starts empty
+          if (lane == 0) {
+            aux.red_f[xpar][warp] = wm0;
+            aux.red_i[xpar][warp] = int(kw);
+          }
+          csync();
+          float m0 = aux.red_f[xpar][0];
+          uint32_t kmin = uint32_t(aux.red_i[xpar][0]);
+#pragma unroll
+          for (int ww = 1; ww < kWarps; ++ww) {
+            m0 = fmax_nan(m0, aux.red_f[xpar][ww]);
+            kmin = min(kmin, uint32_t(aux.red_i[xpar][ww]));
+          }
+          xpar ^= 1;
           float t0 = m0 - job.topp_span;
           if (m0 > -INFINITY && m0 < INFINITY) {
-            // the vectors whose maxima fall in the bins up to the one where kChunk0Vecs of
-            // them are reached; the smallest such maximum bounds what this chunk appends
-            const float mc0 = m0 * c;
-            for (int i = threadIdx.x; i < kBins; i += kThreads) cs.hcnt[i] = 0;
-            csync();
-#pragma unroll
-            for (int u = 0; u < kVecPerThread; ++u) {
-              const int v = u * kThreads + int(threadIdx.x);
-              const bool ok = v >= v_lo && v < v_hi && vm[u] > -INFINITY;
-              hist_add(cs.hcnt, ok ? bin_of(vm[u], c, mc0) : 0, ok);
-            }
-            csync();
-            cs.hist_find((unsigned long long)kChunk0Vecs, false);
-            const int bsel = aux.sel_found ? aux.sel_bin : kBins - 1;
-            float tv = INFINITY;
-#pragma unroll
-            for (int u = 0; u < kVecPerThread; ++u) {
-              const int v = u * kThreads + int(threadIdx.x);
-              if (v >= v_lo && v < v_hi && vm[u] > -INFINITY && bin_of(vm[u], c, mc0) <= bsel)
-                tv = fminf(tv, vm[u]);
-            }
-            tv = creduce<float>(tv, aux.scr_f, OpMin());
-            if (tv < INFINITY) t0 = fmaxf(t0, tv);
+            t0 = fmaxf(t0, key_value<T>(kmin));
+            // the window of kPBins codes starts at the threshold's code, and at most
+            // kPBins - 256 codes below the first chunk's maximum
+            uint32_t kb = Elem<T>::key(t0);
+            const uint32_t ktop = Elem<T>::key(m0) + 256u;
+            if (ktop > kb + uint32_t(kPBins - 1)) kb = ktop - uint32_t(kPBins - 1);
+            pbase = kb;
+            t0 = key_value<T>(kb);  // an exact value: entries of code >= kb are candidates
+          } else {
+            // an empty first chunk (-inf: every entry is appended, the list overflows and
+            // the cluster kernel finishes the row) or a NaN (invalid: nothing is appended)
+            if (!(m0 == m0)) t0 = INFINITY;
+            pbase = Elem<T>::key(t0);
           }
+          lfloor = 0;
           thr = t0;
         }
       }
@@ -934,7 +1120,9 @@ __global__ void __launch_bounds__(kStreamThreads,
                      (v >= v_lo && v < v_hi) ? thr : INFINITY);
       vmax4 = fmaxf(vmax4, vm[u]);  // pad vectors hold -inf; NaN never passes a filter
     }
+    int wadd = 0;  // entries this warp appended in this chunk (uniform in the warp)
     if constexpr (kMode == SM_TOPK) {
+      // the candidates' bits, from the ring again (most vectors hold none)
       if (vmax4 >= thr) {
 #pragma unroll
         for (int u = 0; u < kVecPerThread; ++u) {
@@ -948,9 +1136,6 @@ __global__ void __launch_bounds__(kStreamThreads,
           }
         }
       }
-    }
-    int wadd = 0;  // entries this warp appended in this chunk (uniform in the warp)
-    if constexpr (kCand) {
       int my = 0;
 #pragma unroll
       for (int u = 0; u < kVecPerThread; ++u) my += __popc(cm[u]);
@@ -977,14 +1162,87 @@ __global__ void __launch_bounds__(kStreamThreads,
           }
         }
       }
+    } else if constexpr (kMode == SM_TOPP) {
+      // the candidates' bits from the sums pass, 8 per vector slot u (bit 8 (u % 4) + k of
+      // mb[u / 4])
+      static_assert(kVecPerThread <= 8, "two words of candidate bits per thread");
+      uint32_t mb[2] = {0u, 0u};
+#pragma unroll
+      for (int u = 0; u < kVecPerThread; ++u) mb[u >> 2] |= cm[u] << (8 * (u & 3));
+      // warp-cooperative appends: the warp's candidates in (lane, slot, element) order,
+      // one per lane per round, each lane reading its entry from the ring
+      const int my = __popc(mb[0]) + __popc(mb[1]);
+      int inc = my;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int t = __shfl_up_sync(0xffffffffu, inc, o);
+        if (lane >= o) inc += t;
+      }
+      wadd = __shfl_sync(0xffffffffu, inc, 31);
+      if (wadd) {
+        int wbase = 0;
+        if (lane == 31) wbase = atomicAdd(&aux.ccount, wadd);
+        wbase = __shfl_sync(0xffffffffu, wbase, 31);
+        const unsigned char* rb = ring + size_t(b) * kRingBufBytes;
+        for (int j0 = 0; j0 < wadd; j0 += 32) {
+          const int j = j0 + lane;
+          // the lane holding candidate j: the number of lanes whose inclusive count is <= j
+          int src = 0;
+#pragma unroll
+          for (int st = 16; st > 0; st >>= 1) {
+            const int c_in = __shfl_sync(0xffffffffu, inc, src + st - 1);
+            if (c_in <= j) src += st;
+          }
+          src = min(src, 31);
+          const int ex_s = __shfl_sync(0xffffffffu, inc - my, src);
+          const uint32_t m0s = __shfl_sync(0xffffffffu, mb[0], src);
+          const uint32_t m1s = __shfl_sync(0xffffffffu, mb[1], src);
+          if (j < wadd) {
+            int r = j - ex_s;  // its rank among that lane's candidates
+            const int c0 = __popc(m0s);
+            const int word = r < c0 ? 0 : 1;
+            if (word) r -= c0;
+            const int bit = int(__fns(word ? m1s : m0s, 0u, r + 1));
+            const int u = 4 * word + (bit >> 3), k = bit & 7;
+            const int v = u * kThreads + warp * 32 + src;
+            uint32_t key;
+            if constexpr (E == 2) {
+              const uint32_t h = *reinterpret_cast<const unsigned short*>(rb + 16 * v + 2 * k);
+              key = Elem<T>::key(__uint_as_float(h << 16));
+            } else {
+              key = Elem<T>::key(*reinterpret_cast<const float*>(rb + 16 * v + 4 * k));
+            }
+            const int id = base + (16 * v - s.pad) / E + k;
+            const int pos = wbase + j;
+            const uint32_t rel = key - pbase;
+            if (rel < uint32_t(kPBins)) {
+              if (pos < kCapM) cs.plist[pos] = pcomp(rel, id);
+              atomicAdd(&cs.hcnt[rel], 1u);
+            } else {
+              aux.pover = 1;
+            }
+          }
+        }
+      }
     }
     if (edge) {
       for (int j = e_lo; j < e_hi; ++j) {
         const float x = Elem<T>::load(s.g, j);
-        st.scalar(x, base + j, c, want_ent);
-        if (kCand && x >= thr) {
+        const bool is_cand = kCand && x >= thr;
+        st.scalar(x, base + j, c, want_ent, !is_cand);
+        if (is_cand) {
           const int pos = atomicAdd(&aux.ccount, 1);
-          if (pos < kCapM) cs.cand[pos] = make_comp(Elem<T>::key(x), base + j);
+          if constexpr (kMode == SM_TOPK) {
+            if (pos < kCapM) cs.cand[pos] = make_comp(Elem<T>::key(x), base + j);
+          } else {
+            const uint32_t rel = Elem<T>::key(x) - pbase;
+            if (rel < uint32_t(kPBins)) {
+              if (pos < kCapM) cs.plist[pos] = pcomp(rel, base + j);
+              atomicAdd(&cs.hcnt[rel], 1u);
+            } else {
+              aux.pover = 1;
+            }
+          }
           ++single;  // entries this thread appended one by one (edge elements)
         }
       }
@@ -997,7 +1255,7 @@ __global__ void __launch_bounds__(kStreamThreads,
       wacc += wadd;
       ++wlen;
       if ((kMode == SM_TOPP && wlen == kXchgTopP && q != nchunk - 1) ||
-          (kMode == SM_TOPK && wlen == xchg_k && q != nchunk - 1) || q == 0) {
+          (kMode == SM_TOPK && ((wlen == xchg_k && q != nchunk - 1) || q == 0))) {
         // exchange: the row maximum so far and the entries appended since the last one
         float wm = st.mt;
 #pragma unroll
@@ -1017,7 +1275,11 @@ __global__ void __launch_bounds__(kStreamThreads,
         }
         xpar ^= 1;
         cnt += added;
-        if (kMode == SM_TOPP) thr = fmaxf(thr, mrow - job.topp_span);
+        if (kMode == SM_TOPP) {
+          // the threshold follows the maximum, as an exact value (the code at or below it)
+          const float tn = mrow - job.topp_span;
+          if (tn > thr) thr = key_value<T>(Elem<T>::key(tn));
+        }
         const int rem = nchunk - 1 - q;  // chunks of this row still to come
         if (cnt > kCapM) {
           overflow = true;
@@ -1041,8 +1303,8 @@ __global__ void __launch_bounds__(kStreamThreads,
               thr = fmaxf(thr, key_value<T>(comp_key(kth)));
               if (cnt > kCapTopK / 2) cnt = cs.compact_ge(cnt, kth);
             }
-          } else if (keep < cnt && mrow > -INFINITY && mrow < INFINITY) {
-            cnt = cs.cut(cnt, keep, c, mrow * c, &thr);
+          } else if (keep < cnt) {
+            cnt = cs.p_cut(cnt, keep, pbase, &lfloor, &thr);
           }
         }
         wacc = 0;
@@ -1051,7 +1313,189 @@ __global__ void __launch_bounds__(kStreamThreads,
       }
     }
 
-    if (q == nchunk - 1) {
+    if (kMode == SM_TOPP && q == nchunk - 1) {
+      // ---------------------------------------------------------------- top-p row end
+      // one exchange: per warp the timeout flag, the maximum and the sum below the
+      // threshold, relative to the warp's integer reference ceil(fl(max * c))
+      float wmx = st.mt;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) wmx = fmax_nan(wmx, __shfl_xor_sync(0xffffffffu, wmx, o));
+      const float wref = ceilf(wmx * c);
+      const float dsw = wref - st.mct;  // >= 0 for every thread with a sum
+      unsigned long long zw = (st.sfx && dsw < 64.0f) ? st.sfx >> int(dsw) : 0ull;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) zw += __shfl_xor_sync(0xffffffffu, zw, o);
+      const bool wtmo = __any_sync(0xffffffffu, row_timeout);
+      if (lane == 0) {
+        aux.red_f[xpar][warp] = wmx;
+        aux.red_i[xpar][warp] = wtmo ? 1 : 0;
+        aux.scr_u64[warp] = zw;
+      }
+      csync();
+      const int nall = aux.ccount;  // every append of the row is done
+      float m = aux.red_f[xpar][0];
+      bool tmo = aux.red_i[xpar][0] != 0;
+#pragma unroll
+      for (int ww = 1; ww < kWarps; ++ww) {
+        m = fmax_nan(m, aux.red_f[xpar][ww]);
+        tmo = tmo || aux.red_i[xpar][ww] != 0;
+      }
+      int status = tmo ? ROW_TIMEOUT
+                       : ((m != m || m == INFINITY || m == -INFINITY) ? ROW_INVALID : ROW_OK);
+      const float mc = m * c;
+      // the sum of the entries below the threshold, relative to the row's integer reference
+      // rref = ceil(mc), then in weights exp((l - m) / T)
+      const float rref = ceilf(mc);
+      unsigned long long zb = 0ull;
+#pragma unroll
+      for (int ww = 0; ww < kWarps; ++ww) {
+        const float d = rref - ceilf(aux.red_f[xpar][ww] * c);
+        const unsigned long long z = aux.scr_u64[ww];
+        zb += (z && d < 64.0f) ? z >> int(d) : 0ull;
+      }
+      const double fxw = kFxInv * exp2(double(rref) - double(m) * double(c));
+      const double sbelow = double(zb) * fxw;
+      // its error bound: the weights' fp32 error, the fixed-point roundings (one per
+      // vector, per reference shift and per warp's and thread's final shift)
+      const double guard = kPGuardRel * sbelow + kPGuardAbs +
+                           (double(rj.V) / 8.0 + 66.0 * kThreads) * kPGuardFxUnit * (fxw / kFxInv);
+      const int n = min(nall, kCapM);
+      const bool go = status == ROW_OK && !overflow && nall <= kCapM && !aux.pover;
+      // warp 0: the crossing code over the histogram's occupied bins
+      if (warp == 0) {
+        int j = 0, stable = 0, bsel = -1;
+        double above = 0.0, wc = 0.0;
+        if (go) {
+          const int km = int(Elem<T>::key(m)) - int(pbase);
+          if (km >= 0)
+            bsel = cs.p_cross_warp(min(km, kPBins - 1), pbase, m, iT, rj.top_p, sbelow, -1.0,
+                                   double(rj.top_p) * guard, &j, &above, &wc, &stable);
+          // a crossing below the list's floor, or with too many entries at its code
+          if (bsel < lfloor || cs.hcnt[bsel >= 0 ? bsel : 0] > uint32_t(kPMem)) bsel = -1;
+        }
+        if (lane == 0) {
+          aux.sel_bin = bsel;
+          aux.sel_j = j;
+          aux.sel_stable = stable;
+          aux.sel_above = above + double(j) * wc;  // the kept mass
+          aux.mcount = 0;  // kept ids listed
+          aux.sel_cnt = 0u;  // entries of the crossing code gathered
+        }
+      }
+      csync();
+      const int bsel = aux.sel_bin;
+      if (status == ROW_OK && bsel < 0) status = ROW_FALLBACK;
+      const bool ok = status == ROW_OK;
+      const bool list = ok && rj.kept_ids != nullptr;
+      // the fp32 normaliser, entropy term and kept-id list: every warp takes the entries of
+      // the codes above the crossing code and gathers those of the crossing code; then warp
+      // 0 keeps the j of them with the lowest ids
+      unsigned long long z = 0;
+      long long s1 = 0;
+      auto keep = [&](uint32_t e) {
+        const float xv = key_value<T>(pbase + pcomp_rel(e));
+        const float zx = wexp(xv, c, mc);
+        const float ex = ex2(zx);
+        z += to_fx(ex);
+        if (want_ent) s1 += __float2ll_rn(ent_term(ex, zx) * kS1Fx);
+        if (list) {
+          const int slot = atomicAdd(&aux.mcount, 1);
+          if (slot < kKeptCap) rj.kept_ids[size_t(row) * kKeptCap + slot] = pcomp_id(e);
+        }
+      };
+      if (ok) {
+        for (int i = threadIdx.x; i < n; i += kThreads) {
+          const uint32_t e = cs.plist[i];
+          const int r = int(pcomp_rel(e));
+          if (r > bsel) {
+            keep(e);
+          } else if (r == bsel) {
+            const uint32_t slot = atomicAdd(&aux.sel_cnt, 1u);
+            if (slot < uint32_t(kPMem)) cs.pmem[slot] = e;
+          }
+        }
+      }
+      csync();
+      if (ok && warp == 0) {
+        const int nm = min(int(aux.sel_cnt), kPMem);
+        const int j = aux.sel_j;
+        uint32_t cst = 0u;
+        bool got = false;
+        for (int i = lane; i < nm; i += 32) {
+          const uint32_t e = cs.pmem[i];
+          int ab = 0;
+          for (int q = 0; q < nm; ++q) ab += cs.pmem[q] > e ? 1 : 0;
+          if (ab < j) keep(e);  // one of the j largest composites: the j lowest ids
+          if (ab == j - 1) {
+            cst = e;
+            got = true;
+          }
+        }
+        const unsigned g = __ballot_sync(0xffffffffu, got);
+        if (lane == 0) aux.sel_c32 = g ? 0u : 1u;  // (1: not found)
+        if (g && lane == __ffs(g) - 1) aux.sel_comp = cst;
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        z += __shfl_xor_sync(0xffffffffu, z, o);
+        s1 += __shfl_xor_sync(0xffffffffu, s1, o);
+      }
+      if (lane == 0) {
+        aux.scr_u64[warp] = z;
+        aux.scr_s64[warp] = s1;
+      }
+      csync();
+      const uint32_t cstar = uint32_t(aux.sel_comp);
+      if (ok && aux.sel_c32 != 0u) status = ROW_FALLBACK;
+      if (threadIdx.x == 0) {
+        unsigned long long zfx = 0;
+        long long s1a = 0;
+#pragma unroll
+        for (int ww = 0; ww < kWarps; ++ww) {
+          zfx += aux.scr_u64[ww];
+          s1a += aux.scr_s64[ww];
+        }
+        if (tmo && rj.dev_status) atomicOr(rj.dev_status, 1);
+        const bool settled = status == ROW_OK;
+        if (settled && !aux.sel_stable && rj.refine_rows) {
+          const int li = atomicAdd(rj.refine_count, 1);
+          rj.refine_rows[li] = int32_t(row);
+          rj.refine_z[2 * li] = 0ull;  // the exact normaliser's accumulator
+          rj.refine_z[2 * li + 1] = 0ull;
+        }
+        if (status == ROW_FALLBACK) job.fb_rows[atomicAdd(job.fb_count, 1)] = int32_t(row);
+        if (rj.kept_n)
+          rj.kept_n[row] = (settled && list && aux.mcount <= kKeptCap) ? aux.mcount : 0;
+        const double Z = double(zfx) * kFxInv;
+        const double S1 = double(s1a) / double(kS1Fx);
+        if (rj.stats) {
+          RowStats rs;
+          rs.mc = mc;
+          rs.z = float(Z);
+          rs.entropy = (settled && want_ent) ? float(log(Z) - 0.6931471805599453 * S1 / Z) : 0.0f;
+          rs.thr_key = settled ? pbase + pcomp_rel(cstar) : 0u;
+          rs.cutoff = settled ? pcomp_id(cstar) : INT_MAX;
+          rs.argmax = -1;
+          rs.status = status;
+          rs.c = c;
+          rs.m = m;
+          rs.pad = 0;
+          rs.zd = settled ? aux.sel_above : -1.0;
+          rj.stats[row] = rs;
+        }
+        // the next row starts clean (its first exchange orders this before its appends)
+        aux.ccount = 0;
+        aux.pover = 0;
+      }
+      st.reset();
+      thr = -INFINITY;
+      cnt = 0;
+      wacc = 0;
+      single = 0;
+      wlen = 0;
+      overflow = false;
+      row_timeout = false;
+    } else if (q == nchunk - 1) {
       // ---------------------------------------------------------------- row end
       const bool tmo = csync_or(row_timeout);
       const int nall = aux.ccount;  // every append of the row is done (candidate modes)
@@ -1081,61 +1525,29 @@ __global__ void __launch_bounds__(kStreamThreads,
           zfx = creduce<unsigned long long>(to_fx(sc), aux.scr_u64, OpSum());
           S1 = creduce<double>(double(hc), aux.scr_f64, OpSum());
         }
-      } else {
+      } else if constexpr (kMode == SM_TOPK) {
         if (status == ROW_OK) {
           const int n = min(nall, kCapM);
-          bool ok = !overflow && nall <= kCapM;
+          bool ok = !overflow && nall <= kCapM && n >= rj.top_k;
           uint64_t cstar = 0;
-          if constexpr (kMode == SM_TOPK) {
-            ok = ok && n >= rj.top_k;
-            if (ok) {  // every list is short (kCapTopK <= kRankMax): rank directly
-              if (rj.top_p < 1.0f) {  // the top-p crossing within the top k
-                ok = cs.rank_topp(n, rj.top_k, rj.top_p, m, iT);
-              } else {
-                ok = cs.rank_select(n, 0, rj.top_k);
-              }
-              cstar = aux.sel_comp;
+          if (ok) {  // every list is short (kCapTopK <= kRankMax): rank directly
+            if (rj.top_p < 1.0f) {  // the top-p crossing within the top k
+              ok = cs.rank_topp(n, rj.top_k, rj.top_p, m, iT);
+            } else {
+              ok = cs.rank_select(n, 0, rj.top_k);
             }
-          } else {  // top-p over the whole row: the mass target from the online sums,
-                    // relative to the row's integer reference rref = ceil(mc)
-            const float rref = ceilf(mc);
-            const float dsh = rref - st.mct;  // >= 0 for every thread with a sum
-            const unsigned long long zt = (st.sfx && dsh < 64.0f) ? st.sfx >> int(dsh) : 0ull;
-            const unsigned long long zall = creduce<unsigned long long>(zt, aux.scr_u64, OpSum());
-            unsigned long long target =
-                (unsigned long long)ceil(double(rj.top_p) * double(zall));
-            if (target < 1) target = 1;
-            if (ok) {
-              cs.hist_build(n, 0, c, mc, true, rref);
-              cs.hist_find(target, true);  // not found: the candidates hold too little mass
-              ok = aux.sel_found && cs.resolve(n, 0, c, mc, true, target - aux.sel_before, rref);
-              cstar = aux.sel_comp;
-              if (ok && rj.refine_rows) {
-                // the fp32 masses before and through the crossing; within the guard of the
-                // target the decision goes to the double-precision refinement
-                const unsigned long long before = aux.sel_before + aux.sel_mabove;
-                const unsigned long long through = before + aux.sel_mw;
-                const unsigned long long g =
-                    (unsigned long long)ceil(double(kToppGuard) * double(zall)) + 1ull;
-                if ((target - before <= g || through - target <= g) && threadIdx.x == 0)
-                  rj.refine_rows[atomicAdd(rj.refine_count, 1)] = int32_t(row);
-              }
-            }
+            cstar = aux.sel_comp;
           }
           if (!ok) {
             status = ROW_FALLBACK;
           } else {
-            // normaliser, entropy term and kept-id list over the kept candidates. Rows list
-            // their kept ids (a nucleus of more than kKeptCap entries is not listed); top-k
-            // rows leave the double normaliser to the consumer, which sums it over the list
-            // if it needs it, and top-p rows get it here.
+            // normaliser, entropy term and kept-id list over the kept candidates; the double
+            // normaliser is left to the consumer, which sums it over the list if it needs it
             const bool list = rj.kept_ids != nullptr;
             if (threadIdx.x == 0) aux.mcount = 0;
             csync();
             unsigned long long z = 0;
             long long s1 = 0;
-            Fx128 zdx = fx_zero();
-            if constexpr (kMode == SM_TOPP) zdx = kept_weights_fx<T>(cs.cand, n, cstar, m, iT);
             for (int i = threadIdx.x; i < n; i += kThreads) {
               const uint64_t e = cs.cand[i];
               if (e < cstar) continue;
@@ -1149,7 +1561,6 @@ __global__ void __launch_bounds__(kStreamThreads,
                 if (slot < kKeptCap) rj.kept_ids[size_t(row) * kKeptCap + slot] = comp_id(e);
               }
             }
-            if constexpr (kMode == SM_TOPP) zd = fx_to_double(creduce_fx(zdx, scr_fx(aux)));
             zfx = creduce<unsigned long long>(z, aux.scr_u64, OpSum());
             S1 = double(creduce<long long>(s1, aux.scr_s64, OpSum())) / double(kS1Fx);
             thr_key = comp_key(cstar);
@@ -1191,7 +1602,10 @@ __global__ void __launch_bounds__(kStreamThreads,
       overflow = false;
       row_timeout = false;
       if constexpr (kCand) {
-        if (threadIdx.x == 0) aux.ccount = 0;
+        if (threadIdx.x == 0) {
+          aux.ccount = 0;
+          aux.pover = 0;
+        }
         csync();
       }
     }
