@@ -21,7 +21,7 @@
 namespace sv {
 
 constexpr int kMaxDrawChunks = 128;
-constexpr int kSparsePer = 4;                           // support entries per thread
+constexpr int kSparsePer = 8;                           // support entries per thread
 constexpr int kSparseCap = kSparsePer * kThreads;       // support of a sparse draw
 
 struct DrawSmem {
@@ -219,6 +219,30 @@ __device__ __forceinline__ void load8(const T* row, int v0, int V, bool aligned,
   }
 }
 
+// G groups of 8 entries at v0, v0 + stride, ..., v0 + (G - 1) stride (-inf past V). When
+// every group lies inside an aligned row the G vector loads are issued together, ahead of
+// any use, so that their latencies overlap; otherwise group by group.
+template <typename T, int G>
+__device__ __forceinline__ void load8xG(const T* row, int v0, int stride, int V, bool aligned,
+                                        float (&x)[G][8]) {
+  constexpr int P = Elem<T>::kPerVec;
+  if (aligned && v0 + (G - 1) * stride + 8 <= V) {
+    uint4 w[G][8 / P];
+#pragma unroll
+    for (int g = 0; g < G; ++g)
+#pragma unroll
+      for (int q = 0; q < 8 / P; ++q)
+        w[g][q] = __ldg(reinterpret_cast<const uint4*>(row + v0 + g * stride) + q);
+#pragma unroll
+    for (int g = 0; g < G; ++g)
+#pragma unroll
+      for (int q = 0; q < 8 / P; ++q) Elem<T>::unpack(w[g][q], x[g] + q * P);
+  } else {
+#pragma unroll
+    for (int g = 0; g < G; ++g) load8<T>(row, v0 + g * stride, V, aligned, x[g]);
+  }
+}
+
 // Probability of entry v under the transformed distribution described by s (fp32).
 template <typename T>
 __device__ __forceinline__ float prob(const RowStats& s, float l, int v) {
@@ -251,11 +275,14 @@ static __device__ const double kExp2J[64] = {
 // 15(2), 1989): x = (64 k + j) ln2 / 64 + r with |r| <= ln2 / 128 (ln2 / 64 split into a
 // 32-bit head and a tail, so n * head is exact), e^x = 2^k 2^(j/64) e^r, and e^r by its
 // Taylor series to r^5 (the remainder is below 4e-17 of it). Relative error within a few
-// units in the last place; x below -745 (and -inf) gives 0.
+// units in the last place; x below -745 (and -inf) gives 0. Branch-free, so that the
+// compiler can overlap independent evaluations: 2^k is applied as two exact power-of-two
+// factors (each a normal double), so a subnormal result is rounded once, as by ldexp.
 __device__ __forceinline__ double exp_neg(double x) {
-  if (!(x > -745.0)) return 0.0;
-  const double n = rint(x * 92.33248261689366);  // 64 / ln2
-  double r = fma(-n, 0x1.62e42fee00000p-7, x);
+  const bool zero = !(x > -745.0);  // also -inf and NaN
+  const double xs = zero ? 0.0 : x;
+  const double n = rint(xs * 92.33248261689366);  // 64 / ln2
+  double r = fma(-n, 0x1.62e42fee00000p-7, xs);
   r = fma(-n, 0x1.a39ef35793c76p-39, r);
   const int ni = int(n);
   double p = fma(r, 1.0 / 120.0, 1.0 / 24.0);
@@ -264,9 +291,11 @@ __device__ __forceinline__ double exp_neg(double x) {
   p = fma(p, r, 1.0);
   p = fma(p, r, 1.0);
   const double t = __ldg(&kExp2J[ni & 63]) * p;
-  const int k = ni >> 6;  // floor(n / 64)
-  if (k >= -1022) return t * __longlong_as_double((long long)(k + 1023) << 52);
-  return ldexp(t, k);
+  const int k = ni >> 6;  // floor(n / 64), in [-1075, 0]
+  const int k1 = k >> 1, k2 = k - k1;
+  const double res = t * __longlong_as_double((long long)(k1 + 1023) << 52) *
+                     __longlong_as_double((long long)(k2 + 1023) << 52);
+  return zero ? 0.0 : res;
 }
 
 // Unnormalised weight exp((l - m) / T) of a kept entry, in double (l - m is exact); iT = 1 / T.
@@ -304,16 +333,16 @@ __device__ double row_zd(const RowStats& s, const T* row, int V, double iT, Fx12
   }
   const bool al = (reinterpret_cast<uintptr_t>(row) & 15u) == 0;
   Fx128 acc = fx_zero();
-  // two groups of 8 per iteration, both loaded before either is used
-  for (int v0 = int(threadIdx.x) * 8; v0 < V; v0 += 2 * kThreads * 8) {
-    float x[8], y[8];
-    const int v1 = v0 + kThreads * 8;
-    load8<T>(row, v0, V, al, x);
-    load8<T>(row, v1, V, al, y);
+  // four groups of 8 per iteration, all loaded before any is used
+  for (int v00 = int(threadIdx.x) * 8; v00 < V; v00 += 4 * kThreads * 8) {
+    float x[4][8];
+    load8xG<T, 4>(row, v00, kThreads * 8, V, al, x);
 #pragma unroll
-    for (int k = 0; k < 8; ++k) {
-      if (v0 + k < V) acc = fx_add(acc, fx_from(kept_weight_d<T>(s, iT, x[k], v0 + k)));
-      if (v1 + k < V) acc = fx_add(acc, fx_from(kept_weight_d<T>(s, iT, y[k], v1 + k)));
+    for (int g = 0; g < 4; ++g) {
+      const int v0 = v00 + g * kThreads * 8;
+#pragma unroll
+      for (int k = 0; k < 8; ++k)
+        if (v0 + k < V) acc = fx_add(acc, fx_from(kept_weight_d<T>(s, iT, x[g][k], v0 + k)));
     }
   }
   return fx_to_double(block_sum_fx(acc, scr));

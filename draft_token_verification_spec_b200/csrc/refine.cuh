@@ -52,7 +52,7 @@ __host__ __device__ constexpr size_t refine_smem() {
   return size_t(kRefineCap) * 8 + (sizeof(T) == 2 ? kHistBytes : 0);
 }
 
-constexpr int kZSlices = 16;  // blocks per listed row summing its exact normaliser
+constexpr int kZSlices = 64;  // blocks per listed row summing its exact normaliser
 
 // 128-bit atomic add with carry: concurrent adds of exact terms give the exact total.
 __device__ __forceinline__ void fx_atomic_add(unsigned long long* p, Fx128 a) {
@@ -90,8 +90,7 @@ __global__ void __launch_bounds__(kThreads) topp_zexact_kernel(const RefineJob j
     // four groups of 8 per thread in flight
     for (int v00 = sl * slice + int(threadIdx.x) * 8; v00 < v1; v00 += 8 * kThreads * 4) {
       float x[4][8];
-#pragma unroll
-      for (int g = 0; g < 4; ++g) load8<T>(src, v00 + g * kThreads * 8, v1, al, x[g]);
+      load8xG<T, 4>(src, v00, kThreads * 8, v1, al, x);
 #pragma unroll
       for (int g = 0; g < 4; ++g)
 #pragma unroll
@@ -103,14 +102,17 @@ __global__ void __launch_bounds__(kThreads) topp_zexact_kernel(const RefineJob j
   }
 }
 
-// One block per listed bfloat16 row: the boundary again, from the exact normaliser.
+// One block of kFinThreads per listed bfloat16 row: the boundary again, from the exact
+// normaliser.
+constexpr int kFinThreads = 1024;
 template <typename T>
-__global__ void __launch_bounds__(kThreads) topp_finalize_kernel(const RefineJob j) {
+__global__ void __launch_bounds__(kFinThreads) topp_finalize_kernel(const RefineJob j) {
   static_assert(sizeof(T) == 2, "bfloat16 rows");
   __shared__ StreamAux aux;
   __shared__ uint32_t plist[kCapP];
   __shared__ uint32_t hcnt[kPBins];
   __shared__ uint32_t pmem[kPMem];
+  __shared__ unsigned long long zred[kFinThreads / 32];
   CandSet<T> cs;
   cs.cand = nullptr;
   cs.ranked = nullptr;
@@ -122,6 +124,7 @@ __global__ void __launch_bounds__(kThreads) topp_finalize_kernel(const RefineJob
   const int V = rj.V;
   const long long nlist = *j.count;
   const double iT = 1.0 / double(rj.temp);
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   for (long long li = blockIdx.x; li < nlist; li += gridDim.x) {
     const long long row = j.rows[li];
     const RowStats rs = rj.stats[row];
@@ -136,72 +139,130 @@ __global__ void __launch_bounds__(kThreads) topp_finalize_kernel(const RefineJob
     const uint32_t kmax = Elem<T>::key(rs.m);
     if (kmax > base + uint32_t(kPBins - 1)) base = kmax - uint32_t(kPBins - 1);
     const float t = key_value<T>(base);
-    for (int i = threadIdx.x; i < kPBins; i += kThreads) hcnt[i] = 0u;
+    for (int i = threadIdx.x; i < kPBins; i += kFinThreads) hcnt[i] = 0u;
     if (threadIdx.x == 0) aux.ccount = 0;
     __syncthreads();
-    // eight groups of 8 per thread in flight
-    for (int v00 = int(threadIdx.x) * 8; v00 < V; v00 += 8 * kThreads * 8) {
-      float x[8][8];
+    // four groups of 8 per thread in flight; every thread takes the same number of rounds
+    // (the warp-level appends below need all lanes)
+    for (int r0 = 0; r0 < V; r0 += 4 * kFinThreads * 8) {
+      const int v00 = r0 + int(threadIdx.x) * 8;
+      float x[4][8];
+      load8xG<T, 4>(src, v00, kFinThreads * 8, V, al, x);
 #pragma unroll
-      for (int g = 0; g < 8; ++g) load8<T>(src, v00 + g * kThreads * 8, V, al, x[g]);
+      for (int g = 0; g < 4; ++g) {
+        const int v0 = v00 + g * kFinThreads * 8;
+        uint32_t mk = 0u;
 #pragma unroll
-      for (int g = 0; g < 8; ++g) {
-        const int v0 = v00 + g * kThreads * 8;
+        for (int k = 0; k < 8; ++k) mk |= (x[g][k] >= t && v0 + k < V) ? 1u << k : 0u;
+        // one shared atomic per warp for the list slots
+        const int my = __popc(mk);
+        int inc = my;
 #pragma unroll
-        for (int k = 0; k < 8; ++k) {
-          if (x[g][k] >= t && v0 + k < V) {
-            const uint32_t rel = Elem<T>::key(x[g][k]) - base;  // < kPBins: x <= the maximum
-            const int pos = atomicAdd(&aux.ccount, 1);
-            if (pos < kCapP) plist[pos] = pcomp(rel, v0 + k);
-            atomicAdd(&hcnt[rel], 1u);
-          }
+        for (int o = 1; o < 32; o <<= 1) {
+          const int up = __shfl_up_sync(0xffffffffu, inc, o);
+          if (lane >= o) inc += up;
+        }
+        const int wtot = __shfl_sync(0xffffffffu, inc, 31);
+        if (wtot == 0) continue;  // (uniform in the warp)
+        int wb = 0;
+        if (lane == 31) wb = atomicAdd(&aux.ccount, wtot);
+        int pos = __shfl_sync(0xffffffffu, wb, 31) + inc - my;
+        for (uint32_t m2 = mk; m2 != 0u; m2 &= m2 - 1u, ++pos) {
+          const int k = __ffs(m2) - 1;
+          const uint32_t h = Elem<T>::key(__uint_as_float(
+              uint32_t(reinterpret_cast<const unsigned short*>(src)[v0 + k]) << 16));
+          const uint32_t rel = h - base;  // < kPBins: the entry is at most the maximum
+          if (pos < kCapP) plist[pos] = pcomp(rel, v0 + k);
+          atomicAdd(&hcnt[rel], 1u);
         }
       }
     }
     __syncthreads();
     const int nall = aux.ccount;
-    if (threadIdx.x < 32) {
-      uint32_t cst = 0u;
-      double zk = -1.0;
-      int stable = 0;
-      const bool found = nall <= kCapP && cs.p_select_warp(nall, base, 0, rs.m, iT, rj.top_p, 0.0,
-                                                           zt, 0.0, &cst, &zk, &stable);
-      if (threadIdx.x == 0) {
-        aux.sel_found = found ? 1 : 0;
-        aux.sel_c32 = cst;
-        aux.sel_above = zk;
+    // the crossing code with the exact normaliser (warp 0), over the occupied codes
+    if (warp == 0) {
+      int jj = 0, stable = 0, bsel = -1;
+      double above = 0.0, wc = 0.0;
+      if (nall <= kCapP)
+        bsel = cs.p_cross_warp(int(kmax - base), base, rs.m, iT, rj.top_p, 0.0, zt, 0.0, &jj,
+                               &above, &wc, &stable);
+      if (bsel >= 0 && hcnt[bsel] > uint32_t(kPMem)) bsel = -1;
+      if (lane == 0) {
+        aux.sel_bin = bsel;
+        aux.sel_j = jj;
+        aux.sel_above = above + double(jj) * wc;
+        aux.sel_cnt = 0u;
+        aux.mcount = 0;
       }
     }
     __syncthreads();
-    const bool ok = aux.sel_found != 0;
-    const double zkept = aux.sel_above;
-    int32_t* kids = rj.kept_ids ? rj.kept_ids + size_t(row) * kKeptCap : nullptr;
-    if (!ok) {
+    const int bsel = aux.sel_bin;
+    if (bsel < 0) {
       // unresolved: the listed boundary stands, with its kept list
       if (threadIdx.x == 0 && j.unresolved) atomicAdd(j.unresolved, 1);
       __syncthreads();
       continue;
     }
-    const uint32_t cstar = aux.sel_c32;
-    if (threadIdx.x == 0) aux.mcount = 0;
-    __syncthreads();
+    // kept ids and the fp32 normaliser: the codes above the crossing code by every thread,
+    // the crossing code's entries gathered, then the j with the lowest ids by warp 0
+    int32_t* kids = rj.kept_ids ? rj.kept_ids + size_t(row) * kKeptCap : nullptr;
     unsigned long long z = 0;
-    for (int i = threadIdx.x; i < nall; i += kThreads) {
-      const uint32_t e = plist[i];
-      if (e < cstar) continue;
+    auto keep = [&](uint32_t e) {
       z += to_fx(weight(key_value<T>(base + pcomp_rel(e)), rs.c, rs.mc));
       const int slot = atomicAdd(&aux.mcount, 1);
       if (kids && slot < kKeptCap) kids[slot] = pcomp_id(e);
+    };
+    for (int i = threadIdx.x; i < nall; i += kFinThreads) {
+      const uint32_t e = plist[i];
+      const int r = int(pcomp_rel(e));
+      if (r > bsel) {
+        keep(e);
+      } else if (r == bsel) {
+        const uint32_t slot = atomicAdd(&aux.sel_cnt, 1u);
+        if (slot < uint32_t(kPMem)) pmem[slot] = e;
+      }
     }
-    const unsigned long long zf = creduce<unsigned long long>(z, aux.scr_u64, OpSum());
+    __syncthreads();
+    if (warp == 0) {
+      const int nm = min(int(aux.sel_cnt), kPMem);
+      const int jj = aux.sel_j;
+      uint32_t cst = 0u;
+      bool got = false;
+      for (int i = lane; i < nm; i += 32) {
+        const uint32_t e = pmem[i];
+        int ab = 0;
+        for (int q = 0; q < nm; ++q) ab += pmem[q] > e ? 1 : 0;
+        if (ab < jj) keep(e);
+        if (ab == jj - 1) {
+          cst = e;
+          got = true;
+        }
+      }
+      const unsigned g = __ballot_sync(0xffffffffu, got);
+      if (lane == 0) aux.sel_found = g ? 1 : 0;
+      if (g && lane == __ffs(g) - 1) aux.sel_c32 = cst;
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
+    if (lane == 0) zred[warp] = z;
+    __syncthreads();
     if (threadIdx.x == 0) {
-      RowStats out = rs;
-      out.thr_key = base + pcomp_rel(cstar);
-      out.cutoff = pcomp_id(cstar);
-      out.zd = zkept;
-      out.z = float(double(zf) * kFxInv);
-      rj.stats[row] = out;
-      if (rj.kept_n) rj.kept_n[row] = (kids && aux.mcount <= kKeptCap) ? aux.mcount : 0;
+      unsigned long long zf = 0;
+      for (int w = 0; w < kFinThreads / 32; ++w) zf += zred[w];
+      if (aux.sel_found) {
+        const uint32_t cstar = aux.sel_c32;
+        RowStats out = rs;
+        out.thr_key = base + pcomp_rel(cstar);
+        out.cutoff = pcomp_id(cstar);
+        out.zd = aux.sel_above;
+        out.z = float(double(zf) * kFxInv);
+        rj.stats[row] = out;
+        if (rj.kept_n) rj.kept_n[row] = (kids && aux.mcount <= kKeptCap) ? aux.mcount : 0;
+      } else {
+        // the list was partly rewritten: drop it, the listed boundary stands
+        if (rj.kept_n) rj.kept_n[row] = 0;
+        if (j.unresolved) atomicAdd(j.unresolved, 1);
+      }
     }
     __syncthreads();
   }

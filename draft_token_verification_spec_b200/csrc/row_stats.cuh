@@ -41,7 +41,7 @@ constexpr int kBulkChunk = 16384;
 constexpr int kCandCap = 512;      // candidates one CTA may hold in the top-k filter
 constexpr int kGatherCap = 1024;   // candidates a cluster may hold for exact selection
 constexpr int kMaxCluster = 16;
-constexpr int kKeptCap = 1024;     // kept ids listed per row: top-k rows, top-p nuclei this small
+constexpr int kKeptCap = 2048;     // kept ids listed per row: top-k rows, top-p nuclei this small
 constexpr float kS1Fx = 4294967296.0f;  // 2^32: signed fixed point for entropy terms
 
 struct RowJob {

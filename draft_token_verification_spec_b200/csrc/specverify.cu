@@ -191,7 +191,7 @@ cudaError_t launch_stream(const sv::StreamJob& job, int mode, cudaStream_t s) {
   }
 }
 
-// The top-p refinement. bfloat16 rows: the exact normalisers (four blocks per SM over the
+// The top-p refinement. bfloat16 rows: the exact normalisers (eight blocks per SM over the
 // (row, slice) items), then one block per listed row (one per SM, each walking the list).
 // float32 rows: one block per SM, each walking the listed rows.
 template <typename T>
@@ -216,11 +216,11 @@ cudaError_t launch_refine(const sv::RefineJob& j, cudaStream_t s) {
   const long long g = j.r.rows < sms ? j.r.rows : sms;
   if constexpr (sizeof(T) == 2) {
     const long long items = j.r.rows * sv::kZSlices;
-    const long long gz = items < 4LL * sms ? items : 4LL * sms;
+    const long long gz = items < 8LL * sms ? items : 8LL * sms;
     sv::topp_zexact_kernel<T><<<unsigned(gz), kThreads, 0, s>>>(j);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    sv::topp_finalize_kernel<T><<<unsigned(g), kThreads, 0, s>>>(j);
+    sv::topp_finalize_kernel<T><<<unsigned(g), sv::kFinThreads, 0, s>>>(j);
     return cudaGetLastError();
   } else {
     const size_t dyn = sv::refine_smem<T>();

@@ -152,8 +152,8 @@ __host__ __device__ constexpr size_t stream_dyn_bytes(int mode) {
              : size_t(Ring<SM_TOPP>::kBuf) * Ring<SM_TOPP>::kBufBytes + size_t(kCapP) * 4 +
                    size_t(kPBins) * 4 + size_t(kPMem) * 4;
 }
-// top-p: per warp, the vectors of the first chunk whose maxima set its threshold (1 in 16)
-constexpr int kChunk0WarpVecs = Ring<SM_TOPP>::kVec * 32 / 16;
+// top-p: per warp, the vectors of the first chunk whose maxima set its threshold (1 in 12)
+constexpr int kChunk0WarpVecs = Ring<SM_TOPP>::kVec * 32 / 12;
 static_assert(kPBins % kThreads == 0, "whole histogram bins per consumer thread");
 static_assert(kCapTopK <= kRankMax, "every top-k list is ranked directly");
 static_assert(kStreamMaxTopK <= kThreads, "the top k in rank order: one per thread");
@@ -575,109 +575,6 @@ struct CandSet {
     *above = __shfl_sync(0xffffffffu, ab, cl);
     *w = __shfl_sync(0xffffffffu, wc, cl);
     return __shfl_sync(0xffffffffu, bsel, cl);
-  }
-
-  // Top-p selection over the code histogram (bins >= 0 relative to base) and the list
-  // plist[0..n) (every entry of a code >= lfloor), by one warp (all 32 lanes call it; no
-  // block barrier). The codes are weighed once each in double, exp((l - m) / T); Z is ztot
-  // if that is >= 0, else their total plus zrest (the mass of the entries outside the
-  // histogram). Finds the code where the mass accumulated from the top reaches top_p * Z,
-  // how many of its entries it keeps (j, in id order), and the crossing composite among
-  // them (*cstar), with the kept mass (*zd) and whether the crossing stays put when the
-  // target moves by guard either way (*stable). False if it cannot be settled here (no
-  // crossing within the histogram, a crossing below lfloor, or more than kPMem entries of
-  // the crossing code). Lane L holds the codes kPBins - 1 - 32 L down to kPBins - 32 (L + 1).
-  __device__ bool p_select_warp(int n, uint32_t base, int lfloor, float m, double iT,
-                                float top_p, double zrest, double ztot, double guard,
-                                uint32_t* cstar, double* zd, int* stable) const {
-    constexpr int kPerL = kPBins / 32;
-    const int lane = threadIdx.x & 31;
-    const int top = kPBins - 1 - kPerL * lane;
-    Fx128 tsum = fx_zero();
-    for (int q = 0; q < kPerL; ++q) {
-      const uint32_t cnt = hcnt[top - q];
-      if (cnt)
-        tsum = fx_add(tsum, fx_mul_u32(fx_from(weight_d(key_value<T>(base + uint32_t(top - q)),
-                                                        m, iT)),
-                                       cnt));
-    }
-    Fx128 incl = tsum;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const Fx128 nb = fx_shfl_up(incl, o);
-      if (lane >= o) incl = fx_add(incl, nb);
-    }
-    const Fx128 zh{__shfl_sync(0xffffffffu, incl.lo, 31), __shfl_sync(0xffffffffu, incl.hi, 31)};
-    Fx128 ex = fx_shfl_up(incl, 1);
-    if (lane == 0) ex = fx_zero();
-    const double target = double(top_p) * (ztot >= 0.0 ? ztot : fx_to_double(zh) + zrest);
-    const unsigned hit = __ballot_sync(
-        0xffffffffu, fx_to_double(ex) < target && target <= fx_to_double(incl));
-    if (!hit) return false;  // the histogram holds less than the target
-    const int cl = __ffs(hit) - 1;
-    int bsel = -1, j = 0, stb = 0;
-    double above = 0.0, w = 0.0;
-    if (lane == cl) {
-      Fx128 acc = ex;
-      for (int q = 0; q < kPerL; ++q) {
-        const uint32_t cnt = hcnt[top - q];
-        if (!cnt) continue;
-        const double wq = weight_d(key_value<T>(base + uint32_t(top - q)), m, iT);
-        const Fx128 nacc = fx_add(acc, fx_mul_u32(fx_from(wq), cnt));
-        const double a = fx_to_double(acc), t = fx_to_double(nacc);
-        if (a < target && target <= t) {
-          // the fewest entries of the code that reach the target
-          int jj = int(ceil((target - a) / wq));
-          jj = max(1, min(int(cnt), jj));
-          while (jj > 1 && a + double(jj - 1) * wq >= target) --jj;
-          while (jj < int(cnt) && a + double(jj) * wq < target) ++jj;
-          bsel = top - q;
-          j = jj;
-          above = a;
-          w = wq;
-          stb = (a + double(jj - 1) * wq < target - guard && a + double(jj) * wq >= target + guard)
-                    ? 1 : 0;
-          break;
-        }
-        acc = nacc;
-      }
-    }
-    bsel = __shfl_sync(0xffffffffu, bsel, cl);
-    j = __shfl_sync(0xffffffffu, j, cl);
-    stb = __shfl_sync(0xffffffffu, stb, cl);
-    above = __shfl_sync(0xffffffffu, above, cl);
-    w = __shfl_sync(0xffffffffu, w, cl);
-    if (bsel < lfloor || hcnt[bsel] > uint32_t(kPMem)) return false;  // (bsel < 0 included)
-    // the entries of the crossing code, then the j-th largest of them (the j-th lowest id)
-    int nm = 0;
-    for (int i0 = 0; i0 < n; i0 += 32) {
-      const int i = i0 + lane;
-      const uint32_t e = i < n ? plist[i] : 0u;
-      const bool is = i < n && int(pcomp_rel(e)) == bsel;
-      const unsigned bal = __ballot_sync(0xffffffffu, is);
-      const int slot = nm + __popc(bal & ((1u << lane) - 1u));
-      if (is && slot < kPMem) pmem[slot] = e;
-      nm += __popc(bal);
-    }
-    nm = min(nm, kPMem);
-    __syncwarp();
-    uint32_t cst = 0u;
-    bool got = false;
-    for (int i = lane; i < nm; i += 32) {
-      const uint32_t e = pmem[i];
-      int ab = 0;
-      for (int q = 0; q < nm; ++q) ab += pmem[q] > e ? 1 : 0;
-      if (ab == j - 1) {
-        cst = e;
-        got = true;
-      }
-    }
-    const unsigned g = __ballot_sync(0xffffffffu, got);
-    if (!g) return false;
-    *cstar = __shfl_sync(0xffffffffu, cst, __ffs(g) - 1);
-    *zd = above + double(j) * w;
-    *stable = stb;
-    return true;
   }
 
   // Top-k lists: keeps the candidates of cand[0..n) (n <= kCapTopK) whose composite is

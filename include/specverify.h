@@ -253,7 +253,7 @@ spec_status spec_commit_linear_state(float* state, int B, int H, int dk, int dv,
  * SPEC_STATIC_SCRATCH_BYTES inside the library, one per device; the call allocates
  * nothing and looks the array's address up once per device (with that device current).
  *   - A call whose spec_workspace_size(B, K, V) exceeds SPEC_STATIC_SCRATCH_BYTES returns
- *     SPEC_ERR_WORKSPACE before any CUDA call (32 MiB holds about 8,000 logit rows,
+ *     SPEC_ERR_WORKSPACE before any CUDA call (32 MiB holds about 4,000 logit rows,
  *     B * (2K + 1)).
  *   - Every call on a device uses the same scratch: calls that overlap in time (on
  *     different streams, or from host threads without ordering) race on it and give

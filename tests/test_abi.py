@@ -32,12 +32,12 @@ def test_status_strings_and_kernel_counts(lib):
 
 def _ws(rows):
     up = lambda x: (x + 255) // 256 * 256
-    return (256 + up(48 * rows) + up(4 * rows) + up(rows * 1024 * 4) + up(4 * rows) + up(4 * rows)
+    return (256 + up(48 * rows) + up(4 * rows) + up(rows * 2048 * 4) + up(4 * rows) + up(4 * rows)
             + up(16 * rows))
 
 
 def test_workspace_size(lib):
-    """header, 48-byte row statistics, kept-id counts, up to 1024 kept ids per row, the list
+    """header, 48-byte row statistics, kept-id counts, up to 2048 kept ids per row, the list
     of rows the cluster kernel finishes, the list of refined rows and their exact
     normalisers (16 bytes each)"""
     assert sv.spec_workspace_size(0, 4, 10) == 0
