@@ -180,6 +180,7 @@ struct __align__(16) StreamAux {
   uint32_t scr_u32[kWarps];
   unsigned long long sel_before;
   unsigned long long sel_comp;
+  unsigned long long sel_x[2];  // top-k: the exchange's k-th, by exchange parity
   double sel_above;  // top-p: mass of the codes above the crossing code
   double sel_w;      // top-p: weight of the crossing code
   int sel_j;         // top-p: entries of the crossing code kept
@@ -601,20 +602,17 @@ struct CandSet {
   }
 
   // Short lists (n <= kRankMax, flat): the k-th largest composite among cand[0..n) that are
-  // >= lim, by counting for each the larger ones (composites are distinct) ->
-  // aux->sel_comp. The caller has synchronised the list. False if there is none.
-  __device__ bool rank_select(int n, uint64_t lim, int k) {
-    if (threadIdx.x == 0) aux->sel_comp = 0;
-    csync();
+  // >= lim, by counting for each the larger ones (composites are distinct) -> *out, which
+  // the caller zeroed before a barrier that precedes the call; a barrier must follow before
+  // *out is read. No barrier inside.
+  __device__ void rank_into(int n, uint64_t lim, int k, unsigned long long* out) const {
     for (int i = threadIdx.x; i < n; i += kThreads) {
       const uint64_t e = cand[i];
       if (e < lim) continue;
       int above = 0;
       for (int j = 0; j < n; ++j) above += cand[j] > e ? 1 : 0;
-      if (above == k - 1) aux->sel_comp = e;
+      if (above == k - 1) *out = e;
     }
-    csync();
-    return aux->sel_comp != 0;
   }
 
   // Top-k lists (n <= kRankMax): the top k of cand[0..n) (k <= kThreads) in rank order, then
@@ -916,6 +914,7 @@ __global__ void __launch_bounds__(kStreamThreads, (kMode == SM_TOPK ? SV_TOPK_CT
     };
     uint4 w[kReload ? 1 : kVecPerThread];
     float vm[kVecPerThread];
+    uint32_t cm[kVecPerThread];
 #pragma unroll
     for (int u = 0; u < kVecPerThread; ++u) {
       const uint4 wu = load_vec(u * kThreads + int(threadIdx.x));
@@ -1007,7 +1006,6 @@ __global__ void __launch_bounds__(kStreamThreads, (kMode == SM_TOPK ? SV_TOPK_CT
     }
 
     // ---- the chunk pass
-    uint32_t cm[kVecPerThread];
     float vmax4 = -INFINITY;
 #pragma unroll
     for (int u = 0; u < kVecPerThread; ++u) {
@@ -1162,6 +1160,8 @@ __global__ void __launch_bounds__(kStreamThreads, (kMode == SM_TOPK ? SV_TOPK_CT
           aux.red_f[xpar][warp] = wm;
           aux.red_i[xpar][warp] = wacc + wsingle;
         }
+        if (kMode == SM_TOPK && threadIdx.x == 0) aux.sel_x[xpar] = 0ull;
+        const int xp = xpar;
         csync();
         float mrow = aux.red_f[xpar][0];
         int added = aux.red_i[xpar][0];
@@ -1195,8 +1195,14 @@ __global__ void __launch_bounds__(kStreamThreads, (kMode == SM_TOPK ? SV_TOPK_CT
             // the exact k-th of the entries seen so far becomes the threshold; a short list
             // keeps the entries below it (the row-end selection ranks past them), one past
             // half the capacity drops them
-            if (cnt >= keep && cs.rank_select(cnt, 0, keep)) {
-              const uint64_t kth = aux.sel_comp;
+            bool have = false;
+            if (cnt >= keep) {  // (uniform)
+              cs.rank_into(cnt, 0, keep, &aux.sel_x[xp]);
+              csync();
+              have = aux.sel_x[xp] != 0ull;
+            }
+            if (have) {
+              const uint64_t kth = aux.sel_x[xp];
               thr = fmaxf(thr, key_value<T>(comp_key(kth)));
               if (cnt > kCapTopK / 2) cnt = cs.compact_ge(cnt, kth);
             }
@@ -1392,6 +1398,118 @@ __global__ void __launch_bounds__(kStreamThreads, (kMode == SM_TOPK ? SV_TOPK_CT
       wlen = 0;
       overflow = false;
       row_timeout = false;
+    } else if (kMode == SM_TOPK && q == nchunk - 1) {
+      // ---------------------------------------------------------------- top-k row end
+      // one exchange: per warp the timeout flag and the maximum
+      float wmx = st.mt;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) wmx = fmax_nan(wmx, __shfl_xor_sync(0xffffffffu, wmx, o));
+      const bool wtmo = __any_sync(0xffffffffu, row_timeout);
+      if (lane == 0) {
+        aux.red_f[xpar][warp] = wmx;
+        aux.red_i[xpar][warp] = wtmo ? 1 : 0;
+      }
+      if (threadIdx.x == 0) {
+        aux.sel_comp = 0ull;
+        aux.mcount = 0;
+      }
+      csync();
+      const int nall = aux.ccount;  // every append of the row is done
+      float m = aux.red_f[xpar][0];
+      bool tmo = aux.red_i[xpar][0] != 0;
+#pragma unroll
+      for (int ww = 1; ww < kWarps; ++ww) {
+        m = fmax_nan(m, aux.red_f[xpar][ww]);
+        tmo = tmo || aux.red_i[xpar][ww] != 0;
+      }
+      int status = tmo ? ROW_TIMEOUT
+                       : ((m != m || m == INFINITY || m == -INFINITY) ? ROW_INVALID : ROW_OK);
+      const float mc = m * c;
+      const int n = min(nall, kCapM);
+      const bool go = status == ROW_OK && !overflow && nall <= kCapM && n >= rj.top_k;
+      // the k-th composite (every list is short, kCapTopK <= kRankMax: ranked directly); with
+      // top-p, the crossing within the top k
+      if (go) {
+        if (rj.top_p < 1.0f) {
+          cs.rank_topp(n, rj.top_k, rj.top_p, m, iT);
+        } else {
+          cs.rank_into(n, 0, rj.top_k, &aux.sel_comp);
+          csync();
+        }
+      } else {
+        csync();
+      }
+      const uint64_t cstar = aux.sel_comp;
+      if (status == ROW_OK && cstar == 0ull) status = ROW_FALLBACK;
+      const bool ok = status == ROW_OK;
+      const bool list = ok && rj.kept_ids != nullptr;
+      // normaliser, entropy term and kept-id list over the kept candidates; the double
+      // normaliser is left to the consumer, which sums it over the list if it needs it
+      unsigned long long z = 0;
+      long long s1 = 0;
+      if (ok) {
+        for (int i = threadIdx.x; i < n; i += kThreads) {
+          const uint64_t e = cs.cand[i];
+          if (e < cstar) continue;
+          const float xv = key_value<T>(comp_key(e));
+          const float zx = wexp(xv, c, mc);
+          const float ex = ex2(zx);
+          z += to_fx(ex);
+          if (want_ent) s1 += __float2ll_rn(ent_term(ex, zx) * kS1Fx);
+          if (list) {
+            const int slot = atomicAdd(&aux.mcount, 1);
+            if (slot < kKeptCap) rj.kept_ids[size_t(row) * kKeptCap + slot] = comp_id(e);
+          }
+        }
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        z += __shfl_xor_sync(0xffffffffu, z, o);
+        s1 += __shfl_xor_sync(0xffffffffu, s1, o);
+      }
+      if (lane == 0) {
+        aux.scr_u64[warp] = z;
+        aux.scr_s64[warp] = s1;
+      }
+      csync();
+      if (threadIdx.x == 0) {
+        unsigned long long zfx = 0;
+        long long s1a = 0;
+#pragma unroll
+        for (int ww = 0; ww < kWarps; ++ww) {
+          zfx += aux.scr_u64[ww];
+          s1a += aux.scr_s64[ww];
+        }
+        if (tmo && rj.dev_status) atomicOr(rj.dev_status, 1);
+        if (status == ROW_FALLBACK) job.fb_rows[atomicAdd(job.fb_count, 1)] = int32_t(row);
+        if (rj.kept_n) rj.kept_n[row] = (list && aux.mcount <= kKeptCap) ? aux.mcount : 0;
+        const double Z = double(zfx) * kFxInv;
+        const double S1 = double(s1a) / double(kS1Fx);
+        if (rj.stats) {
+          RowStats rs;
+          rs.mc = mc;
+          rs.z = float(Z);
+          rs.entropy = (ok && want_ent) ? float(log(Z) - 0.6931471805599453 * S1 / Z) : 0.0f;
+          rs.thr_key = ok ? comp_key(cstar) : 0u;
+          rs.cutoff = ok ? comp_id(cstar) : INT_MAX;
+          rs.argmax = -1;
+          rs.status = status;
+          rs.c = c;
+          rs.m = m;
+          rs.pad = 0;
+          rs.zd = -1.0;
+          rj.stats[row] = rs;
+        }
+        aux.ccount = 0;  // the next row starts clean (its first exchange orders this)
+      }
+      st.reset();
+      thr = -INFINITY;
+      cnt = 0;
+      wacc = 0;
+      single = 0;
+      wlen = 0;
+      overflow = false;
+      row_timeout = false;
     } else if (q == nchunk - 1) {
       // ---------------------------------------------------------------- row end
       const bool tmo = csync_or(row_timeout);
@@ -1421,49 +1539,6 @@ __global__ void __launch_bounds__(kStreamThreads, (kMode == SM_TOPK ? SV_TOPK_CT
           }
           zfx = creduce<unsigned long long>(to_fx(sc), aux.scr_u64, OpSum());
           S1 = creduce<double>(double(hc), aux.scr_f64, OpSum());
-        }
-      } else if constexpr (kMode == SM_TOPK) {
-        if (status == ROW_OK) {
-          const int n = min(nall, kCapM);
-          bool ok = !overflow && nall <= kCapM && n >= rj.top_k;
-          uint64_t cstar = 0;
-          if (ok) {  // every list is short (kCapTopK <= kRankMax): rank directly
-            if (rj.top_p < 1.0f) {  // the top-p crossing within the top k
-              ok = cs.rank_topp(n, rj.top_k, rj.top_p, m, iT);
-            } else {
-              ok = cs.rank_select(n, 0, rj.top_k);
-            }
-            cstar = aux.sel_comp;
-          }
-          if (!ok) {
-            status = ROW_FALLBACK;
-          } else {
-            // normaliser, entropy term and kept-id list over the kept candidates; the double
-            // normaliser is left to the consumer, which sums it over the list if it needs it
-            const bool list = rj.kept_ids != nullptr;
-            if (threadIdx.x == 0) aux.mcount = 0;
-            csync();
-            unsigned long long z = 0;
-            long long s1 = 0;
-            for (int i = threadIdx.x; i < n; i += kThreads) {
-              const uint64_t e = cs.cand[i];
-              if (e < cstar) continue;
-              const float xv = key_value<T>(comp_key(e));
-              const float zx = wexp(xv, c, mc);
-              const float ex = ex2(zx);
-              z += to_fx(ex);
-              if (want_ent) s1 += __float2ll_rn(ent_term(ex, zx) * kS1Fx);
-              if (list) {
-                const int slot = atomicAdd(&aux.mcount, 1);
-                if (slot < kKeptCap) rj.kept_ids[size_t(row) * kKeptCap + slot] = comp_id(e);
-              }
-            }
-            zfx = creduce<unsigned long long>(z, aux.scr_u64, OpSum());
-            S1 = double(creduce<long long>(s1, aux.scr_s64, OpSum())) / double(kS1Fx);
-            thr_key = comp_key(cstar);
-            cutoff = comp_id(cstar);
-            listed = list;
-          }
         }
       }
       if (status == ROW_FALLBACK && threadIdx.x == 0)
