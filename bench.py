@@ -244,7 +244,8 @@ def per_config_chain(cfg, greedy, args, dev) -> dict:
     res = {"workload": workload(cfg, greedy)["workload"], "metric_unit": UNIT,
            "value": cfg.B * cfg.K * args.steps / (ms / 1e3), "ms_per_step": ms / args.steps,
            "row_stage_ms": round(row, 4),
-           "roofline": roofline_entry(algorithmic_bytes(cfg, greedy), row),
+           "roofline": {**roofline_entry(algorithmic_bytes(cfg, greedy), row),
+                        "traffic": read_profile_traffic(workload(cfg, greedy)["workload"])},
            "mean_accepted_len": float(accl.mean())}
     del tg, dg, ug, xg, ws
     torch.cuda.empty_cache()
@@ -384,9 +385,12 @@ def run_ours(args, cfg, greedy, rank, world):
     e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e2e_steps, dev, world)
     e2e_value = job_value(cfg.B, cfg.K, world, 1, e2e_ms)
 
-    # the row kernel, the exact finisher (candidate modes only) and the per-batch-row kernel
+    # the row kernel, the exact finisher (candidate modes only), the double-precision top-p
+    # placement (exact normalisers and re-collection, top-p without top-k) and the
+    # per-batch-row kernel
     candidates = not greedy and ((0 < cfg.top_k < cfg.V) or cfg.top_p < 1.0)
-    kernels_per_step = 3 if candidates else 2
+    refined = not greedy and cfg.top_p < 1.0 and not (0 < cfg.top_k < cfg.V)
+    kernels_per_step = 2 + (1 if candidates else 0) + (2 if refined else 0)
     row_avg_ms = float(np.mean(row_ms))
     alg = algorithmic_bytes(cfg, greedy)
     traffic = read_profile_traffic(workload(cfg, greedy)["workload"])

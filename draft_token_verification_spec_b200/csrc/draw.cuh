@@ -139,39 +139,39 @@ __device__ int inverse_cdf_draw(F&& f, int V, float w, DrawSmem& sm) {
 }
 
 // The same draw when every entry outside ids[0..n) (distinct ids, any order,
-// n <= kSparseCap) has mass 0: the support is sorted by id (each id counts the smaller ones)
-// and one block-wide prefix sum replaces the pass over the row, thread t holding sorted
-// positions [kSparsePer t, kSparsePer (t + 1)). mass(v) gives the Fx128 mass of entry v; the
+// n <= kPer * kThreads) has mass 0: the support is sorted by id (each id counts the smaller
+// ones) and one block-wide prefix sum replaces the pass over the row, thread t holding
+// sorted positions [kPer t, kPer (t + 1)). mass(v) gives the Fx128 mass of entry v; the
 // result is identical to inverse_cdf_draw over the whole row with the same masses.
-template <typename F>
-__device__ int sparse_draw(const int32_t* ids, int n, F&& mass, float w, DrawSmem& sm) {
+template <int kPer, typename F>
+__device__ int sparse_draw_n(const int32_t* ids, int n, F&& mass, float w, DrawSmem& sm) {
   const int t = threadIdx.x;
-  int my[kSparsePer];
+  int my[kPer];
 #pragma unroll
-  for (int q = 0; q < kSparsePer; ++q) {
+  for (int q = 0; q < kPer; ++q) {
     const int i = q * kThreads + t;
     my[q] = i < n ? ids[i] : INT_MAX;
     if (i < n) sm.ids[i] = my[q];
   }
   if (t == 0) sm.best = INT_MAX;
   __syncthreads();
-  int rank[kSparsePer];
+  int rank[kPer];
 #pragma unroll
-  for (int q = 0; q < kSparsePer; ++q) {
+  for (int q = 0; q < kPer; ++q) {
     rank[q] = 0;
     if (q * kThreads + t < n)
       for (int j = 0; j < n; ++j) rank[q] += sm.ids[j] < my[q] ? 1 : 0;
   }
   __syncthreads();
 #pragma unroll
-  for (int q = 0; q < kSparsePer; ++q)
+  for (int q = 0; q < kPer; ++q)
     if (q * kThreads + t < n) sm.ids[rank[q]] = my[q];
   __syncthreads();
-  Fx128 r[kSparsePer];
+  Fx128 r[kPer];
   Fx128 own = fx_zero();
 #pragma unroll
-  for (int q = 0; q < kSparsePer; ++q) {
-    const int p = kSparsePer * t + q;
+  for (int q = 0; q < kPer; ++q) {
+    const int p = kPer * t + q;
     r[q] = p < n ? mass(sm.ids[p]) : fx_zero();
     own = fx_add(own, r[q]);
   }
@@ -179,10 +179,10 @@ __device__ int sparse_draw(const int32_t* ids, int n, F&& mass, float w, DrawSme
   Fx128 cum = block_exclusive_scan_fx(own, sm.scr, &S);
   const double target = double(w) * fx_to_double(S);
 #pragma unroll
-  for (int q = 0; q < kSparsePer; ++q) {
+  for (int q = 0; q < kPer; ++q) {
     cum = fx_add(cum, r[q]);
     if (!fx_is_zero(r[q]) && fx_to_double(cum) > target) {
-      atomicMin(&sm.best, sm.ids[kSparsePer * t + q]);
+      atomicMin(&sm.best, sm.ids[kPer * t + q]);
       break;
     }
   }
@@ -195,13 +195,21 @@ __device__ int sparse_draw(const int32_t* ids, int n, F&& mass, float w, DrawSme
     if (t == 0) sm.best = -1;
     __syncthreads();
 #pragma unroll
-    for (int q = 0; q < kSparsePer; ++q)
-      if (!fx_is_zero(r[q])) atomicMax(&sm.best, sm.ids[kSparsePer * t + q]);
+    for (int q = 0; q < kPer; ++q)
+      if (!fx_is_zero(r[q])) atomicMax(&sm.best, sm.ids[kPer * t + q]);
     __syncthreads();
     tok = sm.best;
   }
   __syncthreads();
   return tok;
+}
+
+// Dispatch on the support size: four entries per thread up to 4 * kThreads, else eight
+// (fewer registers for the common short lists).
+template <typename F>
+__device__ int sparse_draw(const int32_t* ids, int n, F&& mass, float w, DrawSmem& sm) {
+  if (n <= 4 * kThreads) return sparse_draw_n<4>(ids, n, mass, w, sm);
+  return sparse_draw_n<kSparsePer>(ids, n, mass, w, sm);
 }
 
 // Loads entries v0..v0+7 of a logit row as floats (-inf past V): 16-byte vector loads
@@ -275,14 +283,11 @@ static __device__ const double kExp2J[64] = {
 // 15(2), 1989): x = (64 k + j) ln2 / 64 + r with |r| <= ln2 / 128 (ln2 / 64 split into a
 // 32-bit head and a tail, so n * head is exact), e^x = 2^k 2^(j/64) e^r, and e^r by its
 // Taylor series to r^5 (the remainder is below 4e-17 of it). Relative error within a few
-// units in the last place; x below -745 (and -inf) gives 0. Branch-free, so that the
-// compiler can overlap independent evaluations: 2^k is applied as two exact power-of-two
-// factors (each a normal double), so a subnormal result is rounded once, as by ldexp.
+// units in the last place; x below -745 (and -inf) gives 0.
 __device__ __forceinline__ double exp_neg(double x) {
-  const bool zero = !(x > -745.0);  // also -inf and NaN
-  const double xs = zero ? 0.0 : x;
-  const double n = rint(xs * 92.33248261689366);  // 64 / ln2
-  double r = fma(-n, 0x1.62e42fee00000p-7, xs);
+  if (!(x > -745.0)) return 0.0;
+  const double n = rint(x * 92.33248261689366);  // 64 / ln2
+  double r = fma(-n, 0x1.62e42fee00000p-7, x);
   r = fma(-n, 0x1.a39ef35793c76p-39, r);
   const int ni = int(n);
   double p = fma(r, 1.0 / 120.0, 1.0 / 24.0);
@@ -291,11 +296,9 @@ __device__ __forceinline__ double exp_neg(double x) {
   p = fma(p, r, 1.0);
   p = fma(p, r, 1.0);
   const double t = __ldg(&kExp2J[ni & 63]) * p;
-  const int k = ni >> 6;  // floor(n / 64), in [-1075, 0]
-  const int k1 = k >> 1, k2 = k - k1;
-  const double res = t * __longlong_as_double((long long)(k1 + 1023) << 52) *
-                     __longlong_as_double((long long)(k2 + 1023) << 52);
-  return zero ? 0.0 : res;
+  const int k = ni >> 6;  // floor(n / 64)
+  if (k >= -1022) return t * __longlong_as_double((long long)(k + 1023) << 52);
+  return ldexp(t, k);
 }
 
 // Unnormalised weight exp((l - m) / T) of a kept entry, in double (l - m is exact); iT = 1 / T.

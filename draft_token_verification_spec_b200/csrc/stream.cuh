@@ -1511,9 +1511,8 @@ __global__ void __launch_bounds__(kStreamThreads, (kMode == SM_TOPK ? SV_TOPK_CT
       overflow = false;
       row_timeout = false;
     } else if (q == nchunk - 1) {
-      // ---------------------------------------------------------------- row end
+      // ---------------------------------------------------------------- row end (greedy, sums)
       const bool tmo = csync_or(row_timeout);
-      const int nall = aux.ccount;  // every append of the row is done (candidate modes)
       const float m = creduce<float>(st.mt, aux.scr_f, OpMaxNan());
       int status = tmo ? ROW_TIMEOUT
                        : ((m != m || m == INFINITY || m == -INFINITY) ? ROW_INVALID : ROW_OK);
