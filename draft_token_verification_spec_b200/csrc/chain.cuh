@@ -110,29 +110,49 @@ __global__ void __launch_bounds__(kThreads) chain_finish_kernel(const ChainJob j
   if (threadIdx.x == 0) s_zpos = -1;
   const int npos = min(K + 1, kZPos);
   if (!j.greedy) {
-    // rows that list their kept ids: the double normaliser over the list, one warp per row
+    // rows that list their kept ids: the double normaliser over the list, eight lanes per
+    // row (four rows per warp at a time), each lane's ids and logits loaded together
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    for (int r = warp; r < 2 * npos; r += kWarps) {
+    const int sub = lane & 7;
+    for (int r0 = warp * 4; r0 < 2 * npos; r0 += 4 * kWarps) {  // (uniform in the warp)
+      const int r = r0 + (lane >> 3);
       const bool tgt = r < npos;
       const int i = tgt ? r : r - npos;
+      const bool live = r < 2 * npos && (tgt || i < K);
       double z = -1.0;
-      if (tgt || i < K) {
-        const RowStats st = tgt ? ts[i] : ds[i];
-        const size_t gr = tgt ? size_t(b) * (K + 1) + i : size_t(j.B) * (K + 1) + size_t(b) * K + i;
-        const int nk = j.kept_n ? j.kept_n[gr] : 0;
+      RowStats st;
+      int nk = 0;
+      size_t gr = 0;
+      if (live) {
+        st = tgt ? ts[i] : ds[i];
+        gr = tgt ? size_t(b) * (K + 1) + i : size_t(j.B) * (K + 1) + size_t(b) * K + i;
+        nk = j.kept_n ? j.kept_n[gr] : 0;
         z = st.zd;
-        if (z < 0.0 && st.status == ROW_OK && nk > 0) {
-          const T* row = tgt ? trow0 + size_t(i) * V : drow0 + size_t(i) * V;
-          const int32_t* ids = j.kept_ids + gr * kKeptCap;
-          Fx128 acc = fx_zero();
-          for (int q = lane; q < nk; q += 32) {
-            const int v = ids[q];
-            acc = fx_add(acc, fx_from(kept_weight_d<T>(st, iT, Elem<T>::load(row, size_t(v)), v)));
+      }
+      const bool sum = live && z < 0.0 && st.status == ROW_OK && nk > 0;
+      Fx128 acc = fx_zero();
+      if (sum) {
+        const T* row = tgt ? trow0 + size_t(i) * V : drow0 + size_t(i) * V;
+        const int32_t* ids = j.kept_ids + gr * kKeptCap;
+        for (int q0 = 0; q0 < nk; q0 += 8 * 8) {
+          int v[8];
+          float x[8];
+#pragma unroll
+          for (int k = 0; k < 8; ++k) {
+            const int q = q0 + 8 * k + sub;
+            v[k] = q < nk ? ids[q] : -1;
           }
-          z = fx_to_double(warp_sum_fx(acc));
+#pragma unroll
+          for (int k = 0; k < 8; ++k) x[k] = v[k] >= 0 ? Elem<T>::load(row, size_t(v[k])) : 0.0f;
+#pragma unroll
+          for (int k = 0; k < 8; ++k)
+            if (v[k] >= 0) acc = fx_add(acc, fx_from(kept_weight_d<T>(st, iT, x[k], v[k])));
         }
       }
-      if (lane == 0) s_zl[tgt ? 0 : 1][i] = z;
+#pragma unroll
+      for (int o = 4; o > 0; o >>= 1) acc = fx_add(acc, fx_shfl_xor(acc, o));
+      if (sum) z = fx_to_double(acc);
+      if (live && sub == 0) s_zl[tgt ? 0 : 1][i] = z;
     }
   }
   __syncthreads();
@@ -261,7 +281,7 @@ __global__ void __launch_bounds__(kThreads) chain_finish_kernel(const ChainJob j
                                prob_d<T>(sq, izq, iT, Elem<T>::load(qrow, size_t(v)), v);
               return fx_from(fmax(d, 0.0));
             },
-            w, sm);
+            w, sm, V);
       }
       if (tok < 0)
         tok = sparse_draw(
@@ -269,7 +289,7 @@ __global__ void __launch_bounds__(kThreads) chain_finish_kernel(const ChainJob j
             [&](int v) {
               return fx_from(kept_weight_d<T>(sp, iT, Elem<T>::load(prow, size_t(v)), v));
             },
-            w, sm);
+            w, sm, V);
     } else {
       if (a < K) {
         const RowStats sq = ds[a];

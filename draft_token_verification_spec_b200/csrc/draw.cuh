@@ -138,34 +138,71 @@ __device__ int inverse_cdf_draw(F&& f, int V, float w, DrawSmem& sm) {
   return tok;
 }
 
+// Ids below this many are sorted through a bitmap in the draw's chunk table (16 KB).
+constexpr int kBitmapIds = kMaxDrawChunks * kWarps * 16 * 8;
+
 // The same draw when every entry outside ids[0..n) (distinct ids, any order,
-// n <= kPer * kThreads) has mass 0: the support is sorted by id (each id counts the smaller
-// ones) and one block-wide prefix sum replaces the pass over the row, thread t holding
-// sorted positions [kPer t, kPer (t + 1)). mass(v) gives the Fx128 mass of entry v; the
-// result is identical to inverse_cdf_draw over the whole row with the same masses.
+// n <= kPer * kThreads) has mass 0: the support is sorted by id and one block-wide prefix
+// sum replaces the pass over the row, thread t holding sorted positions [kPer t, kPer (t + 1)).
+// The sort: long lists of ids below V <= kBitmapIds set bits in a bitmap that the block then
+// reads in order; other lists count for each id the smaller ones. mass(v) gives the Fx128
+// mass of entry v; the result is identical to inverse_cdf_draw over the whole row with the
+// same masses.
 template <int kPer, typename F>
-__device__ int sparse_draw_n(const int32_t* ids, int n, F&& mass, float w, DrawSmem& sm) {
+__device__ int sparse_draw_n(const int32_t* ids, int n, F&& mass, float w, DrawSmem& sm,
+                             int V) {
   const int t = threadIdx.x;
   int my[kPer];
+  const bool bitmap = n > 128 && V > 0 && V <= kBitmapIds;  // (uniform)
+  uint32_t* bm = reinterpret_cast<uint32_t*>(&sm.wchunk[0][0]);
+  const int nw = (V + 31) >> 5;
+  if (bitmap)
+    for (int i = t; i < nw; i += kThreads) bm[i] = 0u;
 #pragma unroll
   for (int q = 0; q < kPer; ++q) {
     const int i = q * kThreads + t;
     my[q] = i < n ? ids[i] : INT_MAX;
-    if (i < n) sm.ids[i] = my[q];
+    if (i < n && !bitmap) sm.ids[i] = my[q];
   }
   if (t == 0) sm.best = INT_MAX;
   __syncthreads();
-  int rank[kPer];
+  if (bitmap) {
 #pragma unroll
-  for (int q = 0; q < kPer; ++q) {
-    rank[q] = 0;
-    if (q * kThreads + t < n)
-      for (int j = 0; j < n; ++j) rank[q] += sm.ids[j] < my[q] ? 1 : 0;
+    for (int q = 0; q < kPer; ++q)
+      if (q * kThreads + t < n) atomicOr(&bm[my[q] >> 5], 1u << (my[q] & 31));
+    __syncthreads();
+    // thread t reads words [t per, (t + 1) per) and writes their ids from its exclusive
+    // prefix count on
+    const int per = (nw + kThreads - 1) / kThreads;
+    int cnt = 0;
+    for (int i = t * per; i < min(nw, (t + 1) * per); ++i) cnt += __popc(bm[i]);
+    const int lane = t & 31, warp = t >> 5;
+    int inc = cnt;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int up = __shfl_up_sync(0xffffffffu, inc, o);
+      if (lane >= o) inc += up;
+    }
+    int* wsum = reinterpret_cast<int*>(sm.scr);
+    if (lane == 31) wsum[warp] = inc;
+    __syncthreads();
+    int pos = inc - cnt;
+    for (int ww = 0; ww < warp; ++ww) pos += wsum[ww];
+    for (int i = t * per; i < min(nw, (t + 1) * per); ++i)
+      for (uint32_t bits = bm[i]; bits != 0u; bits &= bits - 1u) sm.ids[pos++] = 32 * i + __ffs(bits) - 1;
+  } else {
+    int rank[kPer];
+#pragma unroll
+    for (int q = 0; q < kPer; ++q) {
+      rank[q] = 0;
+      if (q * kThreads + t < n)
+        for (int j = 0; j < n; ++j) rank[q] += sm.ids[j] < my[q] ? 1 : 0;
+    }
+    __syncthreads();
+#pragma unroll
+    for (int q = 0; q < kPer; ++q)
+      if (q * kThreads + t < n) sm.ids[rank[q]] = my[q];
   }
-  __syncthreads();
-#pragma unroll
-  for (int q = 0; q < kPer; ++q)
-    if (q * kThreads + t < n) sm.ids[rank[q]] = my[q];
   __syncthreads();
   Fx128 r[kPer];
   Fx128 own = fx_zero();
@@ -207,9 +244,10 @@ __device__ int sparse_draw_n(const int32_t* ids, int n, F&& mass, float w, DrawS
 // Dispatch on the support size: four entries per thread up to 4 * kThreads, else eight
 // (fewer registers for the common short lists).
 template <typename F>
-__device__ int sparse_draw(const int32_t* ids, int n, F&& mass, float w, DrawSmem& sm) {
-  if (n <= 4 * kThreads) return sparse_draw_n<4>(ids, n, mass, w, sm);
-  return sparse_draw_n<kSparsePer>(ids, n, mass, w, sm);
+__device__ int sparse_draw(const int32_t* ids, int n, F&& mass, float w, DrawSmem& sm,
+                           int V = 0) {
+  if (n <= 4 * kThreads) return sparse_draw_n<4>(ids, n, mass, w, sm, V);
+  return sparse_draw_n<kSparsePer>(ids, n, mass, w, sm, V);
 }
 
 // Loads entries v0..v0+7 of a logit row as floats (-inf past V): 16-byte vector loads
