@@ -24,10 +24,9 @@
 // Top-k: the first threshold is a value that k entries of the first chunk reach (per-warp
 // order statistics of per-thread maxima; of vector maxima for k > 128). After the first
 // chunk the consumer warps exchange their counts, and a list of more than k entries sets the
-// threshold to the exact k-th seen so far (ranked directly, the list kept as it is). Further
-// exchanges run every (kCapTopK / 2) / k chunks, so about half the list can fill between
-// two even if every chunk brings k new entries; one past half the capacity is cut to its top
-// k. Rows whose values do not grow along the vocabulary rarely reach the threshold again, and
+// threshold to the exact k-th seen so far (ranked directly) and drops the entries below it.
+// Further exchanges run every (kCapTopK / 2) / k chunks, so about half the list can fill
+// between two even if every chunk brings k new entries. Rows whose values do not grow along the vocabulary rarely reach the threshold again, and
 // a list that still outgrows kCapTopK sends the row to the exact finisher. The short list
 // keeps a top-k CTA small enough for three per SM.
 //
@@ -610,7 +609,7 @@ struct CandSet {
       const uint64_t e = cand[i];
       if (e < lim) continue;
       int above = 0;
-      for (int j = 0; j < n; ++j) above += cand[j] > e ? 1 : 0;
+      for (int j = 0; j < n; ++j) above += cand[j] > e ? 1 : 0;  // (a fixed trip count)
       if (above == k - 1) *out = e;
     }
   }
@@ -1192,9 +1191,8 @@ __global__ void __launch_bounds__(kStreamThreads, (kMode == SM_TOPK ? SV_TOPK_CT
             keep = max(kKeepFloor, int((long long)kKeepTarget * seen / rj.V));
           }
           if constexpr (kMode == SM_TOPK) {
-            // the exact k-th of the entries seen so far becomes the threshold; a short list
-            // keeps the entries below it (the row-end selection ranks past them), one past
-            // half the capacity drops them
+            // the exact k-th of the entries seen so far becomes the threshold, and the list
+            // drops the entries below it
             bool have = false;
             if (cnt >= keep) {  // (uniform)
               cs.rank_into(cnt, 0, keep, &aux.sel_x[xp]);
@@ -1204,7 +1202,7 @@ __global__ void __launch_bounds__(kStreamThreads, (kMode == SM_TOPK ? SV_TOPK_CT
             if (have) {
               const uint64_t kth = aux.sel_x[xp];
               thr = fmaxf(thr, key_value<T>(comp_key(kth)));
-              if (cnt > kCapTopK / 2) cnt = cs.compact_ge(cnt, kth);
+              cnt = cs.compact_ge(cnt, kth);  // the row end then ranks a short list
             }
           } else if (keep < cnt) {
             cnt = cs.p_cut(cnt, keep, pbase, &lfloor, &thr);
