@@ -39,10 +39,11 @@ struct TreeJob {
 enum : int8_t { ND_REJECT = 0, ND_ACCEPT = 1, ND_ERROR = 2, ND_TIMEOUT = 3, ND_NEAR = 4 };
 
 // Relative distance of p from the typical threshold below which the test is re-taken in
-// double precision. The fp32 statistics err by far less: per-thread fp32 sums of at most
+// double precision. The fp32 statistics err by less: per-thread fp32 sums of at most
 // V / 256 + 16 terms (2^-24 each), ex2.approx and exponent roundings; they move p by under
-// 3e-4 relative and the entropy by under 3e-3 for V <= 2^20.
-constexpr float kTreeGuard = 3e-2f;
+// 3e-4 relative and the entropy by under 3e-3 (so the threshold by under 3e-3 relative) for
+// V <= 2^20: the guard leaves a factor of three.
+constexpr float kTreeGuard = 1e-2f;
 
 constexpr int kTreeMaxNodes = 4096;  // SPEC_MAX_TREE_NODES
 
@@ -119,7 +120,8 @@ __global__ void __launch_bounds__(kThreads) tree_finish_kernel(const TreeJob j) 
     test[c] = t;
   }
   __syncthreads();
-  if (!j.greedy) {  // tests too close to call in fp32: again in double, one at a time
+  if (!j.greedy) {  // tests too close to call in fp32: again in double, one parent row at a
+                    // time (its normaliser and entropy serve every child tested against it)
     __shared__ Fx128 zscr[kWarps];
     for (int c = 1; c < N; ++c) {
       if (test[c] != ND_NEAR) continue;  // uniform: test[] is in shared memory
@@ -128,25 +130,33 @@ __global__ void __launch_bounds__(kThreads) tree_finish_kernel(const TreeJob j) 
       const T* prow = rows + size_t(pa) * V;
       const bool al = (reinterpret_cast<uintptr_t>(prow) & 15u) == 0;
       Fx128 z = fx_zero(), h = fx_zero();
-      for (int v0 = int(threadIdx.x) * 8; v0 < V; v0 += kThreads * 8) {
-        float x[8];
-        load8<T>(prow, v0, V, al, x);
+      // four groups of 8 per thread, all loaded before any is used
+      for (int v00 = int(threadIdx.x) * 8; v00 < V; v00 += 4 * kThreads * 8) {
+        float x[4][8];
+        load8xG<T, 4>(prow, v00, kThreads * 8, V, al, x);
 #pragma unroll
-        for (int k = 0; k < 8; ++k) {
-          if (v0 + k >= V || !(x[k] > -INFINITY)) continue;
-          const double d = double(s.m) - double(x[k]);  // >= 0, exact
-          const double e = exp_neg(-d);
-          z = fx_add(z, fx_from(e));
-          h = fx_add(h, fx_from(e * d));
+        for (int g = 0; g < 4; ++g) {
+          const int v0 = v00 + g * kThreads * 8;
+#pragma unroll
+          for (int k = 0; k < 8; ++k) {
+            if (v0 + k >= V || !(x[g][k] > -INFINITY)) continue;
+            const double d = double(s.m) - double(x[g][k]);  // >= 0, exact
+            const double e = exp_neg(-d);
+            z = fx_add(z, fx_from(e));
+            h = fx_add(h, fx_from(e * d));
+          }
         }
       }
       const double zd = fx_to_double(block_sum_fx(z, zscr));
       const double hd = fx_to_double(block_sum_fx(h, zscr));
       if (threadIdx.x == 0) {
         const double H = log(zd) + hd / zd;  // -sum p ln p
-        const double p = exp(double(Elem<T>::load(prow, size_t(tok[c]))) - double(s.m)) / zd;
         const double thr = fmin(double(j.eps), double(j.delta) * exp(-H));
-        test[c] = p > thr ? ND_ACCEPT : ND_REJECT;
+        for (int c2 = c; c2 < N; ++c2) {  // this child and the later ones of the same parent
+          if (test[c2] != ND_NEAR || par[c2] != pa) continue;
+          const double p = exp(double(Elem<T>::load(prow, size_t(tok[c2]))) - double(s.m)) / zd;
+          test[c2] = p > thr ? ND_ACCEPT : ND_REJECT;
+        }
       }
       __syncthreads();
     }
