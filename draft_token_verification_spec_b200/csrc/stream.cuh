@@ -746,26 +746,30 @@ struct RowAcc {
           }
         }
         Elem<T>::unpack(ws, x);
-        float s1 = 0.0f, s2 = 0.0f;
+        // two chains, their exponents and additions in packed pairs
+        float2 s12 = make_float2(0.0f, 0.0f);
+        const float2 c2 = make_float2(c, c), m2 = make_float2(-mct, -mct);
 #pragma unroll
         for (int k = 0; k < P; k += 2) {
-          s1 += ex2(wexp(x[k], c, mct));
-          s2 += ex2(wexp(x[k + 1], c, mct));
+          const float2 z = ffma2(make_float2(x[k], x[k + 1]), c2, m2);
+          s12 = fadd2(s12, make_float2(ex2(z.x), ex2(z.y)));
         }
-        sfx += to_fx(s1 + s2);
+        sfx += to_fx(s12.x + s12.y);
       } else if (want_ent) {
         Elem<T>::unpack(w, x);
 #pragma unroll
         for (int k = 0; k < P; ++k) add(x[k], c, true);
       } else {
         Elem<T>::unpack(w, x);
-        float s2 = 0.0f;
+        // two chains (s and s2), their exponents and additions in packed pairs
+        float2 ss = make_float2(s, 0.0f);
+        const float2 c2 = make_float2(c, c), m2 = make_float2(-mct, -mct);
 #pragma unroll
         for (int k = 0; k < P; k += 2) {
-          s += ex2(wexp(x[k], c, mct));
-          s2 += ex2(wexp(x[k + 1], c, mct));
+          const float2 z = ffma2(make_float2(x[k], x[k + 1]), c2, m2);
+          ss = fadd2(ss, make_float2(ex2(z.x), ex2(z.y)));
         }
-        s += s2;
+        s = ss.x + ss.y;
       }
     }
     mt = fmax_nan(mt, vm);
