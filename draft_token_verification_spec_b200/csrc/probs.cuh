@@ -64,4 +64,60 @@ __global__ void __launch_bounds__(kThreads) residual_sample_kernel(const Residua
   if (threadIdx.x == 0) j.tokens[row] = tok;
 }
 
+// Probability rows from row statistics (spec_logits_to_probs after the streaming kernel):
+// p(v) = kept(v) ? exp2(l_v c - mc) / z : 0, NaN for rows whose statistics are not valid;
+// entropy[row] from the statistics. Work items are (row, segment of kProbsSeg entries),
+// numbered row * seg + segment; each thread takes 8 consecutive entries (one 16-byte load of
+// bfloat16 logits, two 16-byte stores). V % 8 == 0, rows 16-byte aligned.
+constexpr int kProbsSeg = 8 * kThreads;
+struct ProbsJob {
+  const void* logits;       // [rows][V] bfloat16
+  const RowStats* stats;    // [rows]
+  float* probs;             // [rows][V]
+  float* entropy;           // [rows] or NULL
+  long long item_begin, item_end;
+  int V, seg;               // seg = ceil(V / kProbsSeg)
+};
+
+__device__ __forceinline__ void probs_write8(const ProbsJob& j, const RowStats& s, long long row,
+                                             int v0) {
+  const uint4 w = __ldg(reinterpret_cast<const uint4*>(
+      static_cast<const __nv_bfloat16*>(j.logits) + size_t(row) * j.V + v0));
+  float x[8], o[8];
+  Elem<__nv_bfloat16>::unpack(w, x);
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    if (s.status != ROW_OK)
+      o[k] = NAN;
+    else
+      o[k] = kept(Elem<__nv_bfloat16>::key(x[k]), v0 + k, s.thr_key, s.cutoff)
+                 ? weight(x[k], s.c, s.mc) / s.z
+                 : 0.0f;
+  }
+  float4* out = reinterpret_cast<float4*>(j.probs + size_t(row) * j.V + v0);
+  out[0] = make_float4(o[0], o[1], o[2], o[3]);
+  out[1] = make_float4(o[4], o[5], o[6], o[7]);
+}
+
+// Items [item_begin, item_end); none of them may overwrite the statistics of its own rows.
+__global__ void __launch_bounds__(kThreads) probs_write_kernel(const ProbsJob j) {
+  for (long long it = j.item_begin + blockIdx.x; it < j.item_end; it += gridDim.x) {
+    const long long row = it / j.seg;
+    const int v0 = int(it - row * j.seg) * kProbsSeg + 8 * int(threadIdx.x);
+    const RowStats s = j.stats[row];
+    if (v0 < j.V) probs_write8(j, s, row, v0);
+    if (j.entropy && v0 == 0) j.entropy[row] = s.status != ROW_OK ? NAN : s.entropy;
+  }
+}
+
+// Item 0 (the first segment of row 0, which holds the statistics of the first rows): one
+// block reads row 0's statistics before it overwrites them.
+__global__ void __launch_bounds__(kThreads) probs_write_first_kernel(const ProbsJob j) {
+  const RowStats s = j.stats[0];
+  __syncthreads();
+  const int v0 = 8 * int(threadIdx.x);
+  if (v0 < j.V) probs_write8(j, s, 0, v0);
+  if (j.entropy && threadIdx.x == 0) j.entropy[0] = s.status != ROW_OK ? NAN : s.entropy;
+}
+
 }  // namespace sv

@@ -113,6 +113,7 @@ __global__ void __launch_bounds__(kFinThreads) topp_finalize_kernel(const Refine
   __shared__ uint32_t hcnt[kPBins];
   __shared__ uint32_t pmem[kPMem];
   __shared__ unsigned long long zred[kFinThreads / 32];
+  __shared__ long long s1red[kFinThreads / 32];
   CandSet<T> cs;
   cs.cand = nullptr;
   cs.ranked = nullptr;
@@ -142,14 +143,14 @@ __global__ void __launch_bounds__(kFinThreads) topp_finalize_kernel(const Refine
     for (int i = threadIdx.x; i < kPBins; i += kFinThreads) hcnt[i] = 0u;
     if (threadIdx.x == 0) aux.ccount = 0;
     __syncthreads();
-    // four groups of 8 per thread in flight; every thread takes the same number of rounds
+    // two groups of 8 per thread in flight; every thread takes the same number of rounds
     // (the warp-level appends below need all lanes)
-    for (int r0 = 0; r0 < V; r0 += 4 * kFinThreads * 8) {
+    for (int r0 = 0; r0 < V; r0 += 2 * kFinThreads * 8) {
       const int v00 = r0 + int(threadIdx.x) * 8;
-      float x[4][8];
-      load8xG<T, 4>(src, v00, kFinThreads * 8, V, al, x);
+      float x[2][8];
+      load8xG<T, 2>(src, v00, kFinThreads * 8, V, al, x);
 #pragma unroll
-      for (int g = 0; g < 4; ++g) {
+      for (int g = 0; g < 2; ++g) {
         const int v0 = v00 + g * kFinThreads * 8;
         uint32_t mk = 0u;
 #pragma unroll
@@ -206,9 +207,14 @@ __global__ void __launch_bounds__(kFinThreads) topp_finalize_kernel(const Refine
     // kept ids and the fp32 normaliser: the codes above the crossing code by every thread,
     // the crossing code's entries gathered, then the j with the lowest ids by warp 0
     int32_t* kids = rj.kept_ids ? rj.kept_ids + size_t(row) * kKeptCap : nullptr;
+    const bool want_ent = (rj.flags & RS_ENTROPY) != 0;
     unsigned long long z = 0;
+    long long s1 = 0;
     auto keep = [&](uint32_t e) {
-      z += to_fx(weight(key_value<T>(base + pcomp_rel(e)), rs.c, rs.mc));
+      const float zx = wexp(key_value<T>(base + pcomp_rel(e)), rs.c, rs.mc);
+      const float ex = ex2(zx);
+      z += to_fx(ex);
+      if (want_ent) s1 += __float2ll_rn(ent_term(ex, zx) * kS1Fx);
       const int slot = atomicAdd(&aux.mcount, 1);
       if (kids && slot < kKeptCap) kids[slot] = pcomp_id(e);
     };
@@ -243,19 +249,32 @@ __global__ void __launch_bounds__(kFinThreads) topp_finalize_kernel(const Refine
       if (g && lane == __ffs(g) - 1) aux.sel_c32 = cst;
     }
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
-    if (lane == 0) zred[warp] = z;
+    for (int o = 16; o > 0; o >>= 1) {
+      z += __shfl_xor_sync(0xffffffffu, z, o);
+      s1 += __shfl_xor_sync(0xffffffffu, s1, o);
+    }
+    if (lane == 0) {
+      zred[warp] = z;
+      s1red[warp] = s1;
+    }
     __syncthreads();
     if (threadIdx.x == 0) {
       unsigned long long zf = 0;
-      for (int w = 0; w < kFinThreads / 32; ++w) zf += zred[w];
+      long long s1a = 0;
+      for (int w = 0; w < kFinThreads / 32; ++w) {
+        zf += zred[w];
+        s1a += s1red[w];
+      }
       if (aux.sel_found) {
         const uint32_t cstar = aux.sel_c32;
         RowStats out = rs;
         out.thr_key = base + pcomp_rel(cstar);
         out.cutoff = pcomp_id(cstar);
         out.zd = aux.sel_above;
-        out.z = float(double(zf) * kFxInv);
+        const double Z = double(zf) * kFxInv;
+        out.z = float(Z);
+        if (want_ent)
+          out.entropy = float(log(Z) - 0.6931471805599453 * (double(s1a) / double(kS1Fx)) / Z);
         rj.stats[row] = out;
         if (rj.kept_n) rj.kept_n[row] = (kids && aux.mcount <= kKeptCap) ? aux.mcount : 0;
       } else {

@@ -634,6 +634,7 @@ spec_status spec_logits_to_probs(const void* logits, spec_dtype dtype, int rows,
   RowPlan pl;
   if (!plan_rows(V, elem_bytes(dtype), &pl) || !rows_fit(rows, pl.C)) return SPEC_ERR_UNSUPPORTED;
   const bool greedy = temp == 0.0f;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
   sv::RowJob rj = {};
   rj.base0 = logits;
   rj.base1 = logits;
@@ -647,13 +648,60 @@ spec_status spec_logits_to_probs(const void* logits, spec_dtype dtype, int rows,
   rj.temp = temp;
   rj.top_k = (top_k >= 1 && top_k < V) ? top_k : 0;
   rj.top_p = top_p < 1.0f ? top_p : 1.0f;
-  rj.flags = sv::RS_WRITE_PROBS | (greedy ? sv::RS_GREEDY : 0) |
-             ((entropy && !greedy) ? sv::RS_ENTROPY : 0);
-  rj.stats = nullptr;
-  rj.probs = probs;
-  rj.entropy = entropy;
   rj.dev_status = nullptr;
-  return check_launch(launch_row_stats_dt(dtype, rj, pl, static_cast<cudaStream_t>(stream)));
+  // bfloat16 rows: the row statistics by the streaming kernel (with its exact finisher and
+  // the exact top-p placement), kept in the probability buffer itself (its first `head` rows),
+  // then the probabilities in three launches: the rows past the head (their statistics are not
+  // overwritten meanwhile), the head rows but for row 0's first segment (which holds the head
+  // rows' statistics), and that segment
+  const long long R = rows;
+  const size_t o_stats = kStatsOffset;
+  const size_t o_fb = o_stats + up256(size_t(R) * sizeof(sv::RowStats));
+  const size_t o_ref = o_fb + up256(size_t(R) * sizeof(int32_t));
+  const size_t o_refz = o_ref + up256(size_t(R) * sizeof(int32_t));
+  const size_t scratch = o_refz + up256(size_t(R) * 2 * sizeof(unsigned long long));
+  const long long head = (long long)((scratch + size_t(V) * 4 - 1) / (size_t(V) * 4));
+  const bool streamed = dtype == SPEC_BF16 && !greedy && V % 8 == 0 && V >= sv::kProbsSeg &&
+                        aligned16(logits) && aligned16(probs) &&
+                        scratch <= size_t(R) * V * 4 &&
+                        o_stats + size_t(head) * sizeof(sv::RowStats) <= size_t(sv::kProbsSeg) * 4;
+  if (!streamed) {
+    rj.flags = sv::RS_WRITE_PROBS | (greedy ? sv::RS_GREEDY : 0) |
+               ((entropy && !greedy) ? sv::RS_ENTROPY : 0);
+    rj.stats = nullptr;
+    rj.probs = probs;
+    rj.entropy = entropy;
+    return check_launch(launch_row_stats_dt(dtype, rj, pl, s));
+  }
+  char* ws = reinterpret_cast<char*>(probs);
+  int32_t* hdr = reinterpret_cast<int32_t*>(ws);
+  if (cudaMemsetAsync(hdr, 0, kHeaderWords * sizeof(int32_t), s) != cudaSuccess)
+    return SPEC_ERR_CUDA;
+  rj.flags = entropy ? sv::RS_ENTROPY : 0;
+  rj.stats = reinterpret_cast<sv::RowStats*>(ws + o_stats);
+  rj.dev_status = hdr;
+  if (row_stage(dtype, rj, pl, reinterpret_cast<int32_t*>(ws + o_fb), hdr + 1,
+                reinterpret_cast<int32_t*>(ws + o_ref), hdr + 3,
+                reinterpret_cast<unsigned long long*>(ws + o_refz), hdr + 4, s) != cudaSuccess)
+    return SPEC_ERR_CUDA;
+  int dev = 0, sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    return SPEC_ERR_CUDA;
+  const int seg = (V + sv::kProbsSeg - 1) / sv::kProbsSeg;
+  sv::ProbsJob pj = {logits, rj.stats, probs, entropy, head * seg, R * seg, V, seg};
+  for (int part = 0; part < 2; ++part) {
+    const long long items = pj.item_end - pj.item_begin;
+    if (items > 0) {
+      const long long g = items < 8LL * sms ? items : 8LL * sms;
+      sv::probs_write_kernel<<<unsigned(g), kThreads, 0, s>>>(pj);
+      if (cudaGetLastError() != cudaSuccess) return SPEC_ERR_CUDA;
+    }
+    pj.item_begin = 1;
+    pj.item_end = (head < R ? head : R) * seg;
+  }
+  sv::probs_write_first_kernel<<<1, kThreads, 0, s>>>(pj);
+  return check_launch(cudaGetLastError());
 }
 
 spec_status spec_residual_sample(const float* p, const float* q, int rows, int V,

@@ -506,6 +506,35 @@ def test_logits_to_probs(dtype, V, temp, top_k, top_p):
     np.testing.assert_allclose(eg[clear], er[clear], rtol=1e-5, atol=1e-6)
 
 
+@pytest.mark.parametrize("V", [2048, 2056])
+@pytest.mark.parametrize("temp,top_k,top_p", [(1.0, 0, 1.0), (0.8, 50, 1.0), (1.0, 0, 0.9)])
+def test_logits_to_probs_many_rows(V, temp, top_k, top_p):
+    """Hundreds of bfloat16 rows: the row statistics then span several probability rows (the
+    first rows of the output are written last), and invalid rows sit among them."""
+    g = np.random.default_rng(V + top_k)
+    rows = 300
+    x = g.normal(0, 3, (rows, V)).astype(np.float32)
+    x[5, :3] = 30.0
+    logits = specgen.f32_to_bf16_bits(x)
+    logits[0, 7] = 0x7FC0                                  # NaN: row 0 invalid
+    logits[2, :] = 0xFF80                                  # all -inf: row 2 invalid
+    logits[rows - 1, V - 1] = 0x7FC0
+    probs, ent = sv.spec_logits_to_probs(dev(logits), temp, top_k, top_p)
+    torch.cuda.synchronize()
+    pg, eg = probs.cpu().numpy().astype(np.float64), ent.cpu().numpy().astype(np.float64)
+    pr, er, marg, valid = oracle.transform_rows(logits, temp, top_k, top_p)
+    valid = valid.astype(bool)
+    assert not valid[[0, 2, rows - 1]].any() and valid.sum() == rows - 3
+    assert np.isnan(pg[~valid]).all() and np.isnan(eg[~valid]).all()
+    clear = valid & (marg >= 1e-6)
+    assert clear.sum() >= rows - 6
+    big = pr > 1e-30
+    err = np.abs(pg - pr)
+    assert np.all((err <= 1e-5 * pr) | ~big | ~clear[:, None]), err[big & clear[:, None]].max()
+    assert np.all(pg[valid][~big[valid]] < 1e-30)
+    np.testing.assert_allclose(eg[clear], er[clear], rtol=1e-5, atol=1e-6)
+
+
 def test_logits_to_probs_invalid_rows_are_nan():
     x = np.zeros((3, 64), np.float32)
     x[1, 3] = np.nan
