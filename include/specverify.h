@@ -174,7 +174,10 @@ spec_status spec_verify_tree_sampling(const void* target_logits, const void* dra
  *   logits [rows][V]; probs [rows][V] float out: the transformed distribution
  *   (temp == 0: one-hot at the argmax); entropy [rows] float out or NULL: its
  *   entropy in nats. Rows that hold NaN or +inf, or are entirely -inf, get NaN
- *   probabilities and entropy. rows >= 1. */
+ *   probabilities and entropy. rows >= 1. probs must not overlap logits or entropy: the
+ *   call also uses the probs buffer as its scratch space (bfloat16 rows keep their row
+ *   statistics there until the probabilities overwrite them), so its contents are defined
+ *   only once the call's work on the stream has finished. */
 spec_status spec_logits_to_probs(const void* logits, spec_dtype dtype, int rows, int V,
                                  float temp, int top_k, float top_p, float* probs,
                                  float* entropy, void* stream);
