@@ -132,11 +132,13 @@ constexpr int kStreamMaxTopK = 256;             // top-k the candidate path take
 // to that sum, in weights exp((l - m) / T) (max 1). Per entry of depth d = (m - l) log2(e) /
 // T log2 units: c = fl(log2(e) / T) is off by 3 * 2^-24 at most (d * 3 * 2^-24 in the
 // exponent), the exponent fl(l c - r) by 2^-24 of (d + 1), ex2.approx by 2^-22 relative,
-// and the per-vector fp32 sum by 4 * 2^-24; entries with d <= 32 are thus within
-// ln2 * 2^-24 * (4 * 32 + 1) + 2^-22 + 4 * 2^-24 = 5.9e-6 of their weight, and the rest (each
-// below 2^-32, at most 2^20 of them) are off by under 1.5e-9 in all. The fixed-point sums
-// add at most 2^-42 per vector and per reference shift (kPGuardFxUnit).
-constexpr double kPGuardRel = 6.0e-6;
+// and the fp32 sum of a thread's share of a chunk (4 roundings within a vector, one per
+// further vector: at most 10) by 10 * 2^-24; entries with d <= 32 are thus within
+// ln2 * 2^-24 * (4 * 32 + 1) + 2^-22 + 10 * 2^-24 = 6.17e-6 of their weight, and the rest
+// (each below 2^-32, at most 2^20 of them) are off by under 1.5e-9 in all. The fixed-point
+// sums add at most 2^-42 per conversion (one per chunk and thread with a sum, and one per
+// reference shift: fewer than one per vector) and per shift (kPGuardFxUnit).
+constexpr double kPGuardRel = 6.2e-6;
 constexpr double kPGuardAbs = 2.0e-9;
 constexpr double kPGuardFxUnit = 2.2737367544323206e-13;  // 2^-42
 
@@ -649,12 +651,19 @@ struct RowAcc {
   float mct;  // the online sums are relative to it: fl(mt * c); top-p: ceil(fl(mt * c))
   float s, h; // online weight sum and entropy term (log2 units)
   // top-p: the online weight sum of the entries below the candidate threshold as 42-bit
-  // fixed point, relative to the integer reference mct. Each vector's weights are summed in
-  // fp32 and added exactly; a reference that rises by d shifts the sum right by d bits (the
+  // fixed point, relative to the integer reference mct. A thread's weights of one chunk are
+  // summed in fp32 (sp) and added exactly; a reference that rises by d shifts the sum right by
+  // d bits (the
   // exact power of two, truncated below 2^-42), so the sum's error stays within a few fp32
   // roundings per weight (the bound kPGuardRel states) with no floating-point rescale in the
   // loop.
   unsigned long long sfx;
+  float sp;  // top-p: the fp32 sum not yet added to sfx
+
+  __device__ __forceinline__ void flush() {
+    sfx += to_fx(sp);
+    sp = 0.0f;
+  }
 
   __device__ void reset() {
     mt = -INFINITY;
@@ -663,6 +672,7 @@ struct RowAcc {
     s = 0.0f;
     h = 0.0f;
     sfx = 0ull;
+    sp = 0.0f;
   }
 
   // Raises the running maximum to vm (> mt), rescaling the online sums.
@@ -670,6 +680,7 @@ struct RowAcc {
     const float nm = vm * c;
     if constexpr (kMode == SM_TOPP) {
       const float nr = ceilf(nm);
+      flush();
       if (sfx == 0ull) {
         mct = nr;
       } else if (nr > mct) {
@@ -699,8 +710,10 @@ struct RowAcc {
   }
 
   // One 16-byte vector whose first element has row index j0 (entries outside the chunk
-  // hold -inf). vm = its largest value. Top-p: returns the mask of its entries >= t (the
-  // candidates, bit k for entry k), which the sums leave out; 0 in the other modes.
+  // hold -inf). vm = its largest value; the sums' reference already covers it (the caller
+  // raises it to the chunk's maximum first, so the vectors of a chunk carry no dependence
+  // through it). Top-p: returns the mask of its entries >= t (the candidates, bit k for
+  // entry k), which the sums leave out; 0 in the other modes.
   __device__ __forceinline__ uint32_t vec(const uint4& w, float vm, int j0, float c,
                                           bool want_ent, float t) {
     constexpr int P = Elem<T>::kPerVec;
@@ -718,7 +731,6 @@ struct RowAcc {
           if (x[k] == vm) am = j0 + k;
       }
     } else if constexpr (kSums) {
-      if (vm > mt) raise_max(vm, c);
       float x[P];
       if constexpr (kMode == SM_TOPP) {
         // candidates become -inf (weight 0) in the copy the sums read
@@ -754,7 +766,7 @@ struct RowAcc {
           const float2 z = ffma2(make_float2(x[k], x[k + 1]), c2, m2);
           s12 = fadd2(s12, make_float2(ex2(z.x), ex2(z.y)));
         }
-        sfx += to_fx(s12.x + s12.y);
+        sp += s12.x + s12.y;
       } else if (want_ent) {
         Elem<T>::unpack(w, x);
 #pragma unroll
@@ -1009,6 +1021,14 @@ __global__ void __launch_bounds__(kStreamThreads, (kMode == SM_TOPK ? SV_TOPK_CT
     }
 
     // ---- the chunk pass
+    if constexpr (RowAcc<T, kMode>::kSums) {
+      // the sums' reference rises once per chunk, to the largest value of this thread's
+      // vectors (fmaxf passes over a NaN; such a row is invalid)
+      float cmax = -INFINITY;
+#pragma unroll
+      for (int u = 0; u < kVecPerThread; ++u) cmax = fmaxf(cmax, vm[u]);
+      if (cmax > st.mt) st.raise_max(cmax, c);
+    }
     float vmax4 = -INFINITY;
 #pragma unroll
     for (int u = 0; u < kVecPerThread; ++u) {
@@ -1018,6 +1038,7 @@ __global__ void __launch_bounds__(kStreamThreads, (kMode == SM_TOPK ? SV_TOPK_CT
                      (v >= v_lo && v < v_hi) ? thr : INFINITY);
       vmax4 = fmaxf(vmax4, vm[u]);  // pad vectors hold -inf; NaN never passes a filter
     }
+    if constexpr (kMode == SM_TOPP) st.flush();
     int wadd = 0;  // entries this warp appended in this chunk (uniform in the warp)
     if constexpr (kMode == SM_TOPK) {
       // the candidates' bits, from the ring again (most vectors hold none)
