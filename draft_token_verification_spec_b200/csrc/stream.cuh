@@ -733,9 +733,11 @@ struct RowAcc {
     } else if constexpr (kSums) {
       float x[P];
       if constexpr (kMode == SM_TOPP) {
-        // candidates become -inf (weight 0) in the copy the sums read
+        // candidates become -inf (weight 0) in the copy the sums read; bfloat16 vectors take
+        // the packed compares whether or not they hold one (four compares and selects cost
+        // less than a branch between the vectors of a chunk)
         uint4 ws = w;
-        if (vm >= t) {
+        if (sizeof(T) == 2 || vm >= t) {
           if constexpr (sizeof(T) == 2) {
             const __nv_bfloat162 tt = __float2bfloat162_rn(t);  // t is a bfloat16 value
             uint32_t a[4] = {w.x, w.y, w.z, w.w};
