@@ -66,57 +66,73 @@ __global__ void __launch_bounds__(kThreads) residual_sample_kernel(const Residua
 
 // Probability rows from row statistics (spec_logits_to_probs after the streaming kernel):
 // p(v) = kept(v) ? exp2(l_v c - mc) / z : 0, NaN for rows whose statistics are not valid;
-// entropy[row] from the statistics. Work items are (row, segment of kProbsSeg entries),
-// numbered row * seg + segment; each thread takes 8 consecutive entries (one 16-byte load of
-// bfloat16 logits, two 16-byte stores). V % 8 == 0, rows 16-byte aligned.
-constexpr int kProbsSeg = 8 * kThreads;
+// entropy[row] from the statistics. A row is cut into segments of kProbsSeg entries; block
+// (x, y) of the grid writes segment x of rows r_begin + y, r_begin + y + gridDim.y, ... Each
+// thread loads its kProbsVecs 16-byte vectors of bfloat16 logits (8 entries each, kThreads
+// vectors apart) before it computes and stores any, so that several loads are in flight.
+// V % 8 == 0, rows 16-byte aligned.
+constexpr int kProbsVecs = 4;
+constexpr int kProbsSeg = 8 * kProbsVecs * kThreads;  // 8,192 entries
 struct ProbsJob {
   const void* logits;       // [rows][V] bfloat16
   const RowStats* stats;    // [rows]
   float* probs;             // [rows][V]
   float* entropy;           // [rows] or NULL
-  long long item_begin, item_end;
-  int V, seg;               // seg = ceil(V / kProbsSeg)
+  long long r_begin, r_end;
+  long long skip_row;       // the row whose first segment the launch leaves out, or -1
+  int V;
 };
 
-__device__ __forceinline__ void probs_write8(const ProbsJob& j, const RowStats& s, long long row,
-                                             int v0) {
-  const uint4 w = __ldg(reinterpret_cast<const uint4*>(
-      static_cast<const __nv_bfloat16*>(j.logits) + size_t(row) * j.V + v0));
-  float x[8], o[8];
-  Elem<__nv_bfloat16>::unpack(w, x);
+__device__ __forceinline__ void probs_write_seg(const ProbsJob& j, const RowStats& s,
+                                                long long row, int v_base) {
+  const __nv_bfloat16* lg = static_cast<const __nv_bfloat16*>(j.logits) + size_t(row) * j.V;
+  float* out = j.probs + size_t(row) * j.V;
+  uint4 w[kProbsVecs];
 #pragma unroll
-  for (int k = 0; k < 8; ++k) {
-    if (s.status != ROW_OK)
-      o[k] = NAN;
-    else
-      o[k] = kept(Elem<__nv_bfloat16>::key(x[k]), v0 + k, s.thr_key, s.cutoff)
-                 ? weight(x[k], s.c, s.mc) / s.z
-                 : 0.0f;
+  for (int u = 0; u < kProbsVecs; ++u) {
+    const int v0 = v_base + u * 8 * kThreads;
+    w[u] = v0 < j.V ? __ldg(reinterpret_cast<const uint4*>(lg + v0)) : make_uint4(0, 0, 0, 0);
   }
-  float4* out = reinterpret_cast<float4*>(j.probs + size_t(row) * j.V + v0);
-  out[0] = make_float4(o[0], o[1], o[2], o[3]);
-  out[1] = make_float4(o[4], o[5], o[6], o[7]);
+#pragma unroll
+  for (int u = 0; u < kProbsVecs; ++u) {
+    const int v0 = v_base + u * 8 * kThreads;
+    if (v0 >= j.V) continue;
+    float x[8], o[8];
+    Elem<__nv_bfloat16>::unpack(w[u], x);
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      if (s.status != ROW_OK)
+        o[k] = NAN;
+      else
+        o[k] = kept(Elem<__nv_bfloat16>::key(x[k]), v0 + k, s.thr_key, s.cutoff)
+                   ? weight(x[k], s.c, s.mc) / s.z
+                   : 0.0f;
+    }
+    float4* o4 = reinterpret_cast<float4*>(out + v0);
+    o4[0] = make_float4(o[0], o[1], o[2], o[3]);
+    o4[1] = make_float4(o[4], o[5], o[6], o[7]);
+  }
 }
 
-// Items [item_begin, item_end); none of them may overwrite the statistics of its own rows.
+// Rows [r_begin, r_end) but the first segment of skip_row; no block may overwrite the
+// statistics of a row it writes.
 __global__ void __launch_bounds__(kThreads) probs_write_kernel(const ProbsJob j) {
-  for (long long it = j.item_begin + blockIdx.x; it < j.item_end; it += gridDim.x) {
-    const long long row = it / j.seg;
-    const int v0 = int(it - row * j.seg) * kProbsSeg + 8 * int(threadIdx.x);
+  const int v_base = int(blockIdx.x) * kProbsSeg + 8 * int(threadIdx.x);
+  for (long long row = j.r_begin + blockIdx.y; row < j.r_end; row += gridDim.y) {
+    if (row == j.skip_row && blockIdx.x == 0) continue;
     const RowStats s = j.stats[row];
-    if (v0 < j.V) probs_write8(j, s, row, v0);
-    if (j.entropy && v0 == 0) j.entropy[row] = s.status != ROW_OK ? NAN : s.entropy;
+    probs_write_seg(j, s, row, v_base);
+    if (j.entropy && blockIdx.x == 0 && threadIdx.x == 0)
+      j.entropy[row] = s.status != ROW_OK ? NAN : s.entropy;
   }
 }
 
-// Item 0 (the first segment of row 0, which holds the statistics of the first rows): one
-// block reads row 0's statistics before it overwrites them.
+// The first segment of row 0, which holds the statistics of the first rows: one block reads
+// row 0's statistics before it overwrites them.
 __global__ void __launch_bounds__(kThreads) probs_write_first_kernel(const ProbsJob j) {
   const RowStats s = j.stats[0];
   __syncthreads();
-  const int v0 = 8 * int(threadIdx.x);
-  if (v0 < j.V) probs_write8(j, s, 0, v0);
+  probs_write_seg(j, s, 0, 8 * int(threadIdx.x));
   if (j.entropy && threadIdx.x == 0) j.entropy[0] = s.status != ROW_OK ? NAN : s.entropy;
 }
 

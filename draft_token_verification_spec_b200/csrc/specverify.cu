@@ -653,7 +653,7 @@ spec_status spec_logits_to_probs(const void* logits, spec_dtype dtype, int rows,
   // the exact top-p placement), kept in the probability buffer itself (its first `head` rows),
   // then the probabilities in three launches: the rows past the head (their statistics are not
   // overwritten meanwhile), the head rows but for row 0's first segment (which holds the head
-  // rows' statistics), and that segment
+  // rows' statistics: kStatsOffset + head * sizeof(RowStats) bytes at most), and that segment
   const long long R = rows;
   const size_t o_stats = kStatsOffset;
   const size_t o_fb = o_stats + up256(size_t(R) * sizeof(sv::RowStats));
@@ -661,10 +661,11 @@ spec_status spec_logits_to_probs(const void* logits, spec_dtype dtype, int rows,
   const size_t o_refz = o_ref + up256(size_t(R) * sizeof(int32_t));
   const size_t scratch = o_refz + up256(size_t(R) * 2 * sizeof(unsigned long long));
   const long long head = (long long)((scratch + size_t(V) * 4 - 1) / (size_t(V) * 4));
-  const bool streamed = dtype == SPEC_BF16 && !greedy && V % 8 == 0 && V >= sv::kProbsSeg &&
+  const size_t seg0_bytes = size_t(V < sv::kProbsSeg ? V : sv::kProbsSeg) * 4;
+  const bool streamed = dtype == SPEC_BF16 && !greedy && V % 8 == 0 && V >= 2048 &&
                         aligned16(logits) && aligned16(probs) &&
                         scratch <= size_t(R) * V * 4 &&
-                        o_stats + size_t(head) * sizeof(sv::RowStats) <= size_t(sv::kProbsSeg) * 4;
+                        o_stats + size_t(head) * sizeof(sv::RowStats) <= seg0_bytes;
   if (!streamed) {
     rj.flags = sv::RS_WRITE_PROBS | (greedy ? sv::RS_GREEDY : 0) |
                ((entropy && !greedy) ? sv::RS_ENTROPY : 0);
@@ -689,16 +690,20 @@ spec_status spec_logits_to_probs(const void* logits, spec_dtype dtype, int rows,
       cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
     return SPEC_ERR_CUDA;
   const int seg = (V + sv::kProbsSeg - 1) / sv::kProbsSeg;
-  sv::ProbsJob pj = {logits, rj.stats, probs, entropy, head * seg, R * seg, V, seg};
+  sv::ProbsJob pj = {logits, rj.stats, probs, entropy, head, R, -1, V};
   for (int part = 0; part < 2; ++part) {
-    const long long items = pj.item_end - pj.item_begin;
-    if (items > 0) {
-      const long long g = items < 8LL * sms ? items : 8LL * sms;
-      sv::probs_write_kernel<<<unsigned(g), kThreads, 0, s>>>(pj);
+    const long long n = pj.r_end - pj.r_begin;
+    if (n > 0) {
+      // about 16 blocks per SM in all, 65,535 row groups at most
+      long long gy = (16LL * sms + seg - 1) / seg;
+      gy = gy < n ? gy : n;
+      gy = gy < 65535 ? gy : 65535;
+      sv::probs_write_kernel<<<dim3(unsigned(seg), unsigned(gy)), kThreads, 0, s>>>(pj);
       if (cudaGetLastError() != cudaSuccess) return SPEC_ERR_CUDA;
     }
-    pj.item_begin = 1;
-    pj.item_end = (head < R ? head : R) * seg;
+    pj.r_begin = 0;
+    pj.r_end = head < R ? head : R;
+    pj.skip_row = 0;
   }
   sv::probs_write_first_kernel<<<1, kThreads, 0, s>>>(pj);
   return check_launch(cudaGetLastError());
