@@ -86,3 +86,38 @@ def test_noalloc_rejects_logits_off_the_current_device(cuda_device):
         ctypes.c_void_p(acc.data_ptr()), ctypes.c_void_p(out.data_ptr()), None)
     assert rc == sv.SPEC_ERR_INVALID_ARG
     torch.cuda.synchronize()  # nothing was launched, and the context is healthy
+
+
+@pytest.mark.parametrize("cfg", [specgen.CFG5, specgen.CFG3], ids=["topk", "topp"])
+def test_noalloc_call_captures_into_a_cuda_graph(cuda_device, cfg):
+    """After one ordinary call, the no-alloc entry point records into a CUDA graph (global
+    capture mode: an allocating or synchronising call inside would end the capture with an
+    error), and every replay verifies the logits the buffers hold at that moment."""
+    tg, dg, x, u = _inputs(cfg, 8, cuda_device)
+    ref = sv.spec_verify_chain(tg, dg, x, u, cfg.temp, cfg.top_k, cfg.top_p)
+    acc = torch.empty_like(ref[0])
+    out = torch.empty_like(ref[1])
+    sv.spec_verify_chain_noalloc(tg, dg, x, u, cfg.temp, cfg.top_k, cfg.top_p,
+                                 accepted_len=acc, out_tokens=out)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        sv.spec_verify_chain_noalloc(tg, dg, x, u, cfg.temp, cfg.top_k, cfg.top_p,
+                                     accepted_len=acc, out_tokens=out)
+    acc.fill_(-7)
+    out.fill_(-7)
+    g.replay()
+    torch.cuda.synchronize()
+    assert torch.equal(acc, ref[0]) and torch.equal(out, ref[1])
+    # new inputs in the same buffers: the replay verifies them, not the captured values
+    tg2, dg2, x2, u2 = _inputs(cfg, 8, cuda_device)
+    u2.copy_(torch.flip(u2, dims=[0]))
+    ref2 = sv.spec_verify_chain(tg2, dg2, x2, u2, cfg.temp, cfg.top_k, cfg.top_p)
+    tg.copy_(tg2)
+    dg.copy_(dg2)
+    x.copy_(x2)
+    u.copy_(u2)
+    g.replay()
+    torch.cuda.synchronize()
+    assert torch.equal(acc, ref2[0]) and torch.equal(out, ref2[1])
+    del g
