@@ -17,8 +17,9 @@
 //   lstate_factors_kernel: one block per (sequence, head); the Gram products k_t . k_s, the
 //     gates G_t, then w_t and u_t in step order (each step parallel over dk or dv).
 //   lstate_commit_kernel: one block per (sequence, head, 64-column tile of S); the tile stays
-//     in registers: M = U_a - W_a S_0 (a x 64; each warp owns 8 columns and reduces its
-//     16 row lanes by shuffles), then S_a = G_a (S_0 + K_a^T M), written back in place. A
+//     in registers: M = U_a - W_a S_0 (a x 64; partial sums per thread over its rows, then
+//     over the warp's two row groups and the eight warps), then S_a = G_a (S_0 + K_a^T M),
+//     written back in place. A
 //     sequence committing 0 steps (or an invalid length) is not touched. Bandwidth-bound:
 //     one read and one write of the state per committed sequence.
 #pragma once
@@ -103,10 +104,14 @@ struct LsCommitJob {
   int tiles;            // column tiles per head: ceil(dv / kLsCols)
 };
 
-// R rows of S per lane: dk = 16 R (16 row lanes per warp).
-// Dynamic shared memory: keys and w of S steps (S x dk each), then M (S x kLsCols).
+// Thread layout of a commit block: 16 column quads (64 columns) x 16 row groups; the thread
+// with quad q = tid % 16 and row group g = tid / 16 holds rows g, g + 16, ..., g + 16 (R - 1)
+// (dk = 16 R) of columns 4q .. 4q + 3 of the tile. A warp's load or store of one of its rows
+// then covers two whole 256-byte row segments of the tile.
+// Dynamic shared memory: keys and w of S steps (S x dk each), M (S x kLsCols), and the warps'
+// partial sums of M (S x kWarps x kLsCols).
 __host__ __device__ constexpr size_t lstate_commit_smem(int S, int dk) {
-  return size_t(S) * dk * 8 + size_t(S) * kLsCols * 4;
+  return size_t(S) * dk * 8 + size_t(S) * kLsCols * 4 + size_t(S) * kWarps * kLsCols * 4;
 }
 
 // 16-byte global -> shared copy that bypasses the registers (and L1).
@@ -122,6 +127,8 @@ __global__ void __launch_bounds__(kThreads) lstate_commit_kernel(const LsCommitJ
   float* ks = lsm;                                            // [S][dk]
   float* ws = ks + size_t(j.S) * dk;                          // [S][dk]
   float (*mt)[kLsCols] = reinterpret_cast<float (*)[kLsCols]>(ws + size_t(j.S) * dk);
+  float4* red = reinterpret_cast<float4*>(ws + size_t(j.S) * dk + size_t(j.S) * kLsCols);
+  // red[(t * kWarps + warp) * 16 + q]: warp's partial sum of M[t][4q .. 4q + 3]
   const long long blk = blockIdx.x;
   const int tile = int(blk % j.tiles);
   const long long bh = blk / j.tiles;
@@ -152,61 +159,70 @@ __global__ void __launch_bounds__(kThreads) lstate_commit_kernel(const LsCommitJ
   }
   const float ga = j.gamma[size_t(bh) * S + a - 1];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int rl = lane & 15;                          // row lane: rows rl, rl + 16, ...
-  const int cl = warp * 8 + (lane >> 4) * 4;         // first of this lane's 4 columns (in tile)
-  const int col = c0 + cl;
+  const int q = threadIdx.x & 15;                    // column quad: columns 4q .. 4q + 3
+  const int rg = threadIdx.x >> 4;                   // row group: rows rg, rg + 16, ...
+  const int col = c0 + 4 * q;
   const bool live = col < dv;                        // dv % 4 == 0: a quad is all in or out
   float* base = j.state + size_t(bh) * dk * dv;
   float4 x[R];
 #pragma unroll
   for (int r = 0; r < R; ++r)
-    x[r] = live ? *reinterpret_cast<const float4*>(base + size_t(rl + 16 * r) * dv + col)
+    x[r] = live ? *reinterpret_cast<const float4*>(base + size_t(rg + 16 * r) * dv + col)
                 : make_float4(0.f, 0.f, 0.f, 0.f);
   asm volatile("cp.async.wait_all;" ::: "memory");
   __syncthreads();
-  // M[t][c] = U[t][c] - sum_i W[t][i] S[i][c]: partial sums over this lane's rows, then the
-  // 16 row lanes of the warp (xor shuffles keep them within the half-warp)
+  // M[t][c] = U[t][c] - sum_i W[t][i] S[i][c]: partial sums over this thread's rows, the two
+  // row groups of the warp (lanes l and l ^ 16), then the warps' sums in warp order
   for (int t = 0; t < a; ++t) {
     float4 p = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
     for (int r = 0; r < R; ++r) {
-      const float wv = ws[t * dk + rl + 16 * r];
+      const float wv = ws[t * dk + rg + 16 * r];
       p.x = fmaf(wv, x[r].x, p.x);
       p.y = fmaf(wv, x[r].y, p.y);
       p.z = fmaf(wv, x[r].z, p.z);
       p.w = fmaf(wv, x[r].w, p.w);
     }
-#pragma unroll
-    for (int o = 1; o < 16; o <<= 1) {
-      p.x += __shfl_xor_sync(0xffffffffu, p.x, o);
-      p.y += __shfl_xor_sync(0xffffffffu, p.y, o);
-      p.z += __shfl_xor_sync(0xffffffffu, p.z, o);
-      p.w += __shfl_xor_sync(0xffffffffu, p.w, o);
-    }
-    if (rl == 0) {
-      mt[t][cl + 0] -= p.x;
-      mt[t][cl + 1] -= p.y;
-      mt[t][cl + 2] -= p.z;
-      mt[t][cl + 3] -= p.w;
-    }
+    p.x += __shfl_xor_sync(0xffffffffu, p.x, 16);
+    p.y += __shfl_xor_sync(0xffffffffu, p.y, 16);
+    p.z += __shfl_xor_sync(0xffffffffu, p.z, 16);
+    p.w += __shfl_xor_sync(0xffffffffu, p.w, 16);
+    if (lane < 16) red[(t * kWarps + warp) * 16 + q] = p;
   }
-  __syncwarp();  // each warp reads back only its own columns of mt
+  __syncthreads();
+  for (int o = threadIdx.x; o < a * 16; o += kThreads) {
+    const int t = o >> 4, qq = o & 15;
+    float4 sum = red[(t * kWarps) * 16 + qq];
+#pragma unroll
+    for (int w = 1; w < kWarps; ++w) {
+      const float4 v = red[(t * kWarps + w) * 16 + qq];
+      sum.x += v.x;
+      sum.y += v.y;
+      sum.z += v.z;
+      sum.w += v.w;
+    }
+    float4* m = reinterpret_cast<float4*>(&mt[t][4 * qq]);
+    const float4 u4 = *m;
+    *m = make_float4(u4.x - sum.x, u4.y - sum.y, u4.z - sum.z, u4.w - sum.w);
+  }
+  __syncthreads();
   // S_a = G_a (S_0 + K^T M)
 #pragma unroll
   for (int r = 0; r < R; ++r) {
     float4 y = x[r];
     for (int t = 0; t < a; ++t) {
-      const float kv = ks[t * dk + rl + 16 * r];
-      y.x = fmaf(kv, mt[t][cl + 0], y.x);
-      y.y = fmaf(kv, mt[t][cl + 1], y.y);
-      y.z = fmaf(kv, mt[t][cl + 2], y.z);
-      y.w = fmaf(kv, mt[t][cl + 3], y.w);
+      const float kv = ks[t * dk + rg + 16 * r];
+      const float4 m = *reinterpret_cast<const float4*>(&mt[t][4 * q]);
+      y.x = fmaf(kv, m.x, y.x);
+      y.y = fmaf(kv, m.y, y.y);
+      y.z = fmaf(kv, m.z, y.z);
+      y.w = fmaf(kv, m.w, y.w);
     }
     y.x *= ga;
     y.y *= ga;
     y.z *= ga;
     y.w *= ga;
-    if (live) *reinterpret_cast<float4*>(base + size_t(rl + 16 * r) * dv + col) = y;
+    if (live) *reinterpret_cast<float4*>(base + size_t(rg + 16 * r) * dv + col) = y;
   }
 }
 
