@@ -15,7 +15,8 @@
 // only on steps <= t, so one set of factors serves every acceptance length.
 //
 //   lstate_factors_kernel: one block per (sequence, head); the Gram products k_t . k_s, the
-//     gates G_t, then w_t and u_t in step order (each step parallel over dk or dv).
+//     gates G_t, then w_t and u_t by forward substitution over the steps, one column per
+//     thread (the earlier steps of a column stay in shared memory).
 //   lstate_commit_kernel: one block per (sequence, head, 64-column tile of S); the tile stays
 //     in registers: M = U_a - W_a S_0 (a x 64; partial sums per thread over its rows, then
 //     over the warp's two row groups and the eight warps), then S_a = G_a (S_0 + K_a^T M),
@@ -43,22 +44,38 @@ struct LsFactorJob {
   float* gamma;         // [B][H][S]: G_t for t = 1..S
 };
 
+// Dynamic shared memory of a factor block: the keys [S][dk] (overwritten in place by w, each
+// thread's own entries), the Gram products [S][S], and the u values of the thread's current
+// column [S][kThreads].
+__host__ __device__ constexpr size_t lstate_factors_smem(int S, int dk) {
+  return (size_t(S) * dk + size_t(S) * S + size_t(S) * kThreads) * 4;
+}
+
 __global__ void __launch_bounds__(kThreads) lstate_factors_kernel(const LsFactorJob j) {
-  __shared__ float kk[kLsMaxSteps * kLsMaxDk];
-  __shared__ float gram[kLsMaxSteps][kLsMaxSteps];
-  __shared__ float g[kLsMaxSteps];
+  extern __shared__ __align__(16) float fsm[];
+  __shared__ float g[kLsMaxSteps], gi[kLsMaxSteps], bs[kLsMaxSteps];
   const int bh = blockIdx.x, S = j.S, dk = j.dk, dv = j.dv;
+  float* kk = fsm;                          // [S][dk]: k_t, overwritten in place by w_t
+  float* gram = kk + size_t(S) * dk;        // [S][S]: k_t . k_s for s < t
+  float* us = gram + size_t(S) * S;         // [S][kThreads]: v_t, overwritten by u_t
+  // every input is loaded before anything is stored (the outputs may not be assumed apart
+  // from the inputs, so a load after a store would wait for it)
   const float* kin = j.keys + size_t(bh) * S * dk;
   for (int i = threadIdx.x; i < S * dk; i += kThreads) kk[i] = kin[i];
+  if (threadIdx.x < S) {
+    g[threadIdx.x] = j.alpha[size_t(bh) * S + threadIdx.x];
+    bs[threadIdx.x] = j.beta[size_t(bh) * S + threadIdx.x];
+  }
+  __syncthreads();
   if (threadIdx.x == 0) {
     float acc = 1.0f;
     for (int t = 0; t < S; ++t) {
-      acc *= j.alpha[size_t(bh) * S + t];
+      acc *= g[t];
       g[t] = acc;
+      gi[t] = 1.0f / acc;
       j.gamma[size_t(bh) * S + t] = acc;
     }
   }
-  __syncthreads();
   // Gram products k_t . k_s (s < t), one warp per pair
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   for (int p = warp; p < S * S; p += kWarps) {
@@ -68,27 +85,36 @@ __global__ void __launch_bounds__(kThreads) lstate_factors_kernel(const LsFactor
     for (int i = lane; i < dk; i += 32) acc += kk[t * dk + i] * kk[s * dk + i];
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-    if (lane == 0) gram[t][s] = acc;
+    if (lane == 0) gram[t * S + s] = acc;
   }
   __syncthreads();
-  const float* bet = j.beta + size_t(bh) * S;
   float* wout = j.w + size_t(bh) * S * dk;
   float* uout = j.u + size_t(bh) * S * dv;
   const float* vin = j.values + size_t(bh) * S * dv;
-  // w_t and u_t in step order; a thread owns fixed entries, so it reads back only its own
-  // earlier writes
-  for (int t = 0; t < S; ++t) {
-    const float bt = bet[t];
-    for (int i = threadIdx.x; i < dk; i += kThreads) {
+  // w_t and u_t by forward substitution over the steps, one column per thread: the earlier
+  // steps of a column are the thread's own shared-memory entries
+  for (int i = threadIdx.x; i < dk; i += kThreads) {
+    for (int t = 0; t < S; ++t) {
       float x = kk[t * dk + i];
-      for (int s = 0; s < t; ++s) x -= gram[t][s] * wout[s * dk + i];
-      wout[t * dk + i] = bt * x;
+#pragma unroll 8
+      for (int s = 0; s < t; ++s) x -= gram[t * S + s] * kk[s * dk + i];
+      x = bs[t] * x;
+      kk[t * dk + i] = x;
+      wout[t * dk + i] = x;
     }
-    const float inv_g = 1.0f / g[t];
-    for (int i = threadIdx.x; i < dv; i += kThreads) {
-      float x = vin[t * dv + i] * inv_g;
-      for (int s = 0; s < t; ++s) x -= gram[t][s] * uout[s * dv + i];
-      uout[t * dv + i] = bt * x;
+  }
+  for (int i0 = 0; i0 < dv; i0 += kThreads) {
+    const int i = i0 + int(threadIdx.x);
+    if (i < dv) {
+      for (int t = 0; t < S; ++t) us[t * kThreads + threadIdx.x] = vin[t * dv + i];
+      for (int t = 0; t < S; ++t) {
+        float x = us[t * kThreads + threadIdx.x] * gi[t];
+#pragma unroll 8
+        for (int s = 0; s < t; ++s) x -= gram[t * S + s] * us[s * kThreads + threadIdx.x];
+        x = bs[t] * x;
+        us[t * kThreads + threadIdx.x] = x;
+        uout[t * dv + i] = x;
+      }
     }
   }
 }

@@ -727,8 +727,12 @@ spec_status spec_linear_state_factors(const float* alpha, const float* beta, con
   if (S > sv::kLsMaxSteps || dk > sv::kLsMaxDk || (long long)B * H > 0x7fffffffLL)
     return SPEC_ERR_UNSUPPORTED;
   sv::LsFactorJob j = {alpha, beta, keys, values, B, H, S, dk, dv, w, u, gamma};
-  sv::lstate_factors_kernel<<<unsigned(B * H), kThreads, 0, static_cast<cudaStream_t>(stream)>>>(
-      j);
+  const size_t dyn = sv::lstate_factors_smem(S, dk);
+  if (cudaFuncSetAttribute(sv::lstate_factors_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           int(dyn)) != cudaSuccess)
+    return SPEC_ERR_CUDA;
+  sv::lstate_factors_kernel<<<unsigned(B * H), kThreads, dyn,
+                              static_cast<cudaStream_t>(stream)>>>(j);
   return check_launch(cudaGetLastError());
 }
 
