@@ -34,7 +34,7 @@ def _check(gpu, ref, tol=1e-5):
 
 
 @pytest.mark.parametrize("dk,dv,S", [(32, 48, 3), (64, 64, 5), (128, 256, 9), (256, 100, 4),
-                                     (128, 4, 32)])
+                                     (128, 4, 32), (64, 2056, 9)])
 def test_commit_matches_replay(dk, dv, S):
     cfg = specgen.LinearStateConfig("t", 6, 3, dk, dv, S - 1, 0.75, seed=dk + dv + S)
     state, alpha, beta, keys, values, steps = specgen.linear_state_inputs(cfg)
