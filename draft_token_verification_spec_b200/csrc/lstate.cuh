@@ -58,8 +58,9 @@ __global__ void __launch_bounds__(kThreads) lstate_factors_kernel(const LsFactor
   float* kk = fsm;                          // [S][dk]: k_t, overwritten in place by w_t
   float* gram = kk + size_t(S) * dk;        // [S][S]: k_t . k_s for s < t
   float* us = gram + size_t(S) * S;         // [S][kThreads]: v_t, overwritten by u_t
-  // every input is loaded before anything is stored (the outputs may not be assumed apart
-  // from the inputs, so a load after a store would wait for it)
+  // the keys, gates and step weights are loaded before anything is stored, and the values of
+  // a column all at once before its substitution (the outputs may not be assumed apart from
+  // the inputs, so a load placed after a store could not be moved ahead of it)
   const float* kin = j.keys + size_t(bh) * S * dk;
   for (int i = threadIdx.x; i < S * dk; i += kThreads) kk[i] = kin[i];
   if (threadIdx.x < S) {
